@@ -1,0 +1,412 @@
+"""Decode-throughput benchmark of one SSM layer (Mamba-2, Nemotron-scale) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+A step is one rssm_decode call: one token for each of the 256 sequences of a
+Mamba-2 layer with 128 heads x headdim 64 x dstate 128 (4 MiB of fp32 state per
+sequence), 8 groups, window 16, fp32 checkpoint + bf16 read copy, bf16 inputs;
+the fold of a full buffer happens inside the step every 16 tokens.  Inputs are
+seeded synthetic tokens already resident in HBM (cycling through up to 256
+distinct steps); the 512 MiB read copy is larger than L2, so no flush is needed
+between steps.  Prints one JSON line (rank 0).
+
+N > 1 (torchrun): every rank decodes its own 256 sequences (weak scaling, no
+collective on the data path); the time is the max over ranks.
+--impl reference times the fp64 CPU oracle on the host cores instead.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from checkpoint_input_replay_rssm_b200 import inputs as I  # noqa: E402
+from checkpoint_input_replay_rssm_b200 import traffic  # noqa: E402
+
+METRIC = "SSM-layer decode tokens/s and achieved HBM GB/s vs ~8 TB/s roofline (1×B200)"
+WL = I.NEMOTRON
+FALLBACK_HBM_GBS = 6650.0
+PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "m2_replay_decode_b256_h128_p64_n128_w16.traffic.json")
+
+
+def kernel_source_hash() -> str:
+    """Hash of the CUDA sources, to tell whether a stored ncu traffic figure is current."""
+    h = hashlib.sha256()
+    d = os.path.join(ROOT, "checkpoint_input_replay_rssm_b200", "csrc")
+    for f in sorted(os.listdir(d)):
+        if f.endswith((".cu", ".cuh", ".h")):
+            h.update(f.encode())
+            h.update(open(os.path.join(d, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def measured_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        return float(json.load(open(p))["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """Polls NVML (read-only) for SM clock and clock-event reasons during the timed region."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, index: int):
+        self.ok = False
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # no NVML: report that, do not guess
+            self.err = str(e)
+        self.samples, self.reasons = [], 0
+        self._stop = threading.Event()
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                self.reasons |= self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+            except Exception:
+                pass
+            time.sleep(0.002)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "error": self.err}
+        names = [n for bit, n in self.REASONS.items() if self.reasons & bit and n != "gpu_idle"]
+        return {"sm_mhz": float(np.median(self.samples)) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": names, "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------ setup
+def make_layer(wl, mode, state_dtype, consts, device):
+    import torch
+
+    from checkpoint_input_replay_rssm_b200 import rssm
+
+    cfg = rssm.make_config(kind=wl.kind, mode=mode, state_dtype=state_dtype,
+                           input_dtype=wl.input_dtype, batch=wl.batch, nheads=wl.nheads,
+                           headdim=wl.headdim, dstate=wl.dstate, ngroups=wl.ngroups,
+                           window=wl.window, max_draft=1)
+    L = rssm.Layer(cfg, device=device)
+    L.set_params(torch.tensor(consts["A"], dtype=torch.float32, device=device),
+                 torch.tensor(consts["D"], dtype=torch.float32, device=device))
+    L.import_state(torch.from_numpy(consts["S0"]).to(device))
+    return L
+
+
+def host_tokens(wl, n):
+    """n distinct seeded decode steps as pinned host tensors in storage dtypes."""
+    import torch
+
+    out = []
+    for t in range(n):
+        tok = I.token(wl, t)
+        d = {}
+        for k, v in tok.items():
+            ht = I.to_torch(v, wl.input_dtype if k in ("x", "B", "C") else "f32").unsqueeze(1)
+            d[k] = ht.contiguous().pin_memory()
+        out.append(d)
+    return out
+
+
+def timed_loop(L, toks_dev, ys, K, W, sync):
+    """W warm-up then K timed decode steps; per-launch and whole-loop CUDA events."""
+    import torch
+
+    from checkpoint_input_replay_rssm_b200 import rssm
+
+    n = len(toks_dev)
+    ins = [L._inputs(d) for d in toks_dev]
+    yptr = [y.data_ptr() for y in ys]
+    for i in range(W):
+        rssm.rssm_decode(L.h, ins[i % n], yptr[i % len(ys)])
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sync()
+    l0 = L.launches()
+    stream = L.stream
+    t0.record(stream)
+    for i in range(K):
+        j = (W + i) % n
+        starts[i].record(stream)
+        rssm.rssm_decode(L.h, ins[j], yptr[i % len(ys)])
+        ends[i].record(stream)
+    t1.record(stream)
+    sync()
+    launches = L.launches() - l0
+    total_ms = t0.elapsed_time(t1)
+    per = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    return total_ms, float(np.mean(per)), launches
+
+
+def e2e_loop(L, toks_host, K, W, sync):
+    """Public-API decode with host buffers: pinned H2D of the step's inputs, decode,
+    D2H of the step's output, all inside the timed region."""
+    import torch
+
+    dev = {k: torch.empty_like(v, device=L.device) for k, v in toks_host[0].items()}
+    y = torch.empty((L.B, 1, L.H, L.P), dtype=torch.float32, device=L.device)
+    y_host = torch.empty_like(y, device="cpu").pin_memory()
+    n = len(toks_host)
+
+    def step(i):
+        for k, v in toks_host[i % n].items():
+            dev[k].copy_(v, non_blocking=True)
+        L.decode(dev, y=y)
+        y_host.copy_(y, non_blocking=True)
+
+    for i in range(W):
+        step(i)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sync()
+    t0.record(L.stream)
+    for i in range(K):
+        step(W + i)
+    t1.record(L.stream)
+    sync()
+    h2d = sum(v.numel() * v.element_size() for v in toks_host[0].values())
+    return t0.elapsed_time(t1), h2d, y.numel() * y.element_size()
+
+
+# ------------------------------------------------------------------ CPU oracle legs
+def oracle_tokens_per_s(wl, seqs, max_steps, budget_s):
+    """Time the fp64 eager oracle (as it stands) on `seqs` sequences for up to
+    `max_steps` tokens or `budget_s` seconds of oracle time; input generation is
+    outside the timed part."""
+    from oracle import eager
+
+    c = I.constants(wl, seqs=range(seqs))
+    S = np.ascontiguousarray(c["S0"])
+    done, t_used = 0, 0.0
+    for t in range(max_steps):
+        tok = I.token(wl, t, seqs=range(seqs))
+        t0 = time.perf_counter()
+        eager.mamba2_step(S, c["A"], c["D"], tok["x"], tok["dt"], tok["B"], tok["C"])
+        t_used += time.perf_counter() - t0
+        done += 1
+        if t_used >= budget_s:
+            break
+    return seqs * done / t_used, done, t_used, eager.max_threads()
+
+
+def run_reference(args, rank):
+    if rank != 0:
+        return
+    from oracle import eager
+
+    eager.build()
+    seqs = 16
+    K, W = args.steps, args.warmup
+    c = I.constants(WL, seqs=range(seqs))
+    n = min(K + W, 8)
+    toks = [I.token(WL, t, seqs=range(seqs)) for t in range(n)]
+    S = np.ascontiguousarray(c["S0"])
+    for i in range(W):
+        tok = toks[i % n]
+        eager.mamba2_step(S, c["A"], c["D"], tok["x"], tok["dt"], tok["B"], tok["C"])
+    t0 = time.perf_counter()
+    for i in range(K):
+        tok = toks[(W + i) % n]
+        eager.mamba2_step(S, c["A"], c["D"], tok["x"], tok["dt"], tok["B"], tok["C"])
+    dt = time.perf_counter() - t0
+    value = seqs * K / dt
+    sample = (f"fp64 eager oracle (C, OpenMP) on {seqs} of the 256 sequences x 128 heads x 64 x 128, "
+              f"one token per step, inputs pre-generated")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": K, "warmup": W, "ms_per_step": dt * 1e3 / K, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_config(),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": eager.max_threads(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def workload_config():
+    return {"workload": WL.name, "batch_per_gpu": WL.batch, "nheads": WL.nheads, "headdim": WL.headdim,
+            "dstate": WL.dstate, "ngroups": WL.ngroups, "window": WL.window, "checkpoint": "f32",
+            "read_copy": "bf16", "inputs": "bf16",
+            "l2": "no flush: the 512 MiB read copy read every step exceeds the 126 MB L2",
+            "input_steps": "seeded steps resident in HBM, cycled"}
+
+
+# ------------------------------------------------------------------ main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=256)
+    ap.add_argument("--warmup", type=int, default=16)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-eager", action="store_true", help="skip the eager-baseline leg")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle leg")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+
+    import datetime
+
+    import torch
+
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=device)
+
+    def sync():
+        torch.cuda.synchronize(device)
+        if dist is not None:
+            dist.barrier()
+            torch.cuda.synchronize(device)
+
+    from checkpoint_input_replay_rssm_b200 import build, rssm
+
+    if not os.path.exists(build.LIB):
+        build.build()
+    rssm.load()
+
+    K, W = args.steps, args.warmup
+    wl = WL.replace(seed=WL.seed + 7919 * rank)
+    consts = I.constants(wl, f64=False)
+    n_distinct = min(K + W, 256)
+    toks_host = host_tokens(wl, n_distinct)
+    toks_dev = [{k: v.to(device) for k, v in d.items()} for d in toks_host]
+    ys = [torch.empty((wl.batch, 1, wl.nheads, wl.headdim), dtype=torch.float32, device=device)
+          for _ in range(2)]
+
+    L = make_layer(wl, "replay", "bf16", consts, device)
+    sampler = ClockSampler(local)
+    with sampler:
+        total_ms, kern_ms, launches = timed_loop(L, toks_dev, ys, K, W, sync)
+    clocks = sampler.summary()
+    t = torch.tensor([total_ms, kern_ms], dtype=torch.float64, device=device)
+    if dist is not None:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms, kern_ms = float(t[0]), float(t[1])
+    assert L.status()[0] == 0, "device error during the benchmark"
+
+    # e2e through the public API with host buffers (fresh layer, same workload)
+    L.import_state(torch.from_numpy(consts["S0"]).to(device))
+    e2e_ms, h2d, d2h = e2e_loop(L, toks_host, K, W, sync)
+    t = torch.tensor([e2e_ms], dtype=torch.float64, device=device)
+    if dist is not None:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    e2e_ms = float(t[0])
+
+    shape = traffic.Shape("mamba2", wl.headdim, wl.dstate, wl.nheads // wl.ngroups, wl.window, "bf16",
+                          wl.input_dtype)
+    rep = traffic.replay_decode_per_token(shape)
+    units = wl.batch * wl.nheads
+    bytes_per_launch = traffic.total(rep) * units
+    achieved = bytes_per_launch / (kern_ms * 1e-3) / 1e9
+    peak, peak_kind = measured_peak()
+    tr = None
+    if os.path.exists(PROFILE_TRAFFIC):
+        p = json.load(open(PROFILE_TRAFFIC))
+        if p.get("kernel_hash") == kernel_source_hash():
+            tr = p.get("dram_bytes_per_launch")
+
+    eager = None
+    if not args.no_eager:
+        del L
+        torch.cuda.empty_cache()
+        E = make_layer(wl, "eager", "f32", consts, device)
+        e_total, e_kern, _ = timed_loop(E, toks_dev, ys, K, W, sync)
+        t = torch.tensor([e_total, e_kern], dtype=torch.float64, device=device)
+        if dist is not None:
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e_total, e_kern = float(t[0]), float(t[1])
+        eg = traffic.eager_decode_per_token(shape, "f32")
+        eager = {"value": world * wl.batch * K / (e_total * 1e-3), "unit": "tokens/s",
+                 "ms_per_step": e_total / K,
+                 "hbm_gbs": traffic.total(eg) * units / (e_kern * 1e-3) / 1e9,
+                 "bytes_per_token_per_head": traffic.total(eg)}
+        del E
+
+    state_rep, state_eag = traffic.state_bytes(rep), traffic.state_bytes(
+        traffic.eager_decode_per_token(shape, "f32"))
+    line = {
+        "metric": METRIC,
+        "value": world * wl.batch * K / (total_ms * 1e-3),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": W,
+        "ms_per_step": total_ms / K,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f32",
+        "data": "synthetic",
+        "config": workload_config() | {"parallelism": f"dp{world} (independent sequences)"},
+        "hbm_gbs": achieved,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": tr, "peak_source": peak_kind,
+                     "kernel": "m2_replay_kernel<128, bf16, 1>",
+                     "algorithmic_bytes_per_launch": bytes_per_launch,
+                     "kernel_ms_per_launch": kern_ms},
+        "e2e": {"value": world * wl.batch * K / (e2e_ms * 1e-3), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches,
+        "clocks": clocks,
+        "state_bytes_per_token_per_head": {"replay": state_rep, "eager": state_eag,
+                                           "ratio": state_rep / state_eag},
+        "eager": eager,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu:
+        v, done, used, cores = oracle_tokens_per_s(wl, 64, 256, 12.0)
+        line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                                "sample": f"fp64 eager oracle on 64 of 256 sequences x 128 heads, "
+                                          f"{done} steps, {used:.1f} s"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,543 @@
+// rssm_gdn.cuh -- Gated DeltaNet decode kernels for sm_100a (templates; instantiated per dstate).
+//
+// Layer (per sequence b, head h; S is d_v x d_k, rows contiguous along d_k):
+//   S_t = alpha_t S_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,   o_t = S_t q_t
+// GDN's update is the Mamba-2 form plus a delta-rule correction
+// (blog.thibaultmonteiro.fr, "La fiche qu'on reecrit a chaque token"), so the
+// same checkpoint + input-buffer replay applies.  With M_j = alpha_j (I - beta_j k_j k_j^T)
+// and buffered entries 1..L (L counts the query token):
+//   o = S_c M_1 ... M_L q + sum_i beta_i v_i (k_i . M_{i+1} ... M_L q)
+// Sweep r <- q; for j = L..1: c_j = beta_j (k_j . r), r <- alpha_j (r - c_j k_j);
+// then o = S^ r + sum_j c_j v_j.  The kernel never forms r during the sweep: it
+// tracks t_e = k_e . r for every earlier entry e, which obeys
+//   t_e <- alpha_j (t_e - c_j (k_e . k_j)),
+// so with the Gram matrix k_e . k_j computed up front (all warps, in parallel)
+// the serial chain is one shuffle per entry, and
+//   r = (prod_{l} alpha_l) q - sum_i (prod_{l<=i} alpha_l) c_i k_i
+// is assembled afterwards in parallel.  The fold applies the per-token updates
+// in order to each fp32 checkpoint row in registers:
+//   s <- alpha s + (beta v[row] - alpha beta (s . k)) k.
+#pragma once
+#include "rssm_device.cuh"
+#include "rssm_internal.h"
+
+namespace rssm {
+
+struct GArgs {
+    int B, H, P, W, R, T, op, in_bf16;
+    Counters c;
+    float *ckpt;
+    void *rc;
+    float *rc_scale;
+    void *kbuf, *vbuf;   // [B][H][R][N], [B][H][R][P] input dtype
+    float *abuf, *bbuf;  // [B][H][R]
+    void *snap;
+    float *snap_scale;
+    const void *q, *k, *v;      // [B][T][H][N|P]
+    const float *alpha, *beta;  // [B][T][H]
+    float *y;                   // [B][T][H][P]
+    float *out;                 // export target
+};
+
+__host__ __device__ constexpr int gpad4(int n) { return (n + 3) & ~3; }
+
+__host__ __device__ inline size_t gdn_smem_floats(int P, int N, int W, int TQ) {
+    const int E = W + TQ;
+    return (size_t)gpad4(E * N) + gpad4(E * P) + 3 * (size_t)gpad4(E) + gpad4(TQ * N) +
+           gpad4(E * E) + 2 * (size_t)gpad4(TQ * E) + gpad4(TQ * N) + gpad4(TQ * P) + gpad4(TQ) + 8;
+}
+
+struct GSmem {
+    float *sk, *sv, *sal, *sbe, *spr, *sq, *sG, *shq, *sc, *sr, *sdot, *srq;
+    int *si;
+};
+
+__device__ __forceinline__ GSmem gdn_carve(float *sm, int P, int N, int W, int TQ) {
+    const int E = W + TQ;
+    GSmem s;
+    s.sk = sm;                            // [E][N]  k of entries (physical)
+    s.sv = s.sk + gpad4(E * N);           // [E][P]  v of entries (physical)
+    s.sal = s.sv + gpad4(E * P);          // [E]     alpha (physical)
+    s.sbe = s.sal + gpad4(E);             // [E]     beta (physical)
+    s.spr = s.sbe + gpad4(E);             // [E]     prefix products of alpha from e0 (logical)
+    s.sq = s.spr + gpad4(E);              // [TQ][N] queries
+    s.sG = s.sq + gpad4(TQ * N);          // [E][E]  Gram k_e . k_j (logical)
+    s.shq = s.sG + gpad4(E * E);          // [TQ][E] k_e . q_m (logical)
+    s.sc = s.shq + gpad4(TQ * E);         // [TQ][E] sweep coefficients c (logical)
+    s.sr = s.sc + gpad4(TQ * E);          // [TQ][N] swept query r
+    s.sdot = s.sr + gpad4(TQ * N);        // [TQ][P] S^ r per row
+    s.srq = s.sdot + gpad4(TQ * P);       // [TQ]    unused pad
+    s.si = reinterpret_cast<int *>(s.srq + gpad4(TQ));
+    return s;
+}
+
+// Fold-mapping: TPRF lanes per state row, NPT contiguous elements per lane.
+template <int N> struct FoldMap {
+    static constexpr int TPRF = (N >= 32) ? 8 : N / 4;
+    static constexpr int NPT = N / TPRF;
+    static constexpr int RPPF = kThreads / TPRF;
+};
+
+// Stage the new tokens' inputs at physical entries W..W+T-1 and queries.
+__device__ __forceinline__ void gdn_stage_new(const GArgs &a, const GSmem &s, int b, int h, int N,
+                                              int tid) {
+    const int H = a.H, P = a.P, T = a.T, W = a.W;
+    for (int i = tid; i < T * N; i += kThreads) {
+        const int m = i / N, n = i - m * N;
+        const int64_t src = ((int64_t)(b * T + m) * H + h) * N + n;
+        s.sk[(W + m) * N + n] = ld_in(a.k, src, a.in_bf16);
+        s.sq[m * N + n] = ld_in(a.q, src, a.in_bf16);
+    }
+    for (int i = tid; i < T * P; i += kThreads) {
+        const int m = i / P, p = i - m * P;
+        s.sv[(W + m) * P + p] = ld_in(a.v, ((int64_t)(b * T + m) * H + h) * P + p, a.in_bf16);
+    }
+    if (tid < T) {
+        s.sal[W + tid] = a.alpha[(int64_t)(b * T + tid) * H + h];
+        s.sbe[W + tid] = a.beta[(int64_t)(b * T + tid) * H + h];
+    }
+}
+
+// Apply entries [0, L0) (physical base..) to NR rows held as NPT-element lane
+// segments.  Rows are independent; every lane of the warp must call this.
+template <int N, int NR>
+__device__ __forceinline__ void gdn_fold_rows(float (&st)[NR][FoldMap<N>::NPT], const int (&rows)[NR],
+                                              int P, const GSmem &s, int base, int L0, int cseg) {
+    constexpr int NPT = FoldMap<N>::NPT, TPRF = FoldMap<N>::TPRF;
+    for (int e = 0; e < L0; ++e) {
+        const float al = s.sal[base + e], be = s.sbe[base + e];
+        float kk[NPT];
+#pragma unroll
+        for (int j = 0; j < NPT; j += 4) {
+            const float4 k4 = *reinterpret_cast<const float4 *>(s.sk + (base + e) * N + cseg * NPT + j);
+            kk[j] = k4.x; kk[j + 1] = k4.y; kk[j + 2] = k4.z; kk[j + 3] = k4.w;
+        }
+#pragma unroll
+        for (int r = 0; r < NR; ++r) {
+            float d = 0.f;
+#pragma unroll
+            for (int j = 0; j < NPT; ++j) d = fmaf(st[r][j], kk[j], d);
+            d = group_sum<TPRF>(d);
+            const float vr = (rows[r] < P) ? s.sv[(base + e) * P + rows[r]] : 0.f;
+            const float coef = be * vr - al * be * d;
+#pragma unroll
+            for (int j = 0; j < NPT; ++j) st[r][j] = fmaf(al, st[r][j], coef * kk[j]);
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Replay kernel: decode (T = 1), verify (T = K), flush (T = 0), export (T = 0).
+// ---------------------------------------------------------------------------
+template <int N, int RK, int TQ>
+__global__ void __launch_bounds__(kThreads) gdn_replay_kernel(const GArgs a) {
+    constexpr int EPC = Chunk<RK>::EPC;
+    constexpr int TPR = N / EPC;
+    constexpr int RPP = kThreads / TPR;
+    constexpr int RB = 8;
+    using FM = FoldMap<N>;
+    constexpr int NPT = FM::NPT, TPRF = FM::TPRF, RPPF = FM::RPPF, RBF = 4;
+    static_assert(TPR >= 1 && TPR <= 32 && (32 % TPR) == 0, "row must fit a warp");
+
+    extern __shared__ __align__(16) float smem[];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int bh = blockIdx.x;
+    const int H = a.H, P = a.P, W = a.W, R = a.R, T = a.T;
+    const int b = bh / H, h = bh - b * H;
+    const int E = W + TQ;
+    GSmem s = gdn_carve(smem, P, N, W, TQ);
+    const int64_t tile0 = (int64_t)bh * P * N;
+    const bool reads = (a.op == OP_DECODE || a.op == OP_VERIFY);
+
+    // 1. Read-copy loads first (dropped on folding steps).
+    const int c = tid % TPR, r0 = tid / TPR;
+    const uint8_t *rc_tile =
+        (RK == SK_F32) ? reinterpret_cast<const uint8_t *>(a.ckpt + tile0)
+                       : reinterpret_cast<const uint8_t *>(a.rc) + tile0 * Chunk<RK>::BYTES;
+    uint4 rv[RB];
+    float rscale[RB];
+    if (reads) {
+#pragma unroll
+        for (int k = 0; k < RB; ++k) {
+            const int r = r0 + k * RPP;
+            if (r < P) rv[k] = ld_stream(rc_tile + ((size_t)r * TPR + c) * 16);
+            if (RK == SK_FP8) rscale[k] = (r < P) ? __ldg(a.rc_scale + (int64_t)bh * P + r) : 0.f;
+        }
+    }
+
+    // 2. Counters and new-token staging.
+    if (tid == 0) {
+        SeqState ss = read_counters(a.c, b, W);
+        const int L0 = (int)(ss.seq - ss.ckpt);
+        int flush = 0;
+        if (ss.ok) flush = (a.op == OP_FLUSH || a.op == OP_EXPORT) ? (L0 > 0) : (L0 + T > W);
+        s.si[0] = ss.ok;
+        s.si[1] = ss.ok ? L0 : 0;
+        s.si[2] = flush;
+        s.si[3] = (int)(ss.ckpt % R);
+        s.si[4] = (int)(ss.seq % R);
+        if (!ss.ok) {
+            if (h == 0) report(a.c.err, DEV_BAD_COUNTERS, b, h, (int)(ss.seq - ss.ckpt));
+        } else if (a.op != OP_EXPORT) {
+            const int64_t new_seq = (a.op == OP_DECODE) ? ss.seq + 1 : -1;
+            const int64_t new_ckpt = flush ? ss.seq : -1;
+            const int new_pending = (a.op == OP_VERIFY) ? T : -1;
+            arrive_and_publish(a.c, b, H, new_seq, new_ckpt, new_pending, flush);
+        }
+    }
+    gdn_stage_new(a, s, b, h, N, tid);
+    __syncthreads();
+    if (!s.si[0]) return;
+    const int L0 = s.si[1], flush = s.si[2], ckmod = s.si[3], spmod = s.si[4];
+    const int base = W - L0;
+    const int nE = L0 + T;
+    const int e0 = flush ? L0 : 0;
+
+    // 3. Buffered entries.
+    for (int i = tid; i < L0 * N; i += kThreads) {
+        const int e = i / N, n = i - e * N;
+        s.sk[(base + e) * N + n] = ld_in(a.kbuf, ((int64_t)bh * R + (ckmod + e) % R) * N + n, a.in_bf16);
+    }
+    for (int i = tid; i < L0 * P; i += kThreads) {
+        const int e = i / P, p = i - e * P;
+        s.sv[(base + e) * P + p] = ld_in(a.vbuf, ((int64_t)bh * R + (ckmod + e) % R) * P + p, a.in_bf16);
+    }
+    for (int e = tid; e < L0; e += kThreads) {
+        const int64_t slot = (int64_t)bh * R + (ckmod + e) % R;
+        s.sal[base + e] = a.abuf[slot];
+        s.sbe[base + e] = a.bbuf[slot];
+    }
+    __syncthreads();
+
+    if (reads) {
+        // 4. Gram matrix of the replayed keys and their products with the queries.
+        const int n = nE - e0;                       // replayed entries
+        const int ngram = n * (n - 1) / 2;
+        const int nq = T * n;
+        for (int pr = warp; pr < ngram + nq; pr += kWarps) {
+            int ea, eb;
+            const float *va, *vb;
+            if (pr < ngram) {  // unrank pr -> (i < j) over [0, n)
+                int j = (int)((1.f + sqrtf(1.f + 8.f * (float)pr)) * 0.5f);
+                while (j * (j - 1) / 2 > pr) --j;
+                while ((j + 1) * j / 2 <= pr) ++j;
+                const int i = pr - j * (j - 1) / 2;
+                ea = e0 + i; eb = e0 + j;
+                va = s.sk + (base + ea) * N;
+                vb = s.sk + (base + eb) * N;
+            } else {
+                const int m = (pr - ngram) / n;
+                ea = e0 + (pr - ngram) - m * n;
+                eb = -1 - m;
+                va = s.sk + (base + ea) * N;
+                vb = s.sq + m * N;
+            }
+            float d = 0.f;
+            for (int x = lane; x < N; x += 32) d = fmaf(va[x], vb[x], d);
+            d = group_sum<32>(d);
+            if (lane == 0) {
+                if (eb >= 0) s.sG[ea * E + eb] = d;
+                else s.shq[(-1 - eb) * E + ea] = d;
+            }
+        }
+        if (tid == 0) {  // prefix products of alpha from e0
+            float acc = 1.f;
+            for (int e = e0; e < nE; ++e) { acc *= s.sal[base + e]; s.spr[e] = acc; }
+        }
+        __syncthreads();
+        // 5. One warp per query: the backward sweep as a lane-parallel chain.
+        constexpr int CH = (64 + TQ + 31) / 32;  // entries per lane (W <= 64)
+        if (warp < T) {
+            const int m = warp, em = L0 + m;
+            float t[CH];
+#pragma unroll
+            for (int j = 0; j < CH; ++j) {
+                const int e = e0 + lane + 32 * j;
+                t[j] = (e <= em) ? s.shq[m * E + e] : 0.f;
+            }
+            for (int i = em; i >= e0; --i) {
+                const int li = i - e0, src = li & 31, ji = li >> 5;
+                float ti = 0.f;
+#pragma unroll
+                for (int j = 0; j < CH; ++j) if (j == ji) ti = t[j];
+                const float ci = s.sbe[base + i] * __shfl_sync(0xffffffffu, ti, src);
+                const float al = s.sal[base + i];
+                if (lane == 0) s.sc[m * E + i] = ci;
+#pragma unroll
+                for (int j = 0; j < CH; ++j) {
+                    const int e = e0 + lane + 32 * j;
+                    if (e < i) t[j] = al * (t[j] - ci * s.sG[e * E + i]);
+                }
+            }
+        }
+        __syncthreads();
+        // 6. r_m = P_{em} q_m - sum_i P_i c_{m,i} k_i  (P_i: prefix products of alpha).
+        for (int idx = tid; idx < T * N; idx += kThreads) {
+            const int m = idx / N, x = idx - m * N, em = L0 + m;
+            float r = s.spr[em] * s.sq[m * N + x];
+            for (int i = e0; i <= em; ++i) r = fmaf(-s.spr[i] * s.sc[m * E + i], s.sk[(base + i) * N + x], r);
+            s.sr[m * N + x] = r;
+        }
+        __syncthreads();
+    }
+
+    if (flush) {
+        // 7a. Fold the committed entries into the fp32 checkpoint rows.
+        const int cseg = tid % TPRF, q0 = tid / TPRF;
+        for (int rb = 0; rb < P; rb += RBF * RPPF) {
+            float st[RBF][NPT];
+            int rows[RBF];
+#pragma unroll
+            for (int k = 0; k < RBF; ++k) {
+                rows[k] = rb + q0 + k * RPPF;
+#pragma unroll
+                for (int j = 0; j < NPT; j += 4) {
+                    float4 v4 = make_float4(0.f, 0.f, 0.f, 0.f);
+                    if (rows[k] < P) v4 = load_quad<SK_F32>(a.ckpt, tile0 + (int64_t)rows[k] * N + cseg * NPT + j);
+                    st[k][j] = v4.x; st[k][j + 1] = v4.y; st[k][j + 2] = v4.z; st[k][j + 3] = v4.w;
+                }
+            }
+            gdn_fold_rows<N, RBF>(st, rows, P, s, base, L0, cseg);
+#pragma unroll
+            for (int k = 0; k < RBF; ++k) {
+                const bool valid = rows[k] < P;
+                const int64_t el = tile0 + (int64_t)(valid ? rows[k] : 0) * N + cseg * NPT;
+                if (a.op == OP_EXPORT) {
+                    if (valid)
+#pragma unroll
+                        for (int j = 0; j < NPT; j += 4)
+                            *reinterpret_cast<float4 *>(a.out + el + j) =
+                                make_float4(st[k][j], st[k][j + 1], st[k][j + 2], st[k][j + 3]);
+                    continue;
+                }
+                float sc = 1.f;
+                if (RK == SK_FP8) {
+                    float am = 0.f;
+#pragma unroll
+                    for (int j = 0; j < NPT; ++j) am = fmaxf(am, fabsf(st[k][j]));
+                    sc = fp8_scale(group_max<TPRF>(am));
+                    if (valid && cseg == 0) a.rc_scale[(int64_t)bh * P + rows[k]] = sc;
+                }
+                float dots[TQ];
+#pragma unroll
+                for (int m = 0; m < TQ; ++m) dots[m] = 0.f;
+#pragma unroll
+                for (int j = 0; j < NPT; j += 4) {
+                    float4 v4 = make_float4(st[k][j], st[k][j + 1], st[k][j + 2], st[k][j + 3]);
+                    float4 rd = v4;
+                    if (valid) {
+                        store_quad<SK_F32>(a.ckpt, el + j, v4, 0.f, 0.f);
+                        if (RK == SK_BF16) rd = store_quad<SK_BF16>(a.rc, el + j, v4, 0.f, 0.f);
+                        if (RK == SK_FP8) rd = store_quad<SK_FP8>(a.rc, el + j, v4, 0.f, sc);
+                    }
+                    if (reads) {
+#pragma unroll
+                        for (int m = 0; m < TQ; ++m) {
+                            const float4 r4 = *reinterpret_cast<const float4 *>(s.sr + m * N + cseg * NPT + j);
+                            dots[m] += rd.x * r4.x + rd.y * r4.y + rd.z * r4.z + rd.w * r4.w;
+                        }
+                    }
+                }
+                if (reads) {
+#pragma unroll
+                    for (int m = 0; m < TQ; ++m) {
+                        const float d = group_sum<TPRF>(dots[m]);
+                        if (valid && cseg == 0 && m < T) s.sdot[m * P + rows[k]] = d;
+                    }
+                }
+            }
+        }
+    } else if (reads) {
+        // 7b. Read: dot products of the read-copy rows with the swept queries.
+        float Rr[TQ][EPC];
+#pragma unroll
+        for (int m = 0; m < TQ; ++m)
+#pragma unroll
+            for (int j = 0; j < EPC; ++j) Rr[m][j] = (m < T) ? s.sr[m * N + c * EPC + j] : 0.f;
+        for (int rb = 0; rb < P; rb += RB * RPP) {
+            if (rb > 0) {
+#pragma unroll
+                for (int k = 0; k < RB; ++k) {
+                    const int r = rb + r0 + k * RPP;
+                    if (r < P) rv[k] = ld_stream(rc_tile + ((size_t)r * TPR + c) * 16);
+                    if (RK == SK_FP8) rscale[k] = (r < P) ? __ldg(a.rc_scale + (int64_t)bh * P + r) : 0.f;
+                }
+            }
+#pragma unroll
+            for (int k = 0; k < RB; ++k) {
+                const int r = rb + r0 + k * RPP;
+                float v[EPC];
+                if (r < P) unpack<RK>(rv[k], v);
+                else {
+#pragma unroll
+                    for (int j = 0; j < EPC; ++j) v[j] = 0.f;
+                }
+#pragma unroll
+                for (int m = 0; m < TQ; ++m) {
+                    float d = 0.f;
+#pragma unroll
+                    for (int j = 0; j < EPC; ++j) d = fmaf(v[j], Rr[m][j], d);
+                    d = group_sum<TPR>(d);
+                    if (RK == SK_FP8) d *= rscale[k];
+                    if (c == 0 && r < P && m < T) s.sdot[m * P + r] = d;
+                }
+            }
+        }
+    }
+    if (!reads) return;
+    __syncthreads();
+
+    // 8. Outputs o_m = S^ r_m + sum_i c_{m,i} v_i.
+    for (int i = tid; i < T * P; i += kThreads) {
+        const int m = i / P, p = i - m * P;
+        float o = s.sdot[m * P + p];
+        for (int e = e0; e <= L0 + m; ++e) o = fmaf(s.sc[m * E + e], s.sv[(base + e) * P + p], o);
+        a.y[((int64_t)(b * T + m) * H + h) * P + p] = o;
+    }
+
+    // 9. Append the new tokens to the ring.
+    for (int i = tid; i < T * N; i += kThreads) {
+        const int m = i / N, n = i - m * N;
+        copy_in(a.kbuf, ((int64_t)bh * R + (spmod + m) % R) * N + n, a.k,
+                ((int64_t)(b * T + m) * H + h) * N + n, a.in_bf16);
+    }
+    for (int i = tid; i < T * P; i += kThreads) {
+        const int m = i / P, p = i - m * P;
+        copy_in(a.vbuf, ((int64_t)bh * R + (spmod + m) % R) * P + p, a.v,
+                ((int64_t)(b * T + m) * H + h) * P + p, a.in_bf16);
+    }
+    if (tid < T) {
+        const int64_t slot = (int64_t)bh * R + (spmod + tid) % R;
+        a.abuf[slot] = s.sal[W + tid];
+        a.bbuf[slot] = s.sbe[W + tid];
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Eager baseline: decode (state rewritten every token) and verify (K snapshots).
+// ---------------------------------------------------------------------------
+template <int N, int SK, int TQ>
+__global__ void __launch_bounds__(kThreads) gdn_eager_kernel(const GArgs a) {
+    using FM = FoldMap<N>;
+    constexpr int NPT = FM::NPT, TPRF = FM::TPRF, RPPF = FM::RPPF, RBF = 4;
+    extern __shared__ __align__(16) float smem[];
+    const int tid = threadIdx.x;
+    const int bh = blockIdx.x;
+    const int H = a.H, P = a.P, T = a.T, W = a.W;
+    const int b = bh / H, h = bh - b * H;
+    GSmem s = gdn_carve(smem, P, N, W, TQ);
+    const int64_t tile0 = (int64_t)bh * P * N;
+    void *state = (SK == SK_F32) ? (void *)a.ckpt : a.rc;
+    const int64_t state_elems = (int64_t)a.B * H * P * N;
+
+    if (tid == 0) {
+        SeqState st = read_counters(a.c, b, W);
+        if (a.op == OP_DECODE)
+            arrive_and_publish(a.c, b, H, st.seq + 1, st.seq + 1, -1, 0);
+        else
+            arrive_and_publish(a.c, b, H, -1, -1, T, 0);
+    }
+    gdn_stage_new(a, s, b, h, N, tid);
+    __syncthreads();
+
+    const int cseg = tid % TPRF, q0 = tid / TPRF;
+    for (int rb = 0; rb < P; rb += RBF * RPPF) {
+        float st[RBF][NPT];
+        int rows[RBF];
+#pragma unroll
+        for (int k = 0; k < RBF; ++k) {
+            rows[k] = rb + q0 + k * RPPF;
+            const float scl = (SK == SK_FP8 && rows[k] < P) ? __ldg(a.rc_scale + (int64_t)bh * P + rows[k]) : 1.f;
+#pragma unroll
+            for (int j = 0; j < NPT; j += 4) {
+                float4 v4 = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (rows[k] < P) v4 = load_quad<SK>(state, tile0 + (int64_t)rows[k] * N + cseg * NPT + j);
+                st[k][j] = v4.x * scl; st[k][j + 1] = v4.y * scl; st[k][j + 2] = v4.z * scl; st[k][j + 3] = v4.w * scl;
+            }
+        }
+        for (int m = 0; m < T; ++m) {
+            // one token: entry m sits at physical W + m
+            gdn_fold_rows<N, RBF>(st, rows, P, s, W + m, 1, cseg);
+#pragma unroll
+            for (int k = 0; k < RBF; ++k) {
+                const bool valid = rows[k] < P;
+                float d = 0.f;
+#pragma unroll
+                for (int j = 0; j < NPT; ++j) d = fmaf(st[k][j], s.sq[m * N + cseg * NPT + j], d);
+                d = group_sum<TPRF>(d);
+                if (valid && cseg == 0) s.sdot[m * P + rows[k]] = d;
+                const bool last = (m == T - 1);
+                if (a.op == OP_VERIFY || (a.op == OP_DECODE && last)) {
+                    void *dst = state;
+                    float *dscale = a.rc_scale;
+                    if (a.op == OP_VERIFY) {
+                        dst = (SK == SK_F32) ? (void *)(reinterpret_cast<float *>(a.snap) + m * state_elems)
+                                             : (void *)(reinterpret_cast<uint8_t *>(a.snap) + m * state_elems * Chunk<SK>::BYTES);
+                        dscale = a.snap_scale ? a.snap_scale + (int64_t)m * a.B * H * P : nullptr;
+                    }
+                    float sc = 1.f;
+                    if (SK == SK_FP8) {
+                        float am = 0.f;
+#pragma unroll
+                        for (int j = 0; j < NPT; ++j) am = fmaxf(am, fabsf(st[k][j]));
+                        sc = fp8_scale(group_max<TPRF>(am));
+                        if (valid && cseg == 0) dscale[(int64_t)bh * P + rows[k]] = sc;
+                    }
+                    if (valid) {
+                        const int64_t el = tile0 + (int64_t)rows[k] * N + cseg * NPT;
+#pragma unroll
+                        for (int j = 0; j < NPT; j += 4)
+                            store_quad<SK>(dst, el + j, make_float4(st[k][j], st[k][j + 1], st[k][j + 2], st[k][j + 3]), 0.f, sc);
+                    }
+                }
+            }
+        }
+    }
+    __syncthreads();
+    for (int i = tid; i < T * P; i += kThreads) {
+        const int m = i / P, p = i - m * P;
+        a.y[((int64_t)(b * T + m) * H + h) * P + p] = s.sdot[m * P + p];
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Host launchers.
+// ---------------------------------------------------------------------------
+template <int N, int RK, int TQ>
+inline cudaError_t glaunch_replay(const GArgs &a, size_t smem, cudaStream_t st) {
+    auto k = gdn_replay_kernel<N, RK, TQ>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    k<<<a.B * a.H, kThreads, smem, st>>>(a);
+    return cudaGetLastError();
+}
+template <int N, int SK, int TQ>
+inline cudaError_t glaunch_eager(const GArgs &a, size_t smem, cudaStream_t st) {
+    auto k = gdn_eager_kernel<N, SK, TQ>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    k<<<a.B * a.H, kThreads, smem, st>>>(a);
+    return cudaGetLastError();
+}
+template <int N, int TQ>
+inline cudaError_t gdispatch_rk(bool eager, int rk, const GArgs &a, size_t smem, cudaStream_t st) {
+    switch (rk) {
+        case SK_F32: return eager ? glaunch_eager<N, SK_F32, TQ>(a, smem, st) : glaunch_replay<N, SK_F32, TQ>(a, smem, st);
+        case SK_BF16: return eager ? glaunch_eager<N, SK_BF16, TQ>(a, smem, st) : glaunch_replay<N, SK_BF16, TQ>(a, smem, st);
+        default: return eager ? glaunch_eager<N, SK_FP8, TQ>(a, smem, st) : glaunch_replay<N, SK_FP8, TQ>(a, smem, st);
+    }
+}
+template <int N>
+inline cudaError_t gdispatch_tq(bool eager, int rk, int TQ, const GArgs &a, size_t smem, cudaStream_t st) {
+    if (TQ == 1) return gdispatch_rk<N, 1>(eager, rk, a, smem, st);
+    if (TQ == 4) return gdispatch_rk<N, 4>(eager, rk, a, smem, st);
+    return gdispatch_rk<N, 8>(eager, rk, a, smem, st);
+}
+
+// Per-dstate entry point; each instantiation lives in its own translation unit.
+template <int N>
+cudaError_t g_dispatch_n(bool eager, int rk, int TQ, const GArgs &a, size_t smem, cudaStream_t st) {
+    return gdispatch_tq<N>(eager, rk, TQ, a, smem, st);
+}
+
+}  // namespace rssm

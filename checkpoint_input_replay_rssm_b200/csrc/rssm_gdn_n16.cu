@@ -1,0 +1,6 @@
+// Kernel instantiations for dstate = 16.
+#include "rssm_gdn.cuh"
+
+namespace rssm {
+template cudaError_t g_dispatch_n<16>(bool, int, int, const GArgs &, size_t, cudaStream_t);
+}  // namespace rssm

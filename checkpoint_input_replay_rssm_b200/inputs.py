@@ -25,8 +25,6 @@ values (what the oracle consumes) and, via ``to_torch``, in the storage dtype.
 from __future__ import annotations
 
 import dataclasses
-from concurrent.futures import ThreadPoolExecutor
-
 import numpy as np
 
 CONST_TAG = 0xC0_57_A1_7E  # keeps constant streams apart from token streams (t >= 0)
@@ -89,49 +87,50 @@ def _softplus(z: np.ndarray) -> np.ndarray:
 
 
 def round_to(a: np.ndarray, dtype: str) -> np.ndarray:
-    """Round float data to the storage dtype and return it as float64 (exact)."""
+    """Round float data to the storage dtype (via fp32, torch's cast) and return it as
+    float64 holding exactly the rounded values."""
     import torch
 
-    t = torch.from_numpy(np.ascontiguousarray(a, dtype=np.float64))
+    f = np.ascontiguousarray(a, dtype=np.float32)
     if dtype == "f32":
-        t = t.to(torch.float32)
-    elif dtype == "bf16":
-        t = t.to(torch.float32).to(torch.bfloat16)
-    else:
-        raise ValueError(dtype)
-    return t.to(torch.float64).numpy()
+        return f.astype(np.float64)
+    if dtype == "bf16":
+        return torch.from_numpy(f).to(torch.bfloat16).to(torch.float64).numpy()
+    raise ValueError(dtype)
 
 
-def constants(wl: Workload, seqs=None) -> dict:
-    """Per-layer constants and the initial state S_0[seqs] (float64 exact fp32 values)."""
+def constants(wl: Workload, seqs=None, f64: bool = True) -> dict:
+    """Per-layer constants and the initial state S_0[seqs], fp32 values held in
+    float64 (``f64=True``, what the oracle consumes) or in float32."""
     seqs = range(wl.batch) if seqs is None else seqs
     out = {}
     if wl.kind == "mamba2":
         g = _rng(wl.seed, CONST_TAG)
         out["A"] = round_to(-np.exp(g.uniform(0.0, 1.0, wl.nheads)), "f32")
         out["D"] = round_to(g.standard_normal(wl.nheads), "f32")
-    s0 = np.empty((len(seqs), wl.nheads, wl.headdim, wl.dstate))
+    s0 = np.empty((len(seqs), wl.nheads, wl.headdim, wl.dstate), np.float32)
     for i, b in enumerate(seqs):
         s0[i] = _rng(wl.seed, CONST_TAG, b).normal(0.0, wl.state_std,
                                                     (wl.nheads, wl.headdim, wl.dstate))
-    out["S0"] = round_to(s0, "f32")
+    out["S0"] = s0.astype(np.float64) if f64 else s0
     return out
 
 
 def _token_one_seq(wl: Workload, t: int, b: int) -> dict:
     g = _rng(wl.seed, t, b)
     H, P, N = wl.nheads, wl.headdim, wl.dstate
+    f32 = np.float32
     if wl.kind == "mamba2":
         G = wl.ngroups
         return {
-            "x": g.standard_normal((H, P)),
+            "x": g.standard_normal((H, P), dtype=f32),
             "dt": _softplus(g.standard_normal(H) - 2.0),
-            "B": g.standard_normal((G, N)),
-            "C": g.standard_normal((G, N)),
+            "B": g.standard_normal((G, N), dtype=f32),
+            "C": g.standard_normal((G, N), dtype=f32),
         }
-    q = g.standard_normal((H, N))
-    k = g.standard_normal((H, N))
-    v = g.standard_normal((H, P))
+    q = g.standard_normal((H, N), dtype=f32)
+    k = g.standard_normal((H, N), dtype=f32)
+    v = g.standard_normal((H, P), dtype=f32)
     beta = 1.0 / (1.0 + np.exp(-g.standard_normal(H)))
     alpha = np.exp(-_softplus(g.standard_normal(H)))
     q /= np.linalg.norm(q, axis=-1, keepdims=True)
@@ -139,24 +138,15 @@ def _token_one_seq(wl: Workload, t: int, b: int) -> dict:
     return {"q": q, "k": k, "v": v, "beta": beta, "alpha": alpha}
 
 
-_POOL: ThreadPoolExecutor | None = None
-
-
-def token(wl: Workload, t: int, seqs=None, threads: int = 8) -> dict:
+def token(wl: Workload, t: int, seqs=None) -> dict:
     """Inputs of absolute token index t for the given sequences.
 
     Returns float64 arrays shaped [len(seqs), ...] holding the dtype-rounded
     values: Mamba-2 x[b,H,P], dt[b,H], B[b,G,N], C[b,G,N]; GDN q,k[b,H,N],
     v[b,H,P], beta,alpha[b,H].
     """
-    global _POOL
     seqs = list(range(wl.batch)) if seqs is None else list(seqs)
-    if threads > 1 and len(seqs) >= 16:
-        if _POOL is None:
-            _POOL = ThreadPoolExecutor(max_workers=threads)
-        parts = list(_POOL.map(lambda b: _token_one_seq(wl, t, b), seqs))
-    else:
-        parts = [_token_one_seq(wl, t, b) for b in seqs]
+    parts = [_token_one_seq(wl, t, b) for b in seqs]
     out = {k: np.stack([p[k] for p in parts]) for k in parts[0]}
     wide = ("x", "B", "C") if wl.kind == "mamba2" else ("q", "k", "v")
     for k in out:

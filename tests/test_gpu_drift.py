@@ -1,0 +1,89 @@
+"""Dual-precision drift over 4096 decode steps, window sweep (Mamba-2, Nemotron-scale heads).
+
+The ReplaySSM reports keep a high-precision checkpoint for the recurrent update
+and a low-precision copy for reads, so the copy's rounding never re-enters the
+recurrence, unlike a single shared low-precision state whose rounding
+accumulates ("Deux precisions pour le prix d'une", irisproject.cloud).  This
+runs the fp32 checkpoint + per-row e4m3 read copy for W in {4, 8, 16, 32, 64}
+next to the eager single shared fp8 state on the same inputs, and records the
+per-step error against the fp64 oracle.  Eight sequences of 128 heads x 64 x 128
+are decoded (the float comparison subset; every sequence is independent).
+
+Set RSSM_REPORT_DIR to write the per-step error summary as JSON.
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+
+from checkpoint_input_replay_rssm_b200 import inputs as I
+from oracle import eager
+from oracle.replay import ReplayOracle
+from tests.gpu_common import make_layer, oracle_params, rel_err, to_device
+
+pytestmark = pytest.mark.gpu
+
+WINDOWS = (4, 8, 16, 32, 64)
+
+
+def test_fp8_dual_precision_drift_window_sweep():
+    import torch
+
+    wl = I.FP8DRIFT.replace(batch=8)
+    steps = wl.steps
+    c = I.constants(wl)
+    layers = {f"dual_fp8_W{W}": make_layer(wl.replace(window=W), "replay", "fp8")[0] for W in WINDOWS}
+    layers["dual_bf16_W16"] = make_layer(wl, "replay", "bf16")[0]
+    layers["replay_f32_W16"] = make_layer(wl, "replay", "f32")[0]
+    layers["shared_fp8"] = make_layer(wl, "eager", "fp8")[0]
+    layers["shared_bf16"] = make_layer(wl, "eager", "bf16")[0]
+    emu = ReplayOracle("mamba2", c["S0"], 16, params=oracle_params(c), ngroups=wl.ngroups,
+                       read_dtype="fp8")
+    S = np.ascontiguousarray(c["S0"].copy())
+    err = {n: np.zeros(steps) for n in layers}
+    emu_worst = 0.0
+    for t in range(steps):
+        tok = I.token(wl, t)
+        dev = to_device(tok, wl, with_T=False)
+        ys = {n: L.decode(dev) for n, L in layers.items()}
+        y_ref = eager.mamba2_step(S, c["A"], c["D"], tok["x"], tok["dt"], tok["B"], tok["C"])
+        for n, y in ys.items():
+            err[n][t] = rel_err(y[:, 0].double().cpu().numpy(), y_ref)
+        if t < 96:
+            emu_worst = max(emu_worst, rel_err(ys["dual_fp8_W16"][:, 0].double().cpu().numpy(),
+                                               emu.decode(tok)))
+    torch.cuda.synchronize()
+
+    # the GPU's fp8 copy behaves like the emulated e4m3 copy of the same checkpoint
+    assert emu_worst <= 2e-2, emu_worst
+    # rounding of the copy never feeds back: the checkpoint is the fp32 path's, byte for byte
+    ck = {n: layers[n].region("ckpt_off", "ckpt_bytes", torch.int32) for n in
+          ("dual_fp8_W16", "dual_bf16_W16", "replay_f32_W16")}
+    assert torch.equal(ck["dual_fp8_W16"], ck["replay_f32_W16"])
+    assert torch.equal(ck["dual_bf16_W16"], ck["replay_f32_W16"])
+    # the fp32 path stays at fp32 rounding level for 4096 steps
+    assert err["replay_f32_W16"].max() <= 1e-4
+    assert err["dual_bf16_W16"].max() <= 2e-2
+    # no accumulation: the dual path's error level does not grow along the run
+    q = steps // 4
+    for W in WINDOWS:
+        e = err[f"dual_fp8_W{W}"]
+        assert np.median(e[-q:]) <= 1.25 * np.median(e[64:q]) + 1e-3, W
+        assert e.max() < 0.5, W
+
+    report = {
+        "workload": "mamba2 fp8 drift: 8 seqs x 128 heads x 64 x 128, G 8, bf16 inputs, 4096 steps",
+        "metric": "per step max|y - y_fp64| / RMS(y_fp64)",
+        "emulated_fp8_copy_vs_gpu_first96_max": emu_worst,
+        "series": {n: {"median": float(np.median(e)), "p99": float(np.quantile(e, 0.99)),
+                       "max": float(e.max()),
+                       "median_by_quarter": [float(np.median(e[i * q:(i + 1) * q])) for i in range(4)]}
+                   for n, e in err.items()},
+    }
+    out = os.environ.get("RSSM_REPORT_DIR")
+    if out:
+        os.makedirs(out, exist_ok=True)
+        with open(os.path.join(out, "fp8_drift_window_sweep.json"), "w") as f:
+            json.dump(report, f, indent=1)
+    print(json.dumps(report["series"], indent=1))
