@@ -169,7 +169,7 @@ def timed_loop(L, toks_dev, ys, K, W, sync):
     launches = L.launches() - l0
     total_ms = t0.elapsed_time(t1)
     per = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    return total_ms, float(np.mean(per)), launches
+    return total_ms, float(np.mean(per)), launches, per
 
 
 def e2e_loop(L, toks_host, K, W, sync):
@@ -255,8 +255,8 @@ def run_reference(args, rank):
     print(json.dumps(line), flush=True)
 
 
-def workload_config():
-    return {"workload": WL.name, "batch_per_gpu": WL.batch, "nheads": WL.nheads, "headdim": WL.headdim,
+def workload_config(batch=None):
+    return {"workload": WL.name, "batch_per_gpu": batch or WL.batch, "nheads": WL.nheads, "headdim": WL.headdim,
             "dstate": WL.dstate, "ngroups": WL.ngroups, "window": WL.window, "checkpoint": "f32",
             "read_copy": "bf16", "inputs": "bf16",
             "l2": "no flush: the 512 MiB read copy read every step exceeds the 126 MB L2",
@@ -272,6 +272,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-eager", action="store_true", help="skip the eager-baseline leg")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle leg")
+    ap.add_argument("--batch", type=int, default=WL.batch,
+                    help="sequences per GPU (default: the workload's 256; smaller for profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -309,7 +311,7 @@ def main():
     rssm.load()
 
     K, W = args.steps, args.warmup
-    wl = WL.replace(seed=WL.seed + 7919 * rank)
+    wl = WL.replace(seed=WL.seed + 7919 * rank, batch=args.batch)
     consts = I.constants(wl, f64=False)
     n_distinct = min(K + W, 256)
     toks_host = host_tokens(wl, n_distinct)
@@ -320,7 +322,10 @@ def main():
     L = make_layer(wl, "replay", "bf16", consts, device)
     sampler = ClockSampler(local)
     with sampler:
-        total_ms, kern_ms, launches = timed_loop(L, toks_dev, ys, K, W, sync)
+        total_ms, kern_ms, launches, per = timed_loop(L, toks_dev, ys, K, W, sync)
+    fold = [(W + i) >= wl.window and (W + i) % wl.window == 0 for i in range(K)]
+    per_fold = [p for p, f in zip(per, fold) if f]
+    per_read = [p for p, f in zip(per, fold) if not f]
     clocks = sampler.summary()
     t = torch.tensor([total_ms, kern_ms], dtype=torch.float64, device=device)
     if dist is not None:
@@ -354,7 +359,7 @@ def main():
         del L
         torch.cuda.empty_cache()
         E = make_layer(wl, "eager", "f32", consts, device)
-        e_total, e_kern, _ = timed_loop(E, toks_dev, ys, K, W, sync)
+        e_total, e_kern, _, _ = timed_loop(E, toks_dev, ys, K, W, sync)
         t = torch.tensor([e_total, e_kern], dtype=torch.float64, device=device)
         if dist is not None:
             dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -381,13 +386,17 @@ def main():
         "vs_baseline": None,
         "dtype": "f32",
         "data": "synthetic",
-        "config": workload_config() | {"parallelism": f"dp{world} (independent sequences)"},
+        "config": workload_config(wl.batch) | {"parallelism": f"dp{world} (independent sequences)"},
         "hbm_gbs": achieved,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": tr, "peak_source": peak_kind,
                      "kernel": "m2_replay_kernel<128, bf16, 1>",
                      "algorithmic_bytes_per_launch": bytes_per_launch,
-                     "kernel_ms_per_launch": kern_ms},
+                     "kernel_ms_per_launch": kern_ms,
+                     "kernel_ms_fold_step": float(np.mean(per_fold)) if per_fold else None,
+                     "kernel_ms_read_step": float(np.mean(per_read)) if per_read else None,
+                     "read_step_gbs": (traffic.total(traffic.replay_step(shape, wl.window // 2, False))
+                                       * units / (np.mean(per_read) * 1e-3) / 1e9) if per_read else None},
         "e2e": {"value": world * wl.batch * K / (e2e_ms * 1e-3), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches,

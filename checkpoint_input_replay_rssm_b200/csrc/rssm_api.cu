@@ -26,7 +26,8 @@ bool validate(const rssm_config *c, std::string *why) {
     if (c->input_dtype != RSSM_F32 && c->input_dtype != RSSM_BF16) return fail("input_dtype must be F32 or BF16");
     if (c->batch < 1 || c->nheads < 1) return fail("batch and nheads must be >= 1");
     if ((int64_t)c->batch * c->nheads > 0x7fffffffLL) return fail("batch * nheads too large");
-    if (c->headdim < 1 || c->headdim > 256) return fail("headdim must be in 1..256");
+    if (c->headdim < 8 || c->headdim > 256 || c->headdim % 8 != 0)
+        return fail("headdim must be a multiple of 8 in 8..256");
     if (c->dstate != 16 && c->dstate != 32 && c->dstate != 64 && c->dstate != 128)
         return fail("dstate must be 16, 32, 64 or 128");
     if (c->kind == RSSM_MAMBA2 && (c->ngroups < 1 || c->nheads % c->ngroups != 0))
@@ -103,10 +104,15 @@ rssm_status cuda_fail(Ctx *h, cudaError_t e, const char *what) {
     return fail(h, RSSM_ECUDA, m);
 }
 
+bool aligned16(const void *p) { return ((uintptr_t)p & 15) == 0; }
+
 bool inputs_ok(const Ctx *h, const rssm_inputs *in) {
     if (!in) return false;
-    if (h->cfg.kind == RSSM_MAMBA2) return in->x && in->dt && in->Bm && in->Cm;
-    return in->q && in->k && in->v && in->alpha && in->beta;
+    if (h->cfg.kind == RSSM_MAMBA2)
+        return in->x && in->dt && in->Bm && in->Cm && aligned16(in->x) && aligned16(in->Bm) &&
+               aligned16(in->Cm);
+    return in->q && in->k && in->v && in->alpha && in->beta && aligned16(in->q) &&
+           aligned16(in->k) && aligned16(in->v);
 }
 
 cudaError_t launch_kind(Ctx *h, int op, int T, const rssm_inputs *in, float *y, float *out) {
@@ -219,7 +225,7 @@ rssm_status rssm_decode(rssm_handle hh, const rssm_inputs *in, float *y) {
     Ctx *h = (Ctx *)hh;
     if (!h) return RSSM_EINVAL;
     if (h->pending) return fail(h, RSSM_ESTATE, "decode while a verify is pending (commit first)");
-    if (!inputs_ok(h, in) || !y) return fail(h, RSSM_EINVAL, "missing input or output pointer");
+    if (!inputs_ok(h, in) || !y) return fail(h, RSSM_EINVAL, "missing or misaligned input/output pointer (device arrays must be 16-byte aligned)");
     cudaError_t e = launch_kind(h, rssm::OP_DECODE, 1, in, y, nullptr);
     return e == cudaSuccess ? RSSM_OK : cuda_fail(h, e, "decode launch");
 }
@@ -230,7 +236,7 @@ rssm_status rssm_verify(rssm_handle hh, int32_t K, const rssm_inputs *in, float 
     if (h->pending) return fail(h, RSSM_ESTATE, "verify while a verify is pending (commit first)");
     if (K < 1 || K > h->cfg.max_draft || K > h->cfg.window)
         return fail(h, RSSM_EINVAL, "K must be in 1..min(max_draft, window)");
-    if (!inputs_ok(h, in) || !y) return fail(h, RSSM_EINVAL, "missing input or output pointer");
+    if (!inputs_ok(h, in) || !y) return fail(h, RSSM_EINVAL, "missing or misaligned input/output pointer (device arrays must be 16-byte aligned)");
     cudaError_t e = launch_kind(h, rssm::OP_VERIFY, K, in, y, nullptr);
     if (e != cudaSuccess) return cuda_fail(h, e, "verify launch");
     h->pending = K;

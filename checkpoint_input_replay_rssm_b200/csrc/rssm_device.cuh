@@ -221,3 +221,34 @@ __device__ __forceinline__ void arrive_and_publish(const Counters &c, int b, int
 }
 
 }  // namespace rssm
+
+namespace rssm {
+
+// 16-byte global -> shared copy that bypasses registers (Ampere-style cp.async;
+// completion is awaited with cp_async_wait_all + __syncthreads).
+__device__ __forceinline__ void cp_async16(void *smem, const void *gmem) {
+    const unsigned s = (unsigned)__cvta_generic_to_shared(smem);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(s), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+    asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
+// Element i of a raw input-dtype buffer (shared or global) as fp32.
+__device__ __forceinline__ float raw_f(const void *p, int i, int bf16) {
+    return bf16 ? bf16_bits_to_float(reinterpret_cast<const uint16_t *>(p)[i])
+                : reinterpret_cast<const float *>(p)[i];
+}
+
+// Inclusive prefix sum over the warp of one value per lane.
+__device__ __forceinline__ float warp_incl_scan(float v) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const float u = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += u;
+    }
+    return v;
+}
+
+}  // namespace rssm

@@ -11,11 +11,22 @@ extern template cudaError_t m2_dispatch_n<128>(bool, int, int, const M2Args &, s
 
 static int tq_of(int T) { return T <= 1 ? 1 : (T <= 4 ? 4 : 8); }
 
+// Heads per replay CTA: the largest of 4, 2, 1 that divides the heads of a group
+// and keeps the CTA's shared memory within 160 KiB.
+static int m2_heads_per_cta(const rssm_config &cf, int TQ) {
+    const int hpg = cf.nheads / cf.ngroups, ib = cf.input_dtype == RSSM_BF16 ? 2 : 4;
+    for (int hc = 4; hc > 1; hc >>= 1)
+        if (hpg % hc == 0 && m2_lay(hc, cf.headdim, cf.dstate, cf.window, TQ, ib).total <= 160 * 1024)
+            return hc;
+    return 1;
+}
+
 size_t mamba2_smem_bytes(const rssm_config &cf, int T) {
     const int TQ = tq_of(T), P = cf.headdim, N = cf.dstate;
     if (cf.mode == RSSM_EAGER)
         return sizeof(float) * ((size_t)2 * pad4(TQ * P) + 2 * pad4(TQ * N) + 2 * pad4(TQ));
-    return sizeof(float) * m2_smem_floats(P, N, cf.window, TQ);
+    const int ib = cf.input_dtype == RSSM_BF16 ? 2 : 4;
+    return (size_t)m2_lay(m2_heads_per_cta(cf, TQ), P, N, cf.window, TQ, ib).total;
 }
 
 cudaError_t mamba2_launch(const Ctx &h, int op, int T, const rssm_inputs *in, float *y, float *out,
@@ -25,6 +36,7 @@ cudaError_t mamba2_launch(const Ctx &h, int op, int T, const rssm_inputs *in, fl
     a.B = cf.batch; a.H = cf.nheads; a.P = cf.headdim; a.G = cf.ngroups; a.W = cf.window;
     a.R = (int)h.lay.ring; a.T = T; a.op = op; a.in_bf16 = cf.input_dtype == RSSM_BF16;
     a.dt_scales = cf.dt_scales_input;
+    a.HC = m2_heads_per_cta(cf, tq_of(T));
     a.c = h.counters();
     a.A = (const float *)h.at(h.lay.A_off); a.D = (const float *)h.at(h.lay.D_off);
     a.ckpt = h.lay.ckpt_bytes ? (float *)h.at(h.lay.ckpt_off) : nullptr;

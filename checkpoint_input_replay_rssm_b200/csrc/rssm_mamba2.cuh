@@ -29,6 +29,7 @@ namespace rssm {
 
 struct M2Args {
     int B, H, P, G, W, R, T, op, in_bf16, dt_scales;
+    int HC;             // heads per replay CTA (divides H / G)
     Counters c;
     const float *A, *D;
     float *ckpt;        // fp32 [B][H][P][N]
@@ -48,195 +49,267 @@ struct M2Args {
     float *out;         // export target [B][H][P][N]
 };
 
-// Shared-memory carve-up for one CTA (floats unless noted).
-struct M2Smem {
-    float *sx, *sB, *sC, *sdot, *slam, *sdt, *su, *scoef, *sdec;
-    int *si;
+// Shared-memory layout of the replay kernel, in bytes; every region 16-byte aligned.
+// E = W + TQ entry slots: committed entries sit right-aligned before slot W, the
+// tokens of this call at W..W+T-1, so an entry's slot is (W - L0) + its index.
+struct M2Lay {
+    int sx, sB, sC, sCf, sdt, slam, sd, scoef, sdec, sdot, su, ssc, si, total;
 };
-
-// Regions are padded to multiples of 4 floats so every one is 16-byte aligned.
+__host__ __device__ constexpr int a16(int v) { return (v + 15) & ~15; }
 __host__ __device__ constexpr int pad4(int n) { return (n + 3) & ~3; }
-
-__host__ __device__ inline size_t m2_smem_floats(int P, int N, int W, int TQ) {
+__host__ __device__ inline M2Lay m2_lay(int HC, int P, int N, int W, int TQ, int ib) {
     const int E = W + TQ;
-    return (size_t)pad4(E * P) + pad4(E * N) + pad4(TQ * N) + pad4(TQ * P) + 3 * (size_t)pad4(E) +
-           pad4(TQ * E) + pad4(TQ) + 8;
-}
-
-__device__ __forceinline__ M2Smem m2_carve(float *sm, int P, int N, int W, int TQ) {
-    const int E = W + TQ;
-    M2Smem s;
-    s.sx = sm;                           // [E][P]    x of entries (physical index)
-    s.sB = s.sx + pad4(E * P);           // [E][N]    B of entries
-    s.sC = s.sB + pad4(E * N);           // [TQ][N]   C of the query tokens
-    s.sdot = s.sC + pad4(TQ * N);        // [TQ][P]   S^ C per row
-    s.slam = s.sdot + pad4(TQ * P);      // [E]       prefix sums of log decay
-    s.sdt = s.slam + pad4(E);            // [E]       dt of entries
-    s.su = s.sdt + pad4(E);              // [E]       fold weights
-    s.scoef = s.su + pad4(E);            // [TQ][E]   replay coefficients (logical entry index)
-    s.sdec = s.scoef + pad4(TQ * E);     // [TQ]      decay applied to S^ C
-    s.si = reinterpret_cast<int *>(s.sdec + pad4(TQ));
-    return s;
+    M2Lay L{};
+    int o = 0;
+    L.sx = o;    o += a16(HC * E * P * ib);   // raw x of entries      [HC][E][P]
+    L.sB = o;    o += a16(E * N * ib);        // raw B of entries      [E][N]
+    L.sC = o;    o += a16(TQ * N * ib);       // raw C of the queries  [TQ][N]
+    L.sCf = o;   o += a16(TQ * N * 4);        // C as fp32             [TQ][N]
+    L.sdt = o;   o += a16(HC * E * 4);        // dt of entries         [HC][E]
+    L.slam = o;  o += a16(HC * E * 4);        // prefix sums of dt*A   [HC][E]
+    L.sd = o;    o += a16(TQ * E * 4);        // B_e . C_m             [TQ][E]
+    L.scoef = o; o += a16(HC * TQ * E * 4);   // replay coefficients   [HC][TQ][E]
+    L.sdec = o;  o += a16(HC * TQ * 4);       // decay of S^ C         [HC][TQ]
+    L.sdot = o;  o += a16(HC * P * TQ * 4);   // S^ C per state row    [HC*P][TQ]
+    L.su = o;    o += a16(HC * E * 4);        // fold weights          [HC][E]
+    L.ssc = o;   o += a16(HC * P * 4);        // fp8 row scales        [HC*P]
+    L.si = o;    o += 32;                     // counters of the sequence
+    L.total = o;
+    return L;
 }
 
 // ---------------------------------------------------------------------------
 // Replay kernel: decode (T = 1), verify (T = K), flush (T = 0), export (T = 0).
+//
+// One CTA per (sequence b, group g, chunk of HC heads of the group).  The HC
+// heads' state tiles are contiguous, so the CTA streams one block of
+// HC * P * N elements.  Timeline:
+//   1. every thread issues its read-copy chunks (128-bit, L1 no-allocate) --
+//      up to MAXC per thread, all in flight at once;
+//   2. thread 0 reads the sequence counters while cp.async stages the call's
+//      own tokens (C, B, x, dt) in shared memory;
+//   3. one cp.async batch stages the L0 buffered entries (B of the group, x and
+//      dt of the HC heads);
+//   4. warps compute B_e . C_m once for the group and the prefix sums of the log
+//      decays per head (warp scans), then the replay coefficients;
+//   5. the read-copy rows are dotted with C (or, on a fold step, the fp32
+//      checkpoint rows are folded, stored with the requantised copy and dotted);
+//   6. outputs, ring appends; the last CTA of the sequence publishes counters.
 // ---------------------------------------------------------------------------
 template <int N, int RK, int TQ>
-__global__ void __launch_bounds__(kThreads) m2_replay_kernel(const M2Args a) {
+__global__ void __launch_bounds__(kThreads, 2) m2_replay_kernel(const M2Args a) {
     constexpr int EPC = Chunk<RK>::EPC;    // stored elements per 16-byte chunk
-    constexpr int TPR = N / EPC;           // threads per row, read mapping
-    constexpr int RPP = kThreads / TPR;    // rows per pass, read mapping
-    constexpr int RB = 8;                  // rows per thread per batch
-    constexpr int TPR4 = N / 4;            // threads per row, fp32 (quad) mapping
+    constexpr int TPR = N / EPC;           // lanes per state row, read mapping
+    constexpr int MAXC = (TQ == 1) ? 16 : (TQ == 4 ? 8 : 4);  // read-copy chunks in flight per thread
+    constexpr int TPR4 = N / 4;            // lanes per row, fp32 quad mapping (fold)
     constexpr int RPP4 = kThreads / TPR4;
+    constexpr int RB4 = 8;
     static_assert(TPR >= 1 && TPR <= 32 && (32 % TPR) == 0, "row must fit a warp");
-    static_assert(TPR4 >= 1 && TPR4 <= 32, "row must fit a warp");
 
-    extern __shared__ __align__(16) float smem[];
+    extern __shared__ __align__(16) uint8_t smraw[];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int bh = blockIdx.x;
-    const int H = a.H, P = a.P, W = a.W, R = a.R, T = a.T, G = a.G;
-    const int b = bh / H, h = bh - b * H;
-    const int hpg = H / G, g = h / hpg;
+    const int H = a.H, P = a.P, W = a.W, R = a.R, T = a.T, G = a.G, HC = a.HC;
+    const int hpg = H / G, cpg = hpg / HC;
+    const int b = blockIdx.x / (G * cpg);
+    const int rem = blockIdx.x - b * G * cpg;
+    const int g = rem / cpg, hc = rem - g * cpg;
+    const int h0 = g * hpg + hc * HC;
     const int E = W + TQ;
-    M2Smem s = m2_carve(smem, P, N, W, TQ);
-    const int64_t tile0 = (int64_t)bh * P * N;
+    const int bf = a.in_bf16, ib = bf ? 2 : 4;
+    const M2Lay Ly = m2_lay(HC, P, N, W, TQ, ib);
+    uint8_t *sx = smraw + Ly.sx;
+    uint8_t *sB = smraw + Ly.sB;
+    uint8_t *sC = smraw + Ly.sC;
+    float *sCf = reinterpret_cast<float *>(smraw + Ly.sCf);
+    float *sdt = reinterpret_cast<float *>(smraw + Ly.sdt);
+    float *slam = reinterpret_cast<float *>(smraw + Ly.slam);
+    float *sd = reinterpret_cast<float *>(smraw + Ly.sd);
+    float *scoef = reinterpret_cast<float *>(smraw + Ly.scoef);
+    float *sdec = reinterpret_cast<float *>(smraw + Ly.sdec);
+    float *sdot = reinterpret_cast<float *>(smraw + Ly.sdot);
+    float *su = reinterpret_cast<float *>(smraw + Ly.su);
+    float *ssc = reinterpret_cast<float *>(smraw + Ly.ssc);
+    int *si = reinterpret_cast<int *>(smraw + Ly.si);
+    const int64_t row0 = (int64_t)b * H + h0;  // (b, h0)
+    const int64_t tile0 = row0 * P * N;        // first state element of the CTA
+    const int nrows = HC * P;
+    const int nchunks = nrows * TPR;
     const bool reads = (a.op == OP_DECODE || a.op == OP_VERIFY);
+    const int c = tid % TPR;
+    const int xrow = P * ib, brow = N * ib;   // bytes of an x row / a B or C row
+    const int xch = xrow / 16, bch = brow / 16;
 
-    // 1. Read-copy loads first: they do not depend on the counters, and on the
-    //    steps that fold they are simply dropped.
-    const int c = tid % TPR, r0 = tid / TPR;
-    const uint8_t *rc_tile =
+    // 1. Read-copy chunks first (dropped on fold steps).
+    const uint8_t *rc_base =
         (RK == SK_F32) ? reinterpret_cast<const uint8_t *>(a.ckpt + tile0)
                        : reinterpret_cast<const uint8_t *>(a.rc) + tile0 * Chunk<RK>::BYTES;
-    uint4 rv[RB];
-    float rscale[RB];
+    uint4 rv[MAXC];
     if (reads) {
 #pragma unroll
-        for (int k = 0; k < RB; ++k) {
-            const int r = r0 + k * RPP;
-            if (r < P) rv[k] = ld_stream(rc_tile + ((size_t)r * TPR + c) * 16);
-            if (RK == SK_FP8) rscale[k] = (r < P) ? __ldg(a.rc_scale + (int64_t)bh * P + r) : 0.f;
+        for (int j = 0; j < MAXC; ++j) {
+            const int idx = tid + kThreads * j;
+            if (idx < nchunks) rv[j] = ld_stream(rc_base + (size_t)idx * 16);
         }
+        if (RK == SK_FP8)  // the CTA's row scales, contiguous: HC * P floats
+            for (int i = tid; i < nrows / 4; i += kThreads)
+                cp_async16(ssc + 4 * i, a.rc_scale + row0 * P + 4 * i);
     }
 
-    // 2. Counters (thread 0), and the new tokens' inputs (independent of them).
+    // 2. Counters (thread 0) and this call's tokens.
     if (tid == 0) {
         SeqState ss = read_counters(a.c, b, W);
         const int L0 = (int)(ss.seq - ss.ckpt);
         int flush = 0;
         if (ss.ok) flush = (a.op == OP_FLUSH || a.op == OP_EXPORT) ? (L0 > 0) : (L0 + T > W);
-        s.si[0] = ss.ok;
-        s.si[1] = ss.ok ? L0 : 0;
-        s.si[2] = flush;
-        s.si[3] = (int)(ss.ckpt % R);
-        s.si[4] = (int)(ss.seq % R);
+        si[0] = ss.ok;
+        si[1] = ss.ok ? L0 : 0;
+        si[2] = flush;
+        si[3] = (int)(ss.ckpt % R);
+        si[4] = (int)(ss.seq % R);
         if (!ss.ok) {
-            if (h == 0) report(a.c.err, DEV_BAD_COUNTERS, b, h, (int)(ss.seq - ss.ckpt));
+            if (g == 0 && hc == 0) report(a.c.err, DEV_BAD_COUNTERS, b, h0, (int)(ss.seq - ss.ckpt));
         } else if (a.op != OP_EXPORT) {
             const int64_t new_seq = (a.op == OP_DECODE) ? ss.seq + 1 : -1;
             const int64_t new_ckpt = flush ? ss.seq : -1;
             const int new_pending = (a.op == OP_VERIFY) ? T : -1;
-            arrive_and_publish(a.c, b, H, new_seq, new_ckpt, new_pending, flush);
+            arrive_and_publish(a.c, b, H / HC, new_seq, new_ckpt, new_pending, flush);
         }
     }
-    for (int i = tid; i < T * P; i += kThreads) {
-        const int m = i / P, p = i - m * P;
-        s.sx[(W + m) * P + p] = ld_in(a.x, ((int64_t)(b * T + m) * H + h) * P + p, a.in_bf16);
+    for (int i = tid; i < T * bch; i += kThreads) {
+        const int m = i / bch, k = i - m * bch;
+        const int64_t src = (((int64_t)(b * T + m) * G + g) * N) * ib + k * 16;
+        cp_async16(sC + m * brow + k * 16, reinterpret_cast<const uint8_t *>(a.Cm) + src);
+        cp_async16(sB + (W + m) * brow + k * 16, reinterpret_cast<const uint8_t *>(a.Bm) + src);
     }
-    for (int i = tid; i < T * N; i += kThreads) {
-        const int m = i / N, n = i - m * N;
-        const int64_t src = ((int64_t)(b * T + m) * G + g) * N + n;
-        s.sB[(W + m) * N + n] = ld_in(a.Bm, src, a.in_bf16);
-        s.sC[m * N + n] = ld_in(a.Cm, src, a.in_bf16);
+    for (int i = tid; i < T * HC * xch; i += kThreads) {
+        const int m = i / (HC * xch), r2 = i - m * HC * xch;
+        const int hh = r2 / xch, k = r2 - hh * xch;
+        cp_async16(sx + (hh * E + W + m) * xrow + k * 16,
+                   reinterpret_cast<const uint8_t *>(a.x) + (((int64_t)(b * T + m) * H + h0 + hh) * P) * ib + k * 16);
     }
-    if (tid < T) s.sdt[W + tid] = a.dt[(int64_t)(b * T + tid) * H + h];
+    if (tid < T * HC) {
+        const int m = tid / HC, hh = tid - m * HC;
+        sdt[hh * E + W + m] = a.dt[(int64_t)(b * T + m) * H + h0 + hh];
+    }
     __syncthreads();
-    if (!s.si[0]) return;  // counters corrupted: error reported, sequence skipped
-    const int L0 = s.si[1], flush = s.si[2], ckmod = s.si[3], spmod = s.si[4];
-    const int base = W - L0;  // buffered entries sit right-aligned before the new tokens
+    if (!si[0]) {  // counters corrupted: error reported, sequence skipped
+        cp_async_wait_all();
+        return;
+    }
+    const int L0 = si[1], flush = si[2], ckmod = si[3], spmod = si[4];
+    const int base = W - L0;
     const int nE = L0 + T;
 
-    // 3. Buffered entries (logical 0..L0-1 -> physical base..W-1).
-    for (int i = tid; i < L0 * P; i += kThreads) {
-        const int e = i / P, p = i - e * P;
+    // 3. Buffered entries, one cp.async batch.
+    for (int i = tid; i < L0 * bch; i += kThreads) {
+        const int e = i / bch, k = i - e * bch;
         const int slot = (ckmod + e) % R;
-        s.sx[(base + e) * P + p] = ld_in(a.xbuf, ((int64_t)bh * R + slot) * P + p, a.in_bf16);
+        cp_async16(sB + (base + e) * brow + k * 16,
+                   reinterpret_cast<const uint8_t *>(a.Bbuf) + (((int64_t)(b * G + g) * R + slot) * N) * ib + k * 16);
     }
-    for (int i = tid; i < L0 * N; i += kThreads) {
-        const int e = i / N, n = i - e * N;
+    for (int i = tid; i < HC * L0 * xch; i += kThreads) {
+        const int hh = i / (L0 * xch), r2 = i - hh * L0 * xch;
+        const int e = r2 / xch, k = r2 - e * xch;
         const int slot = (ckmod + e) % R;
-        s.sB[(base + e) * N + n] = ld_in(a.Bbuf, ((int64_t)(b * G + g) * R + slot) * N + n, a.in_bf16);
+        cp_async16(sx + (hh * E + base + e) * xrow + k * 16,
+                   reinterpret_cast<const uint8_t *>(a.xbuf) + (((row0 + hh) * R + slot) * P) * ib + k * 16);
     }
-    for (int e = tid; e < L0; e += kThreads) s.sdt[base + e] = a.dtbuf[(int64_t)bh * R + (ckmod + e) % R];
+    for (int i = tid; i < HC * L0; i += kThreads) {
+        const int hh = i / L0, e = i - hh * L0;
+        sdt[hh * E + base + e] = a.dtbuf[(row0 + hh) * R + (ckmod + e) % R];
+    }
+    cp_async_wait_all();
     __syncthreads();
 
-    // 4. Prefix sums of the log decays, fold weights, replay coefficients.
-    const float Ah = a.A[h];
-    if (tid == 0) {
-        float acc = 0.f;
-        for (int e = 0; e < nE; ++e) {
-            acc += s.sdt[base + e] * Ah;
-            s.slam[base + e] = acc;
-        }
-    }
-    __syncthreads();
+    // 4. B_e . C_m for the group (warps), prefix sums of dt*A per head (warp scans).
     const int e0 = flush ? L0 : 0;  // first entry the outputs replay
-    const float lam_fold = (L0 > 0) ? s.slam[base + L0 - 1] : 0.f;
-    const float lam_base = flush ? lam_fold : 0.f;
-    if (flush) {
-        for (int e = tid; e < L0; e += kThreads)
-            s.su[e] = expf(lam_fold - s.slam[base + e]) * (a.dt_scales ? s.sdt[base + e] : 1.f);
-    }
     if (reads) {
-        const int npairs = T * nE;
-        for (int pr = warp; pr < npairs; pr += kWarps) {
+        for (int pr = warp; pr < T * nE; pr += kWarps) {
             const int m = pr / nE, e = pr - m * nE;
             if (e < e0 || e > L0 + m) continue;  // warp-uniform
             float d = 0.f;
-            for (int n = lane; n < N; n += 32) d += s.sB[(base + e) * N + n] * s.sC[m * N + n];
+            for (int n = lane; n < N; n += 32)
+                d = fmaf(raw_f(sB + (base + e) * brow, n, bf), raw_f(sC + m * brow, n, bf), d);
             d = group_sum<32>(d);
-            if (lane == 0)
-                s.scoef[m * E + e] = expf(s.slam[base + L0 + m] - s.slam[base + e]) * d *
-                                     (a.dt_scales ? s.sdt[base + e] : 1.f);
+            if (lane == 0) sd[m * E + e] = d;
         }
-        if (tid < T) s.sdec[tid] = expf(s.slam[base + L0 + tid] - lam_base);
+    }
+    for (int i = tid; i < T * N; i += kThreads) sCf[i] = raw_f(sC, i, bf);
+    for (int hh = warp; hh < HC; hh += kWarps) {
+        const float Ah = a.A[h0 + hh];
+        float carry = 0.f;
+        for (int k0 = 0; k0 < nE; k0 += 32) {
+            const int e = k0 + lane;
+            float v = (e < nE) ? sdt[hh * E + base + e] * Ah : 0.f;
+            v = warp_incl_scan(v) + carry;
+            if (e < nE) slam[hh * E + base + e] = v;
+            carry = __shfl_sync(0xffffffffu, v, 31);
+        }
+    }
+    __syncthreads();
+    if (reads) {
+        for (int i = tid; i < HC * T * nE; i += kThreads) {
+            const int hh = i / (T * nE), r2 = i - hh * T * nE;
+            const int m = r2 / nE, e = r2 - m * nE;
+            if (e < e0 || e > L0 + m) continue;
+            const float* lam = slam + hh * E + base;
+            scoef[(hh * TQ + m) * E + e] = expf(lam[L0 + m] - lam[e]) * sd[m * E + e] *
+                                           (a.dt_scales ? sdt[hh * E + base + e] : 1.f);
+        }
+        for (int i = tid; i < HC * T; i += kThreads) {
+            const int hh = i / T, m = i - hh * T;
+            const float* lam = slam + hh * E + base;
+            sdec[hh * TQ + m] = expf(lam[L0 + m] - (flush ? lam[L0 - 1] : 0.f));
+        }
+    }
+    if (flush) {
+        for (int i = tid; i < HC * L0; i += kThreads) {
+            const int hh = i / L0, e = i - hh * L0;
+            const float* lam = slam + hh * E + base;
+            su[hh * E + e] = expf(lam[L0 - 1] - lam[e]) * (a.dt_scales ? sdt[hh * E + base + e] : 1.f);
+        }
     }
     __syncthreads();
 
     if (flush) {
         // 5a. Fold: fp32 checkpoint rows in quads, TPR4 lanes per row.
         const int c4 = tid % TPR4, q0 = tid / TPR4;
-        const float dec_all = expf(lam_fold);
         float4 Cq[TQ];
 #pragma unroll
-        for (int m = 0; m < TQ; ++m)
-            Cq[m] = (reads && m < T) ? reinterpret_cast<const float4 *>(s.sC + m * N)[c4]
-                                     : make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int rb = 0; rb < P; rb += RB * RPP4) {
-            float4 st[RB];
+        for (int m = 0; m < TQ; ++m) {
+            Cq[m] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (reads && m < T)
+                Cq[m] = make_float4(raw_f(sC + m * brow, 4 * c4, bf), raw_f(sC + m * brow, 4 * c4 + 1, bf),
+                                    raw_f(sC + m * brow, 4 * c4 + 2, bf), raw_f(sC + m * brow, 4 * c4 + 3, bf));
+        }
+        for (int rb = 0; rb < nrows; rb += RB4 * RPP4) {
+            float4 st[RB4];
 #pragma unroll
-            for (int k = 0; k < RB; ++k) {
-                const int r = rb + q0 + k * RPP4;
-                st[k] = (r < P) ? load_quad<SK_F32>(a.ckpt, tile0 + (int64_t)r * N + 4 * c4)
-                                : make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int k = 0; k < RB4; ++k) {
+                const int gr = rb + q0 + k * RPP4;
+                st[k] = (gr < nrows) ? load_quad<SK_F32>(a.ckpt, tile0 + (int64_t)gr * N + 4 * c4)
+                                     : make_float4(0.f, 0.f, 0.f, 0.f);
             }
 #pragma unroll
-            for (int k = 0; k < RB; ++k) {
-                const int r = rb + q0 + k * RPP4;
-                const bool valid = r < P;
+            for (int k = 0; k < RB4; ++k) {
+                const int gr = rb + q0 + k * RPP4;
+                const bool valid = gr < nrows;
+                const int hh = valid ? gr / P : 0, p = valid ? gr - hh * P : 0;
                 float4 v = st[k];
-                v.x *= dec_all; v.y *= dec_all; v.z *= dec_all; v.w *= dec_all;
                 if (valid) {
+                    const float* lam = slam + hh * E + base;
+                    const float dec_all = expf(lam[L0 - 1]);
+                    v.x *= dec_all; v.y *= dec_all; v.z *= dec_all; v.w *= dec_all;
                     for (int e = 0; e < L0; ++e) {
-                        const float w = s.su[e] * s.sx[(base + e) * P + r];
-                        const float4 Bq = reinterpret_cast<const float4 *>(s.sB + (base + e) * N)[c4];
-                        v.x = fmaf(w, Bq.x, v.x); v.y = fmaf(w, Bq.y, v.y);
-                        v.z = fmaf(w, Bq.z, v.z); v.w = fmaf(w, Bq.w, v.w);
+                        const float w = su[hh * E + e] * raw_f(sx + (hh * E + base + e) * xrow, p, bf);
+                        const uint8_t *Br = sB + (base + e) * brow;
+                        v.x = fmaf(w, raw_f(Br, 4 * c4, bf), v.x);
+                        v.y = fmaf(w, raw_f(Br, 4 * c4 + 1, bf), v.y);
+                        v.z = fmaf(w, raw_f(Br, 4 * c4 + 2, bf), v.z);
+                        v.w = fmaf(w, raw_f(Br, 4 * c4 + 3, bf), v.w);
                     }
                 }
-                const int64_t el = tile0 + (int64_t)(valid ? r : 0) * N + 4 * c4;
+                const int64_t el = tile0 + (int64_t)(valid ? gr : 0) * N + 4 * c4;
                 if (a.op == OP_EXPORT) {
                     if (valid) *reinterpret_cast<float4 *>(a.out + el) = v;
                     continue;
@@ -251,7 +324,7 @@ __global__ void __launch_bounds__(kThreads) m2_replay_kernel(const M2Args a) {
                     const float sc = fp8_scale(am);
                     if (valid) {
                         rd = store_quad<SK_FP8>(a.rc, el, v, 0.f, sc);
-                        if (c4 == 0) a.rc_scale[(int64_t)bh * P + r] = sc;
+                        if (c4 == 0) a.rc_scale[row0 * P + gr] = sc;
                     }
                 }
                 if (reads) {
@@ -259,44 +332,54 @@ __global__ void __launch_bounds__(kThreads) m2_replay_kernel(const M2Args a) {
                     for (int m = 0; m < TQ; ++m) {
                         float d = rd.x * Cq[m].x + rd.y * Cq[m].y + rd.z * Cq[m].z + rd.w * Cq[m].w;
                         d = group_sum<TPR4>(d);
-                        if (c4 == 0 && valid && m < T) s.sdot[m * P + r] = d;
+                        if (c4 == 0 && valid && m < T) sdot[gr * TQ + m] = d;
                     }
                 }
             }
         }
     } else if (reads) {
-        // 5b. Read: dot products of the read-copy rows with the query C's.
-        float Cr[TQ][EPC];
+        // 5b. Read: dot products of the read-copy rows with the query C's (held in
+        // registers when they fit, else read from shared memory).
+        constexpr bool kCregs = TQ * EPC <= 64;
+        float Cr[kCregs ? TQ : 1][kCregs ? EPC : 1];
+        if (kCregs) {
 #pragma unroll
-        for (int m = 0; m < TQ; ++m)
+            for (int m = 0; m < (kCregs ? TQ : 1); ++m)
 #pragma unroll
-            for (int j = 0; j < EPC; ++j) Cr[m][j] = (m < T) ? s.sC[m * N + c * EPC + j] : 0.f;
-        for (int rb = 0; rb < P; rb += RB * RPP) {
-            if (rb > 0) {
+                for (int j = 0; j < (kCregs ? EPC : 1); ++j)
+                    Cr[m][j] = (m < T) ? sCf[m * N + c * EPC + j] : 0.f;
+        }
+        for (int r0 = 0; r0 < nchunks; r0 += MAXC * kThreads) {
+            if (r0 > 0) {
 #pragma unroll
-                for (int k = 0; k < RB; ++k) {
-                    const int r = rb + r0 + k * RPP;
-                    if (r < P) rv[k] = ld_stream(rc_tile + ((size_t)r * TPR + c) * 16);
-                    if (RK == SK_FP8) rscale[k] = (r < P) ? __ldg(a.rc_scale + (int64_t)bh * P + r) : 0.f;
+                for (int j = 0; j < MAXC; ++j) {
+                    const int idx = r0 + tid + kThreads * j;
+                    if (idx < nchunks) rv[j] = ld_stream(rc_base + (size_t)idx * 16);
                 }
             }
 #pragma unroll
-            for (int k = 0; k < RB; ++k) {
-                const int r = rb + r0 + k * RPP;
+            for (int j = 0; j < MAXC; ++j) {
+                const int idx = r0 + tid + kThreads * j;
+                const bool valid = idx < nchunks;
                 float v[EPC];
-                if (r < P) unpack<RK>(rv[k], v);
+                if (valid) unpack<RK>(rv[j], v);
                 else {
 #pragma unroll
-                    for (int j = 0; j < EPC; ++j) v[j] = 0.f;
+                    for (int q = 0; q < EPC; ++q) v[q] = 0.f;
                 }
 #pragma unroll
                 for (int m = 0; m < TQ; ++m) {
                     float d = 0.f;
+                    if (kCregs) {
 #pragma unroll
-                    for (int j = 0; j < EPC; ++j) d = fmaf(v[j], Cr[m][j], d);
+                        for (int q = 0; q < EPC; ++q) d = fmaf(v[q], Cr[kCregs ? m : 0][kCregs ? q : 0], d);
+                    } else {
+#pragma unroll
+                        for (int q = 0; q < EPC; ++q) d = fmaf(v[q], sCf[m * N + c * EPC + q], d);
+                    }
                     d = group_sum<TPR>(d);
-                    if (RK == SK_FP8) d *= rscale[k];
-                    if (c == 0 && r < P && m < T) s.sdot[m * P + r] = d;
+                    if (c == 0 && valid && m < T)
+                        sdot[(idx / TPR) * TQ + m] = (RK == SK_FP8) ? d * ssc[idx / TPR] : d;
                 }
             }
         }
@@ -304,30 +387,34 @@ __global__ void __launch_bounds__(kThreads) m2_replay_kernel(const M2Args a) {
     if (!reads) return;
     __syncthreads();
 
-    // 6. Outputs y[b, m, h, :].
-    const float Dh = a.D[h];
-    for (int i = tid; i < T * P; i += kThreads) {
-        const int m = i / P, p = i - m * P;
-        float yv = s.sdec[m] * s.sdot[m * P + p];
-        for (int e = e0; e <= L0 + m; ++e) yv = fmaf(s.scoef[m * E + e], s.sx[(base + e) * P + p], yv);
-        yv = fmaf(Dh, s.sx[(W + m) * P + p], yv);
-        a.y[((int64_t)(b * T + m) * H + h) * P + p] = yv;
+    // 6. Outputs y[b, m, h0 + hh, :] and ring appends (slots seq_pos + m mod R).
+    for (int i = tid; i < T * HC * P; i += kThreads) {
+        const int m = i / (HC * P), r2 = i - m * HC * P;
+        const int hh = r2 / P, p = r2 - hh * P;
+        float yv = sdec[hh * TQ + m] * sdot[(hh * P + p) * TQ + m];
+        const float *cf = scoef + (hh * TQ + m) * E;
+        const uint8_t *xs = sx + (hh * E + base) * xrow;
+        for (int e = e0; e <= L0 + m; ++e) yv = fmaf(cf[e], raw_f(xs + e * xrow, p, bf), yv);
+        yv = fmaf(a.D[h0 + hh], raw_f(sx + (hh * E + W + m) * xrow, p, bf), yv);
+        a.y[((int64_t)(b * T + m) * H + h0 + hh) * P + p] = yv;
     }
-
-    // 7. Append the new tokens to the ring (slots seq_pos + m mod R).
-    for (int i = tid; i < T * P; i += kThreads) {
-        const int m = i / P, p = i - m * P;
+    for (int i = tid; i < T * HC * xch; i += kThreads) {
+        const int m = i / (HC * xch), r2 = i - m * HC * xch;
+        const int hh = r2 / xch, k = r2 - hh * xch;
         const int slot = (spmod + m) % R;
-        copy_in(a.xbuf, ((int64_t)bh * R + slot) * P + p, a.x, ((int64_t)(b * T + m) * H + h) * P + p,
-                a.in_bf16);
+        *reinterpret_cast<uint4 *>(reinterpret_cast<uint8_t *>(a.xbuf) + (((row0 + hh) * R + slot) * P) * ib + k * 16) =
+            *reinterpret_cast<const uint4 *>(sx + (hh * E + W + m) * xrow + k * 16);
     }
-    if (tid < T) a.dtbuf[(int64_t)bh * R + (spmod + tid) % R] = s.sdt[W + tid];
-    if (h % hpg == 0) {  // one head per group writes the group's B
-        for (int i = tid; i < T * N; i += kThreads) {
-            const int m = i / N, n = i - m * N;
+    if (tid < T * HC) {
+        const int m = tid / HC, hh = tid - m * HC;
+        a.dtbuf[(row0 + hh) * R + (spmod + m) % R] = sdt[hh * E + W + m];
+    }
+    if (hc == 0) {  // the group's first CTA writes the group's B
+        for (int i = tid; i < T * bch; i += kThreads) {
+            const int m = i / bch, k = i - m * bch;
             const int slot = (spmod + m) % R;
-            copy_in(a.Bbuf, ((int64_t)(b * G + g) * R + slot) * N + n, a.Bm,
-                    ((int64_t)(b * T + m) * G + g) * N + n, a.in_bf16);
+            *reinterpret_cast<uint4 *>(reinterpret_cast<uint8_t *>(a.Bbuf) + (((int64_t)(b * G + g) * R + slot) * N) * ib + k * 16) =
+                *reinterpret_cast<const uint4 *>(sB + (W + m) * brow + k * 16);
         }
     }
 }
@@ -451,7 +538,7 @@ inline cudaError_t launch_replay_t(const M2Args &a, size_t smem, cudaStream_t st
     auto k = m2_replay_kernel<N, RK, TQ>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    k<<<a.B * a.H, kThreads, smem, st>>>(a);
+    k<<<a.B * (a.H / a.HC), kThreads, smem, st>>>(a);
     return cudaGetLastError();
 }
 template <int N, int SK, int TQ>

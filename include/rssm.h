@@ -91,7 +91,7 @@ typedef struct {
                             the buffer stores them as given.  dt, alpha, beta are fp32. */
     int32_t batch;       /* sequences B >= 1 */
     int32_t nheads;      /* heads H >= 1 */
-    int32_t headdim;     /* P: Mamba-2 headdim, GDN d_v; 1..256 */
+    int32_t headdim;     /* P: Mamba-2 headdim, GDN d_v; a multiple of 8 in 8..256 */
     int32_t dstate;      /* N: Mamba-2 dstate, GDN d_k; one of 16, 32, 64, 128 */
     int32_t ngroups;     /* Mamba-2: G >= 1 dividing H (B/C per group).  GDN: ignored */
     int32_t window;      /* W: buffer window, 1..64 */

@@ -98,6 +98,7 @@ def test_fp8_and_eager_layouts(lib):
 
 @pytest.mark.parametrize("bad", [
     dict(kind=5), dict(dstate=48), dict(dstate=256), dict(headdim=0), dict(headdim=257),
+    dict(headdim=20), dict(headdim=7),
     dict(ngroups=3), dict(window=0), dict(window=65), dict(max_draft=9), dict(max_draft=17),
     dict(batch=0), dict(input_dtype="fp8")])
 def test_invalid_configs_rejected(lib, bad):

@@ -56,7 +56,8 @@ def test_fp8_dual_precision_drift_window_sweep():
     torch.cuda.synchronize()
 
     # the GPU's fp8 copy behaves like the emulated e4m3 copy of the same checkpoint
-    assert emu_worst <= 2e-2, emu_worst
+    # (6e-2: one code rounding the other way at a row's largest element, see test_gpu_mamba2)
+    assert emu_worst <= 6e-2, emu_worst
     # rounding of the copy never feeds back: the checkpoint is the fp32 path's, byte for byte
     ck = {n: layers[n].region("ckpt_off", "ckpt_bytes", torch.int32) for n in
           ("dual_fp8_W16", "dual_bf16_W16", "replay_f32_W16")}

@@ -1,9 +1,13 @@
 """Mamba-2 decode on the GPU against the fp64 CPU oracle.
 
 Tolerances (per step, max |y - y_oracle| <= tol * RMS(y_oracle)): 1e-4 for the
-fp32 read path, 2e-2 for the bf16 read copy, and, for the fp8 read copy, 2e-2
-against the oracle that applies the same e4m3 rounding (the residual is the
-rare code that rounds the other way from an fp32 vs fp64 checkpoint value).
+fp32 read path and 2e-2 for the bf16 read copy against the fp64 oracle.  The e4m3
+copy's own rounding is larger than any fp8 tolerance against fp64 at these
+shapes, so the fp8 path is checked against the oracle that applies the same e4m3
+rounding to its checkpoint: the stored codes must agree except for rare one-step
+differences where the fp32 and fp64 checkpoints straddle a rounding boundary, and
+outputs within 6e-2 * RMS (one such step at a row's largest element moves an
+output by up to amax/14 times |C_n|, a few percent of RMS).
 """
 import numpy as np
 import pytest
@@ -19,7 +23,8 @@ pytestmark = pytest.mark.gpu
 TOL = {"f32": 1e-4, "bf16": 2e-2, "fp8": 2e-2}
 
 
-def _run_decode(wl, mode, read_dtypes, steps, seqs=None, dt_scales=False, emulate=False):
+def _run_decode(wl, mode, read_dtypes, steps, seqs=None, dt_scales=False, emulate=False,
+                return_emu=False):
     """Decode `steps` tokens with one GPU layer per read dtype; compare every step
     against the fp64 eager oracle (and the emulated-rounding oracles)."""
     import torch
@@ -55,6 +60,8 @@ def _run_decode(wl, mode, read_dtypes, steps, seqs=None, dt_scales=False, emulat
             if d in emu:
                 worst_emu[d] = max(worst_emu[d], rel_err(yc, emu[d].decode(sub)))
     torch.cuda.synchronize()
+    if return_emu:
+        return layers, worst, worst_emu, S, emu
     return layers, worst, worst_emu, S
 
 
@@ -76,17 +83,43 @@ def test_tiny_replay_and_eager_fp32_match_oracle():
         assert L.status()[0] == 0
 
 
-@pytest.mark.parametrize("N,P,W,H,G", [(16, 7, 3, 4, 2), (32, 40, 5, 6, 3), (64, 33, 8, 4, 1),
-                                       (128, 20, 2, 2, 2)])
+def fp8_codes_match(L, emu_ckpt, shape):
+    """The GPU's e4m3 read copy against the oracle's e4m3 rounding of its own (fp64)
+    checkpoint: codes may differ only where the fp32 and fp64 checkpoints straddle a
+    rounding boundary -- rarely, and then by one e4m3 step."""
+    import torch
+
+    from oracle import quant
+
+    Bn, H, P, N = shape
+    g_codes = L.region("rc_off", "rc_bytes", torch.uint8).view(torch.float8_e4m3fn).float().view(Bn, H, P, N)
+    g_scale = L.region("rc_scale_off", "rc_scale_bytes", torch.float32).view(Bn, H, P)
+    o_codes, o_scale = quant.e4m3_rows(emu_ckpt.astype(np.float32))
+    g = g_codes.double().cpu().numpy()
+    assert np.allclose(g_scale.double().cpu().numpy(), o_scale, rtol=2 ** -20, atol=0)
+    diff = g != o_codes
+    assert diff.mean() <= 1e-3, diff.mean()
+    if diff.any():
+        grid = np.sort(np.unique(np.abs(torch.arange(256, dtype=torch.uint8).view(torch.float8_e4m3fn)
+                                        .float().numpy())))
+        gi = np.searchsorted(grid, np.abs(g[diff]))
+        oi = np.searchsorted(grid, np.abs(o_codes[diff]))
+        assert np.all(np.abs(gi - oi) <= 1) and np.all(np.sign(g[diff]) * np.sign(o_codes[diff]) >= 0)
+
+
+@pytest.mark.parametrize("N,P,W,H,G", [(16, 8, 3, 4, 2), (32, 40, 5, 6, 3), (64, 24, 8, 4, 1),
+                                       (128, 72, 2, 2, 2), (128, 64, 16, 8, 1)])
 def test_ragged_shapes_all_read_copies(N, P, W, H, G):
-    """Rows not a multiple of the rows per pass, groups of several heads, short windows."""
+    """Rows not a multiple of the rows per pass, 1, 2 or 4 heads per CTA, short windows."""
     wl = I.TINY.replace(batch=3, nheads=H, ngroups=G, headdim=P, dstate=N, window=W, steps=3 * W + 2,
                         seed=11)
-    _, worst, worst_emu, _ = _run_decode(wl, "replay", ["f32", "bf16", "fp8"], wl.steps, emulate=True)
+    layers, worst, worst_emu, _, emu = _run_decode(wl, "replay", ["f32", "bf16", "fp8"], wl.steps,
+                                                   emulate=True, return_emu=True)
     assert worst["f32"] <= TOL["f32"], worst
     assert worst["bf16"] <= TOL["bf16"], worst
     assert worst_emu["bf16"] <= 2e-3, worst_emu
-    assert worst_emu["fp8"] <= TOL["fp8"], worst_emu
+    assert worst_emu["fp8"] <= 6e-2, worst_emu
+    fp8_codes_match(layers["fp8"], emu["fp8"].ckpt, (wl.batch, H, P, N))
 
 
 @pytest.mark.parametrize("sd", ["f32", "bf16", "fp8"])
@@ -99,7 +132,7 @@ def test_eager_baselines(sd):
     if sd == "f32":
         assert worst[sd] <= 1e-4
     else:
-        assert worst_emu[sd] <= TOL[sd], worst_emu
+        assert worst_emu[sd] <= (2e-2 if sd == "bf16" else 6e-2), worst_emu
 
 
 def test_dt_scaled_input_term():

@@ -79,7 +79,7 @@ def test_spec_verify_mamba2_batch512_k4():
 def test_spec_verify_small_all_k():
     """Every K up to max_draft with tight windows (flush on most verifies) and ragged rows."""
     for K, W in ((1, 1), (2, 2), (3, 4), (8, 8)):
-        wl = I.TINY.replace(batch=5, nheads=4, ngroups=2, headdim=12, dstate=32, window=W, steps=0,
+        wl = I.TINY.replace(batch=5, nheads=4, ngroups=2, headdim=16, dstate=32, window=W, steps=0,
                             seed=30 + K, max_draft=K, draft_k=K)
         _spec_run(wl, 12, list(range(5)), {"r32": ("replay", "f32"), "e32": ("eager", "f32")},
                   {"r32": 1e-4, "e32": 1e-4})
