@@ -158,7 +158,11 @@ rssm_status rssm_create(const rssm_config *cfg, void *workspace, size_t workspac
     h->ws = (uint8_t *)workspace;
     h->ws_bytes = workspace_bytes;
     h->stream = (cudaStream_t)stream;
-    cudaError_t e = cudaMemsetAsync(h->ws, 0, L.total_bytes, h->stream);
+    int dev = 0, sms = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e == cudaSuccess && sms > 0) h->num_sms = sms;
+    if (e == cudaSuccess) e = cudaMemsetAsync(h->ws, 0, L.total_bytes, h->stream);
     if (e != cudaSuccess) {
         g_create_error = std::string("zeroing the workspace: ") + cudaGetErrorString(e);
         delete h;

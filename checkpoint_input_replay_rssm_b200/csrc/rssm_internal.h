@@ -19,6 +19,7 @@ struct Ctx {
     cudaStream_t stream = nullptr;
     int pending = 0;            // K of an uncommitted verify (host mirror), 0 if none
     int64_t launches = 0;       // kernels enqueued so far
+    int num_sms = 148;          // SMs of the handle's device (persistent grids)
     std::string err;
 
     void *at(size_t off) const { return ws + off; }

@@ -11,22 +11,32 @@ extern template cudaError_t m2_dispatch_n<128>(bool, int, int, const M2Args &, s
 
 static int tq_of(int T) { return T <= 1 ? 1 : (T <= 4 ? 4 : 8); }
 
-// Heads per replay CTA: the largest of 4, 2, 1 that divides the heads of a group
-// and keeps the CTA's shared memory within 160 KiB.
-static int m2_heads_per_cta(const rssm_config &cf, int TQ) {
+// Replay pipeline shape: heads per item HC (dividing the heads of a group) and
+// stages NS.  Prefer 2 heads per item, then 1, then 4, with the most stages
+// (up to 4) that fit 200 KiB of shared memory; at least 3 stages unless only
+// fewer fit (large windows x wide heads), down to one.
+struct M2Pipe { int HC, NS; size_t smem; };
+static M2Pipe m2_pipe(const rssm_config &cf, int TQ) {
     const int hpg = cf.nheads / cf.ngroups, ib = cf.input_dtype == RSSM_BF16 ? 2 : 4;
-    for (int hc = 4; hc > 1; hc >>= 1)
-        if (hpg % hc == 0 && m2_lay(hc, cf.headdim, cf.dstate, cf.window, TQ, ib).total <= 160 * 1024)
-            return hc;
-    return 1;
+    const int rcb = cf.state_dtype == RSSM_F32 ? 4 : (cf.state_dtype == RSSM_BF16 ? 2 : 1);
+    auto total = [&](int hc, int ns) {
+        return m2_smem_total(ns, hc, cf.headdim, cf.dstate, cf.window, TQ, ib, rcb);
+    };
+    for (int min_ns : {3, 1}) {
+        for (int hc : {2, 1, 4}) {
+            if (hpg % hc != 0) continue;
+            for (int ns = 4; ns >= min_ns; --ns)
+                if (total(hc, ns) <= 200 * 1024) return {hc, ns, (size_t)total(hc, ns)};
+        }
+    }
+    return {1, 1, (size_t)total(1, 1)};
 }
 
 size_t mamba2_smem_bytes(const rssm_config &cf, int T) {
     const int TQ = tq_of(T), P = cf.headdim, N = cf.dstate;
     if (cf.mode == RSSM_EAGER)
         return sizeof(float) * ((size_t)2 * pad4(TQ * P) + 2 * pad4(TQ * N) + 2 * pad4(TQ));
-    const int ib = cf.input_dtype == RSSM_BF16 ? 2 : 4;
-    return (size_t)m2_lay(m2_heads_per_cta(cf, TQ), P, N, cf.window, TQ, ib).total;
+    return m2_pipe(cf, TQ).smem;
 }
 
 cudaError_t mamba2_launch(const Ctx &h, int op, int T, const rssm_inputs *in, float *y, float *out,
@@ -36,7 +46,13 @@ cudaError_t mamba2_launch(const Ctx &h, int op, int T, const rssm_inputs *in, fl
     a.B = cf.batch; a.H = cf.nheads; a.P = cf.headdim; a.G = cf.ngroups; a.W = cf.window;
     a.R = (int)h.lay.ring; a.T = T; a.op = op; a.in_bf16 = cf.input_dtype == RSSM_BF16;
     a.dt_scales = cf.dt_scales_input;
-    a.HC = m2_heads_per_cta(cf, tq_of(T));
+    const M2Pipe pp = m2_pipe(cf, tq_of(T));
+    a.HC = pp.HC;
+    a.NS = pp.NS;
+    {
+        const int items = cf.batch * (cf.nheads / pp.HC);
+        a.grid = items < h.num_sms ? items : h.num_sms;
+    }
     a.c = h.counters();
     a.A = (const float *)h.at(h.lay.A_off); a.D = (const float *)h.at(h.lay.D_off);
     a.ckpt = h.lay.ckpt_bytes ? (float *)h.at(h.lay.ckpt_off) : nullptr;

@@ -24,12 +24,15 @@
 #pragma once
 #include "rssm_device.cuh"
 #include "rssm_internal.h"
+#include "rssm_pipe.cuh"
 
 namespace rssm {
 
 struct M2Args {
     int B, H, P, G, W, R, T, op, in_bf16, dt_scales;
-    int HC;             // heads per replay CTA (divides H / G)
+    int HC;             // heads per replay item (divides H / G)
+    int NS;             // pipeline stages of the replay kernel
+    int grid;           // persistent CTAs of the replay kernel
     Counters c;
     const float *A, *D;
     float *ckpt;        // fp32 [B][H][P][N]
@@ -49,256 +52,358 @@ struct M2Args {
     float *out;         // export target [B][H][P][N]
 };
 
-// Shared-memory layout of the replay kernel, in bytes; every region 16-byte aligned.
-// E = W + TQ entry slots: committed entries sit right-aligned before slot W, the
-// tokens of this call at W..W+T-1, so an entry's slot is (W - L0) + its index.
-struct M2Lay {
-    int sx, sB, sC, sCf, sdt, slam, sd, scoef, sdec, sdot, su, ssc, si, total;
-};
 __host__ __device__ constexpr int a16(int v) { return (v + 15) & ~15; }
 __host__ __device__ constexpr int pad4(int n) { return (n + 3) & ~3; }
-__host__ __device__ inline M2Lay m2_lay(int HC, int P, int N, int W, int TQ, int ib) {
+
+// One pipeline stage of the persistent replay kernel (bytes, 16-byte aligned
+// regions).  A stage carries one unit of work: the state tile of an item (the
+// read copy of HC heads, or one part of their fp32 checkpoint when the item
+// folds) plus everything the item needs from the ring and from this call's
+// tokens.  Entry slots: E = W + TQ; committed entries sit right-aligned before
+// slot W and this call's tokens at W..W+T-1.
+struct M2Stage {
+    int tile, scale, x, B, C, dt, info, bytes;
+};
+constexpr int kTileCap = 32 * 1024;  // bytes of state rows per pipeline unit
+
+__host__ __device__ inline M2Stage m2_stage(int HC, int P, int N, int W, int TQ, int ib, int rcb) {
     const int E = W + TQ;
-    M2Lay L{};
+    M2Stage S{};
     int o = 0;
-    L.sx = o;    o += a16(HC * E * P * ib);   // raw x of entries      [HC][E][P]
-    L.sB = o;    o += a16(E * N * ib);        // raw B of entries      [E][N]
-    L.sC = o;    o += a16(TQ * N * ib);       // raw C of the queries  [TQ][N]
-    L.sCf = o;   o += a16(TQ * N * 4);        // C as fp32             [TQ][N]
-    L.sdt = o;   o += a16(HC * E * 4);        // dt of entries         [HC][E]
-    L.slam = o;  o += a16(HC * E * 4);        // prefix sums of dt*A   [HC][E]
-    L.sd = o;    o += a16(TQ * E * 4);        // B_e . C_m             [TQ][E]
-    L.scoef = o; o += a16(HC * TQ * E * 4);   // replay coefficients   [HC][TQ][E]
-    L.sdec = o;  o += a16(HC * TQ * 4);       // decay of S^ C         [HC][TQ]
-    L.sdot = o;  o += a16(HC * P * TQ * 4);   // S^ C per state row    [HC*P][TQ]
-    L.su = o;    o += a16(HC * E * 4);        // fold weights          [HC][E]
-    L.ssc = o;   o += a16(HC * P * 4);        // fp8 row scales        [HC*P]
-    L.si = o;    o += 32;                     // counters of the sequence
-    L.total = o;
-    return L;
+    S.tile = o;  o += kTileCap;                                  // state rows of the unit
+    S.scale = o; o += (rcb == 1) ? a16(kTileCap / N * 4) : 0;    // fp8 row scales
+    S.x = o;     o += a16(HC * E * P * ib);            // x of entries   [HC][E][P]
+    S.B = o;     o += a16(E * N * ib);                 // B of entries   [E][N]
+    S.C = o;     o += a16(TQ * N * ib);                // C of queries   [TQ][N]
+    S.dt = o;    o += a16(HC * E * 4);                 // dt of entries  [HC][E]
+    S.info = o;  o += 64;                              // unit descriptor
+    S.bytes = o;
+    return S;
 }
+
+// Consumer-side scratch, shared by all units (bytes).
+struct M2Scratch {
+    int sd, slam, scoef, sdec, su, sdot, sCf, flag, bytes;
+};
+__host__ __device__ inline M2Scratch m2_scratch(int HC, int P, int N, int W, int TQ) {
+    const int E = W + TQ;
+    M2Scratch S{};
+    int o = 0;
+    S.sd = o;    o += a16(TQ * E * 4);       // B_e . C_m             [TQ][E]
+    S.slam = o;  o += a16(HC * E * 4);       // prefix sums of dt*A   [HC][E]
+    S.scoef = o; o += a16(HC * TQ * E * 4);  // replay coefficients   [HC][TQ][E]
+    S.sdec = o;  o += a16(HC * TQ * 4);      // decay of S^ C         [HC][TQ]
+    S.su = o;    o += a16(HC * E * 4);       // fold weights          [HC][E]
+    S.sdot = o;  o += a16(HC * P * TQ * 4);  // S^ C per state row    [HC*P][TQ]
+    S.sCf = o;   o += a16(TQ * N * 4);       // C as fp32             [TQ][N]
+    S.flag = o;  o += 16;                    // consumer vote
+    S.bytes = o;
+    return S;
+}
+
+__host__ __device__ inline int m2_smem_total(int NS, int HC, int P, int N, int W, int TQ, int ib, int rcb) {
+    return 16 * NS + NS * m2_stage(HC, P, N, W, TQ, ib, rcb).bytes + m2_scratch(HC, P, N, W, TQ).bytes;
+}
+
+enum { INFO_ITEM = 0, INFO_PART, INFO_NPARTS, INFO_L0, INFO_FLUSH, INFO_CKMOD, INFO_SPMOD };
 
 // ---------------------------------------------------------------------------
 // Replay kernel: decode (T = 1), verify (T = K), flush (T = 0), export (T = 0).
 //
-// One CTA per (sequence b, group g, chunk of HC heads of the group).  The HC
-// heads' state tiles are contiguous, so the CTA streams one block of
-// HC * P * N elements.  Timeline:
-//   1. every thread issues its read-copy chunks (128-bit, L1 no-allocate) --
-//      up to MAXC per thread, all in flight at once;
-//   2. thread 0 reads the sequence counters while cp.async stages the call's
-//      own tokens (C, B, x, dt) in shared memory;
-//   3. one cp.async batch stages the L0 buffered entries (B of the group, x and
-//      dt of the HC heads);
-//   4. warps compute B_e . C_m once for the group and the prefix sums of the log
-//      decays per head (warp scans), then the replay coefficients;
-//   5. the read-copy rows are dotted with C (or, on a fold step, the fp32
-//      checkpoint rows are folded, stored with the requantised copy and dotted);
-//   6. outputs, ring appends; the last CTA of the sequence publishes counters.
+// Persistent: one CTA per SM walks the items (sequence b, group g, chunk of HC
+// heads of the group; the HC state tiles are contiguous) with stride gridDim.
+// Warp 8 is the producer: for each item it reads the sequence counters, decides
+// whether the item folds, and fills the next free stage of an NS-deep ring in
+// shared memory with bulk copies (the read-copy tile, or the fp32 checkpoint in
+// parts when folding, plus the buffered entries and this call's tokens), so up
+// to NS tiles are in flight while the eight consumer warps work.  Consumers,
+// per unit: B_e . C_m and per-head prefix sums of the log decays (first part of
+// an item), then either the read-copy rows dotted with C or the fold of the
+// checkpoint rows (stored with the requantised copy), then outputs and ring
+// appends (last part), and release the stage.  Every barrier wait is bounded.
 // ---------------------------------------------------------------------------
 template <int N, int RK, int TQ>
-__global__ void __launch_bounds__(kThreads, 2) m2_replay_kernel(const M2Args a) {
+__global__ void __launch_bounds__(kThreads + 32, 1) m2_replay_kernel(const M2Args a) {
     constexpr int EPC = Chunk<RK>::EPC;    // stored elements per 16-byte chunk
     constexpr int TPR = N / EPC;           // lanes per state row, read mapping
-    constexpr int MAXC = (TQ == 1) ? 16 : (TQ == 4 ? 8 : 4);  // read-copy chunks in flight per thread
+    constexpr int RCB = Chunk<RK>::BYTES;  // bytes per stored element
     constexpr int TPR4 = N / 4;            // lanes per row, fp32 quad mapping (fold)
     constexpr int RPP4 = kThreads / TPR4;
-    constexpr int RB4 = 8;
     static_assert(TPR >= 1 && TPR <= 32 && (32 % TPR) == 0, "row must fit a warp");
 
-    extern __shared__ __align__(16) uint8_t smraw[];
+    extern __shared__ __align__(128) uint8_t smraw[];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int H = a.H, P = a.P, W = a.W, R = a.R, T = a.T, G = a.G, HC = a.HC;
+    const int H = a.H, P = a.P, W = a.W, R = a.R, T = a.T, G = a.G, HC = a.HC, NS = a.NS;
     const int hpg = H / G, cpg = hpg / HC;
-    const int b = blockIdx.x / (G * cpg);
-    const int rem = blockIdx.x - b * G * cpg;
-    const int g = rem / cpg, hc = rem - g * cpg;
-    const int h0 = g * hpg + hc * HC;
     const int E = W + TQ;
     const int bf = a.in_bf16, ib = bf ? 2 : 4;
-    const M2Lay Ly = m2_lay(HC, P, N, W, TQ, ib);
-    uint8_t *sx = smraw + Ly.sx;
-    uint8_t *sB = smraw + Ly.sB;
-    uint8_t *sC = smraw + Ly.sC;
-    float *sCf = reinterpret_cast<float *>(smraw + Ly.sCf);
-    float *sdt = reinterpret_cast<float *>(smraw + Ly.sdt);
-    float *slam = reinterpret_cast<float *>(smraw + Ly.slam);
-    float *sd = reinterpret_cast<float *>(smraw + Ly.sd);
-    float *scoef = reinterpret_cast<float *>(smraw + Ly.scoef);
-    float *sdec = reinterpret_cast<float *>(smraw + Ly.sdec);
-    float *sdot = reinterpret_cast<float *>(smraw + Ly.sdot);
-    float *su = reinterpret_cast<float *>(smraw + Ly.su);
-    float *ssc = reinterpret_cast<float *>(smraw + Ly.ssc);
-    int *si = reinterpret_cast<int *>(smraw + Ly.si);
-    const int64_t row0 = (int64_t)b * H + h0;  // (b, h0)
-    const int64_t tile0 = row0 * P * N;        // first state element of the CTA
     const int nrows = HC * P;
-    const int nchunks = nrows * TPR;
     const bool reads = (a.op == OP_DECODE || a.op == OP_VERIFY);
-    const int c = tid % TPR;
-    const int xrow = P * ib, brow = N * ib;   // bytes of an x row / a B or C row
-    const int xch = xrow / 16, bch = brow / 16;
+    const int rpp_read = kTileCap / (N * RCB);  // read-copy rows per unit
+    const int rpp_fold = kTileCap / (N * 4);    // fp32 checkpoint rows per unit
+    const int read_parts = (nrows + rpp_read - 1) / rpp_read;
+    const int fold_parts = (nrows + rpp_fold - 1) / rpp_fold;
+    const int xrow = P * ib, brow = N * ib;
+    const M2Stage SG = m2_stage(HC, P, N, W, TQ, ib, RCB);
+    const M2Scratch SC = m2_scratch(HC, P, N, W, TQ);
+    uint64_t *full = reinterpret_cast<uint64_t *>(smraw);
+    uint64_t *empty = full + NS;
+    uint8_t *stages = smraw + 16 * NS;
+    uint8_t *scr = stages + NS * SG.bytes;
+    const int nitems = a.B * (H / HC);
 
-    // 1. Read-copy chunks first (dropped on fold steps).
-    const uint8_t *rc_base =
-        (RK == SK_F32) ? reinterpret_cast<const uint8_t *>(a.ckpt + tile0)
-                       : reinterpret_cast<const uint8_t *>(a.rc) + tile0 * Chunk<RK>::BYTES;
-    uint4 rv[MAXC];
-    if (reads) {
-#pragma unroll
-        for (int j = 0; j < MAXC; ++j) {
-            const int idx = tid + kThreads * j;
-            if (idx < nchunks) rv[j] = ld_stream(rc_base + (size_t)idx * 16);
-        }
-        if (RK == SK_FP8)  // the CTA's row scales, contiguous: HC * P floats
-            for (int i = tid; i < nrows / 4; i += kThreads)
-                cp_async16(ssc + 4 * i, a.rc_scale + row0 * P + 4 * i);
-    }
-
-    // 2. Counters (thread 0) and this call's tokens.
     if (tid == 0) {
-        SeqState ss = read_counters(a.c, b, W);
-        const int L0 = (int)(ss.seq - ss.ckpt);
-        int flush = 0;
-        if (ss.ok) flush = (a.op == OP_FLUSH || a.op == OP_EXPORT) ? (L0 > 0) : (L0 + T > W);
-        si[0] = ss.ok;
-        si[1] = ss.ok ? L0 : 0;
-        si[2] = flush;
-        si[3] = (int)(ss.ckpt % R);
-        si[4] = (int)(ss.seq % R);
-        if (!ss.ok) {
-            if (g == 0 && hc == 0) report(a.c.err, DEV_BAD_COUNTERS, b, h0, (int)(ss.seq - ss.ckpt));
-        } else if (a.op != OP_EXPORT) {
-            const int64_t new_seq = (a.op == OP_DECODE) ? ss.seq + 1 : -1;
-            const int64_t new_ckpt = flush ? ss.seq : -1;
-            const int new_pending = (a.op == OP_VERIFY) ? T : -1;
-            arrive_and_publish(a.c, b, H / HC, new_seq, new_ckpt, new_pending, flush);
+        for (int i = 0; i < NS; ++i) {
+            mbar_init(&full[i], 32);       // the producer warp's lanes (+ bulk-copy bytes)
+            mbar_init(&empty[i], kWarps);  // one arrival per consumer warp
         }
-    }
-    for (int i = tid; i < T * bch; i += kThreads) {
-        const int m = i / bch, k = i - m * bch;
-        const int64_t src = (((int64_t)(b * T + m) * G + g) * N) * ib + k * 16;
-        cp_async16(sC + m * brow + k * 16, reinterpret_cast<const uint8_t *>(a.Cm) + src);
-        cp_async16(sB + (W + m) * brow + k * 16, reinterpret_cast<const uint8_t *>(a.Bm) + src);
-    }
-    for (int i = tid; i < T * HC * xch; i += kThreads) {
-        const int m = i / (HC * xch), r2 = i - m * HC * xch;
-        const int hh = r2 / xch, k = r2 - hh * xch;
-        cp_async16(sx + (hh * E + W + m) * xrow + k * 16,
-                   reinterpret_cast<const uint8_t *>(a.x) + (((int64_t)(b * T + m) * H + h0 + hh) * P) * ib + k * 16);
-    }
-    if (tid < T * HC) {
-        const int m = tid / HC, hh = tid - m * HC;
-        sdt[hh * E + W + m] = a.dt[(int64_t)(b * T + m) * H + h0 + hh];
+        mbar_init_fence();
     }
     __syncthreads();
-    if (!si[0]) {  // counters corrupted: error reported, sequence skipped
-        cp_async_wait_all();
+
+    if (warp == kWarps) {
+        // ================================ producer ================================
+        int s = 0;
+        uint32_t used = 0, ephase = 0;
+        bool dead = false;
+        auto acquire = [&](int st) -> bool {  // warp-uniform
+            if (used & (1u << st)) {
+                int got = 0;
+                if (lane == 0) got = mbar_wait(&empty[st], (ephase >> st) & 1u) ? 1 : 0;
+                got = __shfl_sync(0xffffffffu, got, 0);
+                __syncwarp();
+                if (!got) return false;
+                ephase ^= 1u << st;
+            }
+            used |= 1u << st;
+            return true;
+        };
+        for (int item = blockIdx.x; item < nitems && !dead; item += gridDim.x) {
+            const int b = item / (H / HC);
+            const int rem = item - b * (H / HC);
+            const int g = rem / cpg, hc = rem - g * cpg;
+            const int h0 = g * hpg + hc * HC;
+            const int64_t row0 = (int64_t)b * H + h0;
+            const int64_t tile0 = row0 * P * N;
+            int ok = 0, L0 = 0, flush = 0, ckmod = 0, spmod = 0;
+            if (lane == 0) {
+                SeqState ss = read_counters(a.c, b, W);
+                ok = ss.ok;
+                L0 = (int)(ss.seq - ss.ckpt);
+                if (ok) flush = (a.op == OP_FLUSH || a.op == OP_EXPORT) ? (L0 > 0) : (L0 + T > W);
+                ckmod = (int)(ss.ckpt % R);
+                spmod = (int)(ss.seq % R);
+                if (!ok) {
+                    if (g == 0 && hc == 0) report(a.c.err, DEV_BAD_COUNTERS, b, h0, L0);
+                } else if (a.op != OP_EXPORT) {
+                    arrive_and_publish(a.c, b, H / HC, (a.op == OP_DECODE) ? ss.seq + 1 : -1,
+                                       flush ? ss.seq : -1, (a.op == OP_VERIFY) ? T : -1, flush);
+                }
+            }
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            L0 = __shfl_sync(0xffffffffu, L0, 0);
+            flush = __shfl_sync(0xffffffffu, flush, 0);
+            ckmod = __shfl_sync(0xffffffffu, ckmod, 0);
+            spmod = __shfl_sync(0xffffffffu, spmod, 0);
+            const int nparts = !ok ? 0 : (flush ? fold_parts : (reads ? read_parts : 0));
+            const int base = W - L0;
+            const int n1 = min(L0, R - ckmod);  // entries before the ring wraps
+            for (int part = 0; part < nparts; ++part) {
+                if (!acquire(s)) {
+                    if (lane == 0) report(a.c.err, DEV_PIPE_TIMEOUT, b, h0, 1);
+                    dead = true;
+                    break;
+                }
+                uint8_t *st = stages + s * SG.bytes;
+                int *info = reinterpret_cast<int *>(st + SG.info);
+                float *sdt = reinterpret_cast<float *>(st + SG.dt);
+                if (lane == 0) {
+                    info[INFO_ITEM] = item; info[INFO_PART] = part; info[INFO_NPARTS] = nparts;
+                    info[INFO_L0] = L0; info[INFO_FLUSH] = flush; info[INFO_CKMOD] = ckmod;
+                    info[INFO_SPMOD] = spmod;
+                }
+                for (int i = lane; i < HC * L0; i += 32) {
+                    const int hh = i / L0, e = i - hh * L0;
+                    sdt[hh * E + base + e] = a.dtbuf[(row0 + hh) * R + (ckmod + e) % R];
+                }
+                for (int i = lane; i < HC * T; i += 32) {
+                    const int m = i / HC, hh = i - m * HC;
+                    sdt[hh * E + W + m] = a.dt[(int64_t)(b * T + m) * H + h0 + hh];
+                }
+                // The unit's bulk copies: the same list is walked twice, once to
+                // total the bytes, once to issue (copy k by lane k mod 32).
+                uint32_t tx = 0;
+                int ci = 0;
+                auto copy = [&](bool issue, void *dst, const void *src, uint32_t bytes) {
+                    if (bytes == 0) return;
+                    if (!issue) tx += bytes;
+                    else if ((ci & 31) == lane) bulk_g2s(dst, src, bytes, &full[s]);
+                    ++ci;
+                };
+                auto walk = [&](bool issue) {
+                    ci = 0;
+                    if (flush) {
+                        const int r0 = part * rpp_fold, r1 = min(nrows, r0 + rpp_fold);
+                        copy(issue, st + SG.tile, a.ckpt + tile0 + (int64_t)r0 * N, (uint32_t)((r1 - r0) * N * 4));
+                    } else {
+                        const int r0 = part * rpp_read, r1 = min(nrows, r0 + rpp_read);
+                        const uint8_t *rc = (RK == SK_F32) ? reinterpret_cast<const uint8_t *>(a.ckpt + tile0)
+                                                           : reinterpret_cast<const uint8_t *>(a.rc) + tile0 * RCB;
+                        copy(issue, st + SG.tile, rc + (int64_t)r0 * N * RCB, (uint32_t)((r1 - r0) * N * RCB));
+                        if (RK == SK_FP8)
+                            copy(issue, st + SG.scale, a.rc_scale + row0 * P + r0, (uint32_t)((r1 - r0) * 4));
+                    }
+                    const uint8_t *Bb = reinterpret_cast<const uint8_t *>(a.Bbuf) + ((int64_t)(b * G + g) * R) * brow;
+                    copy(issue, st + SG.B + base * brow, Bb + (int64_t)ckmod * brow, (uint32_t)(n1 * brow));
+                    copy(issue, st + SG.B + (base + n1) * brow, Bb, (uint32_t)((L0 - n1) * brow));
+                    for (int hh = 0; hh < HC; ++hh) {
+                        const uint8_t *xb = reinterpret_cast<const uint8_t *>(a.xbuf) + ((row0 + hh) * R) * xrow;
+                        uint8_t *xd = st + SG.x + (hh * E + base) * xrow;
+                        copy(issue, xd, xb + (int64_t)ckmod * xrow, (uint32_t)(n1 * xrow));
+                        copy(issue, xd + n1 * xrow, xb, (uint32_t)((L0 - n1) * xrow));
+                    }
+                    for (int m = 0; m < T; ++m) {
+                        const int64_t gsrc = (((int64_t)(b * T + m) * G + g) * N) * ib;
+                        copy(issue, st + SG.C + m * brow, reinterpret_cast<const uint8_t *>(a.Cm) + gsrc, (uint32_t)brow);
+                        copy(issue, st + SG.B + (W + m) * brow, reinterpret_cast<const uint8_t *>(a.Bm) + gsrc, (uint32_t)brow);
+                        // x of the HC heads for token m is contiguous
+                        uint8_t *xd = st + SG.x + W * xrow + m * xrow;  // head 0 slot W + m
+                        const uint8_t *xs = reinterpret_cast<const uint8_t *>(a.x) + (((int64_t)(b * T + m) * H + h0) * P) * ib;
+                        for (int hh = 0; hh < HC; ++hh)
+                            copy(issue, xd + hh * E * xrow, xs + hh * xrow, (uint32_t)xrow);
+                    }
+                };
+                walk(false);
+                if (lane == 0) mbar_arrive_expect_tx(&full[s], tx);
+                else mbar_arrive(&full[s]);
+                __syncwarp();
+                walk(true);
+                s = (s + 1 == NS) ? 0 : s + 1;
+            }
+        }
+        if (!dead && acquire(s)) {  // end-of-work unit
+            if (lane == 0) reinterpret_cast<int *>(stages + s * SG.bytes + SG.info)[INFO_ITEM] = -1;
+            mbar_arrive(&full[s]);
+        } else if (lane == 0 && !dead) {
+            report(a.c.err, DEV_PIPE_TIMEOUT, -1, -1, 2);
+        }
         return;
     }
-    const int L0 = si[1], flush = si[2], ckmod = si[3], spmod = si[4];
-    const int base = W - L0;
-    const int nE = L0 + T;
 
-    // 3. Buffered entries, one cp.async batch.
-    for (int i = tid; i < L0 * bch; i += kThreads) {
-        const int e = i / bch, k = i - e * bch;
-        const int slot = (ckmod + e) % R;
-        cp_async16(sB + (base + e) * brow + k * 16,
-                   reinterpret_cast<const uint8_t *>(a.Bbuf) + (((int64_t)(b * G + g) * R + slot) * N) * ib + k * 16);
-    }
-    for (int i = tid; i < HC * L0 * xch; i += kThreads) {
-        const int hh = i / (L0 * xch), r2 = i - hh * L0 * xch;
-        const int e = r2 / xch, k = r2 - e * xch;
-        const int slot = (ckmod + e) % R;
-        cp_async16(sx + (hh * E + base + e) * xrow + k * 16,
-                   reinterpret_cast<const uint8_t *>(a.xbuf) + (((row0 + hh) * R + slot) * P) * ib + k * 16);
-    }
-    for (int i = tid; i < HC * L0; i += kThreads) {
-        const int hh = i / L0, e = i - hh * L0;
-        sdt[hh * E + base + e] = a.dtbuf[(row0 + hh) * R + (ckmod + e) % R];
-    }
-    cp_async_wait_all();
-    __syncthreads();
+    // ================================ consumers ================================
+    float *sd = reinterpret_cast<float *>(scr + SC.sd);
+    float *slam = reinterpret_cast<float *>(scr + SC.slam);
+    float *scoef = reinterpret_cast<float *>(scr + SC.scoef);
+    float *sdec = reinterpret_cast<float *>(scr + SC.sdec);
+    float *su = reinterpret_cast<float *>(scr + SC.su);
+    float *sdot = reinterpret_cast<float *>(scr + SC.sdot);
+    float *sCf = reinterpret_cast<float *>(scr + SC.sCf);
+    int *vote = reinterpret_cast<int *>(scr + SC.flag);
+    const int c = tid % TPR;
+    int s = 0;
+    uint32_t fphase = 0;
+    for (;;) {
+        const bool got = mbar_wait(&full[s], (fphase >> s) & 1u);
+        if (tid == 0) vote[0] = 0;
+        consumer_sync();
+        if (!got) atomicOr(&vote[0], 1);
+        consumer_sync();
+        if (vote[0]) {
+            if (tid == 0) report(a.c.err, DEV_PIPE_TIMEOUT, -1, -1, 3);
+            break;
+        }
+        fphase ^= 1u << s;
+        const uint8_t *st = stages + s * SG.bytes;
+        const int *info = reinterpret_cast<const int *>(st + SG.info);
+        const int item = info[INFO_ITEM];
+        if (item < 0) break;
+        const int part = info[INFO_PART], nparts = info[INFO_NPARTS];
+        const int L0 = info[INFO_L0], flush = info[INFO_FLUSH], spmod = info[INFO_SPMOD];
+        const int b = item / (H / HC);
+        const int rem = item - b * (H / HC);
+        const int g = rem / cpg, hc = rem - g * cpg;
+        const int h0 = g * hpg + hc * HC;
+        const int64_t row0 = (int64_t)b * H + h0;
+        const int64_t tile0 = row0 * P * N;
+        const int base = W - L0, nE = L0 + T;
+        const int e0 = flush ? L0 : 0;  // first entry the outputs replay
+        const uint8_t *sx = st + SG.x;
+        const uint8_t *sB = st + SG.B;
+        const uint8_t *sC = st + SG.C;
+        const float *sdt = reinterpret_cast<const float *>(st + SG.dt);
 
-    // 4. B_e . C_m for the group (warps), prefix sums of dt*A per head (warp scans).
-    const int e0 = flush ? L0 : 0;  // first entry the outputs replay
-    if (reads) {
-        for (int pr = warp; pr < T * nE; pr += kWarps) {
-            const int m = pr / nE, e = pr - m * nE;
-            if (e < e0 || e > L0 + m) continue;  // warp-uniform
-            float d = 0.f;
-            for (int n = lane; n < N; n += 32)
-                d = fmaf(raw_f(sB + (base + e) * brow, n, bf), raw_f(sC + m * brow, n, bf), d);
-            d = group_sum<32>(d);
-            if (lane == 0) sd[m * E + e] = d;
-        }
-    }
-    for (int i = tid; i < T * N; i += kThreads) sCf[i] = raw_f(sC, i, bf);
-    for (int hh = warp; hh < HC; hh += kWarps) {
-        const float Ah = a.A[h0 + hh];
-        float carry = 0.f;
-        for (int k0 = 0; k0 < nE; k0 += 32) {
-            const int e = k0 + lane;
-            float v = (e < nE) ? sdt[hh * E + base + e] * Ah : 0.f;
-            v = warp_incl_scan(v) + carry;
-            if (e < nE) slam[hh * E + base + e] = v;
-            carry = __shfl_sync(0xffffffffu, v, 31);
-        }
-    }
-    __syncthreads();
-    if (reads) {
-        for (int i = tid; i < HC * T * nE; i += kThreads) {
-            const int hh = i / (T * nE), r2 = i - hh * T * nE;
-            const int m = r2 / nE, e = r2 - m * nE;
-            if (e < e0 || e > L0 + m) continue;
-            const float* lam = slam + hh * E + base;
-            scoef[(hh * TQ + m) * E + e] = expf(lam[L0 + m] - lam[e]) * sd[m * E + e] *
-                                           (a.dt_scales ? sdt[hh * E + base + e] : 1.f);
-        }
-        for (int i = tid; i < HC * T; i += kThreads) {
-            const int hh = i / T, m = i - hh * T;
-            const float* lam = slam + hh * E + base;
-            sdec[hh * TQ + m] = expf(lam[L0 + m] - (flush ? lam[L0 - 1] : 0.f));
-        }
-    }
-    if (flush) {
-        for (int i = tid; i < HC * L0; i += kThreads) {
-            const int hh = i / L0, e = i - hh * L0;
-            const float* lam = slam + hh * E + base;
-            su[hh * E + e] = expf(lam[L0 - 1] - lam[e]) * (a.dt_scales ? sdt[hh * E + base + e] : 1.f);
-        }
-    }
-    __syncthreads();
-
-    if (flush) {
-        // 5a. Fold: fp32 checkpoint rows in quads, TPR4 lanes per row.
-        const int c4 = tid % TPR4, q0 = tid / TPR4;
-        float4 Cq[TQ];
-#pragma unroll
-        for (int m = 0; m < TQ; ++m) {
-            Cq[m] = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (reads && m < T)
-                Cq[m] = make_float4(raw_f(sC + m * brow, 4 * c4, bf), raw_f(sC + m * brow, 4 * c4 + 1, bf),
-                                    raw_f(sC + m * brow, 4 * c4 + 2, bf), raw_f(sC + m * brow, 4 * c4 + 3, bf));
-        }
-        for (int rb = 0; rb < nrows; rb += RB4 * RPP4) {
-            float4 st[RB4];
-#pragma unroll
-            for (int k = 0; k < RB4; ++k) {
-                const int gr = rb + q0 + k * RPP4;
-                st[k] = (gr < nrows) ? load_quad<SK_F32>(a.ckpt, tile0 + (int64_t)gr * N + 4 * c4)
-                                     : make_float4(0.f, 0.f, 0.f, 0.f);
+        if (part == 0) {
+            // B_e . C_m once per item; C to fp32; prefix sums of dt*A per head.
+            if (reads) {
+                for (int pr = warp; pr < T * nE; pr += kWarps) {
+                    const int m = pr / nE, e = pr - m * nE;
+                    if (e < e0 || e > L0 + m) continue;  // warp-uniform
+                    float d = 0.f;
+                    for (int n = lane; n < N; n += 32)
+                        d = fmaf(raw_f(sB + (base + e) * brow, n, bf), raw_f(sC + m * brow, n, bf), d);
+                    d = group_sum<32>(d);
+                    if (lane == 0) sd[m * E + e] = d;
+                }
+                for (int i = tid; i < T * N; i += kThreads) sCf[i] = raw_f(sC, i, bf);
             }
+            for (int hh = warp; hh < HC; hh += kWarps) {
+                const float Ah = a.A[h0 + hh];
+                float carry = 0.f;
+                for (int k0 = 0; k0 < nE; k0 += 32) {
+                    const int e = k0 + lane;
+                    float v = (e < nE) ? sdt[hh * E + base + e] * Ah : 0.f;
+                    v = warp_incl_scan(v) + carry;
+                    if (e < nE) slam[hh * E + base + e] = v;
+                    carry = __shfl_sync(0xffffffffu, v, 31);
+                }
+            }
+            consumer_sync();
+            if (reads) {
+                for (int i = tid; i < HC * T * nE; i += kThreads) {
+                    const int hh = i / (T * nE), r2 = i - hh * T * nE;
+                    const int m = r2 / nE, e = r2 - m * nE;
+                    if (e < e0 || e > L0 + m) continue;
+                    const float *lam = slam + hh * E + base;
+                    scoef[(hh * TQ + m) * E + e] = expf(lam[L0 + m] - lam[e]) * sd[m * E + e] *
+                                                   (a.dt_scales ? sdt[hh * E + base + e] : 1.f);
+                }
+                for (int i = tid; i < HC * T; i += kThreads) {
+                    const int hh = i / T, m = i - hh * T;
+                    const float *lam = slam + hh * E + base;
+                    sdec[hh * TQ + m] = expf(lam[L0 + m] - (flush ? lam[L0 - 1] : 0.f));
+                }
+            }
+            if (flush) {
+                for (int i = tid; i < HC * L0; i += kThreads) {
+                    const int hh = i / L0, e = i - hh * L0;
+                    const float *lam = slam + hh * E + base;
+                    su[hh * E + e] = expf(lam[L0 - 1] - lam[e]) * (a.dt_scales ? sdt[hh * E + base + e] : 1.f);
+                }
+            }
+            consumer_sync();
+        }
+
+        if (flush) {
+            // Fold this part's fp32 checkpoint rows (from the stage), store the
+            // checkpoint and the requantised copy, dot the fresh copy with C.
+            const int c4 = tid % TPR4, q0 = tid / TPR4;
+            const int rpp = rpp_fold;
+            const int r0 = part * rpp, r1 = min(nrows, r0 + rpp);
+            const float *tf = reinterpret_cast<const float *>(st + SG.tile);
+            float4 Cq[TQ];
 #pragma unroll
-            for (int k = 0; k < RB4; ++k) {
-                const int gr = rb + q0 + k * RPP4;
-                const bool valid = gr < nrows;
+            for (int m = 0; m < TQ; ++m)
+                Cq[m] = (reads && m < T) ? *reinterpret_cast<const float4 *>(sCf + m * N + 4 * c4)
+                                         : make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int rb = 0; rb < rpp; rb += RPP4) {  // same trip count for every lane
+                const int rl = rb + q0;
+                const int gr = r0 + rl;
+                const bool valid = rl < rpp && gr < r1;
                 const int hh = valid ? gr / P : 0, p = valid ? gr - hh * P : 0;
-                float4 v = st[k];
+                float4 v = valid ? *reinterpret_cast<const float4 *>(tf + rl * N + 4 * c4)
+                                 : make_float4(0.f, 0.f, 0.f, 0.f);
                 if (valid) {
-                    const float* lam = slam + hh * E + base;
-                    const float dec_all = expf(lam[L0 - 1]);
+                    const float dec_all = expf(slam[hh * E + base + L0 - 1]);
                     v.x *= dec_all; v.y *= dec_all; v.z *= dec_all; v.w *= dec_all;
                     for (int e = 0; e < L0; ++e) {
                         const float w = su[hh * E + e] * raw_f(sx + (hh * E + base + e) * xrow, p, bf);
@@ -315,7 +420,7 @@ __global__ void __launch_bounds__(kThreads, 2) m2_replay_kernel(const M2Args a) 
                     continue;
                 }
                 if (valid) *reinterpret_cast<float4 *>(a.ckpt + el) = v;
-                float4 rd = v;  // what the outputs read: the fresh read copy
+                float4 rd = v;
                 if (RK == SK_BF16) {
                     if (valid) rd = store_quad<SK_BF16>(a.rc, el, v, 0.f, 0.f);
                 } else if (RK == SK_FP8) {
@@ -336,33 +441,27 @@ __global__ void __launch_bounds__(kThreads, 2) m2_replay_kernel(const M2Args a) 
                     }
                 }
             }
-        }
-    } else if (reads) {
-        // 5b. Read: dot products of the read-copy rows with the query C's (held in
-        // registers when they fit, else read from shared memory).
-        constexpr bool kCregs = TQ * EPC <= 64;
-        float Cr[kCregs ? TQ : 1][kCregs ? EPC : 1];
-        if (kCregs) {
+        } else if (reads) {
+            // Read: every 16-byte chunk of the staged read copy dotted with C.
+            constexpr bool kCregs = TQ * EPC <= 64;
+            float Cr[kCregs ? TQ : 1][kCregs ? EPC : 1];
+            if (kCregs) {
 #pragma unroll
-            for (int m = 0; m < (kCregs ? TQ : 1); ++m)
+                for (int m = 0; m < (kCregs ? TQ : 1); ++m)
 #pragma unroll
-                for (int j = 0; j < (kCregs ? EPC : 1); ++j)
-                    Cr[m][j] = (m < T) ? sCf[m * N + c * EPC + j] : 0.f;
-        }
-        for (int r0 = 0; r0 < nchunks; r0 += MAXC * kThreads) {
-            if (r0 > 0) {
-#pragma unroll
-                for (int j = 0; j < MAXC; ++j) {
-                    const int idx = r0 + tid + kThreads * j;
-                    if (idx < nchunks) rv[j] = ld_stream(rc_base + (size_t)idx * 16);
-                }
+                    for (int j = 0; j < (kCregs ? EPC : 1); ++j)
+                        Cr[m][j] = (m < T) ? sCf[m * N + c * EPC + j] : 0.f;
             }
-#pragma unroll
-            for (int j = 0; j < MAXC; ++j) {
-                const int idx = r0 + tid + kThreads * j;
+            const uint4 *tile = reinterpret_cast<const uint4 *>(st + SG.tile);
+            const float *ssc = reinterpret_cast<const float *>(st + SG.scale);
+            const int r0 = part * rpp_read, r1 = min(nrows, r0 + rpp_read);
+            const int nchunks = (r1 - r0) * TPR;
+#pragma unroll 4
+            for (int cb = 0; cb < nchunks; cb += kThreads) {  // same trip count for every lane
+                const int idx = cb + tid;
                 const bool valid = idx < nchunks;
                 float v[EPC];
-                if (valid) unpack<RK>(rv[j], v);
+                if (valid) unpack<RK>(tile[idx], v);
                 else {
 #pragma unroll
                     for (int q = 0; q < EPC; ++q) v[q] = 0.f;
@@ -379,43 +478,48 @@ __global__ void __launch_bounds__(kThreads, 2) m2_replay_kernel(const M2Args a) 
                     }
                     d = group_sum<TPR>(d);
                     if (c == 0 && valid && m < T)
-                        sdot[(idx / TPR) * TQ + m] = (RK == SK_FP8) ? d * ssc[idx / TPR] : d;
+                        sdot[(r0 + idx / TPR) * TQ + m] = (RK == SK_FP8) ? d * ssc[idx / TPR] : d;
                 }
             }
         }
-    }
-    if (!reads) return;
-    __syncthreads();
 
-    // 6. Outputs y[b, m, h0 + hh, :] and ring appends (slots seq_pos + m mod R).
-    for (int i = tid; i < T * HC * P; i += kThreads) {
-        const int m = i / (HC * P), r2 = i - m * HC * P;
-        const int hh = r2 / P, p = r2 - hh * P;
-        float yv = sdec[hh * TQ + m] * sdot[(hh * P + p) * TQ + m];
-        const float *cf = scoef + (hh * TQ + m) * E;
-        const uint8_t *xs = sx + (hh * E + base) * xrow;
-        for (int e = e0; e <= L0 + m; ++e) yv = fmaf(cf[e], raw_f(xs + e * xrow, p, bf), yv);
-        yv = fmaf(a.D[h0 + hh], raw_f(sx + (hh * E + W + m) * xrow, p, bf), yv);
-        a.y[((int64_t)(b * T + m) * H + h0 + hh) * P + p] = yv;
-    }
-    for (int i = tid; i < T * HC * xch; i += kThreads) {
-        const int m = i / (HC * xch), r2 = i - m * HC * xch;
-        const int hh = r2 / xch, k = r2 - hh * xch;
-        const int slot = (spmod + m) % R;
-        *reinterpret_cast<uint4 *>(reinterpret_cast<uint8_t *>(a.xbuf) + (((row0 + hh) * R + slot) * P) * ib + k * 16) =
-            *reinterpret_cast<const uint4 *>(sx + (hh * E + W + m) * xrow + k * 16);
-    }
-    if (tid < T * HC) {
-        const int m = tid / HC, hh = tid - m * HC;
-        a.dtbuf[(row0 + hh) * R + (spmod + m) % R] = sdt[hh * E + W + m];
-    }
-    if (hc == 0) {  // the group's first CTA writes the group's B
-        for (int i = tid; i < T * bch; i += kThreads) {
-            const int m = i / bch, k = i - m * bch;
-            const int slot = (spmod + m) % R;
-            *reinterpret_cast<uint4 *>(reinterpret_cast<uint8_t *>(a.Bbuf) + (((int64_t)(b * G + g) * R + slot) * N) * ib + k * 16) =
-                *reinterpret_cast<const uint4 *>(sB + (W + m) * brow + k * 16);
+        if (reads && part == nparts - 1) {
+            consumer_sync();
+            // Outputs y[b, m, h0 + hh, :] and ring appends (slots seq_pos + m mod R).
+            for (int i = tid; i < T * HC * P; i += kThreads) {
+                const int m = i / (HC * P), r2 = i - m * HC * P;
+                const int hh = r2 / P, p = r2 - hh * P;
+                float yv = sdec[hh * TQ + m] * sdot[(hh * P + p) * TQ + m];
+                const float *cf = scoef + (hh * TQ + m) * E;
+                const uint8_t *xs = sx + (hh * E + base) * xrow;
+                for (int e = e0; e <= L0 + m; ++e) yv = fmaf(cf[e], raw_f(xs + e * xrow, p, bf), yv);
+                yv = fmaf(a.D[h0 + hh], raw_f(sx + (hh * E + W + m) * xrow, p, bf), yv);
+                a.y[((int64_t)(b * T + m) * H + h0 + hh) * P + p] = yv;
+            }
+            const int xch = xrow / 16, bch = brow / 16;
+            for (int i = tid; i < T * HC * xch; i += kThreads) {
+                const int m = i / (HC * xch), r2 = i - m * HC * xch;
+                const int hh = r2 / xch, k = r2 - hh * xch;
+                const int slot = (spmod + m) % R;
+                *reinterpret_cast<uint4 *>(reinterpret_cast<uint8_t *>(a.xbuf) + (((row0 + hh) * R + slot) * P) * ib + k * 16) =
+                    *reinterpret_cast<const uint4 *>(sx + (hh * E + W + m) * xrow + k * 16);
+            }
+            if (tid < T * HC) {
+                const int m = tid / HC, hh = tid - m * HC;
+                a.dtbuf[(row0 + hh) * R + (spmod + m) % R] = sdt[hh * E + W + m];
+            }
+            if (hc == 0) {  // the group's first item writes the group's B
+                for (int i = tid; i < T * bch; i += kThreads) {
+                    const int m = i / bch, k = i - m * bch;
+                    const int slot = (spmod + m) % R;
+                    *reinterpret_cast<uint4 *>(reinterpret_cast<uint8_t *>(a.Bbuf) + (((int64_t)(b * G + g) * R + slot) * N) * ib + k * 16) =
+                        *reinterpret_cast<const uint4 *>(sB + (W + m) * brow + k * 16);
+                }
+            }
         }
+        consumer_sync();  // every consumer is done with the stage
+        if (lane == 0) mbar_arrive(&empty[s]);
+        s = (s + 1 == NS) ? 0 : s + 1;
     }
 }
 
@@ -538,7 +642,7 @@ inline cudaError_t launch_replay_t(const M2Args &a, size_t smem, cudaStream_t st
     auto k = m2_replay_kernel<N, RK, TQ>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    k<<<a.B * (a.H / a.HC), kThreads, smem, st>>>(a);
+    k<<<a.grid, kThreads + 32, smem, st>>>(a);
     return cudaGetLastError();
 }
 template <int N, int SK, int TQ>
