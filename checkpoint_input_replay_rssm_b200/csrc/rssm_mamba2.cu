@@ -11,25 +11,30 @@ extern template cudaError_t m2_dispatch_n<128>(bool, int, int, const M2Args &, s
 
 static int tq_of(int T) { return T <= 1 ? 1 : (T <= 4 ? 4 : 8); }
 
-// Replay pipeline shape: heads per item HC (dividing the heads of a group) and
-// stages NS.  Prefer 2 heads per item, then 1, then 4, with the most stages
-// (up to 4) that fit 200 KiB of shared memory; at least 3 stages unless only
-// fewer fit (large windows x wide heads), down to one.
-struct M2Pipe { int HC, NS; size_t smem; };
+// Replay pipeline shape: heads per item HC (dividing the heads of a group),
+// stages NS and CTAs per SM.  Two CTAs per SM (two producers, sixteen consumer
+// warps) when two stages fit 110 KiB each; otherwise one CTA with up to 4 stages
+// in 200 KiB.  Items prefer 2 heads, then 1, then 4.
+struct M2Pipe { int HC, NS, per_sm; size_t smem; };
 static M2Pipe m2_pipe(const rssm_config &cf, int TQ) {
     const int hpg = cf.nheads / cf.ngroups, ib = cf.input_dtype == RSSM_BF16 ? 2 : 4;
     const int rcb = cf.state_dtype == RSSM_F32 ? 4 : (cf.state_dtype == RSSM_BF16 ? 2 : 1);
     auto total = [&](int hc, int ns) {
         return m2_smem_total(ns, hc, cf.headdim, cf.dstate, cf.window, TQ, ib, rcb);
     };
+    for (int hc : {2, 1, 4}) {
+        if (hpg % hc != 0) continue;
+        for (int ns = 3; ns >= 2; --ns)
+            if (total(hc, ns) <= 110 * 1024) return {hc, ns, 2, (size_t)total(hc, ns)};
+    }
     for (int min_ns : {3, 1}) {
         for (int hc : {2, 1, 4}) {
             if (hpg % hc != 0) continue;
             for (int ns = 4; ns >= min_ns; --ns)
-                if (total(hc, ns) <= 200 * 1024) return {hc, ns, (size_t)total(hc, ns)};
+                if (total(hc, ns) <= 200 * 1024) return {hc, ns, 1, (size_t)total(hc, ns)};
         }
     }
-    return {1, 1, (size_t)total(1, 1)};
+    return {1, 1, 1, (size_t)total(1, 1)};
 }
 
 size_t mamba2_smem_bytes(const rssm_config &cf, int T) {
@@ -51,7 +56,8 @@ cudaError_t mamba2_launch(const Ctx &h, int op, int T, const rssm_inputs *in, fl
     a.NS = pp.NS;
     {
         const int items = cf.batch * (cf.nheads / pp.HC);
-        a.grid = items < h.num_sms ? items : h.num_sms;
+        const int ctas = pp.per_sm * h.num_sms;
+        a.grid = items < ctas ? items : ctas;
     }
     a.c = h.counters();
     a.A = (const float *)h.at(h.lay.A_off); a.D = (const float *)h.at(h.lay.D_off);

@@ -83,7 +83,7 @@ __host__ __device__ inline M2Stage m2_stage(int HC, int P, int N, int W, int TQ,
 
 // Consumer-side scratch, shared by all units (bytes).
 struct M2Scratch {
-    int sd, slam, scoef, sdec, su, sdot, sCf, flag, bytes;
+    int sd, slam, scoef, sdec, su, sfdec, sdot, sCf, bytes;
 };
 __host__ __device__ inline M2Scratch m2_scratch(int HC, int P, int N, int W, int TQ) {
     const int E = W + TQ;
@@ -94,9 +94,9 @@ __host__ __device__ inline M2Scratch m2_scratch(int HC, int P, int N, int W, int
     S.scoef = o; o += a16(HC * TQ * E * 4);  // replay coefficients   [HC][TQ][E]
     S.sdec = o;  o += a16(HC * TQ * 4);      // decay of S^ C         [HC][TQ]
     S.su = o;    o += a16(HC * E * 4);       // fold weights          [HC][E]
+    S.sfdec = o; o += a16(HC * 4);           // decay of the folded checkpoint [HC]
     S.sdot = o;  o += a16(HC * P * TQ * 4);  // S^ C per state row    [HC*P][TQ]
     S.sCf = o;   o += a16(TQ * N * 4);       // C as fp32             [TQ][N]
-    S.flag = o;  o += 16;                    // consumer vote
     S.bytes = o;
     return S;
 }
@@ -123,7 +123,7 @@ enum { INFO_ITEM = 0, INFO_PART, INFO_NPARTS, INFO_L0, INFO_FLUSH, INFO_CKMOD, I
 // appends (last part), and release the stage.  Every barrier wait is bounded.
 // ---------------------------------------------------------------------------
 template <int N, int RK, int TQ>
-__global__ void __launch_bounds__(kThreads + 32, 1) m2_replay_kernel(const M2Args a) {
+__global__ void __maxnreg__(112) m2_replay_kernel(const M2Args a) {
     constexpr int EPC = Chunk<RK>::EPC;    // stored elements per 16-byte chunk
     constexpr int TPR = N / EPC;           // lanes per state row, read mapping
     constexpr int RCB = Chunk<RK>::BYTES;  // bytes per stored element
@@ -296,19 +296,25 @@ __global__ void __launch_bounds__(kThreads + 32, 1) m2_replay_kernel(const M2Arg
     float *scoef = reinterpret_cast<float *>(scr + SC.scoef);
     float *sdec = reinterpret_cast<float *>(scr + SC.sdec);
     float *su = reinterpret_cast<float *>(scr + SC.su);
+    float *sfdec = reinterpret_cast<float *>(scr + SC.sfdec);
     float *sdot = reinterpret_cast<float *>(scr + SC.sdot);
     float *sCf = reinterpret_cast<float *>(scr + SC.sCf);
-    int *vote = reinterpret_cast<int *>(scr + SC.flag);
-    const int c = tid % TPR;
+    // read mapping: LPR lanes per state row, CPL chunks per lane, rotated so the
+    // rows of a warp spread over all shared-memory banks
+    constexpr int LPR = TPR < 4 ? TPR : 4;
+    constexpr int CPL = TPR / LPR;
+    constexpr int RPPR = kThreads / LPR;
+    constexpr bool kCregs = TQ * CPL * EPC <= 32;
+    const int q = tid % LPR, rrow = tid / LPR, rot = rrow % CPL;
+    // fold mapping: TPR4 lanes per row (quads), FR rows per thread per unit
+    constexpr int FR = 8;  // = (kTileCap / (N * 4)) / RPP4 for every N
+    static_assert(FR * RPP4 * N * 4 == kTileCap, "fold unit is FR rows per thread");
+    const int c4 = tid % TPR4, q0 = tid / TPR4;
     int s = 0;
     uint32_t fphase = 0;
     for (;;) {
         const bool got = mbar_wait(&full[s], (fphase >> s) & 1u);
-        if (tid == 0) vote[0] = 0;
-        consumer_sync();
-        if (!got) atomicOr(&vote[0], 1);
-        consumer_sync();
-        if (vote[0]) {
+        if (consumer_sync_any(!got)) {
             if (tid == 0) report(a.c.err, DEV_PIPE_TIMEOUT, -1, -1, 3);
             break;
         }
@@ -358,127 +364,156 @@ __global__ void __launch_bounds__(kThreads + 32, 1) m2_replay_kernel(const M2Arg
                 }
             }
             consumer_sync();
-            if (reads) {
-                for (int i = tid; i < HC * T * nE; i += kThreads) {
-                    const int hh = i / (T * nE), r2 = i - hh * T * nE;
-                    const int m = r2 / nE, e = r2 - m * nE;
-                    if (e < e0 || e > L0 + m) continue;
-                    const float *lam = slam + hh * E + base;
-                    scoef[(hh * TQ + m) * E + e] = expf(lam[L0 + m] - lam[e]) * sd[m * E + e] *
-                                                   (a.dt_scales ? sdt[hh * E + base + e] : 1.f);
+            for (int i = tid; i < HC * nE; i += kThreads) {
+                const int hh = i / nE, e = i - hh * nE;
+                const float *lam = slam + hh * E + base;
+                const float se = a.dt_scales ? sdt[hh * E + base + e] : 1.f;
+                if (reads) {
+#pragma unroll
+                    for (int m = 0; m < TQ; ++m)
+                        if (m < T && e >= e0 && e <= L0 + m)
+                            scoef[(hh * TQ + m) * E + e] = expf(lam[L0 + m] - lam[e]) * sd[m * E + e] * se;
                 }
-                for (int i = tid; i < HC * T; i += kThreads) {
-                    const int hh = i / T, m = i - hh * T;
-                    const float *lam = slam + hh * E + base;
-                    sdec[hh * TQ + m] = expf(lam[L0 + m] - (flush ? lam[L0 - 1] : 0.f));
-                }
+                if (flush && e < L0) su[hh * E + e] = expf(lam[L0 - 1] - lam[e]) * se;
             }
-            if (flush) {
-                for (int i = tid; i < HC * L0; i += kThreads) {
-                    const int hh = i / L0, e = i - hh * L0;
-                    const float *lam = slam + hh * E + base;
-                    su[hh * E + e] = expf(lam[L0 - 1] - lam[e]) * (a.dt_scales ? sdt[hh * E + base + e] : 1.f);
-                }
+            for (int i = tid; i < HC; i += kThreads) {
+                const float *lam = slam + i * E + base;
+                sfdec[i] = flush ? expf(lam[L0 - 1]) : 1.f;
+#pragma unroll
+                for (int m = 0; m < TQ; ++m)
+                    if (reads && m < T) sdec[i * TQ + m] = expf(lam[L0 + m] - (flush ? lam[L0 - 1] : 0.f));
             }
             consumer_sync();
         }
 
         if (flush) {
-            // Fold this part's fp32 checkpoint rows (from the stage), store the
+            // Fold this part's fp32 checkpoint rows (staged), FR rows per thread held
+            // in registers, buffered B applied 8 entries at a time; store the
             // checkpoint and the requantised copy, dot the fresh copy with C.
-            const int c4 = tid % TPR4, q0 = tid / TPR4;
-            const int rpp = rpp_fold;
-            const int r0 = part * rpp, r1 = min(nrows, r0 + rpp);
+            const int r0 = part * rpp_fold, nr = min(nrows, r0 + rpp_fold) - r0;
             const float *tf = reinterpret_cast<const float *>(st + SG.tile);
             float4 Cq[TQ];
 #pragma unroll
             for (int m = 0; m < TQ; ++m)
                 Cq[m] = (reads && m < T) ? *reinterpret_cast<const float4 *>(sCf + m * N + 4 * c4)
                                          : make_float4(0.f, 0.f, 0.f, 0.f);
-            for (int rb = 0; rb < rpp; rb += RPP4) {  // same trip count for every lane
-                const int rl = rb + q0;
-                const int gr = r0 + rl;
-                const bool valid = rl < rpp && gr < r1;
-                const int hh = valid ? gr / P : 0, p = valid ? gr - hh * P : 0;
-                float4 v = valid ? *reinterpret_cast<const float4 *>(tf + rl * N + 4 * c4)
-                                 : make_float4(0.f, 0.f, 0.f, 0.f);
-                if (valid) {
-                    const float dec_all = expf(slam[hh * E + base + L0 - 1]);
-                    v.x *= dec_all; v.y *= dec_all; v.z *= dec_all; v.w *= dec_all;
-                    for (int e = 0; e < L0; ++e) {
-                        const float w = su[hh * E + e] * raw_f(sx + (hh * E + base + e) * xrow, p, bf);
-                        const uint8_t *Br = sB + (base + e) * brow;
-                        v.x = fmaf(w, raw_f(Br, 4 * c4, bf), v.x);
-                        v.y = fmaf(w, raw_f(Br, 4 * c4 + 1, bf), v.y);
-                        v.z = fmaf(w, raw_f(Br, 4 * c4 + 2, bf), v.z);
-                        v.w = fmaf(w, raw_f(Br, 4 * c4 + 3, bf), v.w);
-                    }
-                }
-                const int64_t el = tile0 + (int64_t)(valid ? gr : 0) * N + 4 * c4;
-                if (a.op == OP_EXPORT) {
-                    if (valid) *reinterpret_cast<float4 *>(a.out + el) = v;
-                    continue;
-                }
-                if (valid) *reinterpret_cast<float4 *>(a.ckpt + el) = v;
-                float4 rd = v;
-                if (RK == SK_BF16) {
-                    if (valid) rd = store_quad<SK_BF16>(a.rc, el, v, 0.f, 0.f);
-                } else if (RK == SK_FP8) {
-                    float am = fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
-                    am = group_max<TPR4>(am);
-                    const float sc = fp8_scale(am);
-                    if (valid) {
-                        rd = store_quad<SK_FP8>(a.rc, el, v, 0.f, sc);
-                        if (c4 == 0) a.rc_scale[row0 * P + gr] = sc;
-                    }
-                }
-                if (reads) {
+            constexpr int FH = 4;  // rows in registers at a time
+#pragma unroll 1
+            for (int kh = 0; kh < FR; kh += FH) {
+                float4 v[FH];
 #pragma unroll
-                    for (int m = 0; m < TQ; ++m) {
-                        float d = rd.x * Cq[m].x + rd.y * Cq[m].y + rd.z * Cq[m].z + rd.w * Cq[m].w;
-                        d = group_sum<TPR4>(d);
-                        if (c4 == 0 && valid && m < T) sdot[gr * TQ + m] = d;
+                for (int k = 0; k < FH; ++k) {
+                    const int rl = q0 + (kh + k) * RPP4;
+                    v[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+                    if (rl < nr) {
+                        v[k] = *reinterpret_cast<const float4 *>(tf + rl * N + 4 * c4);
+                        const float dc = sfdec[(r0 + rl) / P];
+                        v[k].x *= dc; v[k].y *= dc; v[k].z *= dc; v[k].w *= dc;
+                    }
+                }
+#pragma unroll 1
+                for (int eb = 0; eb < L0; eb += 8) {
+                    float4 Bq[8];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const uint8_t *Br = sB + (base + eb + j) * brow;
+                        Bq[j] = (eb + j < L0) ? make_float4(raw_f(Br, 4 * c4, bf), raw_f(Br, 4 * c4 + 1, bf),
+                                                            raw_f(Br, 4 * c4 + 2, bf), raw_f(Br, 4 * c4 + 3, bf))
+                                              : make_float4(0.f, 0.f, 0.f, 0.f);
+                    }
+#pragma unroll
+                    for (int k = 0; k < FH; ++k) {
+                        const int rl = q0 + (kh + k) * RPP4;
+                        if (rl >= nr) continue;
+                        const int gr = r0 + rl, hh = gr / P, p = gr - hh * P;
+                        const uint8_t *xr = sx + (hh * E + base + eb) * xrow;
+                        const float *uw = su + hh * E + eb;
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            if (eb + j < L0) {
+                                const float w = uw[j] * raw_f(xr + j * xrow, p, bf);
+                                v[k].x = fmaf(w, Bq[j].x, v[k].x); v[k].y = fmaf(w, Bq[j].y, v[k].y);
+                                v[k].z = fmaf(w, Bq[j].z, v[k].z); v[k].w = fmaf(w, Bq[j].w, v[k].w);
+                            }
+                        }
+                    }
+                }
+#pragma unroll
+                for (int k = 0; k < FH; ++k) {
+                    const int rl = q0 + (kh + k) * RPP4;
+                    const bool valid = rl < nr;
+                    const int gr = r0 + rl;
+                    const int64_t el = tile0 + (int64_t)(valid ? gr : 0) * N + 4 * c4;
+                    if (a.op == OP_EXPORT) {
+                        if (valid) *reinterpret_cast<float4 *>(a.out + el) = v[k];
+                        continue;
+                    }
+                    if (valid) *reinterpret_cast<float4 *>(a.ckpt + el) = v[k];
+                    float4 rd = v[k];
+                    if (RK == SK_BF16) {
+                        if (valid) rd = store_quad<SK_BF16>(a.rc, el, v[k], 0.f, 0.f);
+                    } else if (RK == SK_FP8) {
+                        float am = fmaxf(fmaxf(fabsf(v[k].x), fabsf(v[k].y)), fmaxf(fabsf(v[k].z), fabsf(v[k].w)));
+                        am = group_max<TPR4>(am);
+                        const float sc = fp8_scale(am);
+                        if (valid) {
+                            rd = store_quad<SK_FP8>(a.rc, el, v[k], 0.f, sc);
+                            if (c4 == 0) a.rc_scale[row0 * P + gr] = sc;
+                        }
+                    }
+                    if (reads) {
+#pragma unroll
+                        for (int m = 0; m < TQ; ++m) {
+                            float d = rd.x * Cq[m].x + rd.y * Cq[m].y + rd.z * Cq[m].z + rd.w * Cq[m].w;
+                            d = group_sum<TPR4>(d);
+                            if (c4 == 0 && valid && m < T) sdot[gr * TQ + m] = d;
+                        }
                     }
                 }
             }
         } else if (reads) {
-            // Read: every 16-byte chunk of the staged read copy dotted with C.
-            constexpr bool kCregs = TQ * EPC <= 64;
-            float Cr[kCregs ? TQ : 1][kCregs ? EPC : 1];
+            // Read: LPR lanes per staged read-copy row, C fragments in registers.
+            float Cf[kCregs ? TQ : 1][kCregs ? CPL * EPC : 1];
             if (kCregs) {
 #pragma unroll
                 for (int m = 0; m < (kCregs ? TQ : 1); ++m)
 #pragma unroll
-                    for (int j = 0; j < (kCregs ? EPC : 1); ++j)
-                        Cr[m][j] = (m < T) ? sCf[m * N + c * EPC + j] : 0.f;
+                    for (int k = 0; k < (kCregs ? CPL : 1); ++k)
+#pragma unroll
+                        for (int e = 0; e < (kCregs ? EPC : 1); ++e)
+                            Cf[m][k * EPC + e] =
+                                (m < T) ? sCf[m * N + (q + LPR * ((k + rot) % CPL)) * EPC + e] : 0.f;
             }
             const uint4 *tile = reinterpret_cast<const uint4 *>(st + SG.tile);
             const float *ssc = reinterpret_cast<const float *>(st + SG.scale);
-            const int r0 = part * rpp_read, r1 = min(nrows, r0 + rpp_read);
-            const int nchunks = (r1 - r0) * TPR;
-#pragma unroll 4
-            for (int cb = 0; cb < nchunks; cb += kThreads) {  // same trip count for every lane
-                const int idx = cb + tid;
-                const bool valid = idx < nchunks;
-                float v[EPC];
-                if (valid) unpack<RK>(tile[idx], v);
-                else {
+            const int r0 = part * rpp_read, nr = min(nrows, r0 + rpp_read) - r0;
+            for (int rb = 0; rb < nr; rb += RPPR) {  // same trip count for every lane
+                const int rl = rb + rrow;
+                const bool valid = rl < nr;
+                float acc[TQ];
 #pragma unroll
-                    for (int q = 0; q < EPC; ++q) v[q] = 0.f;
+                for (int m = 0; m < TQ; ++m) acc[m] = 0.f;
+#pragma unroll
+                for (int k = 0; k < CPL; ++k) {
+                    const int ch = q + LPR * ((k + rot) % CPL);
+                    float vv[EPC];
+                    if (valid) unpack<RK>(tile[rl * TPR + ch], vv);
+                    else {
+#pragma unroll
+                        for (int e = 0; e < EPC; ++e) vv[e] = 0.f;
+                    }
+#pragma unroll
+                    for (int m = 0; m < TQ; ++m)
+#pragma unroll
+                        for (int e = 0; e < EPC; ++e)
+                            acc[m] = fmaf(vv[e], kCregs ? Cf[kCregs ? m : 0][kCregs ? k * EPC + e : 0]
+                                                        : sCf[m * N + ch * EPC + e], acc[m]);
                 }
 #pragma unroll
                 for (int m = 0; m < TQ; ++m) {
-                    float d = 0.f;
-                    if (kCregs) {
-#pragma unroll
-                        for (int q = 0; q < EPC; ++q) d = fmaf(v[q], Cr[kCregs ? m : 0][kCregs ? q : 0], d);
-                    } else {
-#pragma unroll
-                        for (int q = 0; q < EPC; ++q) d = fmaf(v[q], sCf[m * N + c * EPC + q], d);
-                    }
-                    d = group_sum<TPR>(d);
-                    if (c == 0 && valid && m < T)
-                        sdot[(r0 + idx / TPR) * TQ + m] = (RK == SK_FP8) ? d * ssc[idx / TPR] : d;
+                    const float d = group_sum<LPR>(acc[m]);
+                    if (q == 0 && valid && m < T)
+                        sdot[(r0 + rl) * TQ + m] = (RK == SK_FP8) ? d * ssc[rl] : d;
                 }
             }
         }

@@ -74,4 +74,15 @@ __device__ __forceinline__ void consumer_sync() {
     asm volatile("bar.sync 1, %0;" ::"n"(kThreads) : "memory");
 }
 
+// Consumer barrier that also returns whether any consumer thread passed `bad`.
+__device__ __forceinline__ bool consumer_sync_any(bool bad) {
+    uint32_t any;
+    asm volatile(
+        "{\n .reg .pred p, q;\n setp.ne.u32 q, %1, 0;\n bar.red.or.pred p, 1, %2, q;\n selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(any)
+        : "r"((uint32_t)bad), "n"(kThreads)
+        : "memory");
+    return any != 0;
+}
+
 }  // namespace rssm
