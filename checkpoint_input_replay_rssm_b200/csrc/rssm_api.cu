@@ -64,6 +64,8 @@ void layout(const rssm_config *c, rssm_workspace_layout *L) {
     L->D_off = take(H * 4);
     L->ring = (size_t)c->window + (size_t)(c->max_draft > 1 ? c->max_draft : 1);
     const size_t R = L->ring;
+    L->ring_stride = (R + 3) & ~(size_t)3;
+    const size_t Rs = L->ring_stride;
     if (replay || c->state_dtype == RSSM_F32) {
         L->ckpt_bytes = elems * 4;
         L->ckpt_off = take(L->ckpt_bytes);
@@ -81,10 +83,10 @@ void layout(const rssm_config *c, rssm_workspace_layout *L) {
         L->xbuf_off = take(L->xbuf_bytes);
         L->bbuf_bytes = B * G * R * N * ib;
         L->bbuf_off = take(L->bbuf_bytes);
-        L->sbuf_bytes = B * H * R * 4;
+        L->sbuf_bytes = B * H * Rs * 4;
         L->sbuf_off = take(L->sbuf_bytes);
         if (c->kind == RSSM_GDN) {
-            L->tbuf_bytes = B * H * R * 4;
+            L->tbuf_bytes = B * H * Rs * 4;
             L->tbuf_off = take(L->tbuf_bytes);
         }
     } else if (c->max_draft > 0) {

@@ -20,7 +20,7 @@ cudaError_t gdn_launch(const Ctx &h, int op, int T, const rssm_inputs *in, float
     GArgs a{};
     const rssm_config &cf = h.cfg;
     a.B = cf.batch; a.H = cf.nheads; a.P = cf.headdim; a.W = cf.window;
-    a.R = (int)h.lay.ring; a.T = T; a.op = op; a.in_bf16 = cf.input_dtype == RSSM_BF16;
+    a.R = (int)h.lay.ring; a.Rs = (int)h.lay.ring_stride; a.T = T; a.op = op; a.in_bf16 = cf.input_dtype == RSSM_BF16;
     a.c = h.counters();
     a.ckpt = h.lay.ckpt_bytes ? (float *)h.at(h.lay.ckpt_off) : nullptr;
     a.rc = h.lay.rc_bytes ? h.at(h.lay.rc_off) : nullptr;

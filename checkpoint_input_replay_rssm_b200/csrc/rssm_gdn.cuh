@@ -24,7 +24,7 @@
 namespace rssm {
 
 struct GArgs {
-    int B, H, P, W, R, T, op, in_bf16;
+    int B, H, P, W, R, Rs, T, op, in_bf16;  // Rs: row length of the scalar rings
     Counters c;
     float *ckpt;
     void *rc;
@@ -203,7 +203,7 @@ __global__ void __launch_bounds__(kThreads) gdn_replay_kernel(const GArgs a) {
         s.sv[(base + e) * P + p] = ld_in(a.vbuf, ((int64_t)bh * R + (ckmod + e) % R) * P + p, a.in_bf16);
     }
     for (int e = tid; e < L0; e += kThreads) {
-        const int64_t slot = (int64_t)bh * R + (ckmod + e) % R;
+        const int64_t slot = (int64_t)bh * a.Rs + (ckmod + e) % R;
         s.sal[base + e] = a.abuf[slot];
         s.sbe[base + e] = a.bbuf[slot];
     }
@@ -407,7 +407,7 @@ __global__ void __launch_bounds__(kThreads) gdn_replay_kernel(const GArgs a) {
                 ((int64_t)(b * T + m) * H + h) * P + p, a.in_bf16);
     }
     if (tid < T) {
-        const int64_t slot = (int64_t)bh * R + (spmod + tid) % R;
+        const int64_t slot = (int64_t)bh * a.Rs + (spmod + tid) % R;
         a.abuf[slot] = s.sal[W + tid];
         a.bbuf[slot] = s.sbe[W + tid];
     }

@@ -22,7 +22,7 @@ static M2Pipe m2_pipe(const rssm_config &cf, int TQ) {
     auto total = [&](int hc, int ns) {
         return m2_smem_total(ns, hc, cf.headdim, cf.dstate, cf.window, TQ, ib, rcb);
     };
-    for (int hc : {2, 1, 4}) {
+    for (int hc : {4, 2, 1}) {
         if (hpg % hc != 0) continue;
         for (int ns = 3; ns >= 2; --ns)
             if (total(hc, ns) <= 110 * 1024) return {hc, ns, 2, (size_t)total(hc, ns)};
@@ -49,7 +49,7 @@ cudaError_t mamba2_launch(const Ctx &h, int op, int T, const rssm_inputs *in, fl
     M2Args a{};
     const rssm_config &cf = h.cfg;
     a.B = cf.batch; a.H = cf.nheads; a.P = cf.headdim; a.G = cf.ngroups; a.W = cf.window;
-    a.R = (int)h.lay.ring; a.T = T; a.op = op; a.in_bf16 = cf.input_dtype == RSSM_BF16;
+    a.R = (int)h.lay.ring; a.Rs = (int)h.lay.ring_stride; a.T = T; a.op = op; a.in_bf16 = cf.input_dtype == RSSM_BF16;
     a.dt_scales = cf.dt_scales_input;
     const M2Pipe pp = m2_pipe(cf, tq_of(T));
     a.HC = pp.HC;

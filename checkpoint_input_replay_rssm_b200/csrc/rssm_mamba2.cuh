@@ -29,7 +29,7 @@
 namespace rssm {
 
 struct M2Args {
-    int B, H, P, G, W, R, T, op, in_bf16, dt_scales;
+    int B, H, P, G, W, R, Rs, T, op, in_bf16, dt_scales;  // Rs: dt ring row length
     int HC;             // heads per replay item (divides H / G)
     int NS;             // pipeline stages of the replay kernel
     int grid;           // persistent CTAs of the replay kernel
@@ -62,8 +62,11 @@ __host__ __device__ constexpr int pad4(int n) { return (n + 3) & ~3; }
 // tokens.  Entry slots: E = W + TQ; committed entries sit right-aligned before
 // slot W and this call's tokens at W..W+T-1.
 struct M2Stage {
-    int tile, scale, x, B, C, dt, info, bytes;
+    int tile, scale, x, B, C, dt, dtn, info, bytes;
 };
+// Upper bound of a dt ring row in bytes: the ring has R = W + max(max_draft, 1) <= W + 8
+// slots, rows padded to 4 floats.
+__host__ __device__ constexpr int dt_row_max_bytes(int W) { return ((W + 8 + 3) & ~3) * 4; }
 constexpr int kTileCap = 32 * 1024;  // bytes of state rows per pipeline unit
 
 __host__ __device__ inline M2Stage m2_stage(int HC, int P, int N, int W, int TQ, int ib, int rcb) {
@@ -75,7 +78,8 @@ __host__ __device__ inline M2Stage m2_stage(int HC, int P, int N, int W, int TQ,
     S.x = o;     o += a16(HC * E * P * ib);            // x of entries   [HC][E][P]
     S.B = o;     o += a16(E * N * ib);                 // B of entries   [E][N]
     S.C = o;     o += a16(TQ * N * ib);                // C of queries   [TQ][N]
-    S.dt = o;    o += a16(HC * E * 4);                 // dt of entries  [HC][E]
+    S.dt = o;    o += a16(HC * dt_row_max_bytes(W));   // dt ring rows   [HC][Rs]
+    S.dtn = o;   o += a16(TQ * HC * 4);                // dt of this call's tokens [TQ][HC]
     S.info = o;  o += 64;                              // unit descriptor
     S.bytes = o;
     return S;
@@ -83,7 +87,7 @@ __host__ __device__ inline M2Stage m2_stage(int HC, int P, int N, int W, int TQ,
 
 // Consumer-side scratch, shared by all units (bytes).
 struct M2Scratch {
-    int sd, slam, scoef, sdec, su, sfdec, sdot, sCf, bytes;
+    int sd, slam, scoef, sdec, su, sfdec, sdot, sCf, pdt, bytes;
 };
 __host__ __device__ inline M2Scratch m2_scratch(int HC, int P, int N, int W, int TQ) {
     const int E = W + TQ;
@@ -97,6 +101,7 @@ __host__ __device__ inline M2Scratch m2_scratch(int HC, int P, int N, int W, int
     S.sfdec = o; o += a16(HC * 4);           // decay of the folded checkpoint [HC]
     S.sdot = o;  o += a16(HC * P * TQ * 4);  // S^ C per state row    [HC*P][TQ]
     S.sCf = o;   o += a16(TQ * N * 4);       // C as fp32             [TQ][N]
+    S.pdt = o;   o += a16(32 * HC * TQ * 4); // producer: dt of its 32 prefetched items
     S.bytes = o;
     return S;
 }
@@ -163,6 +168,12 @@ __global__ void __maxnreg__(112) m2_replay_kernel(const M2Args a) {
 
     if (warp == kWarps) {
         // ================================ producer ================================
+        // Items are taken 32 at a time: lane j loads the counters and the token dt's
+        // of the j-th item of the batch (one memory round trip per 32 items); then
+        // the items' units are queued in order.
+        float *pdt = reinterpret_cast<float *>(scr + SC.pdt);
+        const int HT = HC * T;
+        const int nper = H / HC;  // items per sequence
         int s = 0;
         uint32_t used = 0, ephase = 0;
         bool dead = false;
@@ -178,107 +189,104 @@ __global__ void __maxnreg__(112) m2_replay_kernel(const M2Args a) {
             used |= 1u << st;
             return true;
         };
-        for (int item = blockIdx.x; item < nitems && !dead; item += gridDim.x) {
-            const int b = item / (H / HC);
-            const int rem = item - b * (H / HC);
-            const int g = rem / cpg, hc = rem - g * cpg;
-            const int h0 = g * hpg + hc * HC;
-            const int64_t row0 = (int64_t)b * H + h0;
-            const int64_t tile0 = row0 * P * N;
+        for (int bstart = blockIdx.x; bstart < nitems && !dead; bstart += 32 * gridDim.x) {
+            const int mine = bstart + lane * gridDim.x;
             int ok = 0, L0 = 0, flush = 0, ckmod = 0, spmod = 0;
-            if (lane == 0) {
+            if (mine < nitems) {
+                const int b = mine / nper, rem = mine - b * nper;
+                const int g = rem / cpg, hc = rem - g * cpg, h0 = g * hpg + hc * HC;
+                for (int i = 0; i < HT; ++i) {
+                    const int m = i / HC, hh = i - m * HC;
+                    pdt[lane * HT + i] = a.dt[(int64_t)(b * T + m) * H + h0 + hh];
+                }
                 SeqState ss = read_counters(a.c, b, W);
                 ok = ss.ok;
                 L0 = (int)(ss.seq - ss.ckpt);
                 if (ok) flush = (a.op == OP_FLUSH || a.op == OP_EXPORT) ? (L0 > 0) : (L0 + T > W);
                 ckmod = (int)(ss.ckpt % R);
                 spmod = (int)(ss.seq % R);
-                if (!ok) {
-                    if (g == 0 && hc == 0) report(a.c.err, DEV_BAD_COUNTERS, b, h0, L0);
-                } else if (a.op != OP_EXPORT) {
-                    arrive_and_publish(a.c, b, H / HC, (a.op == OP_DECODE) ? ss.seq + 1 : -1,
-                                       flush ? ss.seq : -1, (a.op == OP_VERIFY) ? T : -1, flush);
-                }
+                if (!ok && g == 0 && hc == 0) report(a.c.err, DEV_BAD_COUNTERS, b, h0, L0);
             }
-            ok = __shfl_sync(0xffffffffu, ok, 0);
-            L0 = __shfl_sync(0xffffffffu, L0, 0);
-            flush = __shfl_sync(0xffffffffu, flush, 0);
-            ckmod = __shfl_sync(0xffffffffu, ckmod, 0);
-            spmod = __shfl_sync(0xffffffffu, spmod, 0);
-            const int nparts = !ok ? 0 : (flush ? fold_parts : (reads ? read_parts : 0));
-            const int base = W - L0;
-            const int n1 = min(L0, R - ckmod);  // entries before the ring wraps
-            for (int part = 0; part < nparts; ++part) {
-                if (!acquire(s)) {
-                    if (lane == 0) report(a.c.err, DEV_PIPE_TIMEOUT, b, h0, 1);
-                    dead = true;
-                    break;
-                }
-                uint8_t *st = stages + s * SG.bytes;
-                int *info = reinterpret_cast<int *>(st + SG.info);
-                float *sdt = reinterpret_cast<float *>(st + SG.dt);
-                if (lane == 0) {
-                    info[INFO_ITEM] = item; info[INFO_PART] = part; info[INFO_NPARTS] = nparts;
-                    info[INFO_L0] = L0; info[INFO_FLUSH] = flush; info[INFO_CKMOD] = ckmod;
-                    info[INFO_SPMOD] = spmod;
-                }
-                for (int i = lane; i < HC * L0; i += 32) {
-                    const int hh = i / L0, e = i - hh * L0;
-                    sdt[hh * E + base + e] = a.dtbuf[(row0 + hh) * R + (ckmod + e) % R];
-                }
-                for (int i = lane; i < HC * T; i += 32) {
-                    const int m = i / HC, hh = i - m * HC;
-                    sdt[hh * E + W + m] = a.dt[(int64_t)(b * T + m) * H + h0 + hh];
-                }
-                // The unit's bulk copies: the same list is walked twice, once to
-                // total the bytes, once to issue (copy k by lane k mod 32).
-                uint32_t tx = 0;
-                int ci = 0;
-                auto copy = [&](bool issue, void *dst, const void *src, uint32_t bytes) {
-                    if (bytes == 0) return;
-                    if (!issue) tx += bytes;
-                    else if ((ci & 31) == lane) bulk_g2s(dst, src, bytes, &full[s]);
-                    ++ci;
-                };
-                auto walk = [&](bool issue) {
-                    ci = 0;
-                    if (flush) {
-                        const int r0 = part * rpp_fold, r1 = min(nrows, r0 + rpp_fold);
-                        copy(issue, st + SG.tile, a.ckpt + tile0 + (int64_t)r0 * N, (uint32_t)((r1 - r0) * N * 4));
-                    } else {
-                        const int r0 = part * rpp_read, r1 = min(nrows, r0 + rpp_read);
-                        const uint8_t *rc = (RK == SK_F32) ? reinterpret_cast<const uint8_t *>(a.ckpt + tile0)
-                                                           : reinterpret_cast<const uint8_t *>(a.rc) + tile0 * RCB;
-                        copy(issue, st + SG.tile, rc + (int64_t)r0 * N * RCB, (uint32_t)((r1 - r0) * N * RCB));
-                        if (RK == SK_FP8)
-                            copy(issue, st + SG.scale, a.rc_scale + row0 * P + r0, (uint32_t)((r1 - r0) * 4));
+            __syncwarp();
+            for (int j = 0; j < 32 && !dead; ++j) {
+                const int item = bstart + j * gridDim.x;
+                if (item >= nitems) break;
+                const int iok = __shfl_sync(0xffffffffu, ok, j);
+                const int iL0 = __shfl_sync(0xffffffffu, L0, j);
+                const int ifl = __shfl_sync(0xffffffffu, flush, j);
+                const int ick = __shfl_sync(0xffffffffu, ckmod, j);
+                const int isp = __shfl_sync(0xffffffffu, spmod, j);
+                const int b = item / nper, rem = item - b * nper;
+                const int g = rem / cpg, hc = rem - g * cpg, h0 = g * hpg + hc * HC;
+                const int64_t row0 = (int64_t)b * H + h0;
+                const int64_t tile0 = row0 * P * N;
+                const int nparts = !iok ? 0 : (ifl ? fold_parts : (reads ? read_parts : 0));
+                const int base = W - iL0;
+                const int n1 = min(iL0, R - ick);  // entries before the ring wraps
+                for (int part = 0; part < nparts; ++part) {
+                    if (!acquire(s)) {
+                        if (lane == 0) report(a.c.err, DEV_PIPE_TIMEOUT, b, h0, 1);
+                        dead = true;
+                        break;
                     }
-                    const uint8_t *Bb = reinterpret_cast<const uint8_t *>(a.Bbuf) + ((int64_t)(b * G + g) * R) * brow;
-                    copy(issue, st + SG.B + base * brow, Bb + (int64_t)ckmod * brow, (uint32_t)(n1 * brow));
-                    copy(issue, st + SG.B + (base + n1) * brow, Bb, (uint32_t)((L0 - n1) * brow));
-                    for (int hh = 0; hh < HC; ++hh) {
-                        const uint8_t *xb = reinterpret_cast<const uint8_t *>(a.xbuf) + ((row0 + hh) * R) * xrow;
-                        uint8_t *xd = st + SG.x + (hh * E + base) * xrow;
-                        copy(issue, xd, xb + (int64_t)ckmod * xrow, (uint32_t)(n1 * xrow));
-                        copy(issue, xd + n1 * xrow, xb, (uint32_t)((L0 - n1) * xrow));
+                    uint8_t *st = stages + s * SG.bytes;
+                    int *info = reinterpret_cast<int *>(st + SG.info);
+                    float *dtn = reinterpret_cast<float *>(st + SG.dtn);
+                    if (lane == 0) {
+                        info[INFO_ITEM] = item; info[INFO_PART] = part; info[INFO_NPARTS] = nparts;
+                        info[INFO_L0] = iL0; info[INFO_FLUSH] = ifl; info[INFO_CKMOD] = ick;
+                        info[INFO_SPMOD] = isp;
                     }
-                    for (int m = 0; m < T; ++m) {
-                        const int64_t gsrc = (((int64_t)(b * T + m) * G + g) * N) * ib;
-                        copy(issue, st + SG.C + m * brow, reinterpret_cast<const uint8_t *>(a.Cm) + gsrc, (uint32_t)brow);
-                        copy(issue, st + SG.B + (W + m) * brow, reinterpret_cast<const uint8_t *>(a.Bm) + gsrc, (uint32_t)brow);
-                        // x of the HC heads for token m is contiguous
-                        uint8_t *xd = st + SG.x + W * xrow + m * xrow;  // head 0 slot W + m
-                        const uint8_t *xs = reinterpret_cast<const uint8_t *>(a.x) + (((int64_t)(b * T + m) * H + h0) * P) * ib;
-                        for (int hh = 0; hh < HC; ++hh)
-                            copy(issue, xd + hh * E * xrow, xs + hh * xrow, (uint32_t)xrow);
-                    }
-                };
-                walk(false);
-                if (lane == 0) mbar_arrive_expect_tx(&full[s], tx);
-                else mbar_arrive(&full[s]);
-                __syncwarp();
-                walk(true);
-                s = (s + 1 == NS) ? 0 : s + 1;
+                    for (int i = lane; i < HT; i += 32) dtn[i] = pdt[j * HT + i];
+                    // The unit's bulk copies: the same list is walked twice, once to
+                    // total the bytes, once to issue (copy k by lane k mod 32).
+                    uint32_t tx = 0;
+                    int ci = 0;
+                    auto copy = [&](bool issue, void *dst, const void *src, uint32_t bytes) {
+                        if (bytes == 0) return;
+                        if (!issue) tx += bytes;
+                        else if ((ci & 31) == lane) bulk_g2s(dst, src, bytes, &full[s]);
+                        ++ci;
+                    };
+                    auto walk = [&](bool issue) {
+                        ci = 0;
+                        if (ifl) {
+                            const int r0 = part * rpp_fold, r1 = min(nrows, r0 + rpp_fold);
+                            copy(issue, st + SG.tile, a.ckpt + tile0 + (int64_t)r0 * N, (uint32_t)((r1 - r0) * N * 4));
+                        } else {
+                            const int r0 = part * rpp_read, r1 = min(nrows, r0 + rpp_read);
+                            const uint8_t *rc = (RK == SK_F32) ? reinterpret_cast<const uint8_t *>(a.ckpt + tile0)
+                                                               : reinterpret_cast<const uint8_t *>(a.rc) + tile0 * RCB;
+                            copy(issue, st + SG.tile, rc + (int64_t)r0 * N * RCB, (uint32_t)((r1 - r0) * N * RCB));
+                            if (RK == SK_FP8)
+                                copy(issue, st + SG.scale, a.rc_scale + row0 * P + r0, (uint32_t)((r1 - r0) * 4));
+                        }
+                        copy(issue, st + SG.dt, a.dtbuf + row0 * a.Rs, (uint32_t)(HC * a.Rs * 4));
+                        const uint8_t *Bb = reinterpret_cast<const uint8_t *>(a.Bbuf) + ((int64_t)(b * G + g) * R) * brow;
+                        copy(issue, st + SG.B + base * brow, Bb + (int64_t)ick * brow, (uint32_t)(n1 * brow));
+                        copy(issue, st + SG.B + (base + n1) * brow, Bb, (uint32_t)((iL0 - n1) * brow));
+                        for (int hh = 0; hh < HC; ++hh) {
+                            const uint8_t *xb = reinterpret_cast<const uint8_t *>(a.xbuf) + ((row0 + hh) * R) * xrow;
+                            uint8_t *xd = st + SG.x + (hh * E + base) * xrow;
+                            copy(issue, xd, xb + (int64_t)ick * xrow, (uint32_t)(n1 * xrow));
+                            copy(issue, xd + n1 * xrow, xb, (uint32_t)((iL0 - n1) * xrow));
+                        }
+                        for (int m = 0; m < T; ++m) {
+                            const int64_t gsrc = (((int64_t)(b * T + m) * G + g) * N) * ib;
+                            copy(issue, st + SG.C + m * brow, reinterpret_cast<const uint8_t *>(a.Cm) + gsrc, (uint32_t)brow);
+                            copy(issue, st + SG.B + (W + m) * brow, reinterpret_cast<const uint8_t *>(a.Bm) + gsrc, (uint32_t)brow);
+                            const uint8_t *xs = reinterpret_cast<const uint8_t *>(a.x) + (((int64_t)(b * T + m) * H + h0) * P) * ib;
+                            for (int hh = 0; hh < HC; ++hh)
+                                copy(issue, st + SG.x + (hh * E + W + m) * xrow, xs + hh * xrow, (uint32_t)xrow);
+                        }
+                    };
+                    walk(false);
+                    if (lane == 0) mbar_arrive_expect_tx(&full[s], tx);
+                    else mbar_arrive(&full[s]);
+                    __syncwarp();
+                    walk(true);
+                    s = (s + 1 == NS) ? 0 : s + 1;
+                }
             }
         }
         if (!dead && acquire(s)) {  // end-of-work unit
@@ -286,6 +294,34 @@ __global__ void __maxnreg__(112) m2_replay_kernel(const M2Args a) {
             mbar_arrive(&full[s]);
         } else if (lane == 0 && !dead) {
             report(a.c.err, DEV_PIPE_TIMEOUT, -1, -1, 2);
+        }
+        // Counters: every CTA has read all of its items' counters by now; the last
+        // CTA to get here publishes the new counters of every sequence.
+        if (a.op != OP_EXPORT) {
+            int last = 0;
+            if (lane == 0) {
+                __threadfence();
+                last = (atomicAdd(&a.c.err[4], 1) == (int)gridDim.x - 1) ? 1 : 0;
+            }
+            last = __shfl_sync(0xffffffffu, last, 0);
+            if (last) {
+                __threadfence();
+                for (int b = lane; b < a.B; b += 32) {
+                    SeqState ss = read_counters(a.c, b, W);
+                    if (!ss.ok) continue;
+                    const int L0 = (int)(ss.seq - ss.ckpt);
+                    const int flush = (a.op == OP_FLUSH) ? (L0 > 0) : (L0 + T > W);
+                    if (flush) {
+                        a.c.ckpt_pos[b] = ss.seq;
+                        a.c.flush_count[b] += 1;
+                    }
+                    if (a.op == OP_DECODE) a.c.seq_pos[b] = ss.seq + 1;
+                    if (a.op == OP_VERIFY) a.c.pending[b] = T;
+                }
+                __syncwarp();
+                if (lane == 0) a.c.err[4] = 0;
+                __threadfence();
+            }
         }
         return;
     }
@@ -325,6 +361,7 @@ __global__ void __maxnreg__(112) m2_replay_kernel(const M2Args a) {
         if (item < 0) break;
         const int part = info[INFO_PART], nparts = info[INFO_NPARTS];
         const int L0 = info[INFO_L0], flush = info[INFO_FLUSH], spmod = info[INFO_SPMOD];
+        const int ckmod = info[INFO_CKMOD];
         const int b = item / (H / HC);
         const int rem = item - b * (H / HC);
         const int g = rem / cpg, hc = rem - g * cpg;
@@ -336,7 +373,12 @@ __global__ void __maxnreg__(112) m2_replay_kernel(const M2Args a) {
         const uint8_t *sx = st + SG.x;
         const uint8_t *sB = st + SG.B;
         const uint8_t *sC = st + SG.C;
-        const float *sdt = reinterpret_cast<const float *>(st + SG.dt);
+        const float *dring = reinterpret_cast<const float *>(st + SG.dt);
+        const float *dtn = reinterpret_cast<const float *>(st + SG.dtn);
+        // dt of logical entry e (committed entries from the ring, then this call's tokens)
+        auto dt_of = [&](int hh, int e) -> float {
+            return e < L0 ? dring[hh * a.Rs + (ckmod + e) % R] : dtn[(e - L0) * HC + hh];
+        };
 
         if (part == 0) {
             // B_e . C_m once per item; C to fp32; prefix sums of dt*A per head.
@@ -357,7 +399,7 @@ __global__ void __maxnreg__(112) m2_replay_kernel(const M2Args a) {
                 float carry = 0.f;
                 for (int k0 = 0; k0 < nE; k0 += 32) {
                     const int e = k0 + lane;
-                    float v = (e < nE) ? sdt[hh * E + base + e] * Ah : 0.f;
+                    float v = (e < nE) ? dt_of(hh, e) * Ah : 0.f;
                     v = warp_incl_scan(v) + carry;
                     if (e < nE) slam[hh * E + base + e] = v;
                     carry = __shfl_sync(0xffffffffu, v, 31);
@@ -367,7 +409,7 @@ __global__ void __maxnreg__(112) m2_replay_kernel(const M2Args a) {
             for (int i = tid; i < HC * nE; i += kThreads) {
                 const int hh = i / nE, e = i - hh * nE;
                 const float *lam = slam + hh * E + base;
-                const float se = a.dt_scales ? sdt[hh * E + base + e] : 1.f;
+                const float se = a.dt_scales ? dt_of(hh, e) : 1.f;
                 if (reads) {
 #pragma unroll
                     for (int m = 0; m < TQ; ++m)
@@ -541,7 +583,7 @@ __global__ void __maxnreg__(112) m2_replay_kernel(const M2Args a) {
             }
             if (tid < T * HC) {
                 const int m = tid / HC, hh = tid - m * HC;
-                a.dtbuf[(row0 + hh) * R + (spmod + m) % R] = sdt[hh * E + W + m];
+                a.dtbuf[(row0 + hh) * a.Rs + (spmod + m) % R] = dtn[m * HC + hh];
             }
             if (hc == 0) {  // the group's first item writes the group's B
                 for (int i = tid; i < T * bch; i += kThreads) {

@@ -35,7 +35,7 @@ class rssm_workspace_layout(ctypes.Structure):
     _fields_ = [(n, ctypes.c_size_t) for n in (
         "error_off", "seq_pos_off", "ckpt_pos_off", "pending_off", "flush_count_off", "arrive_off",
         "A_off", "D_off", "ckpt_off", "ckpt_bytes", "rc_off", "rc_bytes", "rc_scale_off",
-        "rc_scale_bytes", "ring", "xbuf_off", "xbuf_bytes", "bbuf_off", "bbuf_bytes", "sbuf_off",
+        "rc_scale_bytes", "ring", "ring_stride", "xbuf_off", "xbuf_bytes", "bbuf_off", "bbuf_bytes", "sbuf_off",
         "sbuf_bytes", "tbuf_off", "tbuf_bytes", "snap_off", "snap_bytes", "total_bytes")]
 
 

@@ -102,7 +102,7 @@ typedef struct {
 /* Byte offsets (from the workspace base) and sizes of every workspace region;
  * a size of 0 means the region is absent in this configuration. */
 typedef struct {
-    size_t error_off;                    /* int32[8]: code, b, h, value, ...       */
+    size_t error_off;                    /* int32[8]: code, b, h, value; [4] is kernel-internal */
     size_t seq_pos_off, ckpt_pos_off;    /* int64[B] each                          */
     size_t pending_off, flush_count_off; /* int32[B] each                          */
     size_t arrive_off;                   /* int32[B] (kernel-internal, kept at 0)  */
@@ -113,10 +113,12 @@ typedef struct {
                                             the state (EAGER, BF16/FP8)            */
     size_t rc_scale_off, rc_scale_bytes; /* fp32[B][H][P] (FP8 only)               */
     size_t ring;                         /* R = window + max(max_draft, 1) slots   */
+    size_t ring_stride;                  /* R rounded up to a multiple of 4: row length of the
+                                            fp32 scalar rings below (16-byte rows) */
     size_t xbuf_off, xbuf_bytes;         /* Mamba-2 x[B][H][R][P]; GDN v[B][H][R][P] (input_dtype) */
     size_t bbuf_off, bbuf_bytes;         /* Mamba-2 B[B][G][R][N]; GDN k[B][H][R][N] (input_dtype) */
-    size_t sbuf_off, sbuf_bytes;         /* Mamba-2 dt[B][H][R]; GDN alpha[B][H][R] (fp32)         */
-    size_t tbuf_off, tbuf_bytes;         /* GDN beta[B][H][R] (fp32)                               */
+    size_t sbuf_off, sbuf_bytes;         /* Mamba-2 dt[B][H][ring_stride]; GDN alpha (fp32)        */
+    size_t tbuf_off, tbuf_bytes;         /* GDN beta[B][H][ring_stride] (fp32)                     */
     size_t snap_off, snap_bytes;         /* EAGER: max_draft snapshots of the state (+ scales)      */
     size_t total_bytes;
 } rssm_workspace_layout;

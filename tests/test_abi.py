@@ -64,7 +64,8 @@ def test_workspace_layout_nemotron_scale(lib):
     assert lay.ring == 17
     assert lay.xbuf_bytes == 256 * 128 * 17 * 64 * 2
     assert lay.bbuf_bytes == 256 * 8 * 17 * 128 * 2
-    assert lay.sbuf_bytes == 256 * 128 * 17 * 4
+    assert lay.ring_stride == 20
+    assert lay.sbuf_bytes == 256 * 128 * 20 * 4
     offs = sorted((getattr(lay, f), f) for f, _ in lay._fields_ if f.endswith("_off"))
     assert all(o % 256 == 0 for o, _ in offs)
     assert rssm.rssm_workspace_bytes(_cfg()) == lay.total_bytes
