@@ -141,8 +141,9 @@ def host_tokens(wl, n):
     return out
 
 
-def timed_loop(L, toks_dev, ys, K, W, sync):
-    """W warm-up then K timed decode steps; per-launch and whole-loop CUDA events."""
+def timed_loop(L, toks_dev, ys, K, W, sync, split=True):
+    """W warm-up then K timed decode steps.  CUDA events on the layer's stream
+    around every call, and (replay) between its prep/flush and replay-read kernels."""
     import torch
 
     from checkpoint_input_replay_rssm_b200 import rssm
@@ -150,26 +151,34 @@ def timed_loop(L, toks_dev, ys, K, W, sync):
     n = len(toks_dev)
     ins = [L._inputs(d) for d in toks_dev]
     yptr = [y.data_ptr() for y in ys]
+    stream = L.stream
     for i in range(W):
         rssm.rssm_decode(L.h, ins[i % n], yptr[i % len(ys)])
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    mk = lambda: torch.cuda.Event(enable_timing=True)
+    starts, mids, ends = [mk() for _ in range(K)], [mk() for _ in range(K)], [mk() for _ in range(K)]
+    for e in mids:  # materialise the CUDA events before handing them to the library
+        e.record(stream)
+    t0, t1 = mk(), mk()
     sync()
     l0 = L.launches()
-    stream = L.stream
     t0.record(stream)
     for i in range(K):
         j = (W + i) % n
+        if split:
+            rssm.rssm_set_split_event(L.h, mids[i].cuda_event)
         starts[i].record(stream)
         rssm.rssm_decode(L.h, ins[j], yptr[i % len(ys)])
         ends[i].record(stream)
     t1.record(stream)
     sync()
+    if split:
+        rssm.rssm_set_split_event(L.h, None)
     launches = L.launches() - l0
     total_ms = t0.elapsed_time(t1)
     per = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    return total_ms, float(np.mean(per)), launches, per
+    prep = [s.elapsed_time(m) for s, m in zip(starts, mids)] if split else None
+    read = [m.elapsed_time(e) for m, e in zip(mids, ends)] if split else None
+    return total_ms, per, prep, read, launches
 
 
 def e2e_loop(L, toks_host, K, W, sync):
@@ -322,15 +331,15 @@ def main():
     L = make_layer(wl, "replay", "bf16", consts, device)
     sampler = ClockSampler(local)
     with sampler:
-        total_ms, kern_ms, launches, per = timed_loop(L, toks_dev, ys, K, W, sync)
+        total_ms, per, prep_ms, read_ms, launches = timed_loop(L, toks_dev, ys, K, W, sync)
     fold = [(W + i) >= wl.window and (W + i) % wl.window == 0 for i in range(K)]
-    per_fold = [p for p, f in zip(per, fold) if f]
-    per_read = [p for p, f in zip(per, fold) if not f]
+    pick = lambda xs, want: [x for x, f in zip(xs, fold) if f == want]
     clocks = sampler.summary()
-    t = torch.tensor([total_ms, kern_ms], dtype=torch.float64, device=device)
+    t = torch.tensor([total_ms, float(np.mean(read_ms)), float(np.mean(prep_ms))], dtype=torch.float64,
+                     device=device)
     if dist is not None:
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms, kern_ms = float(t[0]), float(t[1])
+    total_ms, kern_ms, prep_avg = float(t[0]), float(t[1]), float(t[2])
     assert L.status()[0] == 0, "device error during the benchmark"
 
     # e2e through the public API with host buffers (fresh layer, same workload)
@@ -344,8 +353,10 @@ def main():
     shape = traffic.Shape("mamba2", wl.headdim, wl.dstate, wl.nheads // wl.ngroups, wl.window, "bf16",
                           wl.input_dtype)
     rep = traffic.replay_decode_per_token(shape)
+    win = traffic.replay_decode_window(shape)
     units = wl.batch * wl.nheads
-    bytes_per_launch = traffic.total(rep) * units
+    bytes_per_launch = traffic.total(win["read"]) * units       # replay-read kernel, mean per call
+    prep_bytes = traffic.total(win["prep"]) * units             # prep/flush kernel, mean per call
     achieved = bytes_per_launch / (kern_ms * 1e-3) / 1e9
     peak, peak_kind = measured_peak()
     tr = None
@@ -359,8 +370,8 @@ def main():
         del L
         torch.cuda.empty_cache()
         E = make_layer(wl, "eager", "f32", consts, device)
-        e_total, e_kern, _, _ = timed_loop(E, toks_dev, ys, K, W, sync)
-        t = torch.tensor([e_total, e_kern], dtype=torch.float64, device=device)
+        e_total, e_per, _, _, _ = timed_loop(E, toks_dev, ys, K, W, sync, split=False)
+        t = torch.tensor([e_total, float(np.mean(e_per))], dtype=torch.float64, device=device)
         if dist is not None:
             dist.all_reduce(t, op=dist.ReduceOp.MAX)
         e_total, e_kern = float(t[0]), float(t[1])
@@ -390,13 +401,19 @@ def main():
         "hbm_gbs": achieved,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": tr, "peak_source": peak_kind,
-                     "kernel": "m2_replay_kernel<128, bf16, 1>",
+                     "kernel": "replay_read_kernel<128, bf16, 1>",
                      "algorithmic_bytes_per_launch": bytes_per_launch,
                      "kernel_ms_per_launch": kern_ms,
-                     "kernel_ms_fold_step": float(np.mean(per_fold)) if per_fold else None,
-                     "kernel_ms_read_step": float(np.mean(per_read)) if per_read else None,
-                     "read_step_gbs": (traffic.total(traffic.replay_step(shape, wl.window // 2, False))
-                                       * units / (np.mean(per_read) * 1e-3) / 1e9) if per_read else None},
+                     "read_ms_nonfold_call": float(np.mean(pick(read_ms, False))),
+                     "read_gbs_nonfold_call": traffic.total(traffic.replay_step_split(shape, wl.window // 2, False)["read"])
+                                              * units / (np.mean(pick(read_ms, False)) * 1e-3) / 1e9},
+        "prep_kernel": {"kernel": "m2_prep_kernel<128, bf16, 1>", "ms_per_launch": prep_avg,
+                        "algorithmic_bytes_per_launch": prep_bytes,
+                        "gbs": prep_bytes / (prep_avg * 1e-3) / 1e9,
+                        "ms_nonfold_call": float(np.mean(pick(prep_ms, False))),
+                        "ms_fold_call": float(np.mean(pick(prep_ms, True))) if any(fold) else None},
+        "ms_per_call": {"nonfold": float(np.mean(pick(per, False))),
+                        "fold": float(np.mean(pick(per, True))) if any(fold) else None},
         "e2e": {"value": world * wl.batch * K / (e2e_ms * 1e-3), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches,

@@ -89,6 +89,19 @@ void layout(const rssm_config *c, rssm_workspace_layout *L) {
             L->tbuf_bytes = B * H * Rs * 4;
             L->tbuf_off = take(L->tbuf_bytes);
         }
+        // prep -> read hand-off, rewritten by every decode/verify
+        const size_t TQm = (size_t)(c->max_draft > 1 ? c->max_draft : 1);
+        L->tq_max = TQm;
+        L->seqinfo_bytes = B * 16;
+        L->seqinfo_off = take(L->seqinfo_bytes);
+        L->dec_bytes = B * H * TQm * 4;
+        L->dec_off = take(L->dec_bytes);
+        L->coef_bytes = B * H * TQm * ((size_t)c->window + TQm) * 4;
+        L->coef_off = take(L->coef_bytes);
+        if (c->kind == RSSM_GDN) {
+            L->query_bytes = B * H * TQm * N * 4;
+            L->query_off = take(L->query_bytes);
+        }
     } else if (c->max_draft > 0) {
         L->snap_bytes = (size_t)c->max_draft * (elems * sb + (fp8 ? B * H * P * 4 : 0));
         L->snap_off = take(L->snap_bytes);
@@ -118,7 +131,10 @@ bool inputs_ok(const Ctx *h, const rssm_inputs *in) {
 }
 
 cudaError_t launch_kind(Ctx *h, int op, int T, const rssm_inputs *in, float *y, float *out) {
-    h->launches += 1;
+    // replay decode/verify of Mamba-2 runs the prep/flush kernel and the replay-read kernel
+    const bool two = h->cfg.mode == RSSM_REPLAY && h->cfg.kind == RSSM_MAMBA2 &&
+                     (op == rssm::OP_DECODE || op == rssm::OP_VERIFY);
+    h->launches += two ? 2 : 1;
     if (h->cfg.kind == RSSM_MAMBA2) return rssm::mamba2_launch(*h, op, T, in, y, out, h->stream);
     return rssm::gdn_launch(*h, op, T, in, y, out, h->stream);
 }
@@ -309,6 +325,13 @@ rssm_status rssm_clear_status(rssm_handle hh) {
     if (!h) return RSSM_EINVAL;
     cudaError_t e = cudaMemsetAsync(h->at(h->lay.error_off), 0, 8 * sizeof(int32_t), h->stream);
     return e == cudaSuccess ? RSSM_OK : cuda_fail(h, e, "clear_status");
+}
+
+rssm_status rssm_set_split_event(rssm_handle hh, void *event) {
+    Ctx *h = (Ctx *)hh;
+    if (!h) return RSSM_EINVAL;
+    h->split_event = (cudaEvent_t)event;
+    return RSSM_OK;
 }
 
 int64_t rssm_launch_count(rssm_handle hh) {

@@ -19,7 +19,8 @@ struct Ctx {
     cudaStream_t stream = nullptr;
     int pending = 0;            // K of an uncommitted verify (host mirror), 0 if none
     int64_t launches = 0;       // kernels enqueued so far
-    int num_sms = 148;          // SMs of the handle's device (persistent grids)
+    int num_sms = 148;          // SMs of the handle's device
+    cudaEvent_t split_event = nullptr;  // recorded between prep and read kernels (measurement)
     std::string err;
 
     void *at(size_t off) const { return ws + off; }
@@ -43,6 +44,14 @@ size_t mamba2_smem_bytes(const rssm_config &cf, int T);
 cudaError_t gdn_launch(const Ctx &h, int op, int T, const rssm_inputs *in, float *y, float *out,
                        cudaStream_t st);
 size_t gdn_smem_bytes(const rssm_config &cf, int T);
+
+// The replay-read kernel (rssm_read.cu), shared by both kinds: queries Q[b][row][m][n]
+// at the given element strides, q_group heads per query row.
+cudaError_t launch_read(const Ctx &h, int T, const void *Q, int q_bf16, int q_group, int64_t q_stride_b,
+                        int64_t q_stride_row, int64_t q_stride_m, const void *xnew, const float *D,
+                        float *y, cudaStream_t st);
+int read_heads_per_cta(const rssm_config &cf);
+size_t read_smem_bytes(const rssm_config &cf, int T);
 
 // Kernels shared by both kinds (rssm_common.cu).
 cudaError_t launch_commit(const Ctx &h, const int32_t *accept, cudaStream_t st);

@@ -11,37 +11,22 @@ extern template cudaError_t m2_dispatch_n<128>(bool, int, int, const M2Args &, s
 
 static int tq_of(int T) { return T <= 1 ? 1 : (T <= 4 ? 4 : 8); }
 
-// Replay pipeline shape: heads per item HC (dividing the heads of a group),
-// stages NS and CTAs per SM.  Two CTAs per SM (two producers, sixteen consumer
-// warps) when two stages fit 110 KiB each; otherwise one CTA with up to 4 stages
-// in 200 KiB.  Items prefer 2 heads, then 1, then 4.
-struct M2Pipe { int HC, NS, per_sm; size_t smem; };
-static M2Pipe m2_pipe(const rssm_config &cf, int TQ) {
+// Heads per prep CTA: up to 8 heads of one group (the group's B . C is computed
+// once per CTA), within 160 KiB of shared memory.
+static int m2_prep_heads(const rssm_config &cf, int TQ) {
     const int hpg = cf.nheads / cf.ngroups, ib = cf.input_dtype == RSSM_BF16 ? 2 : 4;
-    const int rcb = cf.state_dtype == RSSM_F32 ? 4 : (cf.state_dtype == RSSM_BF16 ? 2 : 1);
-    auto total = [&](int hc, int ns) {
-        return m2_smem_total(ns, hc, cf.headdim, cf.dstate, cf.window, TQ, ib, rcb);
-    };
-    for (int hc : {4, 2, 1}) {
-        if (hpg % hc != 0) continue;
-        for (int ns = 3; ns >= 2; --ns)
-            if (total(hc, ns) <= 110 * 1024) return {hc, ns, 2, (size_t)total(hc, ns)};
-    }
-    for (int min_ns : {3, 1}) {
-        for (int hc : {2, 1, 4}) {
-            if (hpg % hc != 0) continue;
-            for (int ns = 4; ns >= min_ns; --ns)
-                if (total(hc, ns) <= 200 * 1024) return {hc, ns, 1, (size_t)total(hc, ns)};
-        }
-    }
-    return {1, 1, 1, (size_t)total(1, 1)};
+    for (int hc = 8; hc > 1; --hc)
+        if (hpg % hc == 0 && m2_prep_lay(hc, cf.headdim, cf.dstate, cf.window, TQ, ib).bytes <= 160 * 1024)
+            return hc;
+    return 1;
 }
 
 size_t mamba2_smem_bytes(const rssm_config &cf, int T) {
     const int TQ = tq_of(T), P = cf.headdim, N = cf.dstate;
     if (cf.mode == RSSM_EAGER)
         return sizeof(float) * ((size_t)2 * pad4(TQ * P) + 2 * pad4(TQ * N) + 2 * pad4(TQ));
-    return m2_pipe(cf, TQ).smem;
+    const int ib = cf.input_dtype == RSSM_BF16 ? 2 : 4;
+    return (size_t)m2_prep_lay(m2_prep_heads(cf, TQ), P, N, cf.window, TQ, ib).bytes;
 }
 
 cudaError_t mamba2_launch(const Ctx &h, int op, int T, const rssm_inputs *in, float *y, float *out,
@@ -51,13 +36,13 @@ cudaError_t mamba2_launch(const Ctx &h, int op, int T, const rssm_inputs *in, fl
     a.B = cf.batch; a.H = cf.nheads; a.P = cf.headdim; a.G = cf.ngroups; a.W = cf.window;
     a.R = (int)h.lay.ring; a.Rs = (int)h.lay.ring_stride; a.T = T; a.op = op; a.in_bf16 = cf.input_dtype == RSSM_BF16;
     a.dt_scales = cf.dt_scales_input;
-    const M2Pipe pp = m2_pipe(cf, tq_of(T));
-    a.HC = pp.HC;
-    a.NS = pp.NS;
-    {
-        const int items = cf.batch * (cf.nheads / pp.HC);
-        const int ctas = pp.per_sm * h.num_sms;
-        a.grid = items < ctas ? items : ctas;
+    a.HC = m2_prep_heads(cf, tq_of(T));
+    if (h.lay.seqinfo_bytes) {
+        a.seqinfo = (int4 *)h.at(h.lay.seqinfo_off);
+        a.dec = (float *)h.at(h.lay.dec_off);
+        a.coef = (float *)h.at(h.lay.coef_off);
+        a.TQmax = (int)h.lay.tq_max;
+        a.Emax = cf.window + a.TQmax;
     }
     a.c = h.counters();
     a.A = (const float *)h.at(h.lay.A_off); a.D = (const float *)h.at(h.lay.D_off);
@@ -77,12 +62,22 @@ cudaError_t mamba2_launch(const Ctx &h, int op, int T, const rssm_inputs *in, fl
     const bool eager = cf.mode == RSSM_EAGER;
     const int TQ = tq_of(T);
     const size_t smem = mamba2_smem_bytes(cf, T);
+    cudaError_t e;
     switch (cf.dstate) {
-        case 16: return m2_dispatch_n<16>(eager, cf.state_dtype, TQ, a, smem, st);
-        case 32: return m2_dispatch_n<32>(eager, cf.state_dtype, TQ, a, smem, st);
-        case 64: return m2_dispatch_n<64>(eager, cf.state_dtype, TQ, a, smem, st);
-        default: return m2_dispatch_n<128>(eager, cf.state_dtype, TQ, a, smem, st);
+        case 16: e = m2_dispatch_n<16>(eager, cf.state_dtype, TQ, a, smem, st); break;
+        case 32: e = m2_dispatch_n<32>(eager, cf.state_dtype, TQ, a, smem, st); break;
+        case 64: e = m2_dispatch_n<64>(eager, cf.state_dtype, TQ, a, smem, st); break;
+        default: e = m2_dispatch_n<128>(eager, cf.state_dtype, TQ, a, smem, st); break;
     }
+    if (e != cudaSuccess || eager || !(op == OP_DECODE || op == OP_VERIFY)) return e;
+    if (h.split_event) {
+        e = cudaEventRecord(h.split_event, st);
+        if (e != cudaSuccess) return e;
+    }
+    // replay read: C of the group ([B][T][G][N]) is the query, x the buffered entries
+    const int G = cf.ngroups;
+    return launch_read(h, T, in->Cm, cf.input_dtype == RSSM_BF16, cf.nheads / G, (int64_t)T * G * cf.dstate,
+                       cf.dstate, (int64_t)G * cf.dstate, in->x, (const float *)h.at(h.lay.D_off), y, st);
 }
 
 }  // namespace rssm

@@ -24,15 +24,17 @@
 #pragma once
 #include "rssm_device.cuh"
 #include "rssm_internal.h"
-#include "rssm_pipe.cuh"
+#include "rssm_read.cuh"
 
 namespace rssm {
 
 struct M2Args {
     int B, H, P, G, W, R, Rs, T, op, in_bf16, dt_scales;  // Rs: dt ring row length
-    int HC;             // heads per replay item (divides H / G)
-    int NS;             // pipeline stages of the replay kernel
-    int grid;           // persistent CTAs of the replay kernel
+    int HC;             // heads per prep CTA (divides H / G)
+    int4 *seqinfo;      // per sequence, for the read kernel: {L0, ring slot of entry 0, folded, 0}
+    float *dec;         // [B][H][TQmax] decay of S^ C
+    float *coef;        // [B][H][TQmax][Emax] replay coefficients
+    int TQmax, Emax;
     Counters c;
     const float *A, *D;
     float *ckpt;        // fp32 [B][H][P][N]
@@ -55,514 +57,302 @@ struct M2Args {
 __host__ __device__ constexpr int a16(int v) { return (v + 15) & ~15; }
 __host__ __device__ constexpr int pad4(int n) { return (n + 3) & ~3; }
 
-// One pipeline stage of the persistent replay kernel (bytes, 16-byte aligned
-// regions).  A stage carries one unit of work: the state tile of an item (the
-// read copy of HC heads, or one part of their fp32 checkpoint when the item
-// folds) plus everything the item needs from the ring and from this call's
-// tokens.  Entry slots: E = W + TQ; committed entries sit right-aligned before
-// slot W and this call's tokens at W..W+T-1.
-struct M2Stage {
-    int tile, scale, x, B, C, dt, dtn, info, bytes;
-};
 // Upper bound of a dt ring row in bytes: the ring has R = W + max(max_draft, 1) <= W + 8
 // slots, rows padded to 4 floats.
 __host__ __device__ constexpr int dt_row_max_bytes(int W) { return ((W + 8 + 3) & ~3) * 4; }
-constexpr int kTileCap = 32 * 1024;  // bytes of state rows per pipeline unit
 
-__host__ __device__ inline M2Stage m2_stage(int HC, int P, int N, int W, int TQ, int ib, int rcb) {
-    const int E = W + TQ;
-    M2Stage S{};
-    int o = 0;
-    S.tile = o;  o += kTileCap;                                  // state rows of the unit
-    S.scale = o; o += (rcb == 1) ? a16(kTileCap / N * 4) : 0;    // fp8 row scales
-    S.x = o;     o += a16(HC * E * P * ib);            // x of entries   [HC][E][P]
-    S.B = o;     o += a16(E * N * ib);                 // B of entries   [E][N]
-    S.C = o;     o += a16(TQ * N * ib);                // C of queries   [TQ][N]
-    S.dt = o;    o += a16(HC * dt_row_max_bytes(W));   // dt ring rows   [HC][Rs]
-    S.dtn = o;   o += a16(TQ * HC * 4);                // dt of this call's tokens [TQ][HC]
-    S.info = o;  o += 64;                              // unit descriptor
-    S.bytes = o;
-    return S;
-}
-
-// Consumer-side scratch, shared by all units (bytes).
-struct M2Scratch {
-    int sd, slam, scoef, sdec, su, sfdec, sdot, sCf, pdt, bytes;
+// Shared memory of the prep kernel (bytes, 16-byte aligned regions).  Entry
+// slots: E = W + TQ; committed entries sit right-aligned before slot W, the
+// call's own tokens at W..W+T-1, so logical entry e is slot (W - L0) + e.
+struct M2PrepLay {
+    int sC, sB, sx, dring, dtn, sd, slam, scoef, sdec, su, sfdec, sCf, sdot, si, bytes;
 };
-__host__ __device__ inline M2Scratch m2_scratch(int HC, int P, int N, int W, int TQ) {
+__host__ __device__ inline M2PrepLay m2_prep_lay(int HC, int P, int N, int W, int TQ, int ib) {
     const int E = W + TQ;
-    M2Scratch S{};
+    M2PrepLay L{};
     int o = 0;
-    S.sd = o;    o += a16(TQ * E * 4);       // B_e . C_m             [TQ][E]
-    S.slam = o;  o += a16(HC * E * 4);       // prefix sums of dt*A   [HC][E]
-    S.scoef = o; o += a16(HC * TQ * E * 4);  // replay coefficients   [HC][TQ][E]
-    S.sdec = o;  o += a16(HC * TQ * 4);      // decay of S^ C         [HC][TQ]
-    S.su = o;    o += a16(HC * E * 4);       // fold weights          [HC][E]
-    S.sfdec = o; o += a16(HC * 4);           // decay of the folded checkpoint [HC]
-    S.sdot = o;  o += a16(HC * P * TQ * 4);  // S^ C per state row    [HC*P][TQ]
-    S.sCf = o;   o += a16(TQ * N * 4);       // C as fp32             [TQ][N]
-    S.pdt = o;   o += a16(32 * HC * TQ * 4); // producer: dt of its 32 prefetched items
-    S.bytes = o;
-    return S;
+    L.sC = o;    o += a16(TQ * N * ib);          // raw C of the queries   [TQ][N]
+    L.sB = o;    o += a16(E * N * ib);           // raw B of the entries   [E][N]
+    L.sx = o;    o += a16(HC * E * P * ib);      // raw x of the entries   [HC][E][P]
+    L.dring = o; o += a16(HC * dt_row_max_bytes(W));  // dt ring rows      [HC][Rs]
+    L.dtn = o;   o += a16(TQ * HC * 4);          // dt of the call's tokens [TQ][HC]
+    L.sd = o;    o += a16(TQ * E * 4);           // B_e . C_m              [TQ][E]
+    L.slam = o;  o += a16(HC * E * 4);           // prefix sums of dt*A    [HC][E]
+    L.scoef = o; o += a16(HC * TQ * E * 4);      // replay coefficients    [HC][TQ][E]
+    L.sdec = o;  o += a16(HC * TQ * 4);          // decay of S^ C          [HC][TQ]
+    L.su = o;    o += a16(HC * E * 4);           // fold weights           [HC][E]
+    L.sfdec = o; o += a16(HC * 4);               // decay of the folded checkpoint [HC]
+    L.sCf = o;   o += a16(TQ * N * 4);           // C as fp32              [TQ][N]
+    L.sdot = o;  o += a16(HC * P * TQ * 4);      // fresh copy . C per row [HC*P][TQ]
+    L.si = o;    o += 32;
+    L.bytes = o;
+    return L;
 }
-
-__host__ __device__ inline int m2_smem_total(int NS, int HC, int P, int N, int W, int TQ, int ib, int rcb) {
-    return 16 * NS + NS * m2_stage(HC, P, N, W, TQ, ib, rcb).bytes + m2_scratch(HC, P, N, W, TQ).bytes;
-}
-
-enum { INFO_ITEM = 0, INFO_PART, INFO_NPARTS, INFO_L0, INFO_FLUSH, INFO_CKMOD, INFO_SPMOD };
 
 // ---------------------------------------------------------------------------
-// Replay kernel: decode (T = 1), verify (T = K), flush (T = 0), export (T = 0).
+// Prep / flush kernel: decode (T = 1), verify (T = K), flush and export (T = 0).
 //
-// Persistent: one CTA per SM walks the items (sequence b, group g, chunk of HC
-// heads of the group; the HC state tiles are contiguous) with stride gridDim.
-// Warp 8 is the producer: for each item it reads the sequence counters, decides
-// whether the item folds, and fills the next free stage of an NS-deep ring in
-// shared memory with bulk copies (the read-copy tile, or the fp32 checkpoint in
-// parts when folding, plus the buffered entries and this call's tokens), so up
-// to NS tiles are in flight while the eight consumer warps work.  Consumers,
-// per unit: B_e . C_m and per-head prefix sums of the log decays (first part of
-// an item), then either the read-copy rows dotted with C or the fold of the
-// checkpoint rows (stored with the requantised copy), then outputs and ring
-// appends (last part), and release the stage.  Every barrier wait is bounded.
+// One CTA per (sequence b, group g, chunk of HC heads of the group).  It reads
+// the sequence's counters, stages the group's buffered B, the heads' dt ring
+// rows and the call's tokens, and computes once per group B_e . C_m and per head
+// the prefix sums Lam of dt*A.  Then either
+//   * (no fold) it writes the replay coefficients
+//       coef[e] = e^{Lam_{L0+m} - Lam_e} (B_e . C_m) s_e,   dec = e^{Lam_{L0+m}}
+//     for the read kernel, or
+//   * (fold: len + T > W, or flush/export) it folds the committed entries into
+//     the fp32 checkpoint, S_c <- e^{Lam_L} S_c + sum_e e^{Lam_L - Lam_e} s_e x_e B_e^T,
+//     stores it with the requantised read copy (or writes it out, for export),
+//     and, for decode/verify, computes the outputs from the fresh copy itself.
+// Last it appends the call's tokens to the ring; the last CTA of the sequence
+// publishes the counters.
 // ---------------------------------------------------------------------------
 template <int N, int RK, int TQ>
-__global__ void __maxnreg__(112) m2_replay_kernel(const M2Args a) {
-    constexpr int EPC = Chunk<RK>::EPC;    // stored elements per 16-byte chunk
-    constexpr int TPR = N / EPC;           // lanes per state row, read mapping
-    constexpr int RCB = Chunk<RK>::BYTES;  // bytes per stored element
-    constexpr int TPR4 = N / 4;            // lanes per row, fp32 quad mapping (fold)
+__global__ void __launch_bounds__(kThreads) m2_prep_kernel(const M2Args a) {
+    constexpr int TPR4 = N / 4;  // lanes per row, fp32 quad mapping
     constexpr int RPP4 = kThreads / TPR4;
-    static_assert(TPR >= 1 && TPR <= 32 && (32 % TPR) == 0, "row must fit a warp");
-
-    extern __shared__ __align__(128) uint8_t smraw[];
+    constexpr int FH = 4;        // fold rows held in registers per thread
+    extern __shared__ __align__(16) uint8_t smraw[];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int H = a.H, P = a.P, W = a.W, R = a.R, T = a.T, G = a.G, HC = a.HC, NS = a.NS;
+    const int H = a.H, P = a.P, W = a.W, R = a.R, T = a.T, G = a.G, HC = a.HC;
     const int hpg = H / G, cpg = hpg / HC;
+    const int b = blockIdx.x / (G * cpg);
+    const int rem = blockIdx.x - b * G * cpg;
+    const int g = rem / cpg, hc = rem - g * cpg;
+    const int h0 = g * hpg + hc * HC;
     const int E = W + TQ;
     const int bf = a.in_bf16, ib = bf ? 2 : 4;
+    const M2PrepLay Ly = m2_prep_lay(HC, P, N, W, TQ, ib);
+    uint8_t *sC = smraw + Ly.sC, *sB = smraw + Ly.sB, *sx = smraw + Ly.sx;
+    float *dring = reinterpret_cast<float *>(smraw + Ly.dring);
+    float *dtn = reinterpret_cast<float *>(smraw + Ly.dtn);
+    float *sd = reinterpret_cast<float *>(smraw + Ly.sd);
+    float *slam = reinterpret_cast<float *>(smraw + Ly.slam);
+    float *scoef = reinterpret_cast<float *>(smraw + Ly.scoef);
+    float *sdec = reinterpret_cast<float *>(smraw + Ly.sdec);
+    float *su = reinterpret_cast<float *>(smraw + Ly.su);
+    float *sfdec = reinterpret_cast<float *>(smraw + Ly.sfdec);
+    float *sCf = reinterpret_cast<float *>(smraw + Ly.sCf);
+    float *sdot = reinterpret_cast<float *>(smraw + Ly.sdot);
+    int *si = reinterpret_cast<int *>(smraw + Ly.si);
+    const int64_t row0 = (int64_t)b * H + h0;
+    const int64_t tile0 = row0 * P * N;
     const int nrows = HC * P;
     const bool reads = (a.op == OP_DECODE || a.op == OP_VERIFY);
-    const int rpp_read = kTileCap / (N * RCB);  // read-copy rows per unit
-    const int rpp_fold = kTileCap / (N * 4);    // fp32 checkpoint rows per unit
-    const int read_parts = (nrows + rpp_read - 1) / rpp_read;
-    const int fold_parts = (nrows + rpp_fold - 1) / rpp_fold;
-    const int xrow = P * ib, brow = N * ib;
-    const M2Stage SG = m2_stage(HC, P, N, W, TQ, ib, RCB);
-    const M2Scratch SC = m2_scratch(HC, P, N, W, TQ);
-    uint64_t *full = reinterpret_cast<uint64_t *>(smraw);
-    uint64_t *empty = full + NS;
-    uint8_t *stages = smraw + 16 * NS;
-    uint8_t *scr = stages + NS * SG.bytes;
-    const int nitems = a.B * (H / HC);
+    const int xrow = P * ib, brow = N * ib, xch = xrow / 16, bch = brow / 16;
+    const int Rs = a.Rs;
 
+    // 1. Counters (thread 0) and the call's tokens.
     if (tid == 0) {
-        for (int i = 0; i < NS; ++i) {
-            mbar_init(&full[i], 32);       // the producer warp's lanes (+ bulk-copy bytes)
-            mbar_init(&empty[i], kWarps);  // one arrival per consumer warp
+        SeqState ss = read_counters(a.c, b, W);
+        const int L0 = (int)(ss.seq - ss.ckpt);
+        int flush = 0;
+        if (ss.ok) flush = (a.op == OP_FLUSH || a.op == OP_EXPORT) ? (L0 > 0) : (L0 + T > W);
+        si[0] = ss.ok;
+        si[1] = ss.ok ? L0 : 0;
+        si[2] = flush;
+        si[3] = (int)(ss.ckpt % R);
+        si[4] = (int)(ss.seq % R);
+        if (!ss.ok) {
+            if (g == 0 && hc == 0) report(a.c.err, DEV_BAD_COUNTERS, b, h0, L0);
+            if (reads && g == 0 && hc == 0) a.seqinfo[b] = make_int4(0, 0, 1, 0);  // nothing to read
+        } else {
+            if (reads && g == 0 && hc == 0) a.seqinfo[b] = make_int4(flush ? 0 : L0, (int)(ss.ckpt % R), flush, 0);
+            if (a.op != OP_EXPORT)
+                arrive_and_publish(a.c, b, G * cpg, (a.op == OP_DECODE) ? ss.seq + 1 : -1,
+                                   flush ? ss.seq : -1, (a.op == OP_VERIFY) ? T : -1, flush);
         }
-        mbar_init_fence();
+    }
+    for (int i = tid; i < T * bch; i += kThreads) {
+        const int m = i / bch, k = i - m * bch;
+        const int64_t src = (((int64_t)(b * T + m) * G + g) * N) * ib + k * 16;
+        cp_async16(sC + m * brow + k * 16, reinterpret_cast<const uint8_t *>(a.Cm) + src);
+        cp_async16(sB + (W + m) * brow + k * 16, reinterpret_cast<const uint8_t *>(a.Bm) + src);
+    }
+    for (int i = tid; i < T * HC * xch; i += kThreads) {
+        const int m = i / (HC * xch), r2 = i - m * HC * xch;
+        const int hh = r2 / xch, k = r2 - hh * xch;
+        cp_async16(sx + (hh * E + W + m) * xrow + k * 16,
+                   reinterpret_cast<const uint8_t *>(a.x) + (((int64_t)(b * T + m) * H + h0 + hh) * P) * ib + k * 16);
+    }
+    for (int i = tid; i < T * HC; i += kThreads) {
+        const int m = i / HC, hh = i - m * HC;
+        dtn[m * HC + hh] = a.dt[(int64_t)(b * T + m) * H + h0 + hh];
+    }
+    for (int i = tid; i < HC * Rs / 4; i += kThreads) cp_async16(dring + 4 * i, a.dtbuf + row0 * Rs + 4 * i);
+    __syncthreads();
+    if (!si[0]) {
+        cp_async_wait_all();
+        return;
+    }
+    const int L0 = si[1], flush = si[2], ckmod = si[3], spmod = si[4];
+    const int base = W - L0, nE = L0 + T;
+    const int e0 = flush ? L0 : 0;  // first entry the outputs replay
+
+    // 2. Buffered entries: the group's B (always), the heads' x (only to fold).
+    for (int i = tid; i < L0 * bch; i += kThreads) {
+        const int e = i / bch, k = i - e * bch;
+        const int slot = (ckmod + e) % R;
+        cp_async16(sB + (base + e) * brow + k * 16,
+                   reinterpret_cast<const uint8_t *>(a.Bbuf) + (((int64_t)(b * G + g) * R + slot) * N) * ib + k * 16);
+    }
+    if (flush) {
+        for (int i = tid; i < HC * L0 * xch; i += kThreads) {
+            const int hh = i / (L0 * xch), r2 = i - hh * L0 * xch;
+            const int e = r2 / xch, k = r2 - e * xch;
+            const int slot = (ckmod + e) % R;
+            cp_async16(sx + (hh * E + base + e) * xrow + k * 16,
+                       reinterpret_cast<const uint8_t *>(a.xbuf) + (((row0 + hh) * R + slot) * P) * ib + k * 16);
+        }
+    }
+    cp_async_wait_all();
+    __syncthreads();
+    auto dt_of = [&](int hh, int e) -> float {
+        return e < L0 ? dring[hh * Rs + (ckmod + e) % R] : dtn[(e - L0) * HC + hh];
+    };
+
+    // 3. B_e . C_m once for the group, C as fp32, prefix sums of dt*A per head.
+    if (reads) {
+        for (int pr = warp; pr < T * nE; pr += kWarps) {
+            const int m = pr / nE, e = pr - m * nE;
+            if (e > L0 + m) continue;  // warp-uniform
+            float d = 0.f;
+            for (int n = lane; n < N; n += 32)
+                d = fmaf(raw_f(sB + (base + e) * brow, n, bf), raw_f(sC + m * brow, n, bf), d);
+            d = group_sum<32>(d);
+            if (lane == 0) sd[m * E + e] = d;
+        }
+        for (int i = tid; i < T * N; i += kThreads) sCf[i] = raw_f(sC, i, bf);
+    }
+    for (int hh = warp; hh < HC; hh += kWarps) {
+        const float Ah = a.A[h0 + hh];
+        float carry = 0.f;
+        for (int k0 = 0; k0 < nE; k0 += 32) {
+            const int e = k0 + lane;
+            float v = (e < nE) ? dt_of(hh, e) * Ah : 0.f;
+            v = warp_incl_scan(v) + carry;
+            if (e < nE) slam[hh * E + base + e] = v;
+            carry = __shfl_sync(0xffffffffu, v, 31);
+        }
     }
     __syncthreads();
 
-    if (warp == kWarps) {
-        // ================================ producer ================================
-        // Items are taken 32 at a time: lane j loads the counters and the token dt's
-        // of the j-th item of the batch (one memory round trip per 32 items); then
-        // the items' units are queued in order.
-        float *pdt = reinterpret_cast<float *>(scr + SC.pdt);
-        const int HT = HC * T;
-        const int nper = H / HC;  // items per sequence
-        int s = 0;
-        uint32_t used = 0, ephase = 0;
-        bool dead = false;
-        auto acquire = [&](int st) -> bool {  // warp-uniform
-            if (used & (1u << st)) {
-                int got = 0;
-                if (lane == 0) got = mbar_wait(&empty[st], (ephase >> st) & 1u) ? 1 : 0;
-                got = __shfl_sync(0xffffffffu, got, 0);
-                __syncwarp();
-                if (!got) return false;
-                ephase ^= 1u << st;
-            }
-            used |= 1u << st;
-            return true;
-        };
-        for (int bstart = blockIdx.x; bstart < nitems && !dead; bstart += 32 * gridDim.x) {
-            const int mine = bstart + lane * gridDim.x;
-            int ok = 0, L0 = 0, flush = 0, ckmod = 0, spmod = 0;
-            if (mine < nitems) {
-                const int b = mine / nper, rem = mine - b * nper;
-                const int g = rem / cpg, hc = rem - g * cpg, h0 = g * hpg + hc * HC;
-                for (int i = 0; i < HT; ++i) {
-                    const int m = i / HC, hh = i - m * HC;
-                    pdt[lane * HT + i] = a.dt[(int64_t)(b * T + m) * H + h0 + hh];
-                }
-                SeqState ss = read_counters(a.c, b, W);
-                ok = ss.ok;
-                L0 = (int)(ss.seq - ss.ckpt);
-                if (ok) flush = (a.op == OP_FLUSH || a.op == OP_EXPORT) ? (L0 > 0) : (L0 + T > W);
-                ckmod = (int)(ss.ckpt % R);
-                spmod = (int)(ss.seq % R);
-                if (!ok && g == 0 && hc == 0) report(a.c.err, DEV_BAD_COUNTERS, b, h0, L0);
-            }
-            __syncwarp();
-            for (int j = 0; j < 32 && !dead; ++j) {
-                const int item = bstart + j * gridDim.x;
-                if (item >= nitems) break;
-                const int iok = __shfl_sync(0xffffffffu, ok, j);
-                const int iL0 = __shfl_sync(0xffffffffu, L0, j);
-                const int ifl = __shfl_sync(0xffffffffu, flush, j);
-                const int ick = __shfl_sync(0xffffffffu, ckmod, j);
-                const int isp = __shfl_sync(0xffffffffu, spmod, j);
-                const int b = item / nper, rem = item - b * nper;
-                const int g = rem / cpg, hc = rem - g * cpg, h0 = g * hpg + hc * HC;
-                const int64_t row0 = (int64_t)b * H + h0;
-                const int64_t tile0 = row0 * P * N;
-                const int nparts = !iok ? 0 : (ifl ? fold_parts : (reads ? read_parts : 0));
-                const int base = W - iL0;
-                const int n1 = min(iL0, R - ick);  // entries before the ring wraps
-                for (int part = 0; part < nparts; ++part) {
-                    if (!acquire(s)) {
-                        if (lane == 0) report(a.c.err, DEV_PIPE_TIMEOUT, b, h0, 1);
-                        dead = true;
-                        break;
-                    }
-                    uint8_t *st = stages + s * SG.bytes;
-                    int *info = reinterpret_cast<int *>(st + SG.info);
-                    float *dtn = reinterpret_cast<float *>(st + SG.dtn);
-                    if (lane == 0) {
-                        info[INFO_ITEM] = item; info[INFO_PART] = part; info[INFO_NPARTS] = nparts;
-                        info[INFO_L0] = iL0; info[INFO_FLUSH] = ifl; info[INFO_CKMOD] = ick;
-                        info[INFO_SPMOD] = isp;
-                    }
-                    for (int i = lane; i < HT; i += 32) dtn[i] = pdt[j * HT + i];
-                    // The unit's bulk copies: the same list is walked twice, once to
-                    // total the bytes, once to issue (copy k by lane k mod 32).
-                    uint32_t tx = 0;
-                    int ci = 0;
-                    auto copy = [&](bool issue, void *dst, const void *src, uint32_t bytes) {
-                        if (bytes == 0) return;
-                        if (!issue) tx += bytes;
-                        else if ((ci & 31) == lane) bulk_g2s(dst, src, bytes, &full[s]);
-                        ++ci;
-                    };
-                    auto walk = [&](bool issue) {
-                        ci = 0;
-                        if (ifl) {
-                            const int r0 = part * rpp_fold, r1 = min(nrows, r0 + rpp_fold);
-                            copy(issue, st + SG.tile, a.ckpt + tile0 + (int64_t)r0 * N, (uint32_t)((r1 - r0) * N * 4));
-                        } else {
-                            const int r0 = part * rpp_read, r1 = min(nrows, r0 + rpp_read);
-                            const uint8_t *rc = (RK == SK_F32) ? reinterpret_cast<const uint8_t *>(a.ckpt + tile0)
-                                                               : reinterpret_cast<const uint8_t *>(a.rc) + tile0 * RCB;
-                            copy(issue, st + SG.tile, rc + (int64_t)r0 * N * RCB, (uint32_t)((r1 - r0) * N * RCB));
-                            if (RK == SK_FP8)
-                                copy(issue, st + SG.scale, a.rc_scale + row0 * P + r0, (uint32_t)((r1 - r0) * 4));
-                        }
-                        copy(issue, st + SG.dt, a.dtbuf + row0 * a.Rs, (uint32_t)(HC * a.Rs * 4));
-                        const uint8_t *Bb = reinterpret_cast<const uint8_t *>(a.Bbuf) + ((int64_t)(b * G + g) * R) * brow;
-                        copy(issue, st + SG.B + base * brow, Bb + (int64_t)ick * brow, (uint32_t)(n1 * brow));
-                        copy(issue, st + SG.B + (base + n1) * brow, Bb, (uint32_t)((iL0 - n1) * brow));
-                        for (int hh = 0; hh < HC; ++hh) {
-                            const uint8_t *xb = reinterpret_cast<const uint8_t *>(a.xbuf) + ((row0 + hh) * R) * xrow;
-                            uint8_t *xd = st + SG.x + (hh * E + base) * xrow;
-                            copy(issue, xd, xb + (int64_t)ick * xrow, (uint32_t)(n1 * xrow));
-                            copy(issue, xd + n1 * xrow, xb, (uint32_t)((iL0 - n1) * xrow));
-                        }
-                        for (int m = 0; m < T; ++m) {
-                            const int64_t gsrc = (((int64_t)(b * T + m) * G + g) * N) * ib;
-                            copy(issue, st + SG.C + m * brow, reinterpret_cast<const uint8_t *>(a.Cm) + gsrc, (uint32_t)brow);
-                            copy(issue, st + SG.B + (W + m) * brow, reinterpret_cast<const uint8_t *>(a.Bm) + gsrc, (uint32_t)brow);
-                            const uint8_t *xs = reinterpret_cast<const uint8_t *>(a.x) + (((int64_t)(b * T + m) * H + h0) * P) * ib;
-                            for (int hh = 0; hh < HC; ++hh)
-                                copy(issue, st + SG.x + (hh * E + W + m) * xrow, xs + hh * xrow, (uint32_t)xrow);
-                        }
-                    };
-                    walk(false);
-                    if (lane == 0) mbar_arrive_expect_tx(&full[s], tx);
-                    else mbar_arrive(&full[s]);
-                    __syncwarp();
-                    walk(true);
-                    s = (s + 1 == NS) ? 0 : s + 1;
+    // 4. Replay coefficients and decays (to the read kernel, or kept here to fold).
+    for (int i = tid; i < HC * nE; i += kThreads) {
+        const int hh = i / nE, e = i - hh * nE;
+        const float *lam = slam + hh * E + base;
+        const float se = a.dt_scales ? dt_of(hh, e) : 1.f;
+        if (reads) {
+#pragma unroll
+            for (int m = 0; m < TQ; ++m) {
+                if (m >= T || e > L0 + m) continue;
+                const float cf = expf(lam[L0 + m] - lam[e]) * sd[m * E + e] * se;
+                if (flush) {
+                    if (e >= e0) scoef[(hh * TQ + m) * E + e] = cf;
+                } else {
+                    a.coef[((row0 + hh) * a.TQmax + m) * a.Emax + e] = cf;
                 }
             }
         }
-        if (!dead && acquire(s)) {  // end-of-work unit
-            if (lane == 0) reinterpret_cast<int *>(stages + s * SG.bytes + SG.info)[INFO_ITEM] = -1;
-            mbar_arrive(&full[s]);
-        } else if (lane == 0 && !dead) {
-            report(a.c.err, DEV_PIPE_TIMEOUT, -1, -1, 2);
-        }
-        // Counters: every CTA has read all of its items' counters by now; the last
-        // CTA to get here publishes the new counters of every sequence.
-        if (a.op != OP_EXPORT) {
-            int last = 0;
-            if (lane == 0) {
-                __threadfence();
-                last = (atomicAdd(&a.c.err[4], 1) == (int)gridDim.x - 1) ? 1 : 0;
-            }
-            last = __shfl_sync(0xffffffffu, last, 0);
-            if (last) {
-                __threadfence();
-                for (int b = lane; b < a.B; b += 32) {
-                    SeqState ss = read_counters(a.c, b, W);
-                    if (!ss.ok) continue;
-                    const int L0 = (int)(ss.seq - ss.ckpt);
-                    const int flush = (a.op == OP_FLUSH) ? (L0 > 0) : (L0 + T > W);
-                    if (flush) {
-                        a.c.ckpt_pos[b] = ss.seq;
-                        a.c.flush_count[b] += 1;
-                    }
-                    if (a.op == OP_DECODE) a.c.seq_pos[b] = ss.seq + 1;
-                    if (a.op == OP_VERIFY) a.c.pending[b] = T;
-                }
-                __syncwarp();
-                if (lane == 0) a.c.err[4] = 0;
-                __threadfence();
-            }
-        }
-        return;
+        if (flush && e < L0) su[hh * E + e] = expf(lam[L0 - 1] - lam[e]) * se;
     }
-
-    // ================================ consumers ================================
-    float *sd = reinterpret_cast<float *>(scr + SC.sd);
-    float *slam = reinterpret_cast<float *>(scr + SC.slam);
-    float *scoef = reinterpret_cast<float *>(scr + SC.scoef);
-    float *sdec = reinterpret_cast<float *>(scr + SC.sdec);
-    float *su = reinterpret_cast<float *>(scr + SC.su);
-    float *sfdec = reinterpret_cast<float *>(scr + SC.sfdec);
-    float *sdot = reinterpret_cast<float *>(scr + SC.sdot);
-    float *sCf = reinterpret_cast<float *>(scr + SC.sCf);
-    // read mapping: LPR lanes per state row, CPL chunks per lane, rotated so the
-    // rows of a warp spread over all shared-memory banks
-    constexpr int LPR = TPR < 4 ? TPR : 4;
-    constexpr int CPL = TPR / LPR;
-    constexpr int RPPR = kThreads / LPR;
-    constexpr bool kCregs = TQ * CPL * EPC <= 32;
-    const int q = tid % LPR, rrow = tid / LPR, rot = rrow % CPL;
-    // fold mapping: TPR4 lanes per row (quads), FR rows per thread per unit
-    constexpr int FR = 8;  // = (kTileCap / (N * 4)) / RPP4 for every N
-    static_assert(FR * RPP4 * N * 4 == kTileCap, "fold unit is FR rows per thread");
-    const int c4 = tid % TPR4, q0 = tid / TPR4;
-    int s = 0;
-    uint32_t fphase = 0;
-    for (;;) {
-        const bool got = mbar_wait(&full[s], (fphase >> s) & 1u);
-        if (consumer_sync_any(!got)) {
-            if (tid == 0) report(a.c.err, DEV_PIPE_TIMEOUT, -1, -1, 3);
-            break;
+    for (int i = tid; i < HC; i += kThreads) {
+        const float *lam = slam + i * E + base;
+        sfdec[i] = flush ? expf(lam[L0 - 1]) : 1.f;
+        if (reads) {
+#pragma unroll
+            for (int m = 0; m < TQ; ++m) {
+                if (m >= T) continue;
+                const float dcy = expf(lam[L0 + m] - (flush ? lam[L0 - 1] : 0.f));
+                if (flush) sdec[i * TQ + m] = dcy;
+                else a.dec[(row0 + i) * a.TQmax + m] = dcy;
+            }
         }
-        fphase ^= 1u << s;
-        const uint8_t *st = stages + s * SG.bytes;
-        const int *info = reinterpret_cast<const int *>(st + SG.info);
-        const int item = info[INFO_ITEM];
-        if (item < 0) break;
-        const int part = info[INFO_PART], nparts = info[INFO_NPARTS];
-        const int L0 = info[INFO_L0], flush = info[INFO_FLUSH], spmod = info[INFO_SPMOD];
-        const int ckmod = info[INFO_CKMOD];
-        const int b = item / (H / HC);
-        const int rem = item - b * (H / HC);
-        const int g = rem / cpg, hc = rem - g * cpg;
-        const int h0 = g * hpg + hc * HC;
-        const int64_t row0 = (int64_t)b * H + h0;
-        const int64_t tile0 = row0 * P * N;
-        const int base = W - L0, nE = L0 + T;
-        const int e0 = flush ? L0 : 0;  // first entry the outputs replay
-        const uint8_t *sx = st + SG.x;
-        const uint8_t *sB = st + SG.B;
-        const uint8_t *sC = st + SG.C;
-        const float *dring = reinterpret_cast<const float *>(st + SG.dt);
-        const float *dtn = reinterpret_cast<const float *>(st + SG.dtn);
-        // dt of logical entry e (committed entries from the ring, then this call's tokens)
-        auto dt_of = [&](int hh, int e) -> float {
-            return e < L0 ? dring[hh * a.Rs + (ckmod + e) % R] : dtn[(e - L0) * HC + hh];
-        };
-
-        if (part == 0) {
-            // B_e . C_m once per item; C to fp32; prefix sums of dt*A per head.
-            if (reads) {
-                for (int pr = warp; pr < T * nE; pr += kWarps) {
-                    const int m = pr / nE, e = pr - m * nE;
-                    if (e < e0 || e > L0 + m) continue;  // warp-uniform
-                    float d = 0.f;
-                    for (int n = lane; n < N; n += 32)
-                        d = fmaf(raw_f(sB + (base + e) * brow, n, bf), raw_f(sC + m * brow, n, bf), d);
-                    d = group_sum<32>(d);
-                    if (lane == 0) sd[m * E + e] = d;
-                }
-                for (int i = tid; i < T * N; i += kThreads) sCf[i] = raw_f(sC, i, bf);
-            }
-            for (int hh = warp; hh < HC; hh += kWarps) {
-                const float Ah = a.A[h0 + hh];
-                float carry = 0.f;
-                for (int k0 = 0; k0 < nE; k0 += 32) {
-                    const int e = k0 + lane;
-                    float v = (e < nE) ? dt_of(hh, e) * Ah : 0.f;
-                    v = warp_incl_scan(v) + carry;
-                    if (e < nE) slam[hh * E + base + e] = v;
-                    carry = __shfl_sync(0xffffffffu, v, 31);
+    }
+    if (flush) {
+        __syncthreads();
+        // 5. Fold the committed entries into the fp32 checkpoint rows of the HC
+        //    heads: FH rows per thread in registers, buffered B applied 8 entries
+        //    at a time; store the checkpoint and the requantised copy; dot the
+        //    fresh copy with C.
+        const int c4 = tid % TPR4, q0 = tid / TPR4;
+        float4 Cq[TQ];
+#pragma unroll
+        for (int m = 0; m < TQ; ++m)
+            Cq[m] = (reads && m < T) ? *reinterpret_cast<const float4 *>(sCf + m * N + 4 * c4)
+                                     : make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int rb = 0; rb < nrows; rb += FH * RPP4) {  // same trip count for every lane
+            float4 v[FH];
+#pragma unroll
+            for (int k = 0; k < FH; ++k) {
+                const int gr = rb + q0 + k * RPP4;
+                v[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (gr < nrows) {
+                    v[k] = load_quad<SK_F32>(a.ckpt, tile0 + (int64_t)gr * N + 4 * c4);
+                    const float dc = sfdec[gr / P];
+                    v[k].x *= dc; v[k].y *= dc; v[k].z *= dc; v[k].w *= dc;
                 }
             }
-            consumer_sync();
-            for (int i = tid; i < HC * nE; i += kThreads) {
-                const int hh = i / nE, e = i - hh * nE;
-                const float *lam = slam + hh * E + base;
-                const float se = a.dt_scales ? dt_of(hh, e) : 1.f;
-                if (reads) {
+            for (int eb = 0; eb < L0; eb += 8) {
+                float4 Bq[8];
 #pragma unroll
-                    for (int m = 0; m < TQ; ++m)
-                        if (m < T && e >= e0 && e <= L0 + m)
-                            scoef[(hh * TQ + m) * E + e] = expf(lam[L0 + m] - lam[e]) * sd[m * E + e] * se;
+                for (int j = 0; j < 8; ++j) {
+                    const uint8_t *Br = sB + (base + eb + j) * brow;
+                    Bq[j] = (eb + j < L0) ? make_float4(raw_f(Br, 4 * c4, bf), raw_f(Br, 4 * c4 + 1, bf),
+                                                        raw_f(Br, 4 * c4 + 2, bf), raw_f(Br, 4 * c4 + 3, bf))
+                                          : make_float4(0.f, 0.f, 0.f, 0.f);
                 }
-                if (flush && e < L0) su[hh * E + e] = expf(lam[L0 - 1] - lam[e]) * se;
-            }
-            for (int i = tid; i < HC; i += kThreads) {
-                const float *lam = slam + i * E + base;
-                sfdec[i] = flush ? expf(lam[L0 - 1]) : 1.f;
-#pragma unroll
-                for (int m = 0; m < TQ; ++m)
-                    if (reads && m < T) sdec[i * TQ + m] = expf(lam[L0 + m] - (flush ? lam[L0 - 1] : 0.f));
-            }
-            consumer_sync();
-        }
-
-        if (flush) {
-            // Fold this part's fp32 checkpoint rows (staged), FR rows per thread held
-            // in registers, buffered B applied 8 entries at a time; store the
-            // checkpoint and the requantised copy, dot the fresh copy with C.
-            const int r0 = part * rpp_fold, nr = min(nrows, r0 + rpp_fold) - r0;
-            const float *tf = reinterpret_cast<const float *>(st + SG.tile);
-            float4 Cq[TQ];
-#pragma unroll
-            for (int m = 0; m < TQ; ++m)
-                Cq[m] = (reads && m < T) ? *reinterpret_cast<const float4 *>(sCf + m * N + 4 * c4)
-                                         : make_float4(0.f, 0.f, 0.f, 0.f);
-            constexpr int FH = 4;  // rows in registers at a time
-#pragma unroll 1
-            for (int kh = 0; kh < FR; kh += FH) {
-                float4 v[FH];
 #pragma unroll
                 for (int k = 0; k < FH; ++k) {
-                    const int rl = q0 + (kh + k) * RPP4;
-                    v[k] = make_float4(0.f, 0.f, 0.f, 0.f);
-                    if (rl < nr) {
-                        v[k] = *reinterpret_cast<const float4 *>(tf + rl * N + 4 * c4);
-                        const float dc = sfdec[(r0 + rl) / P];
-                        v[k].x *= dc; v[k].y *= dc; v[k].z *= dc; v[k].w *= dc;
-                    }
-                }
-#pragma unroll 1
-                for (int eb = 0; eb < L0; eb += 8) {
-                    float4 Bq[8];
+                    const int gr = rb + q0 + k * RPP4;
+                    if (gr >= nrows) continue;
+                    const int hh = gr / P, p = gr - hh * P;
+                    const uint8_t *xr = sx + (hh * E + base + eb) * xrow;
+                    const float *uw = su + hh * E + eb;
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
-                        const uint8_t *Br = sB + (base + eb + j) * brow;
-                        Bq[j] = (eb + j < L0) ? make_float4(raw_f(Br, 4 * c4, bf), raw_f(Br, 4 * c4 + 1, bf),
-                                                            raw_f(Br, 4 * c4 + 2, bf), raw_f(Br, 4 * c4 + 3, bf))
-                                              : make_float4(0.f, 0.f, 0.f, 0.f);
-                    }
-#pragma unroll
-                    for (int k = 0; k < FH; ++k) {
-                        const int rl = q0 + (kh + k) * RPP4;
-                        if (rl >= nr) continue;
-                        const int gr = r0 + rl, hh = gr / P, p = gr - hh * P;
-                        const uint8_t *xr = sx + (hh * E + base + eb) * xrow;
-                        const float *uw = su + hh * E + eb;
-#pragma unroll
-                        for (int j = 0; j < 8; ++j) {
-                            if (eb + j < L0) {
-                                const float w = uw[j] * raw_f(xr + j * xrow, p, bf);
-                                v[k].x = fmaf(w, Bq[j].x, v[k].x); v[k].y = fmaf(w, Bq[j].y, v[k].y);
-                                v[k].z = fmaf(w, Bq[j].z, v[k].z); v[k].w = fmaf(w, Bq[j].w, v[k].w);
-                            }
-                        }
-                    }
-                }
-#pragma unroll
-                for (int k = 0; k < FH; ++k) {
-                    const int rl = q0 + (kh + k) * RPP4;
-                    const bool valid = rl < nr;
-                    const int gr = r0 + rl;
-                    const int64_t el = tile0 + (int64_t)(valid ? gr : 0) * N + 4 * c4;
-                    if (a.op == OP_EXPORT) {
-                        if (valid) *reinterpret_cast<float4 *>(a.out + el) = v[k];
-                        continue;
-                    }
-                    if (valid) *reinterpret_cast<float4 *>(a.ckpt + el) = v[k];
-                    float4 rd = v[k];
-                    if (RK == SK_BF16) {
-                        if (valid) rd = store_quad<SK_BF16>(a.rc, el, v[k], 0.f, 0.f);
-                    } else if (RK == SK_FP8) {
-                        float am = fmaxf(fmaxf(fabsf(v[k].x), fabsf(v[k].y)), fmaxf(fabsf(v[k].z), fabsf(v[k].w)));
-                        am = group_max<TPR4>(am);
-                        const float sc = fp8_scale(am);
-                        if (valid) {
-                            rd = store_quad<SK_FP8>(a.rc, el, v[k], 0.f, sc);
-                            if (c4 == 0) a.rc_scale[row0 * P + gr] = sc;
-                        }
-                    }
-                    if (reads) {
-#pragma unroll
-                        for (int m = 0; m < TQ; ++m) {
-                            float d = rd.x * Cq[m].x + rd.y * Cq[m].y + rd.z * Cq[m].z + rd.w * Cq[m].w;
-                            d = group_sum<TPR4>(d);
-                            if (c4 == 0 && valid && m < T) sdot[gr * TQ + m] = d;
+                        if (eb + j < L0) {
+                            const float w = uw[j] * raw_f(xr + j * xrow, p, bf);
+                            v[k].x = fmaf(w, Bq[j].x, v[k].x); v[k].y = fmaf(w, Bq[j].y, v[k].y);
+                            v[k].z = fmaf(w, Bq[j].z, v[k].z); v[k].w = fmaf(w, Bq[j].w, v[k].w);
                         }
                     }
                 }
             }
-        } else if (reads) {
-            // Read: LPR lanes per staged read-copy row, C fragments in registers.
-            float Cf[kCregs ? TQ : 1][kCregs ? CPL * EPC : 1];
-            if (kCregs) {
 #pragma unroll
-                for (int m = 0; m < (kCregs ? TQ : 1); ++m)
-#pragma unroll
-                    for (int k = 0; k < (kCregs ? CPL : 1); ++k)
-#pragma unroll
-                        for (int e = 0; e < (kCregs ? EPC : 1); ++e)
-                            Cf[m][k * EPC + e] =
-                                (m < T) ? sCf[m * N + (q + LPR * ((k + rot) % CPL)) * EPC + e] : 0.f;
-            }
-            const uint4 *tile = reinterpret_cast<const uint4 *>(st + SG.tile);
-            const float *ssc = reinterpret_cast<const float *>(st + SG.scale);
-            const int r0 = part * rpp_read, nr = min(nrows, r0 + rpp_read) - r0;
-            for (int rb = 0; rb < nr; rb += RPPR) {  // same trip count for every lane
-                const int rl = rb + rrow;
-                const bool valid = rl < nr;
-                float acc[TQ];
-#pragma unroll
-                for (int m = 0; m < TQ; ++m) acc[m] = 0.f;
-#pragma unroll
-                for (int k = 0; k < CPL; ++k) {
-                    const int ch = q + LPR * ((k + rot) % CPL);
-                    float vv[EPC];
-                    if (valid) unpack<RK>(tile[rl * TPR + ch], vv);
-                    else {
-#pragma unroll
-                        for (int e = 0; e < EPC; ++e) vv[e] = 0.f;
-                    }
-#pragma unroll
-                    for (int m = 0; m < TQ; ++m)
-#pragma unroll
-                        for (int e = 0; e < EPC; ++e)
-                            acc[m] = fmaf(vv[e], kCregs ? Cf[kCregs ? m : 0][kCregs ? k * EPC + e : 0]
-                                                        : sCf[m * N + ch * EPC + e], acc[m]);
+            for (int k = 0; k < FH; ++k) {
+                const int gr = rb + q0 + k * RPP4;
+                const bool valid = gr < nrows;
+                const int64_t el = tile0 + (int64_t)(valid ? gr : 0) * N + 4 * c4;
+                if (a.op == OP_EXPORT) {
+                    if (valid) *reinterpret_cast<float4 *>(a.out + el) = v[k];
+                    continue;
                 }
+                if (valid) *reinterpret_cast<float4 *>(a.ckpt + el) = v[k];
+                float4 rd = v[k];
+                if (RK == SK_BF16) {
+                    if (valid) rd = store_quad<SK_BF16>(a.rc, el, v[k], 0.f, 0.f);
+                } else if (RK == SK_FP8) {
+                    float am = fmaxf(fmaxf(fabsf(v[k].x), fabsf(v[k].y)), fmaxf(fabsf(v[k].z), fabsf(v[k].w)));
+                    am = group_max<TPR4>(am);
+                    const float sc = fp8_scale(am);
+                    if (valid) {
+                        rd = store_quad<SK_FP8>(a.rc, el, v[k], 0.f, sc);
+                        if (c4 == 0) a.rc_scale[row0 * P + gr] = sc;
+                    }
+                }
+                if (reads) {
 #pragma unroll
-                for (int m = 0; m < TQ; ++m) {
-                    const float d = group_sum<LPR>(acc[m]);
-                    if (q == 0 && valid && m < T)
-                        sdot[(r0 + rl) * TQ + m] = (RK == SK_FP8) ? d * ssc[rl] : d;
+                    for (int m = 0; m < TQ; ++m) {
+                        float d = rd.x * Cq[m].x + rd.y * Cq[m].y + rd.z * Cq[m].z + rd.w * Cq[m].w;
+                        d = group_sum<TPR4>(d);
+                        if (c4 == 0 && valid && m < T) sdot[gr * TQ + m] = d;
+                    }
                 }
             }
         }
-
-        if (reads && part == nparts - 1) {
-            consumer_sync();
-            // Outputs y[b, m, h0 + hh, :] and ring appends (slots seq_pos + m mod R).
+        if (reads) {
+            __syncthreads();
+            // Outputs of the folded sequence: the fresh copy plus the call's own tokens.
             for (int i = tid; i < T * HC * P; i += kThreads) {
                 const int m = i / (HC * P), r2 = i - m * HC * P;
                 const int hh = r2 / P, p = r2 - hh * P;
@@ -573,30 +363,29 @@ __global__ void __maxnreg__(112) m2_replay_kernel(const M2Args a) {
                 yv = fmaf(a.D[h0 + hh], raw_f(sx + (hh * E + W + m) * xrow, p, bf), yv);
                 a.y[((int64_t)(b * T + m) * H + h0 + hh) * P + p] = yv;
             }
-            const int xch = xrow / 16, bch = brow / 16;
-            for (int i = tid; i < T * HC * xch; i += kThreads) {
-                const int m = i / (HC * xch), r2 = i - m * HC * xch;
-                const int hh = r2 / xch, k = r2 - hh * xch;
-                const int slot = (spmod + m) % R;
-                *reinterpret_cast<uint4 *>(reinterpret_cast<uint8_t *>(a.xbuf) + (((row0 + hh) * R + slot) * P) * ib + k * 16) =
-                    *reinterpret_cast<const uint4 *>(sx + (hh * E + W + m) * xrow + k * 16);
-            }
-            if (tid < T * HC) {
-                const int m = tid / HC, hh = tid - m * HC;
-                a.dtbuf[(row0 + hh) * a.Rs + (spmod + m) % R] = dtn[m * HC + hh];
-            }
-            if (hc == 0) {  // the group's first item writes the group's B
-                for (int i = tid; i < T * bch; i += kThreads) {
-                    const int m = i / bch, k = i - m * bch;
-                    const int slot = (spmod + m) % R;
-                    *reinterpret_cast<uint4 *>(reinterpret_cast<uint8_t *>(a.Bbuf) + (((int64_t)(b * G + g) * R + slot) * N) * ib + k * 16) =
-                        *reinterpret_cast<const uint4 *>(sB + (W + m) * brow + k * 16);
-                }
-            }
         }
-        consumer_sync();  // every consumer is done with the stage
-        if (lane == 0) mbar_arrive(&empty[s]);
-        s = (s + 1 == NS) ? 0 : s + 1;
+    }
+    if (!reads) return;
+
+    // 6. Append the call's tokens to the ring (slots seq_pos + m mod R).
+    for (int i = tid; i < T * HC * xch; i += kThreads) {
+        const int m = i / (HC * xch), r2 = i - m * HC * xch;
+        const int hh = r2 / xch, k = r2 - hh * xch;
+        const int slot = (spmod + m) % R;
+        *reinterpret_cast<uint4 *>(reinterpret_cast<uint8_t *>(a.xbuf) + (((row0 + hh) * R + slot) * P) * ib + k * 16) =
+            *reinterpret_cast<const uint4 *>(sx + (hh * E + W + m) * xrow + k * 16);
+    }
+    for (int i = tid; i < T * HC; i += kThreads) {
+        const int m = i / HC, hh = i - m * HC;
+        a.dtbuf[(row0 + hh) * Rs + (spmod + m) % R] = dtn[m * HC + hh];
+    }
+    if (hc == 0) {  // the group's first chunk writes the group's B
+        for (int i = tid; i < T * bch; i += kThreads) {
+            const int m = i / bch, k = i - m * bch;
+            const int slot = (spmod + m) % R;
+            *reinterpret_cast<uint4 *>(reinterpret_cast<uint8_t *>(a.Bbuf) + (((int64_t)(b * G + g) * R + slot) * N) * ib + k * 16) =
+                *reinterpret_cast<const uint4 *>(sB + (W + m) * brow + k * 16);
+        }
     }
 }
 
@@ -716,12 +505,13 @@ __global__ void __launch_bounds__(kThreads) m2_eager_kernel(const M2Args a) {
 // ---------------------------------------------------------------------------
 template <int N, int RK, int TQ>
 inline cudaError_t launch_replay_t(const M2Args &a, size_t smem, cudaStream_t st) {
-    auto k = m2_replay_kernel<N, RK, TQ>;
+    auto k = m2_prep_kernel<N, RK, TQ>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    k<<<a.grid, kThreads + 32, smem, st>>>(a);
+    k<<<a.B * (a.H / a.HC), kThreads, smem, st>>>(a);
     return cudaGetLastError();
 }
+
 template <int N, int SK, int TQ>
 inline cudaError_t launch_eager_t(const M2Args &a, size_t smem, cudaStream_t st) {
     auto k = m2_eager_kernel<N, SK, TQ>;
@@ -746,7 +536,7 @@ inline cudaError_t dispatch_tq(bool eager, int rk, int TQ, const M2Args &a, size
     return dispatch_rk<N, 8>(eager, rk, a, smem, st);
 }
 
-// Per-dstate entry point; each instantiation lives in its own translation unit.
+// Per-dstate entry points; each instantiation lives in its own translation unit.
 template <int N>
 cudaError_t m2_dispatch_n(bool eager, int rk, int TQ, const M2Args &a, size_t smem, cudaStream_t st) {
     return dispatch_tq<N>(eager, rk, TQ, a, smem, st);

@@ -1,0 +1,65 @@
+// rssm_read.cu -- host launcher of the replay-read kernel (rssm_read.cuh).
+#include "rssm_read.cuh"
+
+#include "rssm_internal.h"
+
+namespace rssm {
+
+extern template cudaError_t read_dispatch_n<16>(int, int, const ReadArgs &, size_t, cudaStream_t);
+extern template cudaError_t read_dispatch_n<32>(int, int, const ReadArgs &, size_t, cudaStream_t);
+extern template cudaError_t read_dispatch_n<64>(int, int, const ReadArgs &, size_t, cudaStream_t);
+extern template cudaError_t read_dispatch_n<128>(int, int, const ReadArgs &, size_t, cudaStream_t);
+
+static int tq_of_read(int T) { return T <= 1 ? 1 : (T <= 4 ? 4 : 8); }
+
+// Heads per read CTA: about 32 KiB of read copy per CTA, the heads sharing one
+// query row when a query row serves several heads (Mamba-2 groups).
+int read_heads_per_cta(const rssm_config &cf) {
+    const int rcb = cf.state_dtype == RSSM_F32 ? 4 : (cf.state_dtype == RSSM_BF16 ? 2 : 1);
+    const int qg = cf.kind == RSSM_MAMBA2 ? cf.nheads / cf.ngroups : 1;
+    const int unit = qg > 1 ? qg : cf.nheads;  // heads a CTA may span
+    int want = (32 * 1024) / (cf.headdim * cf.dstate * rcb);
+    if (want < 1) want = 1;
+    int hc = 1;
+    for (int d = 1; d <= unit && d <= want; ++d)
+        if (unit % d == 0 && cf.nheads % d == 0) hc = d;
+    return hc;
+}
+
+size_t read_smem_bytes(const rssm_config &cf, int T) {
+    const int ib = cf.input_dtype == RSSM_BF16 ? 2 : 4;
+    return (size_t)read_lay(read_heads_per_cta(cf), cf.headdim, cf.dstate, cf.window, tq_of_read(T), ib).bytes;
+}
+
+cudaError_t launch_read(const Ctx &h, int T, const void *Q, int q_bf16, int q_group, int64_t q_stride_b,
+                        int64_t q_stride_row, int64_t q_stride_m, const void *xnew, const float *D,
+                        float *y, cudaStream_t st) {
+    const rssm_config &cf = h.cfg;
+    ReadArgs r{};
+    r.B = cf.batch; r.H = cf.nheads; r.P = cf.headdim; r.R = (int)h.lay.ring; r.W = cf.window;
+    r.T = T; r.HC = read_heads_per_cta(cf); r.in_bf16 = cf.input_dtype == RSSM_BF16;
+    r.q_group = q_group; r.q_bf16 = q_bf16;
+    r.q_stride_b = q_stride_b; r.q_stride_row = q_stride_row; r.q_stride_m = q_stride_m;
+    r.Q = Q;
+    r.rc = cf.state_dtype == RSSM_F32 ? h.at(h.lay.ckpt_off) : h.at(h.lay.rc_off);
+    r.rc_scale = h.lay.rc_scale_bytes ? (const float *)h.at(h.lay.rc_scale_off) : nullptr;
+    r.xring = h.at(h.lay.xbuf_off);
+    r.xnew = xnew;
+    r.D = D;
+    r.seqinfo = (const int4 *)h.at(h.lay.seqinfo_off);
+    r.dec = (const float *)h.at(h.lay.dec_off);
+    r.coef = (const float *)h.at(h.lay.coef_off);
+    r.TQmax = (int)h.lay.tq_max;
+    r.Emax = cf.window + r.TQmax;
+    r.y = y;
+    const int TQ = tq_of_read(T);
+    const size_t smem = read_smem_bytes(cf, T);
+    switch (cf.dstate) {
+        case 16: return read_dispatch_n<16>(cf.state_dtype, TQ, r, smem, st);
+        case 32: return read_dispatch_n<32>(cf.state_dtype, TQ, r, smem, st);
+        case 64: return read_dispatch_n<64>(cf.state_dtype, TQ, r, smem, st);
+        default: return read_dispatch_n<128>(cf.state_dtype, TQ, r, smem, st);
+    }
+}
+
+}  // namespace rssm

@@ -1,0 +1,250 @@
+// rssm_read.cuh -- the replay-read kernel (sm_100a), shared by Mamba-2 and Gated DeltaNet.
+//
+// ReplaySSM computes a token's output from the checkpoint and the buffered inputs
+// without writing state ("Tenir le journal plutot que le solde",
+// blog.thibaultmonteiro.fr).  After the prep kernel has turned the buffer into a
+// per-head coefficient table, the output of query m of head h is
+//   y[b,m,h,p] = dec[b,h,m] * (S^[b,h,p,:] . Q[b,h,m,:])
+//                + sum_{e <= L0+m} coef[b,h,m,e] * X_e[p]  + D_h X_{L0+m}[p]
+// with S^ the read copy, X_e the buffered entries (Mamba-2 x, GDN v; e < L0 from
+// the ring, the call's own tokens after), Q the query (Mamba-2 C of the head's
+// group straight from the inputs; GDN the swept query r from the prep kernel).
+// Sequences whose buffer was folded in this call were fully served by the prep
+// kernel and are skipped.
+//
+// One CTA per (sequence, HC heads).  Every thread issues its read-copy chunks
+// (128-bit, L1 no-allocate) first -- they depend on nothing -- then the CTA
+// stages the small operands, dots the rows with the query (LPR lanes per row,
+// chunks interleaved so each warp load covers whole 64-byte row segments), and
+// applies the replay term.  Only ordinary loads and cp.async are used.
+#pragma once
+
+#include "rssm_device.cuh"
+
+namespace rssm {
+
+struct ReadArgs {
+    int B, H, P, R, W, T, HC, in_bf16;
+    int q_group;            // heads per query row (Mamba-2: H / G; GDN: 1)
+    int q_bf16;             // query dtype: 1 = input bf16, 0 = fp32
+    int64_t q_stride_m;     // elements between queries m and m+1 of one (b, query row)
+    int64_t q_stride_b;     // elements between sequences
+    int64_t q_stride_row;   // elements between query rows
+    const void *Q;          // query vectors
+    const void *rc;         // read copy (or the fp32 checkpoint): [B][H][P][N]
+    const float *rc_scale;  // fp8 row scales [B][H][P]
+    const void *xring;      // buffered entries [B][H][R][P] (input dtype)
+    const void *xnew;       // the call's own entries [B][T][H][P] (input dtype)
+    const float *D;         // per-head skip (nullptr: none)
+    const int4 *seqinfo;    // per sequence {L0 replayed from the ring, ring slot of entry 0, folded, 0}
+    const float *dec;       // [B][H][TQmax]
+    const float *coef;      // [B][H][TQmax][Emax]
+    int TQmax, Emax;
+    float *y;               // [B][T][H][P]
+};
+
+// Shared memory of the read kernel (bytes, 16-byte aligned regions).
+struct ReadLay {
+    int q, x, coef, dec, dot, scale, info, bytes;
+};
+__host__ __device__ inline ReadLay read_lay(int HC, int P, int N, int W, int TQ, int ib) {
+    auto al = [](int v) { return (v + 15) & ~15; };
+    const int E = W + TQ;
+    ReadLay L{};
+    int o = 0;
+    L.q = o;    o += al(HC * TQ * N * 4);     // queries as fp32   [HC or 1][TQ][N]
+    L.x = o;    o += al(HC * E * P * ib);     // entries           [HC][E][P] raw
+    L.coef = o; o += al(HC * TQ * E * 4);     // coefficients      [HC][TQ][E]
+    L.dec = o;  o += al(HC * TQ * 4);         // decays            [HC][TQ]
+    L.dot = o;  o += al(HC * P * TQ * 4);     // S^ . Q per row    [HC*P][TQ]
+    L.scale = o; o += al(HC * P * 4);         // fp8 row scales    [HC*P]
+    L.info = o; o += 16;
+    L.bytes = o;
+    return L;
+}
+
+template <int N, int RK, int TQ>
+__global__ void __launch_bounds__(kThreads, TQ == 1 ? 4 : 2) replay_read_kernel(const ReadArgs a) {
+    constexpr int EPC = Chunk<RK>::EPC;   // stored elements per 16-byte chunk
+    constexpr int TPR = N / EPC;          // chunks per state row
+    constexpr int RCB = Chunk<RK>::BYTES;
+    constexpr int LPR = TPR < 4 ? TPR : 4;  // lanes per row
+    constexpr int CPL = TPR / LPR;          // chunks per lane per row
+    constexpr int RPP = kThreads / LPR;     // rows per pass
+    constexpr int MAXC = 8;                 // chunks in flight per thread
+    constexpr int PPR = MAXC / CPL > 0 ? MAXC / CPL : 1;  // passes per round
+    static_assert(CPL <= MAXC, "a lane's chunks of one row must fit a round");
+
+    extern __shared__ __align__(16) uint8_t smraw[];
+    const int tid = threadIdx.x;
+    const int H = a.H, P = a.P, R = a.R, W = a.W, T = a.T, HC = a.HC;
+    const int b = blockIdx.x / (H / HC);
+    const int h0 = (blockIdx.x - b * (H / HC)) * HC;
+    const int bf = a.in_bf16, ib = bf ? 2 : 4;
+    const int E = W + TQ;
+    const ReadLay Ly = read_lay(HC, P, N, W, TQ, ib);
+    float *sq = reinterpret_cast<float *>(smraw + Ly.q);
+    uint8_t *sx = smraw + Ly.x;
+    float *scoef = reinterpret_cast<float *>(smraw + Ly.coef);
+    float *sdec = reinterpret_cast<float *>(smraw + Ly.dec);
+    float *sdot = reinterpret_cast<float *>(smraw + Ly.dot);
+    float *ssc = reinterpret_cast<float *>(smraw + Ly.scale);
+    int *sinfo = reinterpret_cast<int *>(smraw + Ly.info);
+    const int64_t row0 = (int64_t)b * H + h0;
+    const int nrows = HC * P;
+    const uint8_t *tile = reinterpret_cast<const uint8_t *>(a.rc) + row0 * P * N * RCB;
+    const int q = tid % LPR, rrow = tid / LPR;
+
+    // 1. First round of read-copy chunks.
+    uint4 rv[MAXC];
+    auto issue = [&](int pass0) {
+#pragma unroll
+        for (int j = 0; j < PPR; ++j) {
+            const int r = (pass0 + j) * RPP + rrow;
+#pragma unroll
+            for (int k = 0; k < CPL; ++k)
+                if (r < nrows) rv[j * CPL + k] = ld_stream(tile + ((size_t)r * TPR + q + LPR * k) * 16);
+        }
+    };
+    issue(0);
+
+    // 2. Per-sequence info, coefficients, decays, the call's own entries.
+    if (tid == 0) {
+        const int4 si = a.seqinfo[b];
+        sinfo[0] = si.x; sinfo[1] = si.y; sinfo[2] = si.z;
+    }
+    const int xrow = P * ib, xch = xrow / 16;
+    for (int i = tid; i < T * HC * xch; i += kThreads) {
+        const int m = i / (HC * xch), r2 = i - m * HC * xch;
+        const int hh = r2 / xch, k = r2 - hh * xch;
+        cp_async16(sx + (hh * E + W + m) * xrow + k * 16,
+                   reinterpret_cast<const uint8_t *>(a.xnew) + (((int64_t)(b * T + m) * H + h0 + hh) * P) * ib + k * 16);
+    }
+    for (int i = tid; i < HC * T; i += kThreads) {
+        const int hh = i / T, m = i - hh * T;
+        sdec[hh * TQ + m] = a.dec[(row0 + hh) * a.TQmax + m];
+    }
+    // queries: one row for the CTA when its heads share a query row (Mamba-2 groups),
+    // else one per head
+    const bool shared_q = (h0 / a.q_group) == ((h0 + HC - 1) / a.q_group);
+    const int nq = shared_q ? 1 : HC;
+    for (int i = tid; i < nq * T * N; i += kThreads) {
+        const int hq = i / (T * N), r2 = i - hq * T * N;
+        const int m = r2 / N, n = r2 - m * N;
+        const int64_t qi = (int64_t)b * a.q_stride_b + (int64_t)((h0 + hq) / a.q_group) * a.q_stride_row +
+                           (int64_t)m * a.q_stride_m + n;
+        sq[(hq * TQ + m) * N + n] = a.q_bf16 ? bf16_bits_to_float(reinterpret_cast<const uint16_t *>(a.Q)[qi])
+                                             : reinterpret_cast<const float *>(a.Q)[qi];
+    }
+    if (RK == SK_FP8)
+        for (int i = tid; i < nrows / 4; i += kThreads) cp_async16(ssc + 4 * i, a.rc_scale + row0 * P + 4 * i);
+    __syncthreads();
+    const int L0 = sinfo[0], ckmod = sinfo[1], folded = sinfo[2];
+    if (folded) {  // served by the prep kernel
+        cp_async_wait_all();
+        return;
+    }
+    const int base = W - L0;
+    for (int i = tid; i < HC * T * (L0 + T); i += kThreads) {
+        const int hh = i / (T * (L0 + T)), r2 = i - hh * T * (L0 + T);
+        const int m = r2 / (L0 + T), e = r2 - m * (L0 + T);
+        scoef[(hh * TQ + m) * E + e] = (e <= L0 + m) ? a.coef[((row0 + hh) * a.TQmax + m) * a.Emax + e] : 0.f;
+    }
+    for (int i = tid; i < HC * L0 * xch; i += kThreads) {
+        const int hh = i / (L0 * xch), r2 = i - hh * L0 * xch;
+        const int e = r2 / xch, k = r2 - e * xch;
+        const int slot = (ckmod + e) % R;
+        cp_async16(sx + (hh * E + base + e) * xrow + k * 16,
+                   reinterpret_cast<const uint8_t *>(a.xring) + (((row0 + hh) * R + slot) * P) * ib + k * 16);
+    }
+
+    // 3. Rows dotted with their query.
+    if (RK == SK_FP8) {  // the row scales must have landed before the first dot is scaled
+        cp_async_wait_all();
+        __syncthreads();
+    }
+    for (int pass0 = 0; pass0 * RPP < nrows; pass0 += PPR) {
+        if (pass0 > 0) issue(pass0);
+#pragma unroll
+        for (int j = 0; j < PPR; ++j) {
+            const int r = (pass0 + j) * RPP + rrow;
+            const bool valid = r < nrows;
+            float acc[TQ];
+#pragma unroll
+            for (int m = 0; m < TQ; ++m) acc[m] = 0.f;
+            const float *qv = sq + (shared_q ? 0 : (valid ? r / P : 0)) * TQ * N;
+#pragma unroll
+            for (int k = 0; k < CPL; ++k) {
+                float v[EPC];
+                if (valid) unpack<RK>(rv[j * CPL + k], v);
+                else {
+#pragma unroll
+                    for (int e = 0; e < EPC; ++e) v[e] = 0.f;
+                }
+                const int c0 = (q + LPR * k) * EPC;
+#pragma unroll
+                for (int m = 0; m < TQ; ++m) {
+                    const float4 *q4 = reinterpret_cast<const float4 *>(qv + m * N + c0);
+#pragma unroll
+                    for (int e4 = 0; e4 < EPC / 4; ++e4) {
+                        const float4 w = q4[e4];
+                        acc[m] = fmaf(v[4 * e4], w.x, acc[m]);
+                        acc[m] = fmaf(v[4 * e4 + 1], w.y, acc[m]);
+                        acc[m] = fmaf(v[4 * e4 + 2], w.z, acc[m]);
+                        acc[m] = fmaf(v[4 * e4 + 3], w.w, acc[m]);
+                    }
+                }
+            }
+#pragma unroll
+            for (int m = 0; m < TQ; ++m) {
+                const float d = group_sum<LPR>(acc[m]);
+                if (q == 0 && valid && m < T)
+                    sdot[r * TQ + m] = (RK == SK_FP8) ? d * ssc[r] : d;
+            }
+        }
+    }
+    cp_async_wait_all();
+    __syncthreads();
+
+    // 4. y = dec * (S^ . Q) + replay term (+ D x).
+    for (int i = tid; i < T * HC * P; i += kThreads) {
+        const int m = i / (HC * P), r2 = i - m * HC * P;
+        const int hh = r2 / P, p = r2 - hh * P;
+        float yv = sdec[hh * TQ + m] * sdot[(hh * P + p) * TQ + m];
+        const float *cf = scoef + (hh * TQ + m) * E;
+        const uint8_t *xs = sx + (hh * E + base) * xrow;
+        for (int e = 0; e <= L0 + m; ++e) yv = fmaf(cf[e], raw_f(xs + e * xrow, p, bf), yv);
+        if (a.D) yv = fmaf(a.D[h0 + hh], raw_f(sx + (hh * E + W + m) * xrow, p, bf), yv);
+        a.y[((int64_t)(b * T + m) * H + h0 + hh) * P + p] = yv;
+    }
+}
+
+// Host-side launch of one instantiation, and the per-dstate entry point (each
+// dstate is compiled in its own translation unit, rssm_read_n*.cu).
+template <int N, int RK, int TQ>
+inline cudaError_t launch_read_t(const ReadArgs &r, size_t smem, cudaStream_t st) {
+    auto k = replay_read_kernel<N, RK, TQ>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    k<<<r.B * (r.H / r.HC), kThreads, smem, st>>>(r);
+    return cudaGetLastError();
+}
+
+template <int N>
+cudaError_t read_dispatch_n(int rk, int TQ, const ReadArgs &r, size_t smem, cudaStream_t st) {
+    if (TQ == 1) {
+        if (rk == SK_F32) return launch_read_t<N, SK_F32, 1>(r, smem, st);
+        if (rk == SK_BF16) return launch_read_t<N, SK_BF16, 1>(r, smem, st);
+        return launch_read_t<N, SK_FP8, 1>(r, smem, st);
+    }
+    if (TQ == 4) {
+        if (rk == SK_F32) return launch_read_t<N, SK_F32, 4>(r, smem, st);
+        if (rk == SK_BF16) return launch_read_t<N, SK_BF16, 4>(r, smem, st);
+        return launch_read_t<N, SK_FP8, 4>(r, smem, st);
+    }
+    if (rk == SK_F32) return launch_read_t<N, SK_F32, 8>(r, smem, st);
+    if (rk == SK_BF16) return launch_read_t<N, SK_BF16, 8>(r, smem, st);
+    return launch_read_t<N, SK_FP8, 8>(r, smem, st);
+}
+
+}  // namespace rssm

@@ -1,0 +1,6 @@
+// Replay-read kernel instantiations for dstate = 64.
+#include "rssm_read.cuh"
+
+namespace rssm {
+template cudaError_t read_dispatch_n<64>(int, int, const ReadArgs &, size_t, cudaStream_t);
+}  // namespace rssm

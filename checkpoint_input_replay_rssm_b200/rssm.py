@@ -36,7 +36,9 @@ class rssm_workspace_layout(ctypes.Structure):
         "error_off", "seq_pos_off", "ckpt_pos_off", "pending_off", "flush_count_off", "arrive_off",
         "A_off", "D_off", "ckpt_off", "ckpt_bytes", "rc_off", "rc_bytes", "rc_scale_off",
         "rc_scale_bytes", "ring", "ring_stride", "xbuf_off", "xbuf_bytes", "bbuf_off", "bbuf_bytes", "sbuf_off",
-        "sbuf_bytes", "tbuf_off", "tbuf_bytes", "snap_off", "snap_bytes", "total_bytes")]
+        "sbuf_bytes", "tbuf_off", "tbuf_bytes", "snap_off", "snap_bytes", "tq_max", "seqinfo_off",
+        "seqinfo_bytes", "dec_off", "dec_bytes", "coef_off", "coef_bytes", "query_off", "query_bytes",
+        "total_bytes")]
 
 
 class rssm_inputs(ctypes.Structure):
@@ -62,6 +64,7 @@ SIGNATURES = {
     "rssm_read_counters": (ctypes.c_int, [_VP, _VP, _VP, _VP, _VP]),
     "rssm_status_word": (ctypes.c_int, [_VP, _VP]),
     "rssm_clear_status": (ctypes.c_int, [_VP]),
+    "rssm_set_split_event": (ctypes.c_int, [_VP, _VP]),
     "rssm_launch_count": (ctypes.c_int64, [_VP]),
     "rssm_last_error": (ctypes.c_char_p, [_VP]),
 }
@@ -172,6 +175,10 @@ def rssm_status_word(h):
 
 def rssm_clear_status(h):
     _check(load().rssm_clear_status(h), h)
+
+
+def rssm_set_split_event(h, event_ptr):
+    _check(load().rssm_set_split_event(h, event_ptr), h)
 
 
 def rssm_launch_count(h) -> int:

@@ -120,6 +120,12 @@ typedef struct {
     size_t sbuf_off, sbuf_bytes;         /* Mamba-2 dt[B][H][ring_stride]; GDN alpha (fp32)        */
     size_t tbuf_off, tbuf_bytes;         /* GDN beta[B][H][ring_stride] (fp32)                     */
     size_t snap_off, snap_bytes;         /* EAGER: max_draft snapshots of the state (+ scales)      */
+    /* REPLAY: hand-off from the prep kernel to the read kernel within one call */
+    size_t tq_max;                       /* max(max_draft, 1): queries per call            */
+    size_t seqinfo_off, seqinfo_bytes;   /* int32[B][4]                                    */
+    size_t dec_off, dec_bytes;           /* fp32[B][H][tq_max]                             */
+    size_t coef_off, coef_bytes;         /* fp32[B][H][tq_max][window + tq_max]            */
+    size_t query_off, query_bytes;       /* GDN: fp32[B][H][tq_max][dstate] swept queries  */
     size_t total_bytes;
 } rssm_workspace_layout;
 
@@ -197,6 +203,12 @@ RSSM_API rssm_status rssm_read_counters(rssm_handle h, int64_t *seq_pos, int64_t
 RSSM_API rssm_status rssm_status_word(rssm_handle h, int32_t *info);
 /* Enqueue clearing of the device error word. */
 RSSM_API rssm_status rssm_clear_status(rssm_handle h);
+
+/* Measurement hook: when `event` (a cudaEvent_t) is not NULL, every REPLAY
+ * decode/verify records it on the handle's stream between its two kernels (the
+ * prep/flush kernel and the replay-read kernel), so a caller can time them
+ * apart.  NULL (the default) records nothing. */
+RSSM_API rssm_status rssm_set_split_event(rssm_handle h, void *event);
 
 /* Number of kernels this handle has enqueued so far (running total). */
 RSSM_API int64_t rssm_launch_count(rssm_handle h);
