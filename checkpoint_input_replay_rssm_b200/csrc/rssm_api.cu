@@ -96,7 +96,7 @@ void layout(const rssm_config *c, rssm_workspace_layout *L) {
         L->seqinfo_off = take(L->seqinfo_bytes);
         L->dec_bytes = B * H * TQm * 4;
         L->dec_off = take(L->dec_bytes);
-        L->coef_bytes = B * H * TQm * ((size_t)c->window + TQm) * 4;
+        L->coef_bytes = B * H * TQm * (((size_t)c->window + TQm + 3) & ~(size_t)3) * 4;
         L->coef_off = take(L->coef_bytes);
         if (c->kind == RSSM_GDN) {
             L->query_bytes = B * H * TQm * N * 4;

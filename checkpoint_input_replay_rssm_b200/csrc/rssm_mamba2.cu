@@ -42,7 +42,7 @@ cudaError_t mamba2_launch(const Ctx &h, int op, int T, const rssm_inputs *in, fl
         a.dec = (float *)h.at(h.lay.dec_off);
         a.coef = (float *)h.at(h.lay.coef_off);
         a.TQmax = (int)h.lay.tq_max;
-        a.Emax = cf.window + a.TQmax;
+        a.Emax = (cf.window + a.TQmax + 3) & ~3;
     }
     a.c = h.counters();
     a.A = (const float *)h.at(h.lay.A_off); a.D = (const float *)h.at(h.lay.D_off);

@@ -34,7 +34,7 @@ struct M2Args {
     int4 *seqinfo;      // per sequence, for the read kernel: {L0, ring slot of entry 0, folded, 0}
     float *dec;         // [B][H][TQmax] decay of S^ C
     float *coef;        // [B][H][TQmax][Emax] replay coefficients
-    int TQmax, Emax;
+    int TQmax, Emax;    // Emax: padded row length of the coefficient table
     Counters c;
     const float *A, *D;
     float *ckpt;        // fp32 [B][H][P][N]
@@ -62,28 +62,31 @@ __host__ __device__ constexpr int pad4(int n) { return (n + 3) & ~3; }
 __host__ __device__ constexpr int dt_row_max_bytes(int W) { return ((W + 8 + 3) & ~3) * 4; }
 
 // Shared memory of the prep kernel (bytes, 16-byte aligned regions).  Entry
-// slots: E = W + TQ; committed entries sit right-aligned before slot W, the
-// call's own tokens at W..W+T-1, so logical entry e is slot (W - L0) + e.
+// slots of x: E = W + TQ; committed entries sit right-aligned before slot W and
+// the call's own tokens at W..W+T-1, so logical entry e is slot (W - L0) + e.
+// The group's B ring is staged whole (R <= W + 8 rows), with no wait for the
+// counters.
 struct M2PrepLay {
-    int sC, sB, sx, dring, dtn, sd, slam, scoef, sdec, su, sfdec, sCf, sdot, si, bytes;
+    int sC, sBr, sBn, sx, dring, dtn, sd, slam, scoef, sdec, su, sfdec, sCf, sdot, si, bytes;
 };
 __host__ __device__ inline M2PrepLay m2_prep_lay(int HC, int P, int N, int W, int TQ, int ib) {
     const int E = W + TQ;
     M2PrepLay L{};
     int o = 0;
-    L.sC = o;    o += a16(TQ * N * ib);          // raw C of the queries   [TQ][N]
-    L.sB = o;    o += a16(E * N * ib);           // raw B of the entries   [E][N]
-    L.sx = o;    o += a16(HC * E * P * ib);      // raw x of the entries   [HC][E][P]
-    L.dring = o; o += a16(HC * dt_row_max_bytes(W));  // dt ring rows      [HC][Rs]
-    L.dtn = o;   o += a16(TQ * HC * 4);          // dt of the call's tokens [TQ][HC]
-    L.sd = o;    o += a16(TQ * E * 4);           // B_e . C_m              [TQ][E]
-    L.slam = o;  o += a16(HC * E * 4);           // prefix sums of dt*A    [HC][E]
-    L.scoef = o; o += a16(HC * TQ * E * 4);      // replay coefficients    [HC][TQ][E]
-    L.sdec = o;  o += a16(HC * TQ * 4);          // decay of S^ C          [HC][TQ]
-    L.su = o;    o += a16(HC * E * 4);           // fold weights           [HC][E]
+    L.sC = o;    o += a16(TQ * N * ib);          // raw C of the queries     [TQ][N]
+    L.sBr = o;   o += a16((W + 8) * N * ib);     // raw B ring of the group  [R][N]
+    L.sBn = o;   o += a16(TQ * N * ib);          // raw B of the call's tokens [TQ][N]
+    L.sx = o;    o += a16(HC * E * P * ib);      // raw x of the entries     [HC][E][P]
+    L.dring = o; o += a16(HC * dt_row_max_bytes(W));  // dt ring rows        [HC][Rs]
+    L.dtn = o;   o += a16(TQ * HC * 4);          // dt of the call's tokens  [TQ][HC]
+    L.sd = o;    o += a16(TQ * E * 4);           // B_e . C_m                [TQ][E]
+    L.slam = o;  o += a16(HC * E * 4);           // prefix sums of dt*A      [HC][E]
+    L.scoef = o; o += a16(HC * TQ * E * 4);      // replay coefficients      [HC][TQ][E]
+    L.sdec = o;  o += a16(HC * TQ * 4);          // decay of S^ C            [HC][TQ]
+    L.su = o;    o += a16(HC * E * 4);           // fold weights             [HC][E]
     L.sfdec = o; o += a16(HC * 4);               // decay of the folded checkpoint [HC]
-    L.sCf = o;   o += a16(TQ * N * 4);           // C as fp32              [TQ][N]
-    L.sdot = o;  o += a16(HC * P * TQ * 4);      // fresh copy . C per row [HC*P][TQ]
+    L.sCf = o;   o += a16(TQ * N * 4);           // C as fp32                [TQ][N]
+    L.sdot = o;  o += a16(HC * P * TQ * 4);      // fresh copy . C per row   [HC*P][TQ]
     L.si = o;    o += 32;
     L.bytes = o;
     return L;
@@ -92,10 +95,10 @@ __host__ __device__ inline M2PrepLay m2_prep_lay(int HC, int P, int N, int W, in
 // ---------------------------------------------------------------------------
 // Prep / flush kernel: decode (T = 1), verify (T = K), flush and export (T = 0).
 //
-// One CTA per (sequence b, group g, chunk of HC heads of the group).  It reads
-// the sequence's counters, stages the group's buffered B, the heads' dt ring
-// rows and the call's tokens, and computes once per group B_e . C_m and per head
-// the prefix sums Lam of dt*A.  Then either
+// One CTA per (sequence b, group g, chunk of HC heads of the group).  In one
+// round trip it reads the sequence's counters and stages the group's whole B
+// ring, the heads' dt ring rows and the call's tokens; it computes once per
+// group B_e . C_m and per head the prefix sums Lam of dt*A.  Then either
 //   * (no fold) it writes the replay coefficients
 //       coef[e] = e^{Lam_{L0+m} - Lam_e} (B_e . C_m) s_e,   dec = e^{Lam_{L0+m}}
 //     for the read kernel, or
@@ -106,11 +109,13 @@ __host__ __device__ inline M2PrepLay m2_prep_lay(int HC, int P, int N, int W, in
 // Last it appends the call's tokens to the ring; the last CTA of the sequence
 // publishes the counters.
 // ---------------------------------------------------------------------------
-template <int N, int RK, int TQ>
-__global__ void __launch_bounds__(kThreads) m2_prep_kernel(const M2Args a) {
+template <int N, int RK, int TQ, bool BF>
+__global__ void __launch_bounds__(kThreads, 3) m2_prep_kernel(const M2Args a) {
     constexpr int TPR4 = N / 4;  // lanes per row, fp32 quad mapping
     constexpr int RPP4 = kThreads / TPR4;
-    constexpr int FH = 4;        // fold rows held in registers per thread
+    constexpr int FH = 2;        // fold rows held in registers per thread
+    constexpr int FB = 4;        // buffered B entries held in registers per block
+    constexpr int IB = BF ? 2 : 4;
     extern __shared__ __align__(16) uint8_t smraw[];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int H = a.H, P = a.P, W = a.W, R = a.R, T = a.T, G = a.G, HC = a.HC;
@@ -120,9 +125,8 @@ __global__ void __launch_bounds__(kThreads) m2_prep_kernel(const M2Args a) {
     const int g = rem / cpg, hc = rem - g * cpg;
     const int h0 = g * hpg + hc * HC;
     const int E = W + TQ;
-    const int bf = a.in_bf16, ib = bf ? 2 : 4;
-    const M2PrepLay Ly = m2_prep_lay(HC, P, N, W, TQ, ib);
-    uint8_t *sC = smraw + Ly.sC, *sB = smraw + Ly.sB, *sx = smraw + Ly.sx;
+    const M2PrepLay Ly = m2_prep_lay(HC, P, N, W, TQ, IB);
+    uint8_t *sC = smraw + Ly.sC, *sBr = smraw + Ly.sBr, *sBn = smraw + Ly.sBn, *sx = smraw + Ly.sx;
     float *dring = reinterpret_cast<float *>(smraw + Ly.dring);
     float *dtn = reinterpret_cast<float *>(smraw + Ly.dtn);
     float *sd = reinterpret_cast<float *>(smraw + Ly.sd);
@@ -138,10 +142,13 @@ __global__ void __launch_bounds__(kThreads) m2_prep_kernel(const M2Args a) {
     const int64_t tile0 = row0 * P * N;
     const int nrows = HC * P;
     const bool reads = (a.op == OP_DECODE || a.op == OP_VERIFY);
-    const int xrow = P * ib, brow = N * ib, xch = xrow / 16, bch = brow / 16;
+    const int xrow = P * IB, brow = N * IB, xch = xrow / 16, bch = brow / 16;
     const int Rs = a.Rs;
+    auto ldx = [](const uint8_t *p) -> float {
+        return BF ? bf16_bits_to_float(*reinterpret_cast<const uint16_t *>(p)) : *reinterpret_cast<const float *>(p);
+    };
 
-    // 1. Counters (thread 0) and the call's tokens.
+    // 1. Counters (thread 0); everything that does not depend on them, at once.
     if (tid == 0) {
         SeqState ss = read_counters(a.c, b, W);
         const int L0 = (int)(ss.seq - ss.ckpt);
@@ -162,66 +169,63 @@ __global__ void __launch_bounds__(kThreads) m2_prep_kernel(const M2Args a) {
                                    flush ? ss.seq : -1, (a.op == OP_VERIFY) ? T : -1, flush);
         }
     }
-    for (int i = tid; i < T * bch; i += kThreads) {
-        const int m = i / bch, k = i - m * bch;
-        const int64_t src = (((int64_t)(b * T + m) * G + g) * N) * ib + k * 16;
-        cp_async16(sC + m * brow + k * 16, reinterpret_cast<const uint8_t *>(a.Cm) + src);
-        cp_async16(sB + (W + m) * brow + k * 16, reinterpret_cast<const uint8_t *>(a.Bm) + src);
+    {
+        const uint8_t *src = reinterpret_cast<const uint8_t *>(a.Bbuf) + ((int64_t)(b * G + g) * R) * brow;
+        for (int i = tid; i < R * bch; i += kThreads) cp_async16(sBr + i * 16, src + i * 16);
     }
-    for (int i = tid; i < T * HC * xch; i += kThreads) {
-        const int m = i / (HC * xch), r2 = i - m * HC * xch;
-        const int hh = r2 / xch, k = r2 - hh * xch;
-        cp_async16(sx + (hh * E + W + m) * xrow + k * 16,
-                   reinterpret_cast<const uint8_t *>(a.x) + (((int64_t)(b * T + m) * H + h0 + hh) * P) * ib + k * 16);
+    for (int i = tid; i < HC * Rs / 4; i += kThreads) cp_async16(dring + 4 * i, a.dtbuf + row0 * Rs + 4 * i);
+    for (int row = warp; row < T; row += kWarps) {
+        const int64_t src = (((int64_t)(b * T + row) * G + g) * N) * IB;
+        for (int k = lane; k < bch; k += 32) {
+            cp_async16(sC + row * brow + k * 16, reinterpret_cast<const uint8_t *>(a.Cm) + src + k * 16);
+            cp_async16(sBn + row * brow + k * 16, reinterpret_cast<const uint8_t *>(a.Bm) + src + k * 16);
+        }
+    }
+    for (int row = warp; row < T * HC; row += kWarps) {
+        const int m = row / HC, hh = row - m * HC;
+        const uint8_t *src = reinterpret_cast<const uint8_t *>(a.x) + (((int64_t)(b * T + m) * H + h0 + hh) * P) * IB;
+        for (int k = lane; k < xch; k += 32) cp_async16(sx + (hh * E + W + m) * xrow + k * 16, src + k * 16);
     }
     for (int i = tid; i < T * HC; i += kThreads) {
         const int m = i / HC, hh = i - m * HC;
         dtn[m * HC + hh] = a.dt[(int64_t)(b * T + m) * H + h0 + hh];
     }
-    for (int i = tid; i < HC * Rs / 4; i += kThreads) cp_async16(dring + 4 * i, a.dtbuf + row0 * Rs + 4 * i);
+    cp_async_wait_all();
     __syncthreads();
-    if (!si[0]) {
-        cp_async_wait_all();
-        return;
-    }
+    if (!si[0]) return;
     const int L0 = si[1], flush = si[2], ckmod = si[3], spmod = si[4];
     const int base = W - L0, nE = L0 + T;
     const int e0 = flush ? L0 : 0;  // first entry the outputs replay
-
-    // 2. Buffered entries: the group's B (always), the heads' x (only to fold).
-    for (int i = tid; i < L0 * bch; i += kThreads) {
-        const int e = i / bch, k = i - e * bch;
-        const int slot = (ckmod + e) % R;
-        cp_async16(sB + (base + e) * brow + k * 16,
-                   reinterpret_cast<const uint8_t *>(a.Bbuf) + (((int64_t)(b * G + g) * R + slot) * N) * ib + k * 16);
-    }
-    if (flush) {
-        for (int i = tid; i < HC * L0 * xch; i += kThreads) {
-            const int hh = i / (L0 * xch), r2 = i - hh * L0 * xch;
-            const int e = r2 / xch, k = r2 - e * xch;
-            const int slot = (ckmod + e) % R;
-            cp_async16(sx + (hh * E + base + e) * xrow + k * 16,
-                       reinterpret_cast<const uint8_t *>(a.xbuf) + (((row0 + hh) * R + slot) * P) * ib + k * 16);
-        }
-    }
-    cp_async_wait_all();
-    __syncthreads();
+    auto B_of = [&](int e) -> const uint8_t * {  // B of logical entry e
+        return e < L0 ? sBr + ((ckmod + e) % R) * brow : sBn + (e - L0) * brow;
+    };
     auto dt_of = [&](int hh, int e) -> float {
         return e < L0 ? dring[hh * Rs + (ckmod + e) % R] : dtn[(e - L0) * HC + hh];
     };
+    if (flush) {  // the heads' buffered x, needed only to fold
+        const int n1 = min(L0, R - ckmod);
+        for (int row = warp; row < 2 * HC; row += kWarps) {
+            const int hh = row >> 1, second = row & 1;
+            const int cnt = second ? L0 - n1 : n1;
+            const uint8_t *src = reinterpret_cast<const uint8_t *>(a.xbuf) +
+                                 (((row0 + hh) * R + (second ? 0 : ckmod)) * P) * IB;
+            uint8_t *dst = sx + (hh * E + base + (second ? n1 : 0)) * xrow;
+            for (int k = lane; k < cnt * xch; k += 32) cp_async16(dst + k * 16, src + k * 16);
+        }
+    }
 
-    // 3. B_e . C_m once for the group, C as fp32, prefix sums of dt*A per head.
+    // 2. B_e . C_m once for the group, C as fp32, prefix sums of dt*A per head.
     if (reads) {
         for (int pr = warp; pr < T * nE; pr += kWarps) {
             const int m = pr / nE, e = pr - m * nE;
             if (e > L0 + m) continue;  // warp-uniform
+            const uint8_t *Bp = B_of(e);
             float d = 0.f;
-            for (int n = lane; n < N; n += 32)
-                d = fmaf(raw_f(sB + (base + e) * brow, n, bf), raw_f(sC + m * brow, n, bf), d);
+            for (int n = lane; n < N; n += 32) d = fmaf(ldx(Bp + n * IB), ldx(sC + m * brow + n * IB), d);
             d = group_sum<32>(d);
             if (lane == 0) sd[m * E + e] = d;
         }
-        for (int i = tid; i < T * N; i += kThreads) sCf[i] = raw_f(sC, i, bf);
+        for (int i = tid; i < T * N; i += kThreads) sCf[i] = ldx(sC + i * IB);
     }
     for (int hh = warp; hh < HC; hh += kWarps) {
         const float Ah = a.A[h0 + hh];
@@ -236,7 +240,7 @@ __global__ void __launch_bounds__(kThreads) m2_prep_kernel(const M2Args a) {
     }
     __syncthreads();
 
-    // 4. Replay coefficients and decays (to the read kernel, or kept here to fold).
+    // 3. Replay coefficients and decays (to the read kernel, or kept here to fold).
     for (int i = tid; i < HC * nE; i += kThreads) {
         const int hh = i / nE, e = i - hh * nE;
         const float *lam = slam + hh * E + base;
@@ -269,17 +273,13 @@ __global__ void __launch_bounds__(kThreads) m2_prep_kernel(const M2Args a) {
         }
     }
     if (flush) {
+        cp_async_wait_all();
         __syncthreads();
-        // 5. Fold the committed entries into the fp32 checkpoint rows of the HC
-        //    heads: FH rows per thread in registers, buffered B applied 8 entries
-        //    at a time; store the checkpoint and the requantised copy; dot the
+        // 4. Fold the committed entries into the fp32 checkpoint rows of the HC
+        //    heads (FH rows per thread in registers, FB buffered B entries at a
+        //    time), store the checkpoint and the requantised copy, and dot the
         //    fresh copy with C.
         const int c4 = tid % TPR4, q0 = tid / TPR4;
-        float4 Cq[TQ];
-#pragma unroll
-        for (int m = 0; m < TQ; ++m)
-            Cq[m] = (reads && m < T) ? *reinterpret_cast<const float4 *>(sCf + m * N + 4 * c4)
-                                     : make_float4(0.f, 0.f, 0.f, 0.f);
         for (int rb = 0; rb < nrows; rb += FH * RPP4) {  // same trip count for every lane
             float4 v[FH];
 #pragma unroll
@@ -292,13 +292,12 @@ __global__ void __launch_bounds__(kThreads) m2_prep_kernel(const M2Args a) {
                     v[k].x *= dc; v[k].y *= dc; v[k].z *= dc; v[k].w *= dc;
                 }
             }
-            for (int eb = 0; eb < L0; eb += 8) {
-                float4 Bq[8];
+            for (int eb = 0; eb < L0; eb += FB) {
+                float4 Bq[FB];
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const uint8_t *Br = sB + (base + eb + j) * brow;
-                    Bq[j] = (eb + j < L0) ? make_float4(raw_f(Br, 4 * c4, bf), raw_f(Br, 4 * c4 + 1, bf),
-                                                        raw_f(Br, 4 * c4 + 2, bf), raw_f(Br, 4 * c4 + 3, bf))
+                for (int j = 0; j < FB; ++j) {
+                    const uint8_t *Br = B_of(eb + j) + 4 * c4 * IB;
+                    Bq[j] = (eb + j < L0) ? make_float4(ldx(Br), ldx(Br + IB), ldx(Br + 2 * IB), ldx(Br + 3 * IB))
                                           : make_float4(0.f, 0.f, 0.f, 0.f);
                 }
 #pragma unroll
@@ -306,12 +305,12 @@ __global__ void __launch_bounds__(kThreads) m2_prep_kernel(const M2Args a) {
                     const int gr = rb + q0 + k * RPP4;
                     if (gr >= nrows) continue;
                     const int hh = gr / P, p = gr - hh * P;
-                    const uint8_t *xr = sx + (hh * E + base + eb) * xrow;
+                    const uint8_t *xr = sx + (hh * E + base + eb) * xrow + p * IB;
                     const float *uw = su + hh * E + eb;
 #pragma unroll
-                    for (int j = 0; j < 8; ++j) {
+                    for (int j = 0; j < FB; ++j) {
                         if (eb + j < L0) {
-                            const float w = uw[j] * raw_f(xr + j * xrow, p, bf);
+                            const float w = uw[j] * ldx(xr + j * xrow);
                             v[k].x = fmaf(w, Bq[j].x, v[k].x); v[k].y = fmaf(w, Bq[j].y, v[k].y);
                             v[k].z = fmaf(w, Bq[j].z, v[k].z); v[k].w = fmaf(w, Bq[j].w, v[k].w);
                         }
@@ -343,7 +342,8 @@ __global__ void __launch_bounds__(kThreads) m2_prep_kernel(const M2Args a) {
                 if (reads) {
 #pragma unroll
                     for (int m = 0; m < TQ; ++m) {
-                        float d = rd.x * Cq[m].x + rd.y * Cq[m].y + rd.z * Cq[m].z + rd.w * Cq[m].w;
+                        const float4 Cq = *reinterpret_cast<const float4 *>(sCf + m * N + 4 * c4);
+                        float d = rd.x * Cq.x + rd.y * Cq.y + rd.z * Cq.z + rd.w * Cq.w;
                         d = group_sum<TPR4>(d);
                         if (c4 == 0 && valid && m < T) sdot[gr * TQ + m] = d;
                     }
@@ -353,38 +353,39 @@ __global__ void __launch_bounds__(kThreads) m2_prep_kernel(const M2Args a) {
         if (reads) {
             __syncthreads();
             // Outputs of the folded sequence: the fresh copy plus the call's own tokens.
-            for (int i = tid; i < T * HC * P; i += kThreads) {
-                const int m = i / (HC * P), r2 = i - m * HC * P;
+            for (int i = tid; i < T * nrows; i += kThreads) {
+                const int m = i / nrows, r2 = i - m * nrows;
                 const int hh = r2 / P, p = r2 - hh * P;
-                float yv = sdec[hh * TQ + m] * sdot[(hh * P + p) * TQ + m];
+                float yv = sdec[hh * TQ + m] * sdot[r2 * TQ + m];
                 const float *cf = scoef + (hh * TQ + m) * E;
-                const uint8_t *xs = sx + (hh * E + base) * xrow;
-                for (int e = e0; e <= L0 + m; ++e) yv = fmaf(cf[e], raw_f(xs + e * xrow, p, bf), yv);
-                yv = fmaf(a.D[h0 + hh], raw_f(sx + (hh * E + W + m) * xrow, p, bf), yv);
+                const uint8_t *xs = sx + (hh * E + base) * xrow + p * IB;
+                for (int e = e0; e <= L0 + m; ++e) yv = fmaf(cf[e], ldx(xs + e * xrow), yv);
+                yv = fmaf(a.D[h0 + hh], ldx(sx + (hh * E + W + m) * xrow + p * IB), yv);
                 a.y[((int64_t)(b * T + m) * H + h0 + hh) * P + p] = yv;
             }
         }
     }
     if (!reads) return;
 
-    // 6. Append the call's tokens to the ring (slots seq_pos + m mod R).
-    for (int i = tid; i < T * HC * xch; i += kThreads) {
-        const int m = i / (HC * xch), r2 = i - m * HC * xch;
-        const int hh = r2 / xch, k = r2 - hh * xch;
+    // 5. Append the call's tokens to the ring (slots seq_pos + m mod R).
+    for (int row = warp; row < T * HC; row += kWarps) {
+        const int m = row / HC, hh = row - m * HC;
         const int slot = (spmod + m) % R;
-        *reinterpret_cast<uint4 *>(reinterpret_cast<uint8_t *>(a.xbuf) + (((row0 + hh) * R + slot) * P) * ib + k * 16) =
-            *reinterpret_cast<const uint4 *>(sx + (hh * E + W + m) * xrow + k * 16);
+        uint8_t *dst = reinterpret_cast<uint8_t *>(a.xbuf) + (((row0 + hh) * R + slot) * P) * IB;
+        const uint8_t *src = sx + (hh * E + W + m) * xrow;
+        for (int k = lane; k < xch; k += 32)
+            *reinterpret_cast<uint4 *>(dst + k * 16) = *reinterpret_cast<const uint4 *>(src + k * 16);
     }
     for (int i = tid; i < T * HC; i += kThreads) {
         const int m = i / HC, hh = i - m * HC;
         a.dtbuf[(row0 + hh) * Rs + (spmod + m) % R] = dtn[m * HC + hh];
     }
     if (hc == 0) {  // the group's first chunk writes the group's B
-        for (int i = tid; i < T * bch; i += kThreads) {
-            const int m = i / bch, k = i - m * bch;
-            const int slot = (spmod + m) % R;
-            *reinterpret_cast<uint4 *>(reinterpret_cast<uint8_t *>(a.Bbuf) + (((int64_t)(b * G + g) * R + slot) * N) * ib + k * 16) =
-                *reinterpret_cast<const uint4 *>(sB + (W + m) * brow + k * 16);
+        for (int row = warp; row < T; row += kWarps) {
+            const int slot = (spmod + row) % R;
+            uint8_t *dst = reinterpret_cast<uint8_t *>(a.Bbuf) + (((int64_t)(b * G + g) * R + slot) * N) * IB;
+            for (int k = lane; k < bch; k += 32)
+                *reinterpret_cast<uint4 *>(dst + k * 16) = *reinterpret_cast<const uint4 *>(sBn + row * brow + k * 16);
         }
     }
 }
@@ -505,7 +506,7 @@ __global__ void __launch_bounds__(kThreads) m2_eager_kernel(const M2Args a) {
 // ---------------------------------------------------------------------------
 template <int N, int RK, int TQ>
 inline cudaError_t launch_replay_t(const M2Args &a, size_t smem, cudaStream_t st) {
-    auto k = m2_prep_kernel<N, RK, TQ>;
+    auto k = a.in_bf16 ? m2_prep_kernel<N, RK, TQ, true> : m2_prep_kernel<N, RK, TQ, false>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     k<<<a.B * (a.H / a.HC), kThreads, smem, st>>>(a);

@@ -28,7 +28,9 @@ int read_heads_per_cta(const rssm_config &cf) {
 
 size_t read_smem_bytes(const rssm_config &cf, int T) {
     const int ib = cf.input_dtype == RSSM_BF16 ? 2 : 4;
-    return (size_t)read_lay(read_heads_per_cta(cf), cf.headdim, cf.dstate, cf.window, tq_of_read(T), ib).bytes;
+    const int tqm = cf.max_draft > 1 ? cf.max_draft : 1;
+    const int Ep = (cf.window + tqm + 3) & ~3;
+    return (size_t)read_lay(read_heads_per_cta(cf), cf.headdim, cf.dstate, cf.window, tq_of_read(T), ib, Ep).bytes;
 }
 
 cudaError_t launch_read(const Ctx &h, int T, const void *Q, int q_bf16, int q_group, int64_t q_stride_b,
@@ -50,7 +52,7 @@ cudaError_t launch_read(const Ctx &h, int T, const void *Q, int q_bf16, int q_gr
     r.dec = (const float *)h.at(h.lay.dec_off);
     r.coef = (const float *)h.at(h.lay.coef_off);
     r.TQmax = (int)h.lay.tq_max;
-    r.Emax = cf.window + r.TQmax;
+    r.Emax = (cf.window + r.TQmax + 3) & ~3;
     r.y = y;
     const int TQ = tq_of_read(T);
     const size_t smem = read_smem_bytes(cf, T);

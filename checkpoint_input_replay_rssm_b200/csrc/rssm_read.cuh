@@ -39,7 +39,7 @@ struct ReadArgs {
     const int4 *seqinfo;    // per sequence {L0 replayed from the ring, ring slot of entry 0, folded, 0}
     const float *dec;       // [B][H][TQmax]
     const float *coef;      // [B][H][TQmax][Emax]
-    int TQmax, Emax;
+    int TQmax, Emax;        // Emax: padded row length of the coefficient table
     float *y;               // [B][T][H][P]
 };
 
@@ -47,14 +47,14 @@ struct ReadArgs {
 struct ReadLay {
     int q, x, coef, dec, dot, scale, info, bytes;
 };
-__host__ __device__ inline ReadLay read_lay(int HC, int P, int N, int W, int TQ, int ib) {
+__host__ __device__ inline ReadLay read_lay(int HC, int P, int N, int W, int TQ, int ib, int Ep) {
     auto al = [](int v) { return (v + 15) & ~15; };
     const int E = W + TQ;
     ReadLay L{};
     int o = 0;
     L.q = o;    o += al(HC * TQ * N * 4);     // queries as fp32   [HC or 1][TQ][N]
     L.x = o;    o += al(HC * E * P * ib);     // entries           [HC][E][P] raw
-    L.coef = o; o += al(HC * TQ * E * 4);     // coefficients      [HC][TQ][E]
+    L.coef = o; o += al(HC * TQ * Ep * 4);    // coefficients      [HC][TQmax][Ep]
     L.dec = o;  o += al(HC * TQ * 4);         // decays            [HC][TQ]
     L.dot = o;  o += al(HC * P * TQ * 4);     // S^ . Q per row    [HC*P][TQ]
     L.scale = o; o += al(HC * P * 4);         // fp8 row scales    [HC*P]
@@ -63,7 +63,7 @@ __host__ __device__ inline ReadLay read_lay(int HC, int P, int N, int W, int TQ,
     return L;
 }
 
-template <int N, int RK, int TQ>
+template <int N, int RK, int TQ, bool BF>
 __global__ void __launch_bounds__(kThreads, TQ == 1 ? 4 : 2) replay_read_kernel(const ReadArgs a) {
     constexpr int EPC = Chunk<RK>::EPC;   // stored elements per 16-byte chunk
     constexpr int TPR = N / EPC;          // chunks per state row
@@ -73,16 +73,16 @@ __global__ void __launch_bounds__(kThreads, TQ == 1 ? 4 : 2) replay_read_kernel(
     constexpr int RPP = kThreads / LPR;     // rows per pass
     constexpr int MAXC = 8;                 // chunks in flight per thread
     constexpr int PPR = MAXC / CPL > 0 ? MAXC / CPL : 1;  // passes per round
+    constexpr int IB = BF ? 2 : 4;
     static_assert(CPL <= MAXC, "a lane's chunks of one row must fit a round");
 
     extern __shared__ __align__(16) uint8_t smraw[];
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int H = a.H, P = a.P, R = a.R, W = a.W, T = a.T, HC = a.HC;
     const int b = blockIdx.x / (H / HC);
     const int h0 = (blockIdx.x - b * (H / HC)) * HC;
-    const int bf = a.in_bf16, ib = bf ? 2 : 4;
-    const int E = W + TQ;
-    const ReadLay Ly = read_lay(HC, P, N, W, TQ, ib);
+    const int E = W + TQ, Ep = a.Emax;
+    const ReadLay Ly = read_lay(HC, P, N, W, TQ, IB, Ep);
     float *sq = reinterpret_cast<float *>(smraw + Ly.q);
     uint8_t *sx = smraw + Ly.x;
     float *scoef = reinterpret_cast<float *>(smraw + Ly.coef);
@@ -94,6 +94,7 @@ __global__ void __launch_bounds__(kThreads, TQ == 1 ? 4 : 2) replay_read_kernel(
     const int nrows = HC * P;
     const uint8_t *tile = reinterpret_cast<const uint8_t *>(a.rc) + row0 * P * N * RCB;
     const int q = tid % LPR, rrow = tid / LPR;
+    const int xrow = P * IB, xch = xrow / 16;
 
     // 1. First round of read-copy chunks.
     uint4 rv[MAXC];
@@ -108,24 +109,27 @@ __global__ void __launch_bounds__(kThreads, TQ == 1 ? 4 : 2) replay_read_kernel(
     };
     issue(0);
 
-    // 2. Per-sequence info, coefficients, decays, the call's own entries.
+    // 2. Small operands: per-sequence info, the call's entries, decays, the
+    //    coefficient rows of the CTA's heads (contiguous), queries, fp8 scales.
     if (tid == 0) {
         const int4 si = a.seqinfo[b];
         sinfo[0] = si.x; sinfo[1] = si.y; sinfo[2] = si.z;
     }
-    const int xrow = P * ib, xch = xrow / 16;
-    for (int i = tid; i < T * HC * xch; i += kThreads) {
-        const int m = i / (HC * xch), r2 = i - m * HC * xch;
-        const int hh = r2 / xch, k = r2 - hh * xch;
-        cp_async16(sx + (hh * E + W + m) * xrow + k * 16,
-                   reinterpret_cast<const uint8_t *>(a.xnew) + (((int64_t)(b * T + m) * H + h0 + hh) * P) * ib + k * 16);
+    for (int row = warp; row < T * HC; row += kWarps) {  // x of token m, head hh
+        const int m = row / HC, hh = row - m * HC;
+        const uint8_t *src = reinterpret_cast<const uint8_t *>(a.xnew) + (((int64_t)(b * T + m) * H + h0 + hh) * P) * IB;
+        for (int k = lane; k < xch; k += 32) cp_async16(sx + (hh * E + W + m) * xrow + k * 16, src + k * 16);
+    }
+    {
+        const float *src = a.coef + row0 * a.TQmax * Ep;  // [HC][TQmax][Ep], contiguous
+        for (int i = tid; i < HC * a.TQmax * Ep / 4; i += kThreads) cp_async16(scoef + 4 * i, src + 4 * i);
     }
     for (int i = tid; i < HC * T; i += kThreads) {
         const int hh = i / T, m = i - hh * T;
         sdec[hh * TQ + m] = a.dec[(row0 + hh) * a.TQmax + m];
     }
-    // queries: one row for the CTA when its heads share a query row (Mamba-2 groups),
-    // else one per head
+    // queries: one row for the CTA when its heads share a query row (Mamba-2
+    // groups), else one per head
     const bool shared_q = (h0 / a.q_group) == ((h0 + HC - 1) / a.q_group);
     const int nq = shared_q ? 1 : HC;
     for (int i = tid; i < nq * T * N; i += kThreads) {
@@ -145,17 +149,14 @@ __global__ void __launch_bounds__(kThreads, TQ == 1 ? 4 : 2) replay_read_kernel(
         return;
     }
     const int base = W - L0;
-    for (int i = tid; i < HC * T * (L0 + T); i += kThreads) {
-        const int hh = i / (T * (L0 + T)), r2 = i - hh * T * (L0 + T);
-        const int m = r2 / (L0 + T), e = r2 - m * (L0 + T);
-        scoef[(hh * TQ + m) * E + e] = (e <= L0 + m) ? a.coef[((row0 + hh) * a.TQmax + m) * a.Emax + e] : 0.f;
-    }
-    for (int i = tid; i < HC * L0 * xch; i += kThreads) {
-        const int hh = i / (L0 * xch), r2 = i - hh * L0 * xch;
-        const int e = r2 / xch, k = r2 - e * xch;
-        const int slot = (ckmod + e) % R;
-        cp_async16(sx + (hh * E + base + e) * xrow + k * 16,
-                   reinterpret_cast<const uint8_t *>(a.xring) + (((row0 + hh) * R + slot) * P) * ib + k * 16);
+    const int n1 = min(L0, R - ckmod);  // buffered entries before the ring wraps
+    for (int row = warp; row < 2 * HC; row += kWarps) {  // two contiguous runs of slots per head
+        const int hh = row >> 1, second = row & 1;
+        const int cnt = second ? L0 - n1 : n1;
+        const uint8_t *src = reinterpret_cast<const uint8_t *>(a.xring) +
+                             (((row0 + hh) * R + (second ? 0 : ckmod)) * P) * IB;
+        uint8_t *dst = sx + (hh * E + base + (second ? n1 : 0)) * xrow;
+        for (int k = lane; k < cnt * xch; k += 32) cp_async16(dst + k * 16, src + k * 16);
     }
 
     // 3. Rows dotted with their query.
@@ -207,14 +208,23 @@ __global__ void __launch_bounds__(kThreads, TQ == 1 ? 4 : 2) replay_read_kernel(
     __syncthreads();
 
     // 4. y = dec * (S^ . Q) + replay term (+ D x).
-    for (int i = tid; i < T * HC * P; i += kThreads) {
-        const int m = i / (HC * P), r2 = i - m * HC * P;
+    for (int i = tid; i < T * nrows; i += kThreads) {
+        const int m = i / nrows, r2 = i - m * nrows;
         const int hh = r2 / P, p = r2 - hh * P;
-        float yv = sdec[hh * TQ + m] * sdot[(hh * P + p) * TQ + m];
-        const float *cf = scoef + (hh * TQ + m) * E;
-        const uint8_t *xs = sx + (hh * E + base) * xrow;
-        for (int e = 0; e <= L0 + m; ++e) yv = fmaf(cf[e], raw_f(xs + e * xrow, p, bf), yv);
-        if (a.D) yv = fmaf(a.D[h0 + hh], raw_f(sx + (hh * E + W + m) * xrow, p, bf), yv);
+        float yv = sdec[hh * TQ + m] * sdot[r2 * TQ + m];
+        const float *cf = scoef + (hh * a.TQmax + m) * Ep;
+        const uint8_t *xs = sx + (hh * E + base) * xrow + p * IB;
+        for (int e = 0; e <= L0 + m; ++e) {
+            const float xv = BF ? bf16_bits_to_float(*reinterpret_cast<const uint16_t *>(xs + e * xrow))
+                                : *reinterpret_cast<const float *>(xs + e * xrow);
+            yv = fmaf(cf[e], xv, yv);
+        }
+        if (a.D) {
+            const uint8_t *xn = sx + (hh * E + W + m) * xrow + p * IB;
+            const float xv = BF ? bf16_bits_to_float(*reinterpret_cast<const uint16_t *>(xn))
+                                : *reinterpret_cast<const float *>(xn);
+            yv = fmaf(a.D[h0 + hh], xv, yv);
+        }
         a.y[((int64_t)(b * T + m) * H + h0 + hh) * P + p] = yv;
     }
 }
@@ -223,7 +233,7 @@ __global__ void __launch_bounds__(kThreads, TQ == 1 ? 4 : 2) replay_read_kernel(
 // dstate is compiled in its own translation unit, rssm_read_n*.cu).
 template <int N, int RK, int TQ>
 inline cudaError_t launch_read_t(const ReadArgs &r, size_t smem, cudaStream_t st) {
-    auto k = replay_read_kernel<N, RK, TQ>;
+    auto k = r.in_bf16 ? replay_read_kernel<N, RK, TQ, true> : replay_read_kernel<N, RK, TQ, false>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     k<<<r.B * (r.H / r.HC), kThreads, smem, st>>>(r);

@@ -124,7 +124,7 @@ typedef struct {
     size_t tq_max;                       /* max(max_draft, 1): queries per call            */
     size_t seqinfo_off, seqinfo_bytes;   /* int32[B][4]                                    */
     size_t dec_off, dec_bytes;           /* fp32[B][H][tq_max]                             */
-    size_t coef_off, coef_bytes;         /* fp32[B][H][tq_max][window + tq_max]            */
+    size_t coef_off, coef_bytes;         /* fp32[B][H][tq_max][window + tq_max, padded to 4] */
     size_t query_off, query_bytes;       /* GDN: fp32[B][H][tq_max][dstate] swept queries  */
     size_t total_bytes;
 } rssm_workspace_layout;
