@@ -16,7 +16,7 @@ static int tq_of(int T) { return T <= 1 ? 1 : (T <= 4 ? 4 : 8); }
 static int m2_prep_heads(const rssm_config &cf, int TQ) {
     const int hpg = cf.nheads / cf.ngroups, ib = cf.input_dtype == RSSM_BF16 ? 2 : 4;
     for (int hc = 8; hc > 1; --hc)
-        if (hpg % hc == 0 && m2_prep_lay(hc, cf.headdim, cf.dstate, cf.window, TQ, ib).bytes <= 160 * 1024)
+        if (hpg % hc == 0 && m2_prep_lay(hc, cf.headdim, cf.dstate, cf.window, TQ, ib).bytes <= 150 * 1024)
             return hc;
     return 1;
 }
@@ -37,6 +37,8 @@ cudaError_t mamba2_launch(const Ctx &h, int op, int T, const rssm_inputs *in, fl
     a.R = (int)h.lay.ring; a.Rs = (int)h.lay.ring_stride; a.T = T; a.op = op; a.in_bf16 = cf.input_dtype == RSSM_BF16;
     a.dt_scales = cf.dt_scales_input;
     a.HC = m2_prep_heads(cf, tq_of(T));
+    a.cpg = (cf.nheads / cf.ngroups) / a.HC;
+    a.lay = m2_prep_lay(a.HC, cf.headdim, cf.dstate, cf.window, tq_of(T), cf.input_dtype == RSSM_BF16 ? 2 : 4);
     if (h.lay.seqinfo_bytes) {
         a.seqinfo = (int4 *)h.at(h.lay.seqinfo_off);
         a.dec = (float *)h.at(h.lay.dec_off);

@@ -5,54 +5,23 @@
 // Replay representation (ReplaySSM: the output comes from a checkpoint plus a
 // buffer of recent inputs with no state write; the checkpoint is rewritten only
 // when the buffer is full -- blog.thibaultmonteiro.fr, "Tenir le journal plutot
-// que le solde").  With buffered entries 1..L (L counts the token being read)
-// and prefix sums Lam_m = sum_{j<=m} dt_j A_h of the log decays:
-//   y = e^{Lam_L} (S^ C) + sum_i e^{Lam_L - Lam_i} (B_i . C) s_i x_i + D x_L
-//   fold: S_c <- e^{Lam_L} S_c + sum_i e^{Lam_L - Lam_i} s_i x_i B_i^T
+// que le solde").  With buffered entries e = 0..L-1 (the last being the token
+// read) and prefix sums Lam_e = sum_{j<=e} dt_j A_h of the log decays:
+//   y = e^{Lam_{L-1}} (S^ C) + sum_e e^{Lam_{L-1} - Lam_e} (B_e . C) s_e x_e + D x_{L-1}
+//   fold: S_c <- e^{Lam_{L-1}} S_c + sum_e e^{Lam_{L-1} - Lam_e} s_e x_e B_e^T
 // S^ is the read copy (bf16, per-row-scaled e4m3, or the fp32 checkpoint).
 //
-// One CTA per (b, h).  The replay kernel issues its read-copy loads (128-bit,
-// L1 no-allocate) before anything else, reads the sequence counters, stages the
-// buffered inputs in shared memory, and then either
-//   * reads: dot products of every state row with C (and the K draft C's),
-//     reduced with warp shuffles, or
-//   * folds (the buffer is full): loads the fp32 checkpoint, applies the rank-L
-//     update, stores fp32 + requantised copy, and reads the outputs from the
-//     fresh copy -- so a flush never needs a second pass over the state.
-// Then it writes y, appends the new tokens to the ring, and the last CTA of the
-// sequence publishes the counters.
+// A replay decode/verify runs this file's prep/flush kernel, which turns the
+// buffer into per-head replay coefficients (and folds when the buffer is full),
+// then the shared replay-read kernel (rssm_read.cuh).  The eager baseline below
+// rewrites the whole state every token.
 #pragma once
 #include "rssm_device.cuh"
 #include "rssm_internal.h"
+#include "rssm_pipe.cuh"
 #include "rssm_read.cuh"
 
 namespace rssm {
-
-struct M2Args {
-    int B, H, P, G, W, R, Rs, T, op, in_bf16, dt_scales;  // Rs: dt ring row length
-    int HC;             // heads per prep CTA (divides H / G)
-    int4 *seqinfo;      // per sequence, for the read kernel: {L0, ring slot of entry 0, folded, 0}
-    float *dec;         // [B][H][TQmax] decay of S^ C
-    float *coef;        // [B][H][TQmax][Emax] replay coefficients
-    int TQmax, Emax;    // Emax: padded row length of the coefficient table
-    Counters c;
-    const float *A, *D;
-    float *ckpt;        // fp32 [B][H][P][N]
-    void *rc;           // read copy / low-precision state [B][H][P][N]
-    float *rc_scale;    // [B][H][P] (FP8)
-    void *xbuf;         // [B][H][R][P]
-    float *dtbuf;       // [B][H][R]
-    void *Bbuf;         // [B][G][R][N]
-    void *snap;         // eager verify snapshots
-    float *snap_scale;
-    const void *x;      // [B][T][H][P]
-    const float *dt;    // [B][T][H]
-    const void *Bm;     // [B][T][G][N]
-    const void *Cm;     // [B][T][G][N]
-    const int32_t *accept;  // [B] (commit)
-    float *y;           // [B][T][H][P]
-    float *out;         // export target [B][H][P][N]
-};
 
 __host__ __device__ constexpr int a16(int v) { return (v + 15) & ~15; }
 __host__ __device__ constexpr int pad4(int n) { return (n + 3) & ~3; }
@@ -61,18 +30,21 @@ __host__ __device__ constexpr int pad4(int n) { return (n + 3) & ~3; }
 // slots, rows padded to 4 floats.
 __host__ __device__ constexpr int dt_row_max_bytes(int W) { return ((W + 8 + 3) & ~3) * 4; }
 
-// Shared memory of the prep kernel (bytes, 16-byte aligned regions).  Entry
-// slots of x: E = W + TQ; committed entries sit right-aligned before slot W and
-// the call's own tokens at W..W+T-1, so logical entry e is slot (W - L0) + e.
-// The group's B ring is staged whole (R <= W + 8 rows), with no wait for the
-// counters.
+constexpr int kFoldChunk = 16 * 1024;  // bytes of fp32 checkpoint rows per fold stage
+
+// Shared memory of the prep kernel (bytes, 16-byte aligned regions), computed on
+// the host.  Entry slots of x: E = W + TQ; committed entries sit right-aligned
+// before slot W and the call's own tokens at W..W+T-1, so logical entry e is
+// slot (W - L0) + e.  The group's B ring is staged whole (R <= W + 8 rows).
 struct M2PrepLay {
-    int sC, sBr, sBn, sx, dring, dtn, sd, slam, scoef, sdec, su, sfdec, sCf, sdot, si, bytes;
+    int fold, bar, sC, sBr, sBn, sx, dring, dtn, sd, slam, scoef, sdec, su, sfdec, sCf, sdot, si, bytes;
 };
-__host__ __device__ inline M2PrepLay m2_prep_lay(int HC, int P, int N, int W, int TQ, int ib) {
+inline M2PrepLay m2_prep_lay(int HC, int P, int N, int W, int TQ, int ib) {
     const int E = W + TQ;
     M2PrepLay L{};
     int o = 0;
+    L.fold = o;  o += 2 * kFoldChunk;            // fp32 checkpoint rows, two stages
+    L.bar = o;   o += 16;                        // their mbarriers
     L.sC = o;    o += a16(TQ * N * ib);          // raw C of the queries     [TQ][N]
     L.sBr = o;   o += a16((W + 8) * N * ib);     // raw B ring of the group  [R][N]
     L.sBn = o;   o += a16(TQ * N * ib);          // raw B of the call's tokens [TQ][N]
@@ -92,40 +64,71 @@ __host__ __device__ inline M2PrepLay m2_prep_lay(int HC, int P, int N, int W, in
     return L;
 }
 
+struct M2Args {
+    int B, H, P, G, W, R, Rs, T, op, in_bf16, dt_scales;  // Rs: dt ring row length
+    int HC, cpg;        // heads per prep CTA (divides H / G); prep CTAs per group
+    M2PrepLay lay;      // prep kernel shared memory
+    int4 *seqinfo;      // per sequence, for the read kernel: {L0, ring slot of entry 0, folded, 0}
+    float *dec;         // [B][H][TQmax] decay of S^ C
+    float *coef;        // [B][H][TQmax][Emax] replay coefficients
+    int TQmax, Emax;    // Emax: padded row length of the coefficient table
+    Counters c;
+    const float *A, *D;
+    float *ckpt;        // fp32 [B][H][P][N]
+    void *rc;           // read copy / low-precision state [B][H][P][N]
+    float *rc_scale;    // [B][H][P] (FP8)
+    void *xbuf;         // [B][H][R][P]
+    float *dtbuf;       // [B][H][Rs]
+    void *Bbuf;         // [B][G][R][N]
+    void *snap;         // eager verify snapshots
+    float *snap_scale;
+    const void *x;      // [B][T][H][P]
+    const float *dt;    // [B][T][H]
+    const void *Bm;     // [B][T][G][N]
+    const void *Cm;     // [B][T][G][N]
+    float *y;           // [B][T][H][P]
+    float *out;         // export target [B][H][P][N]
+};
+
 // ---------------------------------------------------------------------------
 // Prep / flush kernel: decode (T = 1), verify (T = K), flush and export (T = 0).
 //
-// One CTA per (sequence b, group g, chunk of HC heads of the group).  In one
-// round trip it reads the sequence's counters and stages the group's whole B
-// ring, the heads' dt ring rows and the call's tokens; it computes once per
-// group B_e . C_m and per head the prefix sums Lam of dt*A.  Then either
-//   * (no fold) it writes the replay coefficients
-//       coef[e] = e^{Lam_{L0+m} - Lam_e} (B_e . C_m) s_e,   dec = e^{Lam_{L0+m}}
-//     for the read kernel, or
-//   * (fold: len + T > W, or flush/export) it folds the committed entries into
-//     the fp32 checkpoint, S_c <- e^{Lam_L} S_c + sum_e e^{Lam_L - Lam_e} s_e x_e B_e^T,
-//     stores it with the requantised read copy (or writes it out, for export),
-//     and, for decode/verify, computes the outputs from the fresh copy itself.
-// Last it appends the call's tokens to the ring; the last CTA of the sequence
-// publishes the counters.
+// One CTA per (group chunk of HC heads, sequence b).  In one round trip it reads
+// the sequence's counters and stages the group's whole B ring, the heads' dt
+// ring rows and the call's tokens; then B_e . C_m once for the group and, per
+// head (one warp each), the prefix sums Lam of dt*A and the coefficients.
+//   * no fold: the replay coefficients
+//       coef[m][e] = e^{Lam_{L0+m} - Lam_e} (B_e . C_m) s_e,   dec[m] = e^{Lam_{L0+m}}
+//     go to the read kernel;
+//   * fold (len + T > W, or flush/export): the committed entries are folded into
+//     the fp32 checkpoint, S_c <- e^{Lam_{L0-1}} S_c + sum_e e^{Lam_{L0-1} - Lam_e} s_e x_e B_e^T.
+//     Thread 0 starts bulk copies of the checkpoint rows (16 KiB stages, two in
+//     flight) as soon as it has read the counters; the CTA stores the result
+//     with the requantised read copy (or writes it out, for export) and, for
+//     decode/verify, computes the outputs from the fresh copy itself.
+// Last it appends the call's tokens to the ring, and thread 0 registers the
+// CTA's arrival; the last CTA of the sequence publishes the counters.
 // ---------------------------------------------------------------------------
 template <int N, int RK, int TQ, bool BF>
 __global__ void __launch_bounds__(kThreads, 3) m2_prep_kernel(const M2Args a) {
-    constexpr int TPR4 = N / 4;  // lanes per row, fp32 quad mapping
+    constexpr int TPR4 = N / 4;           // lanes per row, fp32 quad mapping
     constexpr int RPP4 = kThreads / TPR4;
-    constexpr int FH = 2;        // fold rows held in registers per thread
-    constexpr int FB = 4;        // buffered B entries held in registers per block
+    constexpr int FC = kFoldChunk / (N * 4);  // fp32 rows per fold stage
+    constexpr int FH = FC / RPP4;         // rows per thread per stage (= 4)
+    constexpr int FB = 4;                 // buffered B entries held in registers per block
     constexpr int IB = BF ? 2 : 4;
-    extern __shared__ __align__(16) uint8_t smraw[];
+    static_assert(FH * RPP4 == FC, "fold stage is FH rows per thread");
+    extern __shared__ __align__(128) uint8_t smraw[];
+    const M2PrepLay &Ly = a.lay;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int H = a.H, P = a.P, W = a.W, R = a.R, T = a.T, G = a.G, HC = a.HC;
-    const int hpg = H / G, cpg = hpg / HC;
-    const int b = blockIdx.x / (G * cpg);
-    const int rem = blockIdx.x - b * G * cpg;
-    const int g = rem / cpg, hc = rem - g * cpg;
+    const int hpg = H / G;
+    const int b = blockIdx.y;
+    const int g = blockIdx.x / a.cpg, hc = blockIdx.x - g * a.cpg;
     const int h0 = g * hpg + hc * HC;
     const int E = W + TQ;
-    const M2PrepLay Ly = m2_prep_lay(HC, P, N, W, TQ, IB);
+    float *fbuf = reinterpret_cast<float *>(smraw + Ly.fold);
+    uint64_t *fbar = reinterpret_cast<uint64_t *>(smraw + Ly.bar);
     uint8_t *sC = smraw + Ly.sC, *sBr = smraw + Ly.sBr, *sBn = smraw + Ly.sBn, *sx = smraw + Ly.sx;
     float *dring = reinterpret_cast<float *>(smraw + Ly.dring);
     float *dtn = reinterpret_cast<float *>(smraw + Ly.dtn);
@@ -141,16 +144,25 @@ __global__ void __launch_bounds__(kThreads, 3) m2_prep_kernel(const M2Args a) {
     const int64_t row0 = (int64_t)b * H + h0;
     const int64_t tile0 = row0 * P * N;
     const int nrows = HC * P;
+    const int nfc = (nrows + FC - 1) / FC;  // fold stages
     const bool reads = (a.op == OP_DECODE || a.op == OP_VERIFY);
     const int xrow = P * IB, brow = N * IB, xch = xrow / 16, bch = brow / 16;
     const int Rs = a.Rs;
     auto ldx = [](const uint8_t *p) -> float {
         return BF ? bf16_bits_to_float(*reinterpret_cast<const uint16_t *>(p)) : *reinterpret_cast<const float *>(p);
     };
+    auto fold_issue = [&](int c) {  // thread 0: stage c of the checkpoint rows into buffer c & 1
+        const int r0 = c * FC, r1 = min(nrows, r0 + FC);
+        const uint32_t bytes = (uint32_t)((r1 - r0) * N * 4);
+        mbar_arrive_expect_tx(&fbar[c & 1], bytes);
+        bulk_g2s(fbuf + (c & 1) * (FC * N), a.ckpt + tile0 + (int64_t)r0 * N, bytes, &fbar[c & 1]);
+    };
 
-    // 1. Counters (thread 0); everything that does not depend on them, at once.
+    // 1. Counters (thread 0; starts the fold's checkpoint copies when one is due)
+    //    and everything that does not depend on them, at once.
+    SeqState ss{};
     if (tid == 0) {
-        SeqState ss = read_counters(a.c, b, W);
+        ss = read_counters(a.c, b, W);
         const int L0 = (int)(ss.seq - ss.ckpt);
         int flush = 0;
         if (ss.ok) flush = (a.op == OP_FLUSH || a.op == OP_EXPORT) ? (L0 > 0) : (L0 + T > W);
@@ -159,14 +171,18 @@ __global__ void __launch_bounds__(kThreads, 3) m2_prep_kernel(const M2Args a) {
         si[2] = flush;
         si[3] = (int)(ss.ckpt % R);
         si[4] = (int)(ss.seq % R);
+        if (flush) {
+            mbar_init(&fbar[0], 1);
+            mbar_init(&fbar[1], 1);
+            mbar_init_fence();
+            fold_issue(0);
+            if (nfc > 1) fold_issue(1);
+        }
         if (!ss.ok) {
-            if (g == 0 && hc == 0) report(a.c.err, DEV_BAD_COUNTERS, b, h0, L0);
-            if (reads && g == 0 && hc == 0) a.seqinfo[b] = make_int4(0, 0, 1, 0);  // nothing to read
-        } else {
-            if (reads && g == 0 && hc == 0) a.seqinfo[b] = make_int4(flush ? 0 : L0, (int)(ss.ckpt % R), flush, 0);
-            if (a.op != OP_EXPORT)
-                arrive_and_publish(a.c, b, G * cpg, (a.op == OP_DECODE) ? ss.seq + 1 : -1,
-                                   flush ? ss.seq : -1, (a.op == OP_VERIFY) ? T : -1, flush);
+            if (blockIdx.x == 0) report(a.c.err, DEV_BAD_COUNTERS, b, h0, L0);
+            if (reads && blockIdx.x == 0) a.seqinfo[b] = make_int4(0, 0, 1, 0);  // nothing to read
+        } else if (reads && blockIdx.x == 0) {
+            a.seqinfo[b] = make_int4(flush ? 0 : L0, (int)(ss.ckpt % R), flush, 0);
         }
     }
     {
@@ -192,15 +208,16 @@ __global__ void __launch_bounds__(kThreads, 3) m2_prep_kernel(const M2Args a) {
     }
     cp_async_wait_all();
     __syncthreads();
-    if (!si[0]) return;
+    if (!si[0]) return;  // counters corrupted: reported, sequence skipped, no arrival
     const int L0 = si[1], flush = si[2], ckmod = si[3], spmod = si[4];
     const int base = W - L0, nE = L0 + T;
     const int e0 = flush ? L0 : 0;  // first entry the outputs replay
+    auto slot_of = [&](int e) { const int s = ckmod + e; return s >= R ? s - R : s; };
     auto B_of = [&](int e) -> const uint8_t * {  // B of logical entry e
-        return e < L0 ? sBr + ((ckmod + e) % R) * brow : sBn + (e - L0) * brow;
+        return e < L0 ? sBr + slot_of(e) * brow : sBn + (e - L0) * brow;
     };
     auto dt_of = [&](int hh, int e) -> float {
-        return e < L0 ? dring[hh * Rs + (ckmod + e) % R] : dtn[(e - L0) * HC + hh];
+        return e < L0 ? dring[hh * Rs + slot_of(e)] : dtn[(e - L0) * HC + hh];
     };
     if (flush) {  // the heads' buffered x, needed only to fold
         const int n1 = min(L0, R - ckmod);
@@ -214,81 +231,82 @@ __global__ void __launch_bounds__(kThreads, 3) m2_prep_kernel(const M2Args a) {
         }
     }
 
-    // 2. B_e . C_m once for the group, C as fp32, prefix sums of dt*A per head.
+    // 2. B_e . C_m once for the group (warps), C as fp32.
     if (reads) {
         for (int pr = warp; pr < T * nE; pr += kWarps) {
             const int m = pr / nE, e = pr - m * nE;
-            if (e > L0 + m) continue;  // warp-uniform
-            const uint8_t *Bp = B_of(e);
+            if (e > L0 + m || e < e0) continue;  // warp-uniform
+            const uint8_t *Bp = B_of(e), *Cp = sC + m * brow;
             float d = 0.f;
-            for (int n = lane; n < N; n += 32) d = fmaf(ldx(Bp + n * IB), ldx(sC + m * brow + n * IB), d);
+            for (int n = lane; n < N; n += 32) d = fmaf(ldx(Bp + n * IB), ldx(Cp + n * IB), d);
             d = group_sum<32>(d);
             if (lane == 0) sd[m * E + e] = d;
         }
         for (int i = tid; i < T * N; i += kThreads) sCf[i] = ldx(sC + i * IB);
     }
+    __syncthreads();
+
+    // 3. Per head (one warp): prefix sums of dt*A, coefficients, decays.
     for (int hh = warp; hh < HC; hh += kWarps) {
         const float Ah = a.A[h0 + hh];
+        float *lam = slam + hh * E + base;
         float carry = 0.f;
         for (int k0 = 0; k0 < nE; k0 += 32) {
             const int e = k0 + lane;
             float v = (e < nE) ? dt_of(hh, e) * Ah : 0.f;
             v = warp_incl_scan(v) + carry;
-            if (e < nE) slam[hh * E + base + e] = v;
+            if (e < nE) lam[e] = v;
             carry = __shfl_sync(0xffffffffu, v, 31);
         }
-    }
-    __syncthreads();
-
-    // 3. Replay coefficients and decays (to the read kernel, or kept here to fold).
-    for (int i = tid; i < HC * nE; i += kThreads) {
-        const int hh = i / nE, e = i - hh * nE;
-        const float *lam = slam + hh * E + base;
-        const float se = a.dt_scales ? dt_of(hh, e) : 1.f;
-        if (reads) {
+        __syncwarp();
+        const float lam_f = (flush && L0 > 0) ? lam[L0 - 1] : 0.f;
+        for (int e = lane; e < nE; e += 32) {
+            const float se = a.dt_scales ? dt_of(hh, e) : 1.f;
+            if (reads) {
 #pragma unroll
-            for (int m = 0; m < TQ; ++m) {
-                if (m >= T || e > L0 + m) continue;
-                const float cf = expf(lam[L0 + m] - lam[e]) * sd[m * E + e] * se;
-                if (flush) {
-                    if (e >= e0) scoef[(hh * TQ + m) * E + e] = cf;
-                } else {
-                    a.coef[((row0 + hh) * a.TQmax + m) * a.Emax + e] = cf;
+                for (int m = 0; m < TQ; ++m) {
+                    if (m >= T || e > L0 + m || e < e0) continue;
+                    const float cf = expf(lam[L0 + m] - lam[e]) * sd[m * E + e] * se;
+                    if (flush) scoef[(hh * TQ + m) * E + e] = cf;
+                    else a.coef[((row0 + hh) * a.TQmax + m) * a.Emax + e] = cf;
                 }
             }
+            if (flush && e < L0) su[hh * E + e] = expf(lam_f - lam[e]) * se;
         }
-        if (flush && e < L0) su[hh * E + e] = expf(lam[L0 - 1] - lam[e]) * se;
-    }
-    for (int i = tid; i < HC; i += kThreads) {
-        const float *lam = slam + i * E + base;
-        sfdec[i] = flush ? expf(lam[L0 - 1]) : 1.f;
-        if (reads) {
-#pragma unroll
-            for (int m = 0; m < TQ; ++m) {
-                if (m >= T) continue;
-                const float dcy = expf(lam[L0 + m] - (flush ? lam[L0 - 1] : 0.f));
-                if (flush) sdec[i * TQ + m] = dcy;
-                else a.dec[(row0 + i) * a.TQmax + m] = dcy;
-            }
+        if (lane == 0) sfdec[hh] = flush ? expf(lam_f) : 1.f;
+        if (reads && lane < T) {
+            const float dcy = expf(lam[L0 + lane] - lam_f);
+            if (flush) sdec[hh * TQ + lane] = dcy;
+            else a.dec[(row0 + hh) * a.TQmax + lane] = dcy;
         }
     }
+
     if (flush) {
         cp_async_wait_all();
         __syncthreads();
-        // 4. Fold the committed entries into the fp32 checkpoint rows of the HC
-        //    heads (FH rows per thread in registers, FB buffered B entries at a
-        //    time), store the checkpoint and the requantised copy, and dot the
-        //    fresh copy with C.
+        // 4. Fold, one staged 16 KiB block of checkpoint rows at a time (the next
+        //    one in flight): FH rows per thread, FB buffered B entries per block
+        //    in registers; store the checkpoint and the requantised copy, and dot
+        //    the fresh copy with C.
         const int c4 = tid % TPR4, q0 = tid / TPR4;
-        for (int rb = 0; rb < nrows; rb += FH * RPP4) {  // same trip count for every lane
+        bool timed_out = false;
+        for (int c = 0; c < nfc; ++c) {
+            const bool got = mbar_wait(&fbar[c & 1], (c >> 1) & 1);
+            if (__syncthreads_or(!got)) {
+                timed_out = true;
+                break;
+            }
+            const float *tf = fbuf + (c & 1) * (FC * N);
             float4 v[FH];
+            int gr[FH];
 #pragma unroll
             for (int k = 0; k < FH; ++k) {
-                const int gr = rb + q0 + k * RPP4;
+                const int rl = q0 + k * RPP4;
+                gr[k] = c * FC + rl;
                 v[k] = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (gr < nrows) {
-                    v[k] = load_quad<SK_F32>(a.ckpt, tile0 + (int64_t)gr * N + 4 * c4);
-                    const float dc = sfdec[gr / P];
+                if (gr[k] < nrows) {
+                    v[k] = *reinterpret_cast<const float4 *>(tf + rl * N + 4 * c4);
+                    const float dc = sfdec[gr[k] / P];
                     v[k].x *= dc; v[k].y *= dc; v[k].z *= dc; v[k].w *= dc;
                 }
             }
@@ -302,9 +320,8 @@ __global__ void __launch_bounds__(kThreads, 3) m2_prep_kernel(const M2Args a) {
                 }
 #pragma unroll
                 for (int k = 0; k < FH; ++k) {
-                    const int gr = rb + q0 + k * RPP4;
-                    if (gr >= nrows) continue;
-                    const int hh = gr / P, p = gr - hh * P;
+                    if (gr[k] >= nrows) continue;
+                    const int hh = gr[k] / P, p = gr[k] - hh * P;
                     const uint8_t *xr = sx + (hh * E + base + eb) * xrow + p * IB;
                     const float *uw = su + hh * E + eb;
 #pragma unroll
@@ -317,11 +334,12 @@ __global__ void __launch_bounds__(kThreads, 3) m2_prep_kernel(const M2Args a) {
                     }
                 }
             }
+            __syncthreads();  // every thread has its rows of this stage in registers
+            if (tid == 0 && c + 2 < nfc) fold_issue(c + 2);
 #pragma unroll
             for (int k = 0; k < FH; ++k) {
-                const int gr = rb + q0 + k * RPP4;
-                const bool valid = gr < nrows;
-                const int64_t el = tile0 + (int64_t)(valid ? gr : 0) * N + 4 * c4;
+                const bool valid = gr[k] < nrows;
+                const int64_t el = tile0 + (int64_t)(valid ? gr[k] : 0) * N + 4 * c4;
                 if (a.op == OP_EXPORT) {
                     if (valid) *reinterpret_cast<float4 *>(a.out + el) = v[k];
                     continue;
@@ -336,7 +354,7 @@ __global__ void __launch_bounds__(kThreads, 3) m2_prep_kernel(const M2Args a) {
                     const float sc = fp8_scale(am);
                     if (valid) {
                         rd = store_quad<SK_FP8>(a.rc, el, v[k], 0.f, sc);
-                        if (c4 == 0) a.rc_scale[row0 * P + gr] = sc;
+                        if (c4 == 0) a.rc_scale[row0 * P + gr[k]] = sc;
                     }
                 }
                 if (reads) {
@@ -345,10 +363,14 @@ __global__ void __launch_bounds__(kThreads, 3) m2_prep_kernel(const M2Args a) {
                         const float4 Cq = *reinterpret_cast<const float4 *>(sCf + m * N + 4 * c4);
                         float d = rd.x * Cq.x + rd.y * Cq.y + rd.z * Cq.z + rd.w * Cq.w;
                         d = group_sum<TPR4>(d);
-                        if (c4 == 0 && valid && m < T) sdot[gr * TQ + m] = d;
+                        if (c4 == 0 && valid && m < T) sdot[gr[k] * TQ + m] = d;
                     }
                 }
             }
+        }
+        if (timed_out) {  // a checkpoint copy never landed: reported, sequence left as it was
+            if (tid == 0) report(a.c.err, DEV_PIPE_TIMEOUT, b, h0, 0);
+            return;
         }
         if (reads) {
             __syncthreads();
@@ -365,29 +387,36 @@ __global__ void __launch_bounds__(kThreads, 3) m2_prep_kernel(const M2Args a) {
             }
         }
     }
-    if (!reads) return;
 
     // 5. Append the call's tokens to the ring (slots seq_pos + m mod R).
-    for (int row = warp; row < T * HC; row += kWarps) {
-        const int m = row / HC, hh = row - m * HC;
-        const int slot = (spmod + m) % R;
-        uint8_t *dst = reinterpret_cast<uint8_t *>(a.xbuf) + (((row0 + hh) * R + slot) * P) * IB;
-        const uint8_t *src = sx + (hh * E + W + m) * xrow;
-        for (int k = lane; k < xch; k += 32)
-            *reinterpret_cast<uint4 *>(dst + k * 16) = *reinterpret_cast<const uint4 *>(src + k * 16);
-    }
-    for (int i = tid; i < T * HC; i += kThreads) {
-        const int m = i / HC, hh = i - m * HC;
-        a.dtbuf[(row0 + hh) * Rs + (spmod + m) % R] = dtn[m * HC + hh];
-    }
-    if (hc == 0) {  // the group's first chunk writes the group's B
-        for (int row = warp; row < T; row += kWarps) {
-            const int slot = (spmod + row) % R;
-            uint8_t *dst = reinterpret_cast<uint8_t *>(a.Bbuf) + (((int64_t)(b * G + g) * R + slot) * N) * IB;
-            for (int k = lane; k < bch; k += 32)
-                *reinterpret_cast<uint4 *>(dst + k * 16) = *reinterpret_cast<const uint4 *>(sBn + row * brow + k * 16);
+    if (reads) {
+        for (int row = warp; row < T * HC; row += kWarps) {
+            const int m = row / HC, hh = row - m * HC;
+            const int slot = spmod + m >= R ? spmod + m - R : spmod + m;
+            uint8_t *dst = reinterpret_cast<uint8_t *>(a.xbuf) + (((row0 + hh) * R + slot) * P) * IB;
+            const uint8_t *src = sx + (hh * E + W + m) * xrow;
+            for (int k = lane; k < xch; k += 32)
+                *reinterpret_cast<uint4 *>(dst + k * 16) = *reinterpret_cast<const uint4 *>(src + k * 16);
+        }
+        for (int i = tid; i < T * HC; i += kThreads) {
+            const int m = i / HC, hh = i - m * HC;
+            const int slot = spmod + m >= R ? spmod + m - R : spmod + m;
+            a.dtbuf[(row0 + hh) * Rs + slot] = dtn[m * HC + hh];
+        }
+        if (hc == 0) {  // the group's first chunk writes the group's B
+            for (int row = warp; row < T; row += kWarps) {
+                const int slot = spmod + row >= R ? spmod + row - R : spmod + row;
+                uint8_t *dst = reinterpret_cast<uint8_t *>(a.Bbuf) + (((int64_t)(b * G + g) * R + slot) * N) * IB;
+                for (int k = lane; k < bch; k += 32)
+                    *reinterpret_cast<uint4 *>(dst + k * 16) = *reinterpret_cast<const uint4 *>(sBn + row * brow + k * 16);
+            }
         }
     }
+    // 6. This CTA read the counters long ago; its arrival lets the last CTA of the
+    //    sequence publish them.
+    if (tid == 0 && a.op != OP_EXPORT)
+        arrive_and_publish(a.c, b, G * a.cpg, (a.op == OP_DECODE) ? ss.seq + 1 : -1, flush ? ss.seq : -1,
+                           (a.op == OP_VERIFY) ? T : -1, flush);
 }
 
 // ---------------------------------------------------------------------------
@@ -509,7 +538,7 @@ inline cudaError_t launch_replay_t(const M2Args &a, size_t smem, cudaStream_t st
     auto k = a.in_bf16 ? m2_prep_kernel<N, RK, TQ, true> : m2_prep_kernel<N, RK, TQ, false>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    k<<<a.B * (a.H / a.HC), kThreads, smem, st>>>(a);
+    k<<<dim3(a.H / a.HC, a.B), kThreads, smem, st>>>(a);
     return cudaGetLastError();
 }
 

@@ -55,6 +55,7 @@ cudaError_t launch_read(const Ctx &h, int T, const void *Q, int q_bf16, int q_gr
     r.Emax = (cf.window + r.TQmax + 3) & ~3;
     r.y = y;
     const int TQ = tq_of_read(T);
+    r.lay = read_lay(r.HC, cf.headdim, cf.dstate, cf.window, TQ, cf.input_dtype == RSSM_BF16 ? 2 : 4, r.Emax);
     const size_t smem = read_smem_bytes(cf, T);
     switch (cf.dstate) {
         case 16: return read_dispatch_n<16>(cf.state_dtype, TQ, r, smem, st);

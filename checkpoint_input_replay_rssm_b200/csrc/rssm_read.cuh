@@ -23,6 +23,26 @@
 
 namespace rssm {
 
+// Shared memory of the read kernel (bytes, 16-byte aligned regions).
+struct ReadLay {
+    int q, x, coef, dec, dot, scale, info, bytes;
+};
+inline ReadLay read_lay(int HC, int P, int N, int W, int TQ, int ib, int Ep) {
+    auto al = [](int v) { return (v + 15) & ~15; };
+    const int E = W + TQ;
+    ReadLay L{};
+    int o = 0;
+    L.q = o;    o += al(HC * TQ * N * 4);     // queries as fp32   [HC or 1][TQ][N]
+    L.x = o;    o += al(HC * E * P * ib);     // entries           [HC][E][P] raw
+    L.coef = o; o += al(HC * TQ * Ep * 4);    // coefficients      [HC][TQmax][Ep]
+    L.dec = o;  o += al(HC * TQ * 4);         // decays            [HC][TQ]
+    L.dot = o;  o += al(HC * P * TQ * 4);     // S^ . Q per row    [HC*P][TQ]
+    L.scale = o; o += al(HC * P * 4);         // fp8 row scales    [HC*P]
+    L.info = o; o += 16;
+    L.bytes = o;
+    return L;
+}
+
 struct ReadArgs {
     int B, H, P, R, W, T, HC, in_bf16;
     int q_group;            // heads per query row (Mamba-2: H / G; GDN: 1)
@@ -40,28 +60,9 @@ struct ReadArgs {
     const float *dec;       // [B][H][TQmax]
     const float *coef;      // [B][H][TQmax][Emax]
     int TQmax, Emax;        // Emax: padded row length of the coefficient table
+    ReadLay lay;            // shared memory, computed on the host
     float *y;               // [B][T][H][P]
 };
-
-// Shared memory of the read kernel (bytes, 16-byte aligned regions).
-struct ReadLay {
-    int q, x, coef, dec, dot, scale, info, bytes;
-};
-__host__ __device__ inline ReadLay read_lay(int HC, int P, int N, int W, int TQ, int ib, int Ep) {
-    auto al = [](int v) { return (v + 15) & ~15; };
-    const int E = W + TQ;
-    ReadLay L{};
-    int o = 0;
-    L.q = o;    o += al(HC * TQ * N * 4);     // queries as fp32   [HC or 1][TQ][N]
-    L.x = o;    o += al(HC * E * P * ib);     // entries           [HC][E][P] raw
-    L.coef = o; o += al(HC * TQ * Ep * 4);    // coefficients      [HC][TQmax][Ep]
-    L.dec = o;  o += al(HC * TQ * 4);         // decays            [HC][TQ]
-    L.dot = o;  o += al(HC * P * TQ * 4);     // S^ . Q per row    [HC*P][TQ]
-    L.scale = o; o += al(HC * P * 4);         // fp8 row scales    [HC*P]
-    L.info = o; o += 16;
-    L.bytes = o;
-    return L;
-}
 
 template <int N, int RK, int TQ, bool BF>
 __global__ void __launch_bounds__(kThreads, TQ == 1 ? 4 : 2) replay_read_kernel(const ReadArgs a) {
@@ -79,10 +80,10 @@ __global__ void __launch_bounds__(kThreads, TQ == 1 ? 4 : 2) replay_read_kernel(
     extern __shared__ __align__(16) uint8_t smraw[];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int H = a.H, P = a.P, R = a.R, W = a.W, T = a.T, HC = a.HC;
-    const int b = blockIdx.x / (H / HC);
-    const int h0 = (blockIdx.x - b * (H / HC)) * HC;
+    const int b = blockIdx.y;
+    const int h0 = blockIdx.x * HC;
     const int E = W + TQ, Ep = a.Emax;
-    const ReadLay Ly = read_lay(HC, P, N, W, TQ, IB, Ep);
+    const ReadLay &Ly = a.lay;
     float *sq = reinterpret_cast<float *>(smraw + Ly.q);
     uint8_t *sx = smraw + Ly.x;
     float *scoef = reinterpret_cast<float *>(smraw + Ly.coef);
@@ -236,7 +237,7 @@ inline cudaError_t launch_read_t(const ReadArgs &r, size_t smem, cudaStream_t st
     auto k = r.in_bf16 ? replay_read_kernel<N, RK, TQ, true> : replay_read_kernel<N, RK, TQ, false>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    k<<<r.B * (r.H / r.HC), kThreads, smem, st>>>(r);
+    k<<<dim3(r.H / r.HC, r.B), kThreads, smem, st>>>(r);
     return cudaGetLastError();
 }
 
