@@ -47,7 +47,7 @@ size_t gdn_smem_bytes(const rssm_config &cf, int T);
 
 // The replay-read kernel (rssm_read.cu), shared by both kinds: queries Q[b][row][m][n]
 // at the given element strides, q_group heads per query row.
-cudaError_t launch_read(const Ctx &h, int T, const void *Q, int q_bf16, int q_group, int64_t q_stride_b,
+cudaError_t launch_read(const Ctx &h, int op, int T, const void *Q, int q_bf16, int q_group, int64_t q_stride_b,
                         int64_t q_stride_row, int64_t q_stride_m, const void *xnew, const float *D,
                         float *y, cudaStream_t st);
 int read_heads_per_cta(const rssm_config &cf);

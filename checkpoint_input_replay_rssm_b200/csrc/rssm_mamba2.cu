@@ -78,7 +78,7 @@ cudaError_t mamba2_launch(const Ctx &h, int op, int T, const rssm_inputs *in, fl
     }
     // replay read: C of the group ([B][T][G][N]) is the query, x the buffered entries
     const int G = cf.ngroups;
-    return launch_read(h, T, in->Cm, cf.input_dtype == RSSM_BF16, cf.nheads / G, (int64_t)T * G * cf.dstate,
+    return launch_read(h, op, T, in->Cm, cf.input_dtype == RSSM_BF16, cf.nheads / G, (int64_t)T * G * cf.dstate,
                        cf.dstate, (int64_t)G * cf.dstate, in->x, (const float *)h.at(h.lay.D_off), y, st);
 }
 

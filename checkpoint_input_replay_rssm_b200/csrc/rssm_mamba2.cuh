@@ -178,11 +178,14 @@ __global__ void __launch_bounds__(kThreads, 3) m2_prep_kernel(const M2Args a) {
             fold_issue(0);
             if (nfc > 1) fold_issue(1);
         }
+        // seqinfo: {ring entries the read kernel replays, ring slot of entry 0,
+        // folded here, counters valid} -- the read kernel also publishes the
+        // sequence's new counters from it
         if (!ss.ok) {
             if (blockIdx.x == 0) report(a.c.err, DEV_BAD_COUNTERS, b, h0, L0);
-            if (reads && blockIdx.x == 0) a.seqinfo[b] = make_int4(0, 0, 1, 0);  // nothing to read
+            if (reads && blockIdx.x == 0) a.seqinfo[b] = make_int4(0, 0, 1, 0);  // nothing to read or publish
         } else if (reads && blockIdx.x == 0) {
-            a.seqinfo[b] = make_int4(flush ? 0 : L0, (int)(ss.ckpt % R), flush, 0);
+            a.seqinfo[b] = make_int4(flush ? 0 : L0, (int)(ss.ckpt % R), flush, 1);
         }
     }
     {
@@ -412,11 +415,11 @@ __global__ void __launch_bounds__(kThreads, 3) m2_prep_kernel(const M2Args a) {
             }
         }
     }
-    // 6. This CTA read the counters long ago; its arrival lets the last CTA of the
-    //    sequence publish them.
-    if (tid == 0 && a.op != OP_EXPORT)
-        arrive_and_publish(a.c, b, G * a.cpg, (a.op == OP_DECODE) ? ss.seq + 1 : -1, flush ? ss.seq : -1,
-                           (a.op == OP_VERIFY) ? T : -1, flush);
+    // 6. Flush: this CTA read the counters long ago; its arrival lets the last CTA
+    //    of the sequence publish them.  (Decode and verify publish from the read
+    //    kernel, which runs after every prep CTA has read them.)
+    if (tid == 0 && a.op == OP_FLUSH)
+        arrive_and_publish(a.c, b, G * a.cpg, -1, flush ? ss.seq : -1, -1, flush);
 }
 
 // ---------------------------------------------------------------------------

@@ -33,7 +33,7 @@ size_t read_smem_bytes(const rssm_config &cf, int T) {
     return (size_t)read_lay(read_heads_per_cta(cf), cf.headdim, cf.dstate, cf.window, tq_of_read(T), ib, Ep).bytes;
 }
 
-cudaError_t launch_read(const Ctx &h, int T, const void *Q, int q_bf16, int q_group, int64_t q_stride_b,
+cudaError_t launch_read(const Ctx &h, int op, int T, const void *Q, int q_bf16, int q_group, int64_t q_stride_b,
                         int64_t q_stride_row, int64_t q_stride_m, const void *xnew, const float *D,
                         float *y, cudaStream_t st) {
     const rssm_config &cf = h.cfg;
@@ -54,6 +54,8 @@ cudaError_t launch_read(const Ctx &h, int T, const void *Q, int q_bf16, int q_gr
     r.TQmax = (int)h.lay.tq_max;
     r.Emax = (cf.window + r.TQmax + 3) & ~3;
     r.y = y;
+    r.c = h.counters();
+    r.op = op;
     const int TQ = tq_of_read(T);
     r.lay = read_lay(r.HC, cf.headdim, cf.dstate, cf.window, TQ, cf.input_dtype == RSSM_BF16 ? 2 : 4, r.Emax);
     const size_t smem = read_smem_bytes(cf, T);

@@ -56,7 +56,9 @@ struct ReadArgs {
     const void *xring;      // buffered entries [B][H][R][P] (input dtype)
     const void *xnew;       // the call's own entries [B][T][H][P] (input dtype)
     const float *D;         // per-head skip (nullptr: none)
-    const int4 *seqinfo;    // per sequence {L0 replayed from the ring, ring slot of entry 0, folded, 0}
+    const int4 *seqinfo;    // per sequence {L0 replayed from the ring, ring slot of entry 0, folded, valid}
+    Counters c;             // published by the first CTA of each sequence
+    int op;                 // OP_DECODE | OP_VERIFY
     const float *dec;       // [B][H][TQmax]
     const float *coef;      // [B][H][TQmax][Emax]
     int TQmax, Emax;        // Emax: padded row length of the coefficient table
@@ -115,6 +117,17 @@ __global__ void __launch_bounds__(kThreads, TQ == 1 ? 4 : 2) replay_read_kernel(
     if (tid == 0) {
         const int4 si = a.seqinfo[b];
         sinfo[0] = si.x; sinfo[1] = si.y; sinfo[2] = si.z;
+        // Counters of the sequence: every prep CTA has read them (the prep kernel
+        // ran before this one), so the first CTA of the sequence rewrites them.
+        if (blockIdx.x == 0 && si.w) {
+            const int64_t sp = a.c.seq_pos[b];
+            if (si.z) {
+                a.c.ckpt_pos[b] = sp;
+                a.c.flush_count[b] += 1;
+            }
+            if (a.op == OP_DECODE) a.c.seq_pos[b] = sp + 1;
+            else a.c.pending[b] = T;
+        }
     }
     for (int row = warp; row < T * HC; row += kWarps) {  // x of token m, head hh
         const int m = row / HC, hh = row - m * HC;
