@@ -92,7 +92,7 @@ void layout(const rssm_config *c, rssm_workspace_layout *L) {
         // prep -> read hand-off, rewritten by every decode/verify
         const size_t TQm = (size_t)(c->max_draft > 1 ? c->max_draft : 1);
         L->tq_max = TQm;
-        L->seqinfo_bytes = B * 16;
+        L->seqinfo_bytes = B * 16 + 16 + ((B * 4 + 15) & ~(size_t)15);
         L->seqinfo_off = take(L->seqinfo_bytes);
         L->dec_bytes = B * H * TQm * 4;
         L->dec_off = take(L->dec_bytes);
@@ -131,11 +131,8 @@ bool inputs_ok(const Ctx *h, const rssm_inputs *in) {
 }
 
 cudaError_t launch_kind(Ctx *h, int op, int T, const rssm_inputs *in, float *y, float *out) {
-    // replay decode/verify of Mamba-2 runs the prep/flush kernel and the replay-read kernel
-    const bool two = h->cfg.mode == RSSM_REPLAY && h->cfg.kind == RSSM_MAMBA2 &&
-                     (op == rssm::OP_DECODE || op == rssm::OP_VERIFY);
-    h->launches += two ? 2 : 1;
     if (h->cfg.kind == RSSM_MAMBA2) return rssm::mamba2_launch(*h, op, T, in, y, out, h->stream);
+    h->launches += 1;
     return rssm::gdn_launch(*h, op, T, in, y, out, h->stream);
 }
 
@@ -222,6 +219,7 @@ rssm_status rssm_import_state(rssm_handle hh, const float *S) {
     if (h->lay.rc_bytes) h->launches += 1;
     if (e == cudaSuccess)
         e = cudaMemsetAsync(h->at(h->lay.seq_pos_off), 0, h->lay.A_off - h->lay.seq_pos_off, h->stream);
+    h->len_lb = h->len_ub = 0;
     return e == cudaSuccess ? RSSM_OK : cuda_fail(h, e, "import_state");
 }
 

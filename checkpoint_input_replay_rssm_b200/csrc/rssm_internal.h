@@ -18,6 +18,7 @@ struct Ctx {
     size_t ws_bytes = 0;
     cudaStream_t stream = nullptr;
     int pending = 0;            // K of an uncommitted verify (host mirror), 0 if none
+    int len_lb = 0, len_ub = 0; // bounds of every sequence's committed buffer length (host mirror)
     int64_t launches = 0;       // kernels enqueued so far
     int num_sms = 148;          // SMs of the handle's device
     cudaEvent_t split_event = nullptr;  // recorded between prep and read kernels (measurement)
@@ -34,11 +35,16 @@ struct Ctx {
         c.err = (int32_t *)at(lay.error_off);
         return c;
     }
+    // Replay: work list of the flush kernel, after the per-sequence hand-off
+    // (int32 count, 3 pad words, then [batch] sequence indices).
+    int *fold_count() const { return (int *)at(lay.seqinfo_off + (size_t)cfg.batch * 16); }
+    int *fold_list() const { return fold_count() + 4; }
 };
 
 // Kernel launchers (one per layer kind).  op: Op; T tokens appended (0 for
-// flush/export); in/y used by decode/verify, out by export.
-cudaError_t mamba2_launch(const Ctx &h, int op, int T, const rssm_inputs *in, float *y, float *out,
+// flush/export); in/y used by decode/verify, out by export.  mamba2_launch
+// counts its launches and keeps the buffer-length bounds len_lb/len_ub.
+cudaError_t mamba2_launch(Ctx &h, int op, int T, const rssm_inputs *in, float *y, float *out,
                           cudaStream_t st);
 size_t mamba2_smem_bytes(const rssm_config &cf, int T);
 cudaError_t gdn_launch(const Ctx &h, int op, int T, const rssm_inputs *in, float *y, float *out,

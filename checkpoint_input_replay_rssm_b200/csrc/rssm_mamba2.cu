@@ -4,19 +4,30 @@
 
 namespace rssm {
 
-extern template cudaError_t m2_dispatch_n<16>(bool, int, int, const M2Args &, size_t, cudaStream_t);
-extern template cudaError_t m2_dispatch_n<32>(bool, int, int, const M2Args &, size_t, cudaStream_t);
-extern template cudaError_t m2_dispatch_n<64>(bool, int, int, const M2Args &, size_t, cudaStream_t);
-extern template cudaError_t m2_dispatch_n<128>(bool, int, int, const M2Args &, size_t, cudaStream_t);
+extern template cudaError_t m2_dispatch_n<16>(int, int, int, const M2Args &, const M2FoldLay &, size_t, int, cudaStream_t);
+extern template cudaError_t m2_dispatch_n<32>(int, int, int, const M2Args &, const M2FoldLay &, size_t, int, cudaStream_t);
+extern template cudaError_t m2_dispatch_n<64>(int, int, int, const M2Args &, const M2FoldLay &, size_t, int, cudaStream_t);
+extern template cudaError_t m2_dispatch_n<128>(int, int, int, const M2Args &, const M2FoldLay &, size_t, int, cudaStream_t);
 
 static int tq_of(int T) { return T <= 1 ? 1 : (T <= 4 ? 4 : 8); }
+static int in_bytes(const rssm_config &cf) { return cf.input_dtype == RSSM_BF16 ? 2 : 4; }
 
-// Heads per prep CTA: up to 8 heads of one group (the group's B . C is computed
-// once per CTA), within 160 KiB of shared memory.
+// Heads per prep CTA: up to the whole group (its B . C is computed once per CTA),
+// within 48 KiB of shared memory so that many CTAs stay resident.
 static int m2_prep_heads(const rssm_config &cf, int TQ) {
-    const int hpg = cf.nheads / cf.ngroups, ib = cf.input_dtype == RSSM_BF16 ? 2 : 4;
+    const int hpg = cf.nheads / cf.ngroups;
+    for (int hc = 16; hc > 1; --hc)
+        if (hpg % hc == 0 && m2_prep_lay(hc, cf.headdim, cf.dstate, cf.window, TQ, in_bytes(cf)).bytes <= 48 * 1024)
+            return hc;
+    return 1;
+}
+
+// Heads per flush CTA: up to 8 heads of one group, within 112 KiB of shared
+// memory (two CTAs per SM); a single head may take up to 200 KiB.
+static int m2_fold_heads(const rssm_config &cf, int TQ) {
+    const int hpg = cf.nheads / cf.ngroups;
     for (int hc = 8; hc > 1; --hc)
-        if (hpg % hc == 0 && m2_prep_lay(hc, cf.headdim, cf.dstate, cf.window, TQ, ib).bytes <= 150 * 1024)
+        if (hpg % hc == 0 && m2_fold_lay(hc, cf.headdim, cf.dstate, cf.window, TQ, in_bytes(cf)).bytes <= 112 * 1024)
             return hc;
     return 1;
 }
@@ -25,22 +36,36 @@ size_t mamba2_smem_bytes(const rssm_config &cf, int T) {
     const int TQ = tq_of(T), P = cf.headdim, N = cf.dstate;
     if (cf.mode == RSSM_EAGER)
         return sizeof(float) * ((size_t)2 * pad4(TQ * P) + 2 * pad4(TQ * N) + 2 * pad4(TQ));
-    const int ib = cf.input_dtype == RSSM_BF16 ? 2 : 4;
-    return (size_t)m2_prep_lay(m2_prep_heads(cf, TQ), P, N, cf.window, TQ, ib).bytes;
+    const size_t prep = m2_prep_lay(m2_prep_heads(cf, TQ), P, N, cf.window, TQ, in_bytes(cf)).bytes;
+    const size_t fold = m2_fold_lay(m2_fold_heads(cf, TQ), P, N, cf.window, TQ, in_bytes(cf)).bytes;
+    return prep > fold ? prep : fold;
 }
 
-cudaError_t mamba2_launch(const Ctx &h, int op, int T, const rssm_inputs *in, float *y, float *out,
-                          cudaStream_t st) {
+static cudaError_t dispatch(int which, int N, int rk, int TQ, const M2Args &a, const M2FoldLay &lay, size_t smem,
+                            int num_sms, cudaStream_t st) {
+    switch (N) {
+        case 16: return m2_dispatch_n<16>(which, rk, TQ, a, lay, smem, num_sms, st);
+        case 32: return m2_dispatch_n<32>(which, rk, TQ, a, lay, smem, num_sms, st);
+        case 64: return m2_dispatch_n<64>(which, rk, TQ, a, lay, smem, num_sms, st);
+        default: return m2_dispatch_n<128>(which, rk, TQ, a, lay, smem, num_sms, st);
+    }
+}
+
+// Replay decode/verify: prep kernel, flush kernel (only when some sequence's
+// buffer may be too full for the call's tokens: len_ub + T > W), replay-read
+// kernel.  Flush/export: the
+// flush kernel over every sequence.  Eager: one kernel.
+cudaError_t mamba2_launch(Ctx &h, int op, int T, const rssm_inputs *in, float *y, float *out, cudaStream_t st) {
     M2Args a{};
     const rssm_config &cf = h.cfg;
+    const int TQ = tq_of(T), ib = in_bytes(cf);
     a.B = cf.batch; a.H = cf.nheads; a.P = cf.headdim; a.G = cf.ngroups; a.W = cf.window;
-    a.R = (int)h.lay.ring; a.Rs = (int)h.lay.ring_stride; a.T = T; a.op = op; a.in_bf16 = cf.input_dtype == RSSM_BF16;
+    a.R = (int)h.lay.ring; a.Rs = (int)h.lay.ring_stride; a.T = T; a.op = op; a.in_bf16 = ib == 2;
     a.dt_scales = cf.dt_scales_input;
-    a.HC = m2_prep_heads(cf, tq_of(T));
-    a.cpg = (cf.nheads / cf.ngroups) / a.HC;
-    a.lay = m2_prep_lay(a.HC, cf.headdim, cf.dstate, cf.window, tq_of(T), cf.input_dtype == RSSM_BF16 ? 2 : 4);
     if (h.lay.seqinfo_bytes) {
         a.seqinfo = (int4 *)h.at(h.lay.seqinfo_off);
+        a.fold_count = h.fold_count();
+        a.fold_list = h.fold_list();
         a.dec = (float *)h.at(h.lay.dec_off);
         a.coef = (float *)h.at(h.lay.coef_off);
         a.TQmax = (int)h.lay.tq_max;
@@ -61,25 +86,62 @@ cudaError_t mamba2_launch(const Ctx &h, int op, int T, const rssm_inputs *in, fl
     }
     if (in) { a.x = in->x; a.dt = in->dt; a.Bm = in->Bm; a.Cm = in->Cm; }
     a.y = y; a.out = out;
-    const bool eager = cf.mode == RSSM_EAGER;
-    const int TQ = tq_of(T);
-    const size_t smem = mamba2_smem_bytes(cf, T);
-    cudaError_t e;
-    switch (cf.dstate) {
-        case 16: e = m2_dispatch_n<16>(eager, cf.state_dtype, TQ, a, smem, st); break;
-        case 32: e = m2_dispatch_n<32>(eager, cf.state_dtype, TQ, a, smem, st); break;
-        case 64: e = m2_dispatch_n<64>(eager, cf.state_dtype, TQ, a, smem, st); break;
-        default: e = m2_dispatch_n<128>(eager, cf.state_dtype, TQ, a, smem, st); break;
+    const int N = cf.dstate, rk = cf.state_dtype;
+    M2FoldLay flay{};
+
+    if (cf.mode == RSSM_EAGER) {
+        h.launches += 1;
+        return dispatch(M2_EAGER, N, rk, TQ, a, flay, mamba2_smem_bytes(cf, T), h.num_sms, st);
     }
-    if (e != cudaSuccess || eager || !(op == OP_DECODE || op == OP_VERIFY)) return e;
-    if (h.split_event) {
-        e = cudaEventRecord(h.split_event, st);
-        if (e != cudaSuccess) return e;
+    const int fHC = m2_fold_heads(cf, TQ);
+    flay = m2_fold_lay(fHC, cf.headdim, N, cf.window, TQ, ib);
+    M2Args f = a;  // flush kernel arguments
+    f.HC = fHC;
+    f.cpg = (cf.nheads / cf.ngroups) / fHC;
+    if (!(op == OP_DECODE || op == OP_VERIFY)) {  // flush / export
+        h.launches += 1;
+        cudaError_t e = dispatch(M2_FOLD, N, rk, TQ, f, flay, 0, h.num_sms, st);
+        if (e == cudaSuccess && op == OP_FLUSH) h.len_lb = h.len_ub = 0;
+        return e;
     }
-    // replay read: C of the group ([B][T][G][N]) is the query, x the buffered entries
-    const int G = cf.ngroups;
-    return launch_read(h, op, T, in->Cm, cf.input_dtype == RSSM_BF16, cf.nheads / G, (int64_t)T * G * cf.dstate,
-                       cf.dstate, (int64_t)G * cf.dstate, in->x, (const float *)h.at(h.lay.D_off), y, st);
+    const bool fold = h.len_ub + T > cf.window;
+    a.fold_launched = fold;
+    a.HC = m2_prep_heads(cf, TQ);
+    a.cpg = (cf.nheads / cf.ngroups) / a.HC;
+    a.lay = m2_prep_lay(a.HC, cf.headdim, N, cf.window, TQ, ib);
+    h.launches += 1;
+    cudaError_t e = dispatch(M2_PREP, N, rk, TQ, a, flay, (size_t)a.lay.bytes, h.num_sms, st);
+    if (e == cudaSuccess && fold) {
+        h.launches += 1;
+        e = dispatch(M2_FOLD, N, rk, TQ, f, flay, 0, h.num_sms, st);
+    }
+    if (e == cudaSuccess && h.split_event) e = cudaEventRecord(h.split_event, st);
+    if (e == cudaSuccess) {
+        // replay read: C of the group ([B][T][G][N]) is the query, x the buffered entries
+        const int G = cf.ngroups;
+        h.launches += 1;
+        e = launch_read(h, op, T, in->Cm, ib == 2, cf.nheads / G, (int64_t)T * G * N, N, (int64_t)G * N, in->x,
+                        (const float *)h.at(h.lay.D_off), y, st);
+    }
+    if (e != cudaSuccess) {  // leave no stale work list behind
+        cudaMemsetAsync(h.fold_count(), 0, sizeof(int), st);
+        return e;
+    }
+    // Committed lengths after this call (and the commit of a verify, which keeps
+    // 0..T of its tokens): a sequence that folds holds its kept tokens, the others
+    // add them to what they had.
+    const int W = cf.window, kept_min = op == OP_DECODE ? T : 0;
+    if (h.len_lb + T > W) {          // every sequence folded
+        h.len_lb = kept_min;
+        h.len_ub = T;
+    } else if (h.len_ub + T <= W) {  // none did
+        h.len_lb += kept_min;
+        h.len_ub += T;
+    } else {                          // some may have
+        h.len_lb = kept_min;
+        h.len_ub = W;
+    }
+    return cudaSuccess;
 }
 
 }  // namespace rssm

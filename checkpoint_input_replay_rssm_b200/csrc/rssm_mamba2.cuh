@@ -33,32 +33,22 @@ __host__ __device__ constexpr int dt_row_max_bytes(int W) { return ((W + 8 + 3) 
 constexpr int kFoldChunk = 16 * 1024;  // bytes of fp32 checkpoint rows per fold stage
 
 // Shared memory of the prep kernel (bytes, 16-byte aligned regions), computed on
-// the host.  Entry slots of x: E = W + TQ; committed entries sit right-aligned
-// before slot W and the call's own tokens at W..W+T-1, so logical entry e is
-// slot (W - L0) + e.  The group's B ring is staged whole (R <= W + 8 rows).
+// the host.  The group's B ring is staged whole (R <= W + 8 rows).
 struct M2PrepLay {
-    int fold, bar, sC, sBr, sBn, sx, dring, dtn, sd, slam, scoef, sdec, su, sfdec, sCf, sdot, si, bytes;
+    int sC, sBr, sBn, sx, dring, dtn, sd, slam, si, bytes;
 };
 inline M2PrepLay m2_prep_lay(int HC, int P, int N, int W, int TQ, int ib) {
     const int E = W + TQ;
     M2PrepLay L{};
     int o = 0;
-    L.fold = o;  o += 2 * kFoldChunk;            // fp32 checkpoint rows, two stages
-    L.bar = o;   o += 16;                        // their mbarriers
     L.sC = o;    o += a16(TQ * N * ib);          // raw C of the queries     [TQ][N]
     L.sBr = o;   o += a16((W + 8) * N * ib);     // raw B ring of the group  [R][N]
     L.sBn = o;   o += a16(TQ * N * ib);          // raw B of the call's tokens [TQ][N]
-    L.sx = o;    o += a16(HC * E * P * ib);      // raw x of the entries     [HC][E][P]
+    L.sx = o;    o += a16(TQ * HC * P * ib);     // raw x of the call's tokens [TQ][HC][P]
     L.dring = o; o += a16(HC * dt_row_max_bytes(W));  // dt ring rows        [HC][Rs]
     L.dtn = o;   o += a16(TQ * HC * 4);          // dt of the call's tokens  [TQ][HC]
     L.sd = o;    o += a16(TQ * E * 4);           // B_e . C_m                [TQ][E]
     L.slam = o;  o += a16(HC * E * 4);           // prefix sums of dt*A      [HC][E]
-    L.scoef = o; o += a16(HC * TQ * E * 4);      // replay coefficients      [HC][TQ][E]
-    L.sdec = o;  o += a16(HC * TQ * 4);          // decay of S^ C            [HC][TQ]
-    L.su = o;    o += a16(HC * E * 4);           // fold weights             [HC][E]
-    L.sfdec = o; o += a16(HC * 4);               // decay of the folded checkpoint [HC]
-    L.sCf = o;   o += a16(TQ * N * 4);           // C as fp32                [TQ][N]
-    L.sdot = o;  o += a16(HC * P * TQ * 4);      // fresh copy . C per row   [HC*P][TQ]
     L.si = o;    o += 32;
     L.bytes = o;
     return L;
@@ -66,9 +56,12 @@ inline M2PrepLay m2_prep_lay(int HC, int P, int N, int W, int TQ, int ib) {
 
 struct M2Args {
     int B, H, P, G, W, R, Rs, T, op, in_bf16, dt_scales;  // Rs: dt ring row length
-    int HC, cpg;        // heads per prep CTA (divides H / G); prep CTAs per group
+    int HC, cpg;        // heads per CTA (divides H / G); CTAs per group
     M2PrepLay lay;      // prep kernel shared memory
-    int4 *seqinfo;      // per sequence, for the read kernel: {L0, ring slot of entry 0, folded, 0}
+    int4 *seqinfo;      // per sequence, for the read kernel: {L0, ring slot of entry 0, folded, valid}
+    int *fold_count;    // sequences the flush kernel folds in this call (reset by the read kernel)
+    int *fold_list;     // [B] their indices
+    int fold_launched;  // the host launches the flush kernel in this call
     float *dec;         // [B][H][TQmax] decay of S^ C
     float *coef;        // [B][H][TQmax][Emax] replay coefficients
     int TQmax, Emax;    // Emax: padded row length of the coefficient table
@@ -91,33 +84,21 @@ struct M2Args {
 };
 
 // ---------------------------------------------------------------------------
-// Prep / flush kernel: decode (T = 1), verify (T = K), flush and export (T = 0).
+// Prep kernel: decode (T = 1) and verify (T = K).
 //
 // One CTA per (group chunk of HC heads, sequence b).  In one round trip it reads
 // the sequence's counters and stages the group's whole B ring, the heads' dt
-// ring rows and the call's tokens; then B_e . C_m once for the group and, per
-// head (one warp each), the prefix sums Lam of dt*A and the coefficients.
-//   * no fold: the replay coefficients
-//       coef[m][e] = e^{Lam_{L0+m} - Lam_e} (B_e . C_m) s_e,   dec[m] = e^{Lam_{L0+m}}
-//     go to the read kernel;
-//   * fold (len + T > W, or flush/export): the committed entries are folded into
-//     the fp32 checkpoint, S_c <- e^{Lam_{L0-1}} S_c + sum_e e^{Lam_{L0-1} - Lam_e} s_e x_e B_e^T.
-//     Thread 0 starts bulk copies of the checkpoint rows (16 KiB stages, two in
-//     flight) as soon as it has read the counters; the CTA stores the result
-//     with the requantised read copy (or writes it out, for export) and, for
-//     decode/verify, computes the outputs from the fresh copy itself.
-// Last it appends the call's tokens to the ring, and thread 0 registers the
-// CTA's arrival; the last CTA of the sequence publishes the counters.
+// ring rows and the call's tokens.  A sequence whose buffer must be folded first
+// (len + T > W) is left to the flush kernel (m2_fold_kernel).  Otherwise it
+// computes B_e . C_m once for the group and, per head (one warp each), the
+// prefix sums Lam of dt*A and the replay coefficients for the read kernel:
+//     coef[m][e] = e^{Lam_{L0+m} - Lam_e} (B_e . C_m) s_e,   dec[m] = e^{Lam_{L0+m}}.
+// Every sequence's tokens are appended to the ring (slots seq_pos + m mod R);
+// the slots of the entries a fold reads are never among them (R >= W + T).
 // ---------------------------------------------------------------------------
-template <int N, int RK, int TQ, bool BF>
-__global__ void __launch_bounds__(kThreads, 3) m2_prep_kernel(const M2Args a) {
-    constexpr int TPR4 = N / 4;           // lanes per row, fp32 quad mapping
-    constexpr int RPP4 = kThreads / TPR4;
-    constexpr int FC = kFoldChunk / (N * 4);  // fp32 rows per fold stage
-    constexpr int FH = FC / RPP4;         // rows per thread per stage (= 4)
-    constexpr int FB = 4;                 // buffered B entries held in registers per block
+template <int N, int TQ, bool BF>
+__global__ void __launch_bounds__(kThreads, 4) m2_prep_kernel(const M2Args a) {
     constexpr int IB = BF ? 2 : 4;
-    static_assert(FH * RPP4 == FC, "fold stage is FH rows per thread");
     extern __shared__ __align__(128) uint8_t smraw[];
     const M2PrepLay &Ly = a.lay;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -127,65 +108,45 @@ __global__ void __launch_bounds__(kThreads, 3) m2_prep_kernel(const M2Args a) {
     const int g = blockIdx.x / a.cpg, hc = blockIdx.x - g * a.cpg;
     const int h0 = g * hpg + hc * HC;
     const int E = W + TQ;
-    float *fbuf = reinterpret_cast<float *>(smraw + Ly.fold);
-    uint64_t *fbar = reinterpret_cast<uint64_t *>(smraw + Ly.bar);
     uint8_t *sC = smraw + Ly.sC, *sBr = smraw + Ly.sBr, *sBn = smraw + Ly.sBn, *sx = smraw + Ly.sx;
     float *dring = reinterpret_cast<float *>(smraw + Ly.dring);
     float *dtn = reinterpret_cast<float *>(smraw + Ly.dtn);
     float *sd = reinterpret_cast<float *>(smraw + Ly.sd);
     float *slam = reinterpret_cast<float *>(smraw + Ly.slam);
-    float *scoef = reinterpret_cast<float *>(smraw + Ly.scoef);
-    float *sdec = reinterpret_cast<float *>(smraw + Ly.sdec);
-    float *su = reinterpret_cast<float *>(smraw + Ly.su);
-    float *sfdec = reinterpret_cast<float *>(smraw + Ly.sfdec);
-    float *sCf = reinterpret_cast<float *>(smraw + Ly.sCf);
-    float *sdot = reinterpret_cast<float *>(smraw + Ly.sdot);
     int *si = reinterpret_cast<int *>(smraw + Ly.si);
     const int64_t row0 = (int64_t)b * H + h0;
-    const int64_t tile0 = row0 * P * N;
-    const int nrows = HC * P;
-    const int nfc = (nrows + FC - 1) / FC;  // fold stages
-    const bool reads = (a.op == OP_DECODE || a.op == OP_VERIFY);
     const int xrow = P * IB, brow = N * IB, xch = xrow / 16, bch = brow / 16;
     const int Rs = a.Rs;
     auto ldx = [](const uint8_t *p) -> float {
         return BF ? bf16_bits_to_float(*reinterpret_cast<const uint16_t *>(p)) : *reinterpret_cast<const float *>(p);
     };
-    auto fold_issue = [&](int c) {  // thread 0: stage c of the checkpoint rows into buffer c & 1
-        const int r0 = c * FC, r1 = min(nrows, r0 + FC);
-        const uint32_t bytes = (uint32_t)((r1 - r0) * N * 4);
-        mbar_arrive_expect_tx(&fbar[c & 1], bytes);
-        bulk_g2s(fbuf + (c & 1) * (FC * N), a.ckpt + tile0 + (int64_t)r0 * N, bytes, &fbar[c & 1]);
-    };
 
-    // 1. Counters (thread 0; starts the fold's checkpoint copies when one is due)
-    //    and everything that does not depend on them, at once.
-    SeqState ss{};
+    // 1. Counters (thread 0) and everything that does not depend on them, at once.
     if (tid == 0) {
-        ss = read_counters(a.c, b, W);
+        const SeqState ss = read_counters(a.c, b, W);
         const int L0 = (int)(ss.seq - ss.ckpt);
-        int flush = 0;
-        if (ss.ok) flush = (a.op == OP_FLUSH || a.op == OP_EXPORT) ? (L0 > 0) : (L0 + T > W);
+        const int fold = ss.ok && (L0 + T > W);
         si[0] = ss.ok;
         si[1] = ss.ok ? L0 : 0;
-        si[2] = flush;
+        si[2] = fold;
         si[3] = (int)(ss.ckpt % R);
         si[4] = (int)(ss.seq % R);
-        if (flush) {
-            mbar_init(&fbar[0], 1);
-            mbar_init(&fbar[1], 1);
-            mbar_init_fence();
-            fold_issue(0);
-            if (nfc > 1) fold_issue(1);
-        }
         // seqinfo: {ring entries the read kernel replays, ring slot of entry 0,
-        // folded here, counters valid} -- the read kernel also publishes the
-        // sequence's new counters from it
-        if (!ss.ok) {
-            if (blockIdx.x == 0) report(a.c.err, DEV_BAD_COUNTERS, b, h0, L0);
-            if (reads && blockIdx.x == 0) a.seqinfo[b] = make_int4(0, 0, 1, 0);  // nothing to read or publish
-        } else if (reads && blockIdx.x == 0) {
-            a.seqinfo[b] = make_int4(flush ? 0 : L0, (int)(ss.ckpt % R), flush, 1);
+        // folded by the flush kernel, counters valid}; the read kernel also
+        // publishes the sequence's new counters from it
+        if (blockIdx.x == 0) {
+            bool valid = ss.ok;
+            if (!ss.ok) report(a.c.err, DEV_BAD_COUNTERS, b, h0, L0);
+            if (fold) {  // list the sequence for the flush kernel
+                if (a.fold_launched) {
+                    const int j = atomicAdd(a.fold_count, 1);
+                    if (j < a.B) a.fold_list[j] = b;
+                } else {  // the host's bound on buffer lengths was wrong: counters changed outside the API
+                    report(a.c.err, DEV_BAD_COUNTERS, b, h0, L0);
+                    valid = false;
+                }
+            }
+            a.seqinfo[b] = valid ? make_int4(fold ? 0 : L0, (int)(ss.ckpt % R), fold, 1) : make_int4(0, 0, 1, 0);
         }
     }
     {
@@ -203,7 +164,7 @@ __global__ void __launch_bounds__(kThreads, 3) m2_prep_kernel(const M2Args a) {
     for (int row = warp; row < T * HC; row += kWarps) {
         const int m = row / HC, hh = row - m * HC;
         const uint8_t *src = reinterpret_cast<const uint8_t *>(a.x) + (((int64_t)(b * T + m) * H + h0 + hh) * P) * IB;
-        for (int k = lane; k < xch; k += 32) cp_async16(sx + (hh * E + W + m) * xrow + k * 16, src + k * 16);
+        for (int k = lane; k < xch; k += 32) cp_async16(sx + (m * HC + hh) * xrow + k * 16, src + k * 16);
     }
     for (int i = tid; i < T * HC; i += kThreads) {
         const int m = i / HC, hh = i - m * HC;
@@ -211,170 +172,376 @@ __global__ void __launch_bounds__(kThreads, 3) m2_prep_kernel(const M2Args a) {
     }
     cp_async_wait_all();
     __syncthreads();
-    if (!si[0]) return;  // counters corrupted: reported, sequence skipped, no arrival
-    const int L0 = si[1], flush = si[2], ckmod = si[3], spmod = si[4];
-    const int base = W - L0, nE = L0 + T;
-    const int e0 = flush ? L0 : 0;  // first entry the outputs replay
+    if (!si[0]) return;  // counters corrupted: reported, sequence skipped
+    const int L0 = si[1], fold = si[2], ckmod = si[3], spmod = si[4];
+    const int nE = L0 + T;
     auto slot_of = [&](int e) { const int s = ckmod + e; return s >= R ? s - R : s; };
-    auto B_of = [&](int e) -> const uint8_t * {  // B of logical entry e
-        return e < L0 ? sBr + slot_of(e) * brow : sBn + (e - L0) * brow;
-    };
-    auto dt_of = [&](int hh, int e) -> float {
-        return e < L0 ? dring[hh * Rs + slot_of(e)] : dtn[(e - L0) * HC + hh];
-    };
-    if (flush) {  // the heads' buffered x, needed only to fold
-        const int n1 = min(L0, R - ckmod);
-        for (int row = warp; row < 2 * HC; row += kWarps) {
-            const int hh = row >> 1, second = row & 1;
-            const int cnt = second ? L0 - n1 : n1;
-            const uint8_t *src = reinterpret_cast<const uint8_t *>(a.xbuf) +
-                                 (((row0 + hh) * R + (second ? 0 : ckmod)) * P) * IB;
-            uint8_t *dst = sx + (hh * E + base + (second ? n1 : 0)) * xrow;
-            for (int k = lane; k < cnt * xch; k += 32) cp_async16(dst + k * 16, src + k * 16);
-        }
-    }
 
-    // 2. B_e . C_m once for the group (warps), C as fp32.
-    if (reads) {
+    if (!fold) {
+        // 2. B_e . C_m once for the group (warps).
         for (int pr = warp; pr < T * nE; pr += kWarps) {
             const int m = pr / nE, e = pr - m * nE;
-            if (e > L0 + m || e < e0) continue;  // warp-uniform
-            const uint8_t *Bp = B_of(e), *Cp = sC + m * brow;
+            if (e > L0 + m) continue;  // warp-uniform
+            const uint8_t *Bp = e < L0 ? sBr + slot_of(e) * brow : sBn + (e - L0) * brow;
+            const uint8_t *Cp = sC + m * brow;
             float d = 0.f;
             for (int n = lane; n < N; n += 32) d = fmaf(ldx(Bp + n * IB), ldx(Cp + n * IB), d);
             d = group_sum<32>(d);
             if (lane == 0) sd[m * E + e] = d;
         }
-        for (int i = tid; i < T * N; i += kThreads) sCf[i] = ldx(sC + i * IB);
+        __syncthreads();
+        // 3. Per head (one warp): prefix sums of dt*A, coefficients, decays.
+        for (int hh = warp; hh < HC; hh += kWarps) {
+            const float Ah = a.A[h0 + hh];
+            float *lam = slam + hh * E;
+            float carry = 0.f;
+            for (int k0 = 0; k0 < nE; k0 += 32) {
+                const int e = k0 + lane;
+                float v = 0.f;
+                if (e < nE) v = (e < L0 ? dring[hh * Rs + slot_of(e)] : dtn[(e - L0) * HC + hh]) * Ah;
+                v = warp_incl_scan(v) + carry;
+                if (e < nE) lam[e] = v;
+                carry = __shfl_sync(0xffffffffu, v, 31);
+            }
+            __syncwarp();
+            float *crow = a.coef + (row0 + hh) * a.TQmax * a.Emax;
+            for (int e = lane; e < nE; e += 32) {
+                const float se = a.dt_scales ? (e < L0 ? dring[hh * Rs + slot_of(e)] : dtn[(e - L0) * HC + hh]) : 1.f;
+#pragma unroll
+                for (int m = 0; m < TQ; ++m)
+                    if (m < T && e <= L0 + m) crow[m * a.Emax + e] = expf(lam[L0 + m] - lam[e]) * sd[m * E + e] * se;
+            }
+            if (lane < T) a.dec[(row0 + hh) * a.TQmax + lane] = expf(lam[L0 + lane]);
+        }
+    }
+
+    // 4. Append the call's tokens to the ring.
+    for (int row = warp; row < T * HC; row += kWarps) {
+        const int m = row / HC, hh = row - m * HC;
+        const int slot = spmod + m >= R ? spmod + m - R : spmod + m;
+        uint8_t *dst = reinterpret_cast<uint8_t *>(a.xbuf) + (((row0 + hh) * R + slot) * P) * IB;
+        const uint8_t *src = sx + (m * HC + hh) * xrow;
+        for (int k = lane; k < xch; k += 32)
+            *reinterpret_cast<uint4 *>(dst + k * 16) = *reinterpret_cast<const uint4 *>(src + k * 16);
+    }
+    for (int i = tid; i < T * HC; i += kThreads) {
+        const int m = i / HC, hh = i - m * HC;
+        const int slot = spmod + m >= R ? spmod + m - R : spmod + m;
+        a.dtbuf[(row0 + hh) * Rs + slot] = dtn[m * HC + hh];
+    }
+    if (hc == 0) {  // the group's first chunk writes the group's B
+        for (int row = warp; row < T; row += kWarps) {
+            const int slot = spmod + row >= R ? spmod + row - R : spmod + row;
+            uint8_t *dst = reinterpret_cast<uint8_t *>(a.Bbuf) + (((int64_t)(b * G + g) * R + slot) * N) * IB;
+            for (int k = lane; k < bch; k += 32)
+                *reinterpret_cast<uint4 *>(dst + k * 16) = *reinterpret_cast<const uint4 *>(sBn + row * brow + k * 16);
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Flush kernel: fold the committed buffer into the fp32 checkpoint and
+// requantise the read copy ("the checkpoint is rewritten only when the buffer
+// is full", blog.thibaultmonteiro.fr, "Tenir le journal plutot que le solde").
+// Runs for decode/verify calls that find a full buffer (len + T > W; it then
+// also serves that sequence's outputs), and for flush (len > 0) and export
+// (writing the folded state out instead).
+//
+//     S_c <- e^{Lam_{L0-1}} S_c + sum_{e < L0} U_e B_e^T,   U_e[p] = e^{Lam_{L0-1} - Lam_e} s_e x_e[p]
+//
+// is a rank-L0 update: U and B (fp32, in shared memory) give each thread a 4x4
+// register block (4 consecutive rows x 4 columns) updated with two 128-bit
+// shared loads and 16 FMAs per entry.  The checkpoint rows arrive in 16 KiB
+// bulk-copy stages, three in flight; all waits are bounded.
+// ---------------------------------------------------------------------------
+struct M2FoldLay {
+    int stage, bar, sC, sBr, sBn, sx, dring, dtn, U, Bf, slam, su, scoef, sdec, sfdec, sCf, sdot, si, bytes;
+};
+constexpr int kFoldStages = 3;
+inline M2FoldLay m2_fold_lay(int HC, int P, int N, int W, int TQ, int ib) {
+    const int E = W + TQ;
+    M2FoldLay L{};
+    int o = 0;
+    L.stage = o; o += kFoldStages * kFoldChunk;  // fp32 checkpoint rows
+    L.bar = o;   o += 8 * kFoldStages;
+    o = a16(o);
+    L.sC = o;    o += a16(TQ * N * ib);          // raw C of the queries       [TQ][N]
+    L.sBr = o;   o += a16((W + 8) * N * ib);     // raw B ring of the group    [R][N]
+    L.sBn = o;   o += a16(TQ * N * ib);          // raw B of the call's tokens [TQ][N]
+    L.sx = o;    o += a16(HC * E * P * ib);      // raw x of the entries       [HC][E][P]
+    L.dring = o; o += a16(HC * dt_row_max_bytes(W));  // dt ring rows          [HC][Rs]
+    L.dtn = o;   o += a16(TQ * HC * 4);          // dt of the call's tokens    [TQ][HC]
+    L.U = o;     o += a16(HC * W * P * 4);       // fold weights x rows        [HC][L0][P]
+    L.Bf = o;    o += a16(W * N * 4);            // committed B as fp32        [L0][N]
+    L.slam = o;  o += a16(HC * E * 4);           // prefix sums of dt*A        [HC][E]
+    L.su = o;    o += a16(HC * E * 4);           // fold weights               [HC][E]
+    L.scoef = o; o += a16(HC * TQ * E * 4);      // coefficients of the new tokens [HC][TQ][E]
+    L.sdec = o;  o += a16(HC * TQ * 4);          // decay of the fresh copy    [HC][TQ]
+    L.sfdec = o; o += a16(HC * 4);               // decay of the folded checkpoint [HC]
+    L.sCf = o;   o += a16(TQ * N * 4);           // C as fp32                  [TQ][N]
+    L.sdot = o;  o += a16(HC * P * TQ * 4);      // fresh copy . C per row     [HC*P][TQ]
+    L.si = o;    o += 32;
+    L.bytes = o;
+    return L;
+}
+
+template <int N, int RK, int TQ, bool BF>
+__global__ void __launch_bounds__(kThreads, 2) m2_fold_kernel(const M2Args a, const M2FoldLay Ly) {
+    constexpr int Q = N / 4;              // column quads per row
+    constexpr int RG = kThreads / Q;      // row groups per stage
+    constexpr int FC = kFoldChunk / (N * 4);  // fp32 rows per stage (= 4 * RG)
+    constexpr int IB = BF ? 2 : 4;
+    static_assert(FC == 4 * RG, "each thread owns 4 consecutive rows of a stage");
+    extern __shared__ __align__(128) uint8_t smraw[];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int H = a.H, P = a.P, W = a.W, R = a.R, T = a.T, G = a.G, HC = a.HC;
+    const int hpg = H / G;
+    const int E = W + TQ;
+    float *stg = reinterpret_cast<float *>(smraw + Ly.stage);
+    uint64_t *bar = reinterpret_cast<uint64_t *>(smraw + Ly.bar);
+    uint8_t *sC = smraw + Ly.sC, *sBr = smraw + Ly.sBr, *sBn = smraw + Ly.sBn, *sx = smraw + Ly.sx;
+    float *dring = reinterpret_cast<float *>(smraw + Ly.dring);
+    float *dtn = reinterpret_cast<float *>(smraw + Ly.dtn);
+    float *U = reinterpret_cast<float *>(smraw + Ly.U);
+    float *Bf = reinterpret_cast<float *>(smraw + Ly.Bf);
+    float *slam = reinterpret_cast<float *>(smraw + Ly.slam);
+    float *su = reinterpret_cast<float *>(smraw + Ly.su);
+    float *scoef = reinterpret_cast<float *>(smraw + Ly.scoef);
+    float *sdec = reinterpret_cast<float *>(smraw + Ly.sdec);
+    float *sfdec = reinterpret_cast<float *>(smraw + Ly.sfdec);
+    float *sCf = reinterpret_cast<float *>(smraw + Ly.sCf);
+    float *sdot = reinterpret_cast<float *>(smraw + Ly.sdot);
+    int *si = reinterpret_cast<int *>(smraw + Ly.si);
+    const int nrows = HC * P;
+    const int nst = (nrows + FC - 1) / FC;
+    const bool reads = (a.op == OP_DECODE || a.op == OP_VERIFY);
+    const int xrow = P * IB, brow = N * IB, xch = xrow / 16, bch = brow / 16;
+    const int Rs = a.Rs;
+    const int chunks = G * a.cpg;  // CTA work items per sequence
+    auto ldx = [](const uint8_t *p) -> float {
+        return BF ? bf16_bits_to_float(*reinterpret_cast<const uint16_t *>(p)) : *reinterpret_cast<const float *>(p);
+    };
+
+    // Work items (sequence, chunk of HC heads of one group): decode/verify fold
+    // the sequences the prep kernel listed; flush/export visit every sequence.
+    const int nitems = (reads ? min(*a.fold_count, a.B) : a.B) * chunks;
+    if (tid == 0) {
+        for (int k = 0; k < kFoldStages; ++k) mbar_init(&bar[k], 1);
+        mbar_init_fence();
     }
     __syncthreads();
+    uint32_t gs = 0;  // checkpoint stages consumed so far: stage slot gs % 3, phase (gs / 3) & 1
 
-    // 3. Per head (one warp): prefix sums of dt*A, coefficients, decays.
-    for (int hh = warp; hh < HC; hh += kWarps) {
-        const float Ah = a.A[h0 + hh];
-        float *lam = slam + hh * E + base;
-        float carry = 0.f;
-        for (int k0 = 0; k0 < nE; k0 += 32) {
-            const int e = k0 + lane;
-            float v = (e < nE) ? dt_of(hh, e) * Ah : 0.f;
-            v = warp_incl_scan(v) + carry;
-            if (e < nE) lam[e] = v;
-            carry = __shfl_sync(0xffffffffu, v, 31);
+    for (int item = blockIdx.x; item < nitems; item += gridDim.x) {
+        const int b = reads ? a.fold_list[item / chunks] : item / chunks;
+        const int chunk = item % chunks;
+        const int g = chunk / a.cpg, hc = chunk - g * a.cpg;
+        const int h0 = g * hpg + hc * HC;
+        const int64_t row0 = (int64_t)b * H + h0;
+        const int64_t tile0 = row0 * P * N;
+        auto issue = [&](int c) {  // thread 0: stage c of the item's checkpoint rows
+            const int r0 = c * FC, r1 = min(nrows, r0 + FC);
+            const uint32_t bytes = (uint32_t)((r1 - r0) * N * 4);
+            const int k = (gs + c) % kFoldStages;
+            mbar_arrive_expect_tx(&bar[k], bytes);
+            bulk_g2s(stg + k * (FC * N), a.ckpt + tile0 + (int64_t)r0 * N, bytes, &bar[k]);
+        };
+
+        // 1. Counters: fold when the buffer holds committed entries (flush,
+        //    export) or is too full for the call's tokens (decode, verify).
+        SeqState ss{};
+        if (tid == 0) {
+            ss = read_counters(a.c, b, W);
+            const int L0 = (int)(ss.seq - ss.ckpt);
+            const int fold = ss.ok && (reads ? (L0 + T > W) : (L0 > 0));
+            si[0] = fold;
+            si[1] = L0;
+            si[3] = (int)(ss.ckpt % R);
+            if (!ss.ok && !reads && chunk == 0) report(a.c.err, DEV_BAD_COUNTERS, b, h0, L0);
+            if (fold)
+                for (int c = 0; c < kFoldStages && c < nst; ++c) issue(c);
         }
-        __syncwarp();
-        const float lam_f = (flush && L0 > 0) ? lam[L0 - 1] : 0.f;
-        for (int e = lane; e < nE; e += 32) {
-            const float se = a.dt_scales ? dt_of(hh, e) : 1.f;
-            if (reads) {
-#pragma unroll
-                for (int m = 0; m < TQ; ++m) {
-                    if (m >= T || e > L0 + m || e < e0) continue;
-                    const float cf = expf(lam[L0 + m] - lam[e]) * sd[m * E + e] * se;
-                    if (flush) scoef[(hh * TQ + m) * E + e] = cf;
-                    else a.coef[((row0 + hh) * a.TQmax + m) * a.Emax + e] = cf;
-                }
+        __syncthreads();
+        if (!si[0]) {
+            if (tid == 0 && a.op == OP_FLUSH)  // nothing to fold; the CTA still arrives
+                arrive_and_publish(a.c, b, chunks, -1, -1, -1, 0);
+            __syncthreads();
+            continue;
+        }
+        const int L0 = si[1], ckmod = si[3];
+        const int base = W - L0, nE = L0 + T;
+        auto slot_of = [&](int e) { const int s = ckmod + e; return s >= R ? s - R : s; };
+
+        // 2. Stage the buffered entries (B of the group, x and dt of the heads) and the call's tokens.
+        {
+            const uint8_t *src = reinterpret_cast<const uint8_t *>(a.Bbuf) + ((int64_t)(b * G + g) * R) * brow;
+            for (int i = tid; i < R * bch; i += kThreads) cp_async16(sBr + i * 16, src + i * 16);
+        }
+        for (int i = tid; i < HC * Rs / 4; i += kThreads) cp_async16(dring + 4 * i, a.dtbuf + row0 * Rs + 4 * i);
+        {
+            const int n1 = min(L0, R - ckmod);
+            for (int row = warp; row < 2 * HC; row += kWarps) {
+                const int hh = row >> 1, second = row & 1;
+                const int cnt = second ? L0 - n1 : n1;
+                const uint8_t *src = reinterpret_cast<const uint8_t *>(a.xbuf) +
+                                     (((row0 + hh) * R + (second ? 0 : ckmod)) * P) * IB;
+                uint8_t *dst = sx + (hh * E + base + (second ? n1 : 0)) * xrow;
+                for (int k = lane; k < cnt * xch; k += 32) cp_async16(dst + k * 16, src + k * 16);
             }
-            if (flush && e < L0) su[hh * E + e] = expf(lam_f - lam[e]) * se;
         }
-        if (lane == 0) sfdec[hh] = flush ? expf(lam_f) : 1.f;
-        if (reads && lane < T) {
-            const float dcy = expf(lam[L0 + lane] - lam_f);
-            if (flush) sdec[hh * TQ + lane] = dcy;
-            else a.dec[(row0 + hh) * a.TQmax + lane] = dcy;
+        for (int row = warp; row < T; row += kWarps) {
+            const int64_t src = (((int64_t)(b * T + row) * G + g) * N) * IB;
+            for (int k = lane; k < bch; k += 32) {
+                cp_async16(sC + row * brow + k * 16, reinterpret_cast<const uint8_t *>(a.Cm) + src + k * 16);
+                cp_async16(sBn + row * brow + k * 16, reinterpret_cast<const uint8_t *>(a.Bm) + src + k * 16);
+            }
         }
-    }
-
-    if (flush) {
+        for (int row = warp; row < T * HC; row += kWarps) {
+            const int m = row / HC, hh = row - m * HC;
+            const uint8_t *src = reinterpret_cast<const uint8_t *>(a.x) + (((int64_t)(b * T + m) * H + h0 + hh) * P) * IB;
+            for (int k = lane; k < xch; k += 32) cp_async16(sx + (hh * E + W + m) * xrow + k * 16, src + k * 16);
+        }
+        for (int i = tid; i < T * HC; i += kThreads) {
+            const int m = i / HC, hh = i - m * HC;
+            dtn[m * HC + hh] = a.dt[(int64_t)(b * T + m) * H + h0 + hh];
+        }
         cp_async_wait_all();
         __syncthreads();
-        // 4. Fold, one staged 16 KiB block of checkpoint rows at a time (the next
-        //    one in flight): FH rows per thread, FB buffered B entries per block
-        //    in registers; store the checkpoint and the requantised copy, and dot
-        //    the fresh copy with C.
-        const int c4 = tid % TPR4, q0 = tid / TPR4;
-        bool timed_out = false;
-        for (int c = 0; c < nfc; ++c) {
-            const bool got = mbar_wait(&fbar[c & 1], (c >> 1) & 1);
+        auto dt_of = [&](int hh, int e) -> float {
+            return e < L0 ? dring[hh * Rs + slot_of(e)] : dtn[(e - L0) * HC + hh];
+        };
+
+        // 3. Per head (one warp): prefix sums of dt*A, fold weights, decays; C and
+        //    the committed entries' B as fp32.
+        for (int hh = warp; hh < HC; hh += kWarps) {
+            const float Ah = a.A[h0 + hh];
+            float *lam = slam + hh * E;
+            float carry = 0.f;
+            for (int k0 = 0; k0 < nE; k0 += 32) {
+                const int e = k0 + lane;
+                float v = (e < nE) ? dt_of(hh, e) * Ah : 0.f;
+                v = warp_incl_scan(v) + carry;
+                if (e < nE) lam[e] = v;
+                carry = __shfl_sync(0xffffffffu, v, 31);
+            }
+            __syncwarp();
+            const float lam_f = lam[L0 - 1];
+            for (int e = lane; e < L0; e += 32)
+                su[hh * E + e] = expf(lam_f - lam[e]) * (a.dt_scales ? dt_of(hh, e) : 1.f);
+            if (lane == 0) sfdec[hh] = expf(lam_f);
+            if (reads && lane < T) sdec[hh * TQ + lane] = expf(lam[L0 + lane] - lam_f);
+        }
+        for (int i = tid; i < L0 * N; i += kThreads) {
+            const int e = i / N, n = i - e * N;
+            Bf[e * N + n] = ldx(sBr + slot_of(e) * brow + n * IB);
+        }
+        if (reads)
+            for (int i = tid; i < T * N; i += kThreads) sCf[i] = ldx(sC + i * IB);
+        __syncthreads();
+        for (int i = tid; i < HC * L0 * P; i += kThreads) {  // U[hh][e][p] = weight * x
+            const int hh = i / (L0 * P), r2 = i - hh * L0 * P;
+            const int e = r2 / P, p = r2 - e * P;
+            U[(hh * L0 + e) * P + p] = su[hh * E + e] * ldx(sx + (hh * E + base + e) * xrow + p * IB);
+        }
+        if (reads) {  // coefficients of the call's own tokens against the fresh checkpoint
+            for (int pr = warp; pr < T * T; pr += kWarps) {
+                const int m = pr / T, j = pr - m * T;  // entry L0 + j, query m
+                if (j > m) continue;                   // warp-uniform
+                float d = 0.f;
+                for (int n = lane; n < N; n += 32) d = fmaf(ldx(sBn + j * brow + n * IB), sCf[m * N + n], d);
+                d = group_sum<32>(d);
+                if (lane < HC) {
+                    const float *lam = slam + lane * E;
+                    scoef[(lane * TQ + m) * E + L0 + j] =
+                        expf(lam[L0 + m] - lam[L0 + j]) * d * (a.dt_scales ? dtn[j * HC + lane] : 1.f);
+                }
+            }
+        }
+        __syncthreads();
+
+        // 4. Stages of checkpoint rows: fold, store checkpoint and read copy, dot with C.
+        const int q = tid % Q, rg = tid / Q;
+        int failed = -1;  // stage whose copy never landed
+        for (int c = 0; c < nst; ++c) {
+            const int k = (gs + c) % kFoldStages;
+            const bool got = mbar_wait(&bar[k], ((gs + c) / kFoldStages) & 1);
             if (__syncthreads_or(!got)) {
-                timed_out = true;
+                failed = c;
                 break;
             }
-            const float *tf = fbuf + (c & 1) * (FC * N);
-            float4 v[FH];
-            int gr[FH];
+            const int gr0 = c * FC + 4 * rg;  // first of this thread's 4 rows (one head: P % 4 == 0)
+            const bool valid = gr0 < nrows;
+            const int hh = valid ? gr0 / P : 0, p0 = gr0 - hh * P;
+            const float *tf = stg + k * (FC * N) + (4 * rg) * N + 4 * q;
+            const float dc = sfdec[hh];
+            float4 v[4];
 #pragma unroll
-            for (int k = 0; k < FH; ++k) {
-                const int rl = q0 + k * RPP4;
-                gr[k] = c * FC + rl;
-                v[k] = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (gr[k] < nrows) {
-                    v[k] = *reinterpret_cast<const float4 *>(tf + rl * N + 4 * c4);
-                    const float dc = sfdec[gr[k] / P];
-                    v[k].x *= dc; v[k].y *= dc; v[k].z *= dc; v[k].w *= dc;
+            for (int i = 0; i < 4; ++i) {
+                v[i] = valid ? *reinterpret_cast<const float4 *>(tf + i * N) : make_float4(0.f, 0.f, 0.f, 0.f);
+                v[i].x *= dc; v[i].y *= dc; v[i].z *= dc; v[i].w *= dc;
+            }
+            if (valid) {
+                const float *Ur = U + (hh * L0) * P + p0;
+                const float *Br = Bf + 4 * q;
+#pragma unroll 2
+                for (int e = 0; e < L0; ++e) {
+                    const float4 u = *reinterpret_cast<const float4 *>(Ur + e * P);
+                    const float4 bb = *reinterpret_cast<const float4 *>(Br + e * N);
+                    v[0].x = fmaf(u.x, bb.x, v[0].x); v[0].y = fmaf(u.x, bb.y, v[0].y);
+                    v[0].z = fmaf(u.x, bb.z, v[0].z); v[0].w = fmaf(u.x, bb.w, v[0].w);
+                    v[1].x = fmaf(u.y, bb.x, v[1].x); v[1].y = fmaf(u.y, bb.y, v[1].y);
+                    v[1].z = fmaf(u.y, bb.z, v[1].z); v[1].w = fmaf(u.y, bb.w, v[1].w);
+                    v[2].x = fmaf(u.z, bb.x, v[2].x); v[2].y = fmaf(u.z, bb.y, v[2].y);
+                    v[2].z = fmaf(u.z, bb.z, v[2].z); v[2].w = fmaf(u.z, bb.w, v[2].w);
+                    v[3].x = fmaf(u.w, bb.x, v[3].x); v[3].y = fmaf(u.w, bb.y, v[3].y);
+                    v[3].z = fmaf(u.w, bb.z, v[3].z); v[3].w = fmaf(u.w, bb.w, v[3].w);
                 }
             }
-            for (int eb = 0; eb < L0; eb += FB) {
-                float4 Bq[FB];
+            __syncthreads();  // every thread has its rows: the stage buffer is free again
+            if (tid == 0 && c + kFoldStages < nst) issue(c + kFoldStages);
 #pragma unroll
-                for (int j = 0; j < FB; ++j) {
-                    const uint8_t *Br = B_of(eb + j) + 4 * c4 * IB;
-                    Bq[j] = (eb + j < L0) ? make_float4(ldx(Br), ldx(Br + IB), ldx(Br + 2 * IB), ldx(Br + 3 * IB))
-                                          : make_float4(0.f, 0.f, 0.f, 0.f);
-                }
-#pragma unroll
-                for (int k = 0; k < FH; ++k) {
-                    if (gr[k] >= nrows) continue;
-                    const int hh = gr[k] / P, p = gr[k] - hh * P;
-                    const uint8_t *xr = sx + (hh * E + base + eb) * xrow + p * IB;
-                    const float *uw = su + hh * E + eb;
-#pragma unroll
-                    for (int j = 0; j < FB; ++j) {
-                        if (eb + j < L0) {
-                            const float w = uw[j] * ldx(xr + j * xrow);
-                            v[k].x = fmaf(w, Bq[j].x, v[k].x); v[k].y = fmaf(w, Bq[j].y, v[k].y);
-                            v[k].z = fmaf(w, Bq[j].z, v[k].z); v[k].w = fmaf(w, Bq[j].w, v[k].w);
-                        }
-                    }
-                }
-            }
-            __syncthreads();  // every thread has its rows of this stage in registers
-            if (tid == 0 && c + 2 < nfc) fold_issue(c + 2);
-#pragma unroll
-            for (int k = 0; k < FH; ++k) {
-                const bool valid = gr[k] < nrows;
-                const int64_t el = tile0 + (int64_t)(valid ? gr[k] : 0) * N + 4 * c4;
+            for (int i = 0; i < 4; ++i) {
+                const int gr = gr0 + i;
+                const int64_t el = tile0 + (int64_t)(valid ? gr : 0) * N + 4 * q;
                 if (a.op == OP_EXPORT) {
-                    if (valid) *reinterpret_cast<float4 *>(a.out + el) = v[k];
+                    if (valid) *reinterpret_cast<float4 *>(a.out + el) = v[i];
                     continue;
                 }
-                if (valid) *reinterpret_cast<float4 *>(a.ckpt + el) = v[k];
-                float4 rd = v[k];
+                if (valid) *reinterpret_cast<float4 *>(a.ckpt + el) = v[i];
+                float4 rd = v[i];
                 if (RK == SK_BF16) {
-                    if (valid) rd = store_quad<SK_BF16>(a.rc, el, v[k], 0.f, 0.f);
+                    if (valid) rd = store_quad<SK_BF16>(a.rc, el, v[i], 0.f, 0.f);
                 } else if (RK == SK_FP8) {
-                    float am = fmaxf(fmaxf(fabsf(v[k].x), fabsf(v[k].y)), fmaxf(fabsf(v[k].z), fabsf(v[k].w)));
-                    am = group_max<TPR4>(am);
+                    float am = fmaxf(fmaxf(fabsf(v[i].x), fabsf(v[i].y)), fmaxf(fabsf(v[i].z), fabsf(v[i].w)));
+                    am = group_max<Q>(am);
                     const float sc = fp8_scale(am);
                     if (valid) {
-                        rd = store_quad<SK_FP8>(a.rc, el, v[k], 0.f, sc);
-                        if (c4 == 0) a.rc_scale[row0 * P + gr[k]] = sc;
+                        rd = store_quad<SK_FP8>(a.rc, el, v[i], 0.f, sc);
+                        if (q == 0) a.rc_scale[row0 * P + gr] = sc;
                     }
                 }
                 if (reads) {
 #pragma unroll
                     for (int m = 0; m < TQ; ++m) {
-                        const float4 Cq = *reinterpret_cast<const float4 *>(sCf + m * N + 4 * c4);
+                        const float4 Cq = *reinterpret_cast<const float4 *>(sCf + m * N + 4 * q);
                         float d = rd.x * Cq.x + rd.y * Cq.y + rd.z * Cq.z + rd.w * Cq.w;
-                        d = group_sum<TPR4>(d);
-                        if (c4 == 0 && valid && m < T) sdot[gr[k] * TQ + m] = d;
+                        d = group_sum<Q>(d);
+                        if (q == 0 && valid && m < T) sdot[gr * TQ + m] = d;
                     }
                 }
             }
         }
-        if (timed_out) {  // a checkpoint copy never landed: reported, sequence left as it was
-            if (tid == 0) report(a.c.err, DEV_PIPE_TIMEOUT, b, h0, 0);
+        if (failed >= 0) {
+            // A checkpoint copy never landed: report, let the copies still in
+            // flight (stages failed .. failed + 2) land, bounded, and stop.
+            if (tid == 0) {
+                report(a.c.err, DEV_PIPE_TIMEOUT, b, h0, 0);
+                for (int c = failed; c < nst && c < failed + kFoldStages; ++c)
+                    mbar_wait(&bar[(gs + c) % kFoldStages], ((gs + c) / kFoldStages) & 1);
+            }
             return;
         }
+        gs += nst;
         if (reads) {
             __syncthreads();
             // Outputs of the folded sequence: the fresh copy plus the call's own tokens.
@@ -383,43 +550,16 @@ __global__ void __launch_bounds__(kThreads, 3) m2_prep_kernel(const M2Args a) {
                 const int hh = r2 / P, p = r2 - hh * P;
                 float yv = sdec[hh * TQ + m] * sdot[r2 * TQ + m];
                 const float *cf = scoef + (hh * TQ + m) * E;
-                const uint8_t *xs = sx + (hh * E + base) * xrow + p * IB;
-                for (int e = e0; e <= L0 + m; ++e) yv = fmaf(cf[e], ldx(xs + e * xrow), yv);
-                yv = fmaf(a.D[h0 + hh], ldx(sx + (hh * E + W + m) * xrow + p * IB), yv);
+                const uint8_t *xs = sx + (hh * E + W) * xrow + p * IB;  // the call's tokens
+                for (int j = 0; j <= m; ++j) yv = fmaf(cf[L0 + j], ldx(xs + j * xrow), yv);
+                yv = fmaf(a.D[h0 + hh], ldx(xs + m * xrow), yv);
                 a.y[((int64_t)(b * T + m) * H + h0 + hh) * P + p] = yv;
             }
         }
+        if (tid == 0 && a.op == OP_FLUSH)  // flush publishes the sequence's counters here
+            arrive_and_publish(a.c, b, chunks, -1, ss.seq, -1, 1);
+        __syncthreads();  // shared memory is restaged by the next item
     }
-
-    // 5. Append the call's tokens to the ring (slots seq_pos + m mod R).
-    if (reads) {
-        for (int row = warp; row < T * HC; row += kWarps) {
-            const int m = row / HC, hh = row - m * HC;
-            const int slot = spmod + m >= R ? spmod + m - R : spmod + m;
-            uint8_t *dst = reinterpret_cast<uint8_t *>(a.xbuf) + (((row0 + hh) * R + slot) * P) * IB;
-            const uint8_t *src = sx + (hh * E + W + m) * xrow;
-            for (int k = lane; k < xch; k += 32)
-                *reinterpret_cast<uint4 *>(dst + k * 16) = *reinterpret_cast<const uint4 *>(src + k * 16);
-        }
-        for (int i = tid; i < T * HC; i += kThreads) {
-            const int m = i / HC, hh = i - m * HC;
-            const int slot = spmod + m >= R ? spmod + m - R : spmod + m;
-            a.dtbuf[(row0 + hh) * Rs + slot] = dtn[m * HC + hh];
-        }
-        if (hc == 0) {  // the group's first chunk writes the group's B
-            for (int row = warp; row < T; row += kWarps) {
-                const int slot = spmod + row >= R ? spmod + row - R : spmod + row;
-                uint8_t *dst = reinterpret_cast<uint8_t *>(a.Bbuf) + (((int64_t)(b * G + g) * R + slot) * N) * IB;
-                for (int k = lane; k < bch; k += 32)
-                    *reinterpret_cast<uint4 *>(dst + k * 16) = *reinterpret_cast<const uint4 *>(sBn + row * brow + k * 16);
-            }
-        }
-    }
-    // 6. Flush: this CTA read the counters long ago; its arrival lets the last CTA
-    //    of the sequence publish them.  (Decode and verify publish from the read
-    //    kernel, which runs after every prep CTA has read them.)
-    if (tid == 0 && a.op == OP_FLUSH)
-        arrive_and_publish(a.c, b, G * a.cpg, -1, flush ? ss.seq : -1, -1, flush);
 }
 
 // ---------------------------------------------------------------------------
@@ -536,12 +676,29 @@ __global__ void __launch_bounds__(kThreads) m2_eager_kernel(const M2Args a) {
 // ---------------------------------------------------------------------------
 // Host launchers.
 // ---------------------------------------------------------------------------
-template <int N, int RK, int TQ>
-inline cudaError_t launch_replay_t(const M2Args &a, size_t smem, cudaStream_t st) {
-    auto k = a.in_bf16 ? m2_prep_kernel<N, RK, TQ, true> : m2_prep_kernel<N, RK, TQ, false>;
+enum M2Kernel : int { M2_EAGER = 0, M2_PREP = 1, M2_FOLD = 2 };
+
+template <int N, int TQ>
+inline cudaError_t launch_prep_t(const M2Args &a, size_t smem, cudaStream_t st) {
+    auto k = a.in_bf16 ? m2_prep_kernel<N, TQ, true> : m2_prep_kernel<N, TQ, false>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     k<<<dim3(a.H / a.HC, a.B), kThreads, smem, st>>>(a);
+    return cudaGetLastError();
+}
+
+// The flush kernel is persistent: min(work items, resident CTAs) CTAs.
+template <int N, int RK, int TQ>
+inline cudaError_t launch_fold_t(const M2Args &a, const M2FoldLay &lay, int num_sms, cudaStream_t st) {
+    auto k = a.in_bf16 ? m2_fold_kernel<N, RK, TQ, true> : m2_fold_kernel<N, RK, TQ, false>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, lay.bytes);
+    if (e != cudaSuccess) return e;
+    int occ = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k, kThreads, lay.bytes);
+    if (e != cudaSuccess) return e;
+    const int items = a.B * (a.H / a.HC);
+    const int grid = items < num_sms * (occ > 0 ? occ : 1) ? items : num_sms * (occ > 0 ? occ : 1);
+    k<<<grid, kThreads, lay.bytes, st>>>(a, lay);
     return cudaGetLastError();
 }
 
@@ -555,24 +712,30 @@ inline cudaError_t launch_eager_t(const M2Args &a, size_t smem, cudaStream_t st)
 }
 
 template <int N, int TQ>
-inline cudaError_t dispatch_rk(bool eager, int rk, const M2Args &a, size_t smem, cudaStream_t st) {
+inline cudaError_t dispatch_rk(int which, int rk, const M2Args &a, const M2FoldLay &lay, size_t smem, int num_sms,
+                               cudaStream_t st) {
+    if (which == M2_PREP) return launch_prep_t<N, TQ>(a, smem, st);
     switch (rk) {
-        case SK_F32: return eager ? launch_eager_t<N, SK_F32, TQ>(a, smem, st) : launch_replay_t<N, SK_F32, TQ>(a, smem, st);
-        case SK_BF16: return eager ? launch_eager_t<N, SK_BF16, TQ>(a, smem, st) : launch_replay_t<N, SK_BF16, TQ>(a, smem, st);
-        default: return eager ? launch_eager_t<N, SK_FP8, TQ>(a, smem, st) : launch_replay_t<N, SK_FP8, TQ>(a, smem, st);
+        case SK_F32:
+            return which == M2_EAGER ? launch_eager_t<N, SK_F32, TQ>(a, smem, st)
+                                     : launch_fold_t<N, SK_F32, TQ>(a, lay, num_sms, st);
+        case SK_BF16:
+            return which == M2_EAGER ? launch_eager_t<N, SK_BF16, TQ>(a, smem, st)
+                                     : launch_fold_t<N, SK_BF16, TQ>(a, lay, num_sms, st);
+        default:
+            return which == M2_EAGER ? launch_eager_t<N, SK_FP8, TQ>(a, smem, st)
+                                     : launch_fold_t<N, SK_FP8, TQ>(a, lay, num_sms, st);
     }
-}
-template <int N>
-inline cudaError_t dispatch_tq(bool eager, int rk, int TQ, const M2Args &a, size_t smem, cudaStream_t st) {
-    if (TQ == 1) return dispatch_rk<N, 1>(eager, rk, a, smem, st);
-    if (TQ == 4) return dispatch_rk<N, 4>(eager, rk, a, smem, st);
-    return dispatch_rk<N, 8>(eager, rk, a, smem, st);
 }
 
 // Per-dstate entry points; each instantiation lives in its own translation unit.
+// which: M2Kernel; lay: flush kernel shared memory (M2_FOLD); smem: the others'.
 template <int N>
-cudaError_t m2_dispatch_n(bool eager, int rk, int TQ, const M2Args &a, size_t smem, cudaStream_t st) {
-    return dispatch_tq<N>(eager, rk, TQ, a, smem, st);
+cudaError_t m2_dispatch_n(int which, int rk, int TQ, const M2Args &a, const M2FoldLay &lay, size_t smem,
+                          int num_sms, cudaStream_t st) {
+    if (TQ == 1) return dispatch_rk<N, 1>(which, rk, a, lay, smem, num_sms, st);
+    if (TQ == 4) return dispatch_rk<N, 4>(which, rk, a, lay, smem, num_sms, st);
+    return dispatch_rk<N, 8>(which, rk, a, lay, smem, num_sms, st);
 }
 
 }  // namespace rssm

@@ -2,5 +2,5 @@
 #include "rssm_mamba2.cuh"
 
 namespace rssm {
-template cudaError_t m2_dispatch_n<16>(bool, int, int, const M2Args &, size_t, cudaStream_t);
+template cudaError_t m2_dispatch_n<16>(int, int, int, const M2Args &, const M2FoldLay &, size_t, int, cudaStream_t);
 }  // namespace rssm

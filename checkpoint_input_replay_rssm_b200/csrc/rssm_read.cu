@@ -55,6 +55,7 @@ cudaError_t launch_read(const Ctx &h, int op, int T, const void *Q, int q_bf16, 
     r.Emax = (cf.window + r.TQmax + 3) & ~3;
     r.y = y;
     r.c = h.counters();
+    r.fold_count = h.fold_count();
     r.op = op;
     const int TQ = tq_of_read(T);
     r.lay = read_lay(r.HC, cf.headdim, cf.dstate, cf.window, TQ, cf.input_dtype == RSSM_BF16 ? 2 : 4, r.Emax);

@@ -58,6 +58,7 @@ struct ReadArgs {
     const float *D;         // per-head skip (nullptr: none)
     const int4 *seqinfo;    // per sequence {L0 replayed from the ring, ring slot of entry 0, folded, valid}
     Counters c;             // published by the first CTA of each sequence
+    int *fold_count;        // flush kernel work-list length, reset here for the next call
     int op;                 // OP_DECODE | OP_VERIFY
     const float *dec;       // [B][H][TQmax]
     const float *coef;      // [B][H][TQmax][Emax]
@@ -119,6 +120,7 @@ __global__ void __launch_bounds__(kThreads, TQ == 1 ? 4 : 2) replay_read_kernel(
         sinfo[0] = si.x; sinfo[1] = si.y; sinfo[2] = si.z;
         // Counters of the sequence: every prep CTA has read them (the prep kernel
         // ran before this one), so the first CTA of the sequence rewrites them.
+        if (blockIdx.x == 0 && b == 0) *a.fold_count = 0;  // the flush kernel has run
         if (blockIdx.x == 0 && si.w) {
             const int64_t sp = a.c.seq_pos[b];
             if (si.z) {

@@ -122,7 +122,8 @@ typedef struct {
     size_t snap_off, snap_bytes;         /* EAGER: max_draft snapshots of the state (+ scales)      */
     /* REPLAY: hand-off from the prep kernel to the read kernel within one call */
     size_t tq_max;                       /* max(max_draft, 1): queries per call            */
-    size_t seqinfo_off, seqinfo_bytes;   /* int32[B][4]                                    */
+    size_t seqinfo_off, seqinfo_bytes;   /* int32[B][4] per sequence, then the flush kernel's
+                                            work list: int32 count, 3 pad, int32[B] (padded) */
     size_t dec_off, dec_bytes;           /* fp32[B][H][tq_max]                             */
     size_t coef_off, coef_bytes;         /* fp32[B][H][tq_max][window + tq_max, padded to 4] */
     size_t query_off, query_bytes;       /* GDN: fp32[B][H][tq_max][dstate] swept queries  */

@@ -184,3 +184,37 @@ def test_host_misuse_is_refused():
     L.commit(torch.zeros(wl.batch, dtype=torch.int32, device="cuda"))
     L.decode(dev1)
     assert L.status()[0] == 0
+
+
+def test_flush_kernel_launched_only_when_a_buffer_can_be_full():
+    """Plain decode from an empty buffer: the flush kernel runs exactly on the
+    calls that find the buffer full (every W-th), so those calls launch one
+    kernel more; counters changed behind the library's back so that a fold is
+    due when none was scheduled are reported, not silently mis-served."""
+    import torch
+
+    wl = _wl()
+    W = wl.window
+    L, _ = make_layer(wl, "replay", "bf16")
+    per_call = []
+    for t in range(2 * W + 1):
+        l0 = L.launches()
+        L.decode(to_device(I.token(wl, t), wl, with_T=False))
+        per_call.append(L.launches() - l0)
+    fold_calls = [t for t in range(2 * W + 1) if per_call[t] == per_call[0] + 1]
+    assert fold_calls == [W, 2 * W], per_call
+    assert L.counters()[3].tolist() == [2] * wl.batch
+    assert L.status()[0] == 0
+
+    L2, _ = make_layer(wl, "replay", "bf16")
+    for t in range(3):
+        L2.decode(to_device(I.token(wl, t), wl, with_T=False))
+    off = L2.layout.seq_pos_off
+    seq = L2.workspace[off:off + 8 * wl.batch].view(torch.int64)
+    seq[1] = W  # buffer of sequence 1 now claims W entries
+    y = torch.full((wl.batch, 1, wl.nheads, wl.headdim), 7.0, device="cuda")
+    L2.decode(to_device(I.token(wl, 3), wl, with_T=False), y=y)
+    st, info = L2.status()
+    assert st == rssm.RSSM_EDEVICE and info[0] == rssm.RSSM_DEV_BAD_COUNTERS and info[1] == 1
+    assert (y[1] == 7.0).all() and not (y[0] == 7.0).all()
+    assert L2.counters()[0].tolist() == [4, W, 4, 4]
