@@ -34,7 +34,7 @@ inline ReadLay read_lay(int HC, int P, int N, int W, int TQ, int ib, int Ep) {
     int o = 0;
     L.q = o;    o += al(HC * TQ * N * 4);     // queries as fp32   [HC or 1][TQ][N]
     L.x = o;    o += al(HC * E * P * ib);     // entries           [HC][E][P] raw
-    L.coef = o; o += al(HC * TQ * Ep * 4);    // coefficients      [HC][TQmax][Ep]
+    L.coef = o; o += al(HC * TQ * Ep * 4);    // coefficients      [HC][TQ][Ep]
     L.dec = o;  o += al(HC * TQ * 4);         // decays            [HC][TQ]
     L.dot = o;  o += al(HC * P * TQ * 4);     // S^ . Q per row    [HC*P][TQ]
     L.scale = o; o += al(HC * P * 4);         // fp8 row scales    [HC*P]
@@ -136,9 +136,12 @@ __global__ void __launch_bounds__(kThreads, TQ == 1 ? 4 : 2) replay_read_kernel(
         const uint8_t *src = reinterpret_cast<const uint8_t *>(a.xnew) + (((int64_t)(b * T + m) * H + h0 + hh) * P) * IB;
         for (int k = lane; k < xch; k += 32) cp_async16(sx + (hh * E + W + m) * xrow + k * 16, src + k * 16);
     }
-    {
-        const float *src = a.coef + row0 * a.TQmax * Ep;  // [HC][TQmax][Ep], contiguous
-        for (int i = tid; i < HC * a.TQmax * Ep / 4; i += kThreads) cp_async16(scoef + 4 * i, src + 4 * i);
+    {  // rows m < T of each head's [TQmax][Ep] table, to [HC][TQ][Ep]
+        const int per = T * Ep / 4;  // 16-byte chunks per head
+        for (int i = tid; i < HC * per; i += kThreads) {
+            const int hh = i / per, j = i - hh * per;
+            cp_async16(scoef + hh * TQ * Ep + 4 * j, a.coef + (row0 + hh) * a.TQmax * Ep + 4 * j);
+        }
     }
     for (int i = tid; i < HC * T; i += kThreads) {
         const int hh = i / T, m = i - hh * T;
@@ -228,7 +231,7 @@ __global__ void __launch_bounds__(kThreads, TQ == 1 ? 4 : 2) replay_read_kernel(
         const int m = i / nrows, r2 = i - m * nrows;
         const int hh = r2 / P, p = r2 - hh * P;
         float yv = sdec[hh * TQ + m] * sdot[r2 * TQ + m];
-        const float *cf = scoef + (hh * a.TQmax + m) * Ep;
+        const float *cf = scoef + (hh * TQ + m) * Ep;
         const uint8_t *xs = sx + (hh * E + base) * xrow + p * IB;
         for (int e = 0; e <= L0 + m; ++e) {
             const float xv = BF ? bf16_bits_to_float(*reinterpret_cast<const uint16_t *>(xs + e * xrow))

@@ -90,3 +90,54 @@ def test_spec_verify_gdn():
     _spec_run(wl, 14, list(range(6)), {"r32": ("replay", "f32"), "rbf": ("replay", "bf16"),
                                        "e32": ("eager", "f32")},
               {"r32": 1e-4, "rbf": 2e-2, "e32": 1e-4})
+
+
+def test_decode_and_short_verifies_on_a_deep_draft_handle():
+    """A handle sized for 8 drafts serving plain decodes and verifies of fewer
+    drafts (T below the handle's maximum), mixed, across folds: every output
+    against the eager fp64 oracle, counters against the ring model."""
+    import torch
+
+    wl = I.TINY.replace(batch=3, nheads=4, ngroups=2, headdim=24, dstate=32, window=8, steps=0,
+                        seed=61, max_draft=8, draft_k=8, input_dtype="bf16")
+    seqs = list(range(wl.batch))
+    layers = {n: make_layer(wl, mode="replay", state_dtype=sd)[0] for n, sd in (("f32", "f32"), ("bf16", "bf16"))}
+    tols = {"f32": 1e-4, "bf16": 2e-2}
+    c = I.constants(wl, seqs)
+    S_ref = np.ascontiguousarray(c["S0"].copy())
+    rm = RingModel(wl.batch, wl.window, wl.max_draft)
+    t = 0
+    rng = np.random.default_rng(5)
+    for op in ["d", "d", "d", 2, "d", 5, "d", "d", 1, "d", "d", "d", "d", "d", 3, "d", 8, "d"]:
+        if op == "d":
+            tok = I.token(wl, t); t += 1
+            ys = {n: L.decode(to_device(tok, wl, with_T=False)) for n, L in layers.items()}
+            y_ref = eager.step(wl.kind, S_ref, tok, oracle_params(c))
+            for n, y in ys.items():
+                assert rel_err(y[:, 0].double().cpu().numpy(), y_ref) <= tols[n], (n, op)
+            rm.decode()
+            continue
+        K = op
+        toks = I.tokens(wl, t, K); t += K
+        dev = to_device(toks, wl)
+        ys = {n: L.verify(K, dev) for n, L in layers.items()}
+        S_tmp = S_ref.copy()
+        states = []
+        for m in range(K):
+            y_m = eager.step(wl.kind, S_tmp, {k: v[:, m] for k, v in toks.items()}, oracle_params(c))
+            states.append(S_tmp.copy())
+            for n, y in ys.items():
+                assert rel_err(y[:, m].double().cpu().numpy(), y_m) <= tols[n], (n, op, m)
+        a = rng.integers(0, K + 1, wl.batch).astype(np.int32)
+        for L in layers.values():
+            L.commit(torch.tensor(a, device="cuda"))
+        rm.verify(K)
+        rm.commit(a)
+        for b in seqs:
+            if a[b] > 0:
+                S_ref[b] = states[a[b] - 1][b]
+    for n, L in layers.items():
+        sp, ck, pe, fc = L.counters()
+        assert np.array_equal(sp, rm.seq_pos) and np.array_equal(ck, rm.ckpt_pos), n
+        assert np.array_equal(fc, rm.flush_count), n
+        assert L.status()[0] == 0
