@@ -78,7 +78,11 @@ typedef enum { RSSM_F32 = 0, RSSM_BF16 = 1, RSSM_FP8E4M3 = 2 } rssm_dtype;
 typedef enum {
     RSSM_DEV_OK = 0,
     RSSM_DEV_BAD_ACCEPT = 1,  /* accept_len[b] < 0 or > pending[b]; treated as 0 */
-    RSSM_DEV_BAD_COUNTERS = 2 /* seq_pos - ckpt_pos outside [0, window]; sequence skipped */
+    RSSM_DEV_BAD_COUNTERS = 2, /* seq_pos - ckpt_pos outside [0, window], or a fold due that the
+                                  host did not schedule (counters changed outside the API);
+                                  sequence skipped */
+    RSSM_DEV_PIPE_TIMEOUT = 3  /* a bulk copy into shared memory did not complete within 2 s;
+                                  the kernel stopped and the sequence was left as it was */
 } rssm_device_error;
 
 typedef struct {
