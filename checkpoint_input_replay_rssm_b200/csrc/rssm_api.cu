@@ -138,6 +138,12 @@ cudaError_t launch_kind(Ctx *h, int op, int T, const rssm_inputs *in, float *y, 
 
 }  // namespace
 
+namespace rssm {
+rssm_status api_fail(Ctx *h, rssm_status st, const std::string &m) { return fail(h, st, m); }
+rssm_status api_cuda_fail(Ctx *h, cudaError_t e, const char *what) { return cuda_fail(h, e, what); }
+bool api_inputs_ok(const Ctx *h, const rssm_inputs *in) { return inputs_ok(h, in); }
+}  // namespace rssm
+
 extern "C" {
 
 size_t rssm_workspace_bytes(const rssm_config *cfg) {

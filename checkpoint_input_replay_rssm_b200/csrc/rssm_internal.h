@@ -11,6 +11,18 @@
 
 namespace rssm {
 
+// The prep kernel's per-call hand-off to the flush and read kernels: per
+// sequence {entries replayed, ring slot of entry 0, folded, valid}, the flush
+// kernel's work list, and the replay decays and coefficients.
+struct Handoff {
+    int4 *seqinfo;    // [B]
+    int *fold_count;  // one int32, zero between calls
+    int *fold_list;   // [B]
+    float *dec;       // [B][H][tq_max]
+    float *coef;      // [B][H][tq_max][Emax], Emax = window + tq_max rounded up to 4
+    int tq_max;
+};
+
 struct Ctx {
     rssm_config cfg;
     rssm_workspace_layout lay;
@@ -39,13 +51,26 @@ struct Ctx {
     // (int32 count, 3 pad words, then [batch] sequence indices).
     int *fold_count() const { return (int *)at(lay.seqinfo_off + (size_t)cfg.batch * 16); }
     int *fold_list() const { return fold_count() + 4; }
+    // The hand-off in the handle's workspace.
+    Handoff handoff() const {
+        Handoff o{};
+        if (!lay.seqinfo_bytes) return o;
+        o.seqinfo = (int4 *)at(lay.seqinfo_off);
+        o.fold_count = fold_count();
+        o.fold_list = fold_list();
+        o.dec = (float *)at(lay.dec_off);
+        o.coef = (float *)at(lay.coef_off);
+        o.tq_max = (int)lay.tq_max;
+        return o;
+    }
 };
 
 // Kernel launchers (one per layer kind).  op: Op; T tokens appended (0 for
 // flush/export); in/y used by decode/verify, out by export.  mamba2_launch
 // counts its launches and keeps the buffer-length bounds len_lb/len_ub.
+// ho: where the replay decode/verify hand-off lives (nullptr: the workspace's).
 cudaError_t mamba2_launch(Ctx &h, int op, int T, const rssm_inputs *in, float *y, float *out,
-                          cudaStream_t st);
+                          cudaStream_t st, const Handoff *ho = nullptr);
 size_t mamba2_smem_bytes(const rssm_config &cf, int T);
 cudaError_t gdn_launch(const Ctx &h, int op, int T, const rssm_inputs *in, float *y, float *out,
                        cudaStream_t st);
@@ -55,9 +80,14 @@ size_t gdn_smem_bytes(const rssm_config &cf, int T);
 // at the given element strides, q_group heads per query row.
 cudaError_t launch_read(const Ctx &h, int op, int T, const void *Q, int q_bf16, int q_group, int64_t q_stride_b,
                         int64_t q_stride_row, int64_t q_stride_m, const void *xnew, const float *D,
-                        float *y, cudaStream_t st);
+                        float *y, const Handoff &ho, cudaStream_t st);
 int read_heads_per_cta(const rssm_config &cf);
 size_t read_smem_bytes(const rssm_config &cf, int T);
+
+// Argument checks and error recording of the C ABI (rssm_api.cu).
+rssm_status api_fail(Ctx *h, rssm_status st, const std::string &m);
+rssm_status api_cuda_fail(Ctx *h, cudaError_t e, const char *what);
+bool api_inputs_ok(const Ctx *h, const rssm_inputs *in);
 
 // Kernels shared by both kinds (rssm_common.cu).
 cudaError_t launch_commit(const Ctx &h, const int32_t *accept, cudaStream_t st);

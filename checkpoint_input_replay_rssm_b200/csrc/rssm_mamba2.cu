@@ -55,20 +55,22 @@ static cudaError_t dispatch(int which, int N, int rk, int TQ, const M2Args &a, c
 // buffer may be too full for the call's tokens: len_ub + T > W), replay-read
 // kernel.  Flush/export: the
 // flush kernel over every sequence.  Eager: one kernel.
-cudaError_t mamba2_launch(Ctx &h, int op, int T, const rssm_inputs *in, float *y, float *out, cudaStream_t st) {
+cudaError_t mamba2_launch(Ctx &h, int op, int T, const rssm_inputs *in, float *y, float *out, cudaStream_t st,
+                          const Handoff *ho_in) {
+    const Handoff ho = ho_in ? *ho_in : h.handoff();
     M2Args a{};
     const rssm_config &cf = h.cfg;
     const int TQ = tq_of(T), ib = in_bytes(cf);
     a.B = cf.batch; a.H = cf.nheads; a.P = cf.headdim; a.G = cf.ngroups; a.W = cf.window;
     a.R = (int)h.lay.ring; a.Rs = (int)h.lay.ring_stride; a.T = T; a.op = op; a.in_bf16 = ib == 2;
     a.dt_scales = cf.dt_scales_input;
-    if (h.lay.seqinfo_bytes) {
-        a.seqinfo = (int4 *)h.at(h.lay.seqinfo_off);
-        a.fold_count = h.fold_count();
-        a.fold_list = h.fold_list();
-        a.dec = (float *)h.at(h.lay.dec_off);
-        a.coef = (float *)h.at(h.lay.coef_off);
-        a.TQmax = (int)h.lay.tq_max;
+    if (ho.seqinfo) {
+        a.seqinfo = ho.seqinfo;
+        a.fold_count = ho.fold_count;
+        a.fold_list = ho.fold_list;
+        a.dec = ho.dec;
+        a.coef = ho.coef;
+        a.TQmax = ho.tq_max;
         a.Emax = (cf.window + a.TQmax + 3) & ~3;
     }
     a.c = h.counters();
@@ -121,10 +123,10 @@ cudaError_t mamba2_launch(Ctx &h, int op, int T, const rssm_inputs *in, float *y
         const int G = cf.ngroups;
         h.launches += 1;
         e = launch_read(h, op, T, in->Cm, ib == 2, cf.nheads / G, (int64_t)T * G * N, N, (int64_t)G * N, in->x,
-                        (const float *)h.at(h.lay.D_off), y, st);
+                        (const float *)h.at(h.lay.D_off), y, ho, st);
     }
     if (e != cudaSuccess) {  // leave no stale work list behind
-        cudaMemsetAsync(h.fold_count(), 0, sizeof(int), st);
+        cudaMemsetAsync(ho.fold_count, 0, sizeof(int), st);
         return e;
     }
     // Committed lengths after this call (and the commit of a verify, which keeps

@@ -35,7 +35,7 @@ size_t read_smem_bytes(const rssm_config &cf, int T) {
 
 cudaError_t launch_read(const Ctx &h, int op, int T, const void *Q, int q_bf16, int q_group, int64_t q_stride_b,
                         int64_t q_stride_row, int64_t q_stride_m, const void *xnew, const float *D,
-                        float *y, cudaStream_t st) {
+                        float *y, const Handoff &ho, cudaStream_t st) {
     const rssm_config &cf = h.cfg;
     ReadArgs r{};
     r.B = cf.batch; r.H = cf.nheads; r.P = cf.headdim; r.R = (int)h.lay.ring; r.W = cf.window;
@@ -48,14 +48,14 @@ cudaError_t launch_read(const Ctx &h, int op, int T, const void *Q, int q_bf16, 
     r.xring = h.at(h.lay.xbuf_off);
     r.xnew = xnew;
     r.D = D;
-    r.seqinfo = (const int4 *)h.at(h.lay.seqinfo_off);
-    r.dec = (const float *)h.at(h.lay.dec_off);
-    r.coef = (const float *)h.at(h.lay.coef_off);
-    r.TQmax = (int)h.lay.tq_max;
+    r.seqinfo = ho.seqinfo;
+    r.dec = ho.dec;
+    r.coef = ho.coef;
+    r.TQmax = ho.tq_max;
     r.Emax = (cf.window + r.TQmax + 3) & ~3;
     r.y = y;
     r.c = h.counters();
-    r.fold_count = h.fold_count();
+    r.fold_count = ho.fold_count;
     r.op = op;
     const int TQ = tq_of_read(T);
     r.lay = read_lay(r.HC, cf.headdim, cf.dstate, cf.window, TQ, cf.input_dtype == RSSM_BF16 ? 2 : 4, r.Emax);

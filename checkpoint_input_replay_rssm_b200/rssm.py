@@ -58,6 +58,7 @@ SIGNATURES = {
     "rssm_import_state": (ctypes.c_int, [_VP, _VP]),
     "rssm_export_state": (ctypes.c_int, [_VP, _VP]),
     "rssm_decode": (ctypes.c_int, [_VP, _INP, _VP]),
+    "rssm_decode_static_scratch": (ctypes.c_int, [_VP, _INP, _VP]),
     "rssm_verify": (ctypes.c_int, [_VP, _I32, _INP, _VP]),
     "rssm_commit": (ctypes.c_int, [_VP, _VP]),
     "rssm_flush": (ctypes.c_int, [_VP]),
@@ -146,6 +147,10 @@ def rssm_export_state(h, S_ptr: int):
 
 def rssm_decode(h, inputs: rssm_inputs, y_ptr: int):
     _check(load().rssm_decode(h, ctypes.byref(inputs), y_ptr), h)
+
+
+def rssm_decode_static_scratch(h, inputs: rssm_inputs, y_ptr: int):
+    _check(load().rssm_decode_static_scratch(h, ctypes.byref(inputs), y_ptr), h)
 
 
 def rssm_verify(h, K: int, inputs: rssm_inputs, y_ptr: int):
@@ -262,6 +267,12 @@ class Layer:
         y = y if y is not None else self.torch.empty((self.B, 1, self.H, self.P),
                                                      dtype=self.torch.float32, device=self.device)
         rssm_decode(self.h, self._inputs(inputs), self._ptr(y))
+        return y
+
+    def decode_static_scratch(self, inputs: dict, y=None):
+        y = y if y is not None else self.torch.empty((self.B, 1, self.H, self.P),
+                                                     dtype=self.torch.float32, device=self.device)
+        rssm_decode_static_scratch(self.h, self._inputs(inputs), self._ptr(y))
         return y
 
     def verify(self, K: int, inputs: dict, y=None):

@@ -183,6 +183,19 @@ RSSM_API rssm_status rssm_export_state(rssm_handle h, float *S_out);
  * [B][1][H][P]) and commits the token. */
 RSSM_API rssm_status rssm_decode(rssm_handle h, const rssm_inputs *in, float *y);
 
+/* rssm_decode for REPLAY Mamba-2 layers with its per-call scratch (the prep
+ * kernel's hand-off to the flush and read kernels) in one library-owned static
+ * device array of 4 MiB instead of the handle's workspace: for callers that
+ * give each layer memory for its state only and decode the layers one after
+ * another on one stream.  The pages on checkpointed input replay have no
+ * counterpart; the results equal rssm_decode's.  Allocates nothing.  Refused
+ * (RSSM_EINVAL, nothing enqueued) for other layers and when the hand-off
+ * (about batch * nheads * (window + 4) * 4 bytes) exceeds the array.  All calls
+ * on a device share the array, so calls that may run concurrently race.  The
+ * first call on a device looks up the array's address; make one call before
+ * recording calls into a stream capture. */
+RSSM_API rssm_status rssm_decode_static_scratch(rssm_handle h, const rssm_inputs *in, float *y);
+
 /* Speculative verify of K drafts (1 <= K <= max_draft, K <= W) for every
  * sequence: folds where len + K > W, appends the drafts uncommitted and writes
  * y (device fp32 [B][K][H][P]), draft m seeing the committed tokens and drafts
