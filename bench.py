@@ -264,6 +264,30 @@ def run_reference(args, rank):
     print(json.dumps(line), flush=True)
 
 
+def rank_workload(rank: int, batch: int):
+    """The workload one rank decodes: the same layer shapes, its own sequences
+    (seeded per rank), so that N ranks run N independent batches."""
+    return WL.replace(seed=WL.seed + 7919 * rank, batch=batch)
+
+
+def max_over_ranks(dist, values, device):
+    """Element-wise max of per-rank timings (ms) over the process group; the
+    values themselves when there is no group."""
+    if dist is None:
+        return [float(v) for v in values]
+    import torch
+
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def job_tokens_per_s(world: int, batch: int, steps: int, ms: float) -> float:
+    """Whole-job throughput: every rank decoded `batch` sequences for `steps`
+    tokens, and the job took the slowest rank's time."""
+    return world * batch * steps / (ms * 1e-3)
+
+
 def workload_config(batch=None):
     return {"workload": WL.name, "batch_per_gpu": batch or WL.batch, "nheads": WL.nheads, "headdim": WL.headdim,
             "dstate": WL.dstate, "ngroups": WL.ngroups, "window": WL.window, "checkpoint": "f32",
@@ -320,7 +344,7 @@ def main():
     rssm.load()
 
     K, W = args.steps, args.warmup
-    wl = WL.replace(seed=WL.seed + 7919 * rank, batch=args.batch)
+    wl = rank_workload(rank, args.batch)
     consts = I.constants(wl, f64=False)
     n_distinct = min(K + W, 256)
     toks_host = host_tokens(wl, n_distinct)
@@ -335,20 +359,14 @@ def main():
     fold = [(W + i) >= wl.window and (W + i) % wl.window == 0 for i in range(K)]
     pick = lambda xs, want: [x for x, f in zip(xs, fold) if f == want]
     clocks = sampler.summary()
-    t = torch.tensor([total_ms, float(np.mean(read_ms)), float(np.mean(prep_ms))], dtype=torch.float64,
-                     device=device)
-    if dist is not None:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms, kern_ms, prep_avg = float(t[0]), float(t[1]), float(t[2])
+    total_ms, kern_ms, prep_avg = max_over_ranks(dist, [total_ms, float(np.mean(read_ms)), float(np.mean(prep_ms))],
+                                                 device)
     assert L.status()[0] == 0, "device error during the benchmark"
 
     # e2e through the public API with host buffers (fresh layer, same workload)
     L.import_state(torch.from_numpy(consts["S0"]).to(device))
     e2e_ms, h2d, d2h = e2e_loop(L, toks_host, K, W, sync)
-    t = torch.tensor([e2e_ms], dtype=torch.float64, device=device)
-    if dist is not None:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    e2e_ms = float(t[0])
+    (e2e_ms,) = max_over_ranks(dist, [e2e_ms], device)
 
     shape = traffic.Shape("mamba2", wl.headdim, wl.dstate, wl.nheads // wl.ngroups, wl.window, "bf16",
                           wl.input_dtype)
@@ -371,12 +389,9 @@ def main():
         torch.cuda.empty_cache()
         E = make_layer(wl, "eager", "f32", consts, device)
         e_total, e_per, _, _, _ = timed_loop(E, toks_dev, ys, K, W, sync, split=False)
-        t = torch.tensor([e_total, float(np.mean(e_per))], dtype=torch.float64, device=device)
-        if dist is not None:
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e_total, e_kern = float(t[0]), float(t[1])
+        e_total, e_kern = max_over_ranks(dist, [e_total, float(np.mean(e_per))], device)
         eg = traffic.eager_decode_per_token(shape, "f32")
-        eager = {"value": world * wl.batch * K / (e_total * 1e-3), "unit": "tokens/s",
+        eager = {"value": job_tokens_per_s(world, wl.batch, K, e_total), "unit": "tokens/s",
                  "ms_per_step": e_total / K,
                  "hbm_gbs": traffic.total(eg) * units / (e_kern * 1e-3) / 1e9,
                  "bytes_per_token_per_head": traffic.total(eg)}
@@ -386,7 +401,7 @@ def main():
         traffic.eager_decode_per_token(shape, "f32"))
     line = {
         "metric": METRIC,
-        "value": world * wl.batch * K / (total_ms * 1e-3),
+        "value": job_tokens_per_s(world, wl.batch, K, total_ms),
         "unit": "tokens/s",
         "n_gpus": world,
         "steps": K,
@@ -414,7 +429,7 @@ def main():
                         "ms_fold_call": float(np.mean(pick(prep_ms, True))) if any(fold) else None},
         "ms_per_call": {"nonfold": float(np.mean(pick(per, False))),
                         "fold": float(np.mean(pick(per, True))) if any(fold) else None},
-        "e2e": {"value": world * wl.batch * K / (e2e_ms * 1e-3), "unit": "tokens/s",
+        "e2e": {"value": job_tokens_per_s(world, wl.batch, K, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches,
         "clocks": clocks,
