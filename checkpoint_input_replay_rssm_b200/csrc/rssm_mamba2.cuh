@@ -35,7 +35,7 @@ constexpr int kFoldChunk = 16 * 1024;  // bytes of fp32 checkpoint rows per fold
 // Shared memory of the prep kernel (bytes, 16-byte aligned regions), computed on
 // the host.  The group's B ring is staged whole (R <= W + 8 rows).
 struct M2PrepLay {
-    int sC, sBr, sBn, sx, dring, dtn, sd, slam, si, bytes;
+    int sC, sBr, sBn, sx, dring, dtn, sA, sd, slam, si, bytes;
 };
 inline M2PrepLay m2_prep_lay(int HC, int P, int N, int W, int TQ, int ib) {
     const int E = W + TQ;
@@ -47,6 +47,7 @@ inline M2PrepLay m2_prep_lay(int HC, int P, int N, int W, int TQ, int ib) {
     L.sx = o;    o += a16(TQ * HC * P * ib);     // raw x of the call's tokens [TQ][HC][P]
     L.dring = o; o += a16(HC * dt_row_max_bytes(W));  // dt ring rows        [HC][Rs]
     L.dtn = o;   o += a16(TQ * HC * 4);          // dt of the call's tokens  [TQ][HC]
+    L.sA = o;    o += a16(HC * 4);               // A of the heads           [HC]
     L.sd = o;    o += a16(TQ * E * 4);           // B_e . C_m                [TQ][E]
     L.slam = o;  o += a16(HC * E * 4);           // prefix sums of dt*A      [HC][E]
     L.si = o;    o += 32;
@@ -97,7 +98,7 @@ struct M2Args {
 // the slots of the entries a fold reads are never among them (R >= W + T).
 // ---------------------------------------------------------------------------
 template <int N, int TQ, bool BF>
-__global__ void __launch_bounds__(kThreads, 4) m2_prep_kernel(const M2Args a) {
+__global__ void __launch_bounds__(kThreads, 6) m2_prep_kernel(const M2Args a) {
     constexpr int IB = BF ? 2 : 4;
     extern __shared__ __align__(128) uint8_t smraw[];
     const M2PrepLay &Ly = a.lay;
@@ -111,6 +112,7 @@ __global__ void __launch_bounds__(kThreads, 4) m2_prep_kernel(const M2Args a) {
     uint8_t *sC = smraw + Ly.sC, *sBr = smraw + Ly.sBr, *sBn = smraw + Ly.sBn, *sx = smraw + Ly.sx;
     float *dring = reinterpret_cast<float *>(smraw + Ly.dring);
     float *dtn = reinterpret_cast<float *>(smraw + Ly.dtn);
+    float *sA = reinterpret_cast<float *>(smraw + Ly.sA);
     float *sd = reinterpret_cast<float *>(smraw + Ly.sd);
     float *slam = reinterpret_cast<float *>(smraw + Ly.slam);
     int *si = reinterpret_cast<int *>(smraw + Ly.si);
@@ -170,6 +172,7 @@ __global__ void __launch_bounds__(kThreads, 4) m2_prep_kernel(const M2Args a) {
         const int m = i / HC, hh = i - m * HC;
         dtn[m * HC + hh] = a.dt[(int64_t)(b * T + m) * H + h0 + hh];
     }
+    for (int i = tid; i < HC; i += kThreads) sA[i] = a.A[h0 + i];
     cp_async_wait_all();
     __syncthreads();
     if (!si[0]) return;  // counters corrupted: reported, sequence skipped
@@ -178,21 +181,39 @@ __global__ void __launch_bounds__(kThreads, 4) m2_prep_kernel(const M2Args a) {
     auto slot_of = [&](int e) { const int s = ckmod + e; return s >= R ? s - R : s; };
 
     if (!fold) {
-        // 2. B_e . C_m once for the group (warps).
-        for (int pr = warp; pr < T * nE; pr += kWarps) {
-            const int m = pr / nE, e = pr - m * nE;
-            if (e > L0 + m) continue;  // warp-uniform
-            const uint8_t *Bp = e < L0 ? sBr + slot_of(e) * brow : sBn + (e - L0) * brow;
-            const uint8_t *Cp = sC + m * brow;
-            float d = 0.f;
-            for (int n = lane; n < N; n += 32) d = fmaf(ldx(Bp + n * IB), ldx(Cp + n * IB), d);
-            d = group_sum<32>(d);
-            if (lane == 0) sd[m * E + e] = d;
+        // 2. B_e . C_m once for the group: a row is bch 16-byte chunks, one lane
+        //    each, so a warp takes 32 / bch dots at a time.
+        {
+            const int dpw = 32 / bch, dl = lane / bch, c = lane - dl * bch;
+            const int ndots = T * nE;
+            for (int pr0 = warp * dpw; pr0 < ndots; pr0 += kWarps * dpw) {  // warp-uniform
+                const int pr = pr0 + dl;
+                const int m = pr / nE, e = pr - m * nE;
+                float d = 0.f;
+                if (pr < ndots && e <= L0 + m) {
+                    const uint8_t *Bp = e < L0 ? sBr + slot_of(e) * brow : sBn + (e - L0) * brow;
+                    const uint4 bu = *reinterpret_cast<const uint4 *>(Bp + c * 16);
+                    const uint4 cu = *reinterpret_cast<const uint4 *>(sC + m * brow + c * 16);
+                    if (BF) {
+                        const uint32_t bw[4] = {bu.x, bu.y, bu.z, bu.w}, cw[4] = {cu.x, cu.y, cu.z, cu.w};
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            d = fmaf(bf16_bits_to_float(bw[k] & 0xFFFFu), bf16_bits_to_float(cw[k] & 0xFFFFu), d);
+                            d = fmaf(__uint_as_float(bw[k] & 0xFFFF0000u), __uint_as_float(cw[k] & 0xFFFF0000u), d);
+                        }
+                    } else {
+                        d = __uint_as_float(bu.x) * __uint_as_float(cu.x) + __uint_as_float(bu.y) * __uint_as_float(cu.y) +
+                            __uint_as_float(bu.z) * __uint_as_float(cu.z) + __uint_as_float(bu.w) * __uint_as_float(cu.w);
+                    }
+                }
+                for (int o = bch / 2; o > 0; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
+                if (c == 0 && pr < ndots && e <= L0 + m) sd[m * E + e] = d;
+            }
         }
         __syncthreads();
         // 3. Per head (one warp): prefix sums of dt*A, coefficients, decays.
         for (int hh = warp; hh < HC; hh += kWarps) {
-            const float Ah = a.A[h0 + hh];
+            const float Ah = sA[hh];
             float *lam = slam + hh * E;
             float carry = 0.f;
             for (int k0 = 0; k0 < nE; k0 += 32) {
