@@ -110,7 +110,7 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ setup
-def make_layer(wl, mode, state_dtype, consts, device):
+def make_layer(wl, mode, state_dtype, consts, device, max_draft=1):
     import torch
 
     from checkpoint_input_replay_rssm_b200 import rssm
@@ -118,12 +118,107 @@ def make_layer(wl, mode, state_dtype, consts, device):
     cfg = rssm.make_config(kind=wl.kind, mode=mode, state_dtype=state_dtype,
                            input_dtype=wl.input_dtype, batch=wl.batch, nheads=wl.nheads,
                            headdim=wl.headdim, dstate=wl.dstate, ngroups=wl.ngroups,
-                           window=wl.window, max_draft=1)
+                           window=wl.window, max_draft=max_draft)
     L = rssm.Layer(cfg, device=device)
-    L.set_params(torch.tensor(consts["A"], dtype=torch.float32, device=device),
-                 torch.tensor(consts["D"], dtype=torch.float32, device=device))
+    if wl.kind == "mamba2":
+        L.set_params(torch.tensor(consts["A"], dtype=torch.float32, device=device),
+                     torch.tensor(consts["D"], dtype=torch.float32, device=device))
     L.import_state(torch.from_numpy(consts["S0"]).to(device))
     return L
+
+
+def device_tokens(wl, tok, device, with_T):
+    """One seeded token dict (numpy float64) as device tensors in storage dtypes."""
+    wide = ("x", "B", "C", "q", "k", "v")
+    out = {}
+    for k, v in tok.items():
+        t = I.to_torch(v, wl.input_dtype if k in wide else "f32")
+        out[k] = (t if with_T else t.unsqueeze(1)).contiguous().to(device)
+    return out
+
+
+def spec_leg(rank, device, sync, dist, world, rounds, warmup):
+    """Speculative verify + commit on the 512-sequence, 128-head Mamba-2 layer with K = 4
+    drafts and seeded accept lengths a ~ U{0..4}: committed tokens/s, replay (bf16 copy)
+    and the eager snapshot baseline (fp32 state, K snapshots per round)."""
+    import torch
+
+    wl = I.SPECVERIFY.replace(seed=I.SPECVERIFY.seed + 7919 * rank)
+    K = wl.draft_k
+    consts = I.constants(wl, f64=False)
+    n = min(rounds + warmup, 16)
+    toks = [device_tokens(wl, I.tokens(wl, r * K, K), device, True) for r in range(n)]
+    acc = [torch.tensor(I.accept_lengths(wl, r), dtype=torch.int32, device=device) for r in range(n)]
+    kept = [int(a.sum()) for a in acc]
+    out = {}
+    for name, mode, sd in (("replay", "replay", "bf16"), ("eager", "eager", "f32")):
+        L = make_layer(wl, mode, sd, consts, device, max_draft=K)
+        y = torch.empty((wl.batch, K, wl.nheads, wl.headdim), dtype=torch.float32, device=device)
+        for r in range(warmup):
+            L.verify(K, toks[r % n], y=y)
+            L.commit(acc[r % n])
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        sync()
+        e0.record(L.stream)
+        committed = 0
+        for i in range(rounds):
+            r = (warmup + i) % n
+            L.verify(K, toks[r], y=y)
+            L.commit(acc[r])
+            committed += kept[r]
+        e1.record(L.stream)
+        sync()
+        assert L.status()[0] == 0, "device error in the speculative leg"
+        (ms,) = max_over_ranks(dist, [e0.elapsed_time(e1)], device)
+        out[name] = {"value": world * committed / (ms * 1e-3), "unit": "committed tokens/s",
+                     "ms_per_round": ms / rounds}
+        del L
+        torch.cuda.empty_cache()
+    out["config"] = {"workload": wl.name, "batch_per_gpu": wl.batch, "draft_k": K, "rounds": rounds,
+                     "accept": "U{0..K} per sequence and round, seeded", "read_copy": "bf16 (replay)",
+                     "eager_state": "f32 with K snapshots"}
+    out["speedup_vs_eager"] = out["replay"]["value"] / out["eager"]["value"]
+    return out
+
+
+def gdn_leg(rank, device, sync, dist, world, steps, warmup):
+    """Gated DeltaNet decode, 256 sequences x 32 heads x 128 x 128, W = 16: replay (bf16
+    copy) and eager (fp32) tokens/s, with the state bytes per token of each."""
+    import torch
+
+    wl = I.GDN.replace(seed=I.GDN.seed + 7919 * rank)
+    consts = I.constants(wl, f64=False)
+    n = min(steps + warmup, 32)
+    toks = [device_tokens(wl, I.token(wl, t), device, False) for t in range(n)]
+    out = {}
+    for name, mode, sd in (("replay", "replay", "bf16"), ("eager", "eager", "f32")):
+        L = make_layer(wl, mode, sd, consts, device)
+        y = torch.empty((wl.batch, 1, wl.nheads, wl.headdim), dtype=torch.float32, device=device)
+        for t in range(warmup):
+            L.decode(toks[t % n], y=y)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        sync()
+        e0.record(L.stream)
+        for i in range(steps):
+            L.decode(toks[(warmup + i) % n], y=y)
+        e1.record(L.stream)
+        sync()
+        assert L.status()[0] == 0, "device error in the GDN leg"
+        (ms,) = max_over_ranks(dist, [e0.elapsed_time(e1)], device)
+        out[name] = {"value": job_tokens_per_s(world, wl.batch, steps, ms), "unit": "tokens/s",
+                     "ms_per_step": ms / steps}
+        del L
+        torch.cuda.empty_cache()
+    shape = traffic.Shape("gdn", wl.headdim, wl.dstate, 1, wl.window, "bf16", wl.input_dtype)
+    rep, eg = traffic.replay_decode_per_token(shape), traffic.eager_decode_per_token(shape, "f32")
+    units = wl.batch * wl.nheads
+    out["replay"]["hbm_gbs"] = traffic.total(rep) * units * steps / (out["replay"]["ms_per_step"] * steps * 1e-3) / 1e9
+    out["eager"]["hbm_gbs"] = traffic.total(eg) * units * steps / (out["eager"]["ms_per_step"] * steps * 1e-3) / 1e9
+    out["state_bytes_per_token_per_head"] = {"replay": traffic.state_bytes(rep), "eager": traffic.state_bytes(eg),
+                                             "ratio": traffic.state_bytes(rep) / traffic.state_bytes(eg)}
+    out["config"] = {"workload": wl.name, "batch_per_gpu": wl.batch, "nheads": wl.nheads, "d_k": wl.dstate,
+                     "d_v": wl.headdim, "window": wl.window, "read_copy": "bf16", "inputs": wl.input_dtype}
+    return out
 
 
 def host_tokens(wl, n):
@@ -305,6 +400,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-eager", action="store_true", help="skip the eager-baseline leg")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle leg")
+    ap.add_argument("--no-spec", action="store_true", help="skip the speculative-verify leg")
+    ap.add_argument("--no-gdn", action="store_true", help="skip the Gated DeltaNet leg")
     ap.add_argument("--batch", type=int, default=WL.batch,
                     help="sequences per GPU (default: the workload's 256; smaller for profiling)")
     args = ap.parse_args()
@@ -397,6 +494,9 @@ def main():
                  "bytes_per_token_per_head": traffic.total(eg)}
         del E
 
+    spec = None if args.no_spec else spec_leg(rank, device, sync, dist, world, min(K, 64), W)
+    gdn = None if args.no_gdn else gdn_leg(rank, device, sync, dist, world, min(K, 128), W)
+
     state_rep, state_eag = traffic.state_bytes(rep), traffic.state_bytes(
         traffic.eager_decode_per_token(shape, "f32"))
     line = {
@@ -436,6 +536,8 @@ def main():
         "state_bytes_per_token_per_head": {"replay": state_rep, "eager": state_eag,
                                            "ratio": state_rep / state_eag},
         "eager": eager,
+        "spec_verify": spec,
+        "gdn": gdn,
     }
     if rank == 0 and world == 1 and not args.no_cpu:
         v, done, used, cores = oracle_tokens_per_s(wl, 64, 256, 12.0)

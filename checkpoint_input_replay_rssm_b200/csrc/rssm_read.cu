@@ -18,7 +18,7 @@ int read_heads_per_cta(const rssm_config &cf) {
     const int rcb = cf.state_dtype == RSSM_F32 ? 4 : (cf.state_dtype == RSSM_BF16 ? 2 : 1);
     const int qg = cf.kind == RSSM_MAMBA2 ? cf.nheads / cf.ngroups : 1;
     const int unit = qg > 1 ? qg : cf.nheads;  // heads a CTA may span
-    int want = (32 * 1024) / (cf.headdim * cf.dstate * rcb);
+    int want = (64 * 1024) / (cf.headdim * cf.dstate * rcb);
     if (want < 1) want = 1;
     int hc = 1;
     for (int d = 1; d <= unit && d <= want; ++d)

@@ -67,7 +67,9 @@ def replay_step_split(s: Shape, L0: int, fold: bool, T: int = 1) -> dict:
         prep["copy_write"] = state_tile(s, s.read_dtype) if s.read_dtype != "f32" else 0.0
         prep["output"] = T * s.headdim * 4
     else:
-        prep["handoff_write"] = T * ((L0 + T) * 4 + 4) + (T * s.dstate * 4 if s.kind == "gdn" else 0)
+        # Mamba-2 hands per-head coefficients to the read kernel; the Gated
+        # DeltaNet path is one kernel and hands nothing over
+        prep["handoff_write"] = T * ((L0 + T) * 4 + 4) if s.kind == "mamba2" else 0.0
         read = {
             "copy_read": state_tile(s, s.read_dtype),
             "buffer_read": L0 * x,
