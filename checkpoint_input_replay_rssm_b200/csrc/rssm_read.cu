@@ -12,13 +12,17 @@ extern template cudaError_t read_dispatch_n<128>(int, int, const ReadArgs &, siz
 
 static int tq_of_read(int T) { return T <= 1 ? 1 : (T <= 4 ? 4 : 8); }
 
-// Heads per read CTA: about 32 KiB of read copy per CTA, the heads sharing one
-// query row when a query row serves several heads (Mamba-2 groups).
+// Heads per read CTA: about 128 KiB of read copy per CTA, the heads sharing one
+// query row when a query row serves several heads (Mamba-2 groups).  A CTA
+// streams its rows in rounds of 8 x 16 bytes per thread and issues each round
+// before dotting the previous one, so its small operands' round trips overlap
+// the stream; on the 128-head layer 32 KiB gave 0.65 of peak bandwidth, 64 KiB
+// 0.76, 128 KiB 0.81, 256 KiB 0.48 (too few CTAs for the SMs).
 int read_heads_per_cta(const rssm_config &cf) {
     const int rcb = cf.state_dtype == RSSM_F32 ? 4 : (cf.state_dtype == RSSM_BF16 ? 2 : 1);
     const int qg = cf.kind == RSSM_MAMBA2 ? cf.nheads / cf.ngroups : 1;
     const int unit = qg > 1 ? qg : cf.nheads;  // heads a CTA may span
-    int want = (64 * 1024) / (cf.headdim * cf.dstate * rcb);
+    int want = (128 * 1024) / (cf.headdim * cf.dstate * rcb);
     if (want < 1) want = 1;
     int hc = 1;
     for (int d = 1; d <= unit && d <= want; ++d)
