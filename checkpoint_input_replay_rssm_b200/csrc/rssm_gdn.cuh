@@ -37,6 +37,15 @@ struct GArgs {
     const float *alpha, *beta;  // [B][T][H]
     float *y;                   // [B][T][H][P]
     float *out;                 // export target
+    // replay decode/verify: hand-off of the prep kernel to the read kernel
+    int4 *seqinfo;              // [B] {L0 replayed, ring slot of entry 0, folded, valid}
+    float *dec;                 // [B][H][TQmax] (1: the decays are inside the swept query)
+    float *coef;                // [B][H][TQmax][Emax] sweep coefficients c_e
+    float *query;               // [B][H][TQmax][N] swept queries r
+    int TQmax, Emax;
+    int fold_launched;          // the fold-only launch of gdn_replay_kernel follows in this call
+    int fold_only;              // gdn_replay_kernel: only fold (and serve) sequences whose buffer is full
+    int prep_heads;             // gdn_prep_kernel: heads (warps at work) per CTA, <= 8
 };
 
 __host__ __device__ constexpr int gpad4(int n) { return (n + 3) & ~3; }
@@ -149,14 +158,15 @@ __global__ void __launch_bounds__(kThreads) gdn_replay_kernel(const GArgs a) {
     const int64_t tile0 = (int64_t)bh * P * N;
     const bool reads = (a.op == OP_DECODE || a.op == OP_VERIFY);
 
-    // 1. Read-copy loads first (dropped on folding steps).
+    // 1. Read-copy loads first (dropped on folding steps; none in fold-only mode,
+    //    which serves only sequences that fold).
     const int c = tid % TPR, r0 = tid / TPR;
     const uint8_t *rc_tile =
         (RK == SK_F32) ? reinterpret_cast<const uint8_t *>(a.ckpt + tile0)
                        : reinterpret_cast<const uint8_t *>(a.rc) + tile0 * Chunk<RK>::BYTES;
     uint4 rv[RB];
     float rscale[RB];
-    if (reads) {
+    if (reads && !a.fold_only) {
 #pragma unroll
         for (int k = 0; k < RB; ++k) {
             const int r = r0 + k * RPP;
@@ -177,8 +187,8 @@ __global__ void __launch_bounds__(kThreads) gdn_replay_kernel(const GArgs a) {
         s.si[3] = (int)(ss.ckpt % R);
         s.si[4] = (int)(ss.seq % R);
         if (!ss.ok) {
-            if (h == 0) report(a.c.err, DEV_BAD_COUNTERS, b, h, (int)(ss.seq - ss.ckpt));
-        } else if (a.op != OP_EXPORT) {
+            if (h == 0 && !a.fold_only) report(a.c.err, DEV_BAD_COUNTERS, b, h, (int)(ss.seq - ss.ckpt));
+        } else if (a.op != OP_EXPORT && !a.fold_only) {
             const int64_t new_seq = (a.op == OP_DECODE) ? ss.seq + 1 : -1;
             const int64_t new_ckpt = flush ? ss.seq : -1;
             const int new_pending = (a.op == OP_VERIFY) ? T : -1;
@@ -189,6 +199,7 @@ __global__ void __launch_bounds__(kThreads) gdn_replay_kernel(const GArgs a) {
     __syncthreads();
     if (!s.si[0]) return;
     const int L0 = s.si[1], flush = s.si[2], ckmod = s.si[3], spmod = s.si[4];
+    if (a.fold_only && !flush) return;  // served by the prep and read kernels
     const int base = W - L0;
     const int nE = L0 + T;
     const int e0 = flush ? L0 : 0;
@@ -395,7 +406,8 @@ __global__ void __launch_bounds__(kThreads) gdn_replay_kernel(const GArgs a) {
         a.y[((int64_t)(b * T + m) * H + h) * P + p] = o;
     }
 
-    // 9. Append the new tokens to the ring.
+    // 9. Append the new tokens to the ring (fold-only mode: the prep kernel did).
+    if (a.fold_only) return;
     for (int i = tid; i < T * N; i += kThreads) {
         const int m = i / N, n = i - m * N;
         copy_in(a.kbuf, ((int64_t)bh * R + (spmod + m) % R) * N + n, a.k,
@@ -410,6 +422,143 @@ __global__ void __launch_bounds__(kThreads) gdn_replay_kernel(const GArgs a) {
         const int64_t slot = (int64_t)bh * a.Rs + (spmod + tid) % R;
         a.abuf[slot] = s.sal[W + tid];
         a.bbuf[slot] = s.sbe[W + tid];
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Prep kernel of a replay decode/verify: one CTA per (sequence, up to 8 heads),
+// one warp per head.  Thread 0 reads the sequence's counters; each warp stages its
+// head's buffered keys and gates and the call's k, q, then runs the backward
+// sweep for every query m (entries L0+m .. 0):
+//     c_e = beta_e (k_e . r),   r <- alpha_e (r - c_e k_e),   starting from r = q_m,
+// leaving the swept query r_m and the coefficients c for the read kernel,
+// which computes o_m = S^ r_m + sum_e c_e v_e (decay 1: it is inside r).
+// Sequences whose buffer must be folded first (len + T > W) are left to the
+// fold-only launch of gdn_replay_kernel.  Every sequence's tokens are appended
+// to the ring (slots seq_pos + m mod R, never an entry read in this call).
+// ---------------------------------------------------------------------------
+__host__ __device__ inline int gdn_prep_warp_bytes(int N, int W, int TQ, int ib) {
+    const int E = W + TQ;
+    return ((E + TQ) * N * ib + 2 * ((E + 3) & ~3) * 4 + 15) & ~15;
+}
+
+template <int N, int TQ, bool BF>
+__global__ void __launch_bounds__(kThreads) gdn_prep_kernel(const GArgs a) {
+    constexpr int IB = BF ? 2 : 4;
+    constexpr int NL = N >= 32 ? N / 32 : 1;  // key elements per lane (lanes >= N idle when N < 32)
+    extern __shared__ __align__(16) uint8_t gsm[];
+    __shared__ int si[6];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int H = a.H, P = a.P, W = a.W, R = a.R, T = a.T;
+    const int E = W + TQ, Ea = (E + 3) & ~3;
+    const int b = blockIdx.y, h = blockIdx.x * a.prep_heads + warp;
+    if (tid == 0) {
+        const SeqState ss = read_counters(a.c, b, W);
+        const int L0 = (int)(ss.seq - ss.ckpt);
+        const int fold = ss.ok && (L0 + T > W);
+        bool valid = ss.ok;
+        if (blockIdx.x == 0) {
+            if (!ss.ok) report(a.c.err, DEV_BAD_COUNTERS, b, 0, L0);
+            if (fold && !a.fold_launched) {  // the host's bound on buffer lengths was wrong
+                report(a.c.err, DEV_BAD_COUNTERS, b, 0, L0);
+                valid = false;
+            }
+            a.seqinfo[b] = valid ? make_int4(fold ? 0 : L0, (int)(ss.ckpt % R), fold, 1) : make_int4(0, 0, 1, 0);
+        }
+        si[0] = ss.ok;
+        si[1] = ss.ok ? L0 : 0;
+        si[2] = fold;
+        si[3] = (int)(ss.ckpt % R);
+        si[4] = (int)(ss.seq % R);
+    }
+    __syncthreads();
+    if (!si[0] || warp >= a.prep_heads || h >= H) return;
+    const int L0 = si[1], fold = si[2], ckmod = si[3], spmod = si[4];
+    const int64_t bh = (int64_t)b * H + h;
+    const int krow = N * IB, kch = krow / 16;
+    uint8_t *wk = gsm + warp * gdn_prep_warp_bytes(N, W, TQ, IB);  // k rows [E][N] raw
+    uint8_t *wq = wk + E * krow;                                   // q rows [TQ][N] raw
+    float *wal = reinterpret_cast<float *>(wq + TQ * krow);        // alpha [E]
+    float *wbe = wal + Ea;                                         // beta  [E]
+    auto run = [&](uint8_t *dst, const uint8_t *src, int n) {
+        for (int j = lane; j < n; j += 32) cp_async16(dst + 16 * j, src + 16 * j);
+    };
+    const uint8_t *kin = reinterpret_cast<const uint8_t *>(a.k), *qin = reinterpret_cast<const uint8_t *>(a.q);
+    for (int m = 0; m < T; ++m) {
+        const int64_t row = ((int64_t)b * T + m) * H + h;
+        run(wk + (L0 + m) * krow, kin + row * krow, kch);
+        run(wq + m * krow, qin + row * krow, kch);
+    }
+    if (!fold) {
+        const int n1 = min(L0, R - ckmod);
+        const uint8_t *kr = reinterpret_cast<const uint8_t *>(a.kbuf) + bh * R * krow;
+        run(wk, kr + ckmod * krow, n1 * kch);
+        run(wk + n1 * krow, kr, (L0 - n1) * kch);
+        for (int e = lane; e < L0; e += 32) {
+            const int s2 = ckmod + e >= R ? ckmod + e - R : ckmod + e;
+            wal[e] = a.abuf[bh * a.Rs + s2];
+            wbe[e] = a.bbuf[bh * a.Rs + s2];
+        }
+    }
+    if (lane < T) {
+        wal[L0 + lane] = a.alpha[((int64_t)b * T + lane) * H + h];
+        wbe[L0 + lane] = a.beta[((int64_t)b * T + lane) * H + h];
+    }
+    cp_async_wait_all();
+    __syncwarp();
+    auto lde = [&](const uint8_t *row, float (&v)[NL]) {  // this lane's NL elements of a raw row
+        if (NL * lane >= N) {
+#pragma unroll
+            for (int i = 0; i < NL; ++i) v[i] = 0.f;
+            return;
+        }
+#pragma unroll
+        for (int i = 0; i < NL; ++i) {
+            const uint8_t *q = row + (NL * lane + i) * IB;
+            v[i] = BF ? bf16_bits_to_float(*reinterpret_cast<const uint16_t *>(q)) : *reinterpret_cast<const float *>(q);
+        }
+    };
+    if (!fold) {
+        for (int m = 0; m < T; ++m) {
+            float r[NL];
+            lde(wq + m * krow, r);
+            float *crow = a.coef + (bh * a.TQmax + m) * a.Emax;
+            for (int e = L0 + m; e >= 0; --e) {
+                float kv[NL];
+                lde(wk + e * krow, kv);
+                float d = 0.f;
+#pragma unroll
+                for (int i = 0; i < NL; ++i) d = fmaf(kv[i], r[i], d);
+                d = group_sum<32>(d);
+                const float ce = wbe[e] * d, al = wal[e];
+#pragma unroll
+                for (int i = 0; i < NL; ++i) r[i] = al * fmaf(-ce, kv[i], r[i]);
+                if (lane == 0) crow[e] = ce;
+            }
+            if (NL * lane < N) {
+                float *qo = a.query + (bh * a.TQmax + m) * N + NL * lane;
+#pragma unroll
+                for (int i = 0; i < NL; ++i) qo[i] = r[i];
+            }
+            if (lane == 0) a.dec[bh * a.TQmax + m] = 1.f;
+        }
+    }
+    // Append the call's tokens: k from the staged rows, v straight from the
+    // inputs, the gates.
+    const int vch = P * IB / 16;
+    for (int m = 0; m < T; ++m) {
+        const int sl = spmod + m >= R ? spmod + m - R : spmod + m;
+        uint8_t *kd = reinterpret_cast<uint8_t *>(a.kbuf) + (bh * R + sl) * krow;
+        for (int j = lane; j < kch; j += 32)
+            *reinterpret_cast<uint4 *>(kd + 16 * j) = *reinterpret_cast<const uint4 *>(wk + (L0 + m) * krow + 16 * j);
+        uint8_t *vd = reinterpret_cast<uint8_t *>(a.vbuf) + (bh * R + sl) * P * IB;
+        const uint8_t *vs = reinterpret_cast<const uint8_t *>(a.v) + (((int64_t)b * T + m) * H + h) * P * IB;
+        for (int j = lane; j < vch; j += 32)
+            *reinterpret_cast<uint4 *>(vd + 16 * j) = *reinterpret_cast<const uint4 *>(vs + 16 * j);
+        if (lane == 0) {
+            a.abuf[bh * a.Rs + sl] = wal[L0 + m];
+            a.bbuf[bh * a.Rs + sl] = wbe[L0 + m];
+        }
     }
 }
 
@@ -538,6 +687,23 @@ inline cudaError_t gdispatch_tq(bool eager, int rk, int TQ, const GArgs &a, size
 template <int N>
 cudaError_t g_dispatch_n(bool eager, int rk, int TQ, const GArgs &a, size_t smem, cudaStream_t st) {
     return gdispatch_tq<N>(eager, rk, TQ, a, smem, st);
+}
+
+template <int N, int TQ>
+inline cudaError_t launch_gprep_t(const GArgs &a, cudaStream_t st) {
+    auto k = a.in_bf16 ? gdn_prep_kernel<N, TQ, true> : gdn_prep_kernel<N, TQ, false>;
+    const int smem = a.prep_heads * gdn_prep_warp_bytes(N, a.W, TQ, a.in_bf16 ? 2 : 4);
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    k<<<dim3((a.H + a.prep_heads - 1) / a.prep_heads, a.B), kThreads, smem, st>>>(a);
+    return cudaGetLastError();
+}
+
+template <int N>
+cudaError_t g_prep_dispatch_n(int TQ, const GArgs &a, cudaStream_t st) {
+    if (TQ == 1) return launch_gprep_t<N, 1>(a, st);
+    if (TQ == 4) return launch_gprep_t<N, 4>(a, st);
+    return launch_gprep_t<N, 8>(a, st);
 }
 
 }  // namespace rssm

@@ -3,4 +3,5 @@
 
 namespace rssm {
 template cudaError_t g_dispatch_n<128>(bool, int, int, const GArgs &, size_t, cudaStream_t);
+template cudaError_t g_prep_dispatch_n<128>(int, const GArgs &, cudaStream_t);
 }  // namespace rssm

@@ -20,6 +20,7 @@ struct Handoff {
     int *fold_list;   // [B]
     float *dec;       // [B][H][tq_max]
     float *coef;      // [B][H][tq_max][Emax], Emax = window + tq_max rounded up to 4
+    float *query;     // Gated DeltaNet: [B][H][tq_max][dstate] swept queries
     int tq_max;
 };
 
@@ -60,6 +61,7 @@ struct Ctx {
         o.fold_list = fold_list();
         o.dec = (float *)at(lay.dec_off);
         o.coef = (float *)at(lay.coef_off);
+        o.query = lay.query_bytes ? (float *)at(lay.query_off) : nullptr;
         o.tq_max = (int)lay.tq_max;
         return o;
     }
@@ -72,8 +74,25 @@ struct Ctx {
 cudaError_t mamba2_launch(Ctx &h, int op, int T, const rssm_inputs *in, float *y, float *out,
                           cudaStream_t st, const Handoff *ho = nullptr);
 size_t mamba2_smem_bytes(const rssm_config &cf, int T);
-cudaError_t gdn_launch(const Ctx &h, int op, int T, const rssm_inputs *in, float *y, float *out,
+cudaError_t gdn_launch(Ctx &h, int op, int T, const rssm_inputs *in, float *y, float *out,
                        cudaStream_t st);
+
+// Bounds of every sequence's committed buffer length after a replay decode or
+// verify of T tokens (a verify's commit keeps 0..T of them): a sequence that
+// folded holds its kept tokens, the others add them to what they had.
+inline void update_len_bounds(Ctx &h, int op, int T) {
+    const int W = h.cfg.window, kept_min = op == OP_DECODE ? T : 0;
+    if (h.len_lb + T > W) {          // every sequence folded
+        h.len_lb = kept_min;
+        h.len_ub = T;
+    } else if (h.len_ub + T <= W) {  // none did
+        h.len_lb += kept_min;
+        h.len_ub += T;
+    } else {                          // some may have
+        h.len_lb = kept_min;
+        h.len_ub = W;
+    }
+}
 size_t gdn_smem_bytes(const rssm_config &cf, int T);
 
 // The replay-read kernel (rssm_read.cu), shared by both kinds: queries Q[b][row][m][n]

@@ -129,20 +129,7 @@ cudaError_t mamba2_launch(Ctx &h, int op, int T, const rssm_inputs *in, float *y
         cudaMemsetAsync(ho.fold_count, 0, sizeof(int), st);
         return e;
     }
-    // Committed lengths after this call (and the commit of a verify, which keeps
-    // 0..T of its tokens): a sequence that folds holds its kept tokens, the others
-    // add them to what they had.
-    const int W = cf.window, kept_min = op == OP_DECODE ? T : 0;
-    if (h.len_lb + T > W) {          // every sequence folded
-        h.len_lb = kept_min;
-        h.len_ub = T;
-    } else if (h.len_ub + T <= W) {  // none did
-        h.len_lb += kept_min;
-        h.len_ub += T;
-    } else {                          // some may have
-        h.len_lb = kept_min;
-        h.len_ub = W;
-    }
+    update_len_bounds(h, op, T);
     return cudaSuccess;
 }
 
