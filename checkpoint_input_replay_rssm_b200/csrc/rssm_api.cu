@@ -160,6 +160,22 @@ rssm_status rssm_workspace_layout_of(const rssm_config *cfg, rssm_workspace_layo
     return RSSM_OK;
 }
 
+// Largest dynamic shared memory any kernel of this configuration asks for
+// (decode and verify query counts; flush and export use the decode layout).
+static size_t smem_need(const rssm_config &c) {
+    size_t need = 0;
+    const int Ts[2] = {1, c.max_draft > 1 ? c.max_draft : 1};
+    for (int T : Ts) {
+        const size_t k = c.kind == RSSM_MAMBA2 ? rssm::mamba2_smem_bytes(c, T) : rssm::gdn_smem_bytes(c, T);
+        if (k > need) need = k;
+        if (c.mode == RSSM_REPLAY) {
+            const size_t r = rssm::read_smem_bytes(c, T);
+            if (r > need) need = r;
+        }
+    }
+    return need;
+}
+
 rssm_status rssm_create(const rssm_config *cfg, void *workspace, size_t workspace_bytes,
                         void *stream, rssm_handle *out) {
     std::string why;
@@ -178,10 +194,20 @@ rssm_status rssm_create(const rssm_config *cfg, void *workspace, size_t workspac
     h->ws = (uint8_t *)workspace;
     h->ws_bytes = workspace_bytes;
     h->stream = (cudaStream_t)stream;
-    int dev = 0, sms = 0;
+    int dev = 0, sms = 0, optin = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e == cudaSuccess && sms > 0) h->num_sms = sms;
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    if (e == cudaSuccess && optin > 0) {
+        const size_t need = smem_need(*cfg);
+        if (need > (size_t)optin) {
+            g_create_error = "this shape's kernels need " + std::to_string(need) +
+                             " bytes of shared memory per CTA; the device allows " + std::to_string(optin);
+            delete h;
+            return RSSM_EINVAL;
+        }
+    }
     if (e == cudaSuccess) e = cudaMemsetAsync(h->ws, 0, L.total_bytes, h->stream);
     if (e != cudaSuccess) {
         g_create_error = std::string("zeroing the workspace: ") + cudaGetErrorString(e);

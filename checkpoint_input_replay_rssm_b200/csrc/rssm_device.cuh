@@ -201,7 +201,7 @@ __device__ __forceinline__ SeqState read_counters(const Counters &c, int b, int 
     s.seq = c.seq_pos[b];
     s.ckpt = c.ckpt_pos[b];
     const int64_t L = s.seq - s.ckpt;
-    s.ok = (L >= 0 && L <= W) ? 1 : 0;
+    s.ok = (s.ckpt >= 0 && L >= 0 && L <= W) ? 1 : 0;
     return s;
 }
 
@@ -229,6 +229,11 @@ namespace rssm {
 __device__ __forceinline__ void cp_async16(void *smem, const void *gmem) {
     const unsigned s = (unsigned)__cvta_generic_to_shared(smem);
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(s), "l"(gmem) : "memory");
+}
+// 4-byte global -> shared copy (cache-all variant; the 16-byte form is cache-global only).
+__device__ __forceinline__ void cp_async4(void *smem, const void *gmem) {
+    const unsigned s = (unsigned)__cvta_generic_to_shared(smem);
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(s), "l"(gmem) : "memory");
 }
 __device__ __forceinline__ void cp_async_wait_all() {
     asm volatile("cp.async.wait_all;" ::: "memory");

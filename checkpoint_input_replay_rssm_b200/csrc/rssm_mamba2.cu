@@ -24,10 +24,12 @@ static int m2_prep_heads(const rssm_config &cf, int TQ) {
 
 // Heads per flush CTA: up to 8 heads of one group, within 112 KiB of shared
 // memory (two CTAs per SM); a single head may take up to 200 KiB.
+static int ring_slots(const rssm_config &cf) { return cf.window + (cf.max_draft > 1 ? cf.max_draft : 1); }
 static int m2_fold_heads(const rssm_config &cf, int TQ) {
     const int hpg = cf.nheads / cf.ngroups;
     for (int hc = 8; hc > 1; --hc)
-        if (hpg % hc == 0 && m2_fold_lay(hc, cf.headdim, cf.dstate, cf.window, TQ, in_bytes(cf)).bytes <= 112 * 1024)
+        if (hpg % hc == 0 &&
+            m2_fold_lay(hc, cf.headdim, cf.dstate, cf.window, ring_slots(cf), TQ, in_bytes(cf)).bytes <= 112 * 1024)
             return hc;
     return 1;
 }
@@ -37,7 +39,7 @@ size_t mamba2_smem_bytes(const rssm_config &cf, int T) {
     if (cf.mode == RSSM_EAGER)
         return sizeof(float) * ((size_t)2 * pad4(TQ * P) + 2 * pad4(TQ * N) + 2 * pad4(TQ));
     const size_t prep = m2_prep_lay(m2_prep_heads(cf, TQ), P, N, cf.window, TQ, in_bytes(cf)).bytes;
-    const size_t fold = m2_fold_lay(m2_fold_heads(cf, TQ), P, N, cf.window, TQ, in_bytes(cf)).bytes;
+    const size_t fold = m2_fold_lay(m2_fold_heads(cf, TQ), P, N, cf.window, ring_slots(cf), TQ, in_bytes(cf)).bytes;
     return prep > fold ? prep : fold;
 }
 
@@ -96,7 +98,7 @@ cudaError_t mamba2_launch(Ctx &h, int op, int T, const rssm_inputs *in, float *y
         return dispatch(M2_EAGER, N, rk, TQ, a, flay, mamba2_smem_bytes(cf, T), h.num_sms, st);
     }
     const int fHC = m2_fold_heads(cf, TQ);
-    flay = m2_fold_lay(fHC, cf.headdim, N, cf.window, TQ, ib);
+    flay = m2_fold_lay(fHC, cf.headdim, N, cf.window, (int)h.lay.ring, TQ, ib);
     M2Args f = a;  // flush kernel arguments
     f.HC = fHC;
     f.cpg = (cf.nheads / cf.ngroups) / fHC;

@@ -274,36 +274,62 @@ __global__ void __launch_bounds__(kThreads, 6) m2_prep_kernel(const M2Args a) {
 // register block (4 consecutive rows x 4 columns) updated with two 128-bit
 // shared loads and 16 FMAs per entry.  The checkpoint rows arrive in 16 KiB
 // bulk-copy stages, three in flight; all waits are bounded.
+//
+// The kernel is persistent and each CTA walks a list of work items (sequence,
+// HC heads of one group).  Per item, everything small is staged in one round
+// trip that does not wait for the counters (the whole B, x and dt rings, the
+// call's tokens, A and D), and the prefix sums, fold weights and coefficients
+// take one barrier.  In a decode/verify every listed sequence folds, so the
+// checkpoint stages of a CTA's items form one stream: the next item's first
+// stages are issued while the current item's last stages are folded, and a
+// new item starts with its rows already landing.
 // ---------------------------------------------------------------------------
 struct M2FoldLay {
-    int stage, bar, sC, sBr, sBn, sx, dring, dtn, U, Bf, slam, su, scoef, sdec, sfdec, sCf, sdot, si, bytes;
+    int stage, bar, sC, sBr, sBn, sxr, sxn, dring, dtn, sA, sD, U, Bf, scoef, sdec, sfdec, sCf, sdot, si, bytes;
 };
 constexpr int kFoldStages = 3;
-inline M2FoldLay m2_fold_lay(int HC, int P, int N, int W, int TQ, int ib) {
-    const int E = W + TQ;
+// R: ring slots (W + max(max_draft, 1)).
+inline M2FoldLay m2_fold_lay(int HC, int P, int N, int W, int R, int TQ, int ib) {
     M2FoldLay L{};
     int o = 0;
     L.stage = o; o += kFoldStages * kFoldChunk;  // fp32 checkpoint rows
     L.bar = o;   o += 8 * kFoldStages;
     o = a16(o);
-    L.sC = o;    o += a16(TQ * N * ib);          // raw C of the queries       [TQ][N]
-    L.sBr = o;   o += a16((W + 8) * N * ib);     // raw B ring of the group    [R][N]
-    L.sBn = o;   o += a16(TQ * N * ib);          // raw B of the call's tokens [TQ][N]
-    L.sx = o;    o += a16(HC * E * P * ib);      // raw x of the entries       [HC][E][P]
-    L.dring = o; o += a16(HC * dt_row_max_bytes(W));  // dt ring rows          [HC][Rs]
-    L.dtn = o;   o += a16(TQ * HC * 4);          // dt of the call's tokens    [TQ][HC]
-    L.U = o;     o += a16(HC * W * P * 4);       // fold weights x rows        [HC][L0][P]
-    L.Bf = o;    o += a16(W * N * 4);            // committed B as fp32        [L0][N]
-    L.slam = o;  o += a16(HC * E * 4);           // prefix sums of dt*A        [HC][E]
-    L.su = o;    o += a16(HC * E * 4);           // fold weights               [HC][E]
-    L.scoef = o; o += a16(HC * TQ * E * 4);      // coefficients of the new tokens [HC][TQ][E]
-    L.sdec = o;  o += a16(HC * TQ * 4);          // decay of the fresh copy    [HC][TQ]
+    L.sC = o;    o += a16(TQ * N * ib);          // raw C of the queries        [TQ][N]
+    L.sBr = o;   o += a16(R * N * ib);           // raw B ring of the group     [R][N]
+    L.sBn = o;   o += a16(TQ * N * ib);          // raw B of the call's tokens  [TQ][N]
+    L.sxr = o;   o += a16(HC * R * P * ib);      // raw x ring of the heads     [HC][R][P]
+    L.sxn = o;   o += a16(TQ * HC * P * ib);     // raw x of the call's tokens  [TQ][HC][P]
+    L.dring = o; o += a16(HC * pad4(R) * 4);     // dt ring rows                [HC][Rs]
+    L.dtn = o;   o += a16(TQ * HC * 4);          // dt of the call's tokens     [TQ][HC]
+    L.sA = o;    o += a16(HC * 4);               // A of the heads              [HC]
+    L.sD = o;    o += a16(HC * 4);               // D of the heads              [HC]
+    L.U = o;     o += a16(HC * W * P * 4);       // fold weights x rows         [HC][L0][P]
+    L.Bf = o;    o += a16(W * N * 4);            // committed B as fp32         [L0][N]
+    L.scoef = o; o += a16(HC * TQ * TQ * 4);     // coefficients of the call's tokens [HC][TQ][TQ]
+    L.sdec = o;  o += a16(HC * TQ * 4);          // decay of the fresh copy     [HC][TQ]
     L.sfdec = o; o += a16(HC * 4);               // decay of the folded checkpoint [HC]
-    L.sCf = o;   o += a16(TQ * N * 4);           // C as fp32                  [TQ][N]
-    L.sdot = o;  o += a16(HC * P * TQ * 4);      // fresh copy . C per row     [HC*P][TQ]
+    L.sCf = o;   o += a16(TQ * N * 4);           // C as fp32                   [TQ][N]
+    L.sdot = o;  o += a16(HC * P * TQ * 4);      // fresh copy . C per row      [HC*P][TQ]
     L.si = o;    o += 32;
     L.bytes = o;
     return L;
+}
+
+// Sums of four row values over the Q lanes of a row group (Q >= 4, a power of
+// two), exchanging halves first: 2 + 1 + log2(Q/4) shuffles instead of
+// 4 log2(Q).  Lane q of the group returns the sum of row 2*(q >= Q/2) + ((q & Q/4) != 0).
+// Every lane of the warp must call it.
+template <int Q>
+__device__ __forceinline__ float quad_rows_sum(float d0, float d1, float d2, float d3, int q) {
+    const bool hi = (q & (Q / 2)) != 0, hi2 = (q & (Q / 4)) != 0;
+    const float s0 = __shfl_xor_sync(0xffffffffu, hi ? d0 : d2, Q / 2);
+    const float s1 = __shfl_xor_sync(0xffffffffu, hi ? d1 : d3, Q / 2);
+    const float e0 = (hi ? d2 : d0) + s0, e1 = (hi ? d3 : d1) + s1;
+    float f = (hi2 ? e1 : e0) + __shfl_xor_sync(0xffffffffu, hi2 ? e0 : e1, Q / 4);
+#pragma unroll
+    for (int o = Q / 8; o > 0; o >>= 1) f += __shfl_xor_sync(0xffffffffu, f, o);
+    return f;
 }
 
 template <int N, int RK, int TQ, bool BF>
@@ -312,21 +338,23 @@ __global__ void __launch_bounds__(kThreads, 2) m2_fold_kernel(const M2Args a, co
     constexpr int RG = kThreads / Q;      // row groups per stage
     constexpr int FC = kFoldChunk / (N * 4);  // fp32 rows per stage (= 4 * RG)
     constexpr int IB = BF ? 2 : 4;
+    constexpr int kLamChunks = 3;         // entries per head: L0 + T <= W + 8 <= 72 = at most 3 warps of lanes
     static_assert(FC == 4 * RG, "each thread owns 4 consecutive rows of a stage");
+    static_assert(Q >= 4, "quad_rows_sum pairs lanes at Q/2 and Q/4");
     extern __shared__ __align__(128) uint8_t smraw[];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int H = a.H, P = a.P, W = a.W, R = a.R, T = a.T, G = a.G, HC = a.HC;
     const int hpg = H / G;
-    const int E = W + TQ;
     float *stg = reinterpret_cast<float *>(smraw + Ly.stage);
     uint64_t *bar = reinterpret_cast<uint64_t *>(smraw + Ly.bar);
-    uint8_t *sC = smraw + Ly.sC, *sBr = smraw + Ly.sBr, *sBn = smraw + Ly.sBn, *sx = smraw + Ly.sx;
+    uint8_t *sC = smraw + Ly.sC, *sBr = smraw + Ly.sBr, *sBn = smraw + Ly.sBn;
+    uint8_t *sxr = smraw + Ly.sxr, *sxn = smraw + Ly.sxn;
     float *dring = reinterpret_cast<float *>(smraw + Ly.dring);
     float *dtn = reinterpret_cast<float *>(smraw + Ly.dtn);
+    float *sA = reinterpret_cast<float *>(smraw + Ly.sA);
+    float *sD = reinterpret_cast<float *>(smraw + Ly.sD);
     float *U = reinterpret_cast<float *>(smraw + Ly.U);
     float *Bf = reinterpret_cast<float *>(smraw + Ly.Bf);
-    float *slam = reinterpret_cast<float *>(smraw + Ly.slam);
-    float *su = reinterpret_cast<float *>(smraw + Ly.su);
     float *scoef = reinterpret_cast<float *>(smraw + Ly.scoef);
     float *sdec = reinterpret_cast<float *>(smraw + Ly.sdec);
     float *sfdec = reinterpret_cast<float *>(smraw + Ly.sfdec);
@@ -336,80 +364,88 @@ __global__ void __launch_bounds__(kThreads, 2) m2_fold_kernel(const M2Args a, co
     const int nrows = HC * P;
     const int nst = (nrows + FC - 1) / FC;
     const bool reads = (a.op == OP_DECODE || a.op == OP_VERIFY);
+    const bool stream = reads;  // every listed sequence folds: stages run on across items
     const int xrow = P * IB, brow = N * IB, xch = xrow / 16, bch = brow / 16;
     const int Rs = a.Rs;
     const int chunks = G * a.cpg;  // CTA work items per sequence
     auto ldx = [](const uint8_t *p) -> float {
         return BF ? bf16_bits_to_float(*reinterpret_cast<const uint16_t *>(p)) : *reinterpret_cast<const float *>(p);
     };
+    auto ld2 = [](const uint8_t *p) -> float2 {  // two consecutive raw inputs
+        if (BF) {
+            const uint32_t u = *reinterpret_cast<const uint32_t *>(p);
+            return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
+        }
+        return *reinterpret_cast<const float2 *>(p);
+    };
+    auto ld4 = [](const uint8_t *p) -> float4 {  // four consecutive raw inputs
+        if (BF) {
+            const uint2 u = *reinterpret_cast<const uint2 *>(p);
+            return make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xffff0000u),
+                               __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xffff0000u));
+        }
+        return *reinterpret_cast<const float4 *>(p);
+    };
 
     // Work items (sequence, chunk of HC heads of one group): decode/verify fold
     // the sequences the prep kernel listed; flush/export visit every sequence.
     const int nitems = (reads ? min(*a.fold_count, a.B) : a.B) * chunks;
+    auto item_seq = [&](int it) { return reads ? a.fold_list[it / chunks] : it / chunks; };
+    auto item_h0 = [&](int it) {
+        const int chunk = it % chunks, g = chunk / a.cpg;
+        return g * hpg + (chunk - g * a.cpg) * HC;
+    };
     if (tid == 0) {
         for (int k = 0; k < kFoldStages; ++k) mbar_init(&bar[k], 1);
         mbar_init_fence();
     }
     __syncthreads();
-    uint32_t gs = 0;  // checkpoint stages consumed so far: stage slot gs % 3, phase (gs / 3) & 1
+    uint32_t gs = 0;    // checkpoint stages consumed so far: slot gs % 3, phase (gs / 3) & 1
+    int ncur = 0;       // thread 0: stages of the current item issued
+    int nnext = 0;      // thread 0: stages of the next item issued (stream only)
+    int b_next = blockIdx.x < nitems ? item_seq(blockIdx.x) : 0;
 
     for (int item = blockIdx.x; item < nitems; item += gridDim.x) {
-        const int b = reads ? a.fold_list[item / chunks] : item / chunks;
+        const int b = b_next;
+        const int nxt = item + gridDim.x;
+        if (nxt < nitems) b_next = item_seq(nxt);  // first used in the stage loop
         const int chunk = item % chunks;
-        const int g = chunk / a.cpg, hc = chunk - g * a.cpg;
-        const int h0 = g * hpg + hc * HC;
+        const int g = chunk / a.cpg;
+        const int h0 = item_h0(item);
         const int64_t row0 = (int64_t)b * H + h0;
         const int64_t tile0 = row0 * P * N;
-        auto issue = [&](int c) {  // thread 0: stage c of the item's checkpoint rows
+
+        // Thread 0 keeps up to three stages in flight: the current item's, then
+        // (stream) the next item's.  `consumed` stages have been waited for.
+        auto issue = [&](bool next, int c) {
             const int r0 = c * FC, r1 = min(nrows, r0 + FC);
             const uint32_t bytes = (uint32_t)((r1 - r0) * N * 4);
-            const int k = (gs + c) % kFoldStages;
+            const uint32_t s = gs + (next ? nst : 0) + c;
+            const int k = s % kFoldStages;
+            const float *src = next ? a.ckpt + ((int64_t)b_next * H + item_h0(nxt)) * P * N : a.ckpt + tile0;
             mbar_arrive_expect_tx(&bar[k], bytes);
-            bulk_g2s(stg + k * (FC * N), a.ckpt + tile0 + (int64_t)r0 * N, bytes, &bar[k]);
+            bulk_g2s(stg + k * (FC * N), src + (int64_t)r0 * N, bytes, &bar[k]);
+        };
+        auto top_up = [&](uint32_t consumed) {
+            while (gs + ncur + nnext < consumed + kFoldStages) {
+                if (ncur < nst)
+                    issue(false, ncur++);
+                else if (stream && nxt < nitems && nnext < nst)
+                    issue(true, nnext++);
+                else
+                    break;
+            }
         };
 
-        // 1. Counters: fold when the buffer holds committed entries (flush,
-        //    export) or is too full for the call's tokens (decode, verify).
-        SeqState ss{};
-        if (tid == 0) {
-            ss = read_counters(a.c, b, W);
-            const int L0 = (int)(ss.seq - ss.ckpt);
-            const int fold = ss.ok && (reads ? (L0 + T > W) : (L0 > 0));
-            si[0] = fold;
-            si[1] = L0;
-            si[3] = (int)(ss.ckpt % R);
-            if (!ss.ok && !reads && chunk == 0) report(a.c.err, DEV_BAD_COUNTERS, b, h0, L0);
-            if (fold)
-                for (int c = 0; c < kFoldStages && c < nst; ++c) issue(c);
-        }
-        __syncthreads();
-        if (!si[0]) {
-            if (tid == 0 && a.op == OP_FLUSH)  // nothing to fold; the CTA still arrives
-                arrive_and_publish(a.c, b, chunks, -1, -1, -1, 0);
-            __syncthreads();
-            continue;
-        }
-        const int L0 = si[1], ckmod = si[3];
-        const int base = W - L0, nE = L0 + T;
-        auto slot_of = [&](int e) { const int s = ckmod + e; return s >= R ? s - R : s; };
-
-        // 2. Stage the buffered entries (B of the group, x and dt of the heads) and the call's tokens.
+        // 1. Stage the group's B ring, the heads' x and dt rings, A and D, and
+        //    the call's tokens (none of it depends on the counters); read the counters.
         {
             const uint8_t *src = reinterpret_cast<const uint8_t *>(a.Bbuf) + ((int64_t)(b * G + g) * R) * brow;
             for (int i = tid; i < R * bch; i += kThreads) cp_async16(sBr + i * 16, src + i * 16);
+            const uint8_t *xs = reinterpret_cast<const uint8_t *>(a.xbuf) + (row0 * R * P) * IB;
+            for (int i = tid; i < HC * R * xch; i += kThreads) cp_async16(sxr + i * 16, xs + i * 16);
         }
         for (int i = tid; i < HC * Rs / 4; i += kThreads) cp_async16(dring + 4 * i, a.dtbuf + row0 * Rs + 4 * i);
-        {
-            const int n1 = min(L0, R - ckmod);
-            for (int row = warp; row < 2 * HC; row += kWarps) {
-                const int hh = row >> 1, second = row & 1;
-                const int cnt = second ? L0 - n1 : n1;
-                const uint8_t *src = reinterpret_cast<const uint8_t *>(a.xbuf) +
-                                     (((row0 + hh) * R + (second ? 0 : ckmod)) * P) * IB;
-                uint8_t *dst = sx + (hh * E + base + (second ? n1 : 0)) * xrow;
-                for (int k = lane; k < cnt * xch; k += 32) cp_async16(dst + k * 16, src + k * 16);
-            }
-        }
         for (int row = warp; row < T; row += kWarps) {
             const int64_t src = (((int64_t)(b * T + row) * G + g) * N) * IB;
             for (int k = lane; k < bch; k += 32) {
@@ -417,91 +453,132 @@ __global__ void __launch_bounds__(kThreads, 2) m2_fold_kernel(const M2Args a, co
                 cp_async16(sBn + row * brow + k * 16, reinterpret_cast<const uint8_t *>(a.Bm) + src + k * 16);
             }
         }
-        for (int row = warp; row < T * HC; row += kWarps) {
-            const int m = row / HC, hh = row - m * HC;
-            const uint8_t *src = reinterpret_cast<const uint8_t *>(a.x) + (((int64_t)(b * T + m) * H + h0 + hh) * P) * IB;
-            for (int k = lane; k < xch; k += 32) cp_async16(sx + (hh * E + W + m) * xrow + k * 16, src + k * 16);
+        for (int m = warp; m < T; m += kWarps) {  // x of the call's tokens: HC heads are contiguous
+            const uint8_t *src = reinterpret_cast<const uint8_t *>(a.x) + (((int64_t)(b * T + m) * H + h0) * P) * IB;
+            for (int k = lane; k < HC * xch; k += 32) cp_async16(sxn + m * HC * xrow + k * 16, src + k * 16);
         }
         for (int i = tid; i < T * HC; i += kThreads) {
             const int m = i / HC, hh = i - m * HC;
-            dtn[m * HC + hh] = a.dt[(int64_t)(b * T + m) * H + h0 + hh];
+            cp_async4(dtn + i, a.dt + (int64_t)(b * T + m) * H + h0 + hh);
+        }
+        if (tid < HC) cp_async4(sA + tid, a.A + h0 + tid);
+        else if (tid >= 32 && tid < 32 + HC) cp_async4(sD + tid - 32, a.D + h0 + tid - 32);
+        SeqState ss{};
+        if (tid == 0) {
+            if (stream) top_up(gs);
+            ss = read_counters(a.c, b, W);
+            const int L0 = (int)(ss.seq - ss.ckpt);
+            const int fold = ss.ok && (reads ? (L0 + T > W) : (L0 > 0));
+            si[0] = fold;
+            si[1] = L0;
+            si[3] = (int)(ss.ckpt % R);
+            if (!ss.ok && !reads && chunk == 0) report(a.c.err, DEV_BAD_COUNTERS, b, h0, L0);
+            if (!stream && fold) top_up(gs);
         }
         cp_async_wait_all();
         __syncthreads();
+        const bool fold = si[0] != 0;
+        if (!fold && !stream) {
+            if (tid == 0 && a.op == OP_FLUSH)  // nothing to fold; the CTA still arrives
+                arrive_and_publish(a.c, b, chunks, -1, -1, -1, 0);
+            __syncthreads();
+            continue;
+        }
+        // (stream && !fold: counters the prep kernel reported as bad; the item's
+        //  stages are only drained.)
+        const int L0 = fold ? si[1] : 0, ckmod = si[3];
+        auto slot_of = [&](int e) { const int s = ckmod + e; return s >= R ? s - R : s; };
         auto dt_of = [&](int hh, int e) -> float {
             return e < L0 ? dring[hh * Rs + slot_of(e)] : dtn[(e - L0) * HC + hh];
         };
 
-        // 3. Per head (one warp): prefix sums of dt*A, fold weights, decays; C and
-        //    the committed entries' B as fp32.
-        for (int hh = warp; hh < HC; hh += kWarps) {
-            const float Ah = a.A[h0 + hh];
-            float *lam = slam + hh * E;
-            float carry = 0.f;
-            for (int k0 = 0; k0 < nE; k0 += 32) {
-                const int e = k0 + lane;
-                float v = (e < nE) ? dt_of(hh, e) * Ah : 0.f;
-                v = warp_incl_scan(v) + carry;
-                if (e < nE) lam[e] = v;
-                carry = __shfl_sync(0xffffffffu, v, 31);
-            }
-            __syncwarp();
-            const float lam_f = lam[L0 - 1];
-            for (int e = lane; e < L0; e += 32)
-                su[hh * E + e] = expf(lam_f - lam[e]) * (a.dt_scales ? dt_of(hh, e) : 1.f);
-            if (lane == 0) sfdec[hh] = expf(lam_f);
-            if (reads && lane < T) sdec[hh * TQ + lane] = expf(lam[L0 + lane] - lam_f);
-        }
-        for (int i = tid; i < L0 * N; i += kThreads) {
-            const int e = i / N, n = i - e * N;
-            Bf[e * N + n] = ldx(sBr + slot_of(e) * brow + n * IB);
-        }
-        if (reads)
-            for (int i = tid; i < T * N; i += kThreads) sCf[i] = ldx(sC + i * IB);
-        __syncthreads();
-        for (int i = tid; i < HC * L0 * P; i += kThreads) {  // U[hh][e][p] = weight * x
-            const int hh = i / (L0 * P), r2 = i - hh * L0 * P;
-            const int e = r2 / P, p = r2 - e * P;
-            U[(hh * L0 + e) * P + p] = su[hh * E + e] * ldx(sx + (hh * E + base + e) * xrow + p * IB);
-        }
-        if (reads) {  // coefficients of the call's own tokens against the fresh checkpoint
-            for (int pr = warp; pr < T * T; pr += kWarps) {
-                const int m = pr / T, j = pr - m * T;  // entry L0 + j, query m
-                if (j > m) continue;                   // warp-uniform
-                float d = 0.f;
-                for (int n = lane; n < N; n += 32) d = fmaf(ldx(sBn + j * brow + n * IB), sCf[m * N + n], d);
-                d = group_sum<32>(d);
-                if (lane < HC) {
-                    const float *lam = slam + lane * E;
-                    scoef[(lane * TQ + m) * E + L0 + j] =
-                        expf(lam[L0 + m] - lam[L0 + j]) * d * (a.dt_scales ? dtn[j * HC + lane] : 1.f);
+        // 2. Per head (kWarps / HC warps each): prefix sums of dt*A, fold weights,
+        //    decays, the fold-weighted x rows U and the call's own coefficients;
+        //    then B of the committed entries and C as fp32.
+        if (fold) {
+            const int nE = L0 + T;
+            const int wph = kWarps / HC;
+            const int hh = warp / wph, part = warp - hh * wph;
+            if (hh < HC) {
+                const float Ah = sA[hh];
+                float lamr[kLamChunks], sur[kLamChunks];
+                float carry = 0.f;
+#pragma unroll
+                for (int ch = 0; ch < kLamChunks; ++ch) {
+                    lamr[ch] = 0.f;
+                    sur[ch] = 0.f;
+                    if (ch * 32 < nE) {  // warp-uniform
+                        const int e = ch * 32 + lane;
+                        float v = e < nE ? dt_of(hh, e) * Ah : 0.f;
+                        v = warp_incl_scan(v) + carry;
+                        lamr[ch] = v;
+                        carry = __shfl_sync(0xffffffffu, v, 31);
+                    }
+                }
+                auto lam_at = [&](int e) -> float {  // e warp-uniform
+                    const float v = e < 32 ? lamr[0] : (e < 64 ? lamr[1] : lamr[2]);
+                    return __shfl_sync(0xffffffffu, v, e & 31);
+                };
+                const float lam_f = lam_at(L0 - 1);
+#pragma unroll
+                for (int ch = 0; ch < kLamChunks; ++ch) {
+                    const int e = ch * 32 + lane;
+                    if (e < L0) sur[ch] = expf(lam_f - lamr[ch]) * (a.dt_scales ? dt_of(hh, e) : 1.f);
+                    if (part == 0 && reads && e >= L0 && e < nE) sdec[hh * TQ + (e - L0)] = expf(lamr[ch] - lam_f);
+                }
+                if (part == 0 && lane == 0) sfdec[hh] = expf(lam_f);
+                for (int e = part; e < L0; e += wph) {  // U[hh][e][p] = weight_e x_e[p]
+                    const float w = __shfl_sync(0xffffffffu, e < 32 ? sur[0] : (e < 64 ? sur[1] : sur[2]), e & 31);
+                    const uint8_t *xr = sxr + ((hh * R + slot_of(e)) * P) * IB;
+                    float2 *Ur = reinterpret_cast<float2 *>(U + (hh * L0 + e) * P);
+                    for (int p2 = lane; p2 < P / 2; p2 += 32) {
+                        const float2 xv = ld2(xr + 2 * p2 * IB);
+                        Ur[p2] = make_float2(w * xv.x, w * xv.y);
+                    }
+                }
+                if (reads) {  // coefficients of the call's own tokens against the fresh checkpoint
+                    for (int pr = part; pr < T * T; pr += wph) {
+                        const int m = pr / T, j = pr - m * T;  // entry L0 + j, query m
+                        if (j > m) continue;                   // warp-uniform
+                        float d = 0.f;
+                        for (int n = lane; n < N; n += 32) d = fmaf(ldx(sBn + (j * N + n) * IB), ldx(sC + (m * N + n) * IB), d);
+                        d = group_sum<32>(d);
+                        const float lm = lam_at(L0 + m), lj = lam_at(L0 + j);
+                        if (lane == 0)
+                            scoef[(hh * TQ + m) * TQ + j] = expf(lm - lj) * d * (a.dt_scales ? dtn[j * HC + hh] : 1.f);
+                    }
                 }
             }
+            for (int i = tid; i < L0 * (N / 4); i += kThreads) {
+                const int e = i / (N / 4), n4 = i - e * (N / 4);
+                *reinterpret_cast<float4 *>(Bf + e * N + 4 * n4) = ld4(sBr + (slot_of(e) * N + 4 * n4) * IB);
+            }
+            if (reads)
+                for (int i = tid; i < T * N; i += kThreads) sCf[i] = ldx(sC + i * IB);
         }
         __syncthreads();
 
-        // 4. Stages of checkpoint rows: fold, store checkpoint and read copy, dot with C.
+        // 3. Stages of checkpoint rows: fold, store checkpoint and read copy, dot with C.
         const int q = tid % Q, rg = tid / Q;
         int failed = -1;  // stage whose copy never landed
         for (int c = 0; c < nst; ++c) {
-            const int k = (gs + c) % kFoldStages;
-            const bool got = mbar_wait(&bar[k], ((gs + c) / kFoldStages) & 1);
-            if (__syncthreads_or(!got)) {
-                failed = c;
-                break;
-            }
+            const uint32_t s = gs + c;
+            const int k = s % kFoldStages;
+            const bool got = mbar_wait(&bar[k], (s / kFoldStages) & 1);
             const int gr0 = c * FC + 4 * rg;  // first of this thread's 4 rows (one head: P % 4 == 0)
-            const bool valid = gr0 < nrows;
+            const bool valid = fold && gr0 < nrows;
             const int hh = valid ? gr0 / P : 0, p0 = gr0 - hh * P;
-            const float *tf = stg + k * (FC * N) + (4 * rg) * N + 4 * q;
-            const float dc = sfdec[hh];
             float4 v[4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                v[i] = valid ? *reinterpret_cast<const float4 *>(tf + i * N) : make_float4(0.f, 0.f, 0.f, 0.f);
-                v[i].x *= dc; v[i].y *= dc; v[i].z *= dc; v[i].w *= dc;
-            }
+            for (int i = 0; i < 4; ++i) v[i] = make_float4(0.f, 0.f, 0.f, 0.f);
             if (valid) {
+                const float *tf = stg + k * (FC * N) + (4 * rg) * N + 4 * q;
+                const float dc = sfdec[hh];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    v[i] = *reinterpret_cast<const float4 *>(tf + i * N);
+                    v[i].x *= dc; v[i].y *= dc; v[i].z *= dc; v[i].w *= dc;
+                }
                 const float *Ur = U + (hh * L0) * P + p0;
                 const float *Br = Bf + 4 * q;
 #pragma unroll 2
@@ -518,62 +595,79 @@ __global__ void __launch_bounds__(kThreads, 2) m2_fold_kernel(const M2Args a, co
                     v[3].z = fmaf(u.w, bb.z, v[3].z); v[3].w = fmaf(u.w, bb.w, v[3].w);
                 }
             }
-            __syncthreads();  // every thread has its rows: the stage buffer is free again
-            if (tid == 0 && c + kFoldStages < nst) issue(c + kFoldStages);
+            // Every thread has its rows (the stage buffer is free again), and
+            // every thread learns whether any wait gave up.
+            if (__syncthreads_or(!got)) {
+                failed = c;
+                break;
+            }
+            if (tid == 0) top_up(s + 1);
+            if (!fold) continue;  // CTA-uniform
+            float4 rd[4];
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 const int gr = gr0 + i;
                 const int64_t el = tile0 + (int64_t)(valid ? gr : 0) * N + 4 * q;
+                rd[i] = v[i];
                 if (a.op == OP_EXPORT) {
                     if (valid) *reinterpret_cast<float4 *>(a.out + el) = v[i];
                     continue;
                 }
                 if (valid) *reinterpret_cast<float4 *>(a.ckpt + el) = v[i];
-                float4 rd = v[i];
                 if (RK == SK_BF16) {
-                    if (valid) rd = store_quad<SK_BF16>(a.rc, el, v[i], 0.f, 0.f);
+                    if (valid) rd[i] = store_quad<SK_BF16>(a.rc, el, v[i], 0.f, 0.f);
                 } else if (RK == SK_FP8) {
                     float am = fmaxf(fmaxf(fabsf(v[i].x), fabsf(v[i].y)), fmaxf(fabsf(v[i].z), fabsf(v[i].w)));
                     am = group_max<Q>(am);
                     const float sc = fp8_scale(am);
                     if (valid) {
-                        rd = store_quad<SK_FP8>(a.rc, el, v[i], 0.f, sc);
+                        rd[i] = store_quad<SK_FP8>(a.rc, el, v[i], 0.f, sc);
                         if (q == 0) a.rc_scale[row0 * P + gr] = sc;
                     }
                 }
-                if (reads) {
+            }
+            if (reads) {
 #pragma unroll
-                    for (int m = 0; m < TQ; ++m) {
-                        const float4 Cq = *reinterpret_cast<const float4 *>(sCf + m * N + 4 * q);
-                        float d = rd.x * Cq.x + rd.y * Cq.y + rd.z * Cq.z + rd.w * Cq.w;
-                        d = group_sum<Q>(d);
-                        if (q == 0 && valid && m < T) sdot[gr * TQ + m] = d;
-                    }
+                for (int m = 0; m < TQ; ++m) {
+                    const float4 Cq = *reinterpret_cast<const float4 *>(sCf + m * N + 4 * q);
+                    float d[4];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) d[i] = rd[i].x * Cq.x + rd[i].y * Cq.y + rd[i].z * Cq.z + rd[i].w * Cq.w;
+                    const float sum = quad_rows_sum<Q>(d[0], d[1], d[2], d[3], q);
+                    const int r = 2 * ((q & (Q / 2)) != 0) + ((q & (Q / 4)) != 0);
+                    if (valid && m < T && (q & (Q / 4 - 1)) == 0) sdot[(gr0 + r) * TQ + m] = sum;
                 }
             }
         }
         if (failed >= 0) {
             // A checkpoint copy never landed: report, let the copies still in
-            // flight (stages failed .. failed + 2) land, bounded, and stop.
+            // flight (this item's from the failed stage on, the next item's
+            // already issued) land, bounded, and stop.
             if (tid == 0) {
                 report(a.c.err, DEV_PIPE_TIMEOUT, b, h0, 0);
-                for (int c = failed; c < nst && c < failed + kFoldStages; ++c)
+                for (int c = failed; c < ncur; ++c)
                     mbar_wait(&bar[(gs + c) % kFoldStages], ((gs + c) / kFoldStages) & 1);
+                for (int c = 0; c < nnext; ++c)
+                    mbar_wait(&bar[(gs + nst + c) % kFoldStages], ((gs + nst + c) / kFoldStages) & 1);
             }
             return;
         }
         gs += nst;
-        if (reads) {
+        if (tid == 0) {
+            ncur = nnext;
+            nnext = 0;
+        }
+        if (reads && fold) {
             __syncthreads();
             // Outputs of the folded sequence: the fresh copy plus the call's own tokens.
             for (int i = tid; i < T * nrows; i += kThreads) {
                 const int m = i / nrows, r2 = i - m * nrows;
                 const int hh = r2 / P, p = r2 - hh * P;
                 float yv = sdec[hh * TQ + m] * sdot[r2 * TQ + m];
-                const float *cf = scoef + (hh * TQ + m) * E;
-                const uint8_t *xs = sx + (hh * E + W) * xrow + p * IB;  // the call's tokens
-                for (int j = 0; j <= m; ++j) yv = fmaf(cf[L0 + j], ldx(xs + j * xrow), yv);
-                yv = fmaf(a.D[h0 + hh], ldx(xs + m * xrow), yv);
+                const float *cf = scoef + (hh * TQ + m) * TQ;
+                const uint8_t *xs = sxn + (hh * P + p) * IB;  // token j at xs + j * HC * xrow
+                for (int j = 0; j <= m; ++j) yv = fmaf(cf[j], ldx(xs + j * HC * xrow), yv);
+                yv = fmaf(sD[hh], ldx(xs + m * HC * xrow), yv);
                 a.y[((int64_t)(b * T + m) * H + h0 + hh) * P + p] = yv;
             }
         }

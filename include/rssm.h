@@ -159,7 +159,11 @@ RSSM_API rssm_status rssm_workspace_layout_of(const rssm_config *cfg, rssm_works
  * rssm_workspace_bytes(cfg) bytes, 256-byte aligned.  `stream` is a cudaStream_t
  * (NULL = legacy default stream).  Enqueues zeroing of the counters, error word and
  * buffers; the state is zero until rssm_import_state.  The handle (host memory) is
- * freed by rssm_destroy; the workspace stays the caller's. */
+ * freed by rssm_destroy; the workspace stays the caller's.  RSSM_EINVAL (nothing
+ * enqueued) for an invalid cfg, a NULL, misaligned or too small workspace, or a
+ * shape whose kernels need more shared memory per CTA than the current device
+ * allows (large headdim x window x max_draft with fp32 inputs); the reason is in
+ * rssm_last_error(NULL). */
 RSSM_API rssm_status rssm_create(const rssm_config *cfg, void *workspace, size_t workspace_bytes,
                         void *stream, rssm_handle *out);
 RSSM_API rssm_status rssm_destroy(rssm_handle h);
