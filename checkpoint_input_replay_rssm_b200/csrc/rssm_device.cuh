@@ -238,6 +238,15 @@ __device__ __forceinline__ void cp_async4(void *smem, const void *gmem) {
 __device__ __forceinline__ void cp_async_wait_all() {
     asm volatile("cp.async.wait_all;" ::: "memory");
 }
+// Close the copies issued so far into a group (an empty group is allowed), and
+// wait until at most `Pending` of the most recent groups are still in flight.
+__device__ __forceinline__ void cp_async_commit() {
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int Pending>
+__device__ __forceinline__ void cp_async_wait_group() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(Pending) : "memory");
+}
 
 // Element i of a raw input-dtype buffer (shared or global) as fp32.
 __device__ __forceinline__ float raw_f(const void *p, int i, int bf16) {

@@ -273,21 +273,22 @@ __global__ void __launch_bounds__(kThreads, 6) m2_prep_kernel(const M2Args a) {
 // is a rank-L0 update: U and B (fp32, in shared memory) give each thread a 4x4
 // register block (4 consecutive rows x 4 columns) updated with two 128-bit
 // shared loads and 16 FMAs per entry.  The checkpoint rows arrive in 16 KiB
-// bulk-copy stages, three in flight; all waits are bounded.
+// bulk-copy stages, two in flight per CTA (three CTAs per SM); all waits are bounded.
 //
 // The kernel is persistent and each CTA walks a list of work items (sequence,
-// HC heads of one group).  Per item, everything small is staged in one round
-// trip that does not wait for the counters (the whole B, x and dt rings, the
-// call's tokens, A and D), and the prefix sums, fold weights and coefficients
-// take one barrier.  In a decode/verify every listed sequence folds, so the
-// checkpoint stages of a CTA's items form one stream: the next item's first
-// stages are issued while the current item's last stages are folded, and a
-// new item starts with its rows already landing.
+// HC heads of one group).  What an item's prefix sums, fold weights and
+// coefficients read (the whole B, x and dt rings, A, the call's C, B and dt) and
+// its counters are fetched while the previous item's rows are folded, since
+// none of it depends on the counters; that phase then takes one barrier.  In a
+// decode/verify every listed sequence folds, so the checkpoint stages of a CTA's
+// items form one stream: the next item's first stages are issued while the
+// current item's last stages are folded, and a new item starts with its rows
+// already landing.
 // ---------------------------------------------------------------------------
 struct M2FoldLay {
     int stage, bar, sC, sBr, sBn, sxr, sxn, dring, dtn, sA, sD, U, Bf, scoef, sdec, sfdec, sCf, sdot, si, bytes;
 };
-constexpr int kFoldStages = 3;
+constexpr int kFoldStages = 2;
 // R: ring slots (W + max(max_draft, 1)).
 inline M2FoldLay m2_fold_lay(int HC, int P, int N, int W, int R, int TQ, int ib) {
     M2FoldLay L{};
@@ -333,7 +334,7 @@ __device__ __forceinline__ float quad_rows_sum(float d0, float d1, float d2, flo
 }
 
 template <int N, int RK, int TQ, bool BF>
-__global__ void __launch_bounds__(kThreads, 2) m2_fold_kernel(const M2Args a, const M2FoldLay Ly) {
+__global__ void __launch_bounds__(kThreads, 3) m2_fold_kernel(const M2Args a, const M2FoldLay Ly) {
     constexpr int Q = N / 4;              // column quads per row
     constexpr int RG = kThreads / Q;      // row groups per stage
     constexpr int FC = kFoldChunk / (N * 4);  // fp32 rows per stage (= 4 * RG)
@@ -400,22 +401,65 @@ __global__ void __launch_bounds__(kThreads, 2) m2_fold_kernel(const M2Args a, co
         mbar_init_fence();
     }
     __syncthreads();
-    uint32_t gs = 0;    // checkpoint stages consumed so far: slot gs % 3, phase (gs / 3) & 1
+    uint32_t gs = 0;    // checkpoint stages consumed so far: slot gs % kFoldStages, phase (gs / kFoldStages) & 1
     int ncur = 0;       // thread 0: stages of the current item issued
     int nnext = 0;      // thread 0: stages of the next item issued (stream only)
-    int b_next = blockIdx.x < nitems ? item_seq(blockIdx.x) : 0;
+    int64_t cseq = 0, cckpt = 0;  // thread 0: counters of the item about to start
+
+    // Staging of item `it` (sequence bb), all threads, one cp.async group each:
+    // the rings, A and the call's C, B, dt (read before the stage loop), and the
+    // call's x and D (read by the outputs after it).
+    auto stage_main = [&](int it, int bb) {
+        const int g = (it % chunks) / a.cpg, h0 = item_h0(it);
+        const int64_t row0 = (int64_t)bb * H + h0;
+        const uint8_t *src = reinterpret_cast<const uint8_t *>(a.Bbuf) + ((int64_t)(bb * G + g) * R) * brow;
+        for (int i = tid; i < R * bch; i += kThreads) cp_async16(sBr + i * 16, src + i * 16);
+        const uint8_t *xs = reinterpret_cast<const uint8_t *>(a.xbuf) + (row0 * R * P) * IB;
+        for (int i = tid; i < HC * R * xch; i += kThreads) cp_async16(sxr + i * 16, xs + i * 16);
+        for (int i = tid; i < HC * Rs / 4; i += kThreads) cp_async16(dring + 4 * i, a.dtbuf + row0 * Rs + 4 * i);
+        for (int row = warp; row < T; row += kWarps) {
+            const int64_t o = (((int64_t)(bb * T + row) * G + g) * N) * IB;
+            for (int k = lane; k < bch; k += 32) {
+                cp_async16(sC + row * brow + k * 16, reinterpret_cast<const uint8_t *>(a.Cm) + o + k * 16);
+                cp_async16(sBn + row * brow + k * 16, reinterpret_cast<const uint8_t *>(a.Bm) + o + k * 16);
+            }
+        }
+        for (int i = tid; i < T * HC; i += kThreads) {
+            const int m = i / HC, hh = i - m * HC;
+            cp_async4(dtn + i, a.dt + (int64_t)(bb * T + m) * H + h0 + hh);
+        }
+        if (tid < HC) cp_async4(sA + tid, a.A + h0 + tid);
+        cp_async_commit();
+    };
+    auto stage_out = [&](int it, int bb) {
+        const int h0 = item_h0(it);
+        for (int m = warp; m < T; m += kWarps) {  // x of the call's tokens: HC heads are contiguous
+            const uint8_t *src = reinterpret_cast<const uint8_t *>(a.x) + (((int64_t)(bb * T + m) * H + h0) * P) * IB;
+            for (int k = lane; k < HC * xch; k += 32) cp_async16(sxn + m * HC * xrow + k * 16, src + k * 16);
+        }
+        if (tid < HC) cp_async4(sD + tid, a.D + h0 + tid);
+        cp_async_commit();
+    };
+    int b_next = 0;
+    if (blockIdx.x < nitems) {
+        b_next = item_seq(blockIdx.x);
+        stage_main(blockIdx.x, b_next);
+        if (tid == 0) {
+            cseq = a.c.seq_pos[b_next];
+            cckpt = a.c.ckpt_pos[b_next];
+        }
+    }
 
     for (int item = blockIdx.x; item < nitems; item += gridDim.x) {
         const int b = b_next;
         const int nxt = item + gridDim.x;
-        if (nxt < nitems) b_next = item_seq(nxt);  // first used in the stage loop
+        if (nxt < nitems) b_next = item_seq(nxt);  // first used after the item's first barrier
         const int chunk = item % chunks;
-        const int g = chunk / a.cpg;
         const int h0 = item_h0(item);
         const int64_t row0 = (int64_t)b * H + h0;
         const int64_t tile0 = row0 * P * N;
 
-        // Thread 0 keeps up to three stages in flight: the current item's, then
+        // Thread 0 keeps up to kFoldStages stages in flight: the current item's, then
         // (stream) the next item's.  `consumed` stages have been waited for.
         auto issue = [&](bool next, int c) {
             const int r0 = c * FC, r1 = min(nrows, r0 + FC);
@@ -437,37 +481,16 @@ __global__ void __launch_bounds__(kThreads, 2) m2_fold_kernel(const M2Args a, co
             }
         };
 
-        // 1. Stage the group's B ring, the heads' x and dt rings, A and D, and
-        //    the call's tokens (none of it depends on the counters); read the counters.
-        {
-            const uint8_t *src = reinterpret_cast<const uint8_t *>(a.Bbuf) + ((int64_t)(b * G + g) * R) * brow;
-            for (int i = tid; i < R * bch; i += kThreads) cp_async16(sBr + i * 16, src + i * 16);
-            const uint8_t *xs = reinterpret_cast<const uint8_t *>(a.xbuf) + (row0 * R * P) * IB;
-            for (int i = tid; i < HC * R * xch; i += kThreads) cp_async16(sxr + i * 16, xs + i * 16);
-        }
-        for (int i = tid; i < HC * Rs / 4; i += kThreads) cp_async16(dring + 4 * i, a.dtbuf + row0 * Rs + 4 * i);
-        for (int row = warp; row < T; row += kWarps) {
-            const int64_t src = (((int64_t)(b * T + row) * G + g) * N) * IB;
-            for (int k = lane; k < bch; k += 32) {
-                cp_async16(sC + row * brow + k * 16, reinterpret_cast<const uint8_t *>(a.Cm) + src + k * 16);
-                cp_async16(sBn + row * brow + k * 16, reinterpret_cast<const uint8_t *>(a.Bm) + src + k * 16);
-            }
-        }
-        for (int m = warp; m < T; m += kWarps) {  // x of the call's tokens: HC heads are contiguous
-            const uint8_t *src = reinterpret_cast<const uint8_t *>(a.x) + (((int64_t)(b * T + m) * H + h0) * P) * IB;
-            for (int k = lane; k < HC * xch; k += 32) cp_async16(sxn + m * HC * xrow + k * 16, src + k * 16);
-        }
-        for (int i = tid; i < T * HC; i += kThreads) {
-            const int m = i / HC, hh = i - m * HC;
-            cp_async4(dtn + i, a.dt + (int64_t)(b * T + m) * H + h0 + hh);
-        }
-        if (tid < HC) cp_async4(sA + tid, a.A + h0 + tid);
-        else if (tid >= 32 && tid < 32 + HC) cp_async4(sD + tid - 32, a.D + h0 + tid - 32);
+        // 1. The item's x and D; what the counters say (fetched during the
+        //    previous item); the staged rings must have landed.
+        stage_out(item, b);
         SeqState ss{};
         if (tid == 0) {
             if (stream) top_up(gs);
-            ss = read_counters(a.c, b, W);
+            ss.seq = cseq;
+            ss.ckpt = cckpt;
             const int L0 = (int)(ss.seq - ss.ckpt);
+            ss.ok = (ss.ckpt >= 0 && L0 >= 0 && L0 <= W) ? 1 : 0;
             const int fold = ss.ok && (reads ? (L0 + T > W) : (L0 > 0));
             si[0] = fold;
             si[1] = L0;
@@ -475,15 +498,9 @@ __global__ void __launch_bounds__(kThreads, 2) m2_fold_kernel(const M2Args a, co
             if (!ss.ok && !reads && chunk == 0) report(a.c.err, DEV_BAD_COUNTERS, b, h0, L0);
             if (!stream && fold) top_up(gs);
         }
-        cp_async_wait_all();
+        cp_async_wait_group<1>();  // this item's rings (its x and D may still be in flight)
         __syncthreads();
         const bool fold = si[0] != 0;
-        if (!fold && !stream) {
-            if (tid == 0 && a.op == OP_FLUSH)  // nothing to fold; the CTA still arrives
-                arrive_and_publish(a.c, b, chunks, -1, -1, -1, 0);
-            __syncthreads();
-            continue;
-        }
         // (stream && !fold: counters the prep kernel reported as bad; the item's
         //  stages are only drained.)
         const int L0 = fold ? si[1] : 0, ckmod = si[3];
@@ -557,6 +574,23 @@ __global__ void __launch_bounds__(kThreads, 2) m2_fold_kernel(const M2Args a, co
                 for (int i = tid; i < T * N; i += kThreads) sCf[i] = ldx(sC + i * IB);
         }
         __syncthreads();
+        // The rings are free: fetch the next item's, and its counters.
+        if (nxt < nitems) {
+            stage_main(nxt, b_next);
+            if (tid == 0) {
+                cseq = a.c.seq_pos[b_next];
+                cckpt = a.c.ckpt_pos[b_next];
+            }
+        } else {
+            cp_async_commit();  // an empty group keeps the group count uniform
+        }
+        if (!fold && !stream) {
+            if (tid == 0 && a.op == OP_FLUSH)  // nothing to fold; the CTA still arrives
+                arrive_and_publish(a.c, b, chunks, -1, -1, -1, 0);
+            cp_async_wait_group<1>();  // this item's x and D have landed before they are restaged
+            __syncthreads();
+            continue;
+        }
 
         // 3. Stages of checkpoint rows: fold, store checkpoint and read copy, dot with C.
         const int q = tid % Q, rg = tid / Q;
@@ -650,6 +684,7 @@ __global__ void __launch_bounds__(kThreads, 2) m2_fold_kernel(const M2Args a, co
                 for (int c = 0; c < nnext; ++c)
                     mbar_wait(&bar[(gs + nst + c) % kFoldStages], ((gs + nst + c) / kFoldStages) & 1);
             }
+            cp_async_wait_all();
             return;
         }
         gs += nst;
@@ -657,6 +692,7 @@ __global__ void __launch_bounds__(kThreads, 2) m2_fold_kernel(const M2Args a, co
             ncur = nnext;
             nnext = 0;
         }
+        cp_async_wait_group<1>();  // this item's x and D (the next item's rings may be in flight)
         if (reads && fold) {
             __syncthreads();
             // Outputs of the folded sequence: the fresh copy plus the call's own tokens.

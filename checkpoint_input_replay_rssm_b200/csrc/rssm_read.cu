@@ -17,24 +17,32 @@ static int tq_of_read(int T) { return T <= 1 ? 1 : (T <= 4 ? 4 : 8); }
 // streams its rows in rounds of 8 x 16 bytes per thread and issues each round
 // before dotting the previous one, so its small operands' round trips overlap
 // the stream; on the 128-head layer 32 KiB gave 0.65 of peak bandwidth, 64 KiB
-// 0.76, 128 KiB 0.81, 256 KiB 0.48 (too few CTAs for the SMs).
+// 0.76, 128 KiB 0.81, 256 KiB 0.48 (too few CTAs for the SMs).  Shapes with
+// small heads are also held to 64 KiB of shared memory at the largest query
+// count (the buffered entries and coefficients grow with the heads).
+static int read_tqm(const rssm_config &cf) { return cf.max_draft > 1 ? cf.max_draft : 1; }
+static int read_ep(const rssm_config &cf) { return (cf.window + read_tqm(cf) + 3) & ~3; }
+
 int read_heads_per_cta(const rssm_config &cf) {
     const int rcb = cf.state_dtype == RSSM_F32 ? 4 : (cf.state_dtype == RSSM_BF16 ? 2 : 1);
+    const int ib = cf.input_dtype == RSSM_BF16 ? 2 : 4;
     const int qg = cf.kind == RSSM_MAMBA2 ? cf.nheads / cf.ngroups : 1;
     const int unit = qg > 1 ? qg : cf.nheads;  // heads a CTA may span
     int want = (128 * 1024) / (cf.headdim * cf.dstate * rcb);
     if (want < 1) want = 1;
     int hc = 1;
-    for (int d = 1; d <= unit && d <= want; ++d)
-        if (unit % d == 0 && cf.nheads % d == 0) hc = d;
+    for (int d = 2; d <= unit && d <= want; ++d)
+        if (unit % d == 0 && cf.nheads % d == 0 &&
+            read_lay(d, cf.headdim, cf.dstate, cf.window, tq_of_read(read_tqm(cf)), ib, read_ep(cf)).bytes <=
+                64 * 1024)
+            hc = d;
     return hc;
 }
 
 size_t read_smem_bytes(const rssm_config &cf, int T) {
     const int ib = cf.input_dtype == RSSM_BF16 ? 2 : 4;
-    const int tqm = cf.max_draft > 1 ? cf.max_draft : 1;
-    const int Ep = (cf.window + tqm + 3) & ~3;
-    return (size_t)read_lay(read_heads_per_cta(cf), cf.headdim, cf.dstate, cf.window, tq_of_read(T), ib, Ep).bytes;
+    return (size_t)read_lay(read_heads_per_cta(cf), cf.headdim, cf.dstate, cf.window, tq_of_read(T), ib,
+                            read_ep(cf)).bytes;
 }
 
 cudaError_t launch_read(const Ctx &h, int op, int T, const void *Q, int q_bf16, int q_group, int64_t q_stride_b,
