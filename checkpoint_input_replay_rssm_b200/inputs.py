@@ -1,4 +1,4 @@
-"""Seeded synthetic inputs for SSM-layer decode (Mamba-2 and Gated DeltaNet).
+"""Seeded synthetic inputs for SSM-layer decode (Mamba-2, Gated DeltaNet, Kimi Delta Attention).
 
 This module is the only code shared by the CUDA path's tests/benchmark and the
 CPU oracle. It draws random numbers and rounds them to their storage dtype; it
@@ -10,13 +10,14 @@ Stream layout.  Every (seed, token t, sequence b) has its own numpy
 steps can be regenerated without materialising the rest.  Per-layer constants
 (A_h, D_h) come from ``SeedSequence([seed, CONST_TAG])`` and the initial state of
 sequence b from ``SeedSequence([seed, CONST_TAG, b])``.  Draw order per token:
-Mamba-2 x, dt, B, C; Gated DeltaNet q, k, v, beta, alpha.
+Mamba-2 x, dt, B, C; Gated DeltaNet and KDA q, k, v, beta, alpha.
 
 Distributions (the decode workloads of the ReplaySSM reports, restated):
   Mamba-2: x, B, C ~ N(0,1); dt = softplus(N(0,1) - 2); A_h = -exp(U(0,1));
            D_h ~ N(0,1); S_0 ~ N(0, 0.1^2).
   GDN:     q, k = v/|v| with v ~ N(0,1) per head; v ~ N(0,1);
            beta = sigmoid(N(0,1)); alpha = exp(-softplus(N(0,1))); S_0 ~ N(0, 0.1^2).
+  KDA:     as GDN, with alpha drawn the same way for every key channel (alpha[H, d_k]).
 x, B, C (q, k, v) are rounded to the workload's input dtype before either side
 sees them, so buffering them in that dtype is lossless; dt, alpha, beta, A, D are
 rounded to fp32.  Every array is returned as float64 holding exactly the rounded
@@ -36,7 +37,7 @@ class Workload:
     """Shapes and seeds of one decode workload for one SSM layer."""
 
     name: str
-    kind: str  # "mamba2" | "gdn"
+    kind: str  # "mamba2" | "gdn" | "kda"
     batch: int
     nheads: int
     headdim: int  # P: Mamba-2 headdim, GDN d_v
@@ -74,8 +75,11 @@ WORKLOADS = {
     "mamba2_fp8drift_b256_h128_p64_n128_g8": Workload(
         "mamba2_fp8drift_b256_h128_p64_n128_g8", "mamba2", 256, 128, 64, 128, 8, 16, 4096, 4,
         "fp8", "bf16"),
+    # Kimi Delta Attention layer (per-channel gate), the GDN layer's shapes
+    "kda_b256_h32_dk128_dv128_w16": Workload(
+        "kda_b256_h32_dk128_dv128_w16", "kda", 256, 32, 128, 128, 32, 16, 256, 5, "bf16", "bf16"),
 }
-TINY, NEMOTRON, SPECVERIFY, GDN, FP8DRIFT = WORKLOADS.values()
+TINY, NEMOTRON, SPECVERIFY, GDN, FP8DRIFT, KDA = WORKLOADS.values()
 
 
 def _rng(*key: int) -> np.random.Generator:
@@ -132,7 +136,7 @@ def _token_one_seq(wl: Workload, t: int, b: int) -> dict:
     k = g.standard_normal((H, N), dtype=f32)
     v = g.standard_normal((H, P), dtype=f32)
     beta = 1.0 / (1.0 + np.exp(-g.standard_normal(H)))
-    alpha = np.exp(-_softplus(g.standard_normal(H)))
+    alpha = np.exp(-_softplus(g.standard_normal((H, N) if wl.kind == "kda" else H)))
     q /= np.linalg.norm(q, axis=-1, keepdims=True)
     k /= np.linalg.norm(k, axis=-1, keepdims=True)
     return {"q": q, "k": k, "v": v, "beta": beta, "alpha": alpha}
@@ -143,7 +147,7 @@ def token(wl: Workload, t: int, seqs=None) -> dict:
 
     Returns float64 arrays shaped [len(seqs), ...] holding the dtype-rounded
     values: Mamba-2 x[b,H,P], dt[b,H], B[b,G,N], C[b,G,N]; GDN q,k[b,H,N],
-    v[b,H,P], beta,alpha[b,H].
+    v[b,H,P], beta,alpha[b,H]; KDA as GDN with alpha[b,H,N].
     """
     seqs = list(range(wl.batch)) if seqs is None else list(seqs)
     parts = [_token_one_seq(wl, t, b) for b in seqs]

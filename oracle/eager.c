@@ -26,9 +26,19 @@
  *    applied to each row s of S (S is d_v x d_k, row-major, d_k contiguous):
  *      s <- alpha (s - beta (s . k) k) + beta v[row] k
  *
+ *  Kimi Delta Attention layer, per (b, h) (named with Mamba-2 and GDN on the same
+ *  page, section "Des couches rapides sur le papier", and covered by the same
+ *  argument in "La fiche qu'on reecrit"; the pages give no formula, so this is the
+ *  plainest reading: GDN with the scalar gate replaced by a gate per key channel,
+ *  applied before the delta-rule correction):
+ *      S_t = S_{t-1} Diag(alpha_t) (I - beta_t k_t k_t^T) + beta_t v_t k_t^T
+ *      o_t = S_t q_t
+ *    applied to each row s of S:  u = alpha (.) s;  s <- u - beta (u . k) k + beta v[row] k
+ *
  * Layouts (all row-major, float64):
  *   S[B][H][P][N];  Mamba-2: x[B][H][P], dt[B][H], Bm[B][G][N], Cm[B][G][N], y[B][H][P]
  *   GDN (P = d_v, N = d_k): q[B][H][N], k[B][H][N], v[B][H][P], alpha[B][H], beta[B][H], o[B][H][P]
+ *   KDA: as GDN with alpha[B][H][N]
  */
 #include <math.h>
 #include <stdint.h>
@@ -104,6 +114,38 @@ void oracle_gdn_eager_step(int64_t Bn, int64_t H, int64_t P, int64_t N, double *
                 double acc = 0.0;
                 for (int64_t n = 0; n < N; ++n) {
                     double s = al * (row[n] - be * sk * kv[n]) + be * vv[r] * kv[n];
+                    row[n] = s;
+                    acc += s * qv[n];
+                }
+                o[(b * H + h) * P + r] = acc;
+            }
+        }
+    }
+}
+
+void oracle_kda_eager_step(int64_t Bn, int64_t H, int64_t P, int64_t N, double *S,
+                           const double *q, const double *k, const double *v,
+                           const double *alpha, const double *beta, double *o)
+{
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int64_t b = 0; b < Bn; ++b) {
+        for (int64_t h = 0; h < H; ++h) {
+            const double *al = alpha + (b * H + h) * N;
+            const double be = beta[b * H + h];
+            double *Sbh = S + (b * H + h) * P * N;
+            const double *qv = q + (b * H + h) * N;
+            const double *kv = k + (b * H + h) * N;
+            const double *vv = v + (b * H + h) * P;
+            for (int64_t r = 0; r < P; ++r) {
+                double *row = Sbh + r * N;
+                double uk = 0.0;
+                for (int64_t n = 0; n < N; ++n) {
+                    row[n] = al[n] * row[n];  /* u = alpha (.) s */
+                    uk += row[n] * kv[n];
+                }
+                double acc = 0.0;
+                for (int64_t n = 0; n < N; ++n) {
+                    double s = row[n] - be * uk * kv[n] + be * vv[r] * kv[n];
                     row[n] = s;
                     acc += s * qv[n];
                 }

@@ -43,6 +43,8 @@ def _load():
         lib.oracle_mamba2_eager_step.restype = None
         lib.oracle_gdn_eager_step.argtypes = [i64, i64, i64, i64, P, P, P, P, P, P, P]
         lib.oracle_gdn_eager_step.restype = None
+        lib.oracle_kda_eager_step.argtypes = [i64, i64, i64, i64, P, P, P, P, P, P, P]
+        lib.oracle_kda_eager_step.restype = None
         lib.oracle_set_threads.argtypes = [ctypes.c_int]
         lib.oracle_max_threads.restype = ctypes.c_int
         _lib = lib
@@ -102,10 +104,30 @@ def gdn_step(S: np.ndarray, q, k, v, alpha, beta) -> np.ndarray:
     return o
 
 
+def kda_step(S: np.ndarray, q, k, v, alpha, beta) -> np.ndarray:
+    """One eager Kimi Delta Attention token for all (b,h). S[B,H,d_v,d_k] updated in place.
+
+    q,k[B,H,d_k], v[B,H,d_v], alpha[B,H,d_k] (a gate per key channel), beta[B,H].
+    Returns o[B,H,d_v].
+    """
+    lib = _load()
+    assert S.dtype == np.float64 and S.flags.c_contiguous
+    Bn, H, P, N = S.shape
+    q, k, v, alpha, beta = map(_f64, (q, k, v, alpha, beta))
+    assert q.shape == (Bn, H, N) and k.shape == (Bn, H, N) and v.shape == (Bn, H, P)
+    assert alpha.shape == (Bn, H, N) and beta.shape == (Bn, H)
+    o = np.empty((Bn, H, P))
+    lib.oracle_kda_eager_step(Bn, H, P, N, _p(S), _p(q), _p(k), _p(v), _p(alpha), _p(beta),
+                              _p(o))
+    return o
+
+
 def step(kind: str, S: np.ndarray, tok: dict, params: dict | None = None,
          dt_scales_input: bool = False) -> np.ndarray:
-    """Dispatch one eager token of either layer kind (tok: one token, [B,...] arrays)."""
+    """Dispatch one eager token of a layer kind ("mamba2" | "gdn" | "kda"; tok: one token, [B,...] arrays)."""
     if kind == "mamba2":
         return mamba2_step(S, params["A"], params["D"], tok["x"], tok["dt"], tok["B"], tok["C"],
                            dt_scales_input)
+    if kind == "kda":
+        return kda_step(S, tok["q"], tok["k"], tok["v"], tok["alpha"], tok["beta"])
     return gdn_step(S, tok["q"], tok["k"], tok["v"], tok["alpha"], tok["beta"])

@@ -16,6 +16,11 @@ Gated DeltaNet (backward sweep applying the delta-rule factors to q):
     r <- q;  for j = L..1: c_j = beta_j (k_j . r);  r <- alpha_j (r - c_j k_j)
     o = S^ r + sum_j c_j v_j
     fold:  for j = 1..L: S_c <- alpha_j S_c (I - beta_j k_j k_j^T) + beta_j v_j k_j^T
+Kimi Delta Attention (alpha_j a gate per key channel; the same sweep with
+Diag(alpha_j) in place of the scalar):
+    r <- q;  for j = L..1: c_j = beta_j (k_j . r);  r <- alpha_j (.) (r - c_j k_j)
+    o = S^ r + sum_j c_j v_j
+    fold:  for j = 1..L: S_c <- S_c Diag(alpha_j) (I - beta_j k_j k_j^T) + beta_j v_j k_j^T
 S^ is the read copy: the fp32 checkpoint itself, or its bf16 / per-row fp8
 rounding (oracle/quant.py); rounding of the copy never feeds the fold, which
 always starts from the full-precision checkpoint ("Deux precisions pour le prix
@@ -55,7 +60,7 @@ class ReplayOracle:
         else:
             self.buf["k"] = np.zeros((Bn, self.R, H, N))
             self.buf["v"] = np.zeros((Bn, self.R, H, P))
-            self.buf["alpha"] = np.zeros((Bn, self.R, H))
+            self.buf["alpha"] = np.zeros((Bn, self.R, H, N) if kind == "kda" else (Bn, self.R, H))
             self.buf["beta"] = np.zeros((Bn, self.R, H))
 
     # ---------------------------------------------------------------- entries
@@ -80,6 +85,15 @@ class ReplayOracle:
                 out = out + (w * s)[:, None, None] * e["x"][i][:, :, None] * Bh[:, None, :]
             return out
         out = S.copy()
+        if self.kind == "kda":
+            for i in range(e["k"].shape[0]):
+                k, v = e["k"][i], e["v"][i]  # [H,N], [H,P]
+                al, be = e["alpha"][i], e["beta"][i]  # [H,N], [H]
+                u = al[:, None, :] * out
+                uk = np.einsum("hpn,hn->hp", u, k)
+                out = u - be[:, None, None] * uk[:, :, None] * k[:, None, :] \
+                    + be[:, None, None] * v[:, :, None] * k[:, None, :]
+            return out
         for i in range(e["k"].shape[0]):
             k, v = e["k"][i], e["v"][i]  # [H,N], [H,P]
             al, be = e["alpha"][i], e["beta"][i]
@@ -109,7 +123,8 @@ class ReplayOracle:
         o = np.zeros((self.H, self.P))
         for j in range(e["k"].shape[0] - 1, -1, -1):
             c = e["beta"][j] * np.sum(e["k"][j] * r, axis=1)  # [H]
-            r = e["alpha"][j][:, None] * (r - c[:, None] * e["k"][j])
+            al = e["alpha"][j] if self.kind == "kda" else e["alpha"][j][:, None]
+            r = al * (r - c[:, None] * e["k"][j])
             o = o + c[:, None] * e["v"][j]
         return o + np.einsum("hpn,hn->hp", rc, r)
 
