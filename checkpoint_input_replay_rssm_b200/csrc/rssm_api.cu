@@ -20,7 +20,8 @@ bool validate(const rssm_config *c, std::string *why) {
     char buf[256];
     auto fail = [&](const char *m) { if (why) *why = m; return false; };
     if (!c) return fail("config is NULL");
-    if (c->kind != RSSM_MAMBA2 && c->kind != RSSM_GDN) return fail("kind must be MAMBA2 or GDN");
+    if (c->kind != RSSM_MAMBA2 && c->kind != RSSM_GDN && c->kind != RSSM_KDA)
+        return fail("kind must be MAMBA2, GDN or KDA");
     if (c->mode != RSSM_REPLAY && c->mode != RSSM_EAGER) return fail("mode must be REPLAY or EAGER");
     if (c->state_dtype < RSSM_F32 || c->state_dtype > RSSM_FP8E4M3) return fail("bad state_dtype");
     if (c->input_dtype != RSSM_F32 && c->input_dtype != RSSM_BF16) return fail("input_dtype must be F32 or BF16");
@@ -39,7 +40,7 @@ bool validate(const rssm_config *c, std::string *why) {
         return false;
     }
     if (c->dt_scales_input != 0 && c->dt_scales_input != 1) return fail("dt_scales_input must be 0 or 1");
-    if (c->kind == RSSM_GDN && c->dt_scales_input) return fail("dt_scales_input is Mamba-2 only");
+    if (c->kind != RSSM_MAMBA2 && c->dt_scales_input) return fail("dt_scales_input is Mamba-2 only");
     return true;
 }
 
@@ -83,9 +84,9 @@ void layout(const rssm_config *c, rssm_workspace_layout *L) {
         L->xbuf_off = take(L->xbuf_bytes);
         L->bbuf_bytes = B * G * R * N * ib;
         L->bbuf_off = take(L->bbuf_bytes);
-        L->sbuf_bytes = B * H * Rs * 4;
+        L->sbuf_bytes = c->kind == RSSM_KDA ? B * H * R * N * 4 : B * H * Rs * 4;
         L->sbuf_off = take(L->sbuf_bytes);
-        if (c->kind == RSSM_GDN) {
+        if (c->kind != RSSM_MAMBA2) {
             L->tbuf_bytes = B * H * Rs * 4;
             L->tbuf_off = take(L->tbuf_bytes);
         }
@@ -98,7 +99,7 @@ void layout(const rssm_config *c, rssm_workspace_layout *L) {
         L->dec_off = take(L->dec_bytes);
         L->coef_bytes = B * H * TQm * (((size_t)c->window + TQm + 3) & ~(size_t)3) * 4;
         L->coef_off = take(L->coef_bytes);
-        if (c->kind == RSSM_GDN) {
+        if (c->kind != RSSM_MAMBA2) {
             L->query_bytes = B * H * TQm * N * 4;
             L->query_off = take(L->query_bytes);
         }
@@ -127,7 +128,7 @@ bool inputs_ok(const Ctx *h, const rssm_inputs *in) {
         return in->x && in->dt && in->Bm && in->Cm && aligned16(in->x) && aligned16(in->Bm) &&
                aligned16(in->Cm);
     return in->q && in->k && in->v && in->alpha && in->beta && aligned16(in->q) &&
-           aligned16(in->k) && aligned16(in->v);
+           aligned16(in->k) && aligned16(in->v) && (h->cfg.kind != RSSM_KDA || aligned16(in->alpha));
 }
 
 cudaError_t launch_kind(Ctx *h, int op, int T, const rssm_inputs *in, float *y, float *out) {

@@ -12,7 +12,7 @@ extern template cudaError_t g_dispatch_n<128>(bool, int, int, const GArgs &, siz
 static int gtq_of(int T) { return T <= 1 ? 1 : (T <= 4 ? 4 : 8); }
 
 size_t gdn_smem_bytes(const rssm_config &cf, int T) {
-    return sizeof(float) * gdn_smem_floats(cf.headdim, cf.dstate, cf.window, gtq_of(T));
+    return sizeof(float) * gdn_smem_floats(cf.headdim, cf.dstate, cf.window, gtq_of(T), cf.kind == RSSM_KDA);
 }
 
 cudaError_t gdn_launch(Ctx &h, int op, int T, const rssm_inputs *in, float *y, float *out, cudaStream_t st) {
@@ -20,6 +20,7 @@ cudaError_t gdn_launch(Ctx &h, int op, int T, const rssm_inputs *in, float *y, f
     const rssm_config &cf = h.cfg;
     a.B = cf.batch; a.H = cf.nheads; a.P = cf.headdim; a.W = cf.window;
     a.R = (int)h.lay.ring; a.Rs = (int)h.lay.ring_stride; a.T = T; a.op = op; a.in_bf16 = cf.input_dtype == RSSM_BF16;
+    a.kda = cf.kind == RSSM_KDA;
     a.c = h.counters();
     a.ckpt = h.lay.ckpt_bytes ? (float *)h.at(h.lay.ckpt_off) : nullptr;
     a.rc = h.lay.rc_bytes ? h.at(h.lay.rc_off) : nullptr;
@@ -61,7 +62,7 @@ cudaError_t gdn_launch(Ctx &h, int op, int T, const rssm_inputs *in, float *y, f
     a.Emax = (cf.window + a.TQmax + 3) & ~3;
     const bool fold = h.len_ub + T > cf.window;
     a.fold_launched = fold;
-    const int wb = gdn_prep_warp_bytes(N, cf.window, TQ, a.in_bf16 ? 2 : 4);
+    const int wb = gdn_prep_warp_bytes(N, cf.window, TQ, a.in_bf16 ? 2 : 4, a.kda);
     a.prep_heads = (96 * 1024) / wb;
     if (a.prep_heads > kWarps) a.prep_heads = kWarps;
     if (a.prep_heads < 1) a.prep_heads = 1;

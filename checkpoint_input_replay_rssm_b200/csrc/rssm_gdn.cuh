@@ -30,11 +30,11 @@ struct GArgs {
     void *rc;
     float *rc_scale;
     void *kbuf, *vbuf;   // [B][H][R][N], [B][H][R][P] input dtype
-    float *abuf, *bbuf;  // [B][H][R]
+    float *abuf, *bbuf;  // GDN [B][H][Rs] each; KDA alpha [B][H][R][N]
     void *snap;
     float *snap_scale;
     const void *q, *k, *v;      // [B][T][H][N|P]
-    const float *alpha, *beta;  // [B][T][H]
+    const float *alpha, *beta;  // [B][T][H]; KDA alpha [B][T][H][N]
     float *y;                   // [B][T][H][P]
     float *out;                 // export target
     // replay decode/verify: hand-off of the prep kernel to the read kernel
@@ -46,13 +46,15 @@ struct GArgs {
     int fold_launched;          // the fold-only launch of gdn_replay_kernel follows in this call
     int fold_only;              // gdn_replay_kernel: only fold (and serve) sequences whose buffer is full
     int prep_heads;             // gdn_prep_kernel: heads (warps at work) per CTA, <= 8
+    int kda;                    // Kimi Delta Attention: alpha is a gate per key channel
 };
 
 __host__ __device__ constexpr int gpad4(int n) { return (n + 3) & ~3; }
 
-__host__ __device__ inline size_t gdn_smem_floats(int P, int N, int W, int TQ) {
+// KDA keeps a gate row [E][N] where GDN keeps one gate per entry.
+__host__ __device__ inline size_t gdn_smem_floats(int P, int N, int W, int TQ, int kda) {
     const int E = W + TQ;
-    return (size_t)gpad4(E * N) + gpad4(E * P) + 3 * (size_t)gpad4(E) + gpad4(TQ * N) +
+    return (size_t)gpad4(E * N) + gpad4(E * P) + gpad4(kda ? E * N : E) + 2 * (size_t)gpad4(E) + gpad4(TQ * N) +
            gpad4(E * E) + 2 * (size_t)gpad4(TQ * E) + gpad4(TQ * N) + gpad4(TQ * P) + gpad4(TQ) + 8;
 }
 
@@ -61,13 +63,13 @@ struct GSmem {
     int *si;
 };
 
-__device__ __forceinline__ GSmem gdn_carve(float *sm, int P, int N, int W, int TQ) {
+__device__ __forceinline__ GSmem gdn_carve(float *sm, int P, int N, int W, int TQ, int kda) {
     const int E = W + TQ;
     GSmem s;
     s.sk = sm;                            // [E][N]  k of entries (physical)
     s.sv = s.sk + gpad4(E * N);           // [E][P]  v of entries (physical)
-    s.sal = s.sv + gpad4(E * P);          // [E]     alpha (physical)
-    s.sbe = s.sal + gpad4(E);             // [E]     beta (physical)
+    s.sal = s.sv + gpad4(E * P);          // [E]     alpha (physical); KDA [E][N]
+    s.sbe = s.sal + gpad4(kda ? E * N : E);  // [E]  beta (physical)
     s.spr = s.sbe + gpad4(E);             // [E]     prefix products of alpha from e0 (logical)
     s.sq = s.spr + gpad4(E);              // [TQ][N] queries
     s.sG = s.sq + gpad4(TQ * N);          // [E][E]  Gram k_e . k_j (logical)
@@ -101,26 +103,57 @@ __device__ __forceinline__ void gdn_stage_new(const GArgs &a, const GSmem &s, in
         const int m = i / P, p = i - m * P;
         s.sv[(W + m) * P + p] = ld_in(a.v, ((int64_t)(b * T + m) * H + h) * P + p, a.in_bf16);
     }
-    if (tid < T) {
+    if (a.kda) {
+        for (int i = tid; i < T * N; i += kThreads) {
+            const int m = i / N, n = i - m * N;
+            s.sal[(W + m) * N + n] = a.alpha[((int64_t)(b * T + m) * H + h) * N + n];
+        }
+    } else if (tid < T) {
         s.sal[W + tid] = a.alpha[(int64_t)(b * T + tid) * H + h];
-        s.sbe[W + tid] = a.beta[(int64_t)(b * T + tid) * H + h];
     }
+    if (tid < T) s.sbe[W + tid] = a.beta[(int64_t)(b * T + tid) * H + h];
 }
 
 // Apply entries [0, L0) (physical base..) to NR rows held as NPT-element lane
 // segments.  Rows are independent; every lane of the warp must call this.
+// GDN:  s <- alpha s + (beta v[row] - alpha beta (s . k)) k
+// KDA:  u = alpha (.) s;  s <- u + beta (v[row] - u . k) k
 template <int N, int NR>
 __device__ __forceinline__ void gdn_fold_rows(float (&st)[NR][FoldMap<N>::NPT], const int (&rows)[NR],
-                                              int P, const GSmem &s, int base, int L0, int cseg) {
+                                              int P, const GSmem &s, int base, int L0, int cseg, int kda) {
     constexpr int NPT = FoldMap<N>::NPT, TPRF = FoldMap<N>::TPRF;
     for (int e = 0; e < L0; ++e) {
-        const float al = s.sal[base + e], be = s.sbe[base + e];
+        const float be = s.sbe[base + e];
         float kk[NPT];
 #pragma unroll
         for (int j = 0; j < NPT; j += 4) {
             const float4 k4 = *reinterpret_cast<const float4 *>(s.sk + (base + e) * N + cseg * NPT + j);
             kk[j] = k4.x; kk[j + 1] = k4.y; kk[j + 2] = k4.z; kk[j + 3] = k4.w;
         }
+        if (kda) {  // warp-uniform
+            float ga[NPT];
+#pragma unroll
+            for (int j = 0; j < NPT; j += 4) {
+                const float4 g4 = *reinterpret_cast<const float4 *>(s.sal + (base + e) * N + cseg * NPT + j);
+                ga[j] = g4.x; ga[j + 1] = g4.y; ga[j + 2] = g4.z; ga[j + 3] = g4.w;
+            }
+#pragma unroll
+            for (int r = 0; r < NR; ++r) {
+                float d = 0.f;
+#pragma unroll
+                for (int j = 0; j < NPT; ++j) {
+                    st[r][j] *= ga[j];
+                    d = fmaf(st[r][j], kk[j], d);
+                }
+                d = group_sum<TPRF>(d);
+                const float vr = (rows[r] < P) ? s.sv[(base + e) * P + rows[r]] : 0.f;
+                const float coef = be * (vr - d);
+#pragma unroll
+                for (int j = 0; j < NPT; ++j) st[r][j] = fmaf(coef, kk[j], st[r][j]);
+            }
+            continue;
+        }
+        const float al = s.sal[base + e];
 #pragma unroll
         for (int r = 0; r < NR; ++r) {
             float d = 0.f;
@@ -154,7 +187,7 @@ __global__ void __launch_bounds__(kThreads) gdn_replay_kernel(const GArgs a) {
     const int H = a.H, P = a.P, W = a.W, R = a.R, T = a.T;
     const int b = bh / H, h = bh - b * H;
     const int E = W + TQ;
-    GSmem s = gdn_carve(smem, P, N, W, TQ);
+    GSmem s = gdn_carve(smem, P, N, W, TQ, a.kda);
     const int64_t tile0 = (int64_t)bh * P * N;
     const bool reads = (a.op == OP_DECODE || a.op == OP_VERIFY);
 
@@ -215,12 +248,37 @@ __global__ void __launch_bounds__(kThreads) gdn_replay_kernel(const GArgs a) {
     }
     for (int e = tid; e < L0; e += kThreads) {
         const int64_t slot = (int64_t)bh * a.Rs + (ckmod + e) % R;
-        s.sal[base + e] = a.abuf[slot];
+        if (!a.kda) s.sal[base + e] = a.abuf[slot];
         s.sbe[base + e] = a.bbuf[slot];
     }
+    if (a.kda)
+        for (int i = tid; i < L0 * N; i += kThreads) {
+            const int e = i / N, n = i - e * N;
+            s.sal[(base + e) * N + n] = a.abuf[((int64_t)bh * R + (ckmod + e) % R) * N + n];
+        }
     __syncthreads();
 
-    if (reads) {
+    if (reads && a.kda) {
+        // 4-6 (KDA). One warp per query: the backward sweep applied to the query
+        // itself, r <- alpha_i (.) (r - c_i k_i), c_i = beta_i (k_i . r).
+        if (warp < T) {
+            const int m = warp, em = L0 + m;
+            float *r = s.sr + m * N;
+            for (int x = lane; x < N; x += 32) r[x] = s.sq[m * N + x];
+            __syncwarp();
+            for (int i = em; i >= e0; --i) {
+                const float *ki = s.sk + (base + i) * N, *gi = s.sal + (base + i) * N;
+                float d = 0.f;
+                for (int x = lane; x < N; x += 32) d = fmaf(ki[x], r[x], d);
+                d = group_sum<32>(d);
+                const float ci = s.sbe[base + i] * d;
+                if (lane == 0) s.sc[m * E + i] = ci;
+                for (int x = lane; x < N; x += 32) r[x] = gi[x] * fmaf(-ci, ki[x], r[x]);
+                __syncwarp();
+            }
+        }
+        __syncthreads();
+    } else if (reads) {
         // 4. Gram matrix of the replayed keys and their products with the queries.
         const int n = nE - e0;                       // replayed entries
         const int ngram = n * (n - 1) / 2;
@@ -308,7 +366,7 @@ __global__ void __launch_bounds__(kThreads) gdn_replay_kernel(const GArgs a) {
                     st[k][j] = v4.x; st[k][j + 1] = v4.y; st[k][j + 2] = v4.z; st[k][j + 3] = v4.w;
                 }
             }
-            gdn_fold_rows<N, RBF>(st, rows, P, s, base, L0, cseg);
+            gdn_fold_rows<N, RBF>(st, rows, P, s, base, L0, cseg, a.kda);
 #pragma unroll
             for (int k = 0; k < RBF; ++k) {
                 const bool valid = rows[k] < P;
@@ -420,9 +478,14 @@ __global__ void __launch_bounds__(kThreads) gdn_replay_kernel(const GArgs a) {
     }
     if (tid < T) {
         const int64_t slot = (int64_t)bh * a.Rs + (spmod + tid) % R;
-        a.abuf[slot] = s.sal[W + tid];
+        if (!a.kda) a.abuf[slot] = s.sal[W + tid];
         a.bbuf[slot] = s.sbe[W + tid];
     }
+    if (a.kda)
+        for (int i = tid; i < T * N; i += kThreads) {
+            const int m = i / N, n = i - m * N;
+            a.abuf[((int64_t)bh * R + (spmod + m) % R) * N + n] = s.sal[(W + m) * N + n];
+        }
 }
 
 // ---------------------------------------------------------------------------
@@ -437,9 +500,11 @@ __global__ void __launch_bounds__(kThreads) gdn_replay_kernel(const GArgs a) {
 // fold-only launch of gdn_replay_kernel.  Every sequence's tokens are appended
 // to the ring (slots seq_pos + m mod R, never an entry read in this call).
 // ---------------------------------------------------------------------------
-__host__ __device__ inline int gdn_prep_warp_bytes(int N, int W, int TQ, int ib) {
-    const int E = W + TQ;
-    return ((E + TQ) * N * ib + 2 * ((E + 3) & ~3) * 4 + 15) & ~15;
+// Per warp: raw k rows [E][N] and q rows [TQ][N], then the gates (GDN [Ea], KDA
+// [E][N] fp32) and beta [Ea].
+__host__ __device__ inline int gdn_prep_warp_bytes(int N, int W, int TQ, int ib, int kda) {
+    const int E = W + TQ, Ea = (E + 3) & ~3;
+    return ((E + TQ) * N * ib + (kda ? E * N : Ea) * 4 + Ea * 4 + 15) & ~15;
 }
 
 template <int N, int TQ, bool BF>
@@ -476,10 +541,11 @@ __global__ void __launch_bounds__(kThreads) gdn_prep_kernel(const GArgs a) {
     const int L0 = si[1], fold = si[2], ckmod = si[3], spmod = si[4];
     const int64_t bh = (int64_t)b * H + h;
     const int krow = N * IB, kch = krow / 16;
-    uint8_t *wk = gsm + warp * gdn_prep_warp_bytes(N, W, TQ, IB);  // k rows [E][N] raw
+    const int kda = a.kda;
+    uint8_t *wk = gsm + warp * gdn_prep_warp_bytes(N, W, TQ, IB, kda);  // k rows [E][N] raw
     uint8_t *wq = wk + E * krow;                                   // q rows [TQ][N] raw
-    float *wal = reinterpret_cast<float *>(wq + TQ * krow);        // alpha [E]
-    float *wbe = wal + Ea;                                         // beta  [E]
+    float *wal = reinterpret_cast<float *>(wq + TQ * krow);        // alpha [E]; KDA [E][N]
+    float *wbe = wal + (kda ? E * N : Ea);                         // beta  [E]
     auto run = [&](uint8_t *dst, const uint8_t *src, int n) {
         for (int j = lane; j < n; j += 32) cp_async16(dst + 16 * j, src + 16 * j);
     };
@@ -489,19 +555,29 @@ __global__ void __launch_bounds__(kThreads) gdn_prep_kernel(const GArgs a) {
         run(wk + (L0 + m) * krow, kin + row * krow, kch);
         run(wq + m * krow, qin + row * krow, kch);
     }
+    const int gch = N * 4 / 16;  // 16-byte chunks of a KDA gate row
     if (!fold) {
         const int n1 = min(L0, R - ckmod);
         const uint8_t *kr = reinterpret_cast<const uint8_t *>(a.kbuf) + bh * R * krow;
         run(wk, kr + ckmod * krow, n1 * kch);
         run(wk + n1 * krow, kr, (L0 - n1) * kch);
+        if (kda) {
+            const uint8_t *gr = reinterpret_cast<const uint8_t *>(a.abuf) + bh * R * N * 4;
+            run(reinterpret_cast<uint8_t *>(wal), gr + ckmod * N * 4, n1 * gch);
+            run(reinterpret_cast<uint8_t *>(wal + n1 * N), gr, (L0 - n1) * gch);
+        }
         for (int e = lane; e < L0; e += 32) {
             const int s2 = ckmod + e >= R ? ckmod + e - R : ckmod + e;
-            wal[e] = a.abuf[bh * a.Rs + s2];
+            if (!kda) wal[e] = a.abuf[bh * a.Rs + s2];
             wbe[e] = a.bbuf[bh * a.Rs + s2];
         }
     }
+    if (kda)
+        for (int m = 0; m < T; ++m)
+            run(reinterpret_cast<uint8_t *>(wal + (L0 + m) * N),
+                reinterpret_cast<const uint8_t *>(a.alpha + (((int64_t)b * T + m) * H + h) * N), gch);
     if (lane < T) {
-        wal[L0 + lane] = a.alpha[((int64_t)b * T + lane) * H + h];
+        if (!kda) wal[L0 + lane] = a.alpha[((int64_t)b * T + lane) * H + h];
         wbe[L0 + lane] = a.beta[((int64_t)b * T + lane) * H + h];
     }
     cp_async_wait_all();
@@ -530,9 +606,18 @@ __global__ void __launch_bounds__(kThreads) gdn_prep_kernel(const GArgs a) {
 #pragma unroll
                 for (int i = 0; i < NL; ++i) d = fmaf(kv[i], r[i], d);
                 d = group_sum<32>(d);
-                const float ce = wbe[e] * d, al = wal[e];
+                const float ce = wbe[e] * d;
+                if (kda) {  // gate per key channel; lanes past N hold zeros
 #pragma unroll
-                for (int i = 0; i < NL; ++i) r[i] = al * fmaf(-ce, kv[i], r[i]);
+                    for (int i = 0; i < NL; ++i) {
+                        const float g = NL * lane < N ? wal[e * N + NL * lane + i] : 0.f;
+                        r[i] = g * fmaf(-ce, kv[i], r[i]);
+                    }
+                } else {
+                    const float al = wal[e];
+#pragma unroll
+                    for (int i = 0; i < NL; ++i) r[i] = al * fmaf(-ce, kv[i], r[i]);
+                }
                 if (lane == 0) crow[e] = ce;
             }
             if (NL * lane < N) {
@@ -555,8 +640,13 @@ __global__ void __launch_bounds__(kThreads) gdn_prep_kernel(const GArgs a) {
         const uint8_t *vs = reinterpret_cast<const uint8_t *>(a.v) + (((int64_t)b * T + m) * H + h) * P * IB;
         for (int j = lane; j < vch; j += 32)
             *reinterpret_cast<uint4 *>(vd + 16 * j) = *reinterpret_cast<const uint4 *>(vs + 16 * j);
+        if (kda) {
+            float *gd = a.abuf + (bh * R + sl) * N;
+            for (int j = lane; j < N / 4; j += 32)
+                *reinterpret_cast<float4 *>(gd + 4 * j) = *reinterpret_cast<const float4 *>(wal + (L0 + m) * N + 4 * j);
+        }
         if (lane == 0) {
-            a.abuf[bh * a.Rs + sl] = wal[L0 + m];
+            if (!kda) a.abuf[bh * a.Rs + sl] = wal[L0 + m];
             a.bbuf[bh * a.Rs + sl] = wbe[L0 + m];
         }
     }
@@ -574,7 +664,7 @@ __global__ void __launch_bounds__(kThreads) gdn_eager_kernel(const GArgs a) {
     const int bh = blockIdx.x;
     const int H = a.H, P = a.P, T = a.T, W = a.W;
     const int b = bh / H, h = bh - b * H;
-    GSmem s = gdn_carve(smem, P, N, W, TQ);
+    GSmem s = gdn_carve(smem, P, N, W, TQ, a.kda);
     const int64_t tile0 = (int64_t)bh * P * N;
     void *state = (SK == SK_F32) ? (void *)a.ckpt : a.rc;
     const int64_t state_elems = (int64_t)a.B * H * P * N;
@@ -606,7 +696,7 @@ __global__ void __launch_bounds__(kThreads) gdn_eager_kernel(const GArgs a) {
         }
         for (int m = 0; m < T; ++m) {
             // one token: entry m sits at physical W + m
-            gdn_fold_rows<N, RBF>(st, rows, P, s, W + m, 1, cseg);
+            gdn_fold_rows<N, RBF>(st, rows, P, s, W + m, 1, cseg, a.kda);
 #pragma unroll
             for (int k = 0; k < RBF; ++k) {
                 const bool valid = rows[k] < P;
@@ -692,7 +782,7 @@ cudaError_t g_dispatch_n(bool eager, int rk, int TQ, const GArgs &a, size_t smem
 template <int N, int TQ>
 inline cudaError_t launch_gprep_t(const GArgs &a, cudaStream_t st) {
     auto k = a.in_bf16 ? gdn_prep_kernel<N, TQ, true> : gdn_prep_kernel<N, TQ, false>;
-    const int smem = a.prep_heads * gdn_prep_warp_bytes(N, a.W, TQ, a.in_bf16 ? 2 : 4);
+    const int smem = a.prep_heads * gdn_prep_warp_bytes(N, a.W, TQ, a.in_bf16 ? 2 : 4, a.kda);
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     k<<<dim3((a.H + a.prep_heads - 1) / a.prep_heads, a.B), kThreads, smem, st>>>(a);

@@ -16,12 +16,12 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "librssm.so")
 
 RSSM_OK, RSSM_EINVAL, RSSM_ESTATE, RSSM_ECUDA, RSSM_EDEVICE = range(5)
-RSSM_MAMBA2, RSSM_GDN = 0, 1
+RSSM_MAMBA2, RSSM_GDN, RSSM_KDA = 0, 1, 2
 RSSM_REPLAY, RSSM_EAGER = 0, 1
 RSSM_F32, RSSM_BF16, RSSM_FP8E4M3 = 0, 1, 2
 RSSM_DEV_BAD_ACCEPT, RSSM_DEV_BAD_COUNTERS, RSSM_DEV_PIPE_TIMEOUT = 1, 2, 3
 DTYPES = {"f32": RSSM_F32, "bf16": RSSM_BF16, "fp8": RSSM_FP8E4M3}
-KINDS = {"mamba2": RSSM_MAMBA2, "gdn": RSSM_GDN}
+KINDS = {"mamba2": RSSM_MAMBA2, "gdn": RSSM_GDN, "kda": RSSM_KDA}
 MODES = {"replay": RSSM_REPLAY, "eager": RSSM_EAGER}
 
 

@@ -42,8 +42,19 @@ def _x_row(s: Shape) -> float:  # Mamba-2 x / GDN v of one token, one head
     return s.headdim * SB[s.input_dtype]
 
 
-def _key_row(s: Shape) -> float:  # Mamba-2 B (charged per head) / GDN k
+def _key_row(s: Shape) -> float:  # Mamba-2 B (charged per head) / GDN, KDA k
     return s.dstate * SB[s.input_dtype] / _grp(s)
+
+
+def _scalars(s: Shape) -> float:  # per-token fp32 gates: dt; alpha + beta; KDA alpha[d_k] + beta
+    return {"mamba2": 4.0, "gdn": 8.0}.get(s.kind, s.dstate * 4.0 + 4.0)
+
+
+def _handoff(s: Shape, L0: int, T: int) -> float:
+    """Prep -> read hand-off per (b, h): coefficients over the replayed entries and
+    a decay per query; GDN and KDA also hand over the swept query (d_k fp32)."""
+    per_query = (L0 + T) * 4 + 4 + (0 if s.kind == "mamba2" else s.dstate * 4)
+    return T * per_query
 
 
 def replay_step_split(s: Shape, L0: int, fold: bool, T: int = 1) -> dict:
@@ -53,8 +64,8 @@ def replay_step_split(s: Shape, L0: int, fold: bool, T: int = 1) -> dict:
     folded into the checkpoint by this call (then the read kernel skips the head).
     """
     x, k = _x_row(s), _key_row(s)
-    scal = 4 if s.kind == "mamba2" else 8  # dt, or alpha + beta
-    q = k  # Mamba-2 C (group-shared), GDN q
+    scal = _scalars(s)
+    q = k  # Mamba-2 C (group-shared), GDN / KDA q
     prep = {
         "buffer_read": L0 * (k + scal) + (L0 * x if fold else 0.0),
         "inputs": T * (q + k + scal + x),
@@ -67,9 +78,7 @@ def replay_step_split(s: Shape, L0: int, fold: bool, T: int = 1) -> dict:
         prep["copy_write"] = state_tile(s, s.read_dtype) if s.read_dtype != "f32" else 0.0
         prep["output"] = T * s.headdim * 4
     else:
-        # Mamba-2 hands per-head coefficients to the read kernel; the Gated
-        # DeltaNet path is one kernel and hands nothing over
-        prep["handoff_write"] = T * ((L0 + T) * 4 + 4) if s.kind == "mamba2" else 0.0
+        prep["handoff_write"] = _handoff(s, L0, T)
         read = {
             "copy_read": state_tile(s, s.read_dtype),
             "buffer_read": L0 * x,
@@ -104,7 +113,7 @@ def replay_decode_per_token(s: Shape) -> dict:
 def eager_decode_per_token(s: Shape, state_dtype: str = "f32") -> dict:
     x, k = _x_row(s), _key_row(s)
     t = state_tile(s, state_dtype)
-    return {"inputs": (2 * k if s.kind == "mamba2" else 2 * k) + x + (4 if s.kind == "mamba2" else 8),
+    return {"inputs": 2 * k + x + _scalars(s),
             "output": s.headdim * 4, "state_read": t, "state_write": t}
 
 

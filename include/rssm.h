@@ -18,11 +18,12 @@
  * "La fiche qu'on reecrit a chaque token").
  *
  * Layer recurrences, per sequence b and head h (S is headdim x dstate for
- * Mamba-2, d_v x d_k for Gated DeltaNet; rows contiguous along dstate / d_k):
+ * Mamba-2, d_v x d_k for Gated DeltaNet and KDA; rows contiguous along dstate / d_k):
  *   Mamba-2:  S_t = exp(dt_t A_h) S_{t-1} + (s_t x_t) B_t^T,  y_t = S_t C_t + D_h x_t,
  *             s_t = dt_t when cfg.dt_scales_input else 1; B, C shared by the
  *             nheads/ngroups heads of a group.
  *   GDN:      S_t = alpha_t S_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,  o_t = S_t q_t.
+ *   KDA:      S_t = S_{t-1} Diag(alpha_t) (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,  o_t = S_t q_t.
  *
  * Conventions shared by every call:
  *   - The library allocates no device memory.  The caller owns the workspace
@@ -65,7 +66,14 @@ typedef enum {
     RSSM_EDEVICE = 4  /* the device error word is set (rssm_status_word) */
 } rssm_status;
 
-typedef enum { RSSM_MAMBA2 = 0, RSSM_GDN = 1 } rssm_kind;
+/* MAMBA2: S_t = exp(dt_t A_h) S_{t-1} + x_t B_t^T, y_t = S_t C_t + D_h x_t.
+ * GDN (Gated DeltaNet): S_t = alpha_t S_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t k_t^T, o_t = S_t q_t.
+ * KDA (Kimi Delta Attention): GDN with a gate per key channel,
+ *      S_t = S_{t-1} Diag(alpha_t) (I - beta_t k_t k_t^T) + beta_t v_t k_t^T, o_t = S_t q_t
+ * (the three layer kinds of the hybrid models on blog.thibaultmonteiro.fr, "Des couches
+ * rapides sur le papier"; the page names KDA without a formula, and the one above is the
+ * plainest reading: the GDN update with the scalar gate made a diagonal). */
+typedef enum { RSSM_MAMBA2 = 0, RSSM_GDN = 1, RSSM_KDA = 2 } rssm_kind;
 
 /* REPLAY: checkpoint + read copy + input buffer.  EAGER: one state, read and
  * rewritten every token (the baseline); with state_dtype BF16 or FP8E4M3 this is
@@ -91,13 +99,13 @@ typedef struct {
     int32_t state_dtype; /* REPLAY: read-copy dtype (F32 = no copy, outputs read the fp32
                             checkpoint).  EAGER: dtype the single state is stored in.
                             FP8E4M3 uses one fp32 scale per state row (amax / 448). */
-    int32_t input_dtype; /* F32 | BF16: dtype of x, B, C (Mamba-2) or q, k, v (GDN);
+    int32_t input_dtype; /* F32 | BF16: dtype of x, B, C (Mamba-2) or q, k, v (GDN, KDA);
                             the buffer stores them as given.  dt, alpha, beta are fp32. */
     int32_t batch;       /* sequences B >= 1 */
     int32_t nheads;      /* heads H >= 1 */
-    int32_t headdim;     /* P: Mamba-2 headdim, GDN d_v; a multiple of 8 in 8..256 */
-    int32_t dstate;      /* N: Mamba-2 dstate, GDN d_k; one of 16, 32, 64, 128 */
-    int32_t ngroups;     /* Mamba-2: G >= 1 dividing H (B/C per group).  GDN: ignored */
+    int32_t headdim;     /* P: Mamba-2 headdim, GDN/KDA d_v; a multiple of 8 in 8..256 */
+    int32_t dstate;      /* N: Mamba-2 dstate, GDN/KDA d_k; one of 16, 32, 64, 128 */
+    int32_t ngroups;     /* Mamba-2: G >= 1 dividing H (B/C per group).  GDN, KDA: ignored */
     int32_t window;      /* W: buffer window, 1..64 */
     int32_t max_draft;   /* largest K accepted by rssm_verify, 0..8 and <= W */
     int32_t dt_scales_input; /* Mamba-2 only: 1 = input term dt_t x_t B_t^T, 0 = x_t B_t^T */
@@ -119,10 +127,11 @@ typedef struct {
     size_t ring;                         /* R = window + max(max_draft, 1) slots   */
     size_t ring_stride;                  /* R rounded up to a multiple of 4: row length of the
                                             fp32 scalar rings below (16-byte rows) */
-    size_t xbuf_off, xbuf_bytes;         /* Mamba-2 x[B][H][R][P]; GDN v[B][H][R][P] (input_dtype) */
-    size_t bbuf_off, bbuf_bytes;         /* Mamba-2 B[B][G][R][N]; GDN k[B][H][R][N] (input_dtype) */
-    size_t sbuf_off, sbuf_bytes;         /* Mamba-2 dt[B][H][ring_stride]; GDN alpha (fp32)        */
-    size_t tbuf_off, tbuf_bytes;         /* GDN beta[B][H][ring_stride] (fp32)                     */
+    size_t xbuf_off, xbuf_bytes;         /* Mamba-2 x[B][H][R][P]; GDN/KDA v[B][H][R][P] (input_dtype) */
+    size_t bbuf_off, bbuf_bytes;         /* Mamba-2 B[B][G][R][N]; GDN/KDA k[B][H][R][N] (input_dtype) */
+    size_t sbuf_off, sbuf_bytes;         /* Mamba-2 dt[B][H][ring_stride]; GDN alpha[B][H][ring_stride];
+                                            KDA alpha[B][H][R][N] (fp32)                              */
+    size_t tbuf_off, tbuf_bytes;         /* GDN/KDA beta[B][H][ring_stride] (fp32)                 */
     size_t snap_off, snap_bytes;         /* EAGER: max_draft snapshots of the state (+ scales)      */
     /* REPLAY: hand-off from the prep kernel to the read kernel within one call */
     size_t tq_max;                       /* max(max_draft, 1): queries per call            */
@@ -130,7 +139,7 @@ typedef struct {
                                             work list: int32 count, 3 pad, int32[B] (padded) */
     size_t dec_off, dec_bytes;           /* fp32[B][H][tq_max]                             */
     size_t coef_off, coef_bytes;         /* fp32[B][H][tq_max][window + tq_max, padded to 4] */
-    size_t query_off, query_bytes;       /* GDN: fp32[B][H][tq_max][dstate] swept queries  */
+    size_t query_off, query_bytes;       /* GDN/KDA: fp32[B][H][tq_max][dstate] swept queries */
     size_t total_bytes;
 } rssm_workspace_layout;
 
@@ -140,11 +149,11 @@ typedef struct {
     const float *dt;    /* Mamba-2 [B][T][H] fp32 (already softplus-ed, > 0 expected) */
     const void *Bm;     /* Mamba-2 [B][T][G][N] input_dtype */
     const void *Cm;     /* Mamba-2 [B][T][G][N] input_dtype */
-    const void *q;      /* GDN [B][T][H][N] input_dtype */
-    const void *k;      /* GDN [B][T][H][N] input_dtype */
-    const void *v;      /* GDN [B][T][H][P] input_dtype */
-    const float *alpha; /* GDN [B][T][H] fp32 */
-    const float *beta;  /* GDN [B][T][H] fp32 */
+    const void *q;      /* GDN/KDA [B][T][H][N] input_dtype */
+    const void *k;      /* GDN/KDA [B][T][H][N] input_dtype */
+    const void *v;      /* GDN/KDA [B][T][H][P] input_dtype */
+    const float *alpha; /* GDN [B][T][H] fp32; KDA [B][T][H][N] fp32, 16-byte aligned */
+    const float *beta;  /* GDN/KDA [B][T][H] fp32 */
 } rssm_inputs;
 
 typedef struct rssm_ctx *rssm_handle;

@@ -5,7 +5,7 @@ import numpy as np
 
 from checkpoint_input_replay_rssm_b200 import inputs as I
 
-WIDE = {"mamba2": ("x", "B", "C"), "gdn": ("q", "k", "v")}
+WIDE = {"mamba2": ("x", "B", "C"), "gdn": ("q", "k", "v"), "kda": ("q", "k", "v")}
 
 
 def make_layer(wl: I.Workload, mode="replay", state_dtype=None, max_draft=None, dt_scales=False,
