@@ -238,6 +238,18 @@ __device__ __forceinline__ void cp_async4(void *smem, const void *gmem) {
 __device__ __forceinline__ void cp_async_wait_all() {
     asm volatile("cp.async.wait_all;" ::: "memory");
 }
+// Programmatic dependent launch.  A kernel that triggers lets the next kernel of
+// its stream, when that one is launched with programmatic stream serialization,
+// be scheduled once every CTA of this grid has triggered or exited; the next
+// kernel's wait returns when this grid has completed and its writes are visible.
+// Without such a launch both are no-ops.
+__device__ __forceinline__ void pdl_trigger() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 // Close the copies issued so far into a group (an empty group is allowed), and
 // wait until at most `Pending` of the most recent groups are still in flight.
 __device__ __forceinline__ void cp_async_commit() {

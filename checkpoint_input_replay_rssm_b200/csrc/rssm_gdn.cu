@@ -84,7 +84,7 @@ cudaError_t gdn_launch(Ctx &h, int op, int T, const rssm_inputs *in, float *y, f
         // swept queries r ([B][H][TQmax][N], fp32) against the read copy; x = v
         h.launches += 1;
         e = launch_read(h, op, T, ho.query, 0, 1, (int64_t)cf.nheads * a.TQmax * N, (int64_t)a.TQmax * N, N, in->v,
-                        nullptr, y, ho, st);
+                        nullptr, y, ho, st, !fold, !h.split_event);
     }
     if (e != cudaSuccess) {
         cudaMemsetAsync(ho.fold_count, 0, sizeof(int), st);

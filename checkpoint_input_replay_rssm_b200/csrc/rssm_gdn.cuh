@@ -517,6 +517,7 @@ __global__ void __launch_bounds__(kThreads) gdn_prep_kernel(const GArgs a) {
     const int H = a.H, P = a.P, W = a.W, R = a.R, T = a.T;
     const int E = W + TQ, Ea = (E + 3) & ~3;
     const int b = blockIdx.y, h = blockIdx.x * a.prep_heads + warp;
+    pdl_trigger();  // the read kernel may be scheduled as this grid's last CTAs run
     if (tid == 0) {
         const SeqState ss = read_counters(a.c, b, W);
         const int L0 = (int)(ss.seq - ss.ckpt);

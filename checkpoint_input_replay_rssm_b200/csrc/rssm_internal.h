@@ -96,10 +96,12 @@ inline void update_len_bounds(Ctx &h, int op, int T) {
 size_t gdn_smem_bytes(const rssm_config &cf, int T);
 
 // The replay-read kernel (rssm_read.cu), shared by both kinds: queries Q[b][row][m][n]
-// at the given element strides, q_group heads per query row.
+// at the given element strides, q_group heads per query row.  `early`: no flush
+// kernel ran in the call (every sequence is read); `pdl`: the kernel directly
+// follows the prep kernel in the stream and is launched as its programmatic dependent.
 cudaError_t launch_read(const Ctx &h, int op, int T, const void *Q, int q_bf16, int q_group, int64_t q_stride_b,
                         int64_t q_stride_row, int64_t q_stride_m, const void *xnew, const float *D,
-                        float *y, const Handoff &ho, cudaStream_t st);
+                        float *y, const Handoff &ho, cudaStream_t st, bool early, bool pdl);
 int read_heads_per_cta(const rssm_config &cf);
 size_t read_smem_bytes(const rssm_config &cf, int T);
 

@@ -129,7 +129,7 @@ cudaError_t mamba2_launch(Ctx &h, int op, int T, const rssm_inputs *in, float *y
         const int G = cf.ngroups;
         h.launches += 1;
         e = launch_read(h, op, T, in->Cm, ib == 2, cf.nheads / G, (int64_t)T * G * N, N, (int64_t)G * N, in->x,
-                        (const float *)h.at(h.lay.D_off), y, ho, st);
+                        (const float *)h.at(h.lay.D_off), y, ho, st, !fold, !h.split_event);
     }
     if (e != cudaSuccess) {  // leave no stale work list behind
         cudaMemsetAsync(ho.fold_count, 0, sizeof(int), st);

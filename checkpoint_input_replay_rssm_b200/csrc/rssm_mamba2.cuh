@@ -123,6 +123,8 @@ __global__ void __launch_bounds__(kThreads, 6) m2_prep_kernel(const M2Args a) {
         return BF ? bf16_bits_to_float(*reinterpret_cast<const uint16_t *>(p)) : *reinterpret_cast<const float *>(p);
     };
 
+    pdl_trigger();  // the read kernel may be scheduled as this grid's last CTAs run
+
     // 1. Counters (thread 0) and everything that does not depend on them, at once.
     if (tid == 0) {
         const SeqState ss = read_counters(a.c, b, W);

@@ -47,7 +47,7 @@ size_t read_smem_bytes(const rssm_config &cf, int T) {
 
 cudaError_t launch_read(const Ctx &h, int op, int T, const void *Q, int q_bf16, int q_group, int64_t q_stride_b,
                         int64_t q_stride_row, int64_t q_stride_m, const void *xnew, const float *D,
-                        float *y, const Handoff &ho, cudaStream_t st) {
+                        float *y, const Handoff &ho, cudaStream_t st, bool early, bool pdl) {
     const rssm_config &cf = h.cfg;
     ReadArgs r{};
     r.B = cf.batch; r.H = cf.nheads; r.P = cf.headdim; r.R = (int)h.lay.ring; r.W = cf.window;
@@ -69,6 +69,8 @@ cudaError_t launch_read(const Ctx &h, int op, int T, const void *Q, int q_bf16, 
     r.c = h.counters();
     r.fold_count = ho.fold_count;
     r.op = op;
+    r.early = early ? 1 : 0;
+    r.pdl = (early && pdl) ? 1 : 0;
     const int TQ = tq_of_read(T);
     r.lay = read_lay(r.HC, cf.headdim, cf.dstate, cf.window, TQ, cf.input_dtype == RSSM_BF16 ? 2 : 4, r.Emax);
     const size_t smem = read_smem_bytes(cf, T);

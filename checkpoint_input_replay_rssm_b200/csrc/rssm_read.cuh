@@ -16,7 +16,13 @@
 // (128-bit, L1 no-allocate) first -- they depend on nothing -- then the CTA
 // stages the small operands, dots the rows with the query (LPR lanes per row,
 // chunks interleaved so each warp load covers whole 64-byte row segments), and
-// applies the replay term.  Only ordinary loads and cp.async are used.
+// applies the replay term.  Only ordinary loads and cp.async are used.  When no
+// flush kernel ran in the call, the kernel is launched as a programmatic
+// dependent of the prep kernel: its first round of copy loads overlaps the prep
+// kernel's last CTAs, and it waits for the prep kernel's hand-off before
+// reading anything the prep kernel wrote (or rewriting the counters it read).
+// After a flush kernel, the CTA first learns whether its sequence was folded
+// (a folded sequence needs no read copy).
 #pragma once
 
 #include "rssm_device.cuh"
@@ -65,6 +71,9 @@ struct ReadArgs {
     int TQmax, Emax;        // Emax: padded row length of the coefficient table
     ReadLay lay;            // shared memory, computed on the host
     float *y;               // [B][T][H][P]
+    int early;              // no flush kernel ran in this call: every sequence is read, so the
+                            // first read-copy round is issued before anything else
+    int pdl;                // launched as a programmatic dependent of the prep kernel
 };
 
 template <int N, int RK, int TQ, bool BF>
@@ -111,7 +120,14 @@ __global__ void __launch_bounds__(kThreads, TQ == 1 ? 4 : 2) replay_read_kernel(
                 if (r < nrows) rv[j * CPL + k] = ld_stream(tile + ((size_t)r * TPR + q + LPR * k) * 16);
         }
     };
-    issue(0);
+    bool skip_copy = false;  // folded in this call: served by the flush kernel
+    if (!a.early) {          // a flush kernel ran in this call
+        if (tid == 0) sinfo[2] = a.seqinfo[b].z;
+        __syncthreads();
+        skip_copy = sinfo[2] != 0;
+    }
+    if (!skip_copy) issue(0);
+    pdl_wait();  // the prep kernel's hand-off is complete and visible
 
     // 2. Small operands: per-sequence info, the call's entries, decays, the
     //    coefficient rows of the CTA's heads (contiguous), queries, fp8 scales.
@@ -163,7 +179,7 @@ __global__ void __launch_bounds__(kThreads, TQ == 1 ? 4 : 2) replay_read_kernel(
         for (int i = tid; i < nrows / 4; i += kThreads) cp_async16(ssc + 4 * i, a.rc_scale + row0 * P + 4 * i);
     __syncthreads();
     const int L0 = sinfo[0], ckmod = sinfo[1], folded = sinfo[2];
-    if (folded) {  // served by the prep kernel
+    if (folded) {  // served by the flush kernel
         cp_async_wait_all();
         return;
     }
@@ -255,8 +271,17 @@ inline cudaError_t launch_read_t(const ReadArgs &r, size_t smem, cudaStream_t st
     auto k = r.in_bf16 ? replay_read_kernel<N, RK, TQ, true> : replay_read_kernel<N, RK, TQ, false>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    k<<<dim3(r.H / r.HC, r.B), kThreads, smem, st>>>(r);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(r.H / r.HC, r.B);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = r.pdl ? 1 : 0;  // a programmatic dependent of the prep kernel
+    return cudaLaunchKernelEx(&cfg, k, r);
 }
 
 template <int N>
