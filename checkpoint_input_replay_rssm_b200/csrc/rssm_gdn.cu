@@ -12,7 +12,8 @@ extern template cudaError_t g_dispatch_n<128>(bool, int, int, const GArgs &, siz
 static int gtq_of(int T) { return T <= 1 ? 1 : (T <= 4 ? 4 : 8); }
 
 size_t gdn_smem_bytes(const rssm_config &cf, int T) {
-    return sizeof(float) * gdn_smem_floats(cf.headdim, cf.dstate, cf.window, gtq_of(T), cf.kind == RSSM_KDA);
+    return sizeof(float) * gdn_smem_floats(cf.headdim, cf.dstate, cf.window, gtq_of(T), cf.kind == RSSM_KDA,
+                                           cf.input_dtype == RSSM_BF16 ? 2 : 4);
 }
 
 cudaError_t gdn_launch(Ctx &h, int op, int T, const rssm_inputs *in, float *y, float *out, cudaStream_t st) {

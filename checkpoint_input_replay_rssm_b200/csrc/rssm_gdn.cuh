@@ -51,19 +51,28 @@ struct GArgs {
 
 __host__ __device__ constexpr int gpad4(int n) { return (n + 3) & ~3; }
 
-// KDA keeps a gate row [E][N] where GDN keeps one gate per entry.
-__host__ __device__ inline size_t gdn_smem_floats(int P, int N, int W, int TQ, int kda) {
+// KDA keeps a gate row [E][N] where GDN keeps one gate per entry.  After the
+// working arrays, the raw rings (k, v in the input dtype, gates and beta fp32) as
+// staged from global memory, ring slot order, R <= W + 8 slots.
+__host__ __device__ inline size_t gdn_raw_floats(int P, int N, int W, int ib, int kda) {
+    const int Rm = W + 8;
+    return (size_t)gpad4(Rm * N * ib / 4) + gpad4(Rm * P * ib / 4) + gpad4(kda ? Rm * N : Rm) + gpad4(Rm);
+}
+__host__ __device__ inline size_t gdn_smem_floats(int P, int N, int W, int TQ, int kda, int ib) {
     const int E = W + TQ;
     return (size_t)gpad4(E * N) + gpad4(E * P) + gpad4(kda ? E * N : E) + 2 * (size_t)gpad4(E) + gpad4(TQ * N) +
-           gpad4(E * E) + 2 * (size_t)gpad4(TQ * E) + gpad4(TQ * N) + gpad4(TQ * P) + gpad4(TQ) + 8;
+           gpad4(E * E) + 2 * (size_t)gpad4(TQ * E) + gpad4(TQ * N) + gpad4(TQ * P) + gpad4(TQ) + 8 +
+           gdn_raw_floats(P, N, W, ib, kda);
 }
 
 struct GSmem {
     float *sk, *sv, *sal, *sbe, *spr, *sq, *sG, *shq, *sc, *sr, *sdot, *srq;
     int *si;
+    uint8_t *rk, *rv;  // raw k, v rings [R][N], [R][P] (input dtype)
+    float *ra, *rb;    // raw gate ring ([Rs], KDA [R][N]) and beta ring [Rs]
 };
 
-__device__ __forceinline__ GSmem gdn_carve(float *sm, int P, int N, int W, int TQ, int kda) {
+__device__ __forceinline__ GSmem gdn_carve(float *sm, int P, int N, int W, int TQ, int kda, int ib) {
     const int E = W + TQ;
     GSmem s;
     s.sk = sm;                            // [E][N]  k of entries (physical)
@@ -79,12 +88,34 @@ __device__ __forceinline__ GSmem gdn_carve(float *sm, int P, int N, int W, int T
     s.sdot = s.sr + gpad4(TQ * N);        // [TQ][P] S^ r per row
     s.srq = s.sdot + gpad4(TQ * P);       // [TQ]    unused pad
     s.si = reinterpret_cast<int *>(s.srq + gpad4(TQ));
+    float *raw = s.srq + gpad4(TQ) + 8;
+    const int Rm = W + 8;
+    s.rk = reinterpret_cast<uint8_t *>(raw);
+    s.rv = s.rk + 4 * gpad4(Rm * N * ib / 4);
+    s.ra = reinterpret_cast<float *>(s.rv + 4 * gpad4(Rm * P * ib / 4));
+    s.rb = s.ra + gpad4(kda ? Rm * N : Rm);
     return s;
 }
 
-// Fold-mapping: TPRF lanes per state row, NPT contiguous elements per lane.
+// 16 bytes of raw inputs (8 bf16 or 4 fp32) to fp32 in shared memory.
+__device__ __forceinline__ void raw16_to_f32(const uint8_t *src, float *dst, int bf16) {
+    const uint4 u = *reinterpret_cast<const uint4 *>(src);
+    if (bf16) {
+        reinterpret_cast<float4 *>(dst)[0] = make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xffff0000u),
+                                                         __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xffff0000u));
+        reinterpret_cast<float4 *>(dst)[1] = make_float4(__uint_as_float(u.z << 16), __uint_as_float(u.z & 0xffff0000u),
+                                                         __uint_as_float(u.w << 16), __uint_as_float(u.w & 0xffff0000u));
+    } else {
+        *reinterpret_cast<float4 *>(dst) = make_float4(__uint_as_float(u.x), __uint_as_float(u.y),
+                                                       __uint_as_float(u.z), __uint_as_float(u.w));
+    }
+}
+
+// Fold-mapping: TPRF lanes per state row, NPT contiguous elements per lane
+// (16 lanes x 8 at d_k = 128: half the state registers of 8 x 16, so three CTAs
+// share an SM and hide the per-token reduction chain).
 template <int N> struct FoldMap {
-    static constexpr int TPRF = (N >= 32) ? 8 : N / 4;
+    static constexpr int TPRF = (N >= 64) ? 16 : (N >= 32 ? 8 : N / 4);
     static constexpr int NPT = N / TPRF;
     static constexpr int RPPF = kThreads / TPRF;
 };
@@ -139,13 +170,15 @@ __device__ __forceinline__ void gdn_fold_rows(float (&st)[NR][FoldMap<N>::NPT], 
             }
 #pragma unroll
             for (int r = 0; r < NR; ++r) {
-                float d = 0.f;
+                float d0 = 0.f, d1 = 0.f;  // two chains: half the dependent latency
 #pragma unroll
-                for (int j = 0; j < NPT; ++j) {
+                for (int j = 0; j < NPT; j += 2) {
                     st[r][j] *= ga[j];
-                    d = fmaf(st[r][j], kk[j], d);
+                    st[r][j + 1] *= ga[j + 1];
+                    d0 = fmaf(st[r][j], kk[j], d0);
+                    d1 = fmaf(st[r][j + 1], kk[j + 1], d1);
                 }
-                d = group_sum<TPRF>(d);
+                const float d = group_sum<TPRF>(d0 + d1);
                 const float vr = (rows[r] < P) ? s.sv[(base + e) * P + rows[r]] : 0.f;
                 const float coef = be * (vr - d);
 #pragma unroll
@@ -156,10 +189,13 @@ __device__ __forceinline__ void gdn_fold_rows(float (&st)[NR][FoldMap<N>::NPT], 
         const float al = s.sal[base + e];
 #pragma unroll
         for (int r = 0; r < NR; ++r) {
-            float d = 0.f;
+            float d0 = 0.f, d1 = 0.f;  // two chains: half the dependent latency
 #pragma unroll
-            for (int j = 0; j < NPT; ++j) d = fmaf(st[r][j], kk[j], d);
-            d = group_sum<TPRF>(d);
+            for (int j = 0; j < NPT; j += 2) {
+                d0 = fmaf(st[r][j], kk[j], d0);
+                d1 = fmaf(st[r][j + 1], kk[j + 1], d1);
+            }
+            const float d = group_sum<TPRF>(d0 + d1);
             const float vr = (rows[r] < P) ? s.sv[(base + e) * P + rows[r]] : 0.f;
             const float coef = be * vr - al * be * d;
 #pragma unroll
@@ -172,7 +208,7 @@ __device__ __forceinline__ void gdn_fold_rows(float (&st)[NR][FoldMap<N>::NPT], 
 // Replay kernel: decode (T = 1), verify (T = K), flush (T = 0), export (T = 0).
 // ---------------------------------------------------------------------------
 template <int N, int RK, int TQ>
-__global__ void __launch_bounds__(kThreads) gdn_replay_kernel(const GArgs a) {
+__global__ void __launch_bounds__(kThreads, TQ == 1 ? 3 : 1) gdn_replay_kernel(const GArgs a) {
     constexpr int EPC = Chunk<RK>::EPC;
     constexpr int TPR = N / EPC;
     constexpr int RPP = kThreads / TPR;
@@ -187,7 +223,8 @@ __global__ void __launch_bounds__(kThreads) gdn_replay_kernel(const GArgs a) {
     const int H = a.H, P = a.P, W = a.W, R = a.R, T = a.T;
     const int b = bh / H, h = bh - b * H;
     const int E = W + TQ;
-    GSmem s = gdn_carve(smem, P, N, W, TQ, a.kda);
+    const int ib = a.in_bf16 ? 2 : 4;
+    GSmem s = gdn_carve(smem, P, N, W, TQ, a.kda, ib);
     const int64_t tile0 = (int64_t)bh * P * N;
     const bool reads = (a.op == OP_DECODE || a.op == OP_VERIFY);
 
@@ -208,7 +245,21 @@ __global__ void __launch_bounds__(kThreads) gdn_replay_kernel(const GArgs a) {
         }
     }
 
-    // 2. Counters and new-token staging.
+    // 2. The whole rings (raw, slot order: none of it depends on the counters),
+    //    the counters and the new tokens, in one round trip.
+    {
+        const uint8_t *ks = reinterpret_cast<const uint8_t *>(a.kbuf) + (int64_t)bh * R * N * ib;
+        for (int i = tid; i < R * N * ib / 16; i += kThreads) cp_async16(s.rk + 16 * i, ks + 16 * i);
+        const uint8_t *vs = reinterpret_cast<const uint8_t *>(a.vbuf) + (int64_t)bh * R * P * ib;
+        for (int i = tid; i < R * P * ib / 16; i += kThreads) cp_async16(s.rv + 16 * i, vs + 16 * i);
+        if (a.kda) {
+            const float *as = a.abuf + (int64_t)bh * R * N;
+            for (int i = tid; i < R * N / 4; i += kThreads) cp_async16(s.ra + 4 * i, as + 4 * i);
+        } else {
+            for (int i = tid; i < a.Rs / 4; i += kThreads) cp_async16(s.ra + 4 * i, a.abuf + (int64_t)bh * a.Rs + 4 * i);
+        }
+        for (int i = tid; i < a.Rs / 4; i += kThreads) cp_async16(s.rb + 4 * i, a.bbuf + (int64_t)bh * a.Rs + 4 * i);
+    }
     if (tid == 0) {
         SeqState ss = read_counters(a.c, b, W);
         const int L0 = (int)(ss.seq - ss.ckpt);
@@ -229,6 +280,7 @@ __global__ void __launch_bounds__(kThreads) gdn_replay_kernel(const GArgs a) {
         }
     }
     gdn_stage_new(a, s, b, h, N, tid);
+    cp_async_wait_all();
     __syncthreads();
     if (!s.si[0]) return;
     const int L0 = s.si[1], flush = s.si[2], ckmod = s.si[3], spmod = s.si[4];
@@ -237,25 +289,31 @@ __global__ void __launch_bounds__(kThreads) gdn_replay_kernel(const GArgs a) {
     const int nE = L0 + T;
     const int e0 = flush ? L0 : 0;
 
-    // 3. Buffered entries.
-    for (int i = tid; i < L0 * N; i += kThreads) {
-        const int e = i / N, n = i - e * N;
-        s.sk[(base + e) * N + n] = ld_in(a.kbuf, ((int64_t)bh * R + (ckmod + e) % R) * N + n, a.in_bf16);
-    }
-    for (int i = tid; i < L0 * P; i += kThreads) {
-        const int e = i / P, p = i - e * P;
-        s.sv[(base + e) * P + p] = ld_in(a.vbuf, ((int64_t)bh * R + (ckmod + e) % R) * P + p, a.in_bf16);
-    }
-    for (int e = tid; e < L0; e += kThreads) {
-        const int64_t slot = (int64_t)bh * a.Rs + (ckmod + e) % R;
-        if (!a.kda) s.sal[base + e] = a.abuf[slot];
-        s.sbe[base + e] = a.bbuf[slot];
-    }
-    if (a.kda)
-        for (int i = tid; i < L0 * N; i += kThreads) {
-            const int e = i / N, n = i - e * N;
-            s.sal[(base + e) * N + n] = a.abuf[((int64_t)bh * R + (ckmod + e) % R) * N + n];
+    // 3. Buffered entries, from the staged rings (slot (ckmod + e) mod R) to fp32
+    //    rows at their physical entries base + e.
+    {
+        const int kc = N * ib / 16, vc = P * ib / 16;  // 16-byte chunks per row
+        auto slot_of = [&](int e) { const int sl = ckmod + e; return sl >= R ? sl - R : sl; };
+        for (int i = tid; i < L0 * kc; i += kThreads) {
+            const int e = i / kc, c2 = i - e * kc;
+            raw16_to_f32(s.rk + (slot_of(e) * kc + c2) * 16, s.sk + (base + e) * N + c2 * (16 / ib), a.in_bf16);
         }
+        for (int i = tid; i < L0 * vc; i += kThreads) {
+            const int e = i / vc, c2 = i - e * vc;
+            raw16_to_f32(s.rv + (slot_of(e) * vc + c2) * 16, s.sv + (base + e) * P + c2 * (16 / ib), a.in_bf16);
+        }
+        if (a.kda) {
+            for (int i = tid; i < L0 * (N / 4); i += kThreads) {
+                const int e = i / (N / 4), c4 = i - e * (N / 4);
+                *reinterpret_cast<float4 *>(s.sal + (base + e) * N + 4 * c4) =
+                    *reinterpret_cast<const float4 *>(s.ra + slot_of(e) * N + 4 * c4);
+            }
+        }
+        for (int e = tid; e < L0; e += kThreads) {
+            if (!a.kda) s.sal[base + e] = s.ra[slot_of(e)];
+            s.sbe[base + e] = s.rb[slot_of(e)];
+        }
+    }
     __syncthreads();
 
     if (reads && a.kda) {
@@ -665,7 +723,7 @@ __global__ void __launch_bounds__(kThreads) gdn_eager_kernel(const GArgs a) {
     const int bh = blockIdx.x;
     const int H = a.H, P = a.P, T = a.T, W = a.W;
     const int b = bh / H, h = bh - b * H;
-    GSmem s = gdn_carve(smem, P, N, W, TQ, a.kda);
+    GSmem s = gdn_carve(smem, P, N, W, TQ, a.kda, a.in_bf16 ? 2 : 4);
     const int64_t tile0 = (int64_t)bh * P * N;
     void *state = (SK == SK_F32) ? (void *)a.ckpt : a.rc;
     const int64_t state_elems = (int64_t)a.B * H * P * N;
