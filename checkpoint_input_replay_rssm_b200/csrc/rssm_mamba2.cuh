@@ -617,7 +617,7 @@ __global__ void __launch_bounds__(kThreads, 3) m2_fold_kernel(const M2Args a, co
                 }
                 const float *Ur = U + (hh * L0) * P + p0;
                 const float *Br = Bf + 4 * q;
-#pragma unroll 2
+#pragma unroll 4
                 for (int e = 0; e < L0; ++e) {
                     const float4 u = *reinterpret_cast<const float4 *>(Ur + e * P);
                     const float4 bb = *reinterpret_cast<const float4 *>(Br + e * N);
