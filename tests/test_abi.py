@@ -147,3 +147,30 @@ def test_product_path_has_no_oracle_or_fallback():
                 txt = open(os.path.join(dirpath, f)).read()
                 assert "import oracle" not in txt and "from oracle" not in txt, f
                 assert "oracle/" not in txt, f
+
+
+def test_kda_layout_keeps_a_gate_row_per_buffered_token(lib):
+    """Kimi Delta Attention: the gate ring holds d_k fp32 per slot ([B][H][R][N]); GDN one
+    gate per slot ([B][H][ring_stride]); both keep beta and the swept-query hand-off."""
+    kw = dict(nheads=32, headdim=128, dstate=128, ngroups=32)
+    g = rssm.rssm_workspace_layout_of(_cfg(kind="gdn", **kw))
+    k = rssm.rssm_workspace_layout_of(_cfg(kind="kda", **kw))
+    R, Rs = 17, 20
+    assert g.sbuf_bytes == 256 * 32 * Rs * 4
+    assert k.sbuf_bytes == 256 * 32 * R * 128 * 4
+    for lay in (g, k):
+        assert lay.tbuf_bytes == 256 * 32 * Rs * 4
+        assert lay.query_bytes == 256 * 32 * 1 * 128 * 4
+        assert lay.bbuf_bytes == 256 * 32 * R * 128 * 2 and lay.xbuf_bytes == 256 * 32 * R * 128 * 2
+    assert k.total_bytes - g.total_bytes >= k.sbuf_bytes - g.sbuf_bytes - 256
+
+
+def test_kda_config_rules(lib):
+    """KDA is validated like GDN: no dt scaling of the input; groups ignored."""
+    assert rssm.rssm_workspace_bytes(_cfg(kind="kda", nheads=4, ngroups=3)) > 0
+    cfg = _cfg(kind="kda")
+    cfg.dt_scales_input = 1
+    assert rssm.rssm_workspace_bytes(cfg) == 0
+    cfg = _cfg()
+    cfg.kind = 3
+    assert rssm.rssm_workspace_bytes(cfg) == 0
