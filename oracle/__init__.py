@@ -9,6 +9,7 @@ it: only tests/, the smoke check and the benchmark's CPU-baseline leg may.
                       Kimi Delta Attention), OpenMP
   closed_form.py      brute-force unrolled closed forms (tiny inputs)
   ut_form.py          chunked (WY / UT) fold of the delta-rule layers
+  prefill.py          chunked Mamba-2 prefill (outputs and the checkpoint after a prompt)
   replay.py           fp64 checkpoint + buffer formulation, and the single
                       low-precision-state eager comparator
   ring.py             integer model of counters, ring slots, flush, verify/commit
