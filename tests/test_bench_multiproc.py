@@ -70,3 +70,26 @@ def test_single_process_reduction_is_identity():
     import bench
 
     assert bench.max_over_ranks(None, [1.5, 2], None) == [1.5, 2.0]
+
+
+def test_reference_arm_prints_the_contract_line(capsys, oracle_built):
+    """Rank 0 of the reference arm (the fp64 oracle on the host cores) prints one JSON
+    line with the benchmark's keys, the same metric and unit as the main arm."""
+    import argparse
+    import json
+
+    import bench
+
+    bench.run_reference(argparse.Namespace(steps=2, warmup=3, gpus=1), rank=0)
+    lines = [l for l in capsys.readouterr().out.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "impl", "cpu_baseline", "e2e"):
+        assert key in d, key
+    assert d["impl"] == "reference" and d["metric"] == bench.METRIC and d["unit"] == "tokens/s"
+    assert d["steps"] == 2 and d["warmup"] == 3 and d["value"] > 0 and d["higher_is_better"] is True
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    assert d["cpu_baseline"]["value"] == d["value"]
+    assert d["e2e"] == {"value": d["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+    assert d["config"]["workload"] == bench.WL.name
