@@ -9,7 +9,7 @@ appended to the buffer and a rejection only moves the buffer pointer, never
 touching the checkpoint ("Un retour en arriere qui devient trivial",
 irisproject.cloud).
 
-Readings of what the pages leave open (each is listed in the design notes):
+Readings of what the pages leave open:
 * counters per sequence: ``seq_pos`` = committed tokens, ``ckpt_pos`` = tokens
   folded into the checkpoint, ``len = seq_pos - ckpt_pos`` in [0, W];
 * lazy flush: before appending n tokens, fold the committed entries if
