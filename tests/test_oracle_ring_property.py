@@ -2,7 +2,10 @@
 the buffer: per sequence, the list of committed-but-unfolded token indices and the
 pending drafts, with the lazy flush rule (fold before appending n tokens when
 len + n > W).  Random op sequences (hypothesis) must give the same counters after
-every op, and the ring slots of the live entries must stay distinct."""
+every op, and the ring slots of the live entries must stay distinct: after a
+verify (drafts pending, possibly after a fold in the same call) and again after
+its commit.  Within each call, the slots it appends to must also avoid the
+entries the call's own fold reads."""
 import numpy as np
 from hypothesis import given, settings
 from hypothesis import strategies as st
@@ -55,6 +58,27 @@ ops = st.lists(st.tuples(st.sampled_from(["decode", "verify", "flush"]), st.inte
                          st.lists(st.integers(-1, 9), min_size=3, max_size=3)), max_size=60)
 
 
+def _check(rm, lm, W):
+    """Counters equal, and the live entries (committed-but-unfolded plus pending
+    drafts) are the explicit model's, each in its own ring slot."""
+    assert rm.seq_pos.tolist() == lm.seq
+    assert rm.ckpt_pos.tolist() == lm.ckpt
+    assert rm.flush_count.tolist() == lm.flushes
+    assert all(0 <= L <= W for L in rm.length.tolist())
+    for b in range(len(lm.seq)):
+        live = lm.buf[b] + lm.drafts[b]
+        assert rm.live_entries(b) == live
+        assert len({n % rm.R for n in live}) == len(live)  # no live entry shares a slot
+
+
+def _check_call(rm, before, appended):
+    """Within one call, the entries a fold reads (the committed entries before
+    the call) and the slots the call appends to never coincide, fold or not."""
+    for b in range(len(before)):
+        touched = before[b] + appended[b]
+        assert len({n % rm.R for n in touched}) == len(touched)
+
+
 @settings(max_examples=200, deadline=None)
 @given(W=st.integers(1, 12), K=st.integers(0, 8), seq=ops)
 def test_ring_model_equals_explicit_buffer(W, K, seq):
@@ -62,9 +86,11 @@ def test_ring_model_equals_explicit_buffer(W, K, seq):
     B = 3
     rm, lm = RingModel(B, W, K), ListModel(B, W, K)
     for op, k, acc in seq:
+        before = [list(x) for x in lm.buf]
         if op == "decode":
             rm.decode()
             lm.decode()
+            _check_call(rm, before, [[lm.seq[b] - 1] for b in range(B)])
         elif op == "flush":
             rm.flush()
             lm.flush()
@@ -74,17 +100,14 @@ def test_ring_model_equals_explicit_buffer(W, K, seq):
             kk = min(k, K)
             rm.verify(kk)
             lm.verify(kk)
+            _check_call(rm, before, lm.drafts)
+            assert rm.pending.tolist() == [kk] * B
+            _check(rm, lm, W)  # drafts pending, possibly after a fold in the same call
             bad = rm.commit(acc)
             lm.commit(acc)
             assert bad.tolist() == [not (0 <= a <= kk) for a in acc]
-        assert rm.seq_pos.tolist() == lm.seq
-        assert rm.ckpt_pos.tolist() == lm.ckpt
-        assert rm.flush_count.tolist() == lm.flushes
-        assert all(0 <= L <= W for L in rm.length.tolist())
-        for b in range(B):
-            live = lm.buf[b]
-            assert rm.live_entries(b) == live
-            assert len({n % rm.R for n in live}) == len(live)  # no live entry shares a slot
+            assert rm.pending.tolist() == [0] * B
+        _check(rm, lm, W)
 
 
 def test_misuse_is_refused():
