@@ -504,10 +504,10 @@ def main():
     shape = traffic.Shape("mamba2", wl.headdim, wl.dstate, wl.nheads // wl.ngroups, wl.window, "bf16",
                           wl.input_dtype)
     rep = traffic.replay_decode_per_token(shape)
-    win = traffic.fused_decode_window(shape)
+    win = traffic.replay_decode_window(shape)
     units = wl.batch * wl.nheads
-    bytes_per_launch = traffic.total(win["read"]) * units       # fused replay-read kernel, mean per call
-    fold_bytes = traffic.total(traffic.fused_step_split(shape, wl.window, True)["flush"]) * units  # per fold
+    bytes_per_launch = traffic.total(win["read"]) * units       # replay-read kernel, mean per call
+    prep_bytes = traffic.total(win["prep"]) * units             # prep/flush kernel, mean per call
     achieved = bytes_per_launch / (kern_ms * 1e-3) / 1e9
     peak, peak_kind = measured_peak()
     tr = None
@@ -554,16 +554,17 @@ def main():
         "hbm_gbs": achieved,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": tr, "peak_source": peak_kind,
-                     "kernel": "m2_read_fused_kernel<128, bf16, 1>",
+                     "kernel": "replay_read_kernel<128, bf16, 1>",
                      "algorithmic_bytes_per_launch": bytes_per_launch,
                      "kernel_ms_per_launch": kern_ms,
                      "read_ms_nonfold_call": float(np.mean(pick(read_ms, False))),
-                     "read_gbs_nonfold_call": traffic.total(traffic.fused_step_split(shape, wl.window // 2, False)["read"])
+                     "read_gbs_nonfold_call": traffic.total(traffic.replay_step_split(shape, wl.window // 2, False)["read"])
                                               * units / (np.mean(pick(read_ms, False)) * 1e-3) / 1e9},
-        "flush_kernel": {"kernel": "m2_fold_kernel<128, bf16, 1>",
-                         "ms_per_fold_call": float(np.mean(pick(prep_ms, True))) if any(fold) else None,
-                         "algorithmic_bytes_per_launch": fold_bytes,
-                         "gbs": (fold_bytes / (float(np.mean(pick(prep_ms, True))) * 1e-3) / 1e9) if any(fold) else None},
+        "prep_kernel": {"kernel": "m2_prep_kernel<128, bf16, 1>", "ms_per_launch": prep_avg,
+                        "algorithmic_bytes_per_launch": prep_bytes,
+                        "gbs": prep_bytes / (prep_avg * 1e-3) / 1e9,
+                        "ms_nonfold_call": float(np.mean(pick(prep_ms, False))),
+                        "ms_fold_call": float(np.mean(pick(prep_ms, True))) if any(fold) else None},
         "ms_per_call": {"nonfold": float(np.mean(pick(per, False))),
                         "fold": float(np.mean(pick(per, True))) if any(fold) else None},
         "e2e": {"value": job_tokens_per_s(world, wl.batch, K, e2e_ms), "unit": "tokens/s",

@@ -58,23 +58,16 @@ __host__ __device__ inline size_t gdn_raw_floats(int P, int N, int W, int ib, in
     const int Rm = W + 8;
     return (size_t)gpad4(Rm * N * ib / 4) + gpad4(Rm * P * ib / 4) + gpad4(kda ? Rm * N : Rm) + gpad4(Rm);
 }
-// The chunked fold's per-head tables: log-gate prefix sums ([W][N], GDN [W]), the
-// unit lower-triangular system (M, then its inverse in place) [W][W], the keys
-// decayed to the end of the buffer [W][N], and the final decay [N].
-__host__ __device__ inline size_t gdn_chunk_floats(int N, int W, int kda) {
-    return (size_t)gpad4(kda ? W * N : W) + gpad4(W * W) + gpad4(W * N) + gpad4(N);
-}
 __host__ __device__ inline size_t gdn_smem_floats(int P, int N, int W, int TQ, int kda, int ib) {
     const int E = W + TQ;
     return (size_t)gpad4(E * N) + gpad4(E * P) + gpad4(kda ? E * N : E) + 2 * (size_t)gpad4(E) + gpad4(TQ * N) +
            gpad4(E * E) + 2 * (size_t)gpad4(TQ * E) + gpad4(TQ * N) + gpad4(TQ * P) + gpad4(TQ) + 8 +
-           gdn_chunk_floats(N, W, kda) + gdn_raw_floats(P, N, W, ib, kda);
+           gdn_raw_floats(P, N, W, ib, kda);
 }
 
 struct GSmem {
     float *sk, *sv, *sal, *sbe, *spr, *sq, *sG, *shq, *sc, *sr, *sdot, *srq;
     int *si;
-    float *cl, *T, *kh, *dfin;  // chunked fold: log-gate prefix sums, system, decayed keys, final decay
     uint8_t *rk, *rv;  // raw k, v rings [R][N], [R][P] (input dtype)
     float *ra, *rb;    // raw gate ring ([Rs], KDA [R][N]) and beta ring [Rs]
 };
@@ -95,11 +88,7 @@ __device__ __forceinline__ GSmem gdn_carve(float *sm, int P, int N, int W, int T
     s.sdot = s.sr + gpad4(TQ * N);        // [TQ][P] S^ r per row
     s.srq = s.sdot + gpad4(TQ * P);       // [TQ]    unused pad
     s.si = reinterpret_cast<int *>(s.srq + gpad4(TQ));
-    s.cl = s.srq + gpad4(TQ) + 8;         // [W][N] (GDN [W])
-    s.T = s.cl + gpad4(kda ? W * N : W);  // [W][W]
-    s.kh = s.T + gpad4(W * W);            // [W][N]
-    s.dfin = s.kh + gpad4(W * N);         // [N]
-    float *raw = s.dfin + gpad4(N);
+    float *raw = s.srq + gpad4(TQ) + 8;
     const int Rm = W + 8;
     s.rk = reinterpret_cast<uint8_t *>(raw);
     s.rv = s.rk + 4 * gpad4(Rm * N * ib / 4);
@@ -212,204 +201,6 @@ __device__ __forceinline__ void gdn_fold_rows(float (&st)[NR][FoldMap<N>::NPT], 
 #pragma unroll
             for (int j = 0; j < NPT; ++j) st[r][j] = fmaf(al, st[r][j], coef * kk[j]);
         }
-    }
-}
-
-// ---------------------------------------------------------------------------
-// Chunked fold (the WY / UT form of the delta rule).  Per row s of the state the
-// entries i = 0..L-1 apply s_i = g_i (.) s_{i-1} + w_i k_i with
-// w_i = beta_i (v_i[row] - (g_i (.) s_{i-1}) . k_i), g_i the gate (GDN: one per
-// entry; KDA: one per key channel).  With C_i = log g_0 + ... + log g_i and
-// D_ij = exp(C_i - C_j) (the gates of entries j+1..i, always <= 1):
-//   (I + M) w = b,   M_ij = beta_i ((D_ij (.) k_j) . k_i) for j < i,
-//   b_i = beta_i (v_i[row] - s_0 . (exp(C_i) (.) k_i)),
-//   s_L = exp(C_{L-1}) (.) s_0 + sum_j w_j (D_{L-1,j} (.) k_j).
-// The system is the same for every row of the head, so (I + M)^{-1} is formed
-// once, and each row takes L independent dots, a small matrix-vector product and
-// a rank-L update: no per-token reduction chain.  Logs of the gates are clamped at
-// -80 so that a gate of exactly 0 (a full reset) gives no NaN.
-// ---------------------------------------------------------------------------
-
-// Per-head tables, every thread of the CTA; ends with a barrier.  Turns the
-// committed keys (physical entries base .. base + L0 - 1 of s.sk) into the gated
-// keys exp(C_i) (.) k_i in place.
-template <int N>
-__device__ __forceinline__ void gdn_chunk_tables(const GSmem &s, int kda, int base, int L0, int W) {
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    // 1. prefix sums of the log gates, and the final decay
-    if (kda) {
-        for (int n = tid; n < N; n += kThreads) {
-            float acc = 0.f;
-            for (int i = 0; i < L0; ++i) {
-                acc += fmaxf(logf(s.sal[(base + i) * N + n]), -80.f);
-                s.cl[i * N + n] = acc;
-            }
-            s.dfin[n] = expf(acc);
-        }
-    } else if (tid == 0) {
-        float acc = 0.f;
-        for (int i = 0; i < L0; ++i) {
-            acc += fmaxf(logf(s.sal[base + i]), -80.f);
-            s.cl[i] = acc;
-        }
-    }
-    __syncthreads();
-    if (!kda)
-        for (int n = tid; n < N; n += kThreads) s.dfin[n] = expf(s.cl[L0 - 1]);
-    auto clv = [&](int i, int n) -> float { return kda ? s.cl[i * N + n] : s.cl[i]; };
-    // 2. M (strictly lower part of s.T, row stride W): one warp per pair (i > j)
-    const int npair = L0 * (L0 - 1) / 2;
-    for (int pr = warp; pr < npair; pr += kWarps) {
-        int i = (int)((1.f + sqrtf(1.f + 8.f * (float)pr)) * 0.5f);  // pr -> (j < i)
-        while (i * (i - 1) / 2 > pr) --i;
-        while ((i + 1) * i / 2 <= pr) ++i;
-        const int j = pr - i * (i - 1) / 2;
-        const float *ki = s.sk + (base + i) * N, *kj = s.sk + (base + j) * N;
-        float d = 0.f;
-        if (kda) {
-            for (int n = lane; n < N; n += 32) d = fmaf(expf(clv(i, n) - clv(j, n)) * kj[n], ki[n], d);
-            d = group_sum<32>(d);
-        } else {
-            for (int n = lane; n < N; n += 32) d = fmaf(kj[n], ki[n], d);
-            d = group_sum<32>(d) * expf(s.cl[i] - s.cl[j]);
-        }
-        if (lane == 0) s.T[i * W + j] = s.sbe[base + i] * d;
-    }
-    //    keys decayed to the end of the buffer
-    for (int x = tid; x < L0 * N; x += kThreads) {
-        const int j = x / N, n = x - j * N;
-        s.kh[j * N + n] = expf(clv(L0 - 1, n) - clv(j, n)) * s.sk[(base + j) * N + n];
-    }
-    __syncthreads();
-    // 3. (I + M)^{-1} in place (warp 0, rows in order, lanes over columns); the
-    //    other warps gate the committed keys in place.
-    if (warp == 0) {
-        for (int i = 0; i < L0; ++i) {
-            float t0 = 0.f, t1 = 0.f;  // columns lane, lane + 32
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const int c = lane + 32 * h;
-                float t = (c == i) ? 1.f : 0.f;
-                if (c < i)
-                    for (int j = c; j < i; ++j) t = fmaf(-s.T[i * W + j], j == c ? 1.f : s.T[j * W + c], t);
-                if (h == 0) t0 = t; else t1 = t;
-            }
-            __syncwarp();
-            if (lane <= i) s.T[i * W + lane] = t0;
-            if (lane + 32 <= i) s.T[i * W + lane + 32] = t1;
-            __syncwarp();
-        }
-    } else {
-        for (int x = tid - 32; x < L0 * N; x += kThreads - 32) {
-            const int i = x / N, n = x - i * N;
-            s.sk[(base + i) * N + n] *= expf(clv(i, n));
-        }
-    }
-    __syncthreads();
-}
-
-// One row per call group: NR rows held as NPT-element segments by TPRF lanes each;
-// every lane of the warp must call this.  Uses the tables of gdn_chunk_tables.
-template <int N, int NR>
-__device__ __forceinline__ void gdn_fold_rows_chunked(float (&st)[NR][FoldMap<N>::NPT], const int (&rows)[NR],
-                                                      int P, const GSmem &s, int base, int L0, int W, int cseg) {
-    constexpr int NPT = FoldMap<N>::NPT, TPRF = FoldMap<N>::TPRF;
-    constexpr int MAXCH = (64 + TPRF - 1) / TPRF;  // entries come in chunks of TPRF, L0 <= 64
-    const int lane = threadIdx.x & 31, gbase = lane & ~(TPRF - 1);
-    const int nch = (L0 + TPRF - 1) / TPRF;
-#pragma unroll
-    for (int r = 0; r < NR; ++r) {
-        const int row = rows[r] < P ? rows[r] : 0;
-        float b[MAXCH], w[MAXCH];
-#pragma unroll
-        for (int c = 0; c < MAXCH; ++c) {
-            b[c] = 0.f;
-            w[c] = 0.f;
-            if (c < nch) {  // warp-uniform
-                float vals[TPRF];
-#pragma unroll
-                for (int kk = 0; kk < TPRF; ++kk) {
-                    const int i = c * TPRF + kk;
-                    float d = 0.f;
-                    if (i < L0) {
-                        const float *kt = s.sk + (base + i) * N + cseg * NPT;
-#pragma unroll
-                        for (int j = 0; j < NPT; j += 4) {
-                            const float4 k4 = *reinterpret_cast<const float4 *>(kt + j);
-                            d = fmaf(st[r][j], k4.x, d);
-                            d = fmaf(st[r][j + 1], k4.y, d);
-                            d = fmaf(st[r][j + 2], k4.z, d);
-                            d = fmaf(st[r][j + 3], k4.w, d);
-                        }
-                    }
-                    vals[kk] = d;
-                }
-                // reduce-scatter over the TPRF lanes of the row: lane cseg keeps entry c*TPRF + cseg
-#pragma unroll
-                for (int o = TPRF / 2; o > 0; o >>= 1) {
-                    const bool hi = (cseg & o) != 0;
-#pragma unroll
-                    for (int kk = 0; kk < o; ++kk) {
-                        const float send = hi ? vals[kk] : vals[kk + o];
-                        const float keep = hi ? vals[kk + o] : vals[kk];
-                        vals[kk] = keep + __shfl_xor_sync(0xffffffffu, send, o);
-                    }
-                }
-                const int i = c * TPRF + cseg;
-                if (i < L0) b[c] = s.sbe[base + i] * (s.sv[(base + i) * P + row] - vals[0]);
-            }
-        }
-        // w = (I + M)^{-1} b: lane cseg forms w of its entries
-#pragma unroll
-        for (int c2 = 0; c2 < MAXCH; ++c2) {
-            if (c2 < nch) {
-#pragma unroll
-                for (int jj = 0; jj < TPRF; ++jj) {
-                    const int j = c2 * TPRF + jj;
-                    const float bj = __shfl_sync(0xffffffffu, b[c2], gbase + jj);
-                    if (j < L0) {
-#pragma unroll
-                        for (int c = 0; c < MAXCH; ++c) {
-                            const int i = c * TPRF + cseg;
-                            if (c < nch && i < L0 && j <= i) w[c] = fmaf(s.T[i * W + j], bj, w[c]);
-                        }
-                    }
-                }
-            }
-        }
-        // s_L = final decay (.) s_0 + sum_j w_j (decayed k_j)
-        float o[NPT];
-#pragma unroll
-        for (int j = 0; j < NPT; j += 4) {
-            const float4 d4 = *reinterpret_cast<const float4 *>(s.dfin + cseg * NPT + j);
-            o[j] = d4.x * st[r][j];
-            o[j + 1] = d4.y * st[r][j + 1];
-            o[j + 2] = d4.z * st[r][j + 2];
-            o[j + 3] = d4.w * st[r][j + 3];
-        }
-#pragma unroll
-        for (int c2 = 0; c2 < MAXCH; ++c2) {
-            if (c2 < nch) {
-#pragma unroll
-                for (int jj = 0; jj < TPRF; ++jj) {
-                    const int j = c2 * TPRF + jj;
-                    const float wj = __shfl_sync(0xffffffffu, w[c2], gbase + jj);
-                    if (j < L0) {
-                        const float *kh = s.kh + j * N + cseg * NPT;
-#pragma unroll
-                        for (int e = 0; e < NPT; e += 4) {
-                            const float4 k4 = *reinterpret_cast<const float4 *>(kh + e);
-                            o[e] = fmaf(wj, k4.x, o[e]);
-                            o[e + 1] = fmaf(wj, k4.y, o[e + 1]);
-                            o[e + 2] = fmaf(wj, k4.z, o[e + 2]);
-                            o[e + 3] = fmaf(wj, k4.w, o[e + 3]);
-                        }
-                    }
-                }
-            }
-        }
-#pragma unroll
-        for (int j = 0; j < NPT; ++j) st[r][j] = o[j];
     }
 }
 
@@ -618,15 +409,13 @@ __global__ void __launch_bounds__(kThreads, TQ == 1 ? 3 : 1) gdn_replay_kernel(c
     }
 
     if (flush) {
-        // 7a. Fold the committed entries into the fp32 checkpoint rows (chunked form).
-        if (L0 > 0) gdn_chunk_tables<N>(s, a.kda, base, L0, W);
-        constexpr int RBFC = 1;  // rows per thread at a time: the chunked row pass holds more per row
+        // 7a. Fold the committed entries into the fp32 checkpoint rows.
         const int cseg = tid % TPRF, q0 = tid / TPRF;
-        for (int rb = 0; rb < P; rb += RBFC * RPPF) {
-            float st[RBFC][NPT];
-            int rows[RBFC];
+        for (int rb = 0; rb < P; rb += RBF * RPPF) {
+            float st[RBF][NPT];
+            int rows[RBF];
 #pragma unroll
-            for (int k = 0; k < RBFC; ++k) {
+            for (int k = 0; k < RBF; ++k) {
                 rows[k] = rb + q0 + k * RPPF;
 #pragma unroll
                 for (int j = 0; j < NPT; j += 4) {
@@ -635,9 +424,9 @@ __global__ void __launch_bounds__(kThreads, TQ == 1 ? 3 : 1) gdn_replay_kernel(c
                     st[k][j] = v4.x; st[k][j + 1] = v4.y; st[k][j + 2] = v4.z; st[k][j + 3] = v4.w;
                 }
             }
-            if (L0 > 0) gdn_fold_rows_chunked<N, RBFC>(st, rows, P, s, base, L0, W, cseg);
+            gdn_fold_rows<N, RBF>(st, rows, P, s, base, L0, cseg, a.kda);
 #pragma unroll
-            for (int k = 0; k < RBFC; ++k) {
+            for (int k = 0; k < RBF; ++k) {
                 const bool valid = rows[k] < P;
                 const int64_t el = tile0 + (int64_t)(valid ? rows[k] : 0) * N + cseg * NPT;
                 if (a.op == OP_EXPORT) {

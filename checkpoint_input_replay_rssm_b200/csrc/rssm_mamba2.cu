@@ -5,13 +5,9 @@
 namespace rssm {
 
 extern template cudaError_t m2_dispatch_n<16>(int, int, int, const M2Args &, const M2FoldLay &, size_t, int, cudaStream_t);
-extern template cudaError_t m2_readf_dispatch_n<16>(int, int, const M2Args &, const M2ReadLay &, cudaStream_t);
 extern template cudaError_t m2_dispatch_n<32>(int, int, int, const M2Args &, const M2FoldLay &, size_t, int, cudaStream_t);
-extern template cudaError_t m2_readf_dispatch_n<32>(int, int, const M2Args &, const M2ReadLay &, cudaStream_t);
 extern template cudaError_t m2_dispatch_n<64>(int, int, int, const M2Args &, const M2FoldLay &, size_t, int, cudaStream_t);
-extern template cudaError_t m2_readf_dispatch_n<64>(int, int, const M2Args &, const M2ReadLay &, cudaStream_t);
 extern template cudaError_t m2_dispatch_n<128>(int, int, int, const M2Args &, const M2FoldLay &, size_t, int, cudaStream_t);
-extern template cudaError_t m2_readf_dispatch_n<128>(int, int, const M2Args &, const M2ReadLay &, cudaStream_t);
 
 static int tq_of(int T) { return T <= 1 ? 1 : (T <= 4 ? 4 : 8); }
 static int in_bytes(const rssm_config &cf) { return cf.input_dtype == RSSM_BF16 ? 2 : 4; }
@@ -48,18 +44,7 @@ size_t mamba2_smem_bytes(const rssm_config &cf, int T) {
         return sizeof(float) * ((size_t)2 * pad4(TQ * P) + 2 * pad4(TQ * N) + 2 * pad4(TQ));
     const size_t prep = m2_prep_lay(m2_prep_heads(cf, TQ), P, N, cf.window, TQ, in_bytes(cf)).bytes;
     const size_t fold = m2_fold_lay(m2_fold_heads(cf, TQ), P, N, cf.window, ring_slots(cf), TQ, in_bytes(cf)).bytes;
-    const size_t readf = m2_read_lay(read_heads_per_cta(cf), P, N, cf.window, ring_slots(cf), TQ, in_bytes(cf)).bytes;
-    size_t m = prep > fold ? prep : fold;
-    return m > readf ? m : readf;
-}
-
-static cudaError_t dispatch_readf(int N, int rk, int TQ, const M2Args &a, const M2ReadLay &lay, cudaStream_t st) {
-    switch (N) {
-        case 16: return m2_readf_dispatch_n<16>(rk, TQ, a, lay, st);
-        case 32: return m2_readf_dispatch_n<32>(rk, TQ, a, lay, st);
-        case 64: return m2_readf_dispatch_n<64>(rk, TQ, a, lay, st);
-        default: return m2_readf_dispatch_n<128>(rk, TQ, a, lay, st);
-    }
+    return prep > fold ? prep : fold;
 }
 
 static cudaError_t dispatch(int which, int N, int rk, int TQ, const M2Args &a, const M2FoldLay &lay, size_t smem,
@@ -127,28 +112,29 @@ cudaError_t mamba2_launch(Ctx &h, int op, int T, const rssm_inputs *in, float *y
         if (e == cudaSuccess && op == OP_FLUSH) h.len_lb = h.len_ub = 0;
         return e;
     }
-    // Decode/verify: the flush kernel when some buffer may be too full for the
-    // call's tokens (it visits every sequence and folds those; when every buffer
-    // is, its checkpoint stages stream across work items), then the fused
-    // replay-read kernel, which forms the coefficients, appends and publishes.
-    (void)ho;
     const bool fold = h.len_ub + T > cf.window;
-    cudaError_t e = cudaSuccess;
-    if (fold) {
-        f.scan_all = 1;
-        f.all_fold = h.len_lb + T > cf.window;
+    a.fold_launched = fold;
+    a.HC = m2_prep_heads(cf, TQ);
+    a.cpg = (cf.nheads / cf.ngroups) / a.HC;
+    a.lay = m2_prep_lay(a.HC, cf.headdim, N, cf.window, TQ, ib);
+    h.launches += 1;
+    cudaError_t e = dispatch(M2_PREP, N, rk, TQ, a, flay, (size_t)a.lay.bytes, h.num_sms, st);
+    if (e == cudaSuccess && fold) {
         h.launches += 1;
         e = dispatch(M2_FOLD, N, rk, TQ, f, flay, 0, h.num_sms, st);
     }
     if (e == cudaSuccess && h.split_event) e = cudaEventRecord(h.split_event, st);
     if (e == cudaSuccess) {
-        a.fold_launched = fold;
-        a.HC = read_heads_per_cta(cf);
-        const M2ReadLay rlay = m2_read_lay(a.HC, cf.headdim, N, cf.window, (int)h.lay.ring, TQ, ib);
+        // replay read: C of the group ([B][T][G][N]) is the query, x the buffered entries
+        const int G = cf.ngroups;
         h.launches += 1;
-        e = dispatch_readf(N, rk, TQ, a, rlay, st);
+        e = launch_read(h, op, T, in->Cm, ib == 2, cf.nheads / G, (int64_t)T * G * N, N, (int64_t)G * N, in->x,
+                        (const float *)h.at(h.lay.D_off), y, ho, st, !fold, !h.split_event);
     }
-    if (e != cudaSuccess) return e;
+    if (e != cudaSuccess) {  // leave no stale work list behind
+        cudaMemsetAsync(ho.fold_count, 0, sizeof(int), st);
+        return e;
+    }
     update_len_bounds(h, op, T);
     return cudaSuccess;
 }

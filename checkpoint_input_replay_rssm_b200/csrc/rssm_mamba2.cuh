@@ -63,9 +63,6 @@ struct M2Args {
     int *fold_count;    // sequences the flush kernel folds in this call (reset by the read kernel)
     int *fold_list;     // [B] their indices
     int fold_launched;  // the host launches the flush kernel in this call
-    int scan_all;       // flush kernel in decode/verify without a work list: it visits every
-                        // sequence and folds those whose buffer is too full for the call
-    int all_fold;       // ... and every sequence's buffer is (so the stages may stream across items)
     float *dec;         // [B][H][TQmax] decay of S^ C
     float *coef;        // [B][H][TQmax][Emax] replay coefficients
     int TQmax, Emax;    // Emax: padded row length of the coefficient table
@@ -370,8 +367,7 @@ __global__ void __launch_bounds__(kThreads, 3) m2_fold_kernel(const M2Args a, co
     const int nrows = HC * P;
     const int nst = (nrows + FC - 1) / FC;
     const bool reads = (a.op == OP_DECODE || a.op == OP_VERIFY);
-    const bool listed = reads && !a.scan_all;  // decode/verify with the prep kernel's work list
-    const bool stream = reads && (listed || a.all_fold);  // every visited sequence folds
+    const bool stream = reads;  // every listed sequence folds: stages run on across items
     const int xrow = P * IB, brow = N * IB, xch = xrow / 16, bch = brow / 16;
     const int Rs = a.Rs;
     const int chunks = G * a.cpg;  // CTA work items per sequence
@@ -396,8 +392,8 @@ __global__ void __launch_bounds__(kThreads, 3) m2_fold_kernel(const M2Args a, co
 
     // Work items (sequence, chunk of HC heads of one group): decode/verify fold
     // the sequences the prep kernel listed; flush/export visit every sequence.
-    const int nitems = (listed ? min(*a.fold_count, a.B) : a.B) * chunks;
-    auto item_seq = [&](int it) { return listed ? a.fold_list[it / chunks] : it / chunks; };
+    const int nitems = (reads ? min(*a.fold_count, a.B) : a.B) * chunks;
+    auto item_seq = [&](int it) { return reads ? a.fold_list[it / chunks] : it / chunks; };
     auto item_h0 = [&](int it) {
         const int chunk = it % chunks, g = chunk / a.cpg;
         return g * hpg + (chunk - g * a.cpg) * HC;
@@ -720,313 +716,6 @@ __global__ void __launch_bounds__(kThreads, 3) m2_fold_kernel(const M2Args a, co
 }
 
 // ---------------------------------------------------------------------------
-// Fused replay-read kernel (Mamba-2): decode (T = 1) and verify (T = K) in one
-// kernel when no flush kernel is needed, and after the flush kernel otherwise.
-//
-// One CTA per (sequence b, HC heads of one group g).  Every thread first issues
-// its first round of read-copy chunks (they depend on nothing); while they are in
-// flight the CTA reads the sequence's counters and stages the group's B ring, the
-// heads' dt ring rows, A, D and the call's tokens, then computes what the prep
-// kernel used to hand over -- B_e . C_m for the group and, per head (one warp),
-// the prefix sums Lam of dt*A, the replay coefficients
-//     coef[m][e] = e^{Lam_{L0+m} - Lam_e} (B_e . C_m) s_e,   dec[m] = e^{Lam_{L0+m}}
-// -- appends the call's tokens to the ring, and streams the rest of its copy:
-//   y = dec (S^ C_m) + sum_{e <= L0+m} coef[m][e] x_e + D x_{L0+m}.
-// A sequence folded by the flush kernel in this call only appends (the flush
-// kernel served its outputs).  The new counters are published by the last CTA of
-// the sequence to arrive (every CTA has read them by then).
-// ---------------------------------------------------------------------------
-struct M2ReadLay {
-    int q, craw, bring, bnew, x, dring, dtn, sa, sd, dd, coef, dec, dot, scale, info, bytes;
-};
-inline M2ReadLay m2_read_lay(int HC, int P, int N, int W, int R, int TQ, int ib) {
-    const int E = W + TQ, Ep = (E + 3) & ~3;
-    M2ReadLay L{};
-    int o = 0;
-    L.q = o;     o += a16(TQ * N * 4);          // C as fp32                 [TQ][N]
-    L.craw = o;  o += a16(TQ * N * ib);         // raw C of the call          [TQ][N]
-    L.bring = o; o += a16(R * N * ib);          // raw B ring of the group    [R][N]
-    L.bnew = o;  o += a16(TQ * N * ib);         // raw B of the call          [TQ][N]
-    L.x = o;     o += a16(HC * E * P * ib);     // raw x entries              [HC][E][P]
-    L.dring = o; o += a16(HC * pad4(R) * 4);    // dt ring rows               [HC][Rs]
-    L.dtn = o;   o += a16(TQ * HC * 4);         // dt of the call's tokens    [TQ][HC]
-    L.sa = o;    o += a16(HC * 4);              // A of the heads             [HC]
-    L.dd = o;    o += a16(HC * 4);              // D of the heads             [HC]
-    L.sd = o;    o += a16(TQ * Ep * 4);         // B_e . C_m                  [TQ][Ep]
-    L.coef = o;  o += a16(HC * TQ * Ep * 4);    // coefficients               [HC][TQ][Ep]
-    L.dec = o;   o += a16(HC * TQ * 4);         // decays                     [HC][TQ]
-    L.dot = o;   o += a16(HC * P * TQ * 4);     // S^ . C per row             [HC*P][TQ]
-    L.scale = o; o += a16(HC * P * 4);          // fp8 row scales             [HC*P]
-    L.info = o;  o += 32;
-    L.bytes = o;
-    return L;
-}
-
-template <int N, int RK, int TQ, bool BF>
-__global__ void __launch_bounds__(kThreads, TQ == 1 ? 4 : 2) m2_read_fused_kernel(const M2Args a, const M2ReadLay Ly) {
-    constexpr int EPC = Chunk<RK>::EPC;   // stored elements per 16-byte chunk
-    constexpr int TPR = N / EPC;          // chunks per state row
-    constexpr int RCB = Chunk<RK>::BYTES;
-    constexpr int LPR = TPR < 4 ? TPR : 4;  // lanes per row
-    constexpr int CPL = TPR / LPR;          // chunks per lane per row
-    constexpr int RPP = kThreads / LPR;     // rows per pass
-    constexpr int MAXC = 8;                 // chunks in flight per thread
-    constexpr int PPR = MAXC / CPL > 0 ? MAXC / CPL : 1;  // passes per round
-    constexpr int IB = BF ? 2 : 4;
-    constexpr int kLamChunks = 3;           // L0 + T <= W + 8 <= 72 entries
-    static_assert(CPL <= MAXC, "a lane's chunks of one row must fit a round");
-
-    extern __shared__ __align__(128) uint8_t smraw[];
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int H = a.H, P = a.P, R = a.R, W = a.W, T = a.T, HC = a.HC, G = a.G;
-    const int hpg = H / G;
-    const int b = blockIdx.y;
-    const int h0 = blockIdx.x * HC;
-    const int g = h0 / hpg;
-    const bool first_of_group = (h0 % hpg) == 0;
-    const int E = W + TQ, Ep = (E + 3) & ~3;
-    float *sq = reinterpret_cast<float *>(smraw + Ly.q);
-    uint8_t *sC = smraw + Ly.craw, *sBr = smraw + Ly.bring, *sBn = smraw + Ly.bnew, *sx = smraw + Ly.x;
-    float *dring = reinterpret_cast<float *>(smraw + Ly.dring);
-    float *dtn = reinterpret_cast<float *>(smraw + Ly.dtn);
-    float *sA = reinterpret_cast<float *>(smraw + Ly.sa);
-    float *sD = reinterpret_cast<float *>(smraw + Ly.dd);
-    float *sd = reinterpret_cast<float *>(smraw + Ly.sd);
-    float *scoef = reinterpret_cast<float *>(smraw + Ly.coef);
-    float *sdec = reinterpret_cast<float *>(smraw + Ly.dec);
-    float *sdot = reinterpret_cast<float *>(smraw + Ly.dot);
-    float *ssc = reinterpret_cast<float *>(smraw + Ly.scale);
-    int *sinfo = reinterpret_cast<int *>(smraw + Ly.info);
-    const int64_t row0 = (int64_t)b * H + h0;
-    const int nrows = HC * P;
-    const uint8_t *tile = reinterpret_cast<const uint8_t *>(a.rc) + row0 * P * N * RCB;
-    const int q = tid % LPR, rrow = tid / LPR;
-    const int xrow = P * IB, xch = xrow / 16, brow = N * IB, bch = brow / 16;
-    const int Rs = a.Rs;
-    auto ldx = [](const uint8_t *p) -> float {
-        return BF ? bf16_bits_to_float(*reinterpret_cast<const uint16_t *>(p)) : *reinterpret_cast<const float *>(p);
-    };
-
-    // 0. After a flush kernel, learn first whether this sequence was folded
-    //    (then it needs no read copy); the counters are not yet rewritten.
-    bool skip_copy = false;
-    if (a.fold_launched) {
-        if (tid == 0) {
-            const SeqState s0 = read_counters(a.c, b, W);
-            sinfo[5] = s0.ok && (int)(s0.seq - s0.ckpt) + T > W;
-        }
-        __syncthreads();
-        skip_copy = sinfo[5] != 0;
-    }
-
-    // 1. First round of read-copy chunks.
-    uint4 rv[MAXC];
-    auto issue = [&](int pass0) {
-#pragma unroll
-        for (int j = 0; j < PPR; ++j) {
-            const int r = (pass0 + j) * RPP + rrow;
-#pragma unroll
-            for (int k = 0; k < CPL; ++k)
-                if (r < nrows) rv[j * CPL + k] = ld_stream(tile + ((size_t)r * TPR + q + LPR * k) * 16);
-        }
-    };
-    if (!skip_copy) issue(0);
-
-    // 2. Counters (thread 0; this CTA's arrival is registered once they are read)
-    //    and everything that does not depend on them.
-    if (tid == 0) {
-        const SeqState ss = read_counters(a.c, b, W);
-        const int L0 = (int)(ss.seq - ss.ckpt);
-        const int fold = ss.ok && (L0 + T > W);
-        const int valid = ss.ok && !(fold && !a.fold_launched);
-        if (blockIdx.x == 0 && !valid) report(a.c.err, DEV_BAD_COUNTERS, b, 0, L0);
-        sinfo[0] = valid;
-        sinfo[1] = ss.ok ? L0 : 0;
-        sinfo[2] = fold;
-        sinfo[3] = (int)(ss.ckpt % R);
-        sinfo[4] = (int)(ss.seq % R);
-        // new counters, published by the last CTA of the sequence to arrive
-        if (valid)
-            arrive_and_publish(a.c, b, H / HC, a.op == OP_DECODE ? ss.seq + 1 : -1, fold ? ss.seq : -1,
-                               a.op == OP_VERIFY ? T : -1, fold);
-        else
-            arrive_and_publish(a.c, b, H / HC, -1, -1, -1, 0);
-    }
-    {
-        const uint8_t *src = reinterpret_cast<const uint8_t *>(a.Bbuf) + ((int64_t)(b * G + g) * R) * brow;
-        for (int i = tid; i < R * bch; i += kThreads) cp_async16(sBr + i * 16, src + i * 16);
-    }
-    for (int i = tid; i < HC * Rs / 4; i += kThreads) cp_async16(dring + 4 * i, a.dtbuf + row0 * Rs + 4 * i);
-    for (int row = warp; row < T; row += kWarps) {
-        const int64_t o = (((int64_t)(b * T + row) * G + g) * N) * IB;
-        for (int k = lane; k < bch; k += 32) {
-            cp_async16(sC + row * brow + k * 16, reinterpret_cast<const uint8_t *>(a.Cm) + o + k * 16);
-            cp_async16(sBn + row * brow + k * 16, reinterpret_cast<const uint8_t *>(a.Bm) + o + k * 16);
-        }
-    }
-    for (int row = warp; row < T * HC; row += kWarps) {  // x of token m, head hh -> entry W + m
-        const int m = row / HC, hh = row - m * HC;
-        const uint8_t *src = reinterpret_cast<const uint8_t *>(a.x) + (((int64_t)(b * T + m) * H + h0 + hh) * P) * IB;
-        for (int k = lane; k < xch; k += 32) cp_async16(sx + (hh * E + W + m) * xrow + k * 16, src + k * 16);
-    }
-    for (int i = tid; i < T * HC; i += kThreads) {
-        const int m = i / HC, hh = i - m * HC;
-        cp_async4(dtn + i, a.dt + (int64_t)(b * T + m) * H + h0 + hh);
-    }
-    if (tid < HC) cp_async4(sA + tid, a.A + h0 + tid);
-    else if (tid >= 32 && tid < 32 + HC) cp_async4(sD + tid - 32, a.D + h0 + tid - 32);
-    if (RK == SK_FP8)
-        for (int i = tid; i < nrows / 4; i += kThreads) cp_async16(ssc + 4 * i, a.rc_scale + row0 * P + 4 * i);
-    cp_async_wait_all();
-    __syncthreads();
-    const int valid = sinfo[0], L0 = sinfo[1], fold = sinfo[2], ckmod = sinfo[3], spmod = sinfo[4];
-    if (!valid) return;  // counters corrupted: reported, sequence skipped
-    const int base = W - L0, nE = L0 + T;
-    auto slot_of = [&](int e) { const int sl = ckmod + e; return sl >= R ? sl - R : sl; };
-
-    // 3. Append the call's tokens (slots seq_pos + m mod R, never an entry read here).
-    for (int row = warp; row < T * HC; row += kWarps) {
-        const int m = row / HC, hh = row - m * HC;
-        const int sl = spmod + m >= R ? spmod + m - R : spmod + m;
-        uint8_t *dst = reinterpret_cast<uint8_t *>(a.xbuf) + (((row0 + hh) * R + sl) * P) * IB;
-        const uint8_t *src = sx + (hh * E + W + m) * xrow;
-        for (int k = lane; k < xch; k += 32)
-            *reinterpret_cast<uint4 *>(dst + k * 16) = *reinterpret_cast<const uint4 *>(src + k * 16);
-    }
-    for (int i = tid; i < T * HC; i += kThreads) {
-        const int m = i / HC, hh = i - m * HC;
-        const int sl = spmod + m >= R ? spmod + m - R : spmod + m;
-        a.dtbuf[(row0 + hh) * Rs + sl] = dtn[m * HC + hh];
-    }
-    if (first_of_group) {  // the group's first CTA writes the group's B
-        for (int row = warp; row < T; row += kWarps) {
-            const int sl = spmod + row >= R ? spmod + row - R : spmod + row;
-            uint8_t *dst = reinterpret_cast<uint8_t *>(a.Bbuf) + (((int64_t)(b * G + g) * R + sl) * N) * IB;
-            for (int k = lane; k < bch; k += 32)
-                *reinterpret_cast<uint4 *>(dst + k * 16) = *reinterpret_cast<const uint4 *>(sBn + row * brow + k * 16);
-        }
-    }
-    if (fold) return;  // outputs served by the flush kernel
-
-    // 4. The buffered x entries of the replay term (two contiguous runs of slots per
-    //    head), in flight while the coefficients are formed.
-    {
-        const int n1 = min(L0, R - ckmod);
-        for (int row = warp; row < 2 * HC; row += kWarps) {
-            const int hh = row >> 1, second = row & 1;
-            const int cnt = second ? L0 - n1 : n1;
-            const uint8_t *src = reinterpret_cast<const uint8_t *>(a.xbuf) +
-                                 (((row0 + hh) * R + (second ? 0 : ckmod)) * P) * IB;
-            uint8_t *dst = sx + (hh * E + base + (second ? n1 : 0)) * xrow;
-            for (int k = lane; k < cnt * xch; k += 32) cp_async16(dst + k * 16, src + k * 16);
-        }
-    }
-    // C as fp32; B_e . C_m once for the group (one warp per pair, lanes over N)
-    for (int i = tid; i < T * N; i += kThreads) sq[i] = ldx(sC + i * IB);
-    for (int pr = warp; pr < T * nE; pr += kWarps) {
-        const int m = pr / nE, e = pr - m * nE;
-        if (e > L0 + m) continue;  // warp-uniform
-        const uint8_t *Bp = e < L0 ? sBr + slot_of(e) * brow : sBn + (e - L0) * brow;
-        float d = 0.f;
-        for (int n = lane; n < N; n += 32) d = fmaf(ldx(Bp + n * IB), ldx(sC + (m * N + n) * IB), d);
-        d = group_sum<32>(d);
-        if (lane == 0) sd[m * Ep + e] = d;
-    }
-    __syncthreads();
-    // per head (one warp each): prefix sums of dt*A, decays, coefficients
-    for (int hh = warp; hh < HC; hh += kWarps) {
-        const float Ah = sA[hh];
-        auto dt_of = [&](int e) -> float { return e < L0 ? dring[hh * Rs + slot_of(e)] : dtn[(e - L0) * HC + hh]; };
-        float lamr[kLamChunks];
-        float carry = 0.f;
-#pragma unroll
-        for (int ch = 0; ch < kLamChunks; ++ch) {
-            lamr[ch] = 0.f;
-            if (ch * 32 < nE) {  // warp-uniform
-                const int e = ch * 32 + lane;
-                float v = e < nE ? dt_of(e) * Ah : 0.f;
-                v = warp_incl_scan(v) + carry;
-                lamr[ch] = v;
-                carry = __shfl_sync(0xffffffffu, v, 31);
-            }
-        }
-        auto lam_at = [&](int e) -> float {  // e warp-uniform
-            const float v = e < 32 ? lamr[0] : (e < 64 ? lamr[1] : lamr[2]);
-            return __shfl_sync(0xffffffffu, v, e & 31);
-        };
-#pragma unroll
-        for (int m = 0; m < TQ; ++m) {
-            if (m < T) {  // warp-uniform
-                const float lm = lam_at(L0 + m);
-                if (lane == 0) sdec[hh * TQ + m] = expf(lm);
-#pragma unroll
-                for (int ch = 0; ch < kLamChunks; ++ch) {
-                    const int e = ch * 32 + lane;
-                    if (e <= L0 + m)
-                        scoef[(hh * TQ + m) * Ep + e] =
-                            expf(lm - lamr[ch]) * sd[m * Ep + e] * (a.dt_scales ? dt_of(e) : 1.f);
-                }
-            }
-        }
-    }
-    cp_async_wait_all();
-    __syncthreads();
-
-    // 5. Rows dotted with the query (C of the group, shared by the CTA's heads).
-    for (int pass0 = 0; pass0 * RPP < nrows; pass0 += PPR) {
-        if (pass0 > 0) issue(pass0);
-#pragma unroll
-        for (int j = 0; j < PPR; ++j) {
-            const int r = (pass0 + j) * RPP + rrow;
-            const bool ok = r < nrows;
-            float acc[TQ];
-#pragma unroll
-            for (int m = 0; m < TQ; ++m) acc[m] = 0.f;
-#pragma unroll
-            for (int k = 0; k < CPL; ++k) {
-                float v[EPC];
-                if (ok) unpack<RK>(rv[j * CPL + k], v);
-                else {
-#pragma unroll
-                    for (int e = 0; e < EPC; ++e) v[e] = 0.f;
-                }
-                const int c0 = (q + LPR * k) * EPC;
-#pragma unroll
-                for (int m = 0; m < TQ; ++m) {
-                    const float4 *q4 = reinterpret_cast<const float4 *>(sq + m * N + c0);
-#pragma unroll
-                    for (int e4 = 0; e4 < EPC / 4; ++e4) {
-                        const float4 w = q4[e4];
-                        acc[m] = fmaf(v[4 * e4], w.x, acc[m]);
-                        acc[m] = fmaf(v[4 * e4 + 1], w.y, acc[m]);
-                        acc[m] = fmaf(v[4 * e4 + 2], w.z, acc[m]);
-                        acc[m] = fmaf(v[4 * e4 + 3], w.w, acc[m]);
-                    }
-                }
-            }
-#pragma unroll
-            for (int m = 0; m < TQ; ++m) {
-                const float d = group_sum<LPR>(acc[m]);
-                if (q == 0 && ok && m < T) sdot[r * TQ + m] = (RK == SK_FP8) ? d * ssc[r] : d;
-            }
-        }
-    }
-    __syncthreads();
-
-    // 6. y = dec * (S^ . C) + replay term + D x.
-    for (int i = tid; i < T * nrows; i += kThreads) {
-        const int m = i / nrows, r2 = i - m * nrows;
-        const int hh = r2 / P, p = r2 - hh * P;
-        float yv = sdec[hh * TQ + m] * sdot[r2 * TQ + m];
-        const float *cf = scoef + (hh * TQ + m) * Ep;
-        const uint8_t *xs = sx + (hh * E + base) * xrow + p * IB;
-        for (int e = 0; e <= L0 + m; ++e) yv = fmaf(cf[e], ldx(xs + e * xrow), yv);
-        yv = fmaf(sD[hh], ldx(sx + (hh * E + W + m) * xrow + p * IB), yv);
-        a.y[((int64_t)(b * T + m) * H + h0 + hh) * P + p] = yv;
-    }
-}
-
-// ---------------------------------------------------------------------------
 // Eager read-modify-write baseline: decode (T = 1, state rewritten) and verify
 // (T = K drafts applied in registers, K snapshots written, state untouched).
 // The per-token state rewrite is the baseline the ReplaySSM reports start from
@@ -1190,28 +879,6 @@ inline cudaError_t dispatch_rk(int which, int rk, const M2Args &a, const M2FoldL
             return which == M2_EAGER ? launch_eager_t<N, SK_FP8, TQ>(a, smem, st)
                                      : launch_fold_t<N, SK_FP8, TQ>(a, lay, num_sms, st);
     }
-}
-
-// The fused replay-read kernel of decode/verify.
-template <int N, int RK, int TQ>
-inline cudaError_t launch_readf_t(const M2Args &a, const M2ReadLay &lay, cudaStream_t st) {
-    auto k = a.in_bf16 ? m2_read_fused_kernel<N, RK, TQ, true> : m2_read_fused_kernel<N, RK, TQ, false>;
-    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, lay.bytes);
-    if (e != cudaSuccess) return e;
-    k<<<dim3(a.H / a.HC, a.B), kThreads, lay.bytes, st>>>(a, lay);
-    return cudaGetLastError();
-}
-template <int N, int TQ>
-inline cudaError_t readf_rk(int rk, const M2Args &a, const M2ReadLay &lay, cudaStream_t st) {
-    if (rk == SK_F32) return launch_readf_t<N, SK_F32, TQ>(a, lay, st);
-    if (rk == SK_BF16) return launch_readf_t<N, SK_BF16, TQ>(a, lay, st);
-    return launch_readf_t<N, SK_FP8, TQ>(a, lay, st);
-}
-template <int N>
-cudaError_t m2_readf_dispatch_n(int rk, int TQ, const M2Args &a, const M2ReadLay &lay, cudaStream_t st) {
-    if (TQ == 1) return readf_rk<N, 1>(rk, a, lay, st);
-    if (TQ == 4) return readf_rk<N, 4>(rk, a, lay, st);
-    return readf_rk<N, 8>(rk, a, lay, st);
 }
 
 // Per-dstate entry points; each instantiation lives in its own translation unit.

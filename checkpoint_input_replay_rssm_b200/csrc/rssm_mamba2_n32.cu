@@ -3,5 +3,4 @@
 
 namespace rssm {
 template cudaError_t m2_dispatch_n<32>(int, int, int, const M2Args &, const M2FoldLay &, size_t, int, cudaStream_t);
-template cudaError_t m2_readf_dispatch_n<32>(int, int, const M2Args &, const M2ReadLay &, cudaStream_t);
 }  // namespace rssm

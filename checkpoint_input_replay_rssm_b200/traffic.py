@@ -89,40 +89,6 @@ def replay_step_split(s: Shape, L0: int, fold: bool, T: int = 1) -> dict:
     return {"prep": prep, "read": read}
 
 
-def fused_step_split(s: Shape, L0: int, fold: bool, T: int = 1) -> dict:
-    """Mamba-2 with the fused read kernel: bytes per (b, h) of one call, by kernel.
-    The flush kernel (fold calls only) reads the buffer, the call's inputs and the
-    fp32 checkpoint and writes the checkpoint, the copy and y; the fused read kernel
-    reads the counters' worth of buffer (B and dt rings, x entries), the call's
-    inputs and the copy, appends, and writes y."""
-    x, k = _x_row(s), _key_row(s)
-    scal = _scalars(s)
-    q = k
-    read = {"inputs": T * (q + k + scal + x), "append": T * (x + k + scal),
-            "buffer_read": (s.window + 1) * (k + scal)}  # B and dt rings staged whole
-    flush = {}
-    if fold:
-        flush = {"buffer_read": L0 * (k + scal + x), "inputs": T * (q + k + scal + x),
-                 "ckpt_read": state_tile(s, "f32"), "ckpt_write": state_tile(s, "f32"),
-                 "copy_write": state_tile(s, s.read_dtype) if s.read_dtype != "f32" else 0.0,
-                 "output": T * s.headdim * 4}
-    else:
-        read["copy_read"] = state_tile(s, s.read_dtype)
-        read["buffer_read"] += L0 * x
-        read["output"] = T * s.headdim * 4
-    return {"flush": flush, "read": read}
-
-
-def fused_decode_window(s: Shape) -> dict:
-    W = s.window
-    steps = [fused_step_split(s, W, True)] + [fused_step_split(s, L0, False) for L0 in range(1, W)]
-    out = {}
-    for kern in ("flush", "read"):
-        keys = sorted({k for st in steps for k in st[kern]})
-        out[kern] = {k: sum(st[kern].get(k, 0.0) for st in steps) / W for k in keys}
-    return out
-
-
 def replay_decode_window(s: Shape) -> dict:
     """Per-kernel bytes per (b, h) per token, averaged over one window of plain decode."""
     W = s.window
