@@ -1,0 +1,366 @@
+// rssm_prefill.cu -- chunked Mamba-2 prefill on the 5th-generation tensor cores:
+// the outputs of a prompt and the fp32 state after it, the checkpoint a replay
+// decode starts from (rssm_import_state).
+//
+// The prompt is cut into chunks of Q = 128 tokens.  With Lam_i the prefix sums
+// of dt A_h over the chunk's tokens, s_j = dt_j (dt scales the input) or 1, and
+// S the state at the chunk's start (headdim P x dstate N):
+//   CB[i][j]  = C_i . B_j                                           (C B^T, group-shared)
+//   M[i][j]   = e^{Lam_i - Lam_j} CB[i][j] s_j  for j <= i, else 0
+//   y_i       = sum_j M[i][j] x_j + e^{Lam_i} (S C_i) + D x_i
+//   S        <- e^{Lam_last} S + sum_j e^{Lam_last - Lam_j} s_j x_j B_j^T
+// -- the checkpoint + buffered-inputs algebra of the replay read, with the chunk
+// as the buffer (blog.thibaultmonteiro.fr, "Tenir le journal plutot que le
+// solde").  The four products are dense contractions, so each is a tcgen05 MMA
+// with bf16 operands and an fp32 accumulator in tensor memory:
+//   MMA1  CB      = C [Q x N] . B [Q x N]^T                    (M = Q,  N = Q, K = N)
+//   MMA3  Y_inter = C [Q x N] . S [P x N]^T                    (M = Q,  N = P, K = N)
+//   MMA4  S^T    += B^T [N x Q] . (x w)^T [P x Q]^T             (M = N,  N = P, K = Q)
+//   MMA2  Y_intra = M [Q x Q] . x^T [P x Q]^T                   (M = Q,  N = P, K = Q)
+// x, B and C are bf16 and enter exactly; the fp32 operands (S, x w, M) enter as
+// a (hi, lo) pair of bf16 matrices whose sum carries about 16 bits of mantissa,
+// two MMAs each, so every product keeps near-fp32 accuracy.  The state stays
+// in tensor memory, transposed (lane n, column p), across the chunks of a head.
+//
+// One CTA of 128 threads per (sequence, head); thread i owns tensor-memory lane i
+// (token i of the chunk, or state column n).  Per chunk: (A) the threads stage
+// the chunk's C, B, B^T, x^T and (x w)^T and the state's (hi, lo) copy in shared
+// memory and rescale the state by e^{Lam_last} in place; (B) one thread issues
+// MMA1, MMA3 and MMA4; (C) the threads turn CB into M (hi, lo) in the space B
+// and B^T occupied; (D) one thread issues MMA2; (E) the threads write y.  Waits
+// on MMA completion are bounded (2 s) and report RSSM_DEV_PIPE_TIMEOUT.
+#include <cuda_bf16.h>
+
+#include "rssm_internal.h"
+#include "rssm_umma.cuh"
+
+namespace rssm {
+
+namespace {
+
+constexpr int kQ = 128;          // chunk length = MMA M
+constexpr int kN = 128;          // dstate = MMA M of the state update
+constexpr int kPT = 128;         // threads per CTA
+constexpr int kTileQN = kQ * kN * 2;  // one [128 x 128] bf16 tile
+
+struct PrefillArgs {
+    int B, H, P, G, T, dt_scales;
+    const __nv_bfloat16 *x;   // [B][T][H][P]
+    const float *dt;          // [B][T][H]
+    const __nv_bfloat16 *Bm;  // [B][T][G][N]
+    const __nv_bfloat16 *Cm;  // [B][T][G][N]
+    const float *A, *D;       // [H]
+    const float *S0;          // [B][H][P][N] or nullptr (zero state)
+    float *y;                 // [B][T][H][P]
+    float *S_out;             // [B][H][P][N]
+    int *err;                 // {code, b, h, value} or nullptr
+};
+
+// Shared memory (bytes from a 1024-aligned base).
+struct PrefillLay {
+    int C, Bk, Bt, Xt, XwHi, XwLo, SHi, SLo, lam, w, red, bar, tslot, bytes;
+};
+__host__ __device__ inline PrefillLay prefill_lay(int P) {
+    PrefillLay L{};
+    int o = 0;
+    const int xp = P * kQ * 2;  // one [P x Q] bf16 tile
+    const int sp = P * kN * 2;  // one [P x N] bf16 tile
+    L.C = o;    o += kTileQN;   // C  [Q rows, K = N]
+    L.Bk = o;   o += kTileQN;   // B  [Q rows, K = N]      (M hi afterwards)
+    L.Bt = o;   o += kTileQN;   // B^T [N rows, K = Q]     (M lo afterwards)
+    L.Xt = o;   o += xp;        // x^T [P rows, K = Q]
+    L.XwHi = o; o += xp;        // (x w)^T hi
+    L.XwLo = o; o += xp;        // (x w)^T lo
+    L.SHi = o;  o += sp;        // S hi [P rows, K = N]
+    L.SLo = o;  o += sp;        // S lo
+    L.lam = o;  o += kQ * 4;    // Lam_i
+    L.w = o;    o += kQ * 4;    // s_j (dt or 1)
+    L.red = o;  o += 64;        // cross-warp scan carries
+    L.bar = o;  o += 16;        // mbarrier
+    L.tslot = o; o += 16;       // tensor-memory address
+    L.bytes = o;
+    return L;
+}
+
+__device__ __forceinline__ void report_err(int *err, int code, int b, int h, int v) {
+    if (err && atomicCAS(err, 0, code) == 0) {
+        err[1] = b;
+        err[2] = h;
+        err[3] = v;
+    }
+}
+
+__device__ __forceinline__ uint32_t pack2(float a, float b) {
+    __nv_bfloat162 t = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<uint32_t *>(&t);
+}
+
+__global__ void __launch_bounds__(kPT, 1) m2_prefill_kernel(const PrefillArgs a) {
+    extern __shared__ __align__(1024) uint8_t psm[];
+    // the swizzled tiles need a 1024-byte aligned base
+    uint8_t *sm = psm + ((1024 - (smem_u32(psm) & 1023)) & 1023);
+    const int P = a.P;
+    const PrefillLay Ly = prefill_lay(P);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int b = blockIdx.y, h = blockIdx.x;
+    const int H = a.H, G = a.G, T = a.T;
+    const int g = h / (H / G);
+    uint8_t *sC = sm + Ly.C, *sBk = sm + Ly.Bk, *sBt = sm + Ly.Bt, *sXt = sm + Ly.Xt;
+    uint8_t *sXwHi = sm + Ly.XwHi, *sXwLo = sm + Ly.XwLo, *sSHi = sm + Ly.SHi, *sSLo = sm + Ly.SLo;
+    uint8_t *sMHi = sBk, *sMLo = sBt;
+    float *slam = reinterpret_cast<float *>(sm + Ly.lam);
+    float *sw = reinterpret_cast<float *>(sm + Ly.w);
+    float *sred = reinterpret_cast<float *>(sm + Ly.red);
+    uint64_t *bar = reinterpret_cast<uint64_t *>(sm + Ly.bar);
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + Ly.tslot);
+    const uint32_t ncols = (128 + 2 * P) <= 256 ? 256u : 512u;
+    // tensor-memory columns: CB (later Y_intra) at 0, Y_inter at 128, S^T at 128 + P
+    const uint32_t cY1 = 0, cY2 = 128, cS = 128 + (uint32_t)P;
+
+    if (warp == 0) tmem_alloc(tslot, ncols);
+    if (tid == 0) {
+        mbar_init(bar, 1);
+        mbar_init_fence();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tslot;
+    const uint32_t lane_base = tmem + ((uint32_t)(32 * warp) << 16);  // this warp's 32 lanes
+    const float Ah = a.A[h], Dh = a.D[h];
+
+    // The initial state, transposed into tensor memory: lane n holds S0[:, n].
+    for (int p0 = 0; p0 < P; p0 += 32) {
+        float v[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+            v[j] = a.S0 ? a.S0[(((int64_t)b * H + h) * P + p0 + j) * kN + tid] : 0.f;
+        tmem_st32(lane_base + cS + p0, v);
+    }
+
+    uint32_t phase = 0;
+    bool failed = false;
+    const int nchunks = (T + kQ - 1) / kQ;
+    for (int c = 0; c < nchunks && !failed; ++c) {
+        const int t0 = c * kQ, Lc = min(kQ, T - t0);
+        const int i = tid;  // token of the chunk owned by this thread
+        const bool live = i < Lc;
+        const int64_t tok = (int64_t)b * T + t0 + i;
+
+        // (A) Prefix sums of dt*A over the chunk (padding tokens add nothing).
+        const float dti = live ? a.dt[tok * H + h] : 0.f;
+        float v = dti * Ah;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const float u = __shfl_up_sync(0xffffffffu, v, o);
+            if (lane >= o) v += u;
+        }
+        if (lane == 31) sred[warp] = v;
+        __syncthreads();
+        float carry = 0.f;
+        for (int w2 = 0; w2 < warp; ++w2) carry += sred[w2];
+        const float lam = v + carry;
+        slam[i] = lam;
+        sw[i] = live ? (a.dt_scales ? dti : 1.f) : 0.f;
+        __syncthreads();
+        const float lam_last = slam[kQ - 1];
+
+        // C and B rows of token i (K-major rows = tokens), B^T and x^T columns.
+        const uint4 *Crow = reinterpret_cast<const uint4 *>(a.Cm + (tok * G + g) * kN);
+        const uint4 *Brow = reinterpret_cast<const uint4 *>(a.Bm + (tok * G + g) * kN);
+        for (int ch = 0; ch < kN / 8; ++ch) {
+            const uint4 cv = live ? Crow[ch] : make_uint4(0, 0, 0, 0);
+            const uint4 bv = live ? Brow[ch] : make_uint4(0, 0, 0, 0);
+            *reinterpret_cast<uint4 *>(sC + sw128_chunk(i, ch, kQ)) = cv;
+            *reinterpret_cast<uint4 *>(sBk + sw128_chunk(i, ch, kQ)) = bv;
+            const __nv_bfloat16 *be = reinterpret_cast<const __nv_bfloat16 *>(&bv);
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+                *reinterpret_cast<__nv_bfloat16 *>(sBt + sw128_off(8 * ch + e, i, kN)) = be[e];
+        }
+        const float wi = live ? expf(lam_last - lam) * sw[i] : 0.f;
+        const uint4 *Xrow = reinterpret_cast<const uint4 *>(a.x + (tok * H + h) * P);
+        for (int ch = 0; ch < P / 8; ++ch) {
+            const uint4 xv = live ? Xrow[ch] : make_uint4(0, 0, 0, 0);
+            const __nv_bfloat16 *xe = reinterpret_cast<const __nv_bfloat16 *>(&xv);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const int p = 8 * ch + e;
+                *reinterpret_cast<__nv_bfloat16 *>(sXt + sw128_off(p, i, P)) = xe[e];
+                __nv_bfloat16 hi, lo;
+                split_bf16(__bfloat162float(xe[e]) * wi, hi, lo);
+                *reinterpret_cast<__nv_bfloat16 *>(sXwHi + sw128_off(p, i, P)) = hi;
+                *reinterpret_cast<__nv_bfloat16 *>(sXwLo + sw128_off(p, i, P)) = lo;
+            }
+        }
+        // The state at the chunk's start: (hi, lo) copy for MMA3 (S rows p, K = n),
+        // and e^{Lam_last} S back into tensor memory for MMA4 to accumulate onto.
+        const float dec = expf(lam_last);
+        for (int p0 = 0; p0 < P; p0 += 32) {
+            float s[32];
+            tmem_ld32(lane_base + cS + p0, s);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                __nv_bfloat16 hi, lo;
+                split_bf16(s[j], hi, lo);
+                *reinterpret_cast<__nv_bfloat16 *>(sSHi + sw128_off(p0 + j, tid, P)) = hi;
+                *reinterpret_cast<__nv_bfloat16 *>(sSLo + sw128_off(p0 + j, tid, P)) = lo;
+                s[j] *= dec;
+            }
+            tmem_st32(lane_base + cS + p0, s);
+        }
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+
+        // (B) MMA1 (CB), MMA3 (Y_inter, hi and lo), MMA4 (state, hi and lo).
+        if (tid == 0) {
+            const uint32_t aC = smem_u32(sC), aB = smem_u32(sBk), aBt = smem_u32(sBt);
+            for (int ks = 0; ks < kN / 16; ++ks)
+                umma_bf16(tmem + cY1, sw128_desc(aC, kQ, ks), sw128_desc(aB, kQ, ks), idesc_bf16_f32(kQ, kQ), ks > 0);
+            for (int hl = 0; hl < 2; ++hl) {
+                const uint32_t aS = smem_u32(hl ? sSLo : sSHi);
+                for (int ks = 0; ks < kN / 16; ++ks)
+                    umma_bf16(tmem + cY2, sw128_desc(aC, kQ, ks), sw128_desc(aS, P, ks), idesc_bf16_f32(kQ, P),
+                              hl > 0 || ks > 0);
+            }
+            for (int hl = 0; hl < 2; ++hl) {
+                const uint32_t aX = smem_u32(hl ? sXwLo : sXwHi);
+                for (int ks = 0; ks < kQ / 16; ++ks)
+                    umma_bf16(tmem + cS, sw128_desc(aBt, kN, ks), sw128_desc(aX, P, ks), idesc_bf16_f32(kN, P), true);
+            }
+            umma_commit(bar);
+        }
+        __syncwarp();
+        if (!mbar_wait(bar, phase & 1)) failed = true;
+        ++phase;
+        if (__syncthreads_or(failed)) {
+            failed = true;
+            break;
+        }
+        tc_fence_after();
+
+        // (C) M = tril(e^{Lam_i - Lam_j}) (.) CB (.) s_j as (hi, lo), row i per thread.
+        for (int j0 = 0; j0 < kQ; j0 += 32) {
+            float cb[32];
+            tmem_ld32(lane_base + cY1 + j0, cb);
+#pragma unroll
+            for (int ch = 0; ch < 4; ++ch) {
+                uint32_t hw[4], lw[4];
+#pragma unroll
+                for (int e2 = 0; e2 < 4; ++e2) {
+                    float m2[2];
+#pragma unroll
+                    for (int u = 0; u < 2; ++u) {
+                        const int jj = 8 * ch + 2 * e2 + u, j = j0 + jj;
+                        m2[u] = (j <= i) ? expf(lam - slam[j]) * cb[jj] * sw[j] : 0.f;
+                    }
+                    __nv_bfloat16 h0, l0, h1, l1;
+                    split_bf16(m2[0], h0, l0);
+                    split_bf16(m2[1], h1, l1);
+                    hw[e2] = pack2(__bfloat162float(h0), __bfloat162float(h1));
+                    lw[e2] = pack2(__bfloat162float(l0), __bfloat162float(l1));
+                }
+                const int chunk = (j0 >> 3) + ch;
+                *reinterpret_cast<uint4 *>(sMHi + sw128_chunk(i, chunk, kQ)) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+                *reinterpret_cast<uint4 *>(sMLo + sw128_chunk(i, chunk, kQ)) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+            }
+        }
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+
+        // (D) MMA2: Y_intra = M x (hi and lo), over the CB columns.
+        if (tid == 0) {
+            const uint32_t aX = smem_u32(sXt);
+            for (int hl = 0; hl < 2; ++hl) {
+                const uint32_t aM = smem_u32(hl ? sMLo : sMHi);
+                for (int ks = 0; ks < kQ / 16; ++ks)
+                    umma_bf16(tmem + cY1, sw128_desc(aM, kQ, ks), sw128_desc(aX, P, ks), idesc_bf16_f32(kQ, P),
+                              hl > 0 || ks > 0);
+            }
+            umma_commit(bar);
+        }
+        __syncwarp();
+        if (!mbar_wait(bar, phase & 1)) failed = true;
+        ++phase;
+        if (__syncthreads_or(failed)) {
+            failed = true;
+            break;
+        }
+        tc_fence_after();
+
+        // (E) y_i = Y_intra + e^{Lam_i} Y_inter + D x_i.
+        const float di = expf(lam);
+        for (int p0 = 0; p0 < P; p0 += 32) {
+            float y1[32], y2[32];
+            tmem_ld32(lane_base + cY1 + p0, y1);
+            tmem_ld32(lane_base + cY2 + p0, y2);
+            if (live) {
+                const __nv_bfloat16 *xr = a.x + (tok * H + h) * P + p0;
+                float4 *yr = reinterpret_cast<float4 *>(a.y + (tok * H + h) * P + p0);
+#pragma unroll
+                for (int j4 = 0; j4 < 8; ++j4) {
+                    float o[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int j = 4 * j4 + u;
+                        o[u] = fmaf(di, y2[j], y1[j]) + Dh * __bfloat162float(xr[j]);
+                    }
+                    yr[j4] = make_float4(o[0], o[1], o[2], o[3]);
+                }
+            }
+        }
+        tc_fence_before();
+        __syncthreads();  // shared memory and tensor-memory columns are reused by the next chunk
+        tc_fence_after();
+    }
+
+    if (failed) {
+        if (tid == 0) report_err(a.err, DEV_PIPE_TIMEOUT, b, h, 0);
+    } else {
+        // The state after the prompt, S_out[b][h][p][n] from lane n.
+        for (int p0 = 0; p0 < P; p0 += 32) {
+            float s[32];
+            tmem_ld32(lane_base + cS + p0, s);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) a.S_out[(((int64_t)b * H + h) * P + p0 + j) * kN + tid] = s[j];
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem, ncols);
+}
+
+}  // namespace
+
+size_t prefill_smem_bytes(int P) { return (size_t)prefill_lay(P).bytes + 1024; }
+
+}  // namespace rssm
+
+extern "C" RSSM_API rssm_status rssm_mamba2_prefill(const rssm_prefill_config *cfg, const float *A, const float *D,
+                                                    const float *S0, const rssm_inputs *in, float *y, float *S_out,
+                                                    int32_t *dev_error, void *stream) {
+    using namespace rssm;
+    if (!cfg || !A || !D || !in || !in->x || !in->dt || !in->Bm || !in->Cm || !y || !S_out)
+        return RSSM_EINVAL;
+    const rssm_prefill_config &c = *cfg;
+    if (c.batch < 1 || c.nheads < 1 || c.ngroups < 1 || c.nheads % c.ngroups != 0 || c.T < 1) return RSSM_EINVAL;
+    if (c.dstate != kN || c.headdim < 32 || c.headdim > 96 || c.headdim % 32 != 0) return RSSM_EINVAL;
+    if (S0 && S0 == S_out) return RSSM_EINVAL;
+    if (c.dt_scales_input != 0 && c.dt_scales_input != 1) return RSSM_EINVAL;
+    auto al16 = [](const void *p) { return ((uintptr_t)p & 15) == 0; };
+    if (!al16(in->x) || !al16(in->Bm) || !al16(in->Cm) || !al16(y)) return RSSM_EINVAL;
+    PrefillArgs a{};
+    a.B = c.batch; a.H = c.nheads; a.P = c.headdim; a.G = c.ngroups; a.T = c.T; a.dt_scales = c.dt_scales_input;
+    a.x = (const __nv_bfloat16 *)in->x; a.dt = in->dt;
+    a.Bm = (const __nv_bfloat16 *)in->Bm; a.Cm = (const __nv_bfloat16 *)in->Cm;
+    a.A = A; a.D = D; a.S0 = S0; a.y = y; a.S_out = S_out; a.err = (int *)dev_error;
+    const size_t smem = prefill_smem_bytes(c.headdim);
+    cudaError_t e = cudaFuncSetAttribute(m2_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return RSSM_ECUDA;
+    m2_prefill_kernel<<<dim3(c.nheads, c.batch), kPT, smem, (cudaStream_t)stream>>>(a);
+    return cudaGetLastError() == cudaSuccess ? RSSM_OK : RSSM_ECUDA;
+}

@@ -1,0 +1,129 @@
+// rssm_umma.cuh -- 5th-generation tensor-core (tcgen05) primitives for sm_100a:
+// tensor-memory allocation, shared-memory matrix descriptors, the bf16 MMA with
+// an fp32 accumulator in tensor memory, its completion on an mbarrier, and
+// tensor-memory loads and stores.  Inline PTX; no library code.
+//
+// Operand tiles live in shared memory in the K-major layout with the 128-byte
+// swizzle: a tile of R rows (R a multiple of 8) and K bf16 columns (K a
+// multiple of 64) is stored as K/64 column blocks of R x 128 bytes; inside a
+// block, row r occupies bytes [r*128, r*128 + 128) of its 8-row group
+// (groups 1024 bytes apart) and its 16-byte chunk c sits at chunk c ^ (r % 8).
+// Every column block starts on a 1024-byte boundary.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "rssm_pipe.cuh"
+
+namespace rssm {
+
+// Byte offset of bf16 element (r, k) in a K-major 128-byte-swizzled tile of R rows.
+__device__ __forceinline__ uint32_t sw128_off(int r, int k, int R) {
+    const int kb = k >> 6, kk = k & 63;
+    return (uint32_t)(kb * (R * 128) + (r >> 3) * 1024 + (r & 7) * 128 + ((((kk >> 3) ^ (r & 7))) << 4) +
+                      ((kk & 7) << 1));
+}
+// Byte offset of the 16-byte chunk holding elements (r, 8c .. 8c+7).
+__device__ __forceinline__ uint32_t sw128_chunk(int r, int c, int R) {
+    const int kb = c >> 3, cc = c & 7;
+    return (uint32_t)(kb * (R * 128) + (r >> 3) * 1024 + (r & 7) * 128 + ((cc ^ (r & 7)) << 4));
+}
+
+// Shared-memory matrix descriptor of the K slice [16 ks, 16 ks + 16) of such a
+// tile (R rows): start address, stride between 8-row groups 1024 bytes, the
+// 128-byte swizzle, descriptor version 1.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t tile_saddr, int R, int ks) {
+    const uint32_t start = tile_saddr + (uint32_t)((ks >> 2) * (R * 128) + (ks & 3) * 32);
+    uint64_t d = (uint64_t)((start >> 4) & 0x3FFFu);
+    d |= (uint64_t)1 << 16;             // leading-dimension offset (unused for swizzled K-major)
+    d |= (uint64_t)(1024 >> 4) << 32;   // stride-dimension offset: 8-row groups
+    d |= (uint64_t)1 << 46;             // descriptor version
+    d |= (uint64_t)2 << 61;             // 128-byte swizzle
+    return d;
+}
+
+// Instruction descriptor of kind::f16 with bf16 A and B (both K-major) and an
+// fp32 accumulator, M x N.
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// D[tmem] (+)= A[desc] * B[desc]^T, issued by one thread.
+__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                          bool accumulate) {
+    asm volatile(
+        "{\n .reg .pred p;\n setp.ne.u32 p, %4, 0;\n"
+        " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"((uint32_t)accumulate)
+        : "memory");
+}
+
+// Arrive on `bar` once every MMA this thread has issued so far has completed.
+__device__ __forceinline__ void umma_commit(uint64_t *bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+
+// Tensor-memory allocation by one whole warp; the address is written to *slot.
+__device__ __forceinline__ void tmem_alloc(uint32_t *slot, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(slot)),
+                 "r"(ncols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+// Generic-proxy shared-memory writes become visible to the tensor cores' reads.
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+// 32 consecutive fp32 columns of this thread's tensor-memory lane (warp w of a
+// 128-thread group reads lanes 32w .. 32w + 31; taddr carries the lane in its
+// upper half).  Waits for the load.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+          "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),
+          "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+}
+
+// Store 32 consecutive fp32 columns of this thread's lane.  Waits for the store.
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+        "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+        "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+        "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
+        "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+        "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
+        "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])), "r"(__float_as_uint(v[17])),
+        "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])), "r"(__float_as_uint(v[20])),
+        "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])), "r"(__float_as_uint(v[23])),
+        "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])),
+        "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])),
+        "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+        : "memory");
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// fp32 -> (hi, lo) bf16 pair with hi + lo = v to about 2^-16 relative: the
+// split that lets a bf16 tensor-core product carry an fp32 operand.
+__device__ __forceinline__ void split_bf16(float v, __nv_bfloat16 &hi, __nv_bfloat16 &lo) {
+    hi = __float2bfloat16_rn(v);
+    lo = __float2bfloat16_rn(v - __bfloat162float(hi));
+}
+
+}  // namespace rssm

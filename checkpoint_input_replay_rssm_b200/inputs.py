@@ -78,8 +78,13 @@ WORKLOADS = {
     # Kimi Delta Attention layer (per-channel gate), the GDN layer's shapes
     "kda_b256_h32_dk128_dv128_w16": Workload(
         "kda_b256_h32_dk128_dv128_w16", "kda", 256, 32, 128, 128, 32, 16, 256, 5, "bf16", "bf16"),
+    # prompt prefill of the Nemotron-scale layer: 512 prompt tokens per sequence
+    # (steps = prompt length), handing its final state to the decode checkpoint
+    "mamba2_prefill_b256_h128_p64_n128_g8_t512": Workload(
+        "mamba2_prefill_b256_h128_p64_n128_g8_t512", "mamba2", 256, 128, 64, 128, 8, 16, 512, 6,
+        "bf16", "bf16"),
 }
-TINY, NEMOTRON, SPECVERIFY, GDN, FP8DRIFT, KDA = WORKLOADS.values()
+TINY, NEMOTRON, SPECVERIFY, GDN, FP8DRIFT, KDA, PREFILL = WORKLOADS.values()
 
 
 def _rng(*key: int) -> np.random.Generator:

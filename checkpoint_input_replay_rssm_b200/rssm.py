@@ -45,9 +45,15 @@ class rssm_inputs(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in ("x", "dt", "Bm", "Cm", "q", "k", "v", "alpha", "beta")]
 
 
+class rssm_prefill_config(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in (
+        "batch", "nheads", "headdim", "dstate", "ngroups", "T", "dt_scales_input")]
+
+
 # C declarations: name -> (restype, argtypes)
 _VP, _I32, _SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
 _CFGP, _LAYP, _INP = ctypes.POINTER(rssm_config), ctypes.POINTER(rssm_workspace_layout), ctypes.POINTER(rssm_inputs)
+_PCFGP = ctypes.POINTER(rssm_prefill_config)
 SIGNATURES = {
     "rssm_workspace_bytes": (_SZ, [_CFGP]),
     "rssm_workspace_layout_of": (ctypes.c_int, [_CFGP, _LAYP]),
@@ -68,6 +74,7 @@ SIGNATURES = {
     "rssm_set_split_event": (ctypes.c_int, [_VP, _VP]),
     "rssm_launch_count": (ctypes.c_int64, [_VP]),
     "rssm_last_error": (ctypes.c_char_p, [_VP]),
+    "rssm_mamba2_prefill": (ctypes.c_int, [_PCFGP, _VP, _VP, _VP, _INP, _VP, _VP, _VP, _VP]),
 }
 
 _lib = None
@@ -193,6 +200,35 @@ def rssm_launch_count(h) -> int:
 def rssm_last_error(h=None) -> str:
     m = load().rssm_last_error(h)
     return m.decode() if m else ""
+
+
+def rssm_mamba2_prefill(cfg: rssm_prefill_config, A_ptr: int, D_ptr: int, S0_ptr, inputs: rssm_inputs,
+                        y_ptr: int, S_out_ptr: int, err_ptr, stream_ptr):
+    st = load().rssm_mamba2_prefill(ctypes.byref(cfg), A_ptr, D_ptr, S0_ptr, ctypes.byref(inputs), y_ptr,
+                                    S_out_ptr, err_ptr, stream_ptr)
+    if st != RSSM_OK:
+        raise RssmError(st, "rssm_mamba2_prefill refused its arguments" if st == RSSM_EINVAL
+                        else "rssm_mamba2_prefill launch failed")
+
+
+def prefill(x, dt, Bm, Cm, A, D, S0=None, dt_scales_input=False, y=None, S_out=None, err=None, stream=None):
+    """Torch convenience over rssm_mamba2_prefill: x [B,T,H,P] bf16, dt [B,T,H] fp32,
+    Bm/Cm [B,T,G,N] bf16, A/D [H] fp32, S0 [B,H,P,N] fp32 or None.  Returns (y, S_out)."""
+    import torch
+
+    Bn, T, H, P = x.shape
+    G, N = Bm.shape[2], Bm.shape[3]
+    for t, dty in ((x, torch.bfloat16), (Bm, torch.bfloat16), (Cm, torch.bfloat16), (dt, torch.float32),
+                   (A, torch.float32), (D, torch.float32)):
+        assert t.is_cuda and t.is_contiguous() and t.dtype == dty
+    y = y if y is not None else torch.empty((Bn, T, H, P), dtype=torch.float32, device=x.device)
+    S_out = S_out if S_out is not None else torch.empty((Bn, H, P, N), dtype=torch.float32, device=x.device)
+    cfg = rssm_prefill_config(Bn, H, P, N, G, T, int(bool(dt_scales_input)))
+    ins = rssm_inputs(x=x.data_ptr(), dt=dt.data_ptr(), Bm=Bm.data_ptr(), Cm=Cm.data_ptr())
+    st = stream if stream is not None else torch.cuda.current_stream(x.device)
+    rssm_mamba2_prefill(cfg, A.data_ptr(), D.data_ptr(), None if S0 is None else S0.data_ptr(), ins,
+                        y.data_ptr(), S_out.data_ptr(), None if err is None else err.data_ptr(), st.cuda_stream)
+    return y, S_out
 
 
 # ---------------------------------------------------------------- torch owner

@@ -133,7 +133,7 @@ typedef struct {
                                             KDA alpha[B][H][R][N] (fp32)                              */
     size_t tbuf_off, tbuf_bytes;         /* GDN/KDA beta[B][H][ring_stride] (fp32)                 */
     size_t snap_off, snap_bytes;         /* EAGER: max_draft snapshots of the state (+ scales)      */
-    /* REPLAY: hand-off from the prep kernel to the read kernel within one call */
+    /* REPLAY: hand-off from the prep kernel to the flush and read kernels within one call */
     size_t tq_max;                       /* max(max_draft, 1): queries per call            */
     size_t seqinfo_off, seqinfo_bytes;   /* int32[B][4] per sequence, then the flush kernel's
                                             work list: int32 count, 3 pad, int32[B] (padded) */
@@ -196,18 +196,58 @@ RSSM_API rssm_status rssm_export_state(rssm_handle h, float *S_out);
  * [B][1][H][P]) and commits the token. */
 RSSM_API rssm_status rssm_decode(rssm_handle h, const rssm_inputs *in, float *y);
 
-/* rssm_decode for REPLAY Mamba-2 layers with its per-call scratch (the prep
- * kernel's hand-off to the flush and read kernels) in one library-owned static
- * device array of 4 MiB instead of the handle's workspace: for callers that
- * give each layer memory for its state only and decode the layers one after
- * another on one stream.  The pages on checkpointed input replay have no
- * counterpart; the results equal rssm_decode's.  Allocates nothing.  Refused
- * (RSSM_EINVAL, nothing enqueued) for other layers and when the hand-off
- * (about batch * nheads * (window + 4) * 4 bytes) exceeds the array.  All calls
- * on a device share the array, so calls that may run concurrently race.  The
- * first call on a device looks up the array's address; make one call before
- * recording calls into a stream capture. */
+/* rssm_decode with the call's scratch in one library-owned static device array
+ * of 8 MiB instead of the handle's workspace, for callers that cannot allocate
+ * device memory on the decode path (a memory pool fixed before the model loads,
+ * a captured step where an allocation would stall or is not allowed) and that
+ * decode their layers one after another on one stream.  The scratch is the prep
+ * kernel's per-call hand-off to the flush and read kernels.  The pages on
+ * checkpointed input replay have no counterpart; the results equal
+ * rssm_decode's.  Allocates nothing.  REPLAY layers only (EAGER: RSSM_EINVAL).
+ * Refused (RSSM_EINVAL, nothing enqueued) when the hand-off -- batch * 20 + 16 +
+ * batch * nheads * 4 * (1 + round_up4(window + 1)) bytes, plus
+ * batch * nheads * dstate * 4 for GDN/KDA, each region padded to 256 bytes --
+ * exceeds the array.  All calls on a device share the array and leave their
+ * contents in it, so calls that may run concurrently (several streams or
+ * threads) race.  The first call on a device looks up the array's address and
+ * keeps it for the life of the process: make that call before any stream
+ * capture, and do not use this entry point on a device again after
+ * cudaDeviceReset. */
 RSSM_API rssm_status rssm_decode_static_scratch(rssm_handle h, const rssm_inputs *in, float *y);
+
+/* Prompt prefill of a Mamba-2 layer, the step before replay decode: for every
+ * sequence b and head h, run the prompt's T tokens through the recurrence from
+ * the state S0 and write every token's output and the fp32 state after the
+ * prompt -- the checkpoint a decode starts from, to be installed with
+ * rssm_import_state.  The prompt is processed in chunks of 128 tokens: within a
+ * chunk the outputs come from the chunk's own inputs through the decayed pairwise
+ * products C_t . B_s plus the state at the chunk's start, and the state moves to
+ * the next chunk by one decay and a rank-128 update (the checkpoint + buffered
+ * inputs algebra of the replay read, the chunk being the buffer;
+ * blog.thibaultmonteiro.fr, "Tenir le journal plutot que le solde").  The pages
+ * describe no prefill; the result is the eager recurrence's
+ * (y_t = S_t C_t + D x_t) to fp32 accuracy: the products run on the tensor cores
+ * with bf16 operands, the fp32 ones split into two bf16 parts.
+ *   cfg:   batch, nheads, ngroups as for rssm_config; headdim P in {32, 64, 96};
+ *          dstate must be 128; T >= 1 prompt tokens; dt_scales_input 0 or 1.
+ *   A, D:  device fp32 [H].  S0: device fp32 [B][H][P][N], or NULL for a zero state.
+ *   in:    x [B][T][H][P] bf16, dt [B][T][H] fp32, Bm, Cm [B][T][G][N] bf16 (device,
+ *          16-byte aligned; the other fields are ignored).
+ *   y:     device fp32 [B][T][H][P] (16-byte aligned).  S_out: device fp32 [B][H][P][N]
+ *          (may not alias S0).
+ *   dev_error: device int32[4] or NULL; {RSSM_DEV_PIPE_TIMEOUT, b, h, 0} is written
+ *          there if a tensor-core wait gives up (2 s), and that head's S_out is not written.
+ *   stream: cudaStream_t (NULL = legacy default stream).
+ * Enqueues one kernel and returns; allocates nothing.  RSSM_EINVAL (nothing
+ * enqueued) for NULL pointers, unsupported sizes or misaligned arrays. */
+typedef struct {
+    int32_t batch, nheads, headdim, dstate, ngroups;
+    int32_t T;               /* prompt tokens >= 1 */
+    int32_t dt_scales_input; /* 1 = input term dt_t x_t B_t^T, 0 = x_t B_t^T */
+} rssm_prefill_config;
+RSSM_API rssm_status rssm_mamba2_prefill(const rssm_prefill_config *cfg, const float *A, const float *D,
+                                         const float *S0, const rssm_inputs *in, float *y, float *S_out,
+                                         int32_t *dev_error, void *stream);
 
 /* Speculative verify of K drafts (1 <= K <= max_draft, K <= W) for every
  * sequence: folds where len + K > W, appends the drafts uncommitted and writes
