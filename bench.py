@@ -38,14 +38,17 @@ FALLBACK_HBM_GBS = 6650.0
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "m2_replay_decode_b256_h128_p64_n128_w16.traffic.json")
 
 
+TRAFFIC_SOURCES = ("rssm_read.cuh", "rssm_device.cuh")
+
+
 def kernel_source_hash() -> str:
-    """Hash of the CUDA sources, to tell whether a stored ncu traffic figure is current."""
+    """Hash of the sources of the replay-read kernel, to tell whether a stored ncu
+    traffic figure was taken on the kernel as it is now."""
     h = hashlib.sha256()
     d = os.path.join(ROOT, "checkpoint_input_replay_rssm_b200", "csrc")
-    for f in sorted(os.listdir(d)):
-        if f.endswith((".cu", ".cuh", ".h")):
-            h.update(f.encode())
-            h.update(open(os.path.join(d, f), "rb").read())
+    for f in TRAFFIC_SOURCES:
+        h.update(f.encode())
+        h.update(open(os.path.join(d, f), "rb").read())
     return h.hexdigest()[:16]
 
 
@@ -245,6 +248,107 @@ def delta_leg(wl0, rank, device, sync, dist, world, steps, warmup):
     return out
 
 
+def hybrid_leg(device, sync, dist, world, steps, warmup):
+    """A synthetic hybrid decode step on the Nemotron-scale layer shapes: one block
+    of five Mamba-2 layers (this library, replay with a bf16 copy or the eager
+    fp32 baseline) and one attention layer (32 query / 2 key-value heads of 128,
+    4096 cached tokens, bf16), each with bf16 in/out projections of a 4096-wide
+    hidden state, random weights.  Whole-step tokens/s for each SSM mode, and the
+    share of the step spent in the SSM layers' decode calls (a second pass with
+    CUDA events around every decode call)."""
+    import torch
+
+    from checkpoint_input_replay_rssm_b200.hybrid import HybridShape, HybridStack
+
+    shape = HybridShape()
+    out = {}
+    for name, mode, rd in (("replay", "replay", "bf16"), ("eager", "eager", "f32")):
+        st = HybridStack(shape, ssm_mode=mode, read_dtype=rd, seed=11, device=device,
+                         max_steps=warmup + 2 * steps + 2)
+        g = torch.Generator(device=device).manual_seed(12)
+        xs = [torch.randn((shape.batch, shape.d_model), generator=g, device=device).to(torch.bfloat16)
+              for _ in range(8)]
+        for i in range(warmup):
+            st.step(xs[i % 8])
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        sync()
+        e0.record()
+        for i in range(steps):
+            st.step(xs[i % 8])
+        e1.record()
+        sync()
+        (ms,) = max_over_ranks(dist, [e0.elapsed_time(e1)], device)
+        st.ssm_events = []
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record()
+        for i in range(steps):
+            st.step(xs[i % 8])
+        f1.record()
+        sync()
+        ssm_ms = sum(a.elapsed_time(b) for a, b in st.ssm_events)
+        timed_ms = f0.elapsed_time(f1)
+        for L in st.ssm_layers():
+            assert L.status()[0] == 0, "device error in the hybrid leg"
+        out[name] = {"value": job_tokens_per_s(world, shape.batch, steps, ms), "unit": "tokens/s",
+                     "ms_per_step": ms / steps, "ssm_ms_per_step": ssm_ms / steps,
+                     "ssm_share": ssm_ms / timed_ms}
+        del st
+        torch.cuda.empty_cache()
+    out["step_speedup"] = out["eager"]["ms_per_step"] / out["replay"]["ms_per_step"]
+    out["ssm_speedup"] = out["eager"]["ssm_ms_per_step"] / out["replay"]["ssm_ms_per_step"]
+    out["config"] = {"blocks": shape.blocks, "ssm_per_attention": shape.ssm_per_block, "batch_per_gpu": shape.batch,
+                     "d_model": shape.d_model, "ssm_layer": "mamba2 128 heads x 64 x 128, 8 groups, W 16",
+                     "attention": f"{shape.n_q_heads} q / {shape.n_kv_heads} kv heads x {shape.head_dim}, "
+                                  f"{shape.context} cached tokens, bf16, torch SDPA",
+                     "projections": "bf16 torch.matmul, random weights", "steps": steps}
+    return out
+
+
+def prefill_leg(device, sync, dist, world, reps, warmup):
+    """Prompt prefill of the Nemotron-scale layer on the tensor cores: 256 sequences x
+    128 heads, 512-token prompts, seeded device-generated inputs of the decode
+    workload's distributions; prompt tokens/s and the roofline of the kernel."""
+    import torch
+
+    from checkpoint_input_replay_rssm_b200 import rssm
+
+    wl = I.PREFILL
+    Bn, T, H, G, P, N = wl.batch, wl.steps, wl.nheads, wl.ngroups, wl.headdim, wl.dstate
+    g = torch.Generator(device=device).manual_seed(wl.seed)
+    x = torch.randn((Bn, T, H, P), generator=g, device=device).to(torch.bfloat16)
+    dt = torch.nn.functional.softplus(torch.randn((Bn, T, H), generator=g, device=device) - 2.0)
+    Bm = torch.randn((Bn, T, G, N), generator=g, device=device).to(torch.bfloat16)
+    Cm = torch.randn((Bn, T, G, N), generator=g, device=device).to(torch.bfloat16)
+    A = -torch.exp(torch.rand(H, generator=g, device=device))
+    D = torch.randn(H, generator=g, device=device)
+    S0 = 0.1 * torch.randn((Bn, H, P, N), generator=g, device=device)
+    y = torch.empty((Bn, T, H, P), dtype=torch.float32, device=device)
+    S = torch.empty_like(S0)
+    err = torch.zeros(4, dtype=torch.int32, device=device)
+    for _ in range(warmup):
+        rssm.prefill(x, dt, Bm, Cm, A, D, S0, y=y, S_out=S, err=err)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sync()
+    e0.record()
+    for _ in range(reps):
+        rssm.prefill(x, dt, Bm, Cm, A, D, S0, y=y, S_out=S, err=err)
+    e1.record()
+    sync()
+    assert err.tolist() == [0, 0, 0, 0], "device error in the prefill leg"
+    (ms,) = max_over_ranks(dist, [e0.elapsed_time(e1) / reps], device)
+    heads = Bn * H
+    bytes_per_launch = heads * (T * (P * 2 + P * 4 + 4) + P * N * 4 * 2) + Bn * T * G * N * 2 * 2
+    # tensor-core work: per head and 128-token chunk, C B^T (1x), S C (2x), the
+    # state update (2x) and M x (2x), the fp32 operands split in two bf16 parts
+    chunks = -(-T // 128)
+    flops = heads * chunks * (2 * 128 * 128 * N + 2 * 2 * 128 * P * N + 2 * 2 * N * P * 128 + 2 * 2 * 128 * P * 128)
+    return {"value": world * Bn * T / (ms * 1e-3), "unit": "prompt tokens/s", "ms_per_launch": ms,
+            "hbm_gbs": bytes_per_launch / (ms * 1e-3) / 1e9, "algorithmic_bytes_per_launch": bytes_per_launch,
+            "tensor_tflops": flops / (ms * 1e-3) / 1e12, "mma_flops_per_launch": flops,
+            "config": {"workload": wl.name, "batch_per_gpu": Bn, "prompt_tokens": T, "chunk": 128,
+                       "inputs": "bf16 x, B, C; fp32 dt", "state": "fp32 in and out", "y": "fp32"}}
+
+
 def host_tokens(wl, n):
     """n distinct seeded decode steps as pinned host tensors in storage dtypes."""
     import torch
@@ -262,10 +366,12 @@ def host_tokens(wl, n):
 
 def timed_loop(L, toks_dev, ys, K, W, sync, split=True):
     """W warm-up then K timed decode steps (the headline: CUDA events around the whole
-    loop only, so the read kernel may overlap the prep kernel's tail); with ``split``,
-    K more steps with CUDA events on the layer's stream around every call and between
-    its prep/flush and replay-read kernels (an event between them keeps the two
-    kernels apart, so each one's duration is its own)."""
+    loop only, so the read kernel may overlap the prep kernel's tail); then M whole
+    windows (M * window steps, each window holding exactly one folding call) timed
+    the same way, the steady state; with ``split``, K more steps with CUDA events
+    on the layer's stream around every call and between its prep/flush and
+    replay-read kernels (an event between them keeps the two kernels apart, so
+    each one's duration is its own)."""
     import torch
 
     from checkpoint_input_replay_rssm_b200 import rssm
@@ -287,8 +393,19 @@ def timed_loop(L, toks_dev, ys, K, W, sync, split=True):
     sync()
     launches = L.launches() - l0
     total_ms = t0.elapsed_time(t1)
+    win = L.cfg.window
+    M = max(1, round(K / win))
+    t2, t3 = mk(), mk()
+    sync()
+    t2.record(stream)
+    for i in range(M * win):
+        rssm.rssm_decode(L.h, ins[(W + K + i) % n], yptr[i % len(ys)])
+    t3.record(stream)
+    sync()
+    steady = (t2.elapsed_time(t3), M * win)
+    W = W + M * win  # calls since the import, for the per-kernel pass below
     if not split:
-        return total_ms, None, None, None, launches
+        return total_ms, None, None, None, launches, steady
     starts, mids, ends = [mk() for _ in range(K)], [mk() for _ in range(K)], [mk() for _ in range(K)]
     for e in mids:  # materialise the CUDA events before handing them to the library
         e.record(stream)
@@ -301,38 +418,65 @@ def timed_loop(L, toks_dev, ys, K, W, sync, split=True):
     sync()
     rssm.rssm_set_split_event(L.h, None)
     per = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    prep = [s.elapsed_time(m) for s, m in zip(starts, mids)]
+    pre = [s.elapsed_time(m) for s, m in zip(starts, mids)]
     read = [m.elapsed_time(e) for m, e in zip(mids, ends)]
-    return total_ms, per, prep, read, launches
+    return total_ms, per, pre, read, launches, steady
 
 
 def e2e_loop(L, toks_host, K, W, sync):
-    """Public-API decode with host buffers: pinned H2D of the step's inputs, decode,
-    D2H of the step's output, all inside the timed region."""
+    """Public-API decode with host buffers: every step copies its inputs from pinned
+    host memory to the device, decodes, and copies its output y back to pinned host
+    memory, all inside the timed region.  Two sets of device buffers alternate so
+    that step i's input copy (one copy stream) and step i-1's output copy (another)
+    run while the layer's stream decodes; events order each buffer's reuse."""
     import torch
 
-    dev = {k: torch.empty_like(v, device=L.device) for k, v in toks_host[0].items()}
-    y = torch.empty((L.B, 1, L.H, L.P), dtype=torch.float32, device=L.device)
-    y_host = torch.empty_like(y, device="cpu").pin_memory()
     n = len(toks_host)
+    dev = [{k: torch.empty_like(v, device=L.device) for k, v in toks_host[0].items()} for _ in range(2)]
+    y = [torch.empty((L.B, 1, L.H, L.P), dtype=torch.float32, device=L.device) for _ in range(2)]
+    y_host = [torch.empty_like(y[0], device="cpu").pin_memory() for _ in range(2)]
+    comp = torch.cuda.ExternalStream(L.stream) if not isinstance(L.stream, torch.cuda.Stream) else L.stream
+    h2d_s, d2h_s = torch.cuda.Stream(L.device), torch.cuda.Stream(L.device)
+    ev = lambda: torch.cuda.Event()
+    in_ready, in_free = [ev(), ev()], [ev(), ev()]
+    y_ready, y_free = [ev(), ev()], [ev(), ev()]
+    for j in range(2):  # every buffer starts free
+        in_free[j].record(comp)
+        y_free[j].record(d2h_s)
 
     def step(i):
-        for k, v in toks_host[i % n].items():
-            dev[k].copy_(v, non_blocking=True)
-        L.decode(dev, y=y)
-        y_host.copy_(y, non_blocking=True)
+        j = i % 2
+        with torch.cuda.stream(h2d_s):
+            h2d_s.wait_event(in_free[j])
+            for k, v in toks_host[i % n].items():
+                dev[j][k].copy_(v, non_blocking=True)
+            in_ready[j].record(h2d_s)
+        comp.wait_event(in_ready[j])
+        comp.wait_event(y_free[j])
+        L.decode(dev[j], y=y[j])
+        in_free[j].record(comp)
+        y_ready[j].record(comp)
+        with torch.cuda.stream(d2h_s):
+            d2h_s.wait_event(y_ready[j])
+            y_host[j].copy_(y[j], non_blocking=True)
+            y_free[j].record(d2h_s)
 
     for i in range(W):
         step(i)
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     sync()
-    t0.record(L.stream)
+    t0.record(comp)
+    h2d_s.wait_event(t0)
+    d2h_s.wait_event(t0)
     for i in range(K):
         step(W + i)
-    t1.record(L.stream)
+    done = torch.cuda.Event()
+    done.record(d2h_s)
+    comp.wait_event(done)
+    t1.record(comp)
     sync()
     h2d = sum(v.numel() * v.element_size() for v in toks_host[0].values())
-    return t0.elapsed_time(t1), h2d, y.numel() * y.element_size()
+    return t0.elapsed_time(t1), h2d, y[0].numel() * y[0].element_size()
 
 
 # ------------------------------------------------------------------ CPU oracle legs
@@ -434,6 +578,8 @@ def main():
     ap.add_argument("--no-spec", action="store_true", help="skip the speculative-verify leg")
     ap.add_argument("--no-gdn", action="store_true", help="skip the Gated DeltaNet leg")
     ap.add_argument("--no-kda", action="store_true", help="skip the Kimi Delta Attention leg")
+    ap.add_argument("--no-hybrid", action="store_true", help="skip the synthetic hybrid-step leg")
+    ap.add_argument("--no-prefill", action="store_true", help="skip the prefill leg")
     ap.add_argument("--batch", type=int, default=WL.batch,
                     help="sequences per GPU (default: the workload's 256; smaller for profiling)")
     args = ap.parse_args()
@@ -487,41 +633,50 @@ def main():
     L = make_layer(wl, "replay", "bf16", consts, device)
     sampler = ClockSampler(local)
     with sampler:
-        total_ms, per, prep_ms, read_ms, launches = timed_loop(L, toks_dev, ys, K, W, sync)
-    # calls of the per-kernel pass are W + K + i since the import: a call folds at len = window
-    fold = [(W + K + i) >= wl.window and (W + K + i) % wl.window == 0 for i in range(K)]
+        total_ms, per, flush_ms, read_ms, launches, steady = timed_loop(L, toks_dev, ys, K, W, sync)
+    # calls of the per-kernel pass are W + K + M*window + i since the import: a call folds at len = window
+    c0 = W + K + steady[1]
+    fold = [(c0 + i) >= wl.window and (c0 + i) % wl.window == 0 for i in range(K)]
     pick = lambda xs, want: [x for x, f in zip(xs, fold) if f == want]
     clocks = sampler.summary()
-    total_ms, kern_ms, prep_avg = max_over_ranks(dist, [total_ms, float(np.mean(read_ms)), float(np.mean(prep_ms))],
-                                                 device)
+    total_ms, kern_ms, steady_ms = max_over_ranks(dist, [total_ms, float(np.mean(read_ms)), steady[0]], device)
     assert L.status()[0] == 0, "device error during the benchmark"
 
-    # e2e through the public API with host buffers (fresh layer, same workload)
+    # e2e through the public API with host buffers (same layer, state re-imported)
     L.import_state(torch.from_numpy(consts["S0"]).to(device))
     e2e_ms, h2d, d2h = e2e_loop(L, toks_host, K, W, sync)
     (e2e_ms,) = max_over_ranks(dist, [e2e_ms], device)
+    assert L.status()[0] == 0, "device error in the end-to-end loop"
 
     shape = traffic.Shape("mamba2", wl.headdim, wl.dstate, wl.nheads // wl.ngroups, wl.window, "bf16",
                           wl.input_dtype)
     rep = traffic.replay_decode_per_token(shape)
     win = traffic.replay_decode_window(shape)
     units = wl.batch * wl.nheads
-    bytes_per_launch = traffic.total(win["read"]) * units       # replay-read kernel, mean per call
-    prep_bytes = traffic.total(win["prep"]) * units             # prep/flush kernel, mean per call
+    bytes_per_launch = traffic.total(win["read"]) * units       # replay-read kernel, window mean per call
+    sp_fold = traffic.replay_step_split(shape, wl.window, True)
+    fold_bytes = traffic.total(sp_fold["prep"]) * units          # prep + flush kernels of a folding call
+    prep_bytes = traffic.total(traffic.replay_step_split(shape, wl.window // 2, False)["prep"]) * units
     achieved = bytes_per_launch / (kern_ms * 1e-3) / 1e9
     peak, peak_kind = measured_peak()
-    tr = None
+    tr, tr_note = None, "no ncu capture of the current kernel"
     if os.path.exists(PROFILE_TRAFFIC):
         p = json.load(open(PROFILE_TRAFFIC))
         if p.get("kernel_hash") == kernel_source_hash():
-            tr = p.get("dram_bytes_per_launch")
+            # measured DRAM bytes per launch over its own launches, put on the
+            # window-mean basis of `achieved` by the algorithmic bytes of both
+            tr = p["dram_bytes_per_launch"] * bytes_per_launch / p["algorithmic_bytes_same_launches"]
+            tr_note = (f"ncu dram bytes {p['dram_bytes_per_launch']:.4g} per launch over launches with "
+                       f"{p['algorithmic_bytes_same_launches']:.4g} algorithmic bytes, scaled to the window mean")
+    fold_call_ms = float(np.mean(pick(flush_ms, True))) if any(fold) else None
+    prep_call_ms = float(np.mean(pick(flush_ms, False)))
 
     eager = None
     if not args.no_eager:
         del L
         torch.cuda.empty_cache()
         E = make_layer(wl, "eager", "f32", consts, device)
-        e_total, _, _, _, _ = timed_loop(E, toks_dev, ys, K, W, sync, split=False)
+        e_total, _, _, _, _, _ = timed_loop(E, toks_dev, ys, K, W, sync, split=False)
         (e_total,) = max_over_ranks(dist, [e_total], device)
         e_kern = e_total / K  # one kernel per eager call
         eg = traffic.eager_decode_per_token(shape, "f32")
@@ -534,6 +689,8 @@ def main():
     spec = None if args.no_spec else spec_leg(rank, device, sync, dist, world, min(K, 64), W)
     gdn = None if args.no_gdn else delta_leg(I.GDN, rank, device, sync, dist, world, min(K, 128), W)
     kda = None if args.no_kda else delta_leg(I.KDA, rank, device, sync, dist, world, min(K, 128), W)
+    hybrid = None if args.no_hybrid else hybrid_leg(device, sync, dist, world, min(K, 64), W)
+    pre = None if args.no_prefill else prefill_leg(device, sync, dist, world, 5, 3)
 
     state_rep, state_eag = traffic.state_bytes(rep), traffic.state_bytes(
         traffic.eager_decode_per_token(shape, "f32"))
@@ -552,19 +709,24 @@ def main():
         "data": "synthetic",
         "config": workload_config(wl.batch) | {"parallelism": f"dp{world} (independent sequences)"},
         "hbm_gbs": achieved,
+        "steady_state": {"value": job_tokens_per_s(world, wl.batch, steady[1], steady_ms), "unit": "tokens/s",
+                         "ms_per_step": steady_ms / steady[1], "steps": steady[1],
+                         "note": "whole windows: every 16 consecutive calls hold exactly one folding call"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": tr, "peak_source": peak_kind,
+                     "frac": achieved / peak, "traffic": tr, "traffic_basis": tr_note, "peak_source": peak_kind,
                      "kernel": "replay_read_kernel<128, bf16, 1>",
                      "algorithmic_bytes_per_launch": bytes_per_launch,
                      "kernel_ms_per_launch": kern_ms,
                      "read_ms_nonfold_call": float(np.mean(pick(read_ms, False))),
                      "read_gbs_nonfold_call": traffic.total(traffic.replay_step_split(shape, wl.window // 2, False)["read"])
                                               * units / (np.mean(pick(read_ms, False)) * 1e-3) / 1e9},
-        "prep_kernel": {"kernel": "m2_prep_kernel<128, bf16, 1>", "ms_per_launch": prep_avg,
-                        "algorithmic_bytes_per_launch": prep_bytes,
-                        "gbs": prep_bytes / (prep_avg * 1e-3) / 1e9,
-                        "ms_nonfold_call": float(np.mean(pick(prep_ms, False))),
-                        "ms_fold_call": float(np.mean(pick(prep_ms, True))) if any(fold) else None},
+        "prep_kernel": {"kernel": "m2_prep_kernel<128, 1>", "ms_nonfold_call": prep_call_ms,
+                        "algorithmic_bytes_nonfold_call": prep_bytes},
+        "flush_kernel": {"kernel": "m2_fold_kernel<128, bf16, 1>",
+                         "ms_per_fold_call": fold_call_ms, "note": "prep + flush kernels of a folding call",
+                         "algorithmic_bytes_per_fold_call": fold_bytes,
+                         "gbs": fold_bytes / (fold_call_ms * 1e-3) / 1e9 if fold_call_ms else None,
+                         "frac": fold_bytes / (fold_call_ms * 1e-3) / 1e9 / peak if fold_call_ms else None},
         "ms_per_call": {"nonfold": float(np.mean(pick(per, False))),
                         "fold": float(np.mean(pick(per, True))) if any(fold) else None},
         "e2e": {"value": job_tokens_per_s(world, wl.batch, K, e2e_ms), "unit": "tokens/s",
@@ -577,12 +739,25 @@ def main():
         "spec_verify": spec,
         "gdn": gdn,
         "kda": kda,
+        "hybrid_step": hybrid,
+        "prefill": pre,
     }
     if rank == 0 and world == 1 and not args.no_cpu:
+        from oracle import eager as oracle_eager
+
         v, done, used, cores = oracle_tokens_per_s(wl, 64, 256, 12.0)
         line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                                 "sample": f"fp64 eager oracle on 64 of 256 sequences x 128 heads, "
                                           f"{done} steps, {used:.1f} s"}
+        all_threads = oracle_eager.max_threads()
+        oracle_eager.set_threads(1)
+        try:
+            v1, done1, used1, _ = oracle_tokens_per_s(wl, 8, 256, 6.0)
+        finally:
+            oracle_eager.set_threads(all_threads)
+        line["cpu_baseline_1core"] = {"value": v1, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                                      "sample": f"fp64 eager oracle, one thread, on 8 of 256 sequences x 128 "
+                                                f"heads, {done1} steps, {used1:.1f} s"}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if dist is not None:

@@ -16,7 +16,8 @@ size_t gdn_smem_bytes(const rssm_config &cf, int T) {
                                            cf.input_dtype == RSSM_BF16 ? 2 : 4);
 }
 
-cudaError_t gdn_launch(Ctx &h, int op, int T, const rssm_inputs *in, float *y, float *out, cudaStream_t st) {
+cudaError_t gdn_launch(Ctx &h, int op, int T, const rssm_inputs *in, float *y, float *out, cudaStream_t st,
+                       const Handoff *ho_in) {
     GArgs a{};
     const rssm_config &cf = h.cfg;
     a.B = cf.batch; a.H = cf.nheads; a.P = cf.headdim; a.W = cf.window;
@@ -57,7 +58,7 @@ cudaError_t gdn_launch(Ctx &h, int op, int T, const rssm_inputs *in, float *y, f
     // Replay decode/verify: the prep kernel (swept queries, coefficients,
     // appends), the fold-only kernel when some buffer may be too full for the
     // call's tokens, then the shared replay-read kernel.
-    const Handoff ho = h.handoff();
+    const Handoff ho = ho_in ? *ho_in : h.handoff();
     a.seqinfo = ho.seqinfo; a.dec = ho.dec; a.coef = ho.coef; a.query = ho.query;
     a.TQmax = ho.tq_max;
     a.Emax = (cf.window + a.TQmax + 3) & ~3;

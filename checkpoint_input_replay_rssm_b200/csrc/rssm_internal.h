@@ -13,7 +13,8 @@ namespace rssm {
 
 // The prep kernel's per-call hand-off to the flush and read kernels: per
 // sequence {entries replayed, ring slot of entry 0, folded, valid}, the flush
-// kernel's work list, and the replay decays and coefficients.
+// kernel's work list, the replay decays and coefficients, and (Gated DeltaNet,
+// KDA) the swept queries.
 struct Handoff {
     int4 *seqinfo;    // [B]
     int *fold_count;  // one int32, zero between calls
@@ -34,7 +35,7 @@ struct Ctx {
     int len_lb = 0, len_ub = 0; // bounds of every sequence's committed buffer length (host mirror)
     int64_t launches = 0;       // kernels enqueued so far
     int num_sms = 148;          // SMs of the handle's device
-    cudaEvent_t split_event = nullptr;  // recorded between prep and read kernels (measurement)
+    cudaEvent_t split_event = nullptr;  // recorded between prep/flush and read kernels (measurement)
     std::string err;
 
     void *at(size_t off) const { return ws + off; }
@@ -68,14 +69,14 @@ struct Ctx {
 };
 
 // Kernel launchers (one per layer kind).  op: Op; T tokens appended (0 for
-// flush/export); in/y used by decode/verify, out by export.  mamba2_launch
-// counts its launches and keeps the buffer-length bounds len_lb/len_ub.
+// flush/export); in/y used by decode/verify, out by export.  The launchers count
+// their launches and keep the buffer-length bounds len_lb/len_ub.
 // ho: where the replay decode/verify hand-off lives (nullptr: the workspace's).
 cudaError_t mamba2_launch(Ctx &h, int op, int T, const rssm_inputs *in, float *y, float *out,
                           cudaStream_t st, const Handoff *ho = nullptr);
 size_t mamba2_smem_bytes(const rssm_config &cf, int T);
 cudaError_t gdn_launch(Ctx &h, int op, int T, const rssm_inputs *in, float *y, float *out,
-                       cudaStream_t st);
+                       cudaStream_t st, const Handoff *ho = nullptr);
 
 // Bounds of every sequence's committed buffer length after a replay decode or
 // verify of T tokens (a verify's commit keeps 0..T of them): a sequence that

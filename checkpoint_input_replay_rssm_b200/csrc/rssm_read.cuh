@@ -89,7 +89,7 @@ __global__ void __launch_bounds__(kThreads, TQ == 1 ? 4 : 2) replay_read_kernel(
     constexpr int IB = BF ? 2 : 4;
     static_assert(CPL <= MAXC, "a lane's chunks of one row must fit a round");
 
-    extern __shared__ __align__(16) uint8_t smraw[];
+    extern __shared__ __align__(128) uint8_t smraw[];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int H = a.H, P = a.P, R = a.R, W = a.W, T = a.T, HC = a.HC;
     const int b = blockIdx.y;

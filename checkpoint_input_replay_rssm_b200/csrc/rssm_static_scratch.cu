@@ -1,27 +1,33 @@
 // rssm_static_scratch.cu -- rssm_decode_static_scratch: the replay decode with
-// its per-call hand-off (prep kernel -> flush and read kernels) kept in one
-// file-scope device array instead of the handle's workspace.
+// its per-call scratch kept in one file-scope device array instead of the
+// handle's workspace.
 //
-// Who needs it: a caller that budgets device memory per layer for the layer's
-// state alone and runs the layers' decodes one after another on one stream.
-// Each handle's workspace carries its own hand-off region (for a 256-sequence,
-// 128-head, window-16 layer about 2.7 MB), rewritten by every call and dead
-// between calls; such a caller wants the hand-off of every layer in one shared
-// array that the library owns and that needs no allocation, at run time or at
-// set-up: the array is part of the loaded module.
+// Who needs it: callers that cannot allocate device memory on the decode path --
+// an engine whose memory pool is fixed before the model is loaded, or a step
+// captured once and replayed, where a cudaMalloc would stall every stream of the
+// device or is not allowed at all -- and that give each layer memory for its
+// state only, decoding the layers one after another on one stream.  Every
+// replay decode passes a per-call hand-off from its prep kernel to its flush
+// and read kernels (per-sequence ring info, the flush work list, the replay
+// decays and coefficients, and for Gated DeltaNet / KDA the swept queries:
+// about 2.8 MB for a 256-sequence, 128-head Mamba-2 layer with window 16 and
+// 4.7 MB for a 256-sequence, 32-head, d_k 128 GDN layer), rewritten by every
+// call and dead between calls.  Here every layer shares one such array, part of
+// the loaded module: nothing is allocated, at run time or at set-up.
 //
 // The method itself (the pages on checkpointed input replay) has no such entry
 // point; it computes exactly what rssm_decode computes, with the same kernels.
 //
 // Limits and sharing:
-//   - the hand-off of one decode call must fit kStaticScratchBytes; larger
-//     layers are refused with RSSM_EINVAL before anything is enqueued;
-//   - all calls on a device share the array: calls whose kernels can overlap
-//     (several streams, several host threads) race on it and must not be
-//     issued concurrently;
+//   - the hand-off of one decode call must fit kStaticScratchBytes (8 MiB);
+//     larger layers are refused with RSSM_EINVAL before anything is enqueued;
+//   - all calls on a device share the array and each call leaves its contents
+//     behind: calls whose kernels can overlap (several streams, several host
+//     threads) race on it and must not be issued concurrently;
 //   - the first call on a device looks up the array's device address
-//     (cudaGetSymbolAddress) with that device current; a caller that records
-//     its calls into a stream capture makes one call before capturing.
+//     (cudaGetSymbolAddress) with that device current and keeps it for the life
+//     of the process: make that first call before any stream capture, and do not
+//     use the entry point again on a device after cudaDeviceReset.
 #include <mutex>
 #include <string>
 
@@ -29,7 +35,7 @@
 
 namespace {
 
-constexpr size_t kStaticScratchBytes = 4u << 20;  // 4 MiB
+constexpr size_t kStaticScratchBytes = 8u << 20;  // 8 MiB
 constexpr int kMaxDevices = 64;
 
 __device__ __align__(256) uint8_t g_handoff_scratch[kStaticScratchBytes];
@@ -39,19 +45,22 @@ void *g_addr[kMaxDevices] = {};
 
 size_t up256(size_t v) { return (v + 255) & ~(size_t)255; }
 
-// Offsets of the decode hand-off (one query per call) inside the array.
+// Offsets of one decode call's hand-off (one query per call) inside the array;
+// the swept queries only for the delta-rule layers.
 struct Carve {
-    size_t seqinfo, fold, dec, coef, total;
+    size_t seqinfo, fold, dec, coef, query, total;
 };
 Carve carve(const rssm_config &c) {
-    const size_t B = c.batch, H = c.nheads;
-    const size_t Emax = ((size_t)c.window + 1 + 3) & ~(size_t)3;
+    const size_t B = c.batch, H = c.nheads, N = c.dstate;
+    const size_t Emax = ((size_t)c.window + 1 + 3) & ~(size_t)3;  // window + 1 entries, padded to 4
     Carve k{};
     size_t o = 0;
     k.seqinfo = o; o = up256(o + B * 16);
     k.fold = o;    o = up256(o + 16 + B * 4);  // count, 3 pad words, list[B]
     k.dec = o;     o = up256(o + B * H * 4);
     k.coef = o;    o = up256(o + B * H * Emax * 4);
+    k.query = o;
+    if (c.kind != RSSM_MAMBA2) o = up256(o + B * H * N * 4);
     k.total = o;
     return k;
 }
@@ -80,8 +89,8 @@ extern "C" RSSM_API rssm_status rssm_decode_static_scratch(rssm_handle hh, const
     using namespace rssm;
     Ctx *h = (Ctx *)hh;
     if (!h) return RSSM_EINVAL;
-    if (h->cfg.mode != RSSM_REPLAY || h->cfg.kind != RSSM_MAMBA2)
-        return api_fail(h, RSSM_EINVAL, "decode_static_scratch: only REPLAY Mamba-2 layers have a hand-off");
+    if (h->cfg.mode != RSSM_REPLAY)
+        return api_fail(h, RSSM_EINVAL, "decode_static_scratch: only REPLAY layers have a per-call hand-off");
     if (h->pending) return api_fail(h, RSSM_ESTATE, "decode while a verify is pending (commit first)");
     if (!api_inputs_ok(h, in) || !y)
         return api_fail(h, RSSM_EINVAL,
@@ -91,7 +100,9 @@ extern "C" RSSM_API rssm_status rssm_decode_static_scratch(rssm_handle hh, const
         return api_fail(h, RSSM_EINVAL,
                         "decode_static_scratch: the hand-off needs " + std::to_string(k.total) +
                             " bytes; the static array holds " + std::to_string(kStaticScratchBytes) +
-                            " (batch * nheads * (window + 4) * 4 bytes must stay below it)");
+                            " (needed: batch * 20 + 16 + batch * nheads * 4 * (1 + round_up4(window + 1)) bytes,"
+                            " plus batch * nheads * dstate * 4 for a delta-rule layer, each region padded to 256"
+                            " bytes)");
     void *base = nullptr;
     cudaError_t e = scratch_address(&base);
     if (e != cudaSuccess) return api_cuda_fail(h, e, "decode_static_scratch: cudaGetSymbolAddress");
@@ -102,10 +113,13 @@ extern "C" RSSM_API rssm_status rssm_decode_static_scratch(rssm_handle hh, const
     ho.fold_list = ho.fold_count + 4;
     ho.dec = (float *)(p + k.dec);
     ho.coef = (float *)(p + k.coef);
+    ho.query = h->cfg.kind == RSSM_MAMBA2 ? nullptr : (float *)(p + k.query);
     ho.tq_max = 1;
     // The work-list length must start at zero; the read kernel leaves it zero,
     // but a call refused or failed half-way on another handle may not have.
     e = cudaMemsetAsync(ho.fold_count, 0, sizeof(int), h->stream);
-    if (e == cudaSuccess) e = mamba2_launch(*h, OP_DECODE, 1, in, y, nullptr, h->stream, &ho);
+    if (e == cudaSuccess)
+        e = h->cfg.kind == RSSM_MAMBA2 ? mamba2_launch(*h, OP_DECODE, 1, in, y, nullptr, h->stream, &ho)
+                                       : gdn_launch(*h, OP_DECODE, 1, in, y, nullptr, h->stream, &ho);
     return e == cudaSuccess ? RSSM_OK : api_cuda_fail(h, e, "decode_static_scratch launch");
 }

@@ -6,8 +6,12 @@ recurrence, unlike a single shared low-precision state whose rounding
 accumulates ("Deux precisions pour le prix d'une", irisproject.cloud).  This
 runs the fp32 checkpoint + per-row e4m3 read copy for W in {4, 8, 16, 32, 64}
 next to the eager single shared fp8 state on the same inputs, and records the
-per-step error against the fp64 oracle.  Eight sequences of 128 heads x 64 x 128
-are decoded (the float comparison subset; every sequence is independent).
+per-step error against the fp64 oracle.  The layers hold the workload's 256
+sequences of 128 heads x 64 x 128; eight of them (a fixed spread from first to
+last) follow their own seeded input streams for all 4096 steps and are compared
+with the oracle, the other 248 replay a cycle of the workload's first 16 seeded
+steps (sequences are independent: their inputs change no compared output, and
+their counters are checked against the ring model on the full batch).
 
 Set RSSM_REPORT_DIR to write the per-step error summary as JSON.
 """
@@ -20,6 +24,7 @@ import pytest
 from checkpoint_input_replay_rssm_b200 import inputs as I
 from oracle import eager
 from oracle.replay import ReplayOracle
+from oracle.ring import RingModel
 from tests.gpu_common import make_layer, oracle_params, rel_err, to_device
 
 pytestmark = pytest.mark.gpu
@@ -30,28 +35,38 @@ WINDOWS = (4, 8, 16, 32, 64)
 def test_fp8_dual_precision_drift_window_sweep():
     import torch
 
-    wl = I.FP8DRIFT.replace(batch=8)
+    wl = I.FP8DRIFT
     steps = wl.steps
-    c = I.constants(wl)
-    layers = {f"dual_fp8_W{W}": make_layer(wl.replace(window=W), "replay", "fp8")[0] for W in WINDOWS}
-    layers["dual_bf16_W16"] = make_layer(wl, "replay", "bf16")[0]
-    layers["replay_f32_W16"] = make_layer(wl, "replay", "f32")[0]
-    layers["shared_fp8"] = make_layer(wl, "eager", "fp8")[0]
-    layers["shared_bf16"] = make_layer(wl, "eager", "bf16")[0]
+    seqs = [0, 37, 74, 111, 148, 185, 222, 255]
+    full = I.constants(wl, f64=False)
+    layers = {f"dual_fp8_W{W}": make_layer(wl.replace(window=W), "replay", "fp8", consts=full)[0]
+              for W in WINDOWS}
+    layers["dual_bf16_W16"] = make_layer(wl, "replay", "bf16", consts=full)[0]
+    layers["replay_f32_W16"] = make_layer(wl, "replay", "f32", consts=full)[0]
+    layers["shared_fp8"] = make_layer(wl, "eager", "fp8", consts=full)[0]
+    layers["shared_bf16"] = make_layer(wl, "eager", "bf16", consts=full)[0]
+    del full
+    c = I.constants(wl, seqs)
     emu = ReplayOracle("mamba2", c["S0"], 16, params=oracle_params(c), ngroups=wl.ngroups,
                        read_dtype="fp8")
     S = np.ascontiguousarray(c["S0"].copy())
+    npool = 16
+    pool = [to_device(I.token(wl, t), wl, with_T=False) for t in range(npool)]
+    idx = torch.tensor(seqs, device="cuda")
     err = {n: np.zeros(steps) for n in layers}
     emu_worst = 0.0
     for t in range(steps):
-        tok = I.token(wl, t)
-        dev = to_device(tok, wl, with_T=False)
-        ys = {n: L.decode(dev) for n, L in layers.items()}
+        tok = I.token(wl, t, seqs)
+        sub = to_device(tok, wl, with_T=False)
+        dev = {k: v.clone() for k, v in pool[t % npool].items()}
+        for k in dev:
+            dev[k][idx] = sub[k]
+        ys = {n: L.decode(dev)[seqs, 0] for n, L in layers.items()}
         y_ref = eager.mamba2_step(S, c["A"], c["D"], tok["x"], tok["dt"], tok["B"], tok["C"])
         for n, y in ys.items():
-            err[n][t] = rel_err(y[:, 0].double().cpu().numpy(), y_ref)
+            err[n][t] = rel_err(y.double().cpu().numpy(), y_ref)
         if t < 96:
-            emu_worst = max(emu_worst, rel_err(ys["dual_fp8_W16"][:, 0].double().cpu().numpy(),
+            emu_worst = max(emu_worst, rel_err(ys["dual_fp8_W16"].double().cpu().numpy(),
                                                emu.decode(tok)))
     torch.cuda.synchronize()
 
@@ -59,10 +74,20 @@ def test_fp8_dual_precision_drift_window_sweep():
     # (6e-2: one code rounding the other way at a row's largest element, see test_gpu_mamba2)
     assert emu_worst <= 6e-2, emu_worst
     # rounding of the copy never feeds back: the checkpoint is the fp32 path's, byte for byte
-    ck = {n: layers[n].region("ckpt_off", "ckpt_bytes", torch.int32) for n in
-          ("dual_fp8_W16", "dual_bf16_W16", "replay_f32_W16")}
-    assert torch.equal(ck["dual_fp8_W16"], ck["replay_f32_W16"])
-    assert torch.equal(ck["dual_bf16_W16"], ck["replay_f32_W16"])
+    ckpt = {n: layers[n].region("ckpt_off", "ckpt_bytes", torch.int32) for n in
+            ("dual_fp8_W16", "dual_bf16_W16", "replay_f32_W16")}
+    assert torch.equal(ckpt["dual_fp8_W16"], ckpt["replay_f32_W16"])
+    assert torch.equal(ckpt["dual_bf16_W16"], ckpt["replay_f32_W16"])
+    # counters of the whole batch follow the ring model (a fold every W steps)
+    for W in WINDOWS:
+        rm = RingModel(wl.batch, W, 1)
+        for _ in range(steps):
+            rm.decode()
+        sp, ck, pe, fc = layers[f"dual_fp8_W{W}"].counters()
+        assert np.array_equal(sp, rm.seq_pos) and np.array_equal(ck, rm.ckpt_pos), W
+        assert np.array_equal(fc, rm.flush_count) and np.array_equal(pe, rm.pending), W
+    for L in layers.values():
+        assert L.status()[0] == 0
     # the fp32 path stays at fp32 rounding level for 4096 steps
     assert err["replay_f32_W16"].max() <= 1e-4
     assert err["dual_bf16_W16"].max() <= 2e-2
@@ -74,7 +99,8 @@ def test_fp8_dual_precision_drift_window_sweep():
         assert e.max() < 0.5, W
 
     report = {
-        "workload": "mamba2 fp8 drift: 8 seqs x 128 heads x 64 x 128, G 8, bf16 inputs, 4096 steps",
+        "workload": "mamba2 fp8 drift: 256 seqs x 128 heads x 64 x 128, G 8, bf16 inputs, 4096 steps; "
+                    "8 seqs compared",
         "metric": "per step max|y - y_fp64| / RMS(y_fp64)",
         "emulated_fp8_copy_vs_gpu_first96_max": emu_worst,
         "series": {n: {"median": float(np.median(e)), "p99": float(np.quantile(e, 0.99)),

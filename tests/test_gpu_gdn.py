@@ -89,9 +89,10 @@ def test_eager_baselines(sd):
 
 def test_gdn_layer_full_size_sampled():
     """Batch 256 x 32 heads x 128 x 128, W = 16, 256 steps, bf16 read copy and fp32
-    read path; sampled sequences against the fp64 oracle, every counter exact."""
+    read path; 16 sequences (first, last, both sides of the halfway and quarter
+    marks) at every step against the fp64 oracle, every counter exact."""
     wl = I.GDN
-    seqs = [0, 77, 255]
+    seqs = [0, 1, 2, 63, 64, 100, 127, 128, 129, 150, 191, 192, 200, 230, 254, 255]
     layers, worst, _, S = _run(wl, "replay", ["bf16", "f32"], wl.steps, seqs=seqs)
     assert worst["bf16"] <= TOL["bf16"], worst
     assert worst["f32"] <= TOL["f32"], worst

@@ -133,10 +133,11 @@ def test_flush_and_export_match_the_oracle():
 
 def test_kda_layer_full_size_sampled():
     """Batch 256 x 32 heads x 128 x 128, W = 16, bf16 read copy and fp32 read path,
-    48 steps (two folds); sampled sequences against the fp64 oracle, counters exact."""
+    256 steps (16 folds); 16 sequences (first, last, both sides of the halfway and
+    quarter marks) at every step against the fp64 oracle, counters exact."""
     wl = I.KDA
-    steps = 48
-    seqs = [0, 101, 255]
+    steps = wl.steps
+    seqs = [0, 1, 2, 63, 64, 100, 127, 128, 129, 150, 191, 192, 200, 230, 254, 255]
     layers, worst, _, S = _run(wl, "replay", ["bf16", "f32"], steps, seqs=seqs)
     assert worst["bf16"] <= TOL["bf16"], worst
     assert worst["f32"] <= TOL["f32"], worst

@@ -145,10 +145,11 @@ def test_dt_scaled_input_term():
 def test_nemotron_layer_full_size_sampled():
     """Batch 256 x 128 heads x 64 x 128 (4 MiB fp32 state per sequence), W = 16,
     256 steps, bf16 read copy and fp32 read path in the launch configuration the
-    benchmark times; outputs of sampled sequences against the fp64 oracle, counters
-    of every sequence against the ring model."""
+    benchmark times; outputs of 16 sequences (first, last, both sides of the
+    halfway and quarter marks) at every one of the 256 steps against the fp64
+    oracle, counters of every sequence against the ring model."""
     wl = I.NEMOTRON
-    seqs = [0, 101, 255]
+    seqs = [0, 1, 2, 63, 64, 100, 127, 128, 129, 150, 191, 192, 200, 230, 254, 255]
     layers, worst, _, S = _run_decode(wl, "replay", ["bf16", "f32"], wl.steps, seqs=seqs)
     assert worst["bf16"] <= TOL["bf16"], worst
     assert worst["f32"] <= TOL["f32"], worst

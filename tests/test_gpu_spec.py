@@ -67,10 +67,11 @@ def _spec_run(wl, rounds, seqs, layers_spec, tols):
 
 def test_spec_verify_mamba2_batch512_k4():
     """Nemotron-scale layer at batch 512, K = 4; replay (bf16 copy, fp32 path) and the
-    eager snapshot baseline.  48 rounds cover several flushes per sequence at W = 16."""
+    eager snapshot baseline, all 128 rounds of the workload (many folds per sequence
+    at W = 16); floats on 16 sequences, integers on all 512."""
     wl = I.SPECVERIFY
     seqs = list(range(3, 512, 32))  # 16 sequences
-    _spec_run(wl, 48, seqs,
+    _spec_run(wl, wl.steps, seqs,
               {"replay_bf16": ("replay", "bf16"), "replay_f32": ("replay", "f32"),
                "eager_f32": ("eager", "f32")},
               {"replay_bf16": 2e-2, "replay_f32": 1e-4, "eager_f32": 1e-4})
