@@ -206,13 +206,13 @@ def spec_leg(rank, device, sync, dist, world, rounds, warmup):
     return out
 
 
-def delta_leg(wl0, rank, device, sync, dist, world, steps, warmup):
+def delta_leg(wl0, rank, device, sync, dist, world, steps, warmup, batch=None):
     """Gated DeltaNet or Kimi Delta Attention decode, 256 sequences x 32 heads x 128 x 128,
     W = 16: replay (bf16 copy) and eager (fp32) tokens/s, with the state bytes per token
     of each."""
     import torch
 
-    wl = wl0.replace(seed=wl0.seed + 7919 * rank)
+    wl = wl0.replace(seed=wl0.seed + 7919 * rank, batch=batch or wl0.batch)
     consts = I.constants(wl, f64=False)
     n = min(steps + warmup, 32)
     toks = [device_tokens(wl, I.token(wl, t), device, False) for t in range(n)]
@@ -304,7 +304,7 @@ def hybrid_leg(device, sync, dist, world, steps, warmup):
     return out
 
 
-def prefill_leg(device, sync, dist, world, reps, warmup):
+def prefill_leg(device, sync, dist, world, reps, warmup, batch=None):
     """Prompt prefill of the Nemotron-scale layer on the tensor cores: 256 sequences x
     128 heads, 512-token prompts, seeded device-generated inputs of the decode
     workload's distributions; prompt tokens/s and the roofline of the kernel."""
@@ -312,7 +312,7 @@ def prefill_leg(device, sync, dist, world, reps, warmup):
 
     from checkpoint_input_replay_rssm_b200 import rssm
 
-    wl = I.PREFILL
+    wl = I.PREFILL.replace(batch=batch or I.PREFILL.batch)
     Bn, T, H, G, P, N = wl.batch, wl.steps, wl.nheads, wl.ngroups, wl.headdim, wl.dstate
     g = torch.Generator(device=device).manual_seed(wl.seed)
     x = torch.randn((Bn, T, H, P), generator=g, device=device).to(torch.bfloat16)
@@ -581,7 +581,8 @@ def main():
     ap.add_argument("--no-hybrid", action="store_true", help="skip the synthetic hybrid-step leg")
     ap.add_argument("--no-prefill", action="store_true", help="skip the prefill leg")
     ap.add_argument("--batch", type=int, default=WL.batch,
-                    help="sequences per GPU (default: the workload's 256; smaller for profiling)")
+                    help="sequences per GPU (default: the workload's 256; smaller for profiling; applies to "
+                         "the decode, GDN, KDA and prefill legs)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -687,10 +688,11 @@ def main():
         del E
 
     spec = None if args.no_spec else spec_leg(rank, device, sync, dist, world, min(K, 64), W)
-    gdn = None if args.no_gdn else delta_leg(I.GDN, rank, device, sync, dist, world, min(K, 128), W)
-    kda = None if args.no_kda else delta_leg(I.KDA, rank, device, sync, dist, world, min(K, 128), W)
+    small = args.batch if args.batch != WL.batch else None  # a smaller batch for profiling applies to every leg
+    gdn = None if args.no_gdn else delta_leg(I.GDN, rank, device, sync, dist, world, min(K, 128), W, small)
+    kda = None if args.no_kda else delta_leg(I.KDA, rank, device, sync, dist, world, min(K, 128), W, small)
     hybrid = None if args.no_hybrid else hybrid_leg(device, sync, dist, world, min(K, 64), W)
-    pre = None if args.no_prefill else prefill_leg(device, sync, dist, world, 5, 3)
+    pre = None if args.no_prefill else prefill_leg(device, sync, dist, world, 5, 3, small)
 
     state_rep, state_eag = traffic.state_bytes(rep), traffic.state_bytes(
         traffic.eager_decode_per_token(shape, "f32"))

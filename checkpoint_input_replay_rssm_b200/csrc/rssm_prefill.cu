@@ -22,10 +22,13 @@
 // two MMAs each, so every product keeps near-fp32 accuracy.  The state stays
 // in tensor memory, transposed (lane n, column p), across the chunks of a head.
 //
-// One CTA of 128 threads per (sequence, head); thread i owns tensor-memory lane i
-// (token i of the chunk, or state column n).  Per chunk: (A) the threads stage
-// the chunk's C, B, B^T, x^T and (x w)^T and the state's (hi, lo) copy in shared
-// memory and rescale the state by e^{Lam_last} in place; (B) one thread issues
+// One CTA of 256 threads per (sequence, head): thread t owns tensor-memory lane
+// t mod 128 (token i of the chunk, or state column n) and half of that row's
+// columns, so two warps share each lane quarter.  Per chunk: (A) the threads issue
+// the chunk's global reads at once (C and B rows by cp.async into their
+// swizzled rows, x into registers), then stage x^T and (x w)^T, the state's
+// (hi, lo) copy and B^T in shared memory and rescale the state by e^{Lam_last}
+// in place; (B) one thread issues
 // MMA1, MMA3 and MMA4; (C) the threads turn CB into M (hi, lo) in the space B
 // and B^T occupied; (D) one thread issues MMA2; (E) the threads write y.  Waits
 // on MMA completion are bounded (2 s) and report RSSM_DEV_PIPE_TIMEOUT.
@@ -40,7 +43,7 @@ namespace {
 
 constexpr int kQ = 128;          // chunk length = MMA M
 constexpr int kN = 128;          // dstate = MMA M of the state update
-constexpr int kPT = 128;         // threads per CTA
+constexpr int kPT = 256;         // threads per CTA: two halves of 128, one lane (row) each
 constexpr int kTileQN = kQ * kN * 2;  // one [128 x 128] bf16 tile
 
 struct PrefillArgs {
@@ -95,13 +98,16 @@ __device__ __forceinline__ uint32_t pack2(float a, float b) {
     return *reinterpret_cast<uint32_t *>(&t);
 }
 
+template <int P>
 __global__ void __launch_bounds__(kPT, 1) m2_prefill_kernel(const PrefillArgs a) {
+    constexpr int PH = P / 2;  // p columns handled by each half of the CTA (a multiple of 16)
     extern __shared__ __align__(1024) uint8_t psm[];
     // the swizzled tiles need a 1024-byte aligned base
     uint8_t *sm = psm + ((1024 - (smem_u32(psm) & 1023)) & 1023);
-    const int P = a.P;
     const PrefillLay Ly = prefill_lay(P);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int row = tid & (kQ - 1);  // tensor-memory lane: token i of the chunk, or state column n
+    const int half = tid >> 7;       // which half of the columns this thread works on
     const int b = blockIdx.y, h = blockIdx.x;
     const int H = a.H, G = a.G, T = a.T;
     const int g = h / (H / G);
@@ -126,16 +132,17 @@ __global__ void __launch_bounds__(kPT, 1) m2_prefill_kernel(const PrefillArgs a)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tslot;
-    const uint32_t lane_base = tmem + ((uint32_t)(32 * warp) << 16);  // this warp's 32 lanes
+    const uint32_t lane_base = tmem + ((uint32_t)(32 * (warp & 3)) << 16);  // this warp's 32 lanes
     const float Ah = a.A[h], Dh = a.D[h];
+    const int p_lo = half * PH;  // this thread's p columns: [p_lo, p_lo + PH)
+    const int64_t head = (int64_t)b * H + h;
 
     // The initial state, transposed into tensor memory: lane n holds S0[:, n].
-    for (int p0 = 0; p0 < P; p0 += 32) {
-        float v[32];
+    for (int j0 = 0; j0 < PH; j0 += 16) {
+        float v[16];
 #pragma unroll
-        for (int j = 0; j < 32; ++j)
-            v[j] = a.S0 ? a.S0[(((int64_t)b * H + h) * P + p0 + j) * kN + tid] : 0.f;
-        tmem_st32(lane_base + cS + p0, v);
+        for (int j = 0; j < 16; ++j) v[j] = a.S0 ? a.S0[(head * P + p_lo + j0 + j) * kN + row] : 0.f;
+        tmem_st16(lane_base + cS + p_lo + j0, v);
     }
 
     uint32_t phase = 0;
@@ -143,49 +150,62 @@ __global__ void __launch_bounds__(kPT, 1) m2_prefill_kernel(const PrefillArgs a)
     const int nchunks = (T + kQ - 1) / kQ;
     for (int c = 0; c < nchunks && !failed; ++c) {
         const int t0 = c * kQ, Lc = min(kQ, T - t0);
-        const int i = tid;  // token of the chunk owned by this thread
+        const int i = row;  // token of the chunk owned by this thread
         const bool live = i < Lc;
         const int64_t tok = (int64_t)b * T + t0 + i;
 
-        // (A) Prefix sums of dt*A over the chunk (padding tokens add nothing).
+        // (A) The chunk's global reads, all issued first: this half's 16-byte chunks
+        //     of the C and B rows of token i by cp.async straight into their K-major
+        //     rows (rows = tokens), this half's part of x row i and dt_i into registers.
+        const uint8_t *Crow = reinterpret_cast<const uint8_t *>(a.Cm + (tok * G + g) * kN);
+        const uint8_t *Brow = reinterpret_cast<const uint8_t *>(a.Bm + (tok * G + g) * kN);
+        constexpr int CH = kN / 16;  // row chunks per half
+#pragma unroll
+        for (int k = 0; k < CH; ++k) {
+            const int ch = half * CH + k;
+            if (live) {
+                cp_async16(sC + sw128_chunk(i, ch, kQ), Crow + 16 * ch);
+                cp_async16(sBk + sw128_chunk(i, ch, kQ), Brow + 16 * ch);
+            } else {
+                *reinterpret_cast<uint4 *>(sC + sw128_chunk(i, ch, kQ)) = make_uint4(0, 0, 0, 0);
+                *reinterpret_cast<uint4 *>(sBk + sw128_chunk(i, ch, kQ)) = make_uint4(0, 0, 0, 0);
+            }
+        }
+        cp_async_commit();
+        uint4 xv[PH / 8];
+        const uint4 *Xrow = reinterpret_cast<const uint4 *>(a.x + (tok * H + h) * P + p_lo);
+#pragma unroll
+        for (int k = 0; k < PH / 8; ++k) xv[k] = live ? Xrow[k] : make_uint4(0, 0, 0, 0);
         const float dti = live ? a.dt[tok * H + h] : 0.f;
+
+        // Prefix sums of dt*A over the chunk (padding tokens add nothing); both
+        // halves scan, the first publishes.
         float v = dti * Ah;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const float u = __shfl_up_sync(0xffffffffu, v, o);
             if (lane >= o) v += u;
         }
-        if (lane == 31) sred[warp] = v;
+        if (half == 0 && lane == 31) sred[warp] = v;
         __syncthreads();
         float carry = 0.f;
-        for (int w2 = 0; w2 < warp; ++w2) carry += sred[w2];
+        for (int w2 = 0; w2 < (warp & 3); ++w2) carry += sred[w2];
         const float lam = v + carry;
-        slam[i] = lam;
-        sw[i] = live ? (a.dt_scales ? dti : 1.f) : 0.f;
+        if (half == 0) {
+            slam[i] = lam;
+            sw[i] = live ? (a.dt_scales ? dti : 1.f) : 0.f;
+        }
         __syncthreads();
         const float lam_last = slam[kQ - 1];
 
-        // C and B rows of token i (K-major rows = tokens), B^T and x^T columns.
-        const uint4 *Crow = reinterpret_cast<const uint4 *>(a.Cm + (tok * G + g) * kN);
-        const uint4 *Brow = reinterpret_cast<const uint4 *>(a.Bm + (tok * G + g) * kN);
-        for (int ch = 0; ch < kN / 8; ++ch) {
-            const uint4 cv = live ? Crow[ch] : make_uint4(0, 0, 0, 0);
-            const uint4 bv = live ? Brow[ch] : make_uint4(0, 0, 0, 0);
-            *reinterpret_cast<uint4 *>(sC + sw128_chunk(i, ch, kQ)) = cv;
-            *reinterpret_cast<uint4 *>(sBk + sw128_chunk(i, ch, kQ)) = bv;
-            const __nv_bfloat16 *be = reinterpret_cast<const __nv_bfloat16 *>(&bv);
-#pragma unroll
-            for (int e = 0; e < 8; ++e)
-                *reinterpret_cast<__nv_bfloat16 *>(sBt + sw128_off(8 * ch + e, i, kN)) = be[e];
-        }
+        // x^T and (x w)^T columns of this half's p (w_i = e^{Lam_last - Lam_i} s_i), as (hi, lo).
         const float wi = live ? expf(lam_last - lam) * sw[i] : 0.f;
-        const uint4 *Xrow = reinterpret_cast<const uint4 *>(a.x + (tok * H + h) * P);
-        for (int ch = 0; ch < P / 8; ++ch) {
-            const uint4 xv = live ? Xrow[ch] : make_uint4(0, 0, 0, 0);
-            const __nv_bfloat16 *xe = reinterpret_cast<const __nv_bfloat16 *>(&xv);
+#pragma unroll
+        for (int k = 0; k < PH / 8; ++k) {
+            const __nv_bfloat16 *xe = reinterpret_cast<const __nv_bfloat16 *>(&xv[k]);
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
-                const int p = 8 * ch + e;
+                const int p = p_lo + 8 * k + e;
                 *reinterpret_cast<__nv_bfloat16 *>(sXt + sw128_off(p, i, P)) = xe[e];
                 __nv_bfloat16 hi, lo;
                 split_bf16(__bfloat162float(xe[e]) * wi, hi, lo);
@@ -196,18 +216,29 @@ __global__ void __launch_bounds__(kPT, 1) m2_prefill_kernel(const PrefillArgs a)
         // The state at the chunk's start: (hi, lo) copy for MMA3 (S rows p, K = n),
         // and e^{Lam_last} S back into tensor memory for MMA4 to accumulate onto.
         const float dec = expf(lam_last);
-        for (int p0 = 0; p0 < P; p0 += 32) {
-            float s[32];
-            tmem_ld32(lane_base + cS + p0, s);
+        for (int j0 = 0; j0 < PH; j0 += 16) {
+            float st[16];
+            tmem_ld16(lane_base + cS + p_lo + j0, st);
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
+            for (int j = 0; j < 16; ++j) {
                 __nv_bfloat16 hi, lo;
-                split_bf16(s[j], hi, lo);
-                *reinterpret_cast<__nv_bfloat16 *>(sSHi + sw128_off(p0 + j, tid, P)) = hi;
-                *reinterpret_cast<__nv_bfloat16 *>(sSLo + sw128_off(p0 + j, tid, P)) = lo;
-                s[j] *= dec;
+                split_bf16(st[j], hi, lo);
+                *reinterpret_cast<__nv_bfloat16 *>(sSHi + sw128_off(p_lo + j0 + j, row, P)) = hi;
+                *reinterpret_cast<__nv_bfloat16 *>(sSLo + sw128_off(p_lo + j0 + j, row, P)) = lo;
+                st[j] *= dec;
             }
-            tmem_st32(lane_base + cS + p0, s);
+            tmem_st16(lane_base + cS + p_lo + j0, st);
+        }
+        // B^T columns from this thread's own B chunks once they have landed.
+        cp_async_wait_all();
+#pragma unroll
+        for (int k = 0; k < CH; ++k) {
+            const int ch = half * CH + k;
+            const uint4 bv = *reinterpret_cast<const uint4 *>(sBk + sw128_chunk(i, ch, kQ));
+            const __nv_bfloat16 *be = reinterpret_cast<const __nv_bfloat16 *>(&bv);
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+                *reinterpret_cast<__nv_bfloat16 *>(sBt + sw128_off(8 * ch + e, i, kN)) = be[e];
         }
         fence_async_smem();
         tc_fence_before();
@@ -241,8 +272,8 @@ __global__ void __launch_bounds__(kPT, 1) m2_prefill_kernel(const PrefillArgs a)
         }
         tc_fence_after();
 
-        // (C) M = tril(e^{Lam_i - Lam_j}) (.) CB (.) s_j as (hi, lo), row i per thread.
-        for (int j0 = 0; j0 < kQ; j0 += 32) {
+        // (C) M = tril(e^{Lam_i - Lam_j}) (.) CB (.) s_j as (hi, lo): row i, this half's 64 columns j.
+        for (int j0 = half * 64; j0 < half * 64 + 64; j0 += 32) {
             float cb[32];
             tmem_ld32(lane_base + cY1 + j0, cb);
 #pragma unroll
@@ -292,22 +323,23 @@ __global__ void __launch_bounds__(kPT, 1) m2_prefill_kernel(const PrefillArgs a)
         }
         tc_fence_after();
 
-        // (E) y_i = Y_intra + e^{Lam_i} Y_inter + D x_i.
+        // (E) y_i = Y_intra + e^{Lam_i} Y_inter + D x_i over this half's p.
         const float di = expf(lam);
-        for (int p0 = 0; p0 < P; p0 += 32) {
-            float y1[32], y2[32];
-            tmem_ld32(lane_base + cY1 + p0, y1);
-            tmem_ld32(lane_base + cY2 + p0, y2);
+        for (int j0 = 0; j0 < PH; j0 += 16) {
+            float y1[16], y2[16];
+            tmem_ld16(lane_base + cY1 + p_lo + j0, y1);
+            tmem_ld16(lane_base + cY2 + p_lo + j0, y2);
             if (live) {
-                const __nv_bfloat16 *xr = a.x + (tok * H + h) * P + p0;
-                float4 *yr = reinterpret_cast<float4 *>(a.y + (tok * H + h) * P + p0);
+                float4 *yr = reinterpret_cast<float4 *>(a.y + (tok * H + h) * P + p_lo + j0);
 #pragma unroll
-                for (int j4 = 0; j4 < 8; ++j4) {
+                for (int j4 = 0; j4 < 4; ++j4) {
                     float o[4];
 #pragma unroll
                     for (int u = 0; u < 4; ++u) {
                         const int j = 4 * j4 + u;
-                        o[u] = fmaf(di, y2[j], y1[j]) + Dh * __bfloat162float(xr[j]);
+                        const uint4 &xw = xv[(j0 + j) >> 3];
+                        const __nv_bfloat16 *xe = reinterpret_cast<const __nv_bfloat16 *>(&xw);
+                        o[u] = fmaf(di, y2[j], y1[j]) + Dh * __bfloat162float(xe[(j0 + j) & 7]);
                     }
                     yr[j4] = make_float4(o[0], o[1], o[2], o[3]);
                 }
@@ -322,11 +354,11 @@ __global__ void __launch_bounds__(kPT, 1) m2_prefill_kernel(const PrefillArgs a)
         if (tid == 0) report_err(a.err, DEV_PIPE_TIMEOUT, b, h, 0);
     } else {
         // The state after the prompt, S_out[b][h][p][n] from lane n.
-        for (int p0 = 0; p0 < P; p0 += 32) {
-            float s[32];
-            tmem_ld32(lane_base + cS + p0, s);
+        for (int j0 = 0; j0 < PH; j0 += 16) {
+            float st[16];
+            tmem_ld16(lane_base + cS + p_lo + j0, st);
 #pragma unroll
-            for (int j = 0; j < 32; ++j) a.S_out[(((int64_t)b * H + h) * P + p0 + j) * kN + tid] = s[j];
+            for (int j = 0; j < 16; ++j) a.S_out[(head * P + p_lo + j0 + j) * kN + row] = st[j];
         }
     }
     tc_fence_before();
@@ -359,8 +391,9 @@ extern "C" RSSM_API rssm_status rssm_mamba2_prefill(const rssm_prefill_config *c
     a.Bm = (const __nv_bfloat16 *)in->Bm; a.Cm = (const __nv_bfloat16 *)in->Cm;
     a.A = A; a.D = D; a.S0 = S0; a.y = y; a.S_out = S_out; a.err = (int *)dev_error;
     const size_t smem = prefill_smem_bytes(c.headdim);
-    cudaError_t e = cudaFuncSetAttribute(m2_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    auto k = c.headdim == 32 ? m2_prefill_kernel<32> : (c.headdim == 64 ? m2_prefill_kernel<64> : m2_prefill_kernel<96>);
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return RSSM_ECUDA;
-    m2_prefill_kernel<<<dim3(c.nheads, c.batch), kPT, smem, (cudaStream_t)stream>>>(a);
+    k<<<dim3(c.nheads, c.batch), kPT, smem, (cudaStream_t)stream>>>(a);
     return cudaGetLastError() == cudaSuccess ? RSSM_OK : RSSM_ECUDA;
 }
