@@ -49,6 +49,12 @@ struct GArgs {
     int kda;                    // Kimi Delta Attention: alpha is a gate per key channel
 };
 
+// The fold of a decode call on the tensor cores (rssm_gdn_fold_tc.cu): used in
+// place of the fold-only launch of gdn_replay_kernel when d_k = d_v = 128,
+// T = 1 and W <= 32.
+bool gdn_fold_tc_eligible(const GArgs &a, int P, int N);
+cudaError_t gdn_fold_tc(const GArgs &a, int rk, cudaStream_t st);
+
 __host__ __device__ constexpr int gpad4(int n) { return (n + 3) & ~3; }
 
 // KDA keeps a gate row [E][N] where GDN keeps one gate per entry.  After the
@@ -728,12 +734,16 @@ __global__ void __launch_bounds__(kThreads) gdn_eager_kernel(const GArgs a) {
     void *state = (SK == SK_F32) ? (void *)a.ckpt : a.rc;
     const int64_t state_elems = (int64_t)a.B * H * P * N;
 
-    if (tid == 0) {
-        SeqState st = read_counters(a.c, b, W);
-        if (a.op == OP_DECODE)
-            arrive_and_publish(a.c, b, H, st.seq + 1, st.seq + 1, -1, 0);
-        else
-            arrive_and_publish(a.c, b, H, -1, -1, T, 0);
+    // No other CTA of an eager launch reads the counters, so the sequence's first
+    // head's CTA rewrites them alone (no arrival count, no fence).
+    if (tid == 0 && h == 0) {
+        if (a.op == OP_DECODE) {
+            const int64_t s1 = a.c.seq_pos[b] + 1;
+            a.c.seq_pos[b] = s1;
+            a.c.ckpt_pos[b] = s1;
+        } else {
+            a.c.pending[b] = T;
+        }
     }
     gdn_stage_new(a, s, b, h, N, tid);
     __syncthreads();
