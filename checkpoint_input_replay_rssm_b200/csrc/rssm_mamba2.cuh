@@ -722,7 +722,7 @@ __global__ void __launch_bounds__(kThreads, 3) m2_fold_kernel(const M2Args a, co
 // (blog.thibaultmonteiro.fr, "La fiche qu'on reecrit a chaque token").
 // ---------------------------------------------------------------------------
 template <int N, int SK, int TQ>
-__global__ void __launch_bounds__(kThreads) m2_eager_kernel(const M2Args a) {
+__global__ void __launch_bounds__(kThreads, (TQ == 1 && SK != SK_FP8) ? 4 : 1) m2_eager_kernel(const M2Args a) {
     constexpr int TPR4 = N / 4;
     constexpr int RPP4 = kThreads / TPR4;
     constexpr int RB = 8;
@@ -742,12 +742,28 @@ __global__ void __launch_bounds__(kThreads) m2_eager_kernel(const M2Args a) {
     void *state = (SK == SK_F32) ? (void *)a.ckpt : a.rc;
     const int64_t state_elems = (int64_t)a.B * H * P * N;
 
-    if (tid == 0) {
-        SeqState st = read_counters(a.c, b, a.W);
-        if (a.op == OP_DECODE)
-            arrive_and_publish(a.c, b, H, st.seq + 1, st.seq + 1, -1, 0);
-        else
-            arrive_and_publish(a.c, b, H, -1, -1, T, 0);
+    // The first batch of state rows is requested before the inputs are staged,
+    // so the tile's HBM latency overlaps the prologue.
+    const int c4 = tid % TPR4, q0 = tid / TPR4;
+    float4 st[RB];
+    float scl[RB];
+#pragma unroll
+    for (int k = 0; k < RB; ++k) {
+        const int r = q0 + k * RPP4;
+        st[k] = (r < P) ? load_quad<SK>(state, tile0 + (int64_t)r * N + 4 * c4) : make_float4(0.f, 0.f, 0.f, 0.f);
+        scl[k] = (SK == SK_FP8 && r < P) ? __ldg(a.rc_scale + (int64_t)bh * P + r) : 1.f;
+    }
+
+    // No other CTA of an eager launch reads the counters, so the sequence's first
+    // head's CTA rewrites them alone (no arrival count, no fence).
+    if (tid == 0 && h == 0) {
+        if (a.op == OP_DECODE) {
+            const int64_t s1 = a.c.seq_pos[b] + 1;
+            a.c.seq_pos[b] = s1;
+            a.c.ckpt_pos[b] = s1;
+        } else {
+            a.c.pending[b] = T;
+        }
     }
     for (int i = tid; i < T * P; i += kThreads) {
         const int m = i / P, p = i - m * P;
@@ -766,16 +782,15 @@ __global__ void __launch_bounds__(kThreads) m2_eager_kernel(const M2Args a) {
     }
     __syncthreads();
 
-    const int c4 = tid % TPR4, q0 = tid / TPR4;
     for (int rb = 0; rb < P; rb += RB * RPP4) {
-        float4 st[RB];
-        float scl[RB];
+        if (rb > 0) {
 #pragma unroll
-        for (int k = 0; k < RB; ++k) {
-            const int r = rb + q0 + k * RPP4;
-            st[k] = (r < P) ? load_quad<SK>(state, tile0 + (int64_t)r * N + 4 * c4)
-                            : make_float4(0.f, 0.f, 0.f, 0.f);
-            scl[k] = (SK == SK_FP8 && r < P) ? __ldg(a.rc_scale + (int64_t)bh * P + r) : 1.f;
+            for (int k = 0; k < RB; ++k) {
+                const int r = rb + q0 + k * RPP4;
+                st[k] = (r < P) ? load_quad<SK>(state, tile0 + (int64_t)r * N + 4 * c4)
+                                : make_float4(0.f, 0.f, 0.f, 0.f);
+                scl[k] = (SK == SK_FP8 && r < P) ? __ldg(a.rc_scale + (int64_t)bh * P + r) : 1.f;
+            }
         }
 #pragma unroll
         for (int k = 0; k < RB; ++k) {
