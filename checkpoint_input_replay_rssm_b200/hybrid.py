@@ -7,9 +7,11 @@ kernel alone (irisproject.cloud, "Des chiffres").  This stand-in builds such a
 stack with random weights (there is no trained model here): each block is
 ``ssm_per_block`` Mamba-2 layers decoded by librssm (replay or the eager
 baseline) and one attention layer.  Every layer projects the hidden state in
-and out with plain bf16 GEMMs (torch.matmul); the attention layer appends the
-token's key and value to a bf16 cache and attends over it with
-torch.nn.functional.scaled_dot_product_attention (grouped-query).  The Mamba-2
+and out with plain bf16 GEMMs (torch.matmul) after an RMS normalisation of its
+input (pre-norm residual blocks, as in the hybrid models); the attention layer
+appends the token's key and value to a bf16 cache and attends over it with
+torch.nn.functional.scaled_dot_product_attention (grouped-query: the query heads
+of a key/value head stacked as its query rows; flash or memory-efficient kernel).  The Mamba-2
 layer's short convolution and output gate are left out: they carry no decode
 state that the method changes.
 
@@ -92,13 +94,24 @@ class HybridStack:
                 "k": rnd(s.batch, s.n_kv_heads, cap, s.head_dim, scale=1.0).to(bf),
                 "v": rnd(s.batch, s.n_kv_heads, cap, s.head_dim, scale=1.0).to(bf),
             }))
+        # torch's SDPA is held to its flash and memory-efficient kernels: its
+        # default dispatch may pick a backend that builds an execution plan per
+        # new sequence length, which a decode meets every step (tens of
+        # milliseconds of host time per new length).
+        from torch.nn.attention import SDPBackend, sdpa_kernel
+
+        self._sdpa_backends = lambda: sdpa_kernel([SDPBackend.FLASH_ATTENTION, SDPBackend.EFFICIENT_ATTENTION])
         self.pos = s.context  # next cache position
         self.cap = s.context + max_steps
-        self.ssm_events = None  # set by time_ssm(): CUDA events around every SSM decode
+        self.ssm_events = None  # a list here records CUDA events around every SSM decode call
+
+    def _norm(self, x):
+        xf = x.float()
+        return (xf * self.torch.rsqrt(xf.pow(2).mean(dim=-1, keepdim=True) + 1e-6)).to(self.torch.bfloat16)
 
     def _ssm(self, x, p):
         torch, s = self.torch, self.s
-        u = x @ p["w_in"]
+        u = self._norm(x) @ p["w_in"]
         HP, H, GN = s.nheads * s.headdim, s.nheads, s.ngroups * s.dstate
         inputs = {
             "x": u[:, :HP].reshape(s.batch, 1, H, s.headdim).contiguous(),
@@ -119,11 +132,18 @@ class HybridStack:
 
     def _attn(self, x, p):
         torch, s = self.torch, self.s
-        q = (x @ p["wq"]).reshape(s.batch, s.n_q_heads, 1, s.head_dim)
-        p["k"][:, :, self.pos] = (x @ p["wk"]).reshape(s.batch, s.n_kv_heads, s.head_dim)
-        p["v"][:, :, self.pos] = (x @ p["wv"]).reshape(s.batch, s.n_kv_heads, s.head_dim)
+        xn = self._norm(x)
+        # One decode token: the query heads that share a key/value head attend to
+        # the same cache, so they are stacked as that head's query rows
+        # ([batch, kv heads, query heads per kv head, head_dim]); query head j
+        # uses key/value head j // (n_q_heads / n_kv_heads), as in grouped-query
+        # attention, and no mask applies.
+        q = (xn @ p["wq"]).reshape(s.batch, s.n_kv_heads, s.n_q_heads // s.n_kv_heads, s.head_dim)
+        p["k"][:, :, self.pos] = (xn @ p["wk"]).reshape(s.batch, s.n_kv_heads, s.head_dim)
+        p["v"][:, :, self.pos] = (xn @ p["wv"]).reshape(s.batch, s.n_kv_heads, s.head_dim)
         n = self.pos + 1
-        o = torch.nn.functional.scaled_dot_product_attention(q, p["k"][:, :, :n], p["v"][:, :, :n], enable_gqa=True)
+        with self._sdpa_backends():
+            o = torch.nn.functional.scaled_dot_product_attention(q, p["k"][:, :, :n], p["v"][:, :, :n])
         return x + o.reshape(s.batch, s.n_q_heads * s.head_dim) @ p["wo"]
 
     def step(self, x):
