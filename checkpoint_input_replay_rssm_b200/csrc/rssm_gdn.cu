@@ -79,12 +79,7 @@ cudaError_t gdn_launch(Ctx &h, int op, int T, const rssm_inputs *in, float *y, f
     if (e == cudaSuccess && fold) {
         GArgs f = a;
         f.fold_only = 1;
-        if (gdn_fold_tc_eligible(f, cf.headdim, N)) {  // the tensor-core fold (rssm_gdn_fold_tc.cu)
-            h.launches += 1;
-            e = gdn_fold_tc(f, cf.state_dtype, st);
-        } else {
-            e = v1(f);
-        }
+        e = v1(f);
     }
     if (e == cudaSuccess && h.split_event) e = cudaEventRecord(h.split_event, st);
     if (e == cudaSuccess) {

@@ -49,12 +49,6 @@ struct GArgs {
     int kda;                    // Kimi Delta Attention: alpha is a gate per key channel
 };
 
-// The fold of a decode call on the tensor cores (rssm_gdn_fold_tc.cu): used in
-// place of the fold-only launch of gdn_replay_kernel when d_k = d_v = 128,
-// T = 1 and W <= 32.
-bool gdn_fold_tc_eligible(const GArgs &a, int P, int N);
-cudaError_t gdn_fold_tc(const GArgs &a, int rk, cudaStream_t st);
-
 __host__ __device__ constexpr int gpad4(int n) { return (n + 3) & ~3; }
 
 // KDA keeps a gate row [E][N] where GDN keeps one gate per entry.  After the
@@ -151,63 +145,100 @@ __device__ __forceinline__ void gdn_stage_new(const GArgs &a, const GSmem &s, in
     if (tid < T) s.sbe[W + tid] = a.beta[(int64_t)(b * T + tid) * H + h];
 }
 
+// Packed pairs of fp32 (sm_100 .f32x2 arithmetic): one instruction updates two elements.
+__device__ __forceinline__ unsigned long long f2_pack(float a, float b) {
+    unsigned long long r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+    return r;
+}
+__device__ __forceinline__ void f2_unpack(unsigned long long v, float &a, float &b) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+__device__ __forceinline__ unsigned long long f2_fma(unsigned long long a, unsigned long long b, unsigned long long c) {
+    unsigned long long d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ unsigned long long f2_mul(unsigned long long a, unsigned long long b) {
+    unsigned long long d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
 // Apply entries [0, L0) (physical base..) to NR rows held as NPT-element lane
 // segments.  Rows are independent; every lane of the warp must call this.
 // GDN:  s <- alpha s + (beta v[row] - alpha beta (s . k)) k
 // KDA:  u = alpha (.) s;  s <- u + beta (v[row] - u . k) k
+// The row segments are held as packed pairs for the length of the call, so the
+// per-entry dot and update take one .f32x2 instruction per two elements; the
+// pair broadcasts (alpha per entry, the coefficient per row) are amortised over
+// the segment.
 template <int N, int NR>
 __device__ __forceinline__ void gdn_fold_rows(float (&st)[NR][FoldMap<N>::NPT], const int (&rows)[NR],
                                               int P, const GSmem &s, int base, int L0, int cseg, int kda) {
-    constexpr int NPT = FoldMap<N>::NPT, TPRF = FoldMap<N>::TPRF;
+    constexpr int NPT = FoldMap<N>::NPT, TPRF = FoldMap<N>::TPRF, NP2 = NPT / 2;
+    unsigned long long s2[NR][NP2];
+#pragma unroll
+    for (int r = 0; r < NR; ++r)
+#pragma unroll
+        for (int j = 0; j < NP2; ++j) s2[r][j] = f2_pack(st[r][2 * j], st[r][2 * j + 1]);
     for (int e = 0; e < L0; ++e) {
         const float be = s.sbe[base + e];
-        float kk[NPT];
+        unsigned long long k2[NP2];
 #pragma unroll
         for (int j = 0; j < NPT; j += 4) {
             const float4 k4 = *reinterpret_cast<const float4 *>(s.sk + (base + e) * N + cseg * NPT + j);
-            kk[j] = k4.x; kk[j + 1] = k4.y; kk[j + 2] = k4.z; kk[j + 3] = k4.w;
+            k2[j / 2] = f2_pack(k4.x, k4.y);
+            k2[j / 2 + 1] = f2_pack(k4.z, k4.w);
         }
         if (kda) {  // warp-uniform
-            float ga[NPT];
+            unsigned long long g2[NP2];
 #pragma unroll
             for (int j = 0; j < NPT; j += 4) {
                 const float4 g4 = *reinterpret_cast<const float4 *>(s.sal + (base + e) * N + cseg * NPT + j);
-                ga[j] = g4.x; ga[j + 1] = g4.y; ga[j + 2] = g4.z; ga[j + 3] = g4.w;
+                g2[j / 2] = f2_pack(g4.x, g4.y);
+                g2[j / 2 + 1] = f2_pack(g4.z, g4.w);
             }
 #pragma unroll
             for (int r = 0; r < NR; ++r) {
-                float d0 = 0.f, d1 = 0.f;  // two chains: half the dependent latency
+                unsigned long long d2 = 0ull;
 #pragma unroll
-                for (int j = 0; j < NPT; j += 2) {
-                    st[r][j] *= ga[j];
-                    st[r][j + 1] *= ga[j + 1];
-                    d0 = fmaf(st[r][j], kk[j], d0);
-                    d1 = fmaf(st[r][j + 1], kk[j + 1], d1);
+                for (int j = 0; j < NP2; ++j) {
+                    s2[r][j] = f2_mul(s2[r][j], g2[j]);
+                    d2 = f2_fma(s2[r][j], k2[j], d2);
                 }
-                const float d = group_sum<TPRF>(d0 + d1);
+                float dl, dh;
+                f2_unpack(d2, dl, dh);
+                const float d = group_sum<TPRF>(dl + dh);
                 const float vr = (rows[r] < P) ? s.sv[(base + e) * P + rows[r]] : 0.f;
                 const float coef = be * (vr - d);
+                const unsigned long long c2 = f2_pack(coef, coef);
 #pragma unroll
-                for (int j = 0; j < NPT; ++j) st[r][j] = fmaf(coef, kk[j], st[r][j]);
+                for (int j = 0; j < NP2; ++j) s2[r][j] = f2_fma(c2, k2[j], s2[r][j]);
             }
             continue;
         }
         const float al = s.sal[base + e];
+        const unsigned long long a2 = f2_pack(al, al);
 #pragma unroll
         for (int r = 0; r < NR; ++r) {
-            float d0 = 0.f, d1 = 0.f;  // two chains: half the dependent latency
+            unsigned long long d2 = 0ull;
 #pragma unroll
-            for (int j = 0; j < NPT; j += 2) {
-                d0 = fmaf(st[r][j], kk[j], d0);
-                d1 = fmaf(st[r][j + 1], kk[j + 1], d1);
-            }
-            const float d = group_sum<TPRF>(d0 + d1);
+            for (int j = 0; j < NP2; ++j) d2 = f2_fma(s2[r][j], k2[j], d2);
+            float dl, dh;
+            f2_unpack(d2, dl, dh);
+            const float d = group_sum<TPRF>(dl + dh);
             const float vr = (rows[r] < P) ? s.sv[(base + e) * P + rows[r]] : 0.f;
             const float coef = be * vr - al * be * d;
+            const unsigned long long c2 = f2_pack(coef, coef);
 #pragma unroll
-            for (int j = 0; j < NPT; ++j) st[r][j] = fmaf(al, st[r][j], coef * kk[j]);
+            for (int j = 0; j < NP2; ++j) s2[r][j] = f2_fma(a2, s2[r][j], f2_mul(c2, k2[j]));
         }
     }
+#pragma unroll
+    for (int r = 0; r < NR; ++r)
+#pragma unroll
+        for (int j = 0; j < NP2; ++j) f2_unpack(s2[r][j], st[r][2 * j], st[r][2 * j + 1]);
 }
 
 // ---------------------------------------------------------------------------

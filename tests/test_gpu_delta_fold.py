@@ -1,12 +1,8 @@
-"""The tensor-core fold of Gated DeltaNet and Kimi Delta Attention decode calls
-(d_k = d_v = 128, W <= 32) against the fp64 CPU oracle.
-
-The fold's two products run as split-bf16 MMAs (about 16 bits per operand) and
-the checkpoint passes through in fp32, so the fp32 read path keeps the 1e-4 x
-RMS output tolerance of the sequential fold and the exported state stays within
-1e-4 x RMS of the oracle's.  Windows cover one and two 16-entry MMA slices and
-ragged buffer lengths (a window not a multiple of 16 pads the slice with
-entries that contribute nothing); both input dtypes; every read copy.
+"""The Gated DeltaNet and Kimi Delta Attention decode fold at d_k = d_v = 128
+against the fp64 CPU oracle: windows from 1 to 32 entries (ragged lengths
+included), both input dtypes, every read copy, buffers of different lengths
+folding on different calls, and the read copy checked bit for bit against the
+rounding of the fp32 checkpoint.
 
 The low-precision copies are compared with the oracle's emulated copy (the
 rounding of its fp64 checkpoint).  An fp32 checkpoint within eps of the fp64
@@ -29,7 +25,7 @@ pytestmark = pytest.mark.gpu
 
 
 def _wl(kind, W, input_dtype, batch=3, nheads=2):
-    return I.Workload(name=f"{kind}_foldtc_w{W}", kind=kind, batch=batch, nheads=nheads, headdim=128, dstate=128,
+    return I.Workload(name=f"{kind}_fold_w{W}", kind=kind, batch=batch, nheads=nheads, headdim=128, dstate=128,
                       ngroups=nheads, window=W, steps=3 * W + 2, seed=400 + W, read_dtype="f32",
                       input_dtype=input_dtype)
 
@@ -91,8 +87,8 @@ def test_fold_fp32_inputs(kind):
 def test_fold_with_staggered_buffers(kind):
     """Sequences whose buffers fold on different calls: one verify of 4 drafts
     with accept lengths 0..4 leaves the buffers at different lengths, so every
-    later fold call serves some sequences from the tensor-core fold and leaves
-    the rest to the read kernel.  Compared with the oracle's bf16 read copy."""
+    later fold call serves some sequences from the fold kernel and leaves the
+    rest to the read kernel.  Compared with the oracle's bf16 read copy."""
     import torch
 
     wl = _wl(kind, 16, "bf16", batch=10)
@@ -120,7 +116,7 @@ def test_fold_with_staggered_buffers(kind):
 
 @pytest.mark.parametrize("kind", ["gdn", "kda"])
 def test_read_copy_is_the_rounded_checkpoint_after_folds(kind):
-    """After several tensor-core folds the read copy equals the rounding of the
+    """After several folds the read copy equals the rounding of the
     fp32 checkpoint, bit for bit: bf16 round-to-nearest-even, and for fp8 the
     per-row scale amax / 448 (correctly rounded) with e4m3(value / scale)
     (torch's casts, which the oracle's quantisers are pinned to)."""
