@@ -841,6 +841,97 @@ __global__ void __launch_bounds__(kThreads, (TQ == 1 && SK != SK_FP8) ? 4 : 1) m
     }
 }
 
+// Eager decode (T = 1) with two heads of one group per CTA: both heads' state
+// rows are requested before anything else and the group's B and C are staged
+// once, so each CTA keeps 2 x P x N state elements in flight and its prologue is
+// shared by two heads.  Per element it computes exactly what m2_eager_kernel
+// computes (the same operations in the same order).  Requires P <= 8 rows per
+// thread x (kThreads / (N / 4)) and an even number of heads per group.
+template <int N, int SK>
+__global__ void __launch_bounds__(kThreads, SK == SK_FP8 ? 2 : 3) m2_eager_decode2_kernel(const M2Args a) {
+    constexpr int TPR4 = N / 4;
+    constexpr int RPP4 = kThreads / TPR4;
+    constexpr int RB = 8;
+    extern __shared__ __align__(16) float smem[];
+    const int tid = threadIdx.x;
+    const int H = a.H, P = a.P, G = a.G;
+    const int bh0 = 2 * blockIdx.x;
+    const int b = bh0 / H, h0 = bh0 - b * H;
+    const int g = h0 / (H / G);
+    float *sx = smem;                 // [2][P]
+    float *sB = sx + pad4(2 * P);     // [N]
+    float *sC = sB + pad4(N);         // [N]
+    float *sdot = sC + pad4(N);       // [2][P]
+    float *sa = sdot + pad4(2 * P);   // [2] decay
+    float *ss = sa + 4;               // [2] input scale
+    void *state = (SK == SK_F32) ? (void *)a.ckpt : a.rc;
+
+    const int c4 = tid % TPR4, q0 = tid / TPR4;
+    float4 st[2][RB];
+    float scl[2][RB];
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+        for (int k = 0; k < RB; ++k) {
+            const int r = q0 + k * RPP4;
+            const int64_t row = (int64_t)(bh0 + hh) * P + r;
+            st[hh][k] = (r < P) ? load_quad<SK>(state, row * N + 4 * c4) : make_float4(0.f, 0.f, 0.f, 0.f);
+            scl[hh][k] = (SK == SK_FP8 && r < P) ? __ldg(a.rc_scale + row) : 1.f;
+        }
+
+    // No other CTA of an eager launch reads the counters, so the CTA of the
+    // sequence's first heads rewrites them alone (no arrival count, no fence).
+    if (tid == 0 && h0 == 0) {
+        const int64_t s1 = a.c.seq_pos[b] + 1;
+        a.c.seq_pos[b] = s1;
+        a.c.ckpt_pos[b] = s1;
+    }
+    for (int i = tid; i < 2 * P; i += kThreads) sx[i] = ld_in(a.x, (int64_t)(b * H + h0) * P + i, a.in_bf16);
+    for (int i = tid; i < N; i += kThreads) {
+        const int64_t src = ((int64_t)b * G + g) * N + i;
+        sB[i] = ld_in(a.Bm, src, a.in_bf16);
+        sC[i] = ld_in(a.Cm, src, a.in_bf16);
+    }
+    if (tid < 2) {
+        const float dtv = a.dt[(int64_t)b * H + h0 + tid];
+        sa[tid] = expf(dtv * a.A[h0 + tid]);
+        ss[tid] = a.dt_scales ? dtv : 1.f;
+    }
+    __syncthreads();
+
+    const float4 Bq = reinterpret_cast<const float4 *>(sB)[c4];
+    const float4 Cq = reinterpret_cast<const float4 *>(sC)[c4];
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+        const float am = sa[hh], sc_in = ss[hh];
+        const int64_t tile0 = (int64_t)(bh0 + hh) * P * N;
+#pragma unroll
+        for (int k = 0; k < RB; ++k) {
+            const int r = q0 + k * RPP4;
+            const bool valid = r < P;
+            const int64_t el = tile0 + (int64_t)(valid ? r : 0) * N + 4 * c4;
+            float4 v = st[hh][k];
+            if (SK == SK_FP8) { v.x *= scl[hh][k]; v.y *= scl[hh][k]; v.z *= scl[hh][k]; v.w *= scl[hh][k]; }
+            const float w = sc_in * (valid ? sx[hh * P + r] : 0.f);
+            v.x = fmaf(am, v.x, w * Bq.x); v.y = fmaf(am, v.y, w * Bq.y);
+            v.z = fmaf(am, v.z, w * Bq.z); v.w = fmaf(am, v.w, w * Bq.w);
+            float d = v.x * Cq.x + v.y * Cq.y + v.z * Cq.z + v.w * Cq.w;
+            d = group_sum<TPR4>(d);
+            if (c4 == 0 && valid) sdot[hh * P + r] = d;  // output from the fp32 value
+            float sc = 1.f;
+            if (SK == SK_FP8) {
+                const float amx = fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
+                sc = fp8_scale(group_max<TPR4>(amx));
+                if (valid && c4 == 0) a.rc_scale[(int64_t)(bh0 + hh) * P + r] = sc;
+            }
+            if (valid) store_quad<SK>(state, el, v, 0.f, sc);
+        }
+    }
+    __syncthreads();
+    for (int i = tid; i < 2 * P; i += kThreads)
+        a.y[(int64_t)(b * H + h0) * P + i] = sdot[i] + a.D[h0 + i / P] * sx[i];
+}
+
 // ---------------------------------------------------------------------------
 // Host launchers.
 // ---------------------------------------------------------------------------
@@ -872,6 +963,15 @@ inline cudaError_t launch_fold_t(const M2Args &a, const M2FoldLay &lay, int num_
 
 template <int N, int SK, int TQ>
 inline cudaError_t launch_eager_t(const M2Args &a, size_t smem, cudaStream_t st) {
+    constexpr int kRows = 8 * (kThreads / (N / 4));  // state rows one pass of the two-head kernel covers
+    if (TQ == 1 && a.op == OP_DECODE && a.T == 1 && (a.H / a.G) % 2 == 0 && a.P <= kRows) {
+        auto k2 = m2_eager_decode2_kernel<N, SK>;
+        const int smem2 = (int)sizeof(float) * (2 * pad4(2 * a.P) + 2 * pad4(N) + 8);
+        cudaError_t e = cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, smem2);
+        if (e != cudaSuccess) return e;
+        k2<<<a.B * a.H / 2, kThreads, smem2, st>>>(a);
+        return cudaGetLastError();
+    }
     auto k = m2_eager_kernel<N, SK, TQ>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
