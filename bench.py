@@ -299,7 +299,7 @@ def hybrid_leg(device, sync, dist, world, steps, warmup):
     out["config"] = {"blocks": shape.blocks, "ssm_per_attention": shape.ssm_per_block, "batch_per_gpu": shape.batch,
                      "d_model": shape.d_model, "ssm_layer": "mamba2 128 heads x 64 x 128, 8 groups, W 16",
                      "attention": f"{shape.n_q_heads} q / {shape.n_kv_heads} kv heads x {shape.head_dim}, "
-                                  f"{shape.context} cached tokens, bf16, torch SDPA",
+                                  f"{shape.context} cached tokens, bf16, torch SDPA (flash / memory-efficient kernels)",
                      "projections": "bf16 torch.matmul, random weights", "steps": steps}
     return out
 
