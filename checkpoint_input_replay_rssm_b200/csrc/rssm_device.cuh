@@ -170,6 +170,22 @@ __device__ __forceinline__ float group_max(float v) {
     return v;
 }
 
+// Sums of four row values over the Q lanes of a row group (Q >= 4, a power of
+// two), exchanging halves first: 2 + 1 + log2(Q/4) shuffles instead of
+// 4 log2(Q).  Lane q of the group returns the sum of row 2*(q >= Q/2) + ((q & Q/4) != 0).
+// Every lane of the warp must call it.
+template <int Q>
+__device__ __forceinline__ float quad_rows_sum(float d0, float d1, float d2, float d3, int q) {
+    const bool hi = (q & (Q / 2)) != 0, hi2 = (q & (Q / 4)) != 0;
+    const float s0 = __shfl_xor_sync(0xffffffffu, hi ? d0 : d2, Q / 2);
+    const float s1 = __shfl_xor_sync(0xffffffffu, hi ? d1 : d3, Q / 2);
+    const float e0 = (hi ? d2 : d0) + s0, e1 = (hi ? d3 : d1) + s1;
+    float f = (hi2 ? e1 : e0) + __shfl_xor_sync(0xffffffffu, hi2 ? e0 : e1, Q / 4);
+#pragma unroll
+    for (int o = Q / 8; o > 0; o >>= 1) f += __shfl_xor_sync(0xffffffffu, f, o);
+    return f;
+}
+
 __device__ __forceinline__ float ld_in(const void *p, int64_t i, int bf16) {
     return bf16 ? bf16_bits_to_float(reinterpret_cast<const uint16_t *>(p)[i])
                 : reinterpret_cast<const float *>(p)[i];

@@ -165,18 +165,27 @@ __device__ __forceinline__ unsigned long long f2_mul(unsigned long long a, unsig
     return d;
 }
 
-// Apply entries [0, L0) (physical base..) to NR rows held as NPT-element lane
-// segments.  Rows are independent; every lane of the warp must call this.
+// Apply entries [0, L0) (physical base..) to the NR = 4 rows a thread holds as
+// NPT-element lane segments (TPRF lanes per row).  Rows are independent; every
+// lane of the warp must call this.
 // GDN:  s <- alpha s + (beta v[row] - alpha beta (s . k)) k
 // KDA:  u = alpha (.) s;  s <- u + beta (v[row] - u . k) k
 // The row segments are held as packed pairs for the length of the call, so the
-// per-entry dot and update take one .f32x2 instruction per two elements; the
-// pair broadcasts (alpha per entry, the coefficient per row) are amortised over
-// the segment.
+// per-entry dot and update take one .f32x2 instruction per two elements.  The
+// four rows' dots are reduced together (quad_rows_sum: 5 shuffles instead of
+// 4 log2(TPRF)); each lane then holds one row's sum, reads that row's v and
+// forms its coefficient, and the four coefficients are broadcast back from the
+// lanes that hold them.
 template <int N, int NR>
 __device__ __forceinline__ void gdn_fold_rows(float (&st)[NR][FoldMap<N>::NPT], const int (&rows)[NR],
                                               int P, const GSmem &s, int base, int L0, int cseg, int kda) {
     constexpr int NPT = FoldMap<N>::NPT, TPRF = FoldMap<N>::TPRF, NP2 = NPT / 2;
+    static_assert(NR == 4 && TPRF >= 4, "four rows per thread, reduced over at least four lanes");
+    const int lane = threadIdx.x & 31;
+    const int qrow = 2 * ((cseg & (TPRF / 2)) != 0) + ((cseg & (TPRF / 4)) != 0);  // the row this lane's sum belongs to
+    const int myrow = qrow == 0 ? rows[0] : (qrow == 1 ? rows[1] : (qrow == 2 ? rows[2] : rows[3]));
+    const bool myvalid = myrow < P;
+    const int gbase = lane & ~(TPRF - 1);  // first lane of this row group
     unsigned long long s2[NR][NP2];
 #pragma unroll
     for (int r = 0; r < NR; ++r)
@@ -191,6 +200,7 @@ __device__ __forceinline__ void gdn_fold_rows(float (&st)[NR][FoldMap<N>::NPT], 
             k2[j / 2] = f2_pack(k4.x, k4.y);
             k2[j / 2 + 1] = f2_pack(k4.z, k4.w);
         }
+        float dp[NR];
         if (kda) {  // warp-uniform
             unsigned long long g2[NP2];
 #pragma unroll
@@ -209,30 +219,41 @@ __device__ __forceinline__ void gdn_fold_rows(float (&st)[NR][FoldMap<N>::NPT], 
                 }
                 float dl, dh;
                 f2_unpack(d2, dl, dh);
-                const float d = group_sum<TPRF>(dl + dh);
-                const float vr = (rows[r] < P) ? s.sv[(base + e) * P + rows[r]] : 0.f;
-                const float coef = be * (vr - d);
-                const unsigned long long c2 = f2_pack(coef, coef);
+                dp[r] = dl + dh;
+            }
+        } else {
+#pragma unroll
+            for (int r = 0; r < NR; ++r) {
+                unsigned long long d2 = 0ull;
+#pragma unroll
+                for (int j = 0; j < NP2; ++j) d2 = f2_fma(s2[r][j], k2[j], d2);
+                float dl, dh;
+                f2_unpack(d2, dl, dh);
+                dp[r] = dl + dh;
+            }
+        }
+        const float d = quad_rows_sum<TPRF>(dp[0], dp[1], dp[2], dp[3], cseg);
+        const float vr = myvalid ? s.sv[(base + e) * P + myrow] : 0.f;
+        const float al = kda ? 1.f : s.sal[base + e];
+        const float coef = kda ? be * (vr - d) : be * vr - al * be * d;
+        float cr[NR];
+#pragma unroll
+        for (int r = 0; r < NR; ++r) cr[r] = __shfl_sync(0xffffffffu, coef, gbase + r * (TPRF / 4));
+        if (kda) {
+#pragma unroll
+            for (int r = 0; r < NR; ++r) {
+                const unsigned long long c2 = f2_pack(cr[r], cr[r]);
 #pragma unroll
                 for (int j = 0; j < NP2; ++j) s2[r][j] = f2_fma(c2, k2[j], s2[r][j]);
             }
-            continue;
-        }
-        const float al = s.sal[base + e];
-        const unsigned long long a2 = f2_pack(al, al);
+        } else {
+            const unsigned long long a2 = f2_pack(al, al);
 #pragma unroll
-        for (int r = 0; r < NR; ++r) {
-            unsigned long long d2 = 0ull;
+            for (int r = 0; r < NR; ++r) {
+                const unsigned long long c2 = f2_pack(cr[r], cr[r]);
 #pragma unroll
-            for (int j = 0; j < NP2; ++j) d2 = f2_fma(s2[r][j], k2[j], d2);
-            float dl, dh;
-            f2_unpack(d2, dl, dh);
-            const float d = group_sum<TPRF>(dl + dh);
-            const float vr = (rows[r] < P) ? s.sv[(base + e) * P + rows[r]] : 0.f;
-            const float coef = be * vr - al * be * d;
-            const unsigned long long c2 = f2_pack(coef, coef);
-#pragma unroll
-            for (int j = 0; j < NP2; ++j) s2[r][j] = f2_fma(a2, s2[r][j], f2_mul(c2, k2[j]));
+                for (int j = 0; j < NP2; ++j) s2[r][j] = f2_fma(a2, s2[r][j], f2_mul(c2, k2[j]));
+            }
         }
     }
 #pragma unroll

@@ -319,22 +319,6 @@ inline M2FoldLay m2_fold_lay(int HC, int P, int N, int W, int R, int TQ, int ib)
     return L;
 }
 
-// Sums of four row values over the Q lanes of a row group (Q >= 4, a power of
-// two), exchanging halves first: 2 + 1 + log2(Q/4) shuffles instead of
-// 4 log2(Q).  Lane q of the group returns the sum of row 2*(q >= Q/2) + ((q & Q/4) != 0).
-// Every lane of the warp must call it.
-template <int Q>
-__device__ __forceinline__ float quad_rows_sum(float d0, float d1, float d2, float d3, int q) {
-    const bool hi = (q & (Q / 2)) != 0, hi2 = (q & (Q / 4)) != 0;
-    const float s0 = __shfl_xor_sync(0xffffffffu, hi ? d0 : d2, Q / 2);
-    const float s1 = __shfl_xor_sync(0xffffffffu, hi ? d1 : d3, Q / 2);
-    const float e0 = (hi ? d2 : d0) + s0, e1 = (hi ? d3 : d1) + s1;
-    float f = (hi2 ? e1 : e0) + __shfl_xor_sync(0xffffffffu, hi2 ? e0 : e1, Q / 4);
-#pragma unroll
-    for (int o = Q / 8; o > 0; o >>= 1) f += __shfl_xor_sync(0xffffffffu, f, o);
-    return f;
-}
-
 template <int N, int RK, int TQ, bool BF>
 __global__ void __launch_bounds__(kThreads, 3) m2_fold_kernel(const M2Args a, const M2FoldLay Ly) {
     constexpr int Q = N / 4;              // column quads per row
@@ -722,7 +706,7 @@ __global__ void __launch_bounds__(kThreads, 3) m2_fold_kernel(const M2Args a, co
 // (blog.thibaultmonteiro.fr, "La fiche qu'on reecrit a chaque token").
 // ---------------------------------------------------------------------------
 template <int N, int SK, int TQ>
-__global__ void __launch_bounds__(kThreads, (TQ == 1 && SK != SK_FP8) ? 4 : 1) m2_eager_kernel(const M2Args a) {
+__global__ void __launch_bounds__(kThreads) m2_eager_kernel(const M2Args a) {
     constexpr int TPR4 = N / 4;
     constexpr int RPP4 = kThreads / TPR4;
     constexpr int RB = 8;
@@ -742,28 +726,12 @@ __global__ void __launch_bounds__(kThreads, (TQ == 1 && SK != SK_FP8) ? 4 : 1) m
     void *state = (SK == SK_F32) ? (void *)a.ckpt : a.rc;
     const int64_t state_elems = (int64_t)a.B * H * P * N;
 
-    // The first batch of state rows is requested before the inputs are staged,
-    // so the tile's HBM latency overlaps the prologue.
-    const int c4 = tid % TPR4, q0 = tid / TPR4;
-    float4 st[RB];
-    float scl[RB];
-#pragma unroll
-    for (int k = 0; k < RB; ++k) {
-        const int r = q0 + k * RPP4;
-        st[k] = (r < P) ? load_quad<SK>(state, tile0 + (int64_t)r * N + 4 * c4) : make_float4(0.f, 0.f, 0.f, 0.f);
-        scl[k] = (SK == SK_FP8 && r < P) ? __ldg(a.rc_scale + (int64_t)bh * P + r) : 1.f;
-    }
-
-    // No other CTA of an eager launch reads the counters, so the sequence's first
-    // head's CTA rewrites them alone (no arrival count, no fence).
-    if (tid == 0 && h == 0) {
-        if (a.op == OP_DECODE) {
-            const int64_t s1 = a.c.seq_pos[b] + 1;
-            a.c.seq_pos[b] = s1;
-            a.c.ckpt_pos[b] = s1;
-        } else {
-            a.c.pending[b] = T;
-        }
+    if (tid == 0) {
+        SeqState st = read_counters(a.c, b, a.W);
+        if (a.op == OP_DECODE)
+            arrive_and_publish(a.c, b, H, st.seq + 1, st.seq + 1, -1, 0);
+        else
+            arrive_and_publish(a.c, b, H, -1, -1, T, 0);
     }
     for (int i = tid; i < T * P; i += kThreads) {
         const int m = i / P, p = i - m * P;
@@ -782,15 +750,16 @@ __global__ void __launch_bounds__(kThreads, (TQ == 1 && SK != SK_FP8) ? 4 : 1) m
     }
     __syncthreads();
 
+    const int c4 = tid % TPR4, q0 = tid / TPR4;
     for (int rb = 0; rb < P; rb += RB * RPP4) {
-        if (rb > 0) {
+        float4 st[RB];
+        float scl[RB];
 #pragma unroll
-            for (int k = 0; k < RB; ++k) {
-                const int r = rb + q0 + k * RPP4;
-                st[k] = (r < P) ? load_quad<SK>(state, tile0 + (int64_t)r * N + 4 * c4)
-                                : make_float4(0.f, 0.f, 0.f, 0.f);
-                scl[k] = (SK == SK_FP8 && r < P) ? __ldg(a.rc_scale + (int64_t)bh * P + r) : 1.f;
-            }
+        for (int k = 0; k < RB; ++k) {
+            const int r = rb + q0 + k * RPP4;
+            st[k] = (r < P) ? load_quad<SK>(state, tile0 + (int64_t)r * N + 4 * c4)
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
+            scl[k] = (SK == SK_FP8 && r < P) ? __ldg(a.rc_scale + (int64_t)bh * P + r) : 1.f;
         }
 #pragma unroll
         for (int k = 0; k < RB; ++k) {

@@ -71,6 +71,7 @@ cudaError_t launch_read(const Ctx &h, int op, int T, const void *Q, int q_bf16, 
     r.op = op;
     r.early = early ? 1 : 0;
     r.pdl = (early && pdl) ? 1 : 0;
+    r.q_ready = (Q != (const void *)ho.query) ? 1 : 0;  // Mamba-2: the call's C; GDN / KDA: the swept queries
     const int TQ = tq_of_read(T);
     r.lay = read_lay(r.HC, cf.headdim, cf.dstate, cf.window, TQ, cf.input_dtype == RSSM_BF16 ? 2 : 4, r.Emax);
     const size_t smem = read_smem_bytes(cf, T);

@@ -74,6 +74,7 @@ struct ReadArgs {
     int early;              // no flush kernel ran in this call: every sequence is read, so the
                             // first read-copy round is issued before anything else
     int pdl;                // launched as a programmatic dependent of the prep kernel
+    int q_ready;            // the queries are the caller's input, not the prep kernel's output
 };
 
 template <int N, int RK, int TQ, bool BF>
@@ -127,57 +128,123 @@ __global__ void __launch_bounds__(kThreads, TQ == 1 ? 4 : 2) replay_read_kernel(
         skip_copy = sinfo[2] != 0;
     }
     if (!skip_copy) issue(0);
-    pdl_wait();  // the prep kernel's hand-off is complete and visible
+    // The read copy, its fp8 row scales and (for Mamba-2) the queries are not
+    // written by the prep kernel.  When no flush kernel runs in this call and the
+    // queries are the caller's input, every round of the stream is dotted before
+    // the prep kernel's hand-off is awaited; otherwise it is awaited here.
+    const bool stream_first = a.early && a.q_ready;
+    if (!stream_first) pdl_wait();  // the prep kernel's hand-off is complete and visible
 
-    // 2. Small operands: per-sequence info, the call's entries, decays, the
-    //    coefficient rows of the CTA's heads (contiguous), queries, fp8 scales.
-    if (tid == 0) {
-        const int4 si = a.seqinfo[b];
-        sinfo[0] = si.x; sinfo[1] = si.y; sinfo[2] = si.z;
-        // Counters of the sequence: every prep CTA has read them (the prep kernel
-        // ran before this one), so the first CTA of the sequence rewrites them.
-        if (blockIdx.x == 0 && b == 0) *a.fold_count = 0;  // the flush kernel has run
-        if (blockIdx.x == 0 && si.w) {
-            const int64_t sp = a.c.seq_pos[b];
-            if (si.z) {
-                a.c.ckpt_pos[b] = sp;
-                a.c.flush_count[b] += 1;
-            }
-            if (a.op == OP_DECODE) a.c.seq_pos[b] = sp + 1;
-            else a.c.pending[b] = T;
-        }
-    }
-    for (int row = warp; row < T * HC; row += kWarps) {  // x of token m, head hh
-        const int m = row / HC, hh = row - m * HC;
-        const uint8_t *src = reinterpret_cast<const uint8_t *>(a.xnew) + (((int64_t)(b * T + m) * H + h0 + hh) * P) * IB;
-        for (int k = lane; k < xch; k += 32) cp_async16(sx + (hh * E + W + m) * xrow + k * 16, src + k * 16);
-    }
-    {  // rows m < T of each head's [TQmax][Ep] table, to [HC][TQ][Ep]
-        const int per = T * Ep / 4;  // 16-byte chunks per head
-        for (int i = tid; i < HC * per; i += kThreads) {
-            const int hh = i / per, j = i - hh * per;
-            cp_async16(scoef + hh * TQ * Ep + 4 * j, a.coef + (row0 + hh) * a.TQmax * Ep + 4 * j);
-        }
-    }
-    for (int i = tid; i < HC * T; i += kThreads) {
-        const int hh = i / T, m = i - hh * T;
-        sdec[hh * TQ + m] = a.dec[(row0 + hh) * a.TQmax + m];
-    }
-    // queries: one row for the CTA when its heads share a query row (Mamba-2
-    // groups), else one per head
+    // Queries: one row for the CTA when its heads share a query row (Mamba-2
+    // groups), else one per head; fp8 row scales.
     const bool shared_q = (h0 / a.q_group) == ((h0 + HC - 1) / a.q_group);
     const int nq = shared_q ? 1 : HC;
-    for (int i = tid; i < nq * T * N; i += kThreads) {
-        const int hq = i / (T * N), r2 = i - hq * T * N;
-        const int m = r2 / N, n = r2 - m * N;
-        const int64_t qi = (int64_t)b * a.q_stride_b + (int64_t)((h0 + hq) / a.q_group) * a.q_stride_row +
-                           (int64_t)m * a.q_stride_m + n;
-        sq[(hq * TQ + m) * N + n] = a.q_bf16 ? bf16_bits_to_float(reinterpret_cast<const uint16_t *>(a.Q)[qi])
-                                             : reinterpret_cast<const float *>(a.Q)[qi];
+    auto stage_queries = [&]() {
+        for (int i = tid; i < nq * T * N; i += kThreads) {
+            const int hq = i / (T * N), r2 = i - hq * T * N;
+            const int m = r2 / N, n = r2 - m * N;
+            const int64_t qi = (int64_t)b * a.q_stride_b + (int64_t)((h0 + hq) / a.q_group) * a.q_stride_row +
+                               (int64_t)m * a.q_stride_m + n;
+            sq[(hq * TQ + m) * N + n] = a.q_bf16 ? bf16_bits_to_float(reinterpret_cast<const uint16_t *>(a.Q)[qi])
+                                                 : reinterpret_cast<const float *>(a.Q)[qi];
+        }
+        if (RK == SK_FP8)
+            for (int i = tid; i < nrows / 4; i += kThreads) cp_async16(ssc + 4 * i, a.rc_scale + row0 * P + 4 * i);
+    };
+    // The prep kernel's hand-off: per-sequence info (and the counters it read,
+    // rewritten by the sequence's first CTA), the call's entries, decays and the
+    // coefficient rows of the CTA's heads (contiguous).
+    auto stage_handoff = [&]() {
+        if (tid == 0) {
+            const int4 si = a.seqinfo[b];
+            sinfo[0] = si.x; sinfo[1] = si.y; sinfo[2] = si.z;
+            // Every prep CTA has read the counters (the prep kernel has completed),
+            // so the first CTA of the sequence rewrites them.
+            if (blockIdx.x == 0 && b == 0) *a.fold_count = 0;  // the flush kernel has run
+            if (blockIdx.x == 0 && si.w) {
+                const int64_t sp = a.c.seq_pos[b];
+                if (si.z) {
+                    a.c.ckpt_pos[b] = sp;
+                    a.c.flush_count[b] += 1;
+                }
+                if (a.op == OP_DECODE) a.c.seq_pos[b] = sp + 1;
+                else a.c.pending[b] = T;
+            }
+        }
+        for (int row = warp; row < T * HC; row += kWarps) {  // x of token m, head hh
+            const int m = row / HC, hh = row - m * HC;
+            const uint8_t *src = reinterpret_cast<const uint8_t *>(a.xnew) + (((int64_t)(b * T + m) * H + h0 + hh) * P) * IB;
+            for (int k = lane; k < xch; k += 32) cp_async16(sx + (hh * E + W + m) * xrow + k * 16, src + k * 16);
+        }
+        {  // rows m < T of each head's [TQmax][Ep] table, to [HC][TQ][Ep]
+            const int per = T * Ep / 4;  // 16-byte chunks per head
+            for (int i = tid; i < HC * per; i += kThreads) {
+                const int hh = i / per, j = i - hh * per;
+                cp_async16(scoef + hh * TQ * Ep + 4 * j, a.coef + (row0 + hh) * a.TQmax * Ep + 4 * j);
+            }
+        }
+        for (int i = tid; i < HC * T; i += kThreads) {
+            const int hh = i / T, m = i - hh * T;
+            sdec[hh * TQ + m] = a.dec[(row0 + hh) * a.TQmax + m];
+        }
+    };
+    // The rows dotted with their query, round after round of the copy.
+    auto stream = [&]() {
+        for (int pass0 = 0; pass0 * RPP < nrows; pass0 += PPR) {
+            if (pass0 > 0) issue(pass0);
+#pragma unroll
+            for (int j = 0; j < PPR; ++j) {
+                const int r = (pass0 + j) * RPP + rrow;
+                const bool valid = r < nrows;
+                float acc[TQ];
+#pragma unroll
+                for (int m = 0; m < TQ; ++m) acc[m] = 0.f;
+                const float *qv = sq + (shared_q ? 0 : (valid ? r / P : 0)) * TQ * N;
+#pragma unroll
+                for (int k = 0; k < CPL; ++k) {
+                    float v[EPC];
+                    if (valid) unpack<RK>(rv[j * CPL + k], v);
+                    else {
+#pragma unroll
+                        for (int e = 0; e < EPC; ++e) v[e] = 0.f;
+                    }
+                    const int c0 = (q + LPR * k) * EPC;
+#pragma unroll
+                    for (int m = 0; m < TQ; ++m) {
+                        const float4 *q4 = reinterpret_cast<const float4 *>(qv + m * N + c0);
+#pragma unroll
+                        for (int e4 = 0; e4 < EPC / 4; ++e4) {
+                            const float4 w = q4[e4];
+                            acc[m] = fmaf(v[4 * e4], w.x, acc[m]);
+                            acc[m] = fmaf(v[4 * e4 + 1], w.y, acc[m]);
+                            acc[m] = fmaf(v[4 * e4 + 2], w.z, acc[m]);
+                            acc[m] = fmaf(v[4 * e4 + 3], w.w, acc[m]);
+                        }
+                    }
+                }
+#pragma unroll
+                for (int m = 0; m < TQ; ++m) {
+                    const float d = group_sum<LPR>(acc[m]);
+                    if (q == 0 && valid && m < T)
+                        sdot[r * TQ + m] = (RK == SK_FP8) ? d * ssc[r] : d;
+                }
+            }
+        }
+    };
+
+    if (stream_first) {
+        stage_queries();
+        cp_async_wait_all();  // fp8 row scales
+        __syncthreads();
+        stream();
+        pdl_wait();  // the prep kernel's hand-off is complete and visible
+        stage_handoff();
+        __syncthreads();
+    } else {
+        stage_handoff();
+        stage_queries();
+        __syncthreads();
     }
-    if (RK == SK_FP8)
-        for (int i = tid; i < nrows / 4; i += kThreads) cp_async16(ssc + 4 * i, a.rc_scale + row0 * P + 4 * i);
-    __syncthreads();
     const int L0 = sinfo[0], ckmod = sinfo[1], folded = sinfo[2];
     if (folded) {  // served by the flush kernel
         cp_async_wait_all();
@@ -193,51 +260,12 @@ __global__ void __launch_bounds__(kThreads, TQ == 1 ? 4 : 2) replay_read_kernel(
         uint8_t *dst = sx + (hh * E + base + (second ? n1 : 0)) * xrow;
         for (int k = lane; k < cnt * xch; k += 32) cp_async16(dst + k * 16, src + k * 16);
     }
-
-    // 3. Rows dotted with their query.
-    if (RK == SK_FP8) {  // the row scales must have landed before the first dot is scaled
-        cp_async_wait_all();
-        __syncthreads();
-    }
-    for (int pass0 = 0; pass0 * RPP < nrows; pass0 += PPR) {
-        if (pass0 > 0) issue(pass0);
-#pragma unroll
-        for (int j = 0; j < PPR; ++j) {
-            const int r = (pass0 + j) * RPP + rrow;
-            const bool valid = r < nrows;
-            float acc[TQ];
-#pragma unroll
-            for (int m = 0; m < TQ; ++m) acc[m] = 0.f;
-            const float *qv = sq + (shared_q ? 0 : (valid ? r / P : 0)) * TQ * N;
-#pragma unroll
-            for (int k = 0; k < CPL; ++k) {
-                float v[EPC];
-                if (valid) unpack<RK>(rv[j * CPL + k], v);
-                else {
-#pragma unroll
-                    for (int e = 0; e < EPC; ++e) v[e] = 0.f;
-                }
-                const int c0 = (q + LPR * k) * EPC;
-#pragma unroll
-                for (int m = 0; m < TQ; ++m) {
-                    const float4 *q4 = reinterpret_cast<const float4 *>(qv + m * N + c0);
-#pragma unroll
-                    for (int e4 = 0; e4 < EPC / 4; ++e4) {
-                        const float4 w = q4[e4];
-                        acc[m] = fmaf(v[4 * e4], w.x, acc[m]);
-                        acc[m] = fmaf(v[4 * e4 + 1], w.y, acc[m]);
-                        acc[m] = fmaf(v[4 * e4 + 2], w.z, acc[m]);
-                        acc[m] = fmaf(v[4 * e4 + 3], w.w, acc[m]);
-                    }
-                }
-            }
-#pragma unroll
-            for (int m = 0; m < TQ; ++m) {
-                const float d = group_sum<LPR>(acc[m]);
-                if (q == 0 && valid && m < T)
-                    sdot[r * TQ + m] = (RK == SK_FP8) ? d * ssc[r] : d;
-            }
+    if (!stream_first) {
+        if (RK == SK_FP8) {  // the row scales must have landed before the first dot is scaled
+            cp_async_wait_all();
+            __syncthreads();
         }
+        stream();
     }
     cp_async_wait_all();
     __syncthreads();
