@@ -817,7 +817,7 @@ __global__ void __launch_bounds__(kThreads) m2_eager_kernel(const M2Args a) {
 // computes (the same operations in the same order).  Requires P <= 8 rows per
 // thread x (kThreads / (N / 4)) and an even number of heads per group.
 template <int N, int SK>
-__global__ void __launch_bounds__(kThreads, SK == SK_FP8 ? 2 : 3) m2_eager_decode2_kernel(const M2Args a) {
+__global__ void __launch_bounds__(kThreads, SK == SK_FP8 ? 2 : 4) m2_eager_decode2_kernel(const M2Args a) {
     constexpr int TPR4 = N / 4;
     constexpr int RPP4 = kThreads / TPR4;
     constexpr int RB = 8;

@@ -45,6 +45,7 @@ constexpr int kQ = 128;          // chunk length = MMA M
 constexpr int kN = 128;          // dstate = MMA M of the state update
 constexpr int kPT = 256;         // threads per CTA: two halves of 128, one lane (row) each
 constexpr int kTileQN = kQ * kN * 2;  // one [128 x 128] bf16 tile
+constexpr float kLog2e = 1.4426950408889634f;
 
 struct PrefillArgs {
     int B, H, P, G, T, dt_scales;
@@ -61,7 +62,7 @@ struct PrefillArgs {
 
 // Shared memory (bytes from a 1024-aligned base).
 struct PrefillLay {
-    int C, Bk, Bt, Xt, XwHi, XwLo, SHi, SLo, lam, w, red, bar, tslot, bytes;
+    int C, Bk, Bt, Xt, XwHi, XwLo, SHi, SLo, lam, lam2, w, red, bar, tslot, bytes;
 };
 __host__ __device__ inline PrefillLay prefill_lay(int P) {
     PrefillLay L{};
@@ -77,6 +78,7 @@ __host__ __device__ inline PrefillLay prefill_lay(int P) {
     L.SHi = o;  o += sp;        // S hi [P rows, K = N]
     L.SLo = o;  o += sp;        // S lo
     L.lam = o;  o += kQ * 4;    // Lam_i
+    L.lam2 = o; o += kQ * 4;    // Lam_i log2(e)
     L.w = o;    o += kQ * 4;    // s_j (dt or 1)
     L.red = o;  o += 64;        // cross-warp scan carries
     L.bar = o;  o += 16;        // mbarrier
@@ -115,6 +117,7 @@ __global__ void __launch_bounds__(kPT, 1) m2_prefill_kernel(const PrefillArgs a)
     uint8_t *sXwHi = sm + Ly.XwHi, *sXwLo = sm + Ly.XwLo, *sSHi = sm + Ly.SHi, *sSLo = sm + Ly.SLo;
     uint8_t *sMHi = sBk, *sMLo = sBt;
     float *slam = reinterpret_cast<float *>(sm + Ly.lam);
+    float *slam2 = reinterpret_cast<float *>(sm + Ly.lam2);  // Lam log2(e): e^{Lam_i - Lam_j} = 2^{Lam2_i - Lam2_j}
     float *sw = reinterpret_cast<float *>(sm + Ly.w);
     float *sred = reinterpret_cast<float *>(sm + Ly.red);
     uint64_t *bar = reinterpret_cast<uint64_t *>(sm + Ly.bar);
@@ -193,6 +196,7 @@ __global__ void __launch_bounds__(kPT, 1) m2_prefill_kernel(const PrefillArgs a)
         const float lam = v + carry;
         if (half == 0) {
             slam[i] = lam;
+            slam2[i] = lam * kLog2e;
             sw[i] = live ? (a.dt_scales ? dti : 1.f) : 0.f;
         }
         __syncthreads();
@@ -273,7 +277,20 @@ __global__ void __launch_bounds__(kPT, 1) m2_prefill_kernel(const PrefillArgs a)
         tc_fence_after();
 
         // (C) M = tril(e^{Lam_i - Lam_j}) (.) CB (.) s_j as (hi, lo): row i, this half's 64 columns j.
+        //     A warp holds rows 32 (w mod 4) .. + 31: a 32-column block wholly above their
+        //     diagonal is zero and skips the exponentials (2^{Lam2_i - Lam2_j} elsewhere).
+        const float lam2 = lam * kLog2e;
+        const int warp_last_row = 32 * (warp & 3) + 31;
         for (int j0 = half * 64; j0 < half * 64 + 64; j0 += 32) {
+            if (j0 > warp_last_row) {  // warp-uniform
+#pragma unroll
+                for (int ch = 0; ch < 4; ++ch) {
+                    const int chunk = (j0 >> 3) + ch;
+                    *reinterpret_cast<uint4 *>(sMHi + sw128_chunk(i, chunk, kQ)) = make_uint4(0, 0, 0, 0);
+                    *reinterpret_cast<uint4 *>(sMLo + sw128_chunk(i, chunk, kQ)) = make_uint4(0, 0, 0, 0);
+                }
+                continue;
+            }
             float cb[32];
             tmem_ld32(lane_base + cY1 + j0, cb);
 #pragma unroll
@@ -285,7 +302,7 @@ __global__ void __launch_bounds__(kPT, 1) m2_prefill_kernel(const PrefillArgs a)
 #pragma unroll
                     for (int u = 0; u < 2; ++u) {
                         const int jj = 8 * ch + 2 * e2 + u, j = j0 + jj;
-                        m2[u] = (j <= i) ? expf(lam - slam[j]) * cb[jj] * sw[j] : 0.f;
+                        m2[u] = (j <= i) ? exp2f(lam2 - slam2[j]) * cb[jj] * sw[j] : 0.f;
                     }
                     __nv_bfloat16 h0, l0, h1, l1;
                     split_bf16(m2[0], h0, l0);
