@@ -145,26 +145,6 @@ __device__ __forceinline__ void gdn_stage_new(const GArgs &a, const GSmem &s, in
     if (tid < T) s.sbe[W + tid] = a.beta[(int64_t)(b * T + tid) * H + h];
 }
 
-// Packed pairs of fp32 (sm_100 .f32x2 arithmetic): one instruction updates two elements.
-__device__ __forceinline__ unsigned long long f2_pack(float a, float b) {
-    unsigned long long r;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
-    return r;
-}
-__device__ __forceinline__ void f2_unpack(unsigned long long v, float &a, float &b) {
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
-}
-__device__ __forceinline__ unsigned long long f2_fma(unsigned long long a, unsigned long long b, unsigned long long c) {
-    unsigned long long d;
-    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-    return d;
-}
-__device__ __forceinline__ unsigned long long f2_mul(unsigned long long a, unsigned long long b) {
-    unsigned long long d;
-    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-    return d;
-}
-
 // Apply entries [0, L0) (physical base..) to the NR = 4 rows a thread holds as
 // NPT-element lane segments (TPRF lanes per row).  Rows are independent; every
 // lane of the warp must call this.

@@ -601,18 +601,31 @@ __global__ void __launch_bounds__(kThreads, 3) m2_fold_kernel(const M2Args a, co
                 }
                 const float *Ur = U + (hh * L0) * P + p0;
                 const float *Br = Bf + 4 * q;
+                // Rank-L0 update on packed pairs: row i's columns (x, y) and (z, w)
+                // each take one .f32x2 FMA per entry with u_i broadcast to both halves.
+                unsigned long long vp[4][2];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    vp[i][0] = f2_pack(v[i].x, v[i].y);
+                    vp[i][1] = f2_pack(v[i].z, v[i].w);
+                }
 #pragma unroll 4
                 for (int e = 0; e < L0; ++e) {
                     const float4 u = *reinterpret_cast<const float4 *>(Ur + e * P);
                     const float4 bb = *reinterpret_cast<const float4 *>(Br + e * N);
-                    v[0].x = fmaf(u.x, bb.x, v[0].x); v[0].y = fmaf(u.x, bb.y, v[0].y);
-                    v[0].z = fmaf(u.x, bb.z, v[0].z); v[0].w = fmaf(u.x, bb.w, v[0].w);
-                    v[1].x = fmaf(u.y, bb.x, v[1].x); v[1].y = fmaf(u.y, bb.y, v[1].y);
-                    v[1].z = fmaf(u.y, bb.z, v[1].z); v[1].w = fmaf(u.y, bb.w, v[1].w);
-                    v[2].x = fmaf(u.z, bb.x, v[2].x); v[2].y = fmaf(u.z, bb.y, v[2].y);
-                    v[2].z = fmaf(u.z, bb.z, v[2].z); v[2].w = fmaf(u.z, bb.w, v[2].w);
-                    v[3].x = fmaf(u.w, bb.x, v[3].x); v[3].y = fmaf(u.w, bb.y, v[3].y);
-                    v[3].z = fmaf(u.w, bb.z, v[3].z); v[3].w = fmaf(u.w, bb.w, v[3].w);
+                    const unsigned long long b01 = f2_pack(bb.x, bb.y), b23 = f2_pack(bb.z, bb.w);
+                    const float uv[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const unsigned long long ui = f2_pack(uv[i], uv[i]);
+                        vp[i][0] = f2_fma(ui, b01, vp[i][0]);
+                        vp[i][1] = f2_fma(ui, b23, vp[i][1]);
+                    }
+                }
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    f2_unpack(vp[i][0], v[i].x, v[i].y);
+                    f2_unpack(vp[i][1], v[i].z, v[i].w);
                 }
             }
             // Every thread has its rows (the stage buffer is free again), and
