@@ -186,26 +186,6 @@ __device__ __forceinline__ float quad_rows_sum(float d0, float d1, float d2, flo
     return f;
 }
 
-// Packed pairs of fp32 (sm_100 .f32x2 arithmetic): one instruction updates two elements.
-__device__ __forceinline__ unsigned long long f2_pack(float a, float b) {
-    unsigned long long r;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
-    return r;
-}
-__device__ __forceinline__ void f2_unpack(unsigned long long v, float &a, float &b) {
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
-}
-__device__ __forceinline__ unsigned long long f2_fma(unsigned long long a, unsigned long long b, unsigned long long c) {
-    unsigned long long d;
-    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-    return d;
-}
-__device__ __forceinline__ unsigned long long f2_mul(unsigned long long a, unsigned long long b) {
-    unsigned long long d;
-    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-    return d;
-}
-
 __device__ __forceinline__ float ld_in(const void *p, int64_t i, int bf16) {
     return bf16 ? bf16_bits_to_float(reinterpret_cast<const uint16_t *>(p)[i])
                 : reinterpret_cast<const float *>(p)[i];

@@ -19,6 +19,7 @@
 //   s <- alpha s + (beta v[row] - alpha beta (s . k)) k.
 #pragma once
 #include "rssm_device.cuh"
+#include "rssm_pair.cuh"
 #include "rssm_internal.h"
 
 namespace rssm {

@@ -17,6 +17,7 @@
 // rewrites the whole state every token.
 #pragma once
 #include "rssm_device.cuh"
+#include "rssm_pair.cuh"
 #include "rssm_internal.h"
 #include "rssm_pipe.cuh"
 #include "rssm_read.cuh"
