@@ -22,9 +22,10 @@
 // two MMAs each, so every product keeps near-fp32 accuracy.  The state stays
 // in tensor memory, transposed (lane n, column p), across the chunks of a head.
 //
-// One CTA of 256 threads per (sequence, head): thread t owns tensor-memory lane
-// t mod 128 (token i of the chunk, or state column n) and half of that row's
-// columns, so two warps share each lane quarter.  Per chunk: (A) the threads issue
+// One CTA of 128 NG threads per (sequence, head): thread t owns tensor-memory
+// lane t mod 128 (token i of the chunk, or state column n) and one of NG column
+// groups of that row, so NG warps share each lane quarter (NG = 4 for headdim 64,
+// 2 otherwise: a group's p columns stay a multiple of 16).  Per chunk: (A) the threads issue
 // the chunk's global reads at once (C and B rows by cp.async into their
 // swizzled rows, x into registers), then stage x^T and (x w)^T, the state's
 // (hi, lo) copy and B^T in shared memory and rescale the state by e^{Lam_last}
@@ -43,7 +44,7 @@ namespace {
 
 constexpr int kQ = 128;          // chunk length = MMA M
 constexpr int kN = 128;          // dstate = MMA M of the state update
-constexpr int kPT = 256;         // threads per CTA: two halves of 128, one lane (row) each
+constexpr int kRows = 128;       // threads per column group: one tensor-memory lane (row) each
 constexpr int kTileQN = kQ * kN * 2;  // one [128 x 128] bf16 tile
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -100,16 +101,22 @@ __device__ __forceinline__ uint32_t pack2(float a, float b) {
     return *reinterpret_cast<uint32_t *>(&t);
 }
 
-template <int P>
-__global__ void __launch_bounds__(kPT, 1) m2_prefill_kernel(const PrefillArgs a) {
-    constexpr int PH = P / 2;  // p columns handled by each half of the CTA (a multiple of 16)
+template <int P, int NG>
+__global__ void __launch_bounds__(kRows * NG, 1) m2_prefill_kernel(const PrefillArgs a) {
+    constexpr int PH = P / NG;  // p columns handled by each column group (a multiple of 16)
+    static_assert(PH % 16 == 0, "a column group's p columns are loaded 16 at a time");
+    // headdim 64: x, x w and the state copy are written as MN-major tiles (row = token
+    // or state column, 128 bytes of p) and B is read MN-major by MMA4, so no operand
+    // is transposed element by element; one MN block, so its stride is never used.
+    constexpr bool kMN = (P == 64);
+    constexpr uint32_t kMNBlock = 1024;
     extern __shared__ __align__(1024) uint8_t psm[];
     // the swizzled tiles need a 1024-byte aligned base
     uint8_t *sm = psm + ((1024 - (smem_u32(psm) & 1023)) & 1023);
     const PrefillLay Ly = prefill_lay(P);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int row = tid & (kQ - 1);  // tensor-memory lane: token i of the chunk, or state column n
-    const int half = tid >> 7;       // which half of the columns this thread works on
+    const int grp = tid >> 7;        // which column group this thread works on
     const int b = blockIdx.y, h = blockIdx.x;
     const int H = a.H, G = a.G, T = a.T;
     const int g = h / (H / G);
@@ -137,7 +144,7 @@ __global__ void __launch_bounds__(kPT, 1) m2_prefill_kernel(const PrefillArgs a)
     const uint32_t tmem = *tslot;
     const uint32_t lane_base = tmem + ((uint32_t)(32 * (warp & 3)) << 16);  // this warp's 32 lanes
     const float Ah = a.A[h], Dh = a.D[h];
-    const int p_lo = half * PH;  // this thread's p columns: [p_lo, p_lo + PH)
+    const int p_lo = grp * PH;  // this thread's p columns: [p_lo, p_lo + PH)
     const int64_t head = (int64_t)b * H + h;
 
     // The initial state, transposed into tensor memory: lane n holds S0[:, n].
@@ -157,15 +164,15 @@ __global__ void __launch_bounds__(kPT, 1) m2_prefill_kernel(const PrefillArgs a)
         const bool live = i < Lc;
         const int64_t tok = (int64_t)b * T + t0 + i;
 
-        // (A) The chunk's global reads, all issued first: this half's 16-byte chunks
+        // (A) The chunk's global reads, all issued first: this group's 16-byte chunks
         //     of the C and B rows of token i by cp.async straight into their K-major
-        //     rows (rows = tokens), this half's part of x row i and dt_i into registers.
+        //     rows (rows = tokens), this group's part of x row i and dt_i into registers.
         const uint8_t *Crow = reinterpret_cast<const uint8_t *>(a.Cm + (tok * G + g) * kN);
         const uint8_t *Brow = reinterpret_cast<const uint8_t *>(a.Bm + (tok * G + g) * kN);
-        constexpr int CH = kN / 16;  // row chunks per half
+        constexpr int CH = kN / 8 / NG;  // 16-byte row chunks per group
 #pragma unroll
         for (int k = 0; k < CH; ++k) {
-            const int ch = half * CH + k;
+            const int ch = grp * CH + k;
             if (live) {
                 cp_async16(sC + sw128_chunk(i, ch, kQ), Crow + 16 * ch);
                 cp_async16(sBk + sw128_chunk(i, ch, kQ), Brow + 16 * ch);
@@ -181,20 +188,20 @@ __global__ void __launch_bounds__(kPT, 1) m2_prefill_kernel(const PrefillArgs a)
         for (int k = 0; k < PH / 8; ++k) xv[k] = live ? Xrow[k] : make_uint4(0, 0, 0, 0);
         const float dti = live ? a.dt[tok * H + h] : 0.f;
 
-        // Prefix sums of dt*A over the chunk (padding tokens add nothing); both
-        // halves scan, the first publishes.
+        // Prefix sums of dt*A over the chunk (padding tokens add nothing); every
+        // group scans, the first publishes.
         float v = dti * Ah;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const float u = __shfl_up_sync(0xffffffffu, v, o);
             if (lane >= o) v += u;
         }
-        if (half == 0 && lane == 31) sred[warp] = v;
+        if (grp == 0 && lane == 31) sred[warp] = v;
         __syncthreads();
         float carry = 0.f;
         for (int w2 = 0; w2 < (warp & 3); ++w2) carry += sred[w2];
         const float lam = v + carry;
-        if (half == 0) {
+        if (grp == 0) {
             slam[i] = lam;
             slam2[i] = lam * kLog2e;
             sw[i] = live ? (a.dt_scales ? dti : 1.f) : 0.f;
@@ -202,47 +209,89 @@ __global__ void __launch_bounds__(kPT, 1) m2_prefill_kernel(const PrefillArgs a)
         __syncthreads();
         const float lam_last = slam[kQ - 1];
 
-        // x^T and (x w)^T columns of this half's p (w_i = e^{Lam_last - Lam_i} s_i), as (hi, lo).
+        // x and x w (w_i = e^{Lam_last - Lam_i} s_i, as (hi, lo)) for this group's p:
+        // with headdim 64 as row i of MN-major tiles (one 16-byte chunk per 8 p),
+        // otherwise as columns of the transposed K-major tiles.
         const float wi = live ? expf(lam_last - lam) * sw[i] : 0.f;
 #pragma unroll
         for (int k = 0; k < PH / 8; ++k) {
             const __nv_bfloat16 *xe = reinterpret_cast<const __nv_bfloat16 *>(&xv[k]);
+            if constexpr (kMN) {
+                uint32_t hw[4], lw[4];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const int p = p_lo + 8 * k + e;
-                *reinterpret_cast<__nv_bfloat16 *>(sXt + sw128_off(p, i, P)) = xe[e];
-                __nv_bfloat16 hi, lo;
-                split_bf16(__bfloat162float(xe[e]) * wi, hi, lo);
-                *reinterpret_cast<__nv_bfloat16 *>(sXwHi + sw128_off(p, i, P)) = hi;
-                *reinterpret_cast<__nv_bfloat16 *>(sXwLo + sw128_off(p, i, P)) = lo;
+                for (int e2 = 0; e2 < 4; ++e2) {
+                    __nv_bfloat16 h0, l0, h1, l1;
+                    split_bf16(__bfloat162float(xe[2 * e2]) * wi, h0, l0);
+                    split_bf16(__bfloat162float(xe[2 * e2 + 1]) * wi, h1, l1);
+                    hw[e2] = pack2(__bfloat162float(h0), __bfloat162float(h1));
+                    lw[e2] = pack2(__bfloat162float(l0), __bfloat162float(l1));
+                }
+                const uint32_t off = sw128_chunk(i, (p_lo >> 3) + k, kQ);
+                *reinterpret_cast<uint4 *>(sXt + off) = xv[k];
+                *reinterpret_cast<uint4 *>(sXwHi + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+                *reinterpret_cast<uint4 *>(sXwLo + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+            } else {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const int p = p_lo + 8 * k + e;
+                    *reinterpret_cast<__nv_bfloat16 *>(sXt + sw128_off(p, i, P)) = xe[e];
+                    __nv_bfloat16 hi, lo;
+                    split_bf16(__bfloat162float(xe[e]) * wi, hi, lo);
+                    *reinterpret_cast<__nv_bfloat16 *>(sXwHi + sw128_off(p, i, P)) = hi;
+                    *reinterpret_cast<__nv_bfloat16 *>(sXwLo + sw128_off(p, i, P)) = lo;
+                }
             }
         }
-        // The state at the chunk's start: (hi, lo) copy for MMA3 (S rows p, K = n),
-        // and e^{Lam_last} S back into tensor memory for MMA4 to accumulate onto.
+        // The state at the chunk's start: (hi, lo) copy for MMA3 (S rows p, K = n;
+        // with headdim 64 MN-major, row n holding this lane's p run), and
+        // e^{Lam_last} S back into tensor memory for MMA4 to accumulate onto.
         const float dec = expf(lam_last);
         for (int j0 = 0; j0 < PH; j0 += 16) {
             float st[16];
             tmem_ld16(lane_base + cS + p_lo + j0, st);
+            if constexpr (kMN) {
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                __nv_bfloat16 hi, lo;
-                split_bf16(st[j], hi, lo);
-                *reinterpret_cast<__nv_bfloat16 *>(sSHi + sw128_off(p_lo + j0 + j, row, P)) = hi;
-                *reinterpret_cast<__nv_bfloat16 *>(sSLo + sw128_off(p_lo + j0 + j, row, P)) = lo;
-                st[j] *= dec;
+                for (int c8 = 0; c8 < 2; ++c8) {
+                    uint32_t hw[4], lw[4];
+#pragma unroll
+                    for (int e2 = 0; e2 < 4; ++e2) {
+                        __nv_bfloat16 h0, l0, h1, l1;
+                        split_bf16(st[8 * c8 + 2 * e2], h0, l0);
+                        split_bf16(st[8 * c8 + 2 * e2 + 1], h1, l1);
+                        hw[e2] = pack2(__bfloat162float(h0), __bfloat162float(h1));
+                        lw[e2] = pack2(__bfloat162float(l0), __bfloat162float(l1));
+                    }
+                    const uint32_t off = sw128_chunk(row, ((p_lo + j0) >> 3) + c8, kN);
+                    *reinterpret_cast<uint4 *>(sSHi + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+                    *reinterpret_cast<uint4 *>(sSLo + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+                }
+#pragma unroll
+                for (int j = 0; j < 16; ++j) st[j] *= dec;
+            } else {
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    __nv_bfloat16 hi, lo;
+                    split_bf16(st[j], hi, lo);
+                    *reinterpret_cast<__nv_bfloat16 *>(sSHi + sw128_off(p_lo + j0 + j, row, P)) = hi;
+                    *reinterpret_cast<__nv_bfloat16 *>(sSLo + sw128_off(p_lo + j0 + j, row, P)) = lo;
+                    st[j] *= dec;
+                }
             }
             tmem_st16(lane_base + cS + p_lo + j0, st);
         }
-        // B^T columns from this thread's own B chunks once they have landed.
         cp_async_wait_all();
+        // B^T columns from this thread's own B chunks once they have landed (with
+        // headdim 64 MMA4 reads the B tile itself MN-major).
+        if constexpr (!kMN) {
 #pragma unroll
-        for (int k = 0; k < CH; ++k) {
-            const int ch = half * CH + k;
-            const uint4 bv = *reinterpret_cast<const uint4 *>(sBk + sw128_chunk(i, ch, kQ));
-            const __nv_bfloat16 *be = reinterpret_cast<const __nv_bfloat16 *>(&bv);
+            for (int k = 0; k < CH; ++k) {
+                const int ch = grp * CH + k;
+                const uint4 bv = *reinterpret_cast<const uint4 *>(sBk + sw128_chunk(i, ch, kQ));
+                const __nv_bfloat16 *be = reinterpret_cast<const __nv_bfloat16 *>(&bv);
 #pragma unroll
-            for (int e = 0; e < 8; ++e)
-                *reinterpret_cast<__nv_bfloat16 *>(sBt + sw128_off(8 * ch + e, i, kN)) = be[e];
+                for (int e = 0; e < 8; ++e)
+                    *reinterpret_cast<__nv_bfloat16 *>(sBt + sw128_off(8 * ch + e, i, kN)) = be[e];
+            }
         }
         fence_async_smem();
         tc_fence_before();
@@ -257,13 +306,16 @@ __global__ void __launch_bounds__(kPT, 1) m2_prefill_kernel(const PrefillArgs a)
             for (int hl = 0; hl < 2; ++hl) {
                 const uint32_t aS = smem_u32(hl ? sSLo : sSHi);
                 for (int ks = 0; ks < kN / 16; ++ks)
-                    umma_bf16(tmem + cY2, sw128_desc(aC, kQ, ks), sw128_desc(aS, P, ks), idesc_bf16_f32(kQ, P),
-                              hl > 0 || ks > 0);
+                    umma_bf16(tmem + cY2, sw128_desc(aC, kQ, ks),
+                              kMN ? sw128_mn_desc(aS, kMNBlock, ks) : sw128_desc(aS, P, ks),
+                              idesc_bf16_f32_mn(kQ, P, false, kMN), hl > 0 || ks > 0);
             }
             for (int hl = 0; hl < 2; ++hl) {
                 const uint32_t aX = smem_u32(hl ? sXwLo : sXwHi);
                 for (int ks = 0; ks < kQ / 16; ++ks)
-                    umma_bf16(tmem + cS, sw128_desc(aBt, kN, ks), sw128_desc(aX, P, ks), idesc_bf16_f32(kN, P), true);
+                    umma_bf16(tmem + cS, kMN ? sw128_mn_desc(aB, kQ * 128, ks) : sw128_desc(aBt, kN, ks),
+                              kMN ? sw128_mn_desc(aX, kMNBlock, ks) : sw128_desc(aX, P, ks),
+                              idesc_bf16_f32_mn(kN, P, kMN, kMN), true);
             }
             umma_commit(bar);
         }
@@ -276,12 +328,12 @@ __global__ void __launch_bounds__(kPT, 1) m2_prefill_kernel(const PrefillArgs a)
         }
         tc_fence_after();
 
-        // (C) M = tril(e^{Lam_i - Lam_j}) (.) CB (.) s_j as (hi, lo): row i, this half's 64 columns j.
+        // (C) M = tril(e^{Lam_i - Lam_j}) (.) CB (.) s_j as (hi, lo): row i, this group's kQ / NG columns j.
         //     A warp holds rows 32 (w mod 4) .. + 31: a 32-column block wholly above their
         //     diagonal is zero and skips the exponentials (2^{Lam2_i - Lam2_j} elsewhere).
         const float lam2 = lam * kLog2e;
         const int warp_last_row = 32 * (warp & 3) + 31;
-        for (int j0 = half * 64; j0 < half * 64 + 64; j0 += 32) {
+        for (int j0 = grp * (kQ / NG); j0 < (grp + 1) * (kQ / NG); j0 += 32) {
             if (j0 > warp_last_row) {  // warp-uniform
 #pragma unroll
                 for (int ch = 0; ch < 4; ++ch) {
@@ -326,8 +378,9 @@ __global__ void __launch_bounds__(kPT, 1) m2_prefill_kernel(const PrefillArgs a)
             for (int hl = 0; hl < 2; ++hl) {
                 const uint32_t aM = smem_u32(hl ? sMLo : sMHi);
                 for (int ks = 0; ks < kQ / 16; ++ks)
-                    umma_bf16(tmem + cY1, sw128_desc(aM, kQ, ks), sw128_desc(aX, P, ks), idesc_bf16_f32(kQ, P),
-                              hl > 0 || ks > 0);
+                    umma_bf16(tmem + cY1, sw128_desc(aM, kQ, ks),
+                              kMN ? sw128_mn_desc(aX, kMNBlock, ks) : sw128_desc(aX, P, ks),
+                              idesc_bf16_f32_mn(kQ, P, false, kMN), hl > 0 || ks > 0);
             }
             umma_commit(bar);
         }
@@ -340,7 +393,7 @@ __global__ void __launch_bounds__(kPT, 1) m2_prefill_kernel(const PrefillArgs a)
         }
         tc_fence_after();
 
-        // (E) y_i = Y_intra + e^{Lam_i} Y_inter + D x_i over this half's p.
+        // (E) y_i = Y_intra + e^{Lam_i} Y_inter + D x_i over this group's p.
         const float di = expf(lam);
         for (int j0 = 0; j0 < PH; j0 += 16) {
             float y1[16], y2[16];
@@ -408,9 +461,11 @@ extern "C" RSSM_API rssm_status rssm_mamba2_prefill(const rssm_prefill_config *c
     a.Bm = (const __nv_bfloat16 *)in->Bm; a.Cm = (const __nv_bfloat16 *)in->Cm;
     a.A = A; a.D = D; a.S0 = S0; a.y = y; a.S_out = S_out; a.err = (int *)dev_error;
     const size_t smem = prefill_smem_bytes(c.headdim);
-    auto k = c.headdim == 32 ? m2_prefill_kernel<32> : (c.headdim == 64 ? m2_prefill_kernel<64> : m2_prefill_kernel<96>);
+    const int ng = c.headdim == 64 ? 4 : 2;
+    auto k = c.headdim == 32 ? m2_prefill_kernel<32, 2>
+                             : (c.headdim == 64 ? m2_prefill_kernel<64, 4> : m2_prefill_kernel<96, 2>);
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return RSSM_ECUDA;
-    k<<<dim3(c.nheads, c.batch), kPT, smem, (cudaStream_t)stream>>>(a);
+    k<<<dim3(c.nheads, c.batch), kRows * ng, smem, (cudaStream_t)stream>>>(a);
     return cudaGetLastError() == cudaSuccess ? RSSM_OK : RSSM_ECUDA;
 }

@@ -3,8 +3,8 @@
 // an fp32 accumulator in tensor memory, its completion on an mbarrier, and
 // tensor-memory loads and stores.  Inline PTX; no library code.
 //
-// Operand tiles live in shared memory in the K-major layout with the 128-byte
-// swizzle: a tile of R rows (R a multiple of 8) and K bf16 columns (K a
+// Operand tiles live in shared memory in the 128-byte-swizzled layout, read
+// K-major or MN-major.  K-major: a tile of R rows (R a multiple of 8) and K bf16 columns (K a
 // multiple of 64) is stored as K/64 column blocks of R x 128 bytes; inside a
 // block, row r occupies bytes [r*128, r*128 + 128) of its 8-row group
 // (groups 1024 bytes apart) and its 16-byte chunk c sits at chunk c ^ (r % 8).
@@ -43,10 +43,28 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t tile_saddr, int R, int k
     return d;
 }
 
+// The same 128-byte-swizzled atoms read MN-major: K rows of 64 MN elements
+// (128 bytes; element (k, m) of an MN block sits where a K-major tile keeps
+// element (row k, column m)), 8-row K groups 1024 bytes apart, MN blocks of 64
+// elements `mn_stride` bytes apart.  Descriptor of the K slice [16 ks, 16 ks + 16).
+__device__ __forceinline__ uint64_t sw128_mn_desc(uint32_t tile_saddr, uint32_t mn_stride, int ks) {
+    const uint32_t start = tile_saddr + (uint32_t)ks * 2048u;
+    uint64_t d = (uint64_t)((start >> 4) & 0x3FFFu);
+    d |= (uint64_t)((mn_stride >> 4) & 0x3FFFu) << 16;  // leading-dimension offset: MN blocks
+    d |= (uint64_t)(1024 >> 4) << 32;                    // stride-dimension offset: 8-row K groups
+    d |= (uint64_t)1 << 46;                              // descriptor version
+    d |= (uint64_t)2 << 61;                              // 128-byte swizzle
+    return d;
+}
+
 // Instruction descriptor of kind::f16 with bf16 A and B (both K-major) and an
 // fp32 accumulator, M x N.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
     return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+// The same with A and / or B read MN-major (the descriptor's transpose bits).
+__host__ __device__ constexpr uint32_t idesc_bf16_f32_mn(int M, int N, bool a_mn, bool b_mn) {
+    return idesc_bf16_f32(M, N) | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16);
 }
 
 // D[tmem] (+)= A[desc] * B[desc]^T, issued by one thread.
