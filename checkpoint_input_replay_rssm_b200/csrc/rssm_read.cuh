@@ -112,14 +112,11 @@ __global__ void __launch_bounds__(kThreads, TQ == 1 ? 4 : 2) replay_read_kernel(
 
     // 1. First round of read-copy chunks.
     uint4 rv[MAXC];
-    auto issue = [&](int pass0) {
+    auto issue_pass = [&](int pass, int off) {  // the pass's chunks into rv[off ..]
+        const int r = pass * RPP + rrow;
 #pragma unroll
-        for (int j = 0; j < PPR; ++j) {
-            const int r = (pass0 + j) * RPP + rrow;
-#pragma unroll
-            for (int k = 0; k < CPL; ++k)
-                if (r < nrows) rv[j * CPL + k] = ld_stream(tile + ((size_t)r * TPR + q + LPR * k) * 16);
-        }
+        for (int k = 0; k < CPL; ++k)
+            if (r < nrows) rv[off + k] = ld_stream(tile + ((size_t)r * TPR + q + LPR * k) * 16);
     };
     bool skip_copy = false;  // folded in this call: served by the flush kernel
     if (!a.early) {          // a flush kernel ran in this call
@@ -127,7 +124,10 @@ __global__ void __launch_bounds__(kThreads, TQ == 1 ? 4 : 2) replay_read_kernel(
         __syncthreads();
         skip_copy = sinfo[2] != 0;
     }
-    if (!skip_copy) issue(0);
+    if (!skip_copy) {
+#pragma unroll
+        for (int j = 0; j < PPR; ++j) issue_pass(j, j * CPL);
+    }
     // The read copy, its fp8 row scales and (for Mamba-2) the queries are not
     // written by the prep kernel.  When no flush kernel runs in this call and the
     // queries are the caller's input, every round of the stream is dotted before
@@ -188,46 +188,61 @@ __global__ void __launch_bounds__(kThreads, TQ == 1 ? 4 : 2) replay_read_kernel(
             sdec[hh * TQ + m] = a.dec[(row0 + hh) * a.TQmax + m];
         }
     };
-    // The rows dotted with their query, round after round of the copy.
+    // The rows dotted with their query, round after round of the copy.  A round
+    // is two halves; a half's next chunks go out as soon as it has been dotted,
+    // so the other half's loads are in flight while it is.
+    auto dot_pass = [&](int pass, int off) {
+        const int r = pass * RPP + rrow;
+        const bool valid = r < nrows;
+        float acc[TQ];
+#pragma unroll
+        for (int m = 0; m < TQ; ++m) acc[m] = 0.f;
+        const float *qv = sq + (shared_q ? 0 : (valid ? r / P : 0)) * TQ * N;
+#pragma unroll
+        for (int k = 0; k < CPL; ++k) {
+            float v[EPC];
+            if (valid) unpack<RK>(rv[off + k], v);
+            else {
+#pragma unroll
+                for (int e = 0; e < EPC; ++e) v[e] = 0.f;
+            }
+            const int c0 = (q + LPR * k) * EPC;
+#pragma unroll
+            for (int m = 0; m < TQ; ++m) {
+                const float4 *q4 = reinterpret_cast<const float4 *>(qv + m * N + c0);
+#pragma unroll
+                for (int e4 = 0; e4 < EPC / 4; ++e4) {
+                    const float4 w = q4[e4];
+                    acc[m] = fmaf(v[4 * e4], w.x, acc[m]);
+                    acc[m] = fmaf(v[4 * e4 + 1], w.y, acc[m]);
+                    acc[m] = fmaf(v[4 * e4 + 2], w.z, acc[m]);
+                    acc[m] = fmaf(v[4 * e4 + 3], w.w, acc[m]);
+                }
+            }
+        }
+#pragma unroll
+        for (int m = 0; m < TQ; ++m) {
+            const float d = group_sum<LPR>(acc[m]);
+            if (q == 0 && valid && m < T)
+                sdot[r * TQ + m] = (RK == SK_FP8) ? d * ssc[r] : d;
+        }
+    };
     auto stream = [&]() {
-        for (int pass0 = 0; pass0 * RPP < nrows; pass0 += PPR) {
-            if (pass0 > 0) issue(pass0);
+        constexpr int HP = PPR / 2;  // passes in a round's first half (0: one pass per round)
+        const int npass = (nrows + RPP - 1) / RPP;
+        for (int p0 = 0; p0 < npass; p0 += PPR) {
+            const bool more = p0 + PPR < npass;
 #pragma unroll
-            for (int j = 0; j < PPR; ++j) {
-                const int r = (pass0 + j) * RPP + rrow;
-                const bool valid = r < nrows;
-                float acc[TQ];
+            for (int j = 0; j < HP; ++j) dot_pass(p0 + j, j * CPL);
+            if (more) {
 #pragma unroll
-                for (int m = 0; m < TQ; ++m) acc[m] = 0.f;
-                const float *qv = sq + (shared_q ? 0 : (valid ? r / P : 0)) * TQ * N;
+                for (int j = 0; j < HP; ++j) issue_pass(p0 + PPR + j, j * CPL);
+            }
 #pragma unroll
-                for (int k = 0; k < CPL; ++k) {
-                    float v[EPC];
-                    if (valid) unpack<RK>(rv[j * CPL + k], v);
-                    else {
+            for (int j = HP; j < PPR; ++j) dot_pass(p0 + j, j * CPL);
+            if (more) {
 #pragma unroll
-                        for (int e = 0; e < EPC; ++e) v[e] = 0.f;
-                    }
-                    const int c0 = (q + LPR * k) * EPC;
-#pragma unroll
-                    for (int m = 0; m < TQ; ++m) {
-                        const float4 *q4 = reinterpret_cast<const float4 *>(qv + m * N + c0);
-#pragma unroll
-                        for (int e4 = 0; e4 < EPC / 4; ++e4) {
-                            const float4 w = q4[e4];
-                            acc[m] = fmaf(v[4 * e4], w.x, acc[m]);
-                            acc[m] = fmaf(v[4 * e4 + 1], w.y, acc[m]);
-                            acc[m] = fmaf(v[4 * e4 + 2], w.z, acc[m]);
-                            acc[m] = fmaf(v[4 * e4 + 3], w.w, acc[m]);
-                        }
-                    }
-                }
-#pragma unroll
-                for (int m = 0; m < TQ; ++m) {
-                    const float d = group_sum<LPR>(acc[m]);
-                    if (q == 0 && valid && m < T)
-                        sdot[r * TQ + m] = (RK == SK_FP8) ? d * ssc[r] : d;
-                }
+                for (int j = HP; j < PPR; ++j) issue_pass(p0 + PPR + j, j * CPL);
             }
         }
     };
