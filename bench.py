@@ -423,29 +423,29 @@ def timed_loop(L, toks_dev, ys, K, W, sync, split=True):
     return total_ms, per, pre, read, launches, steady
 
 
-def e2e_loop(L, toks_host, K, W, sync):
+def e2e_loop(L, toks_host, K, W, sync, nbuf=4):
     """Public-API decode with host buffers: every step copies its inputs from pinned
     host memory to the device, decodes, and copies its output y back to pinned host
-    memory, all inside the timed region.  Two sets of device buffers alternate so
-    that step i's input copy (one copy stream) and step i-1's output copy (another)
-    run while the layer's stream decodes; events order each buffer's reuse."""
+    memory, all inside the timed region.  `nbuf` sets of device buffers rotate so
+    that later steps' input copies (one copy stream) and earlier steps' output copies
+    (another) run while the layer's stream decodes; events order each buffer's reuse."""
     import torch
 
     n = len(toks_host)
-    dev = [{k: torch.empty_like(v, device=L.device) for k, v in toks_host[0].items()} for _ in range(2)]
-    y = [torch.empty((L.B, 1, L.H, L.P), dtype=torch.float32, device=L.device) for _ in range(2)]
-    y_host = [torch.empty_like(y[0], device="cpu").pin_memory() for _ in range(2)]
+    dev = [{k: torch.empty_like(v, device=L.device) for k, v in toks_host[0].items()} for _ in range(nbuf)]
+    y = [torch.empty((L.B, 1, L.H, L.P), dtype=torch.float32, device=L.device) for _ in range(nbuf)]
+    y_host = [torch.empty_like(y[0], device="cpu").pin_memory() for _ in range(nbuf)]
     comp = torch.cuda.ExternalStream(L.stream) if not isinstance(L.stream, torch.cuda.Stream) else L.stream
     h2d_s, d2h_s = torch.cuda.Stream(L.device), torch.cuda.Stream(L.device)
     ev = lambda: torch.cuda.Event()
-    in_ready, in_free = [ev(), ev()], [ev(), ev()]
-    y_ready, y_free = [ev(), ev()], [ev(), ev()]
-    for j in range(2):  # every buffer starts free
+    in_ready, in_free = [ev() for _ in range(nbuf)], [ev() for _ in range(nbuf)]
+    y_ready, y_free = [ev() for _ in range(nbuf)], [ev() for _ in range(nbuf)]
+    for j in range(nbuf):  # every buffer starts free
         in_free[j].record(comp)
         y_free[j].record(d2h_s)
 
     def step(i):
-        j = i % 2
+        j = i % nbuf
         with torch.cuda.stream(h2d_s):
             h2d_s.wait_event(in_free[j])
             for k, v in toks_host[i % n].items():
@@ -580,6 +580,8 @@ def main():
     ap.add_argument("--no-kda", action="store_true", help="skip the Kimi Delta Attention leg")
     ap.add_argument("--no-hybrid", action="store_true", help="skip the synthetic hybrid-step leg")
     ap.add_argument("--no-prefill", action="store_true", help="skip the prefill leg")
+    ap.add_argument("--e2e-buffers", type=int, default=4,
+                    help="device buffer sets rotating in the end-to-end loop (2 or more)")
     ap.add_argument("--batch", type=int, default=WL.batch,
                     help="sequences per GPU (default: the workload's 256; smaller for profiling; applies to "
                          "the decode, GDN, KDA and prefill legs)")
@@ -645,7 +647,7 @@ def main():
 
     # e2e through the public API with host buffers (same layer, state re-imported)
     L.import_state(torch.from_numpy(consts["S0"]).to(device))
-    e2e_ms, h2d, d2h = e2e_loop(L, toks_host, K, W, sync)
+    e2e_ms, h2d, d2h = e2e_loop(L, toks_host, K, W, sync, nbuf=max(2, args.e2e_buffers))
     (e2e_ms,) = max_over_ranks(dist, [e2e_ms], device)
     assert L.status()[0] == 0, "device error in the end-to-end loop"
 
