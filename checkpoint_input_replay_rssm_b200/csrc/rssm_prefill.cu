@@ -122,7 +122,9 @@ __global__ void __launch_bounds__(kRows * NG, 1) m2_prefill_kernel(const Prefill
     const int g = h / (H / G);
     uint8_t *sC = sm + Ly.C, *sBk = sm + Ly.Bk, *sBt = sm + Ly.Bt, *sXt = sm + Ly.Xt;
     uint8_t *sXwHi = sm + Ly.XwHi, *sXwLo = sm + Ly.XwLo, *sSHi = sm + Ly.SHi, *sSLo = sm + Ly.SLo;
-    uint8_t *sMHi = sBk, *sMLo = sBt;
+    // M (hi, lo) for MMA2: over B and B^T; with headdim 64 (no B^T tile in use) over
+    // B^T and the (x w) pair, so that C and B are free for the next chunk's rows.
+    uint8_t *sMHi = kMN ? sBt : sBk, *sMLo = kMN ? sXwHi : sBt;
     float *slam = reinterpret_cast<float *>(sm + Ly.lam);
     float *slam2 = reinterpret_cast<float *>(sm + Ly.lam2);  // Lam log2(e): e^{Lam_i - Lam_j} = 2^{Lam2_i - Lam2_j}
     float *sw = reinterpret_cast<float *>(sm + Ly.w);
@@ -157,6 +159,27 @@ __global__ void __launch_bounds__(kRows * NG, 1) m2_prefill_kernel(const Prefill
 
     uint32_t phase = 0;
     bool failed = false;
+    constexpr int CH = kN / 8 / NG;  // 16-byte row chunks per group
+    // C and B rows of token `row` of chunk cc (this group's chunks), zeros past the prompt.
+    auto stage_cb = [&](int cc) {
+        const int tc0 = cc * kQ;
+        const bool lv = row < min(kQ, T - tc0);
+        const int64_t tk = (int64_t)b * T + tc0 + row;
+        const uint8_t *Crow = reinterpret_cast<const uint8_t *>(a.Cm + (tk * G + g) * kN);
+        const uint8_t *Brow = reinterpret_cast<const uint8_t *>(a.Bm + (tk * G + g) * kN);
+#pragma unroll
+        for (int k = 0; k < CH; ++k) {
+            const int ch = grp * CH + k;
+            if (lv) {
+                cp_async16(sC + sw128_chunk(row, ch, kQ), Crow + 16 * ch);
+                cp_async16(sBk + sw128_chunk(row, ch, kQ), Brow + 16 * ch);
+            } else {
+                *reinterpret_cast<uint4 *>(sC + sw128_chunk(row, ch, kQ)) = make_uint4(0, 0, 0, 0);
+                *reinterpret_cast<uint4 *>(sBk + sw128_chunk(row, ch, kQ)) = make_uint4(0, 0, 0, 0);
+            }
+        }
+        cp_async_commit();
+    };
     const int nchunks = (T + kQ - 1) / kQ;
     for (int c = 0; c < nchunks && !failed; ++c) {
         const int t0 = c * kQ, Lc = min(kQ, T - t0);
@@ -166,22 +189,9 @@ __global__ void __launch_bounds__(kRows * NG, 1) m2_prefill_kernel(const Prefill
 
         // (A) The chunk's global reads, all issued first: this group's 16-byte chunks
         //     of the C and B rows of token i by cp.async straight into their K-major
-        //     rows (rows = tokens), this group's part of x row i and dt_i into registers.
-        const uint8_t *Crow = reinterpret_cast<const uint8_t *>(a.Cm + (tok * G + g) * kN);
-        const uint8_t *Brow = reinterpret_cast<const uint8_t *>(a.Bm + (tok * G + g) * kN);
-        constexpr int CH = kN / 8 / NG;  // 16-byte row chunks per group
-#pragma unroll
-        for (int k = 0; k < CH; ++k) {
-            const int ch = grp * CH + k;
-            if (live) {
-                cp_async16(sC + sw128_chunk(i, ch, kQ), Crow + 16 * ch);
-                cp_async16(sBk + sw128_chunk(i, ch, kQ), Brow + 16 * ch);
-            } else {
-                *reinterpret_cast<uint4 *>(sC + sw128_chunk(i, ch, kQ)) = make_uint4(0, 0, 0, 0);
-                *reinterpret_cast<uint4 *>(sBk + sw128_chunk(i, ch, kQ)) = make_uint4(0, 0, 0, 0);
-            }
-        }
-        cp_async_commit();
+        //     rows (rows = tokens; with headdim 64 issued during the previous chunk),
+        //     this group's part of x row i and dt_i into registers.
+        if (!(kMN && c > 0)) stage_cb(c);
         uint4 xv[PH / 8];
         const uint4 *Xrow = reinterpret_cast<const uint4 *>(a.x + (tok * H + h) * P + p_lo);
 #pragma unroll
@@ -327,6 +337,11 @@ __global__ void __launch_bounds__(kRows * NG, 1) m2_prefill_kernel(const Prefill
             break;
         }
         tc_fence_after();
+        // The MMAs reading C and B have completed: with headdim 64 the next chunk's
+        // rows go into them now and land while this chunk finishes.
+        if constexpr (kMN) {
+            if (c + 1 < nchunks) stage_cb(c + 1);
+        }
 
         // (C) M = tril(e^{Lam_i - Lam_j}) (.) CB (.) s_j as (hi, lo): row i, this group's kQ / NG columns j.
         //     A warp holds rows 32 (w mod 4) .. + 31: a 32-column block wholly above their
@@ -420,6 +435,7 @@ __global__ void __launch_bounds__(kRows * NG, 1) m2_prefill_kernel(const Prefill
         tc_fence_after();
     }
 
+    cp_async_wait_all();  // a chunk's rows still in flight after a failed wait
     if (failed) {
         if (tid == 0) report_err(a.err, DEV_PIPE_TIMEOUT, b, h, 0);
     } else {
