@@ -24,14 +24,16 @@
 //
 // One CTA of 128 NG threads per (sequence, head): thread t owns tensor-memory
 // lane t mod 128 (token i of the chunk, or state column n) and one of NG column
-// groups of that row, so NG warps share each lane quarter (NG = 4 for headdim 64,
-// 2 otherwise: a group's p columns stay a multiple of 16).  Per chunk: (A) the threads issue
-// the chunk's global reads at once (C and B rows by cp.async into their
-// swizzled rows, x into registers), then stage x^T and (x w)^T, the state's
-// (hi, lo) copy and B^T in shared memory and rescale the state by e^{Lam_last}
-// in place; (B) one thread issues
-// MMA1, MMA3 and MMA4; (C) the threads turn CB into M (hi, lo) in the space B
-// and B^T occupied; (D) one thread issues MMA2; (E) the threads write y.  Waits
+// groups of that row, so NG warps share each lane quarter (NG = 4 for headdim
+// 64, 2 otherwise: a group's p columns stay a multiple of 16).  Per chunk:
+// (A) the threads issue the chunk's global reads at once (C and B rows by
+// cp.async into their swizzled rows, x into registers), then stage x and (x w),
+// the state's (hi, lo) copy and, below headdim 64, B^T in shared memory -- at
+// headdim 64 as MN-major tiles written 16 bytes at a time, otherwise transposed
+// into K-major tiles -- and rescale the state by e^{Lam_last} in place; (B) one
+// thread issues MMA1, MMA3 and MMA4; (C) the threads turn CB into M (hi, lo)
+// (over B and B^T; at headdim 64 over B^T and (x w), while the next chunk's C
+// and B rows land); (D) one thread issues MMA2; (E) the threads write y.  Waits
 // on MMA completion are bounded (2 s) and report RSSM_DEV_PIPE_TIMEOUT.
 #include <cuda_bf16.h>
 
