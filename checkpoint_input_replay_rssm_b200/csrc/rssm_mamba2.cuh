@@ -915,6 +915,122 @@ __global__ void __launch_bounds__(kThreads, SK == SK_FP8 ? 2 : 4) m2_eager_decod
         a.y[(int64_t)(b * H + h0) * P + i] = sdot[i] + a.D[h0 + i / P] * sx[i];
 }
 
+// Eager decode (T = 1) of an fp32 state as one stream: a persistent grid whose
+// CTAs walk the heads (b, h) gridDim apart.  Each head's P x N fp32 tile arrives
+// by one bulk copy into one of kEagerStages shared-memory stages, issued
+// kEagerStages - 1 heads ahead, so a CTA keeps up to two tiles in flight while it
+// updates the third; the update itself is what m2_eager_kernel computes (the
+// same operations in the same order), read from shared memory and written back
+// with 128-bit stores.  A head's x row, its group's B and C and its dt, A and D
+// are loaded into registers one head ahead.  Waits are bounded.
+constexpr int kEagerStages = 3;
+template <int N>
+__global__ void __launch_bounds__(kThreads, 2) m2_eager_stream_kernel(const M2Args a) {
+    constexpr int TPR4 = N / 4;            // threads per state row (one float4 each)
+    constexpr int RPP4 = kThreads / TPR4;  // rows per pass
+    extern __shared__ __align__(128) uint8_t esm[];
+    const int tid = threadIdx.x;
+    const int H = a.H, P = a.P, G = a.G;
+    const int hpg = H / G;
+    const int nitems = a.B * H;
+    const int tile = P * N;  // floats
+    float *stg = reinterpret_cast<float *>(esm);                 // [kEagerStages][P][N]
+    float *sx = stg + kEagerStages * tile;                        // [2][P]
+    float *sB = sx + 2 * pad4(P);                                 // [2][N]
+    float *sC = sB + 2 * N;                                       // [2][N]
+    float *sdot = sC + 2 * N;                                     // [P]
+    float *ssc = sdot + pad4(P);                                  // [2][4]: decay, input scale, D
+    uint64_t *bar = reinterpret_cast<uint64_t *>(ssc + 8);        // [kEagerStages]
+    const int c4 = tid % TPR4, q0 = tid / TPR4;
+
+    if (tid == 0) {
+        for (int k = 0; k < kEagerStages; ++k) mbar_init(&bar[k], 1);
+        mbar_init_fence();
+    }
+    __syncthreads();
+    auto issue = [&](int li) {  // thread 0: the tile of the CTA's li-th head into stage li % kEagerStages
+        const int it = blockIdx.x + li * gridDim.x;
+        if (it >= nitems) return;
+        const int k = li % kEagerStages;
+        mbar_arrive_expect_tx(&bar[k], (uint32_t)(tile * 4));
+        bulk_g2s(stg + k * tile, a.ckpt + (int64_t)it * tile, (uint32_t)(tile * 4), &bar[k]);
+    };
+    if (tid == 0)
+        for (int li = 0; li < kEagerStages - 1; ++li) issue(li);
+
+    // The small inputs of head `it`, in registers: x[tid], B[tid], C[tid]; threads
+    // 0..2 hold the decay, the input scale and D.
+    float rx = 0.f, rB = 0.f, rC = 0.f, rs = 0.f;
+    auto load_small = [&](int it) {
+        if (it >= nitems) return;
+        const int b = it / H, h = it - b * H, g = h / hpg;
+        if (tid < P) rx = ld_in(a.x, (int64_t)it * P + tid, a.in_bf16);
+        if (tid < N) {
+            const int64_t src = ((int64_t)b * G + g) * N + tid;
+            rB = ld_in(a.Bm, src, a.in_bf16);
+            rC = ld_in(a.Cm, src, a.in_bf16);
+        }
+        if (tid == 0) rs = expf(a.dt[it] * a.A[h]);
+        if (tid == 1) rs = a.dt_scales ? a.dt[it] : 1.f;
+        if (tid == 2) rs = a.D[h];
+    };
+    load_small(blockIdx.x);
+
+    int li = 0;
+    for (int it = blockIdx.x; it < nitems; it += gridDim.x, ++li) {
+        const int b = it / H, h = it - b * H;
+        const int k = li % kEagerStages, sl = li & 1;
+        // This head's small inputs to shared memory; the next head's into registers.
+        if (tid < P) sx[sl * pad4(P) + tid] = rx;
+        if (tid < N) {
+            sB[sl * N + tid] = rB;
+            sC[sl * N + tid] = rC;
+        }
+        if (tid < 3) ssc[sl * 4 + tid] = rs;
+        load_small(it + gridDim.x);
+        if (tid == 0) {
+            issue(li + kEagerStages - 1);  // its stage was freed at the end of the previous head
+            if (h == 0) {  // no other CTA of an eager launch reads the sequence's counters
+                const int64_t s1 = a.c.seq_pos[b] + 1;
+                a.c.seq_pos[b] = s1;
+                a.c.ckpt_pos[b] = s1;
+            }
+        }
+        const bool got = mbar_wait(&bar[k], (uint32_t)((li / kEagerStages) & 1));
+        if (__syncthreads_or(!got)) {
+            if (tid == 0) {
+                report(a.c.err, DEV_PIPE_TIMEOUT, b, h, 0);
+                for (int j = 0; j < kEagerStages; ++j)  // copies still in flight land (bounded) before exit
+                    if (it + j * (int)gridDim.x < nitems)
+                        mbar_wait(&bar[(li + j) % kEagerStages], (uint32_t)(((li + j) / kEagerStages) & 1));
+            }
+            return;
+        }
+        const float am = ssc[sl * 4], sc_in = ssc[sl * 4 + 1];
+        const float4 Bq = reinterpret_cast<const float4 *>(sB + sl * N)[c4];
+        const float4 Cq = reinterpret_cast<const float4 *>(sC + sl * N)[c4];
+        const float *st = stg + k * tile;
+        float *dst = a.ckpt + (int64_t)it * tile;
+        for (int r = q0; r < P; r += RPP4) {
+            float4 v = *reinterpret_cast<const float4 *>(st + r * N + 4 * c4);
+            const float w = sc_in * sx[sl * pad4(P) + r];
+            v.x = fmaf(am, v.x, w * Bq.x); v.y = fmaf(am, v.y, w * Bq.y);
+            v.z = fmaf(am, v.z, w * Bq.z); v.w = fmaf(am, v.w, w * Bq.w);
+            float d = v.x * Cq.x + v.y * Cq.y + v.z * Cq.z + v.w * Cq.w;
+            d = group_sum<TPR4>(d);
+            if (c4 == 0) sdot[r] = d;  // output from the fp32 value
+            *reinterpret_cast<float4 *>(dst + r * N + 4 * c4) = v;
+        }
+        __syncthreads();  // the stage is free again and every row's dot is in sdot
+        if (tid < P) a.y[(int64_t)it * P + tid] = sdot[tid] + ssc[sl * 4 + 2] * sx[sl * pad4(P) + tid];
+    }
+}
+
+inline size_t m2_eager_stream_smem(int P, int N) {
+    return sizeof(float) * ((size_t)kEagerStages * P * N + 2 * pad4(P) + 4 * N + pad4(P) + 8) +
+           sizeof(uint64_t) * kEagerStages;
+}
+
 // ---------------------------------------------------------------------------
 // Host launchers.
 // ---------------------------------------------------------------------------
@@ -947,6 +1063,19 @@ inline cudaError_t launch_fold_t(const M2Args &a, const M2FoldLay &lay, int num_
 template <int N, int SK, int TQ>
 inline cudaError_t launch_eager_t(const M2Args &a, size_t smem, cudaStream_t st) {
     constexpr int kRows = 8 * (kThreads / (N / 4));  // state rows one pass of the two-head kernel covers
+    const size_t ssm = m2_eager_stream_smem(a.P, N);
+    if (SK == SK_F32 && TQ == 1 && a.op == OP_DECODE && a.T == 1 && a.P <= kThreads && ssm <= 112 * 1024) {
+        auto ks = m2_eager_stream_kernel<N>;
+        cudaError_t e = cudaFuncSetAttribute(ks, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ssm);
+        if (e != cudaSuccess) return e;
+        int dev = 0, sms = 0, occ = 0;
+        if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+        if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+        if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, ks, kThreads, ssm)) != cudaSuccess) return e;
+        const int items = a.B * a.H, cap = sms * (occ > 0 ? occ : 1);
+        ks<<<items < cap ? items : cap, kThreads, ssm, st>>>(a);
+        return cudaGetLastError();
+    }
     if (TQ == 1 && a.op == OP_DECODE && a.T == 1 && (a.H / a.G) % 2 == 0 && a.P <= kRows) {
         auto k2 = m2_eager_decode2_kernel<N, SK>;
         const int smem2 = (int)sizeof(float) * (2 * pad4(2 * a.P) + 2 * pad4(N) + 8);
