@@ -135,6 +135,19 @@ def test_eager_baselines(sd):
         assert worst_emu[sd] <= (2e-2 if sd == "bf16" else 6e-2), worst_emu
 
 
+def test_eager_stream_many_heads_per_cta():
+    """The streamed fp32 eager decode at 1 280 heads (about four per CTA of its
+    persistent grid, so every shared-memory stage is reused and its mbarrier phase
+    flips), 6 steps; six sequences against the fp64 eager oracle, the counters of
+    all of them against the plain count."""
+    wl = I.TINY.replace(batch=80, nheads=16, ngroups=2, headdim=64, dstate=128, window=4, steps=6, seed=21)
+    seqs = [0, 1, 39, 40, 78, 79]
+    layers, worst, _, _ = _run_decode(wl, "eager", ["f32"], wl.steps, seqs=seqs)
+    assert worst["f32"] <= 1e-4, worst
+    sp, ck, pe, fc = layers["f32"].counters()
+    assert sp.tolist() == [wl.steps] * wl.batch and ck.tolist() == [wl.steps] * wl.batch
+
+
 def test_dt_scaled_input_term():
     wl = I.TINY.replace(batch=2, nheads=4, ngroups=2, headdim=16, dstate=16, window=3, steps=12, seed=13)
     for mode in ("replay", "eager"):
