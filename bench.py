@@ -425,14 +425,30 @@ def timed_loop(L, toks_dev, ys, K, W, sync, split=True):
 
 def e2e_loop(L, toks_host, K, W, sync, nbuf=4):
     """Public-API decode with host buffers: every step copies its inputs from pinned
-    host memory to the device, decodes, and copies its output y back to pinned host
-    memory, all inside the timed region.  `nbuf` sets of device buffers rotate so
+    host memory to the device (one copy per step), decodes, and copies its output y
+    back to pinned host memory, all inside the timed region.  `nbuf` sets of device buffers rotate so
     that later steps' input copies (one copy stream) and earlier steps' output copies
     (another) run while the layer's stream decodes; events order each buffer's reuse."""
     import torch
 
     n = len(toks_host)
-    dev = [{k: torch.empty_like(v, device=L.device) for k, v in toks_host[0].items()} for _ in range(nbuf)]
+    # A step's inputs travel as one copy: each host step packed into one pinned
+    # buffer (every input at a 256-byte offset), the device inputs views of one buffer.
+    keys = list(toks_host[0].keys())
+    nbytes = {k: toks_host[0][k].numel() * toks_host[0][k].element_size() for k in keys}
+    offs, total = {}, 0
+    for k in keys:
+        offs[k] = total
+        total += (nbytes[k] + 255) // 256 * 256
+    host_packed = []
+    for d in toks_host:
+        buf = torch.zeros(total, dtype=torch.uint8).pin_memory()
+        for k in keys:
+            buf[offs[k]:offs[k] + nbytes[k]].copy_(d[k].contiguous().view(-1).view(torch.uint8))
+        host_packed.append(buf)
+    dev_buf = [torch.empty(total, dtype=torch.uint8, device=L.device) for _ in range(nbuf)]
+    dev = [{k: dev_buf[j][offs[k]:offs[k] + nbytes[k]].view(toks_host[0][k].dtype).view(toks_host[0][k].shape)
+            for k in keys} for j in range(nbuf)]
     y = [torch.empty((L.B, 1, L.H, L.P), dtype=torch.float32, device=L.device) for _ in range(nbuf)]
     y_host = [torch.empty_like(y[0], device="cpu").pin_memory() for _ in range(nbuf)]
     comp = torch.cuda.ExternalStream(L.stream) if not isinstance(L.stream, torch.cuda.Stream) else L.stream
@@ -448,8 +464,7 @@ def e2e_loop(L, toks_host, K, W, sync, nbuf=4):
         j = i % nbuf
         with torch.cuda.stream(h2d_s):
             h2d_s.wait_event(in_free[j])
-            for k, v in toks_host[i % n].items():
-                dev[j][k].copy_(v, non_blocking=True)
+            dev_buf[j].copy_(host_packed[i % n], non_blocking=True)
             in_ready[j].record(h2d_s)
         comp.wait_event(in_ready[j])
         comp.wait_event(y_free[j])
@@ -475,8 +490,7 @@ def e2e_loop(L, toks_host, K, W, sync, nbuf=4):
     comp.wait_event(done)
     t1.record(comp)
     sync()
-    h2d = sum(v.numel() * v.element_size() for v in toks_host[0].values())
-    return t0.elapsed_time(t1), h2d, y[0].numel() * y[0].element_size()
+    return t0.elapsed_time(t1), total, y[0].numel() * y[0].element_size()
 
 
 # ------------------------------------------------------------------ CPU oracle legs
