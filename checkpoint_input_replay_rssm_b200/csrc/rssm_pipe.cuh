@@ -1,5 +1,6 @@
-// rssm_pipe.cuh -- mbarrier + bulk-copy (TMA, non-multicast) primitives for the
-// persistent producer/consumer decode kernels, with time-bounded waits.
+// rssm_pipe.cuh -- mbarrier and bulk-copy primitives (a global tile into the
+// issuing CTA's own shared memory) for the persistent kernels, with
+// time-bounded waits.
 #pragma once
 
 #include "rssm_device.cuh"
