@@ -423,32 +423,48 @@ def timed_loop(L, toks_dev, ys, K, W, sync, split=True):
     return total_ms, per, pre, read, launches, steady
 
 
-def e2e_loop(L, toks_host, K, W, sync, nbuf=4):
-    """Public-API decode with host buffers: every step copies its inputs from pinned
-    host memory to the device (one copy per step), decodes, and copies its output y
-    back to pinned host memory, all inside the timed region.  `nbuf` sets of device buffers rotate so
-    that later steps' input copies (one copy stream) and earlier steps' output copies
-    (another) run while the layer's stream decodes; events order each buffer's reuse."""
+def pack_inputs(toks_host, pin):
+    """Each step's input tensors packed into one byte buffer (pinned when `pin`),
+    every input at a 256-byte offset, so that a step's inputs travel as one copy.
+    Returns the buffers, the offsets by input name and the buffer length."""
     import torch
 
-    n = len(toks_host)
-    # A step's inputs travel as one copy: each host step packed into one pinned
-    # buffer (every input at a 256-byte offset), the device inputs views of one buffer.
     keys = list(toks_host[0].keys())
     nbytes = {k: toks_host[0][k].numel() * toks_host[0][k].element_size() for k in keys}
     offs, total = {}, 0
     for k in keys:
         offs[k] = total
         total += (nbytes[k] + 255) // 256 * 256
-    host_packed = []
+    out = []
     for d in toks_host:
-        buf = torch.zeros(total, dtype=torch.uint8).pin_memory()
+        buf = torch.zeros(total, dtype=torch.uint8)
         for k in keys:
             buf[offs[k]:offs[k] + nbytes[k]].copy_(d[k].contiguous().view(-1).view(torch.uint8))
-        host_packed.append(buf)
+        out.append(buf.pin_memory() if pin else buf)
+    return out, offs, total
+
+
+def input_views(buf, like, offs):
+    """The inputs inside one packed buffer, as tensors shaped and typed like `like`."""
+    return {k: buf[o:o + like[k].numel() * like[k].element_size()].view(like[k].dtype).view(like[k].shape)
+            for k, o in offs.items()}
+
+
+def e2e_loop(L, toks_host, K, W, sync, nbuf=4):
+    """Public-API decode with host buffers: every step copies its inputs from pinned
+    host memory to the device (one copy per step), decodes, and copies its output y
+    back to pinned host memory, all inside the timed region.  `nbuf` sets of device
+    buffers rotate so that later steps' input copies (one copy stream) and earlier
+    steps' output copies (another) run while the layer's stream decodes; events
+    order each buffer's reuse."""
+    import torch
+
+    n = len(toks_host)
+    # A step's inputs travel as one copy: each host step packed into one pinned
+    # buffer, the device inputs views of one device buffer with the same layout.
+    host_packed, offs, total = pack_inputs(toks_host, pin=True)
     dev_buf = [torch.empty(total, dtype=torch.uint8, device=L.device) for _ in range(nbuf)]
-    dev = [{k: dev_buf[j][offs[k]:offs[k] + nbytes[k]].view(toks_host[0][k].dtype).view(toks_host[0][k].shape)
-            for k in keys} for j in range(nbuf)]
+    dev = [input_views(dev_buf[j], toks_host[0], offs) for j in range(nbuf)]
     y = [torch.empty((L.B, 1, L.H, L.P), dtype=torch.float32, device=L.device) for _ in range(nbuf)]
     y_host = [torch.empty_like(y[0], device="cpu").pin_memory() for _ in range(nbuf)]
     comp = torch.cuda.ExternalStream(L.stream) if not isinstance(L.stream, torch.cuda.Stream) else L.stream
