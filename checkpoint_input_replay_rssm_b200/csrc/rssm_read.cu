@@ -14,9 +14,9 @@ static int tq_of_read(int T) { return T <= 1 ? 1 : (T <= 4 ? 4 : 8); }
 
 // Heads per read CTA: about 128 KiB of read copy per CTA, the heads sharing one
 // query row when a query row serves several heads (Mamba-2 groups).  A CTA
-// streams its rows in rounds of 8 x 16 bytes per thread and issues each round
-// before dotting the previous one, so its small operands' round trips overlap
-// the stream; on the 128-head layer 32 KiB gave 0.65 of peak bandwidth, 64 KiB
+// streams its rows in rounds of 8 x 16 bytes per thread, each half of a round
+// reissued as soon as it has been dotted, and its small operands' round trips
+// overlap the stream; on the 128-head layer 32 KiB gave 0.65 of peak bandwidth, 64 KiB
 // 0.76, 128 KiB 0.81, 256 KiB 0.48 (too few CTAs for the SMs).  Shapes with
 // small heads are also held to 64 KiB of shared memory at the largest query
 // count (the buffered entries and coefficients grow with the heads).
